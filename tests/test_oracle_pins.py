@@ -1,0 +1,376 @@
+"""Pins for the fp64 oracle: checks against what the pages and mathematics fix.
+
+None of these re-types the oracle's formulas: each compares the oracle with a
+closed form, an exact rational computation, a brute-force search, an invariant,
+an exhaustive enumeration, a special case that reduces to a simpler method, or a
+value the pages print (tests/golden).
+"""
+from fractions import Fraction
+import itertools
+import os
+
+import numpy as np
+import pytest
+
+import datagen
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bf16(a):
+    return datagen.f32_to_bf16_bits(np.asarray(a, dtype=np.float32))
+
+
+def f32(b):
+    return datagen.bf16_bits_to_f32(b)
+
+
+# --------------------------------------------------------------------------
+# H: diagonal Gauss-Newton proxy (Sparsity Induction sec. 2C)
+# --------------------------------------------------------------------------
+
+def test_H_closed_form_constant_columns():
+    # a column of constant +-c has mean square exactly c^2
+    T, K = 300, 6
+    c = np.array([0.5, 1.0, 3.0, 0.125, 7.0, 1.5], dtype=np.float32)
+    signs = np.where(np.random.default_rng(0).integers(0, 2, (T, K)) > 0, 1.0, -1.0)
+    X = bf16(signs * c[None, :])
+    H = oracle.hessian_diag(X)
+    assert np.array_equal(H, (c.astype(np.float64) ** 2))
+
+
+def test_H_exact_rational_small():
+    # exact rational mean of the bf16 squares bounds the oracle's rounding error
+    X = datagen.make_activations(257, 40, seed=3, n_outliers=3)
+    H = oracle.hessian_diag(X)
+    xs = f32(X).astype(np.float64)
+    for j in range(X.shape[1]):
+        exact = sum(Fraction(float(v)) ** 2 for v in xs[:, j]) / X.shape[0]
+        err = abs(Fraction(float(H[j])) - exact)
+        # each of at most T+2 roundings is within 2^-53 relative of a partial sum <= total
+        assert err <= exact * Fraction(X.shape[0] + 2, 2 ** 53)
+
+
+def test_H_power_of_two_scaling_is_exact():
+    # scaling a channel by 2^k scales H by 4^k exactly (the O(d_in) refresh
+    # of Sparsity Induction sec. 2C reduces to this for power-of-two scales)
+    X = datagen.make_activations(200, 16, seed=5)
+    xf = f32(X)
+    scale = np.array([2.0 ** ((j % 5) - 2) for j in range(16)], dtype=np.float32)
+    X2 = bf16(xf * scale[None, :])
+    assert np.array_equal(f32(X2), xf * scale[None, :])  # scaling exact in bf16
+    H, H2 = oracle.hessian_diag(X), oracle.hessian_diag(X2)
+    assert np.array_equal(H2, H * (scale.astype(np.float64) ** 2))
+
+
+def test_H_canonical_vs_naive_and_single_chunk():
+    X = datagen.make_activations(1000, 64, seed=7, n_outliers=2)
+    Hc = oracle.hessian_diag(X)
+    Hn = oracle.hessian_diag(X, naive=True)
+    assert np.all(np.abs(Hc - Hn) <= 1e-12 * np.abs(Hn))
+    # with at most one chunk of tokens the canonical order is the sequential one
+    Xs = X[: oracle.H_CHUNK]
+    assert np.array_equal(oracle.hessian_diag(Xs), oracle.hessian_diag(Xs, naive=True))
+
+
+def test_H_outlier_channels_scale_400x_in_expectation():
+    X = datagen.make_activations(4096, 512, seed=0, n_outliers=4)
+    H = oracle.hessian_diag(X)
+    cols = datagen.outlier_columns(512, 4, 0)
+    rest = np.setdiff1d(np.arange(512), cols)
+    ratio = H[cols].mean() / H[rest].mean()
+    assert 360 < ratio < 440
+
+
+# --------------------------------------------------------------------------
+# S: Hessian-aware score (SparseForge) and latent magnitude (Sparse-BitNet)
+# --------------------------------------------------------------------------
+
+def test_S_special_values():
+    H = np.array([0.0, 1.0, 4.0, 0.25], dtype=np.float64)
+    W = bf16([[0.0, 1.0, -2.0, 0.5], [3.0, -0.0, 1.0, -1.0]])
+    S = oracle.score_hessian(H, W, 0.0)
+    # exact small dyadic cases: (H + 0) * w^2
+    assert np.array_equal(S, np.array([[0, 1, 16, 0.0625], [0, 0, 4, 0.25]], dtype=np.float32))
+    # H = 0: score is eps * w^2
+    S2 = oracle.score_hessian(np.zeros(4), W, 0.5)
+    assert np.array_equal(S2, np.array([[0, 0.5, 2, 0.125], [4.5, 0, 0.5, 0.5]], dtype=np.float32))
+
+
+def test_S_magnitude_exact():
+    W = datagen.make_weight(8, 24, 0.02, seed=1)
+    S = oracle.score_magnitude(W)
+    assert np.array_equal(S, np.abs(f32(W)))
+
+
+def test_S_constant_H_reduces_to_magnitude_mask():
+    # constant H: (H+eps)W^2 is monotone in |W|, so the mask equals the
+    # magnitude-pruning mask (SALR sec. on static magnitude masks; Sparse-BitNet sec. 2)
+    W = datagen.make_weight(64, 96, 0.02, seed=2)
+    for (n, m) in ((2, 4), (6, 8), (4, 6), (3, 8)):
+        mh, _, _ = oracle.prune(oracle.score_hessian(np.full(96, 0.7), W, 1e-8), W, n, m)
+        mm, _, _ = oracle.prune(oracle.score_magnitude(W), W, n, m)
+        assert np.array_equal(mh, mm)
+
+
+def test_S_eps0_ranks_like_wanda():
+    # Sparsity Induction sec. 2C: with eps = 0, H_j W^2 ranks like Wanda's
+    # |W| * ||X_j||_2 (= |W| sqrt(T H_j)); compare on groups with separated scores
+    T, K, R = 64, 64, 32
+    X = datagen.make_activations(T, K, seed=11, n_outliers=2)
+    W = datagen.make_weight(R, K, 0.02, seed=12)
+    H = oracle.hessian_diag(X)
+    S = oracle.score_hessian(H, W, 0.0)
+    xf = f32(X).astype(np.float64)
+    wanda = np.abs(f32(W).astype(np.float64)) * np.sqrt((xf ** 2).sum(axis=0))[None, :]
+    for (n, m) in ((2, 4), (6, 8)):
+        mh, _, _ = oracle.prune(S, W, n, m)
+        bits = ((mh[:, :, None] >> np.arange(32, dtype=np.uint32)) & 1).reshape(R, -1)[:, :K]
+        wg = wanda.reshape(R, K // m, m)
+        srt = np.sort(wg, axis=2)
+        gap = (srt[:, :, m - n] - srt[:, :, m - n - 1]) / np.maximum(srt[:, :, m - n], 1e-300)
+        ok = gap > 1e-6
+        order = np.argsort(-wg, axis=2, kind="stable")[:, :, :n]
+        ref = np.zeros((R, K // m, m), dtype=bool)
+        np.put_along_axis(ref, order, True, axis=2)
+        got = bits.reshape(R, K // m, m).astype(bool)
+        assert ok.mean() > 0.95
+        assert np.array_equal(got[ok], ref[ok])
+
+
+# --------------------------------------------------------------------------
+# mask: top-n per group (SparseForge hard target), exact n per group
+# --------------------------------------------------------------------------
+
+def _bits(mask, K):
+    R = mask.shape[0]
+    return ((mask[:, :, None] >> np.arange(32, dtype=np.uint32)) & 1).reshape(R, -1)[:, :K]
+
+
+@pytest.mark.parametrize("m", [4, 6, 8, 10])
+def test_mask_brute_force_all_subsets(m):
+    # for every n < m, the kept set maximises the group's score sum; among equal
+    # maxima it is the lexicographically smallest index set (= lower index wins ties)
+    R = 40
+    S = datagen.tie_heavy_scores(R, m * 3, seed=m)
+    V = bf16(np.arange(R * m * 3, dtype=np.float32).reshape(R, -1) % 97 + 1)
+    for n in range(1, m):
+        mask, vals, meta = oracle.prune(S, V, n, m)
+        bits = _bits(mask, m * 3)
+        for r in range(R):
+            for g in range(3):
+                s = S[r, g * m:(g + 1) * m].astype(np.int64)
+                best = None
+                for sub in itertools.combinations(range(m), n):  # lexicographic order
+                    tot = int(s[list(sub)].sum())
+                    if best is None or tot > best[0]:
+                        best = (tot, sub)
+                got = tuple(np.nonzero(bits[r, g * m:(g + 1) * m])[0])
+                assert got == best[1]
+                # compressed values: kept V in ascending column order
+                assert list(vals[r, g * n:(g + 1) * n]) == [V[r, g * m + q] for q in best[1]]
+
+
+def test_mask_exactly_n_per_group_with_ragged_tail():
+    for (n, m, K) in ((2, 4, 1030), (6, 8, 8195), (4, 6, 1003), (8, 10, 207), (1, 3, 10)):
+        W = datagen.make_weight(9, K, 0.02, seed=K)
+        S = oracle.score_magnitude(W)
+        mask, vals, _ = oracle.prune(S, W, n, m)
+        G = oracle.n_groups(K, m)
+        allbits = _bits(mask, G * m).reshape(9, G, m)
+        assert np.all(allbits.sum(axis=2) == n)
+        # words past G*m are zero
+        full = ((mask[:, :, None] >> np.arange(32, dtype=np.uint32)) & 1).reshape(9, -1)
+        assert full[:, G * m:].sum() == 0
+        # padding survives only when the tail has fewer than n real columns, as value 0
+        tail = K - (G - 1) * m
+        pad_kept = allbits[:, G - 1, tail:].sum(axis=1)
+        assert np.all(pad_kept == max(0, n - tail))
+
+
+def test_mask_ties_and_signed_zero():
+    S = np.array([[1, 1, 1, 1, -0.0, 0.0, 0.0, -0.0]], dtype=np.float32)
+    V = bf16([[1, 2, 3, 4, 5, 6, 7, 8]])
+    mask, vals, meta = oracle.prune(np.abs(S), V, 2, 4)
+    assert list(_bits(mask, 8)[0]) == [1, 1, 0, 0, 1, 1, 0, 0]
+    assert meta[0, 0] == (0 | 1 << 2) | ((0 | 1 << 2) << 4)
+    S2 = S.copy()
+    S2[0, 4] = -0.0  # -0 == +0 is a tie
+    mask2, _, _ = oracle.prune(S2, V, 2, 4)
+    assert np.array_equal(mask, mask2)
+
+
+def test_meta24_encoding_matches_mask():
+    W = datagen.make_weight(16, 64, 0.02, seed=4)
+    mask, vals, meta = oracle.prune(oracle.score_magnitude(W), W, 2, 4)
+    bits = _bits(mask, 64)
+    for r in range(16):
+        for g in range(16):
+            idx = list(np.nonzero(bits[r, 4 * g:4 * g + 4])[0])
+            nib = (meta[r, g // 2] >> (4 * (g % 2))) & 0xF
+            assert nib == idx[0] | (idx[1] << 2)
+
+
+# --------------------------------------------------------------------------
+# slide: SlideSparse sliding-window decomposition, exhaustive
+# --------------------------------------------------------------------------
+
+def _golden_lines(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+@pytest.mark.parametrize("Ns", [2, 3, 4, 5])
+def test_slide_exhaustive_every_group_mask(Ns):
+    m = 2 * Ns
+    n = m - 2
+    masks = list(itertools.combinations(range(m), n))
+    assert len(masks) == {2: 6, 3: 15, 4: 28, 5: 45}[Ns]
+    R = len(masks)
+    S = np.zeros((R, m), dtype=np.float32)
+    for r, sub in enumerate(masks):
+        S[r, list(sub)] = 1.0
+    V = bf16(np.arange(1, R * m + 1, dtype=np.float32).reshape(R, m))
+    mask, vals, _ = oracle.prune(S, V, n, m)
+    wmeta = oracle.slide_pack(mask, m, m)
+    for r in range(R):
+        for w in range(Ns - 1):
+            nib = (wmeta[r, w // 2] >> (4 * (w % 2))) & 0xF
+            a, b = nib & 3, nib >> 2
+            assert 0 <= a < b <= 3  # exactly 2 survivors per width-4 window
+        # reconstruction is bit-exact
+    Wd = oracle.slide_unpack(vals, wmeta, m, m)
+    assert np.array_equal(Wd, oracle.dense_masked(mask, V, m))
+    # necessity: Ns-2 windows hold at most 2(Ns-2) < 2Ns-2 survivors
+    assert 2 * (Ns - 2) < n
+
+
+def test_slide_windows_match_pages_example():
+    # the lift map of 6:8 places window w over columns 2w..2w+3 (pieces 1-4, 3-6, 5-8)
+    rows = _golden_lines("slidesparse_windows_6of8.txt")
+    K, m = 8, 8
+    X = bf16(np.arange(1, K + 1, dtype=np.float32)[None, :])
+    XL = f32(oracle.lift(X, m))[0]
+    for (w, first, last) in rows:
+        w, first, last = int(w), int(first), int(last)
+        assert list(XL[4 * (w - 1):4 * w]) == list(range(first, last + 1))
+
+
+def test_slide_expansion_and_bound_match_pages():
+    for (pat, N, nwin, gam, spd) in _golden_lines("slidesparse_bounds.txt"):
+        N = int(N)
+        m = 2 * N
+        K = 96 * m
+        assert oracle.lifted_cols(K, m) // 4 // (K // m) == int(nwin)
+        assert Fraction(oracle.lifted_cols(K, m), K) == Fraction(gam)
+        # sparse pipe does half the lifted MACs: dense K vs K'/2 -> bound N/(N-1)
+        assert Fraction(K, oracle.lifted_cols(K, m) // 2) == Fraction(spd)
+    for Ns in (2, 3, 4, 5):
+        m = 2 * Ns
+        assert Fraction(oracle.lifted_cols(40 * m, m), 40 * m) == Fraction(2) - Fraction(2, Ns)
+
+
+def test_slide_rejects_non_slide_masks():
+    S = np.zeros((1, 8), dtype=np.float32)
+    S[0, :5] = 1
+    mask, _, _ = oracle.prune(S, bf16(np.ones((1, 8))), 5, 8)
+    with pytest.raises(ValueError):
+        oracle.slide_pack(mask, 8, 8)
+
+
+# --------------------------------------------------------------------------
+# lift + GEMM identity; GEMM against exact integer arithmetic
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n,m,K", [(2, 4, 64), (4, 6, 66), (6, 8, 80), (8, 10, 70), (6, 8, 83), (4, 6, 61)])
+def test_lifted_times_packed_equals_masked_bitexact(n, m, K):
+    T, R = 13, 11
+    X = datagen.make_activations(T, K, seed=K + m, n_outliers=2)
+    W = datagen.make_weight(R, K, 0.02, seed=K * m)
+    res = oracle.run_layer(X, W, n, m)
+    XL = oracle.lift(X, m)
+    Y1 = oracle.gemm_lifted(XL, res["vals"], res["wmeta"], K, m)
+    Y2 = oracle.gemm_masked(X, res["mask"], W, m)
+    Y3 = oracle.gemm_dense(X, oracle.slide_unpack(res["vals"], res["wmeta"], K, m))
+    assert np.array_equal(Y1, Y2)
+    assert np.array_equal(Y2, Y3)
+
+
+def test_gemm_exact_on_small_integers():
+    # integer-valued bf16 inputs: every fp64 partial sum is exact, so the oracle
+    # must equal integer matrix multiplication of the masked matrix
+    T, K, R = 17, 48, 9
+    X = datagen.small_int_bf16((T, K), seed=1, tensor_id=2)
+    W = datagen.small_int_bf16((R, K), seed=1, tensor_id=1)
+    for (n, m) in ((2, 4), (6, 8), (4, 6)):
+        S = oracle.score_magnitude(W)
+        mask, vals, _ = oracle.prune(S, W, n, m)
+        Wm = f32(oracle.dense_masked(mask, W, K)).astype(np.int64)
+        ref = f32(X).astype(np.int64) @ Wm.T
+        Y = oracle.gemm_masked(X, mask, W, m)
+        assert np.array_equal(Y, ref.astype(np.float64))
+        # transposition check: a single nonzero weight picks one column of X
+    W1 = np.zeros((R, K), dtype=np.uint16)
+    W1[3, 5] = bf16([2.0])[0]
+    mask1 = np.zeros((R, oracle.mask_words(K, 4)), dtype=np.uint32)
+    mask1[3, 0] = 1 << 5
+    Y = oracle.gemm_masked(X, mask1, W1, 4)
+    assert np.array_equal(Y[:, 3], 2.0 * f32(X)[:, 5].astype(np.float64))
+    assert np.count_nonzero(np.delete(Y, 3, axis=1)) == 0
+
+
+def test_gemm_row_sampling_matches_full():
+    X = datagen.make_activations(20, 32, seed=9)
+    W = datagen.make_weight(7, 32, 0.02, seed=9)
+    res = oracle.run_layer(X, W, 2, 4)
+    rows = np.array([19, 0, 7], dtype=np.int64)
+    full = oracle.gemm_masked(X, res["mask"], W, 4)
+    assert np.array_equal(oracle.gemm_masked(X, res["mask"], W, 4, rows=rows), full[rows])
+
+
+# --------------------------------------------------------------------------
+# ternary absmean quantisation (Sparse-BitNet)
+# --------------------------------------------------------------------------
+
+def test_ternary_closed_form():
+    W = bf16([[1.0, -2.0, 1.0, 2.0], [-1.0, 2.0, 0.5, -0.5]])
+    # mean |W| = (1+2+1+2+1+2+0.5+0.5)/8 = 1.25; W/gamma: 0.8 -> 1, 1.6 -> 1, 0.4 -> 0
+    g, Wq = oracle.ternary(W)
+    assert g == 1.25
+    q = f32(Wq)
+    assert np.array_equal(q, np.array([[1.25, -1.25, 1.25, 1.25], [-1.25, 1.25, 0, 0]], dtype=np.float32))
+    # half-way case rounds to even (0): |w| / gamma == 0.5 exactly
+    W2 = bf16([[1.0, 3.0, 0.0, 0.0]])  # gamma = 1.0, 1/1=1 -> 1; 3 -> clip 1; 0 -> 0
+    g2, Wq2 = oracle.ternary(W2)
+    assert g2 == 1.0 and list(f32(Wq2)[0]) == [1.0, 1.0, 0.0, 0.0]
+    W3 = bf16([[0.5, 1.5, 0.0, 0.0]])  # gamma = 0.5: 1.0 -> 1, 3 -> 1
+    W4 = bf16([[1.0, 1.0, 1.0, 1.0, 0.5, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0]])
+    g4, Wq4 = oracle.ternary(W4)  # gamma = 4.5/18 = 0.25: 0.5/0.25 = 2 -> 1; 1/0.25 -> 1
+    assert g4 == 0.25 and f32(Wq4)[0, 4] == 0.25
+    W5 = bf16([[0.5, 0.5, 1.5, 1.5]])  # gamma = 1.0: 0.5 -> tie -> 0 (even); 1.5 -> 2 -> clip 1
+    g5, Wq5 = oracle.ternary(W5)
+    assert g5 == 1.0 and list(f32(Wq5)[0]) == [0.0, 0.0, 1.0, 1.0]
+    assert oracle.ternary(W3)[0] == 0.5
+
+
+def test_ternary_gaussian_zero_fraction():
+    # for Gaussian W, |w| < gamma/2 with gamma = E|w| = sigma sqrt(2/pi):
+    # P = erf(sqrt(2/pi)/2 / sqrt(2)) ~= 0.3101
+    W = datagen.make_weight(256, 1024, 0.02, seed=0)
+    g, Wq = oracle.ternary(W)
+    frac = np.mean(Wq == 0)
+    assert abs(g - 0.02 * np.sqrt(2 / np.pi)) < 2e-4
+    assert abs(frac - 0.3101) < 0.005
+
+
+def test_f64_to_bf16_rounding():
+    assert oracle.f64_to_bf16(1.0) == 0x3F80
+    assert oracle.f64_to_bf16(-2.0) == 0xC000
+    # 1 + 2^-8 is a tie between 1 and 1+2^-7 -> even (1.0)
+    assert oracle.f64_to_bf16(1.0 + 2 ** -8) == 0x3F80
+    assert oracle.f64_to_bf16(1.0 + 2 ** -8 + 2 ** -40) == 0x3F81
+    assert oracle.f64_to_bf16(1.0 + 3 * 2 ** -8) == 0x3F82  # tie, odd -> up
+    # agrees with fp32 rounding where no double rounding can occur
+    for v in (0.0123, 3.75, 1e-3, 123.456):
+        assert oracle.f64_to_bf16(v) == int(datagen.f32_to_bf16_bits(np.array([v], dtype=np.float32))[0])
