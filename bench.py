@@ -1,0 +1,468 @@
+#!/usr/bin/env python
+"""Benchmark of the N:M-pruned linear layer hot path on B200.
+
+One step = one pass of the whole path over one layer of synthetic input:
+  a1 H = mean_t x^2            (nm_hessian_diag, part of nm_score)
+  a2 S = (H + eps) W^2         (nm_score)
+  a3 top-n per group + compress (nm_prune_compress)
+  a4 sliding-window pack       (slide_pack, m > 4)
+  a6 operand preparation       (nm_sparse_prepare)
+  a5+a7 lift-in-staging sparse GEMM Y = X W_sparse^T (nm_sparse_gemm)
+  a8 own dense GEMM on the masked W (nm_dense_gemm), the speedup reference.
+
+Prints ONE JSON line.  `value` is the sparse GEMM's effective TFLOP/s,
+2*T*R*K / t_gemm summed over all ranks' layers; the other stages are timed in
+the same steps and reported in `stages_ms`.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   (the fp64 CPU oracle on a sample)
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import datagen  # noqa: E402
+
+DEFAULT_WORKLOAD = "slide_6of8_4096"
+METRIC = "N:M sparse GEMM effective TFLOP/s, % of 2:4 TC peak, speedup vs own dense"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def workload_config(layer: datagen.Layer, l2_note: str):
+    G = (layer.K + layer.m - 1) // layer.m
+    KL = G * (layer.m // 2 - 1) * 4
+    return {
+        "workload": layer.name, "R": layer.R, "K": layer.K, "T": layer.T,
+        "pattern": f"{layer.n}:{layer.m}", "lifted_K": KL, "score": layer.score,
+        "ternary": layer.ternary, "eps": layer.eps, "x_outlier_channels": layer.x_outliers,
+        "w_sigma": layer.w_sigma, "seed": layer.seed, "l2": l2_note,
+    }
+
+
+# --------------------------------------------------------------------------
+# clocks sampled with nvidia-smi during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm_, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm_)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import semi_structured_sparse_diag_b200 as nm
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    layer = datagen.WORKLOADS[args.workload]
+    # weak scaling: every rank prunes and multiplies its own layer (seed = rank)
+    X_h, W_h = datagen.layer_inputs(layer, seed=layer.seed + rank)
+    R, K, T, n, m = layer.R, layer.K, layer.T, layer.n, layer.m
+    lib = nm.load()
+    stream = torch.cuda.current_stream()
+
+    def dev_bf16(a):
+        return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    X = dev_bf16(X_h)
+    W = dev_bf16(W_h)
+    G = (K + m - 1) // m
+    KL = G * (m // 2 - 1) * 4
+    KLpad = (KL + 127) // 128 * 128
+    # persistent buffers (allocated once, outside the timed region)
+    H = torch.empty(K, dtype=torch.float64, device=dev)
+    S = torch.empty((R, K), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(1, lib.nm_hessian_workspace_bytes(T, K)), dtype=torch.uint8, device=dev)
+    mask = torch.empty((R, (G * m + 31) // 32), dtype=torch.int32, device=dev)
+    vals = torch.empty((R, G * n), dtype=torch.bfloat16, device=dev)
+    meta = torch.empty((R, (G + 1) // 2), dtype=torch.uint8, device=dev) if m == 4 else None
+    nw = G * (m // 2 - 1)
+    wmeta = torch.empty((R, (nw + 1) // 2), dtype=torch.uint8, device=dev) if m > 4 else None
+    packed = torch.empty(lib.nm_sparse_prepare_bytes(R, K, m), dtype=torch.uint8, device=dev)
+    ldy = (R + 7) // 8 * 8
+    Y = torch.empty((T, ldy), dtype=torch.bfloat16, device=dev)
+    Yd = torch.empty((T, ldy), dtype=torch.bfloat16, device=dev)
+    V = W
+    Wq = gamma = tws = None
+    if layer.ternary:
+        Wq = torch.empty((R, K), dtype=torch.bfloat16, device=dev)
+        gamma = torch.empty(1, dtype=torch.float64, device=dev)
+        tws = torch.empty(lib.nm_ternary_workspace_bytes(R), dtype=torch.uint8, device=dev)
+        V = Wq
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    s = stream.cuda_stream
+
+    def chk(st, what):
+        if st != 0:
+            raise nm.NMError(f"{what}: {lib.nm_status_string(st).decode()}")
+
+    stage_names = ["score", "prune", "slide_pack", "prepare", "sparse_gemm", "dense_gemm"]
+    launches_per_step = 0
+
+    def step(ev=None, Xs=X, Ws=W):
+        nonlocal launches_per_step
+        cnt = 0
+        Vs = Wq if layer.ternary else Ws
+        if ev is not None:
+            ev[0].record(stream)
+        if layer.ternary:
+            chk(lib.nm_ternary_quantize(Ws.data_ptr(), R, K, K, Wq.data_ptr(), gamma.data_ptr(),
+                                        tws.data_ptr(), tws.numel(), s), "ternary")
+            cnt += 3
+        if layer.score == "hessian":
+            chk(lib.nm_score(Xs.data_ptr(), T, K, Ws.data_ptr(), R, K, K, layer.eps, H.data_ptr(),
+                             S.data_ptr(), ws.data_ptr(), ws.numel(), s), "score")
+            cnt += 3 if T > 128 else 2  # H chunk (+ finish) + score
+        else:
+            chk(lib.nm_score(None, 0, 0, Ws.data_ptr(), R, K, K, 0.0, None, S.data_ptr(), None, 0, s),
+                "score")
+            cnt += 1
+        if ev is not None:
+            ev[1].record(stream)
+        chk(lib.nm_prune_compress(S.data_ptr(), K, Vs.data_ptr(), K, R, K, n, m, mask.data_ptr(),
+                                  vals.data_ptr(), meta.data_ptr() if meta is not None else None, s),
+            "prune")
+        cnt += 1
+        if ev is not None:
+            ev[2].record(stream)
+        if m > 4:
+            chk(lib.slide_pack(mask.data_ptr(), R, K, m, wmeta.data_ptr(), s), "slide_pack")
+            cnt += 1
+        if ev is not None:
+            ev[3].record(stream)
+        wm = meta if m == 4 else wmeta
+        chk(lib.nm_sparse_prepare(vals.data_ptr(), wm.data_ptr(), R, K, m, packed.data_ptr(),
+                                  packed.numel(), s), "prepare")
+        cnt += 2
+        if ev is not None:
+            ev[4].record(stream)
+        chk(lib.nm_sparse_gemm(Xs.data_ptr(), T, K, K, packed.data_ptr(), R, m, Y.data_ptr(), ldy, s),
+            "sparse_gemm")
+        cnt += 1
+        if ev is not None:
+            ev[5].record(stream)
+        chk(lib.nm_dense_gemm(Xs.data_ptr(), T, K, K, Wdense.data_ptr(), R, K, Yd.data_ptr(), ldy, s),
+            "dense_gemm")
+        cnt += 1
+        if ev is not None:
+            ev[6].record(stream)
+        launches_per_step = cnt
+
+    # comparator input: the masked weights as a dense matrix (set-up, not timed)
+    Wdense = torch.empty_like(W)
+    step_pre = True
+    if step_pre:
+        # one untimed pass produces the mask; densify it for the dense GEMM
+        Wdense.copy_(W)
+        step()
+        torch.cuda.synchronize()
+        nm.check_device_error()
+        bits = ((mask.view(torch.int32).unsqueeze(-1) >> torch.arange(32, device=dev, dtype=torch.int32)) & 1)
+        bits = bits.reshape(R, -1)[:, :K].bool()
+        Wdense = torch.where(bits, V, torch.zeros_like(V)).contiguous()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    nm.check_device_error()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    clocks = ClockSampler(local) if rank == 0 else None
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()  # L2 flush between timed steps (outside the events)
+        step(evs[i])
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop() if clocks else None
+    nm.check_device_error()
+
+    stage_ms = {k: 0.0 for k in stage_names}
+    step_ms = 0.0
+    for e in evs:
+        for j, k in enumerate(stage_names):
+            stage_ms[k] += e[j].elapsed_time(e[j + 1])
+        step_ms += e[0].elapsed_time(e[6])
+    stage_ms = {k: v / args.steps for k, v in stage_ms.items()}
+    step_ms /= args.steps
+    gemm_ms = stage_ms["sparse_gemm"]
+    dense_ms = stage_ms["dense_gemm"]
+    if world > 1:
+        t = torch.tensor([step_ms, gemm_ms, dense_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms, gemm_ms, dense_ms = t.tolist()
+
+    # ------------------------------------------------ end-to-end through the C ABI
+    Xh = torch.from_numpy(X_h.view(np.int16)).pin_memory()
+    Wh = torch.from_numpy(W_h.view(np.int16)).pin_memory()
+    Yh = torch.empty((T, ldy), dtype=torch.int16).pin_memory()
+    Xe = torch.empty_like(X)
+    We = torch.empty_like(W)
+    e2e_steps = max(1, min(args.steps, 5))
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = 0.0
+    for _ in range(e2e_steps):
+        flush.zero_()
+        e0.record(stream)
+        Xe.view(torch.int16).copy_(Xh, non_blocking=True)
+        We.view(torch.int16).copy_(Wh, non_blocking=True)
+        step(None, Xe, We)
+        Yh.copy_(Y.view(torch.int16), non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms += e0.elapsed_time(e1)
+    e2e_ms /= e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+    nm.check_device_error()
+
+    hbm, bf16_tf, peak_src = peaks()
+    sparse_peak = 2.0 * bf16_tf  # 2:4 sparse bf16 = 2 x dense bf16 (nominal 4.5 / 2.25)
+    flops_eff = 2.0 * T * R * K                 # dense-equivalent of the original layer
+    flops_lift = 2.0 * T * R * KLpad            # dense-equivalent of the lifted 2:4 problem
+    value = world * flops_eff / (gemm_ms * 1e-3) / 1e12
+    achieved = flops_lift / (gemm_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": workload_config(layer, "flushed between steps (256 MiB write)"),
+        "pct_of_2to4_peak": round(100.0 * achieved / sparse_peak, 2),
+        "speedup_vs_own_dense": round(dense_ms / gemm_ms, 4),
+        "speedup_bound": round(K / (KL / 2), 4),
+        "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+        "roofline": {
+            "kernel": "k_gemm<MODE_SPLIFT>" if m > 4 else "k_gemm<MODE_SP24>",
+            "bound": "tensor",
+            "achieved": round(achieved, 2),
+            "peak": round(sparse_peak, 1),
+            "peak_source": f"2 x {peak_src} dense bf16 burst ({bf16_tf} TFLOP/s)",
+            "unit": "TFLOP/s",
+            "frac": round(achieved / sparse_peak, 4),
+            "traffic": None,
+            "per_unit": "2*R*K'pad flops per token; units per launch = T tokens",
+        },
+        "e2e": {
+            "value": round(world * flops_eff / (e2e_ms * 1e-3) / 1e12, 3),
+            "unit": "TFLOP/s",
+            "ms_per_step": round(e2e_ms, 4),
+            "h2d_bytes_per_step": int(X_h.nbytes + W_h.nbytes),
+            "d2h_bytes_per_step": int(T * ldy * 2),
+            "note": "whole step (all stages) with pinned H2D of X, W and D2H of Y in the timed region",
+        },
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(layer, X_h, W_h, budget_s=args.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------
+# the oracle on a bounded sample (CPU baseline and the reference arm)
+# --------------------------------------------------------------------------
+def oracle_sample_step(layer, X_h, W_h, rows_w: int, tok: int):
+    """One oracle step on a sample: H on all of X; S/prune/pack on `rows_w`
+    weight rows; fp64 GEMM of `tok` tokens against those rows.  Returns
+    (seconds, sample flops (dense-equivalent), stage seconds)."""
+    import oracle
+    t0 = time.perf_counter()
+    Wsub = np.ascontiguousarray(W_h[:rows_w])
+    V = Wsub
+    if layer.ternary:
+        _, V = oracle.ternary(Wsub)
+    if layer.score == "hessian":
+        H = oracle.hessian_diag(X_h)
+        S = oracle.score_hessian(H, Wsub, layer.eps)
+    else:
+        S = oracle.score_magnitude(Wsub)
+    t1 = time.perf_counter()
+    mask, vals, meta = oracle.prune(S, V, layer.n, layer.m)
+    if layer.m > 4:
+        oracle.slide_pack(mask, layer.K, layer.m)
+    t2 = time.perf_counter()
+    rows = np.arange(tok, dtype=np.int64)
+    oracle.gemm_masked(X_h, mask, V, layer.m, rows=rows)
+    t3 = time.perf_counter()
+    return t3 - t0, 2.0 * tok * rows_w * layer.K, {"score": t1 - t0, "prune_pack": t2 - t1,
+                                                   "gemm": t3 - t2}
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def _sample_size(layer, budget_s):
+    # ~1 GFLOP/s-per-core class fp64 loops: size the GEMM sample to the budget
+    rows_w = min(layer.R, 1024)
+    tok = max(1, min(layer.T, int(budget_s * 0.25e9 * _cores() / (2.0 * rows_w * layer.K))))
+    return rows_w, tok
+
+
+def cpu_baseline(layer, X_h, W_h, budget_s=10.0):
+    rows_w, tok = _sample_size(layer, budget_s)
+    sec, flops, stages = oracle_sample_step(layer, X_h, W_h, rows_w, tok)
+    return {
+        "value": round(flops / stages["gemm"] / 1e12, 6),
+        "unit": "TFLOP/s",
+        "cores": _cores(),
+        "kind": "oracle",
+        "sample": (f"{layer.name}: H over all {layer.T} tokens, score+prune+pack on {rows_w} of "
+                   f"{layer.R} weight rows, fp64 GEMM of {tok} tokens x {rows_w} rows x K={layer.K}; "
+                   f"value = sample GEMM flops / oracle GEMM seconds; step {sec:.2f} s"),
+        "stage_seconds": {k: round(v, 3) for k, v in stages.items()},
+    }
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    layer = datagen.WORKLOADS[args.workload]
+    X_h, W_h = datagen.layer_inputs(layer)
+    rows_w, tok = _sample_size(layer, args.cpu_seconds / 2)
+    for _ in range(args.warmup):
+        oracle_sample_step(layer, X_h, W_h, min(rows_w, 128), 1)
+    secs, gsecs, flops = [], [], 0.0
+    for _ in range(args.steps):
+        s, f, st = oracle_sample_step(layer, X_h, W_h, rows_w, tok)
+        secs.append(s)
+        gsecs.append(st["gemm"])
+        flops = f
+    value = flops / (sum(gsecs) / len(gsecs)) / 1e12
+    sample = (f"{layer.name}: per step H over all {layer.T} tokens, score+prune+pack on {rows_w} of "
+              f"{layer.R} weight rows, fp64 GEMM of {tok} tokens x {rows_w} rows x K={layer.K}")
+    line = {
+        "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * sum(secs) / len(secs), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(layer, "host memory (CPU oracle)"),
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _cores(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(datagen.WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

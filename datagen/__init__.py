@@ -27,9 +27,10 @@ TID_OUTLIER_COLS = 3
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     """Round fp32 values to bf16 (round-to-nearest-even); returns uint16 bit patterns."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    rounding_bias = ((u >> 16) & 1) + 0x7FFF
-    out = ((u + rounding_bias) >> 16).astype(np.uint16)
+    u = a.view(np.uint32)
+    # finite values never overflow 32 bits here (max 0xFF7FFFFF + 0x8000)
+    rounding_bias = ((u >> np.uint32(16)) & np.uint32(1)) + np.uint32(0x7FFF)
+    out = ((u + rounding_bias) >> np.uint32(16)).astype(np.uint16)
     nan = np.isnan(a)
     if nan.any():
         out[nan] = 0x7FC0

@@ -1,0 +1,197 @@
+/*
+ * nmsparse.h -- C ABI of the B200 (sm_100a) N:M-pruned linear layer.
+ *
+ * The hot path these calls implement, with the passage that defines each step
+ * (page title, section):
+ *   nm_hessian_diag   H_j = mean_t x_{t,j}^2, the diagonal Gauss-Newton proxy of
+ *                     the input activations. Sparsity Induction for Accurate
+ *                     Post-Training Pruning of LLMs (arXiv 2602.21652), sec. 2C
+ *                     "Efficientie: Snelle Hessian Update".
+ *   nm_score          s = (H + eps) * W^2. SparseForge (arXiv 2605.06402),
+ *                     "Estimativa de Importancia Consciente do Hessiano".
+ *                     With X == NULL: s = |W_latent|, Sparse-BitNet (arXiv
+ *                     2603.05168) sec. 2 "Geracao de Mascara Baseada em Magnitude".
+ *   nm_prune_compress keep the top-n scores of every group of m consecutive
+ *                     weights along the input dimension (ties -> lower index),
+ *                     compress the kept values, emit 2:4 metadata.
+ *                     SparseForge "Mistura Progressiva" (hard top-N target);
+ *                     Sparse-BitNet sec. 1 (N:M definition) and sec. 2
+ *                     ("Quantizar e depois Mascarar": the values compressed are
+ *                     whatever V the caller passes, e.g. ternary W_q).
+ *   slide_pack        (2N-2):2N -> N-1 overlapping width-4 windows at stride 2,
+ *                     each 2:4. SlideSparse (arXiv 2603.05232) sec. 2A.
+ *   lift_activations  X'[t, g*4(N-1) + 4w + i] = X[t, g*2N + 2w + i].
+ *                     SlideSparse sec. 2B "Elevacao de Ativacao".
+ *   nm_sparse_prepare canonical values + window metadata -> the GEMM's operand
+ *                     layout. SlideSparse sec. 2C item 2 (initialisation phase).
+ *   nm_sparse_gemm    Y = X * W_sparse^T on the sparse tensor cores; for
+ *                     (2N-2):2N the lift happens inside the GEMM's shared-memory
+ *                     staging. SlideSparse sec. 2C item 3 (online phase).
+ *   nm_dense_gemm     Y = X * W^T, dense tcgen05 GEMM (the comparison point).
+ *   nm_ternary_quantize  gamma = mean|W|, W_q = clip(rint(W/gamma),-1,1)*gamma.
+ *                     Sparse-BitNet sec. 1 item 1 (BitNet b1.58 ternary weights).
+ *
+ * Conventions shared by every call
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates nothing; its only state is one device error word.
+ *   - bf16 tensors are passed as uint16_t bit patterns.  Matrices are row-major
+ *     with a leading dimension (elements) ld >= the row length.
+ *   - X is [T x K] (tokens x in-features), W is [R x K] (out x in features),
+ *     Y is [T x R].  Groups of m run along K.  G = ceil(K/m), the tail group is
+ *     zero-padded (score 0, value 0).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and returns an nm_status.  Argument errors are detected on
+ *     the host before anything is launched; in that case nothing is launched and
+ *     no output is touched.  The library never aborts, exits or traps.
+ *   - Pointers given to TMA-fed calls (the GEMMs and nm_sparse_prepare's
+ *     output) must be 16-byte aligned and their leading dimensions multiples of
+ *     8 elements; other calls need 16-byte aligned X/W/S and ld % 8 == 0 too.
+ *     Violations return NM_ERR_ALIGN.
+ *   - Outputs are fully overwritten, padding included.
+ *   - Kernels that wait on barriers give up after about one second, record
+ *     NM_ERR_TIMEOUT in the device error word and return; read it with
+ *     nm_check_device_error.
+ */
+#ifndef NMSPARSE_H
+#define NMSPARSE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NM_OK = 0,
+    NM_ERR_NULL = 1,         /* a required pointer is NULL */
+    NM_ERR_SHAPE = 2,        /* a size is < 1, an ld is too small, or a size is too large */
+    NM_ERR_ALIGN = 3,        /* pointer not 16-byte aligned or ld not a multiple of 8 */
+    NM_ERR_UNSUPPORTED = 4,  /* n:m pattern not supported by this call */
+    NM_ERR_WORKSPACE = 5,    /* workspace or packed buffer smaller than required */
+    NM_ERR_CUDA = 6,         /* a CUDA runtime/driver call failed */
+    NM_ERR_TIMEOUT = 7,      /* a device-side barrier wait gave up (device error word) */
+    NM_ERR_DEVICE = 8        /* a device-side consistency check failed (device error word) */
+} nm_status;
+
+/* Human-readable name of a status code.  Never NULL. */
+const char *nm_status_string(int status);
+
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device.  Returns NM_OK, NM_ERR_TIMEOUT, NM_ERR_DEVICE or NM_ERR_CUDA. */
+nm_status nm_check_device_error(void *stream);
+
+/* Library version, (major << 16) | minor. */
+int nm_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* a1: diagonal Gauss-Newton proxy (Sparsity Induction, sec. 2C).
+ *   H[j] = (1/T) * sum_t X[t,j]^2 in fp64, summed in a fixed order: tokens in
+ *   chunks of 128 (each chunk in ascending t), chunk partials in ascending
+ *   chunk order, one correctly rounded division by T.  The result is therefore
+ *   bit-identical run to run and to any implementation of that order.
+ *   X  : [T x K] bf16, ldx >= K.          H : [K] fp64 (output).
+ *   ws : scratch of nm_hessian_workspace_bytes(T, K) bytes (may be NULL when
+ *        that is 0, i.e. T <= 128).  Contents on return are unspecified.   */
+size_t nm_hessian_workspace_bytes(int64_t T, int64_t K);
+nm_status nm_hessian_diag(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, double *H,
+                          void *ws, size_t ws_bytes, void *stream);
+
+/* a1 + a2: importance score (SparseForge, Hessian-aware importance).
+ *   X != NULL: H = nm_hessian_diag(X) (written to H, which must be non-NULL),
+ *              S[i,j] = fp32( (H[j] + eps) * W[i,j]^2 ), fp64 add and multiply,
+ *              one round-to-nearest-even to fp32.
+ *   X == NULL: S[i,j] = |W[i,j]| (latent-magnitude score; H, ws unused).
+ *   W : [R x K] bf16, ldw >= K.  S : [R x K] fp32, row stride K (output).
+ *   ws: as for nm_hessian_diag.                                             */
+nm_status nm_score(const uint16_t *X, int64_t T, int64_t ldx, const uint16_t *W, int64_t R,
+                   int64_t K, int64_t ldw, double eps, double *H, float *S, void *ws,
+                   size_t ws_bytes, void *stream);
+
+/* a2 only, from a given H: S[i,j] = fp32((H[j] + eps) * W[i,j]^2). */
+nm_status nm_score_from_hessian(const double *H, double eps, const uint16_t *W, int64_t R,
+                                int64_t K, int64_t ldw, float *S, void *stream);
+
+/* a3: group top-n selection, compression and 2:4 metadata.
+ *   S     : [R x K] fp32 scores (>= 0, finite), row stride lds >= K.
+ *   V     : [R x K] bf16 values to compress (W, or ternary W_q), ldv >= K.
+ *   n, m  : 1 <= n < m <= 16.
+ *   mask  : [R x ceil(G*m/32)] uint32 (output): bit (c%32) of word c/32 of a
+ *           row is set iff column c is kept (padding columns included; bits
+ *           past G*m are zero).
+ *   vals  : [R x G*n] bf16 (output): the kept values of each group in
+ *           ascending column order (a kept padding column stores 0).
+ *   meta24: [R x ceil(G/2)] bytes (output, only when m == 4, else may be NULL):
+ *           one nibble per group, idx0 | idx1 << 2 (idx0 < idx1), the even
+ *           group in the low nibble.
+ * Ties go to the lower column index; -0 and +0 tie.                         */
+nm_status nm_prune_compress(const float *S, int64_t lds, const uint16_t *V, int64_t ldv,
+                            int64_t R, int64_t K, int n, int m, uint32_t *mask, uint16_t *vals,
+                            uint8_t *meta24, void *stream);
+
+/* a4: sliding-window pack (SlideSparse, sec. 2A), m = 2N in {4, 6, 8, 10},
+ * n = m - 2.  Survivor k (0-based, ascending) of a group goes to window k/2,
+ * in-window index q_k - 2*(k/2) in [0, 3].  The window values are exactly
+ * nm_prune_compress's `vals`; only the metadata is new.
+ *   mask  : as written by nm_prune_compress with n = m - 2.
+ *   wmeta : [R x ceil(G*(N-1)/2)] bytes (output), one nibble idx0 | idx1 << 2
+ *           per window in (group, window) order, even window in the low nibble.
+ * A group that does not hold exactly m-2 survivors sets NM_ERR_DEVICE in the
+ * device error word (its nibbles are written as 0).                        */
+nm_status slide_pack(const uint32_t *mask, int64_t R, int64_t K, int m, uint8_t *wmeta,
+                     void *stream);
+
+/* a5 (standalone form): activation lifting (SlideSparse, sec. 2B).
+ *   XL[t, g*4(N-1) + 4w + i] = X[t, g*m + 2w + i], 0 where g*m+2w+i >= K.
+ *   X : [T x K] bf16, ldx >= K.  XL : [T x G*(N-1)*4] bf16, ldxl >= that.
+ * nm_sparse_gemm does this inside its staging; this call exists for tests and
+ * for the two-pass (lift, then GEMM on a 2:4 problem of width K') variant.  */
+nm_status lift_activations(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, int m,
+                           uint16_t *XL, int64_t ldxl, void *stream);
+
+/* a6: operand preparation (SlideSparse sec. 2C item 2, initialisation).
+ * Lays the window values and window metadata of a layer out in the order and
+ * tiling nm_sparse_gemm reads (padded rows and windows hold zero values and
+ * the index pair (0,1)).  For m == 4 the metadata is meta24 (identical to the
+ * window metadata of a 2:4 pattern).  The packed buffer is opaque; its size
+ * is nm_sparse_prepare_bytes(R, K, m).                                      */
+size_t nm_sparse_prepare_bytes(int64_t R, int64_t K, int m);
+nm_status nm_sparse_prepare(const uint16_t *vals, const uint8_t *wmeta, int64_t R, int64_t K,
+                            int m, void *packed, size_t packed_bytes, void *stream);
+
+/* a7: sparse GEMM (SlideSparse sec. 2C item 3; 2:4 sparse tensor cores).
+ *   Y[t, r] = sum_k X[t,k] * (mask (.) V)[r,k], fp32 accumulation in tensor
+ *   memory, bf16 output (round to nearest even).
+ *   X : [T x K] bf16, ldx >= K, ldx % 8 == 0.   Y : [T x R] bf16, ldy >= R.
+ *   packed: from nm_sparse_prepare(..., R, K, m, ...).  m in {4, 6, 8, 10};
+ *   for m > 4 the activations are lifted inside the kernel's shared-memory
+ *   staging (no X' in global memory).                                       */
+nm_status nm_sparse_gemm(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
+                         const void *packed, int64_t R, int m, uint16_t *Y, int64_t ldy,
+                         void *stream);
+
+/* a8: dense reference GEMM on the tensor cores, Y = X * W^T (W = mask (.) V
+ * densified by the caller), fp32 accumulation, bf16 output.                */
+nm_status nm_dense_gemm(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, const uint16_t *W,
+                        int64_t R, int64_t ldw, uint16_t *Y, int64_t ldy, void *stream);
+
+/* Ternary absmean quantisation (Sparse-BitNet sec. 1 item 1), input
+ * preparation of the ternary 6:8 layer.
+ *   gamma = (sum over rows, ascending, of each row's ascending-column sum of
+ *            |W|, in fp64) / (R*K);
+ *   q     = clip(rint(W / gamma), -1, 1) (fp64 division, ties to even);
+ *   W_q   = q * bf16(gamma), bf16(gamma) rounded to nearest even from fp64,
+ *           zeros stored as +0.
+ *   W : [R x K] bf16, ldw >= K.  Wq : [R x K] bf16 (output, row stride K).
+ *   gamma : one fp64 on the device (output).  ws : nm_ternary_workspace_bytes(R).
+ * If bf16(gamma) falls outside the normal bf16 range the device error word
+ * gets NM_ERR_DEVICE and Wq is all zero.                                    */
+size_t nm_ternary_workspace_bytes(int64_t R);
+nm_status nm_ternary_quantize(const uint16_t *W, int64_t R, int64_t K, int64_t ldw, uint16_t *Wq,
+                              double *gamma, void *ws, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NMSPARSE_H */

@@ -134,7 +134,7 @@ def prune(S: np.ndarray, V: np.ndarray, n: int, m: int):
     G = n_groups(K, m)
     mask = np.empty((R, mask_words(K, m)), dtype=np.uint32)
     vals = np.empty((R, G * n), dtype=np.uint16)
-    meta = np.empty((R, (G + 1) // 2), dtype=np.uint8) if m == 4 else None
+    meta = np.empty((R, (G + 1) // 2), dtype=np.uint8) if (m == 4 and n == 2) else None
     rc = _load().oracle_prune(_p(S), K, _p(V), K, R, K, n, m, _p(mask), _p(vals),
                               _p(meta) if meta is not None else None)
     if rc != 0:

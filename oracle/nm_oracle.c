@@ -139,7 +139,8 @@ void oracle_score_magnitude(const uint16_t *W, int64_t R, int64_t K, int64_t ldw
  * kept values in ascending column order, 2:4 metadata when m == 4.
  *   mask   : [R x ceil(G*m/32)] u32, bit (c % 32) of word c/32 = position c kept
  *   vals   : [R x G*n] bf16 bits
- *   meta24 : [R x ceil(G/2)] bytes, nibble idx0 | idx1<<2, even group low nibble
+ *   meta24 : [R x ceil(G/2)] bytes, only for 2:4 (n == 2, m == 4): nibble
+ *            idx0 | idx1<<2, even group in the low nibble
  * Returns 0, or -1 on an unsupported n:m or a non-finite / negative score.   */
 int oracle_prune(const float *S, int64_t lds, const uint16_t *V, int64_t ldv, int64_t R, int64_t K,
                  int n, int m, uint32_t *mask, uint16_t *vals, uint8_t *meta24) {
@@ -152,7 +153,7 @@ int oracle_prune(const float *S, int64_t lds, const uint16_t *V, int64_t ldv, in
     for (int64_t i = 0; i < R; ++i) {
         uint32_t *mrow = mask + i * mwords;
         memset(mrow, 0, (size_t)mwords * sizeof(uint32_t));
-        if (m == 4 && meta24) memset(meta24 + i * mbytes, 0, (size_t)mbytes);
+        if (m == 4 && n == 2 && meta24) memset(meta24 + i * mbytes, 0, (size_t)mbytes);
         for (int64_t g = 0; g < G; ++g) {
             float s[16];
             uint16_t v[16];
@@ -181,7 +182,7 @@ int oracle_prune(const float *S, int64_t lds, const uint16_t *V, int64_t ldv, in
                 vals[i * (G * n) + g * n + k] = v[idx[k]];
             }
             if (kept != n) bad = 1;
-            if (m == 4 && meta24) {
+            if (m == 4 && n == 2 && meta24) {
                 uint8_t nib = (uint8_t)(idx[0] | (idx[1] << 2));
                 meta24[i * mbytes + g / 2] |= (uint8_t)(nib << (4 * (g % 2)));
             }

@@ -1,0 +1,259 @@
+"""B200 (sm_100a) N:M-pruned linear layer: Python binding of libnmsparse.so.
+
+Argument marshalling only.  Every step of the path runs in the CUDA kernels of
+``libnmsparse.so`` (declared in ``include/nmsparse.h``); PyTorch supplies device
+memory and the current stream.  There is no CPU fallback: if the library is
+missing and cannot be built, importing the functions below raises.
+
+bf16 tensors may be given as ``torch.bfloat16`` or as ``torch.uint16`` /
+``torch.int16`` bit patterns; outputs are ``torch.bfloat16``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import build as _build
+
+__all__ = [
+    "NMError", "load", "hessian_diag", "score", "score_from_hessian", "prune_compress",
+    "slide_pack", "lift_activations", "sparse_prepare", "sparse_gemm", "dense_gemm",
+    "ternary_quantize", "check_device_error", "EXPORTED",
+]
+
+EXPORTED = (
+    "nm_status_string", "nm_check_device_error", "nm_version",
+    "nm_hessian_workspace_bytes", "nm_hessian_diag", "nm_score", "nm_score_from_hessian",
+    "nm_prune_compress", "slide_pack", "lift_activations", "nm_sparse_prepare_bytes",
+    "nm_sparse_prepare", "nm_sparse_gemm", "nm_dense_gemm", "nm_ternary_workspace_bytes",
+    "nm_ternary_quantize",
+)
+
+_P, _I64, _I, _D, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_size_t
+_SIGS = {
+    "nm_status_string": (ctypes.c_char_p, [_I]),
+    "nm_check_device_error": (_I, [_P]),
+    "nm_version": (_I, []),
+    "nm_hessian_workspace_bytes": (_SZ, [_I64, _I64]),
+    "nm_hessian_diag": (_I, [_P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "nm_score": (_I, [_P, _I64, _I64, _P, _I64, _I64, _I64, _D, _P, _P, _P, _SZ, _P]),
+    "nm_score_from_hessian": (_I, [_P, _D, _P, _I64, _I64, _I64, _P, _P]),
+    "nm_prune_compress": (_I, [_P, _I64, _P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P]),
+    "slide_pack": (_I, [_P, _I64, _I64, _I, _P, _P]),
+    "lift_activations": (_I, [_P, _I64, _I64, _I64, _I, _P, _I64, _P]),
+    "nm_sparse_prepare_bytes": (_SZ, [_I64, _I64, _I]),
+    "nm_sparse_prepare": (_I, [_P, _P, _I64, _I64, _I, _P, _SZ, _P]),
+    "nm_sparse_gemm": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I, _P, _I64, _P]),
+    "nm_dense_gemm": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _I64, _P]),
+    "nm_ternary_workspace_bytes": (_SZ, [_I64]),
+    "nm_ternary_quantize": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _SZ, _P]),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class NMError(RuntimeError):
+    pass
+
+
+def load() -> ctypes.CDLL:
+    """Load (building first if missing or stale) the CUDA library."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _build.build()
+            if not os.path.exists(path):
+                raise NMError(f"CUDA library not found at {path}")
+            lib = ctypes.CDLL(path)
+            for name, (res, args) in _SIGS.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        msg = load().nm_status_string(status).decode()
+        raise NMError(f"{what}: {msg}")
+
+
+def _stream(stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else t.data_ptr()
+
+
+def _dev(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise NMError(f"{name} must be a CUDA tensor")
+    return t
+
+
+def _bf16(t: torch.Tensor, name: str) -> torch.Tensor:
+    _dev(t, name)
+    if t.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
+        raise NMError(f"{name} must be bf16 (or 16-bit bit patterns), got {t.dtype}")
+    if t.stride(-1) != 1:
+        raise NMError(f"{name} must have unit stride in its last dimension")
+    return t
+
+
+def _ld(t: torch.Tensor) -> int:
+    return t.stride(0) if t.dim() == 2 else t.shape[-1]
+
+
+def check_device_error(stream=None):
+    """Synchronise and raise if a kernel recorded a timeout or a device check."""
+    _check(load().nm_check_device_error(_stream(stream)), "device error word")
+
+
+def hessian_diag(X, H=None, ws=None, stream=None):
+    X = _bf16(X, "X")
+    T, K = X.shape
+    lib = load()
+    if H is None:
+        H = torch.empty(K, dtype=torch.float64, device=X.device)
+    need = lib.nm_hessian_workspace_bytes(T, K)
+    if ws is None and need:
+        ws = torch.empty(need, dtype=torch.uint8, device=X.device)
+    _check(lib.nm_hessian_diag(_ptr(X), T, K, _ld(X), _ptr(H), _ptr(ws),
+                               ws.numel() * ws.element_size() if ws is not None else 0,
+                               _stream(stream)), "nm_hessian_diag")
+    return H
+
+
+def score_from_hessian(H, W, eps, S=None, stream=None):
+    W = _bf16(W, "W")
+    R, K = W.shape
+    if S is None:
+        S = torch.empty((R, K), dtype=torch.float32, device=W.device)
+    _check(load().nm_score_from_hessian(_ptr(H), float(eps), _ptr(W), R, K, _ld(W), _ptr(S),
+                                        _stream(stream)), "nm_score_from_hessian")
+    return S
+
+
+def score(X, W, eps=1e-8, H=None, S=None, ws=None, stream=None):
+    """Hessian-aware score (X given) or latent-magnitude score (X is None).
+    Returns (H or None, S)."""
+    W = _bf16(W, "W")
+    R, K = W.shape
+    lib = load()
+    if S is None:
+        S = torch.empty((R, K), dtype=torch.float32, device=W.device)
+    if X is None:
+        _check(lib.nm_score(None, 0, 0, _ptr(W), R, K, _ld(W), 0.0, None, _ptr(S), None, 0,
+                            _stream(stream)), "nm_score")
+        return None, S
+    X = _bf16(X, "X")
+    T = X.shape[0]
+    if X.shape[1] != K:
+        raise NMError("X and W disagree on K")
+    if H is None:
+        H = torch.empty(K, dtype=torch.float64, device=W.device)
+    need = lib.nm_hessian_workspace_bytes(T, K)
+    if ws is None and need:
+        ws = torch.empty(need, dtype=torch.uint8, device=W.device)
+    _check(lib.nm_score(_ptr(X), T, _ld(X), _ptr(W), R, K, _ld(W), float(eps), _ptr(H), _ptr(S),
+                        _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)), "nm_score")
+    return H, S
+
+
+def n_groups(K, m):
+    return (K + m - 1) // m
+
+
+def prune_compress(S, V, n, m, K=None, stream=None):
+    """Returns (mask int32 [R x words], vals bf16 [R x G*n], meta24 uint8 or None)."""
+    _dev(S, "S")
+    V = _bf16(V, "V")
+    R, K = V.shape
+    G = n_groups(K, m)
+    dev = V.device
+    mask = torch.empty((R, (G * m + 31) // 32), dtype=torch.int32, device=dev)
+    vals = torch.empty((R, G * n), dtype=torch.bfloat16, device=dev)
+    meta = torch.empty((R, (G + 1) // 2), dtype=torch.uint8, device=dev) if (m == 4 and n == 2) else None
+    _check(load().nm_prune_compress(_ptr(S), S.stride(0), _ptr(V), _ld(V), R, K, n, m, _ptr(mask),
+                                    _ptr(vals), _ptr(meta), _stream(stream)), "nm_prune_compress")
+    return mask, vals, meta
+
+
+def slide_pack(mask, K, m, stream=None):
+    _dev(mask, "mask")
+    R = mask.shape[0]
+    nw = n_groups(K, m) * (m // 2 - 1)
+    wmeta = torch.empty((R, (nw + 1) // 2), dtype=torch.uint8, device=mask.device)
+    _check(load().slide_pack(_ptr(mask), R, K, m, _ptr(wmeta), _stream(stream)), "slide_pack")
+    return wmeta
+
+
+def lifted_cols(K, m):
+    return n_groups(K, m) * (m // 2 - 1) * 4
+
+
+def lift_activations(X, m, XL=None, stream=None):
+    X = _bf16(X, "X")
+    T, K = X.shape
+    KL = lifted_cols(K, m)
+    if XL is None:
+        XL = torch.empty((T, (KL + 7) // 8 * 8), dtype=torch.bfloat16, device=X.device)[:, :KL]
+    _check(load().lift_activations(_ptr(X), T, K, _ld(X), m, _ptr(XL), _ld(XL), _stream(stream)),
+           "lift_activations")
+    return XL
+
+
+def sparse_prepare(vals, wmeta, R, K, m, packed=None, stream=None):
+    lib = load()
+    need = lib.nm_sparse_prepare_bytes(R, K, m)
+    if need == 0:
+        raise NMError("nm_sparse_prepare_bytes: unsupported shape or pattern")
+    if packed is None:
+        packed = torch.empty(need, dtype=torch.uint8, device=vals.device)
+    _check(lib.nm_sparse_prepare(_ptr(vals), _ptr(wmeta), R, K, m, _ptr(packed),
+                                 packed.numel() * packed.element_size(), _stream(stream)),
+           "nm_sparse_prepare")
+    return packed
+
+
+def sparse_gemm(X, packed, R, m, Y=None, stream=None):
+    X = _bf16(X, "X")
+    T, K = X.shape
+    if Y is None:
+        Y = torch.empty((T, (R + 7) // 8 * 8), dtype=torch.bfloat16, device=X.device)[:, :R]
+    _check(load().nm_sparse_gemm(_ptr(X), T, K, _ld(X), _ptr(packed), R, m, _ptr(Y), _ld(Y),
+                                 _stream(stream)), "nm_sparse_gemm")
+    return Y
+
+
+def dense_gemm(X, W, Y=None, stream=None):
+    X = _bf16(X, "X")
+    W = _bf16(W, "W")
+    T, K = X.shape
+    R = W.shape[0]
+    if Y is None:
+        Y = torch.empty((T, (R + 7) // 8 * 8), dtype=torch.bfloat16, device=X.device)[:, :R]
+    _check(load().nm_dense_gemm(_ptr(X), T, K, _ld(X), _ptr(W), R, _ld(W), _ptr(Y), _ld(Y),
+                                _stream(stream)), "nm_dense_gemm")
+    return Y
+
+
+def ternary_quantize(W, stream=None):
+    """Returns (W_q bf16 [R x K], gamma fp64 device scalar)."""
+    W = _bf16(W, "W")
+    R, K = W.shape
+    lib = load()
+    Wq = torch.empty((R, K), dtype=torch.bfloat16, device=W.device)
+    gamma = torch.empty(1, dtype=torch.float64, device=W.device)
+    ws = torch.empty(lib.nm_ternary_workspace_bytes(R), dtype=torch.uint8, device=W.device)
+    _check(lib.nm_ternary_quantize(_ptr(W), R, K, _ld(W), _ptr(Wq), _ptr(gamma), _ptr(ws),
+                                   ws.numel(), _stream(stream)), "nm_ternary_quantize")
+    return Wq, gamma

@@ -1,0 +1,40 @@
+// nm_api.cu -- status strings, the device error word and library metadata.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "nm_common.cuh"
+
+namespace nm {
+__device__ uint32_t g_error_word = 0;
+}  // namespace nm
+
+extern "C" const char *nm_status_string(int status) {
+    switch (status) {
+        case NM_OK: return "NM_OK";
+        case NM_ERR_NULL: return "NM_ERR_NULL: a required pointer is NULL";
+        case NM_ERR_SHAPE: return "NM_ERR_SHAPE: invalid or too large size / leading dimension";
+        case NM_ERR_ALIGN: return "NM_ERR_ALIGN: pointer not 16-byte aligned or ld not a multiple of 8";
+        case NM_ERR_UNSUPPORTED: return "NM_ERR_UNSUPPORTED: n:m pattern not supported by this call";
+        case NM_ERR_WORKSPACE: return "NM_ERR_WORKSPACE: workspace or packed buffer too small";
+        case NM_ERR_CUDA: return "NM_ERR_CUDA: a CUDA call failed";
+        case NM_ERR_TIMEOUT: return "NM_ERR_TIMEOUT: a device-side barrier wait gave up";
+        case NM_ERR_DEVICE: return "NM_ERR_DEVICE: a device-side consistency check failed";
+        default: return "unknown nm_status";
+    }
+}
+
+extern "C" int nm_version(void) { return (1 << 16) | 0; }
+
+extern "C" nm_status nm_check_device_error(void *stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return NM_ERR_CUDA;
+    uint32_t word = 0;
+    if (cudaMemcpyFromSymbol(&word, nm::g_error_word, sizeof(word)) != cudaSuccess) return NM_ERR_CUDA;
+    if (word != 0) {
+        const uint32_t zero = 0;
+        if (cudaMemcpyToSymbol(nm::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return NM_ERR_CUDA;
+    }
+    if (word & nm::ERRBIT_TIMEOUT) return NM_ERR_TIMEOUT;
+    if (word & nm::ERRBIT_DEVICE) return NM_ERR_DEVICE;
+    return NM_OK;
+}

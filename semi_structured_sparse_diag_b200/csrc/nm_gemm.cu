@@ -1,0 +1,467 @@
+// nm_gemm.cu -- tcgen05 dense and 2:4-sparse GEMMs with TMA staging, the
+// SlideSparse activation lift fused into the shared-memory staging, and the
+// operand-preparation kernel.
+//
+// Problem: Y[T x R] = X[T x K] * W^T.  The tensor core computes D = A * B^T
+// with A = weight tile (128 rows of W, K-major), B = activation tile (BN
+// tokens, K-major) and D in tensor memory: lane = row of W, column = token.
+//
+// Sparse operand (SlideSparse, sec. 2A/2C): every width-4 window along the
+// lifted dimension K' holds exactly two kept weights, so W' is 2:4 and runs on
+// tcgen05.mma.sp: A holds 2 values per window (K'/2 per row), the 4-bit index
+// pair of each window sits in tensor memory (copied from shared memory with
+// tcgen05.cp).  For (2N-2):2N patterns the B tile is the lifted activation
+// X', built by four warps from a raw X tile in shared memory (sec. 2B).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "nm_common.cuh"
+
+namespace nm {
+
+constexpr int BM = 128;          // weight rows per tile (MMA M)
+constexpr int GEMM_THREADS = 256;
+constexpr int EBLK_BYTES = 2048; // metadata of 128 rows x 128 lifted columns
+
+// ---------------------------------------------------------------------------
+// packed operand layout (opaque to callers):
+//   [0, Rpad*KLpad)                  values, row-major [Rpad x KLpad/2] bf16
+//   [Rpad*KLpad, + Rpad*KLpad/8)     metadata blocks, (row tile, K' block)
+//                                    order, 2048 bytes each
+// KLpad = K' rounded up to 128, Rpad = R rounded up to 128.
+// ---------------------------------------------------------------------------
+struct PackedGeom {
+    int64_t G, nwin, KL, KLpad, Rpad, nkb, vals_bytes, meta_bytes;
+};
+
+__host__ __device__ inline PackedGeom packed_geom(int64_t R, int64_t K, int m) {
+    PackedGeom p;
+    p.G = (K + m - 1) / m;
+    p.nwin = p.G * (m / 2 - 1);
+    p.KL = p.nwin * 4;
+    p.KLpad = (p.KL + 127) / 128 * 128;
+    p.Rpad = (R + 127) / 128 * 128;
+    p.nkb = p.KLpad / 128;
+    p.vals_bytes = p.Rpad * p.KLpad;       // Rpad x KLpad/2 bf16
+    p.meta_bytes = p.Rpad * p.KLpad / 8;   // 4 bits per window of 4
+    return p;
+}
+
+// Metadata block byte b of a (128 row x 128 lifted column) tile holds the index
+// pairs of two adjacent windows of one row.  The order is the one
+// tcgen05.cp.128x128b + tcgen05.mma.sp expect for kind::f16 with M = 128:
+//   lane L = b/16 = m0 + 8*k1 + 16*m2, byte-in-lane = 4*k2 + 2*m1 + kh,
+//   row = m0 + 8*m1 + 16*m2, first lifted column = 8*kh + 16*k1 + 32*k2.
+// (k2 selects the tensor-memory column, i.e. the MMA k-step of 32 columns.)
+__host__ __device__ inline void meta_byte_coords(int b, int &row, int &col) {
+    const int L = b >> 4, within = b & 15;
+    const int k2 = within >> 2, m1 = (within >> 1) & 1, kh = within & 1;
+    const int m0 = L & 7, k1 = (L >> 3) & 1, m2 = L >> 4;
+    row = m0 + 8 * m1 + 16 * m2;
+    col = 8 * kh + 16 * k1 + 32 * k2;
+}
+
+__global__ void __launch_bounds__(256)
+    k_prepare_vals(const uint16_t *__restrict__ vals, int64_t R, int64_t rowlen, int64_t Rpad,
+                   int64_t KLh, uint16_t *__restrict__ out) {
+    const int64_t total = Rpad * KLh;
+    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = idx / KLh, c = idx - r * KLh;
+        out[idx] = (r < R && c < rowlen) ? vals[r * rowlen + c] : static_cast<uint16_t>(0);
+    }
+}
+
+__global__ void __launch_bounds__(256)
+    k_prepare_meta(const uint8_t *__restrict__ wmeta, int64_t R, int64_t nwin, int64_t wbytes,
+                   int64_t nkb, int64_t nblocks, uint8_t *__restrict__ out) {
+    const int64_t total = nblocks * EBLK_BYTES;
+    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t blk = idx / EBLK_BYTES;
+        const int b = static_cast<int>(idx - blk * EBLK_BYTES);
+        const int64_t mt = blk / nkb, kb = blk - mt * nkb;
+        int rl, cl;
+        meta_byte_coords(b, rl, cl);
+        const int64_t row = mt * BM + rl;
+        const int64_t wi = kb * 32 + cl / 4;  // even window index
+        uint32_t lo = 0x4u, hi = 0x4u;        // padding: pair (0,1) over zero values
+        if (row < R && wi < nwin) {
+            const uint32_t byte = wmeta[row * wbytes + wi / 2];
+            lo = byte & 0xFu;
+            if (wi + 1 < nwin) hi = byte >> 4;
+        }
+        out[idx] = static_cast<uint8_t>(lo | (hi << 4));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// GEMM kernel
+//   MODE_DENSE : A = W tile [128 x 64] per stage, 4 MMAs (K = 16 each).
+//   MODE_SP24  : A = packed values [128 x 64] (= 128 lifted columns), B = X
+//                tile [BN x 128] by TMA, E = 2 KB, 4 sparse MMAs (K = 32).
+//   MODE_SPLIFT: as MODE_SP24 but B is built by four warps from a raw X tile
+//                [BN x 128 columns] (natural window order).
+// Warp roles: 0 = TMA producer, 1 = MMA issuer + tensor-memory owner,
+// 4..7 = lift (MODE_SPLIFT) then epilogue (tensor memory -> bf16 -> TMA store).
+// ---------------------------------------------------------------------------
+enum { MODE_DENSE = 0, MODE_SP24 = 1, MODE_SPLIFT = 2 };
+
+template <int MODE, int BN>
+struct GemmCfg {
+    static constexpr bool SPARSE = MODE != MODE_DENSE;
+    static constexpr int A_BYTES = BM * 128;                              // 16 KB
+    static constexpr int B_BYTES = SPARSE ? BN * 256 : BN * 128;         // 128 or 64 K cols
+    static constexpr int X_BYTES = MODE == MODE_SPLIFT ? BN * 256 : 0;    // raw X, 128 cols
+    static constexpr int E_BYTES = SPARSE ? EBLK_BYTES : 0;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + X_BYTES + E_BYTES;
+    static constexpr int STAGES = MODE == MODE_DENSE ? 6 : (MODE == MODE_SP24 ? 4 : 2);
+    static constexpr int OUT_BYTES = BN * BM * 2;
+    static constexpr int TMEM_COLS = SPARSE ? (BN + 4 <= 256 ? 256 : 512) : (BN <= 128 ? 128 : 256);
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+    static constexpr uint32_t TX_BYTES = A_BYTES + (MODE == MODE_SPLIFT ? X_BYTES : B_BYTES) + E_BYTES;
+    static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+    static_assert(OUT_BYTES <= STAGE_BYTES * STAGES, "epilogue staging");
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+template <int MODE, int BN>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+           const __grid_constant__ CUtensorMap tmY, const uint8_t *__restrict__ meta, int64_t nkb,
+           int m, int nwin) {
+    using C = GemmCfg<MODE, BN>;
+    constexpr int S = C::STAGES;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S * C::STAGE_BYTES);
+    uint64_t *full = bars, *empty = bars + S, *lifted = bars + 2 * S, *accum = bars + 3 * S;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * S + 1);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int mt = blockIdx.x, nt = blockIdx.y;
+
+    auto stA = [&](int s) { return smem + s * C::STAGE_BYTES; };
+    auto stB = [&](int s) { return smem + s * C::STAGE_BYTES + C::A_BYTES; };
+    auto stX = [&](int s) { return smem + s * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES; };
+    auto stE = [&](int s) {
+        return smem + s * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES + C::X_BYTES;
+    };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&lifted[s], 4);
+        }
+        mbar_init(accum, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+        prefetch_tmap(&tmY);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t tmem_e = tmem_base + BN;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int64_t kb = 0;
+            for (; kb < nkb; ++kb) {
+                const int s = static_cast<int>(kb % S);
+                const uint32_t ph = static_cast<uint32_t>((kb / S) & 1);
+                if (kb >= S && !mbar_wait(&empty[s], ph ^ 1u)) { *abort_flag = 1; break; }
+                mbar_arrive_expect_tx(&full[s], C::TX_BYTES);
+                if (MODE == MODE_DENSE) {
+                    tma_load_2d(stA(s), &tmA, &full[s], static_cast<int32_t>(kb * 64), mt * BM);
+                    tma_load_2d(stB(s), &tmB, &full[s], static_cast<int32_t>(kb * 64), nt * BN);
+                } else {
+                    tma_load_2d(stA(s), &tmA, &full[s], static_cast<int32_t>(kb * 64), mt * BM);
+                    bulk_load(stE(s), meta + (static_cast<int64_t>(mt) * nkb + kb) * EBLK_BYTES,
+                              EBLK_BYTES, &full[s]);
+                    if (MODE == MODE_SP24) {
+                        tma_load_2d(stB(s), &tmB, &full[s], static_cast<int32_t>(kb * 128), nt * BN);
+                        tma_load_2d(stB(s) + BN * 128, &tmB, &full[s],
+                                    static_cast<int32_t>(kb * 128 + 64), nt * BN);
+                    } else {
+                        const int64_t g_first = (kb * 32) / nwin;
+                        const int32_t c0 = static_cast<int32_t>((g_first * m) & ~static_cast<int64_t>(7));
+                        tma_load_2d(stX(s), &tmB, &full[s], c0, nt * BN);
+                    }
+                }
+            }
+            if (*abort_flag) {  // let copies already issued land before exiting
+                const int64_t issued = kb;
+                for (int64_t j = (issued > S ? issued - S : 0); j < issued; ++j)
+                    mbar_wait(&full[j % S], static_cast<uint32_t>((j / S) & 1));
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = make_idesc_bf16(BM, BN, C::SPARSE, 0);
+            bool ok = true;
+            for (int64_t kb = 0; kb < nkb && ok; ++kb) {
+                const int s = static_cast<int>(kb % S);
+                const uint32_t ph = static_cast<uint32_t>((kb / S) & 1);
+                if (!mbar_wait(&full[s], ph)) { ok = false; break; }
+                if (MODE == MODE_SPLIFT && !mbar_wait(&lifted[s], ph)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(stA(s)), b0 = smem_u32(stB(s));
+                if (MODE == MODE_DENSE) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint64_t ad = make_sdesc(a0 + j * 32, 16, 1024, 2);
+                        const uint64_t bd = make_sdesc(b0 + j * 32, 16, 1024, 2);
+                        mma_bf16(tmem_base, ad, bd, idesc, (kb > 0 || j > 0) ? 1u : 0u);
+                    }
+                } else {
+                    tmem_cp_128x128b(tmem_e, make_sdesc(smem_u32(stE(s)), 2048, 128, 0));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint64_t ad = make_sdesc(a0 + j * 32, 16, 1024, 2);
+                        const uint64_t bd =
+                            make_sdesc(b0 + (j >> 1) * (BN * 128) + (j & 1) * 64, 16, 1024, 2);
+                        const uint32_t id = idesc | static_cast<uint32_t>(j & 1);
+                        mma_sp_bf16(tmem_base, ad, bd, tmem_e + (j & ~1), id,
+                                    (kb > 0 || j > 0) ? 1u : 0u);
+                    }
+                }
+                mma_commit(&empty[s]);
+            }
+            if (ok) mma_commit(accum);
+            else *abort_flag = 1;
+        }
+    } else if (warp >= 4) {
+        const int ew = warp - 4;
+        bool ok = true;
+        if (MODE == MODE_SPLIFT) {
+            // -------------------------------------------------------- lift
+            for (int64_t kb = 0; kb < nkb; ++kb) {
+                const int s = static_cast<int>(kb % S);
+                const uint32_t ph = static_cast<uint32_t>((kb / S) & 1);
+                ok = __all_sync(0xffffffffu, mbar_wait(&full[s], ph));
+                if (!ok) break;
+                const int64_t W0 = kb * 32;
+                const int64_t g_first = W0 / nwin;
+                const int64_t c0 = (g_first * m) & ~static_cast<int64_t>(7);
+                const int64_t wi = W0 + lane;
+                const int64_t g = wi / nwin;
+                const int w = static_cast<int>(wi - g * nwin);
+                const int src = static_cast<int>(g * m + 2 * w - c0);  // even, <= 124
+                const uint8_t *xs = stX(s);
+                uint8_t *bs = stB(s);
+                const int chunk = lane >> 1;  // 16-byte chunk = 2 windows
+                const int atom = chunk >> 3, cj = chunk & 7;
+                for (int r = ew; r < BN; r += 4) {
+                    const uint32_t *xrow = reinterpret_cast<const uint32_t *>(xs + r * 256);
+                    const uint32_t lo = xrow[src >> 1], hi = xrow[(src >> 1) + 1];
+                    uint8_t *dst = bs + atom * (BN * 128) + r * 128 + ((cj ^ (r & 7)) << 4) +
+                                   ((lane & 1) << 3);
+                    *reinterpret_cast<uint2 *>(dst) = make_uint2(lo, hi);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&lifted[s]);
+            }
+        }
+        // ------------------------------------------------------------ epilogue
+        // each warp owns 32 weight rows (its tensor-memory lane quarter) and
+        // stores them with its own TMA store: no cross-warp barrier.
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(accum, 0));
+        if (ok) {
+            tc_fence_after();
+            uint16_t *stage_out = reinterpret_cast<uint16_t *>(smem) + ew * (BN * 32);  // [BN][32]
+#pragma unroll 1
+            for (int cc = 0; cc < BN / 32; ++cc) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + cc * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const uint32_t b = pack_bf16x2(__uint_as_float(v[j]), 0.0f) & 0xFFFFu;
+                    stage_out[(cc * 32 + j) * 32 + lane] = static_cast<uint16_t>(b);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(&tmY, stage_out, mt * BM + ew * 32, nt * BN);
+                bulk_commit_group();
+                bulk_wait_group_read0();
+            }
+            __syncwarp();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace nm
+
+// ===========================================================================
+// host side: tensor maps and the C ABI
+// ===========================================================================
+using namespace nm;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows x cols] matrix with row stride ld
+bool make_tmap_bf16(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, int64_t ld,
+                    uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+template <int MODE, int BN>
+nm_status launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &y,
+                      const uint8_t *meta, int64_t nkb, int m, int nwin, int64_t R, int64_t T,
+                      cudaStream_t s) {
+    using C = GemmCfg<MODE, BN>;
+    static bool attr_done[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NM_ERR_CUDA;
+    if (!attr_done[dev]) {
+        if (cudaFuncSetAttribute(k_gemm<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES) != cudaSuccess)
+            return NM_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    const int64_t mt = (R + BM - 1) / BM, ntl = (T + BN - 1) / BN;
+    if (mt > 0x7FFFFFFF || ntl > 65535) return NM_ERR_SHAPE;
+    dim3 grid(static_cast<unsigned>(mt), static_cast<unsigned>(ntl));
+    k_gemm<MODE, BN><<<grid, GEMM_THREADS, C::SMEM_BYTES, s>>>(a, b, y, meta, nkb, m, nwin);
+    return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
+}
+
+constexpr int GEMM_BN = 128;
+
+}  // namespace
+
+extern "C" size_t nm_sparse_prepare_bytes(int64_t R, int64_t K, int m) {
+    if (R < 1 || K < 1 || (m != 4 && m != 6 && m != 8 && m != 10)) return 0;
+    const PackedGeom p = packed_geom(R, K, m);
+    return static_cast<size_t>(p.vals_bytes + p.meta_bytes);
+}
+
+extern "C" nm_status nm_sparse_prepare(const uint16_t *vals, const uint8_t *wmeta, int64_t R,
+                                       int64_t K, int m, void *packed, size_t packed_bytes,
+                                       void *stream) {
+    if (!vals || !wmeta || !packed) return NM_ERR_NULL;
+    if (R < 1 || K < 1) return NM_ERR_SHAPE;
+    if (m != 4 && m != 6 && m != 8 && m != 10) return NM_ERR_UNSUPPORTED;
+    if (!aligned16(packed)) return NM_ERR_ALIGN;
+    const PackedGeom p = packed_geom(R, K, m);
+    if (packed_bytes < static_cast<size_t>(p.vals_bytes + p.meta_bytes)) return NM_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t n = m - 2;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+    int64_t blocks = (p.Rpad * (p.KLpad / 2) + 255) / 256;
+    k_prepare_vals<<<static_cast<unsigned>(blocks < cap ? blocks : cap), 256, 0, s>>>(
+        vals, R, p.G * n, p.Rpad, p.KLpad / 2, static_cast<uint16_t *>(packed));
+    const int64_t nblocks = (p.Rpad / BM) * p.nkb;
+    blocks = (nblocks * EBLK_BYTES + 255) / 256;
+    k_prepare_meta<<<static_cast<unsigned>(blocks < cap ? blocks : cap), 256, 0, s>>>(
+        wmeta, R, p.nwin, (p.nwin + 1) / 2, p.nkb, nblocks,
+        static_cast<uint8_t *>(packed) + p.vals_bytes);
+    return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
+}
+
+extern "C" nm_status nm_sparse_gemm(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
+                                    const void *packed, int64_t R, int m, uint16_t *Y, int64_t ldy,
+                                    void *stream) {
+    if (!X || !packed || !Y) return NM_ERR_NULL;
+    if (T < 1 || K < 1 || R < 1 || ldx < K || ldy < R) return NM_ERR_SHAPE;
+    if (m != 4 && m != 6 && m != 8 && m != 10) return NM_ERR_UNSUPPORTED;
+    if (!aligned16(X) || !aligned16(Y) || !aligned16(packed) || (ldx % 8) != 0 || (ldy % 8) != 0)
+        return NM_ERR_ALIGN;
+    const PackedGeom p = packed_geom(R, K, m);
+    CUtensorMap ta, tb, ty;
+    if (!make_tmap_bf16(&ta, packed, p.Rpad, p.KLpad / 2, p.KLpad / 2, 64, BM, true))
+        return NM_ERR_CUDA;
+    if (!make_tmap_bf16(&ty, Y, T, R, ldy, 32, GEMM_BN, false)) return NM_ERR_CUDA;
+    const uint8_t *meta = static_cast<const uint8_t *>(packed) + p.vals_bytes;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (m == 4) {
+        if (!make_tmap_bf16(&tb, X, T, K, ldx, 64, GEMM_BN, true)) return NM_ERR_CUDA;
+        return launch_gemm<MODE_SP24, GEMM_BN>(ta, tb, ty, meta, p.nkb, m, 1, R, T, s);
+    }
+    if (!make_tmap_bf16(&tb, X, T, K, ldx, 128, GEMM_BN, false)) return NM_ERR_CUDA;
+    return launch_gemm<MODE_SPLIFT, GEMM_BN>(ta, tb, ty, meta, p.nkb, m,
+                                             static_cast<int>(m / 2 - 1), R, T, s);
+}
+
+extern "C" nm_status nm_dense_gemm(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
+                                   const uint16_t *W, int64_t R, int64_t ldw, uint16_t *Y,
+                                   int64_t ldy, void *stream) {
+    if (!X || !W || !Y) return NM_ERR_NULL;
+    if (T < 1 || K < 1 || R < 1 || ldx < K || ldw < K || ldy < R) return NM_ERR_SHAPE;
+    if (!aligned16(X) || !aligned16(W) || !aligned16(Y) || (ldx % 8) != 0 || (ldw % 8) != 0 ||
+        (ldy % 8) != 0)
+        return NM_ERR_ALIGN;
+    CUtensorMap ta, tb, ty;
+    if (!make_tmap_bf16(&ta, W, R, K, ldw, 64, BM, true)) return NM_ERR_CUDA;
+    if (!make_tmap_bf16(&tb, X, T, K, ldx, 64, GEMM_BN, true)) return NM_ERR_CUDA;
+    if (!make_tmap_bf16(&ty, Y, T, R, ldy, 32, GEMM_BN, false)) return NM_ERR_CUDA;
+    const int64_t nkb = (K + 63) / 64;
+    return launch_gemm<MODE_DENSE, GEMM_BN>(ta, tb, ty, nullptr, nkb, 4, 1, R, T,
+                                            reinterpret_cast<cudaStream_t>(stream));
+}

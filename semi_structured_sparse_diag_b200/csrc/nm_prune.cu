@@ -1,0 +1,603 @@
+// nm_prune.cu -- score, prune/compress, slide pack, lift and ternary kernels.
+//
+// All of these are HBM-streaming kernels: each reads its operand once with
+// coalesced vector loads and writes its outputs once.  Bit-exact by
+// construction with any implementation of the same definitions:
+//   * H uses a fixed summation order (chunks of 128 tokens);
+//   * S uses fp64 add/multiply with explicit round-to-nearest intrinsics (no
+//     FMA contraction) and one fp64 -> fp32 rounding;
+//   * selection is integer logic on fp32 comparisons.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "nm_common.cuh"
+
+namespace nm {
+
+constexpr int H_CHUNK = 128;   // tokens per partial sum of H
+constexpr int H_COLS = 2;      // columns per thread in the H reduction
+constexpr int H_THREADS = 256;
+constexpr int H_UNROLL = 16;
+
+__device__ __forceinline__ double bf16_to_f64(uint16_t b) {
+    return static_cast<double>(__uint_as_float(static_cast<uint32_t>(b) << 16));
+}
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// ---------------------------------------------------------------------------
+// a1: column sums of squares, one partial per chunk of 128 tokens.
+//   grid.x: column blocks of H_THREADS*H_COLS columns; grid.y: token chunk.
+//   When there is a single chunk the kernel writes H directly.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(H_THREADS) k_colsumsq_chunk(const uint16_t *__restrict__ X,
+                                                              int64_t T, int64_t K, int64_t ldx,
+                                                              double *__restrict__ out,
+                                                              int direct) {
+    const int64_t col = (static_cast<int64_t>(blockIdx.x) * H_THREADS + threadIdx.x) * H_COLS;
+    if (col >= K) return;
+    const int64_t t0 = static_cast<int64_t>(blockIdx.y) * H_CHUNK;
+    const int64_t t1 = t0 + H_CHUNK < T ? t0 + H_CHUNK : T;
+    double p0 = 0.0, p1 = 0.0;
+    const uint16_t *base = X + t0 * ldx + col;
+    if (col + 1 < K) {
+        int64_t t = t0;
+        for (; t + H_UNROLL <= t1; t += H_UNROLL) {
+            uint32_t v[H_UNROLL];
+#pragma unroll
+            for (int u = 0; u < H_UNROLL; ++u)
+                v[u] = __ldg(reinterpret_cast<const uint32_t *>(base + (t - t0 + u) * ldx));
+#pragma unroll
+            for (int u = 0; u < H_UNROLL; ++u) {
+                const double a = bf16_to_f64(static_cast<uint16_t>(v[u] & 0xFFFFu));
+                const double b = bf16_to_f64(static_cast<uint16_t>(v[u] >> 16));
+                p0 = __dadd_rn(p0, __dmul_rn(a, a));
+                p1 = __dadd_rn(p1, __dmul_rn(b, b));
+            }
+        }
+        for (; t < t1; ++t) {
+            const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(base + (t - t0) * ldx));
+            const double a = bf16_to_f64(static_cast<uint16_t>(v & 0xFFFFu));
+            const double b = bf16_to_f64(static_cast<uint16_t>(v >> 16));
+            p0 = __dadd_rn(p0, __dmul_rn(a, a));
+            p1 = __dadd_rn(p1, __dmul_rn(b, b));
+        }
+    } else {  // last single column
+        for (int64_t t = t0; t < t1; ++t) {
+            const double a = bf16_to_f64(__ldg(base + (t - t0) * ldx));
+            p0 = __dadd_rn(p0, __dmul_rn(a, a));
+        }
+    }
+    if (direct) {
+        const double dT = static_cast<double>(T);
+        out[col] = __ddiv_rn(p0, dT);
+        if (col + 1 < K) out[col + 1] = __ddiv_rn(p1, dT);
+    } else {
+        double *dst = out + static_cast<int64_t>(blockIdx.y) * K + col;
+        dst[0] = p0;
+        if (col + 1 < K) dst[1] = p1;
+    }
+}
+
+// sums the chunk partials in ascending chunk order, then divides by T
+__global__ void k_colsumsq_finish(const double *__restrict__ part, int64_t nchunks, int64_t T,
+                                  int64_t K, double *__restrict__ H) {
+    const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (j >= K) return;
+    double total = 0.0;
+    for (int64_t c = 0; c < nchunks; ++c) total = __dadd_rn(total, part[c * K + j]);
+    H[j] = __ddiv_rn(total, static_cast<double>(T));
+}
+
+// ---------------------------------------------------------------------------
+// a2: S = fp32((H + eps) * W^2) (or |W| when H == nullptr), 8 elements/thread.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float score_one(const double *__restrict__ H, double eps, int64_t j,
+                                           uint16_t wb) {
+    if (H == nullptr) return fabsf(bf16_to_f32(wb));
+    const double w = bf16_to_f64(wb);
+    const double h = __dadd_rn(__ldg(H + j), eps);
+    return __double2float_rn(__dmul_rn(h, __dmul_rn(w, w)));
+}
+
+__global__ void __launch_bounds__(256) k_score(const double *__restrict__ H, double eps,
+                                               const uint16_t *__restrict__ W, int64_t R,
+                                               int64_t K, int64_t ldw, float *__restrict__ S) {
+    const int64_t cpr = (K + 7) / 8;  // 8-element chunks per row
+    const int64_t total = R * cpr;
+    const bool vec_store = (K % 4) == 0;
+    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t i = idx / cpr;
+        const int64_t j0 = (idx - i * cpr) * 8;
+        const uint16_t *wrow = W + i * ldw;
+        float *srow = S + i * K;
+        if (j0 + 8 <= K) {
+            const uint4 wv = __ldg(reinterpret_cast<const uint4 *>(wrow + j0));
+            const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
+            float s[8];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                s[2 * u] = score_one(H, eps, j0 + 2 * u, static_cast<uint16_t>(wr[u] & 0xFFFFu));
+                s[2 * u + 1] = score_one(H, eps, j0 + 2 * u + 1, static_cast<uint16_t>(wr[u] >> 16));
+            }
+            if (vec_store) {
+                float4 *d = reinterpret_cast<float4 *>(srow + j0);
+                d[0] = make_float4(s[0], s[1], s[2], s[3]);
+                d[1] = make_float4(s[4], s[5], s[6], s[7]);
+            } else {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) srow[j0 + u] = s[u];
+            }
+        } else {
+            for (int64_t j = j0; j < K; ++j) srow[j] = score_one(H, eps, j, wrow[j]);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a3: group top-n + compression + 2:4 metadata.  One thread per group, one
+// block per (row, 256-group slice).  Mask words of a warp's 32 groups are
+// assembled in shared memory (32*m bits = m whole words, word-aligned).
+// ---------------------------------------------------------------------------
+constexpr int PRUNE_THREADS = 256;
+
+template <int M>
+__device__ __forceinline__ void load_group(const float *__restrict__ srow,
+                                           const uint16_t *__restrict__ vrow, int64_t c0,
+                                           int64_t K, int m_rt, float *s, uint16_t *v) {
+    const int m = M > 0 ? M : m_rt;
+    if (M > 0 && c0 + M <= K) {
+        if constexpr (M % 4 == 0) {
+#pragma unroll
+            for (int q = 0; q < M; q += 4) {
+                const float4 f = __ldg(reinterpret_cast<const float4 *>(srow + c0 + q));
+                s[q] = f.x; s[q + 1] = f.y; s[q + 2] = f.z; s[q + 3] = f.w;
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < M; q += 2) {
+                const float2 f = __ldg(reinterpret_cast<const float2 *>(srow + c0 + q));
+                s[q] = f.x; s[q + 1] = f.y;
+            }
+        }
+        if constexpr (M % 8 == 0) {
+#pragma unroll
+            for (int q = 0; q < M; q += 8) {
+                const uint4 u = __ldg(reinterpret_cast<const uint4 *>(vrow + c0 + q));
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    v[q + 2 * e] = static_cast<uint16_t>(w[e] & 0xFFFFu);
+                    v[q + 2 * e + 1] = static_cast<uint16_t>(w[e] >> 16);
+                }
+            }
+        } else if constexpr (M % 4 == 0) {
+#pragma unroll
+            for (int q = 0; q < M; q += 4) {
+                const uint2 u = __ldg(reinterpret_cast<const uint2 *>(vrow + c0 + q));
+                v[q] = u.x & 0xFFFFu; v[q + 1] = u.x >> 16; v[q + 2] = u.y & 0xFFFFu; v[q + 3] = u.y >> 16;
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < M; q += 2) {
+                const uint32_t u = __ldg(reinterpret_cast<const uint32_t *>(vrow + c0 + q));
+                v[q] = u & 0xFFFFu; v[q + 1] = u >> 16;
+            }
+        }
+    } else {
+        for (int q = 0; q < m; ++q) {
+            const int64_t c = c0 + q;
+            if (c < K) { s[q] = __ldg(srow + c); v[q] = __ldg(vrow + c); }
+            else { s[q] = 0.0f; v[q] = 0; }
+        }
+    }
+}
+
+template <int M>
+__global__ void __launch_bounds__(PRUNE_THREADS)
+    k_prune(const float *__restrict__ S, int64_t lds, const uint16_t *__restrict__ V, int64_t ldv,
+            int64_t K, int64_t G, int n, int m_rt, uint32_t *__restrict__ mask,
+            uint16_t *__restrict__ vals, uint8_t *__restrict__ meta24) {
+    const int m = M > 0 ? M : m_rt;
+    __shared__ uint32_t words[PRUNE_THREADS / 32][16];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t row = blockIdx.y;
+    const int64_t g = static_cast<int64_t>(blockIdx.x) * PRUNE_THREADS + threadIdx.x;
+    const bool valid = g < G;
+    const int64_t mwords = (G * m + 31) / 32;
+
+    if (lane < 16) words[warp][lane] = 0u;
+    __syncwarp();
+
+    float s[16];
+    uint16_t v[16];
+    uint32_t keepbits = 0;
+    uint32_t nib = 0;
+    if (valid) {
+        load_group<M>(S + row * lds, V + row * ldv, g * m, K, m, s, v);
+        int kept = 0;
+        uint16_t out[16];
+        int i0 = 0, i1 = 0;
+#pragma unroll
+        for (int q = 0; q < (M > 0 ? M : 16); ++q) {
+            if (q >= m) break;
+            int rank = 0;
+#pragma unroll
+            for (int p = 0; p < (M > 0 ? M : 16); ++p) {
+                if (p >= m) break;
+                rank += (s[p] > s[q] || (s[p] == s[q] && p < q)) ? 1 : 0;
+            }
+            if (rank < n) {
+                keepbits |= 1u << q;
+                if (kept == 0) i0 = q;
+                if (kept == 1) i1 = q;
+                out[kept++] = v[q];
+            }
+        }
+        nib = static_cast<uint32_t>(i0 | (i1 << 2));
+        // compressed values, ascending column order
+        uint16_t *dst = vals + row * (G * n) + g * n;
+        if (M == 4 && n == 2) {
+            *reinterpret_cast<uint32_t *>(dst) = out[0] | (static_cast<uint32_t>(out[1]) << 16);
+        } else if (n % 8 == 0 && ((G * n) % 8) == 0) {
+            for (int k = 0; k < n; k += 8)
+                *reinterpret_cast<uint4 *>(dst + k) = make_uint4(
+                    out[k] | (static_cast<uint32_t>(out[k + 1]) << 16),
+                    out[k + 2] | (static_cast<uint32_t>(out[k + 3]) << 16),
+                    out[k + 4] | (static_cast<uint32_t>(out[k + 5]) << 16),
+                    out[k + 6] | (static_cast<uint32_t>(out[k + 7]) << 16));
+        } else if (n % 2 == 0) {
+            for (int k = 0; k < n; k += 2)
+                *reinterpret_cast<uint32_t *>(dst + k) =
+                    out[k] | (static_cast<uint32_t>(out[k + 1]) << 16);
+        } else {
+            for (int k = 0; k < n; ++k) dst[k] = out[k];
+        }
+        // mask bits: this group's m bits at offset (g % 32) * m in the warp's words
+        const uint32_t off = static_cast<uint32_t>(lane) * m;
+        atomicOr(&words[warp][off >> 5], keepbits << (off & 31));
+        if ((off & 31) + m > 32) atomicOr(&words[warp][(off >> 5) + 1], keepbits >> (32 - (off & 31)));
+    }
+    __syncwarp();
+    const int64_t g_warp0 = g - lane;
+    const int64_t w0 = g_warp0 * m / 32;
+    if (lane < m && g_warp0 < G && w0 + lane < mwords) mask[row * mwords + w0 + lane] = words[warp][lane];
+
+    if (M == 4 && meta24 != nullptr && n == 2) {
+        const uint32_t other = __shfl_down_sync(0xffffffffu, nib, 1);
+        const int64_t mbytes = (G + 1) / 2;
+        if ((lane & 1) == 0 && valid) {
+            const uint32_t hi = (g + 1 < G) ? other : 0u;
+            meta24[row * mbytes + g / 2] = static_cast<uint8_t>(nib | (hi << 4));
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a4: sliding-window pack.  One thread per group; the window nibbles of a
+// warp's 32 groups are assembled in shared memory and written as bytes.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(PRUNE_THREADS)
+    k_slide_pack(const uint32_t *__restrict__ mask, int64_t G, int m, int64_t mwords,
+                 int64_t wbytes, uint8_t *__restrict__ wmeta) {
+    const int Ns = m / 2;
+    const int nwin = Ns - 1;
+    __shared__ uint32_t words[PRUNE_THREADS / 32][16];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t row = blockIdx.y;
+    const int64_t g = static_cast<int64_t>(blockIdx.x) * PRUNE_THREADS + threadIdx.x;
+    if (lane < 16) words[warp][lane] = 0u;
+    __syncwarp();
+    if (g < G) {
+        const int64_t b0 = g * m;
+        const uint32_t *mrow = mask + row * mwords;
+        const uint64_t lo = mrow[b0 >> 5];
+        const uint64_t hi = ((b0 >> 5) + 1 < mwords) ? mrow[(b0 >> 5) + 1] : 0u;
+        const uint32_t bits =
+            static_cast<uint32_t>(((hi << 32) | lo) >> (b0 & 31)) & ((1u << m) - 1u);
+        int q[16];
+        int cnt = 0;
+        for (int p = 0; p < m; ++p)
+            if ((bits >> p) & 1u) { if (cnt < 16) q[cnt] = p; ++cnt; }
+        uint32_t nibs = 0;  // nwin nibbles, window w at bits 4w
+        if (cnt != m - 2) {
+            raise_error(ERRBIT_DEVICE);
+        } else {
+            for (int w = 0; w < nwin; ++w) {
+                const int a = q[2 * w] - 2 * w, b = q[2 * w + 1] - 2 * w;
+                if (a < 0 || b > 3 || a >= b) { raise_error(ERRBIT_DEVICE); nibs = 0; break; }
+                nibs |= static_cast<uint32_t>(a | (b << 2)) << (4 * w);
+            }
+        }
+        // warp-local bit offset of this group's first window nibble
+        const uint32_t off = static_cast<uint32_t>(lane) * nwin * 4;
+        const int nb = nwin * 4;
+        atomicOr(&words[warp][off >> 5], nibs << (off & 31));
+        if ((off & 31) + nb > 32) atomicOr(&words[warp][(off >> 5) + 1], nibs >> (32 - (off & 31)));
+    }
+    __syncwarp();
+    // this warp's windows start at window (g - lane) * nwin, an even index
+    const int64_t g_warp0 = g - lane;
+    if (g_warp0 < G) {
+        const int64_t byte0 = g_warp0 * nwin / 2;
+        const int nbytes = 16 * nwin;  // 32 groups * nwin nibbles / 2
+        for (int b = lane; b < nbytes; b += 32) {
+            if (byte0 + b < wbytes)
+                wmeta[row * wbytes + byte0 + b] =
+                    static_cast<uint8_t>((words[warp][b >> 2] >> (8 * (b & 3))) & 0xFFu);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a5 (standalone): activation lift.  One thread per (token, group); window w
+// of a group is the column pairs (w, w+1) of that group, as 32-bit words.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    k_lift(const uint16_t *__restrict__ X, int64_t T, int64_t K, int64_t ldx, int m, int64_t G,
+           uint16_t *__restrict__ XL, int64_t ldxl) {
+    const int Ns = m / 2, nwin = Ns - 1;
+    const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t t = blockIdx.y;
+    if (g >= G || t >= T) return;
+    const uint16_t *src = X + t * ldx + g * m;
+    uint16_t *dst = XL + t * ldxl + g * nwin * 4;
+    uint32_t x[8];  // m/2 column pairs
+    if (g * m + m <= K) {
+        for (int p = 0; p < Ns; ++p) x[p] = __ldg(reinterpret_cast<const uint32_t *>(src) + p);
+    } else {
+        for (int p = 0; p < Ns; ++p) {
+            const int64_t c = g * m + 2 * p;
+            const uint32_t a = c < K ? __ldg(src + 2 * p) : 0u;
+            const uint32_t b = c + 1 < K ? __ldg(src + 2 * p + 1) : 0u;
+            x[p] = a | (b << 16);
+        }
+    }
+    uint32_t *d32 = reinterpret_cast<uint32_t *>(dst);
+    for (int w = 0; w < nwin; ++w) {
+        d32[2 * w] = x[w];
+        d32[2 * w + 1] = x[w + 1];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// ternary absmean quantisation
+// ---------------------------------------------------------------------------
+__global__ void k_row_abs_sum(const uint16_t *__restrict__ W, int64_t R, int64_t K, int64_t ldw,
+                              double *__restrict__ rowsum) {
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= R) return;
+    const uint16_t *w = W + i * ldw;
+    double s = 0.0;
+    int64_t j = 0;
+    for (; j + 8 <= K; j += 8) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(w + j));
+        const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            s = __dadd_rn(s, fabs(bf16_to_f64(static_cast<uint16_t>(q[e] & 0xFFFFu))));
+            s = __dadd_rn(s, fabs(bf16_to_f64(static_cast<uint16_t>(q[e] >> 16))));
+        }
+    }
+    for (; j < K; ++j) s = __dadd_rn(s, fabs(bf16_to_f64(w[j])));
+    rowsum[i] = s;
+}
+
+// fp64 -> bf16 bits, round to nearest even, normal range only (0xFFFF if not
+// representable as a normal bf16 or zero).  From the IEEE-754 definition.
+__device__ uint32_t f64_to_bf16_bits(double v) {
+    const unsigned long long u = static_cast<unsigned long long>(__double_as_longlong(v));
+    const uint32_t sign = static_cast<uint32_t>(u >> 63) << 15;
+    const int biased = static_cast<int>((u >> 52) & 0x7FFull);
+    const unsigned long long frac = u & 0xFFFFFFFFFFFFFull;
+    if (biased == 0 && frac == 0) return sign;
+    int e = biased - 1023;
+    if (e < -126 || e > 127) return 0xFFFFu;
+    // significand with the implicit bit: 53 bits; bf16 keeps the top 8
+    const unsigned long long sig = frac | (1ull << 52);
+    unsigned long long top = sig >> 45;
+    const unsigned long long tail = sig & ((1ull << 45) - 1ull);
+    const bool up = tail > (1ull << 44) || (tail == (1ull << 44) && (top & 1ull));
+    top += up ? 1ull : 0ull;
+    if (top >> 8) { top >>= 1; ++e; }
+    if (e > 127) return 0xFFFFu;
+    return sign | (static_cast<uint32_t>(e + 127) << 7) | static_cast<uint32_t>(top & 0x7Full);
+}
+
+__global__ void k_gamma(const double *__restrict__ rowsum, int64_t R, int64_t K,
+                        double *__restrict__ gamma_out, uint32_t *__restrict__ gb_out) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    double total = 0.0;
+    for (int64_t i = 0; i < R; ++i) total = __dadd_rn(total, rowsum[i]);
+    const double gamma = __ddiv_rn(total, __dmul_rn(static_cast<double>(R), static_cast<double>(K)));
+    uint32_t gb = f64_to_bf16_bits(gamma);
+    if (gamma == 0.0 || gb == 0xFFFFu) {
+        raise_error(ERRBIT_DEVICE);
+        gb = 0xFFFFu;
+    }
+    *gamma_out = gamma;
+    *gb_out = gb;
+}
+
+__global__ void __launch_bounds__(256)
+    k_ternary_apply(const uint16_t *__restrict__ W, int64_t R, int64_t K, int64_t ldw,
+                    const double *__restrict__ gamma_p, const uint32_t *__restrict__ gb_p,
+                    uint16_t *__restrict__ Wq) {
+    const double gamma = *gamma_p;
+    const uint32_t gb = *gb_p;
+    const int64_t total = R * K;
+    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t i = idx / K, j = idx - i * K;
+        uint16_t out = 0;
+        if (gb != 0xFFFFu) {
+            double q = rint(__ddiv_rn(bf16_to_f64(W[i * ldw + j]), gamma));
+            q = q > 1.0 ? 1.0 : (q < -1.0 ? -1.0 : q);
+            out = q == 0.0 ? 0 : static_cast<uint16_t>(q > 0.0 ? gb : (gb | 0x8000u));
+        }
+        Wq[idx] = out;
+    }
+}
+
+}  // namespace nm
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+using namespace nm;
+
+namespace {
+
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline nm_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
+}
+
+inline int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+}  // namespace
+
+extern "C" size_t nm_hessian_workspace_bytes(int64_t T, int64_t K) {
+    if (T <= 0 || K <= 0) return 0;
+    const int64_t nchunks = (T + H_CHUNK - 1) / H_CHUNK;
+    return nchunks > 1 ? static_cast<size_t>(nchunks) * static_cast<size_t>(K) * sizeof(double) : 0;
+}
+
+extern "C" nm_status nm_hessian_diag(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
+                                     double *H, void *ws, size_t ws_bytes, void *stream) {
+    if (!X || !H) return NM_ERR_NULL;
+    if (T < 1 || K < 1 || ldx < K) return NM_ERR_SHAPE;
+    if (!aligned16(X) || (ldx % 8) != 0) return NM_ERR_ALIGN;
+    const size_t need = nm_hessian_workspace_bytes(T, K);
+    if (need > 0 && (!ws || ws_bytes < need)) return NM_ERR_WORKSPACE;
+    const int64_t nchunks = (T + H_CHUNK - 1) / H_CHUNK;
+    if (nchunks > 65535) return NM_ERR_SHAPE;
+    const int64_t col_threads = (K + H_COLS - 1) / H_COLS;
+    dim3 grid(static_cast<unsigned>((col_threads + H_THREADS - 1) / H_THREADS),
+              static_cast<unsigned>(nchunks));
+    cudaStream_t s = as_stream(stream);
+    if (nchunks == 1) {
+        k_colsumsq_chunk<<<grid, H_THREADS, 0, s>>>(X, T, K, ldx, H, 1);
+        return launch_status();
+    }
+    double *part = static_cast<double *>(ws);
+    k_colsumsq_chunk<<<grid, H_THREADS, 0, s>>>(X, T, K, ldx, part, 0);
+    k_colsumsq_finish<<<static_cast<unsigned>((K + 255) / 256), 256, 0, s>>>(part, nchunks, T, K, H);
+    return launch_status();
+}
+
+extern "C" nm_status nm_score_from_hessian(const double *H, double eps, const uint16_t *W,
+                                           int64_t R, int64_t K, int64_t ldw, float *S,
+                                           void *stream) {
+    if (!W || !S) return NM_ERR_NULL;
+    if (R < 1 || K < 1 || ldw < K) return NM_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(S) || (ldw % 8) != 0) return NM_ERR_ALIGN;
+    const int64_t work = R * ((K + 7) / 8);
+    int64_t blocks = (work + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+    if (blocks > cap) blocks = cap;
+    k_score<<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(H, eps, W, R, K, ldw, S);
+    return launch_status();
+}
+
+extern "C" nm_status nm_score(const uint16_t *X, int64_t T, int64_t ldx, const uint16_t *W,
+                              int64_t R, int64_t K, int64_t ldw, double eps, double *H, float *S,
+                              void *ws, size_t ws_bytes, void *stream) {
+    if (!W || !S) return NM_ERR_NULL;
+    if (R < 1 || K < 1 || ldw < K) return NM_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(S) || (ldw % 8) != 0) return NM_ERR_ALIGN;
+    if (X == nullptr) return nm_score_from_hessian(nullptr, 0.0, W, R, K, ldw, S, stream);
+    if (!H) return NM_ERR_NULL;
+    const nm_status st = nm_hessian_diag(X, T, K, ldx, H, ws, ws_bytes, stream);
+    if (st != NM_OK) return st;
+    return nm_score_from_hessian(H, eps, W, R, K, ldw, S, stream);
+}
+
+extern "C" nm_status nm_prune_compress(const float *S, int64_t lds, const uint16_t *V, int64_t ldv,
+                                       int64_t R, int64_t K, int n, int m, uint32_t *mask,
+                                       uint16_t *vals, uint8_t *meta24, void *stream) {
+    if (!S || !V || !mask || !vals) return NM_ERR_NULL;
+    if (m == 4 && n == 2 && !meta24) return NM_ERR_NULL;
+    if (R < 1 || K < 1 || lds < K || ldv < K) return NM_ERR_SHAPE;
+    if (m < 2 || m > 16 || n < 1 || n >= m) return NM_ERR_UNSUPPORTED;
+    if (!aligned16(S) || !aligned16(V) || !aligned16(vals) || !aligned16(mask) ||
+        (lds % 8) != 0 || (ldv % 8) != 0)
+        return NM_ERR_ALIGN;
+    if (R > 65535) return NM_ERR_SHAPE;
+    const int64_t G = (K + m - 1) / m;
+    dim3 grid(static_cast<unsigned>((G + PRUNE_THREADS - 1) / PRUNE_THREADS), static_cast<unsigned>(R));
+    cudaStream_t s = as_stream(stream);
+    uint8_t *meta = (m == 4 && n == 2) ? meta24 : nullptr;
+    switch (m) {
+        case 4: k_prune<4><<<grid, PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
+        case 6: k_prune<6><<<grid, PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
+        case 8: k_prune<8><<<grid, PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
+        case 10: k_prune<10><<<grid, PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
+        default: k_prune<0><<<grid, PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
+    }
+    return launch_status();
+}
+
+extern "C" nm_status slide_pack(const uint32_t *mask, int64_t R, int64_t K, int m, uint8_t *wmeta,
+                                void *stream) {
+    if (!mask || !wmeta) return NM_ERR_NULL;
+    if (R < 1 || K < 1) return NM_ERR_SHAPE;
+    if (m != 4 && m != 6 && m != 8 && m != 10) return NM_ERR_UNSUPPORTED;
+    if (R > 65535) return NM_ERR_SHAPE;
+    const int64_t G = (K + m - 1) / m;
+    const int64_t mwords = (G * m + 31) / 32;
+    const int64_t wbytes = (G * (m / 2 - 1) + 1) / 2;
+    dim3 grid(static_cast<unsigned>((G + PRUNE_THREADS - 1) / PRUNE_THREADS), static_cast<unsigned>(R));
+    k_slide_pack<<<grid, PRUNE_THREADS, 0, as_stream(stream)>>>(mask, G, m, mwords, wbytes, wmeta);
+    return launch_status();
+}
+
+extern "C" nm_status lift_activations(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, int m,
+                                      uint16_t *XL, int64_t ldxl, void *stream) {
+    if (!X || !XL) return NM_ERR_NULL;
+    if (m != 4 && m != 6 && m != 8 && m != 10) return NM_ERR_UNSUPPORTED;
+    const int64_t G = (K + m - 1) / m;
+    const int64_t KL = G * (m / 2 - 1) * 4;
+    if (T < 1 || K < 1 || ldx < K || ldxl < KL) return NM_ERR_SHAPE;
+    if (!aligned16(X) || !aligned16(XL) || (ldx % 8) != 0 || (ldxl % 8) != 0) return NM_ERR_ALIGN;
+    if (T > 65535) return NM_ERR_SHAPE;
+    dim3 grid(static_cast<unsigned>((G + 255) / 256), static_cast<unsigned>(T));
+    k_lift<<<grid, 256, 0, as_stream(stream)>>>(X, T, K, ldx, m, G, XL, ldxl);
+    return launch_status();
+}
+
+extern "C" size_t nm_ternary_workspace_bytes(int64_t R) {
+    return R > 0 ? static_cast<size_t>(R) * sizeof(double) + 16 : 0;
+}
+
+extern "C" nm_status nm_ternary_quantize(const uint16_t *W, int64_t R, int64_t K, int64_t ldw,
+                                         uint16_t *Wq, double *gamma, void *ws, size_t ws_bytes,
+                                         void *stream) {
+    if (!W || !Wq || !gamma || !ws) return NM_ERR_NULL;
+    if (R < 1 || K < 1 || ldw < K) return NM_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(ws) || (ldw % 8) != 0) return NM_ERR_ALIGN;
+    if (ws_bytes < nm_ternary_workspace_bytes(R)) return NM_ERR_WORKSPACE;
+    cudaStream_t s = as_stream(stream);
+    double *rowsum = static_cast<double *>(ws);
+    uint32_t *gb = reinterpret_cast<uint32_t *>(rowsum + R);
+    k_row_abs_sum<<<static_cast<unsigned>((R + 127) / 128), 128, 0, s>>>(W, R, K, ldw, rowsum);
+    k_gamma<<<1, 32, 0, s>>>(rowsum, R, K, gamma, gb);
+    int64_t blocks = (R * K + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+    if (blocks > cap) blocks = cap;
+    k_ternary_apply<<<static_cast<unsigned>(blocks), 256, 0, s>>>(W, R, K, ldw, gamma, gb, Wq);
+    return launch_status();
+}

@@ -1,0 +1,85 @@
+"""Host-side checks of the C ABI (no GPU needed): the library builds for
+sm_100a, loads, exports every function include/nmsparse.h declares, and its
+argument validation rejects bad calls before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import semi_structured_sparse_diag_b200 as nm
+from nm_testutil import packed_geometry
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "nmsparse.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([A-Za-z_]\w*)\s*\(", src, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "defined")))
+
+
+def test_header_matches_exports():
+    lib = nm.load()
+    decl = declared_functions()
+    assert len(decl) >= 14
+    assert sorted(nm.EXPORTED) == decl
+    for name in decl:
+        assert getattr(lib, name) is not None
+
+
+def test_status_strings_and_version():
+    lib = nm.load()
+    assert lib.nm_status_string(0) == b"NM_OK"
+    for code in range(1, 9):
+        assert lib.nm_status_string(code).startswith(b"NM_ERR_")
+    assert lib.nm_status_string(99) == b"unknown nm_status"
+    assert lib.nm_version() >> 16 == 1
+
+
+def test_size_queries():
+    lib = nm.load()
+    assert lib.nm_hessian_workspace_bytes(128, 512) == 0
+    assert lib.nm_hessian_workspace_bytes(129, 512) == 2 * 512 * 8
+    assert lib.nm_hessian_workspace_bytes(8192, 4096) == 64 * 4096 * 8
+    for (R, K, m) in ((256, 512, 4), (4096, 4096, 8), (131, 1003, 6), (28672, 8192, 10), (1, 1, 4)):
+        g = packed_geometry(R, K, m)
+        assert lib.nm_sparse_prepare_bytes(R, K, m) == g["vals_bytes"] + g["meta_bytes"]
+    assert lib.nm_sparse_prepare_bytes(256, 512, 5) == 0
+    assert lib.nm_sparse_prepare_bytes(0, 512, 4) == 0
+    assert lib.nm_ternary_workspace_bytes(100) >= 800
+
+
+# fake but 16-byte aligned device addresses: validation fails before any use
+A = 0x10000
+MIS = 0x10002
+
+
+@pytest.mark.parametrize("call,expect", [
+    (lambda l: l.nm_hessian_diag(None, 4, 4, 8, A, None, 0, None), 1),
+    (lambda l: l.nm_hessian_diag(A, 0, 4, 8, A, None, 0, None), 2),
+    (lambda l: l.nm_hessian_diag(A, 4, 9, 8, A, None, 0, None), 2),
+    (lambda l: l.nm_hessian_diag(MIS, 4, 4, 8, A, None, 0, None), 3),
+    (lambda l: l.nm_hessian_diag(A, 4, 4, 12, A, None, 0, None), 3),
+    (lambda l: l.nm_hessian_diag(A, 300, 4, 8, A, None, 0, None), 5),
+    (lambda l: l.nm_prune_compress(A, 8, A, 8, 4, 8, 2, 17, A, A, A, None), 4),
+    (lambda l: l.nm_prune_compress(A, 8, A, 8, 4, 8, 4, 4, A, A, A, None), 4),
+    (lambda l: l.nm_prune_compress(A, 8, A, 8, 4, 8, 2, 4, A, A, None, None), 1),
+    (lambda l: l.nm_prune_compress(A, 8, MIS, 8, 4, 8, 2, 4, A, A, A, None), 3),
+    (lambda l: l.slide_pack(A, 4, 8, 7, A, None), 4),
+    (lambda l: l.slide_pack(A, 4, 8, 12, A, None), 4),
+    (lambda l: l.lift_activations(A, 4, 8, 8, 5, A, 8, None), 4),
+    (lambda l: l.lift_activations(A, 4, 8, 8, 8, A, 8, None), 2),
+    (lambda l: l.nm_sparse_prepare(A, A, 4, 8, 4, A, 1, None), 5),
+    (lambda l: l.nm_sparse_prepare(A, A, 4, 8, 4, MIS, 1 << 20, None), 3),
+    (lambda l: l.nm_sparse_gemm(A, 4, 8, 8, A, 4, 9, A, 8, None), 4),
+    (lambda l: l.nm_sparse_gemm(A, 4, 8, 8, A, 4, 4, A, 12, None), 3),
+    (lambda l: l.nm_sparse_gemm(A, 4, 8, 4, A, 4, 4, A, 8, None), 2),
+    (lambda l: l.nm_dense_gemm(A, 4, 8, 8, None, 4, 8, A, 8, None), 1),
+    (lambda l: l.nm_dense_gemm(A, 4, 8, 8, A, 4, 8, MIS, 8, None), 3),
+    (lambda l: l.nm_ternary_quantize(A, 4, 8, 8, A, A, A, 1, None), 5),
+])
+def test_argument_validation(call, expect):
+    assert call(nm.load()) == expect

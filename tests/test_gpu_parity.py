@@ -1,0 +1,242 @@
+"""GPU parity: every C-ABI call of libnmsparse against the fp64 CPU oracle.
+
+Bit-exact for H, S, masks, values, metadata, window metadata, the lifted
+activations and the packed GEMM operand; GEMM outputs within
+max|Y - Y64| / max|Y64| <= 1e-2 of the oracle's fp64 product.
+"""
+import numpy as np
+import pytest
+import torch
+
+import datagen
+import oracle
+from nm_testutil import (bf16_to_f64, decode_packed, packed_geometry, rel_err, to_dev, to_host,
+                         to_host_u16, wmeta_nibbles)
+
+pytestmark = pytest.mark.gpu
+
+GEMM_TOL = 1e-2
+
+
+@pytest.fixture(scope="module")
+def nm():
+    import semi_structured_sparse_diag_b200 as nm
+    nm.load()
+    return nm
+
+
+def _sync_ok(nm):
+    torch.cuda.synchronize()
+    nm.check_device_error()
+
+
+# ---------------------------------------------------------------- a1 / a2
+@pytest.mark.parametrize("T,K,ld", [(128, 512, 512), (1000, 520, 520), (1, 7, 8), (129, 3, 8),
+                                    (2048, 4096, 4096), (300, 517, 528), (257, 96, 104)])
+def test_hessian_bitexact(nm, T, K, ld):
+    X = datagen.make_activations(T, K, seed=T + K, n_outliers=min(4, K))
+    H = nm.hessian_diag(to_dev(X, ld))
+    _sync_ok(nm)
+    assert np.array_equal(to_host(H), oracle.hessian_diag(X))
+
+
+@pytest.mark.parametrize("R,K,ld", [(256, 512, 512), (33, 1030, 1032), (5, 13, 16), (64, 4096, 4096)])
+def test_score_bitexact(nm, R, K, ld):
+    X = datagen.make_activations(77, K, seed=R, n_outliers=2)
+    W = datagen.make_weight(R, K, 0.02, seed=R + 1)
+    H, S = nm.score(to_dev(X), to_dev(W, ld), eps=1e-8)
+    _, Sm = nm.score(None, to_dev(W, ld))
+    _sync_ok(nm)
+    Ho = oracle.hessian_diag(X)
+    assert np.array_equal(to_host(H), Ho)
+    assert np.array_equal(to_host(S), oracle.score_hessian(Ho, W, 1e-8))
+    assert np.array_equal(to_host(Sm), oracle.score_magnitude(W))
+
+
+# ---------------------------------------------------------------- a3
+@pytest.mark.parametrize("n,m,R,K", [(2, 4, 64, 512), (6, 8, 33, 1030), (4, 6, 17, 1003),
+                                     (8, 10, 9, 207), (2, 4, 3, 9), (1, 4, 8, 64), (3, 4, 8, 60),
+                                     (2, 8, 5, 100), (5, 16, 4, 99), (1, 3, 6, 10), (6, 8, 128, 4096)])
+@pytest.mark.parametrize("kind", ["gauss", "ties"])
+def test_prune_bitexact(nm, n, m, R, K, kind):
+    W = datagen.make_weight(R, K, 0.02, seed=K + m)
+    if kind == "gauss":
+        S = oracle.score_magnitude(W)
+    else:
+        S = datagen.tie_heavy_scores(R, K, seed=n + m, levels=3)
+        S[:, ::7] = -0.0  # signed zeros tie with +0
+    ld = (K + 7) // 8 * 8
+    Sd = torch.from_numpy(np.pad(S, ((0, 0), (0, ld - K)))).cuda()[:, :K]
+    mask, vals, meta = nm.prune_compress(Sd, to_dev(W, ld), n, m)
+    _sync_ok(nm)
+    om, ov, ometa = oracle.prune(np.abs(S) if kind == "ties" else S, W, n, m)
+    assert np.array_equal(to_host(mask).view(np.uint32), om)
+    assert np.array_equal(to_host_u16(vals), ov)
+    if ometa is not None:
+        assert np.array_equal(to_host(meta), ometa)
+
+
+# ---------------------------------------------------------------- a4 / a5
+@pytest.mark.parametrize("m,R,K", [(4, 64, 512), (6, 20, 1003), (8, 33, 1030), (10, 9, 207),
+                                   (8, 4, 8), (6, 128, 4096), (10, 7, 8195)])
+def test_slide_pack_bitexact(nm, m, R, K):
+    W = datagen.make_weight(R, K, 0.02, seed=m * K)
+    S = oracle.score_magnitude(W)
+    om, ov, _ = oracle.prune(S, W, m - 2, m)
+    wm = nm.slide_pack(torch.from_numpy(om.view(np.int32)).cuda(), K, m)
+    _sync_ok(nm)
+    assert np.array_equal(to_host(wm), oracle.slide_pack(om, K, m))
+
+
+def test_slide_pack_flags_bad_mask(nm):
+    # a 5:8 mask is not (m-2):m: the kernel records NM_ERR_DEVICE, nothing hangs
+    S = np.zeros((1, 8), dtype=np.float32)
+    S[0, :5] = 1
+    om, _, _ = oracle.prune(S, datagen.f32_to_bf16_bits(np.ones((1, 8), np.float32)), 5, 8)
+    nm.slide_pack(torch.from_numpy(om.view(np.int32)).cuda(), 8, 8)
+    torch.cuda.synchronize()
+    with pytest.raises(nm.NMError, match="NM_ERR_DEVICE"):
+        nm.check_device_error()
+    nm.check_device_error()  # cleared
+
+
+@pytest.mark.parametrize("m,T,K", [(4, 16, 64), (6, 33, 1003), (8, 17, 1030), (10, 5, 207),
+                                   (8, 128, 4096), (6, 3, 9)])
+def test_lift_bitexact(nm, m, T, K):
+    X = datagen.make_activations(T, K, seed=T * m)
+    ld = (K + 7) // 8 * 8
+    XL = nm.lift_activations(to_dev(X, ld), m)
+    _sync_ok(nm)
+    assert np.array_equal(to_host_u16(XL), oracle.lift(X, m))
+
+
+# ---------------------------------------------------------------- a6
+@pytest.mark.parametrize("m,R,K", [(4, 256, 512), (8, 130, 1030), (6, 64, 1003), (10, 200, 2050),
+                                   (4, 1, 9)])
+def test_prepare_layout_bitexact(nm, m, R, K):
+    W = datagen.make_weight(R, K, 0.02, seed=R * m)
+    res = oracle.run_layer(None, W, m - 2, m, score="magnitude")
+    wm = res["meta24"] if m == 4 else res["wmeta"]
+    packed = nm.sparse_prepare(to_dev(res["vals"]), torch.from_numpy(wm).cuda(), R, K, m)
+    _sync_ok(nm)
+    g = packed_geometry(R, K, m)
+    assert packed.numel() == g["vals_bytes"] + g["meta_bytes"]
+    vals, nib, pad_ok = decode_packed(to_host(packed), R, K, m)
+    assert pad_ok
+    assert np.array_equal(vals, res["vals"])
+    assert np.array_equal(nib, wmeta_nibbles(wm, g["nwin"]))
+
+
+# ---------------------------------------------------------------- a7 / a8
+def _layer(R, K, T, n, m, seed, outliers=0):
+    X = datagen.make_activations(T, K, seed=seed, n_outliers=outliers)
+    W = datagen.make_weight(R, K, 0.02, seed=seed + 1)
+    res = oracle.run_layer(X, W, n, m)
+    return X, W, res
+
+
+def _gemm_sparse(nm, X, res, R, K, m, ldx=None):
+    wm = res["meta24"] if m == 4 else res["wmeta"]
+    packed = nm.sparse_prepare(to_dev(res["vals"]), torch.from_numpy(wm).cuda(), R, K, m)
+    Y = nm.sparse_gemm(to_dev(X, ldx), packed, R, m)
+    _sync_ok(nm)
+    return bf16_to_f64(to_host_u16(Y))
+
+
+@pytest.mark.parametrize("m,R,K,T", [(4, 256, 512, 128), (4, 130, 1030, 200), (4, 128, 128, 1),
+                                     (6, 256, 1536, 128), (8, 256, 1024, 128), (10, 256, 1280, 128),
+                                     (6, 131, 1003, 77), (8, 200, 1030, 257), (10, 129, 2050, 16),
+                                     (8, 384, 4096, 384)])
+def test_sparse_gemm_vs_oracle(nm, m, R, K, T):
+    X, W, res = _layer(R, K, T, m - 2, m, seed=R + K + T, outliers=2)
+    Y = _gemm_sparse(nm, X, res, R, K, m, ldx=(K + 7) // 8 * 8)
+    Y64 = oracle.gemm_masked(X, res["mask"], W, m)
+    assert rel_err(Y, Y64) <= GEMM_TOL
+
+
+@pytest.mark.parametrize("m", [6, 8, 10])
+def test_fused_lift_equals_two_pass(nm, m):
+    # lift_activations + a 2:4 GEMM of width K' gives the same fp32 tensor-core
+    # sums as the fused kernel (same K' order, same tiles): identical bits
+    R, K, T = 256, 1030, 130
+    X, W, res = _layer(R, K, T, m - 2, m, seed=m)
+    Yf = _gemm_sparse(nm, X, res, R, K, m, ldx=1032)
+    XL = nm.lift_activations(to_dev(X, 1032), m)
+    KL = XL.shape[1]
+    packed24 = nm.sparse_prepare(to_dev(res["vals"]), torch.from_numpy(res["wmeta"]).cuda(), R, KL, 4)
+    Y2 = nm.sparse_gemm(XL, packed24, R, 4)
+    _sync_ok(nm)
+    assert np.array_equal(bf16_to_f64(to_host_u16(Y2)), Yf)
+
+
+@pytest.mark.parametrize("R,K,T", [(256, 512, 128), (130, 1030, 200), (128, 64, 1), (384, 4096, 384)])
+def test_dense_gemm_vs_oracle_and_torch(nm, R, K, T):
+    X, W, res = _layer(R, K, T, 2, 4, seed=R * 3 + T)
+    Wd = oracle.dense_masked(res["mask"], W, K)
+    ld = (K + 7) // 8 * 8
+    Yd = nm.dense_gemm(to_dev(X, ld), to_dev(Wd, ld))
+    _sync_ok(nm)
+    Y = bf16_to_f64(to_host_u16(Yd))
+    Y64 = oracle.gemm_dense(X, Wd)
+    assert rel_err(Y, Y64) <= GEMM_TOL
+    Yt = (to_dev(X).float() @ to_dev(Wd).float().T).double().cpu().numpy()
+    assert rel_err(Y, Yt) <= GEMM_TOL
+
+
+# ---------------------------------------------------------------- ternary
+@pytest.mark.parametrize("R,K", [(64, 256), (11008 // 8, 4096 // 4), (3, 13)])
+def test_ternary_bitexact(nm, R, K):
+    W = datagen.make_weight(R, K, 0.02, seed=R)
+    ld = (K + 7) // 8 * 8
+    Wq, gamma = nm.ternary_quantize(to_dev(W, ld))
+    _sync_ok(nm)
+    g, oWq = oracle.ternary(W)
+    assert to_host(gamma)[0] == g
+    assert np.array_equal(to_host_u16(Wq), oWq)
+
+
+# ---------------------------------------------------------------- whole path
+def _device_pipeline(nm, X, W, n, m, eps=1e-8, score="hessian", ternary=False):
+    Xd, Wd = to_dev(X), to_dev(W)
+    V = Wd
+    if ternary:
+        V, _ = nm.ternary_quantize(Wd)
+    H, S = nm.score(Xd if score == "hessian" else None, Wd, eps=eps)
+    mask, vals, meta = nm.prune_compress(S, V, n, m)
+    wm = meta if m == 4 else nm.slide_pack(mask, W.shape[1], m)
+    packed = nm.sparse_prepare(vals, wm, W.shape[0], W.shape[1], m)
+    Y = nm.sparse_gemm(Xd, packed, W.shape[0], m)
+    _sync_ok(nm)
+    return dict(H=H, S=S, mask=mask, vals=vals, wm=wm, Y=Y, V=V)
+
+
+def _check_pipeline(nm, layer, n_rows=64):
+    X, W = datagen.layer_inputs(layer)
+    out = _device_pipeline(nm, X, W, layer.n, layer.m, layer.eps, layer.score, layer.ternary)
+    ref = oracle.run_layer(X, W, layer.n, layer.m, layer.eps, layer.score, layer.ternary)
+    if ref["H"] is not None:
+        assert np.array_equal(to_host(out["H"]), ref["H"])
+    assert np.array_equal(to_host(out["mask"]).view(np.uint32), ref["mask"])
+    assert np.array_equal(to_host_u16(out["vals"]), ref["vals"])
+    wm_ref = ref["meta24"] if layer.m == 4 else ref["wmeta"]
+    assert np.array_equal(to_host(out["wm"]), wm_ref)
+    rows = np.sort(np.random.default_rng(layer.T).choice(layer.T, size=min(n_rows, layer.T), replace=False))
+    Y = bf16_to_f64(to_host_u16(out["Y"][torch.from_numpy(rows).cuda()]))
+    Y64 = oracle.gemm_masked(X, ref["mask"], ref["V"], layer.m, rows=rows)
+    assert rel_err(Y, Y64) <= GEMM_TOL
+    # every output row is finite and the unsampled rows are not left unwritten
+    Yall = out["Y"].float()
+    assert torch.isfinite(Yall).all()
+
+
+@pytest.mark.parametrize("name", ["small_2of4", "slide_6of8_4096", "ternary_6of8_gate",
+                                  "llama7b_q_T8192", "llama7b_gate_T2048", "llama7b_down_T128",
+                                  "llama7b_q_T16"])
+def test_workload_pipeline(nm, name):
+    _check_pipeline(nm, datagen.WORKLOADS[name], n_rows=128 if name == "small_2of4" else 32)
+
+
+@pytest.mark.parametrize("name", ["llama70b_up_4of6", "llama70b_down_8of10",
+                                  "llama70b_up_2of4", "llama70b_down_6of8"])
+def test_workload_pipeline_70b(nm, name):
+    _check_pipeline(nm, datagen.WORKLOADS[name], n_rows=8)
