@@ -44,7 +44,7 @@ def test_hessian_bitexact(nm, T, K, ld):
 def test_score_bitexact(nm, R, K, ld):
     X = datagen.make_activations(77, K, seed=R, n_outliers=2)
     W = datagen.make_weight(R, K, 0.02, seed=R + 1)
-    H, S = nm.score(to_dev(X), to_dev(W, ld), eps=1e-8)
+    H, S = nm.score(to_dev(X, ld), to_dev(W, ld), eps=1e-8)
     _, Sm = nm.score(None, to_dev(W, ld))
     _sync_ok(nm)
     Ho = oracle.hessian_diag(X)
