@@ -33,7 +33,8 @@
  *
  * Conventions shared by every call
  *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
- *     allocates nothing; its only state is one device error word.
+ *     allocates nothing; its only state is one device error word and the static
+ *     scratch array of nm_hessian_diag_noalloc.
  *   - bf16 tensors are passed as uint16_t bit patterns.  Matrices are row-major
  *     with a leading dimension (elements) ld >= the row length.
  *   - X is [T x K] (tokens x in-features), W is [R x K] (out x in features),
@@ -71,7 +72,8 @@ typedef enum {
     NM_ERR_WORKSPACE = 5,    /* workspace or packed buffer smaller than required */
     NM_ERR_CUDA = 6,         /* a CUDA runtime/driver call failed */
     NM_ERR_TIMEOUT = 7,      /* a device-side barrier wait gave up (device error word) */
-    NM_ERR_DEVICE = 8        /* a device-side consistency check failed (device error word) */
+    NM_ERR_DEVICE = 8,       /* a device-side consistency check failed (device error word) */
+    NM_ERR_TOO_LARGE = 9     /* problem needs more than an allocation-free call's static scratch */
 } nm_status;
 
 /* Human-readable name of a status code.  Never NULL. */
@@ -96,6 +98,32 @@ int nm_version(void);
 size_t nm_hessian_workspace_bytes(int64_t T, int64_t K);
 nm_status nm_hessian_diag(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, double *H,
                           void *ws, size_t ws_bytes, void *stream);
+
+/* Allocation-free variant of nm_hessian_diag.  The papers have no counterpart:
+ * this is a convenience of this library for callers that cannot allocate
+ * device memory -- for example a plugin running inside a host framework that
+ * owns all device memory and hands its plugins no allocator, or a
+ * latency-critical loop where a cudaMalloc/cudaFree (which may synchronise the
+ * device) is not acceptable.  It computes exactly what nm_hessian_diag computes
+ * (same kernels, same summation order, bit-identical H) but keeps the chunk
+ * partial sums in a fixed scratch array inside the library instead of a
+ * caller-provided workspace.  The caller still passes X and H.
+ *   Limit: ceil(T/128) * K <= NM_HESSIAN_NOALLOC_MAX_PARTIALS (8 MiB of fp64
+ *   partials, e.g. T = 4096 with K up to 32768, or T = 8192 with K up to
+ *   16384); larger problems return NM_ERR_TOO_LARGE and launch nothing.
+ *   Memory: the scratch is a static device array; every GPU that loads the
+ *   library holds those 8 MiB until the process exits.
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (with that device current); make that first call before any stream
+ *   capture.  It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   Sharing: all calls on a device share the one array and it keeps the last
+ *   call's contents (every partial is written before it is read, so nothing
+ *   needs clearing).  Calls whose kernels may overlap on the GPU -- on
+ *   different streams, or from different host threads -- race on the array
+ *   and must be serialised by the caller.                                   */
+#define NM_HESSIAN_NOALLOC_MAX_PARTIALS 1048576
+nm_status nm_hessian_diag_noalloc(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, double *H,
+                                  void *stream);
 
 /* a1 + a2: importance score (SparseForge, Hessian-aware importance).
  *   X != NULL: H = nm_hessian_diag(X) (written to H, which must be non-NULL),

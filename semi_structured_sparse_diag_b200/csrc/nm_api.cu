@@ -19,6 +19,7 @@ extern "C" const char *nm_status_string(int status) {
         case NM_ERR_CUDA: return "NM_ERR_CUDA: a CUDA call failed";
         case NM_ERR_TIMEOUT: return "NM_ERR_TIMEOUT: a device-side barrier wait gave up";
         case NM_ERR_DEVICE: return "NM_ERR_DEVICE: a device-side consistency check failed";
+        case NM_ERR_TOO_LARGE: return "NM_ERR_TOO_LARGE: problem exceeds the static scratch of an allocation-free call";
         default: return "unknown nm_status";
     }
 }

@@ -10,6 +10,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "nm_common.cuh"
 
 namespace nm {
@@ -599,5 +601,61 @@ extern "C" nm_status nm_ternary_quantize(const uint16_t *W, int64_t R, int64_t K
     const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
     if (blocks > cap) blocks = cap;
     k_ternary_apply<<<static_cast<unsigned>(blocks), 256, 0, s>>>(W, R, K, ldw, gamma, gb, Wq);
+    return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free H reduction: the chunk partials live in this file-scope
+// device array instead of a caller workspace.  Host code must not pass the
+// array's name to a kernel (on the host it is only a stand-in symbol): its
+// device address is looked up once per device with cudaGetSymbolAddress.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) double g_hessian_noalloc_scratch[NM_HESSIAN_NOALLOC_MAX_PARTIALS];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+double *g_noalloc_ptr[kMaxDevices] = {};
+
+// device address of the scratch array for the current device (set-up on first use)
+nm_status noalloc_scratch(double **out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NM_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_hessian_noalloc_scratch) != cudaSuccess || p == nullptr)
+            return NM_ERR_CUDA;
+        g_noalloc_ptr[dev] = static_cast<double *>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return NM_OK;
+}
+
+}  // namespace
+
+extern "C" nm_status nm_hessian_diag_noalloc(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
+                                             double *H, void *stream) {
+    if (!X || !H) return NM_ERR_NULL;
+    if (T < 1 || K < 1 || ldx < K) return NM_ERR_SHAPE;
+    if (!aligned16(X) || (ldx % 8) != 0) return NM_ERR_ALIGN;
+    const int64_t nchunks = (T + H_CHUNK - 1) / H_CHUNK;
+    if (nchunks > 65535) return NM_ERR_SHAPE;
+    if (nchunks > 1 && nchunks * K > static_cast<int64_t>(NM_HESSIAN_NOALLOC_MAX_PARTIALS))
+        return NM_ERR_TOO_LARGE;
+    const int64_t col_threads = (K + H_COLS - 1) / H_COLS;
+    dim3 grid(static_cast<unsigned>((col_threads + H_THREADS - 1) / H_THREADS),
+              static_cast<unsigned>(nchunks));
+    cudaStream_t s = as_stream(stream);
+    if (nchunks == 1) {
+        k_colsumsq_chunk<<<grid, H_THREADS, 0, s>>>(X, T, K, ldx, H, 1);
+        return launch_status();
+    }
+    double *part = nullptr;
+    const nm_status st = noalloc_scratch(&part);
+    if (st != NM_OK) return st;
+    k_colsumsq_chunk<<<grid, H_THREADS, 0, s>>>(X, T, K, ldx, part, 0);
+    k_colsumsq_finish<<<static_cast<unsigned>((K + 255) / 256), 256, 0, s>>>(part, nchunks, T, K, H);
     return launch_status();
 }
