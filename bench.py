@@ -446,6 +446,51 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_probe(args):
+    """Tensor-pipe and HBM probes (calibration, not the bench line)."""
+    import torch
+
+    import semi_structured_sparse_diag_b200 as nm
+    lib = nm.load()
+    dev = torch.device("cuda", 0)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    out = {"probe": "tcgen05 MMA-only loop and HBM copy", "sms": sms, "mma": [], "copy": None}
+    cyc = torch.zeros(sms, dtype=torch.int64, device=dev)
+    ns = torch.zeros(sms, dtype=torch.int64, device=dev)
+    s = torch.cuda.current_stream().cuda_stream
+    iters = 4096
+    clocks = ClockSampler(0)
+    for sparse in (0, 1):
+        for n in (128, 192, 256):
+            for rep in range(2):
+                st = lib.nm_probe_mma(sparse, n, sms, iters, cyc.data_ptr(), ns.data_ptr(), s)
+                if st != 0:
+                    raise nm.NMError(lib.nm_status_string(st).decode())
+                torch.cuda.synchronize()
+            nm.check_device_error()
+            kk = 32 if sparse else 16
+            flops_cta = 4.0 * iters * 2 * 128 * n * kk  # dense-equivalent (logical K)
+            t = ns.double().max().item() * 1e-9
+            c = cyc.double().median().item()
+            out["mma"].append({"sparse": sparse, "N": n, "tflops_dense_equiv": round(sms * flops_cta / t / 1e12, 1),
+                               "flop_per_clk_per_sm": round(flops_cta / c, 1),
+                               "clk_per_instr": round(c / (4 * iters), 2)})
+    nbytes = 2 << 30
+    a = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    b = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    best = 0.0
+    for _ in range(5):
+        e0.record()
+        st = lib.nm_probe_copy(a.data_ptr(), b.data_ptr(), nbytes, sms * 8, s)
+        e1.record()
+        torch.cuda.synchronize()
+        best = max(best, 2 * nbytes / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    out["copy"] = {"GB_per_s_read_plus_write": round(best, 1), "bytes": nbytes}
+    out["clocks"] = clocks.stop()
+    print(json.dumps(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -455,7 +500,11 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(datagen.WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--probe", action="store_true", help="run the tensor-pipe / HBM probes instead")
     args = ap.parse_args()
+    if args.probe:
+        run_probe(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

@@ -1,0 +1,46 @@
+/*
+ * nmsparse_probe.h -- measurement probes of libnmsparse (not part of the hot
+ * path; the papers have no counterpart).  They calibrate the roofline
+ * denominators on the chip the library runs on.
+ */
+#ifndef NMSPARSE_PROBE_H
+#define NMSPARSE_PROBE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "nmsparse.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Tensor-pipe probe: `ctas` CTAs (one per SM when ctas <= SM count) each issue
+ * 4*iters back-to-back tcgen05.mma (sparse = 0: kind::f16 M=128 K=16) or
+ * tcgen05.mma.sp (sparse = 1: M=128, K=32 logical) instructions with N = n
+ * (128, 192 or 256) on operands resident in shared memory, accumulating in
+ * tensor memory.  cycles[i] / nanos[i] (device arrays of `ctas` entries,
+ * caller-owned) receive CTA i's SM clock cycles and global-timer nanoseconds
+ * from the first issue to the completion of the last MMA.                   */
+nm_status nm_probe_mma(int sparse, int n, int ctas, int iters, unsigned long long *cycles,
+                       unsigned long long *nanos, void *stream);
+
+/* HBM probe: dst[i] = src[i] for `bytes` bytes (16-byte aligned, multiple of
+ * 16), grid of `blocks` CTAs of 256 threads with 16-byte streaming accesses. */
+nm_status nm_probe_copy(const void *src, void *dst, size_t bytes, int blocks, void *stream);
+
+/* Ablation baseline: the single-CTA, one-tile-per-CTA tcgen05 GEMM (128 x 128
+ * tiles, M = 128 instructions) that nm_sparse_gemm / nm_dense_gemm replace with
+ * the persistent CTA-pair kernel.  sparse = 1: W_or_packed is the output of
+ * nm_sparse_prepare(..., R, K, m = 4, ...) (ldw unused); sparse = 0: W_or_packed
+ * is a dense bf16 [R x K] matrix with leading dimension ldw.  Same arguments,
+ * alignment rules and output as the library GEMMs.                          */
+nm_status nm_gemm_1cta(int sparse, const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
+                       const void *W_or_packed, int64_t R, int64_t ldw, uint16_t *Y, int64_t ldy,
+                       void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NMSPARSE_PROBE_H */

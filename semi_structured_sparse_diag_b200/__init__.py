@@ -29,7 +29,7 @@ EXPORTED = (
     "nm_hessian_workspace_bytes", "nm_hessian_diag", "nm_score", "nm_score_from_hessian",
     "nm_prune_compress", "slide_pack", "lift_activations", "nm_sparse_prepare_bytes",
     "nm_sparse_prepare", "nm_sparse_gemm", "nm_dense_gemm", "nm_ternary_workspace_bytes",
-    "nm_ternary_quantize", "nm_hessian_diag_noalloc",
+    "nm_ternary_quantize", "nm_hessian_diag_noalloc", "nm_probe_mma", "nm_probe_copy", "nm_gemm_1cta",
 )
 
 _P, _I64, _I, _D, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_size_t
@@ -51,6 +51,9 @@ _SIGS = {
     "nm_ternary_workspace_bytes": (_SZ, [_I64]),
     "nm_ternary_quantize": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "nm_hessian_diag_noalloc": (_I, [_P, _I64, _I64, _I64, _P, _P]),
+    "nm_probe_mma": (_I, [_I, _I, _I, _I, _P, _P, _P]),
+    "nm_probe_copy": (_I, [_P, _P, _SZ, _I, _P]),
+    "nm_gemm_1cta": (_I, [_I, _P, _I64, _I64, _I64, _P, _I64, _I64, _P, _I64, _P]),
 }
 
 _lock = threading.Lock()

@@ -29,9 +29,23 @@ constexpr int EBLK_BYTES = 2048; // metadata of 128 rows x 128 lifted columns
 // ---------------------------------------------------------------------------
 // packed operand layout (opaque to callers):
 //   [0, Rpad*KLpad)                  values, row-major [Rpad x KLpad/2] bf16
-//   [Rpad*KLpad, + Rpad*KLpad/8)     metadata blocks, (row tile, K' block)
-//                                    order, 2048 bytes each
-// KLpad = K' rounded up to 128, Rpad = R rounded up to 128.
+//   [Rpad*KLpad, + Rpad*KLpad/8)     metadata blocks, (row tile of 128, K'
+//                                    block of 128) order, 2048 bytes each
+// Rpad = R rounded up to 256 (one CTA pair tile), KLpad = nkb * 128.
+//
+// K' order.  A K' block holds 32 windows ("slots") of 4 lifted columns.
+//   m = 4, 6, 10: natural order: slot s of block kb is window wi = 32*kb + s,
+//                 i.e. group wi / nwin, window wi % nwin (nwin = m/2 - 1).
+//   m = 8       : blocks come in threes per 32 groups (256 columns of X):
+//                 block 3j   : groups 32j .. 32j+15, windows 0 and 2 of each
+//                              group = columns 8g .. 8g+7 of X, in X's order;
+//                 block 3j+1 : groups 32j+16 .. 32j+31, likewise;
+//                 block 3j+2 : window 1 (columns 8g+2 .. 8g+5) of groups
+//                              32j .. 32j+31.
+//                 Blocks 3j and 3j+1 are plain tiles of X (TMA loads them into
+//                 the operand buffer); only block 3j+2 is built by the lift.
+// Any consistent K' order gives the same product, because A (values and
+// index pairs) and B (lifted activations) are permuted together.
 // ---------------------------------------------------------------------------
 struct PackedGeom {
     int64_t G, nwin, KL, KLpad, Rpad, nkb, vals_bytes, meta_bytes;
@@ -42,17 +56,38 @@ __host__ __device__ inline PackedGeom packed_geom(int64_t R, int64_t K, int m) {
     p.G = (K + m - 1) / m;
     p.nwin = p.G * (m / 2 - 1);
     p.KL = p.nwin * 4;
-    p.KLpad = (p.KL + 127) / 128 * 128;
-    p.Rpad = (R + 127) / 128 * 128;
-    p.nkb = p.KLpad / 128;
+    p.nkb = m == 8 ? 3 * ((p.G + 31) / 32) : (p.KL + 127) / 128;
+    p.KLpad = p.nkb * 128;
+    p.Rpad = (R + 255) / 256 * 256;
     p.vals_bytes = p.Rpad * p.KLpad;       // Rpad x KLpad/2 bf16
     p.meta_bytes = p.Rpad * p.KLpad / 8;   // 4 bits per window of 4
     return p;
 }
 
+// (group, window) held by slot s of K' block kb
+__host__ __device__ inline void slot_window(int m, int64_t kb, int s, int64_t &g, int &w) {
+    if (m == 8) {
+        const int64_t j = kb / 3;
+        const int type = static_cast<int>(kb - 3 * j);
+        if (type < 2) {
+            g = 32 * j + 16 * type + s / 2;
+            w = 2 * (s & 1);
+        } else {
+            g = 32 * j + s;
+            w = 1;
+        }
+    } else {
+        const int nwin = m / 2 - 1;
+        const int64_t wi = 32 * kb + s;
+        g = wi / nwin;
+        w = static_cast<int>(wi - g * nwin);
+    }
+}
+
 // Metadata block byte b of a (128 row x 128 lifted column) tile holds the index
-// pairs of two adjacent windows of one row.  The order is the one
-// tcgen05.cp.128x128b + tcgen05.mma.sp expect for kind::f16 with M = 128:
+// pairs of two adjacent slots of one row.  The order is the one
+// tcgen05.cp.128x128b + tcgen05.mma.sp expect for kind::f16 with 128 rows
+// per CTA:
 //   lane L = b/16 = m0 + 8*k1 + 16*m2, byte-in-lane = 4*k2 + 2*m1 + kh,
 //   row = m0 + 8*m1 + 16*m2, first lifted column = 8*kh + 16*k1 + 32*k2.
 // (k2 selects the tensor-memory column, i.e. the MMA k-step of 32 columns.)
@@ -65,20 +100,27 @@ __host__ __device__ inline void meta_byte_coords(int b, int &row, int &col) {
 }
 
 __global__ void __launch_bounds__(256)
-    k_prepare_vals(const uint16_t *__restrict__ vals, int64_t R, int64_t rowlen, int64_t Rpad,
-                   int64_t KLh, uint16_t *__restrict__ out) {
+    k_prepare_vals(const uint16_t *__restrict__ vals, int64_t R, int64_t G, int n, int m,
+                   int64_t Rpad, int64_t KLh, uint16_t *__restrict__ out) {
     const int64_t total = Rpad * KLh;
+    const int64_t rowlen = G * n;
     for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
          idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int64_t r = idx / KLh, c = idx - r * KLh;
-        out[idx] = (r < R && c < rowlen) ? vals[r * rowlen + c] : static_cast<uint16_t>(0);
+        int64_t g;
+        int w;
+        slot_window(m, c / 64, static_cast<int>((c % 64) / 2), g, w);
+        uint16_t v = 0;
+        if (r < R && g < G) v = vals[r * rowlen + g * n + 2 * w + (c & 1)];
+        out[idx] = v;
     }
 }
 
 __global__ void __launch_bounds__(256)
-    k_prepare_meta(const uint8_t *__restrict__ wmeta, int64_t R, int64_t nwin, int64_t wbytes,
+    k_prepare_meta(const uint8_t *__restrict__ wmeta, int64_t R, int64_t G, int m, int64_t wbytes,
                    int64_t nkb, int64_t nblocks, uint8_t *__restrict__ out) {
     const int64_t total = nblocks * EBLK_BYTES;
+    const int nwin = m / 2 - 1;
     for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
          idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int64_t blk = idx / EBLK_BYTES;
@@ -87,19 +129,23 @@ __global__ void __launch_bounds__(256)
         int rl, cl;
         meta_byte_coords(b, rl, cl);
         const int64_t row = mt * BM + rl;
-        const int64_t wi = kb * 32 + cl / 4;  // even window index
-        uint32_t lo = 0x4u, hi = 0x4u;        // padding: pair (0,1) over zero values
-        if (row < R && wi < nwin) {
-            const uint32_t byte = wmeta[row * wbytes + wi / 2];
-            lo = byte & 0xFu;
-            if (wi + 1 < nwin) hi = byte >> 4;
+        uint32_t nib[2] = {0x4u, 0x4u};  // padding: pair (0,1) over zero values
+        for (int h = 0; h < 2; ++h) {
+            int64_t g;
+            int w;
+            slot_window(m, kb, cl / 4 + h, g, w);
+            if (row < R && g < G) {
+                const int64_t wi = g * nwin + w;
+                nib[h] = (wmeta[row * wbytes + wi / 2] >> (4 * (wi & 1))) & 0xFu;
+            }
         }
-        out[idx] = static_cast<uint8_t>(lo | (hi << 4));
+        out[idx] = static_cast<uint8_t>(nib[0] | (nib[1] << 4));
     }
 }
 
 // ---------------------------------------------------------------------------
-// GEMM kernel
+// Single-CTA, one-tile-per-CTA GEMM (kept as the 1-CTA baseline of the
+// ablation entry point; the library's GEMMs use the CTA-pair kernel below).
 //   MODE_DENSE : A = W tile [128 x 64] per stage, 4 MMAs (K = 16 each).
 //   MODE_SP24  : A = packed values [128 x 64] (= 128 lifted columns), B = X
 //                tile [BN x 128] by TMA, E = 2 KB, 4 sparse MMAs (K = 32).
@@ -130,7 +176,7 @@ struct GemmCfg {
 
 template <int MODE, int BN>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
-    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    k_gemm_1cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const __grid_constant__ CUtensorMap tmY, const uint8_t *__restrict__ meta, int64_t nkb,
            int m, int nwin) {
     using C = GemmCfg<MODE, BN>;
@@ -314,6 +360,329 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
 }
 
+
+// ===========================================================================
+// Persistent CTA-pair GEMM (tcgen05 cta_group::2).
+//
+// A cluster of two CTAs computes 256 weight rows x 256 tokens per tile: CTA r
+// holds weight rows [128r, 128r+128) of the tile (its A) and tokens
+// [128r, 128r+128) (its half of B).  The leader CTA (rank 0) issues every
+// MMA; the tensor core reads A and B from both CTAs' shared memory, so each
+// CTA feeds only half of B -- for the sparse instruction this halves the
+// shared-memory reads per CTA and keeps the tensor pipe at its full rate
+// (shared memory feeds the tensor core at 128 bytes/clock/SM).
+//
+// Warp roles (both CTAs):
+//   warp 0      TMA producer: A (+ metadata E, + B where B is a plain tile of
+//               X), completion bytes signalled on the leader's full[s];
+//   warp 1      tensor-memory owner; in the leader also the MMA issuer;
+//   warps 4-11  epilogue: tensor memory -> bf16 -> TMA store, 32 weight rows
+//               x 128 tokens each;
+//   warps 12-15 lift (SLIFT / SP68 modes): build this CTA's lifted B half of a
+//               stage from X in global memory (SlideSparse sec. 2B), then
+//               arrive on the leader's lifted[s].
+// Stages: a ring of S shared-memory stages per CTA; empty[s] and acc_full[b]
+// are armed in both CTAs by multicast tcgen05.commit from the leader.
+// ===========================================================================
+enum { PMODE_DENSE = 0, PMODE_SP24 = 1, PMODE_SPLIFT = 2, PMODE_SP68 = 3 };
+
+template <int MODE>
+struct PairCfg {
+    static constexpr bool SPARSE = MODE != PMODE_DENSE;
+    static constexpr bool LIFT = MODE == PMODE_SPLIFT || MODE == PMODE_SP68;
+    static constexpr int BN = 256;                 // tokens per tile (both CTAs)
+    static constexpr int BH = 128;                 // tokens per CTA
+    static constexpr int A_BYTES = BM * 128;       // 128 rows x 128 bytes
+    static constexpr int B_BYTES = SPARSE ? BH * 256 : BH * 128;
+    static constexpr int E_BYTES = SPARSE ? EBLK_BYTES : 0;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + E_BYTES;
+    static constexpr int STAGES = SPARSE ? 4 : 6;
+    static constexpr int ACC_BUFS = SPARSE ? 1 : 2;     // accumulators of BN columns
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int TMEM_E = 256;                  // metadata columns (sparse)
+    static constexpr int EPI_WARPS = 8;
+    static constexpr int EPI_BYTES = EPI_WARPS * 32 * 32 * 2;
+    static constexpr int THREADS = LIFT ? 512 : 384;
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
+    static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+    static_assert(!SPARSE || TMEM_E >= ACC_BUFS * BN, "tensor memory");
+};
+
+__device__ __forceinline__ bool pair_needs_lift(int mode, int64_t kb) {
+    return mode == PMODE_SPLIFT || (mode == PMODE_SP68 && (kb % 3) == 2);
+}
+
+// B by TMA: the stage's B half is a plain tile of X
+__device__ __forceinline__ bool pair_b_by_tma(int mode, int64_t kb) {
+    return mode == PMODE_DENSE || mode == PMODE_SP24 || (mode == PMODE_SP68 && (kb % 3) != 2);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
+    k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
+                const uint16_t *__restrict__ X, int64_t T, int64_t K, int64_t ldx, int64_t R,
+                int64_t nkb, int m) {
+    using C = PairCfg<MODE>;
+    constexpr int S = C::STAGES;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    uint8_t *epi_smem = smem + S * C::STAGE_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(epi_smem + C::EPI_BYTES);
+    uint64_t *full = bars, *empty = bars + S, *lifted = bars + 2 * S;
+    uint64_t *acc_full = bars + 3 * S, *acc_empty = bars + 3 * S + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * S + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int64_t cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    const int64_t n_t = (T + C::BN - 1) / C::BN;
+    const int64_t n_m = (R + 255) / 256;
+    const int64_t ntiles = n_t * n_m;
+
+    auto stA = [&](int s) { return smem + s * C::STAGE_BYTES; };
+    auto stB = [&](int s) { return smem + s * C::STAGE_BYTES + C::A_BYTES; };
+    auto stE = [&](int s) { return smem + s * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES; };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&lifted[s], 8);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 2 * C::EPI_WARPS);
+        }
+        fence_barrier_init();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+        prefetch_tmap(&tmY);
+        if (C::SPARSE) prefetch_tmap(&tmE);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            int64_t it = 0;
+            bool ok = true;
+            for (int64_t tile = cluster; tile < ntiles && ok; tile += nclusters) {
+                const int64_t nt = tile % n_t, mt2 = tile / n_t;
+                const int32_t arow = static_cast<int32_t>(mt2 * 256 + rank * 128);
+                const int32_t brow = static_cast<int32_t>(nt * C::BN + rank * C::BH);
+                for (int64_t kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = static_cast<int>(it % S);
+                    const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
+                    if (it >= S && !mbar_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
+                    const bool btma = pair_b_by_tma(MODE, kb);
+                    if (rank == 0) {
+                        const uint32_t tx = 2u * static_cast<uint32_t>(
+                            C::A_BYTES + C::E_BYTES + (btma ? C::B_BYTES : 0));
+                        mbar_arrive_expect_tx(&full[s], tx);
+                    }
+                    const uint32_t bar = mapa_shared(&full[s], 0);
+                    tma_load_2d_pair(stA(s), &tmA, bar, static_cast<int32_t>(kb * 64), arow);
+                    if (C::SPARSE)
+                        tma_load_2d_pair(stE(s), &tmE, bar, 0,
+                                         static_cast<int32_t>(((mt2 * 2 + rank) * nkb + kb) * 8));
+                    if (btma) {
+                        if (MODE == PMODE_DENSE) {
+                            tma_load_2d_pair(stB(s), &tmB, bar, static_cast<int32_t>(kb * 64), brow);
+                        } else {
+                            const int64_t x0 = MODE == PMODE_SP24 ? kb * 128
+                                                                  : (kb / 3) * 256 + (kb % 3) * 128;
+                            tma_load_2d_pair(stB(s), &tmB, bar, static_cast<int32_t>(x0), brow);
+                            tma_load_2d_pair(stB(s) + C::BH * 128, &tmB, bar,
+                                             static_cast<int32_t>(x0 + 64), brow);
+                        }
+                    }
+                }
+            }
+            if (!ok && rank == 0) {  // let copies already issued land before exiting
+                for (int64_t j = (it > S ? it - S : 0); j < it; ++j)
+                    mbar_wait(&full[j % S], static_cast<uint32_t>((j / S) & 1));
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (rank == 0 && lane == 0) {
+            const uint32_t idesc = make_idesc_bf16(256, C::BN, C::SPARSE, 0);
+            int64_t it = 0, ti = 0;
+            uint32_t lbits = 0;
+            bool ok = true;
+            for (int64_t tile = cluster; tile < ntiles && ok; tile += nclusters, ++ti) {
+                const int buf = static_cast<int>(ti % C::ACC_BUFS);
+                const uint32_t aph = static_cast<uint32_t>((ti / C::ACC_BUFS) & 1);
+                if (ti >= C::ACC_BUFS && !mbar_wait_cluster(&acc_empty[buf], aph ^ 1u)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t dcol = tmem_base + static_cast<uint32_t>(buf * C::BN);
+                for (int64_t kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = static_cast<int>(it % S);
+                    const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
+                    if (!mbar_wait(&full[s], ph)) { ok = false; break; }
+                    if (pair_needs_lift(MODE, kb)) {
+                        if (!mbar_wait_cluster(&lifted[s], (lbits >> s) & 1u)) { ok = false; break; }
+                        lbits ^= 1u << s;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(stA(s)), b0 = smem_u32(stB(s));
+                    if (!C::SPARSE) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            mma_bf16_pair(dcol, make_sdesc(a0 + j * 32, 16, 1024, 2),
+                                          make_sdesc(b0 + j * 32, 16, 1024, 2), idesc,
+                                          (kb > 0 || j > 0) ? 1u : 0u);
+                    } else {
+                        const uint32_t te = tmem_base + C::TMEM_E;
+                        tmem_cp_128x128b_pair(te, make_sdesc(smem_u32(stE(s)), 2048, 128, 0));
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            mma_sp_bf16_pair(
+                                dcol, make_sdesc(a0 + j * 32, 16, 1024, 2),
+                                make_sdesc(b0 + (j >> 1) * (C::BH * 128) + (j & 1) * 64, 16, 1024, 2),
+                                te + (j & ~1), idesc | static_cast<uint32_t>(j & 1),
+                                (kb > 0 || j > 0) ? 1u : 0u);
+                    }
+                    mma_commit_pair(&empty[s]);
+                }
+                if (ok) mma_commit_pair(&acc_full[buf]);
+            }
+        }
+    } else if (warp >= 4 && warp < 12) {
+        // ---------------------------------------------------------- epilogue
+        const int q = warp & 3;              // tensor-memory lane quarter
+        const int h = (warp - 4) >> 2;       // token half of the tile
+        uint16_t *stage_out = reinterpret_cast<uint16_t *>(epi_smem) + (warp - 4) * 1024;
+        const uint32_t acc_empty_cl0 = mapa_shared(&acc_empty[0], 0);
+        const uint32_t acc_empty_cl1 = mapa_shared(&acc_empty[1], 0);
+        int64_t ti = 0;
+        for (int64_t tile = cluster; tile < ntiles; tile += nclusters, ++ti) {
+            const int64_t nt = tile % n_t, mt2 = tile / n_t;
+            const int buf = static_cast<int>(ti % C::ACC_BUFS);
+            const uint32_t aph = static_cast<uint32_t>((ti / C::ACC_BUFS) & 1);
+            if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], aph))) break;
+            tc_fence_after();
+            uint32_t packed[64];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                       static_cast<uint32_t>(buf * C::BN + h * 128 + c * 32),
+                                   v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    packed[c * 16 + i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(buf == 0 ? acc_empty_cl0 : acc_empty_cl1);
+            const int32_t yr = static_cast<int32_t>(mt2 * 256 + rank * 128 + q * 32);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (lane == 0) bulk_wait_group_read0();
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    stage_out[(2 * i) * 32 + lane] = static_cast<uint16_t>(packed[c * 16 + i] & 0xFFFFu);
+                    stage_out[(2 * i + 1) * 32 + lane] = static_cast<uint16_t>(packed[c * 16 + i] >> 16);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmY, stage_out, yr,
+                                 static_cast<int32_t>(nt * C::BN + h * 128 + c * 32));
+                    bulk_commit_group();
+                }
+            }
+        }
+        if (lane == 0) bulk_wait_group0();
+        __syncwarp();
+    } else if (C::LIFT && warp >= 12) {
+        // ---------------------------------------------------------- lift
+        const int lw = warp - 12;
+        const int nwin = m / 2 - 1;
+        int64_t it = 0;
+        bool ok = true;
+        for (int64_t tile = cluster; tile < ntiles && ok; tile += nclusters) {
+            const int64_t nt = tile % n_t;
+            const int64_t t0 = nt * C::BN + rank * C::BH;
+            for (int64_t kb = 0; kb < nkb; ++kb, ++it) {
+                if (!pair_needs_lift(MODE, kb)) continue;
+                const int s = static_cast<int>(it % S);
+                const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
+                if (it >= S && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u))) {
+                    ok = false;
+                    break;
+                }
+                int64_t g;
+                int w;
+                slot_window(m, kb, lane, g, w);
+                const int64_t col = g * m + 2 * w;  // first of the window's 4 columns
+                const bool full_cols = col + 4 <= K;
+                (void)nwin;
+                uint8_t *bs = stB(s);
+                const int chunk = (lane & 15) >> 1, atom = lane >> 4;
+                for (int r0 = lw; r0 < C::BH; r0 += 32) {
+                    uint32_t lo[8], hi[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int row = r0 + 4 * u;
+                        const int64_t t = t0 + row;
+                        lo[u] = 0u;
+                        hi[u] = 0u;
+                        if (t < T) {
+                            const uint16_t *src = X + t * ldx + col;
+                            if (full_cols) {
+                                lo[u] = __ldg(reinterpret_cast<const uint32_t *>(src));
+                                hi[u] = __ldg(reinterpret_cast<const uint32_t *>(src) + 1);
+                            } else {
+                                uint32_t e[4];
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) e[i] = col + i < K ? __ldg(src + i) : 0u;
+                                lo[u] = e[0] | (e[1] << 16);
+                                hi[u] = e[2] | (e[3] << 16);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int row = r0 + 4 * u;
+                        uint8_t *dst = bs + atom * (C::BH * 128) + row * 128 +
+                                       ((chunk ^ (row & 7)) << 4) + ((lane & 1) << 3);
+                        *reinterpret_cast<uint2 *>(dst) = make_uint2(lo[u], hi[u]);
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(&lifted[s], 0));
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    }
+}
+
 }  // namespace nm
 
 // ===========================================================================
@@ -342,57 +711,104 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D bf16 tensor map over a row-major [rows x cols] matrix with row stride ld
-bool make_tmap_bf16(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, int64_t ld,
-                    uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
+// 2-D tensor map over a row-major [rows x cols] matrix with row stride ld (elements)
+bool make_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, int esize, const void *base,
+                  int64_t rows, int64_t cols, int64_t ld, uint32_t box_cols, uint32_t box_rows,
+                  bool swizzle128) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * esize};
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
-                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+    CUresult r = fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
                     swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
-inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-inline int sm_count() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
+bool make_tmap_bf16(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, int64_t ld,
+                    uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
+    return make_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, rows, cols, ld, box_cols,
+                        box_rows, swizzle128);
 }
 
-template <int MODE, int BN>
-nm_status launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &y,
-                      const uint8_t *meta, int64_t nkb, int m, int nwin, int64_t R, int64_t T,
-                      cudaStream_t s) {
-    using C = GemmCfg<MODE, BN>;
-    static bool attr_done[64] = {};
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count() {
+    static int n[64] = {};
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NM_ERR_CUDA;
-    if (!attr_done[dev]) {
-        if (cudaFuncSetAttribute(k_gemm<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_BYTES) != cudaSuccess)
-            return NM_ERR_CUDA;
-        attr_done[dev] = true;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return 148;
+    if (n[dev] == 0) {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        n[dev] = v > 0 ? v : 148;
     }
+    return n[dev];
+}
+
+// one flag per kernel instantiation and device (kernels of different modes
+// share a signature, so the cache is keyed on the kernel itself)
+template <auto kernel>
+bool set_smem_attr(int bytes) {
+    static bool done[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    if (!done[dev]) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+            cudaSuccess)
+            return false;
+        done[dev] = true;
+    }
+    return true;
+}
+
+// ---- single-CTA kernel (ablation baseline)
+constexpr int GEMM_BN = 128;
+
+template <int MODE, int BN>
+nm_status launch_gemm_1cta(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &y,
+                           const uint8_t *meta, int64_t nkb, int m, int nwin, int64_t R,
+                           int64_t T, cudaStream_t s) {
+    using Cfg = GemmCfg<MODE, BN>;
+    if (!set_smem_attr<k_gemm_1cta<MODE, BN>>(Cfg::SMEM_BYTES)) return NM_ERR_CUDA;
     const int64_t mt = (R + BM - 1) / BM, ntl = (T + BN - 1) / BN;
     if (mt > 0x7FFFFFFF || ntl > 65535) return NM_ERR_SHAPE;
     dim3 grid(static_cast<unsigned>(mt), static_cast<unsigned>(ntl));
-    k_gemm<MODE, BN><<<grid, GEMM_THREADS, C::SMEM_BYTES, s>>>(a, b, y, meta, nkb, m, nwin);
+    k_gemm_1cta<MODE, BN><<<grid, GEMM_THREADS, Cfg::SMEM_BYTES, s>>>(a, b, y, meta, nkb, m, nwin);
     return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
 }
 
-constexpr int GEMM_BN = 128;
+// ---- persistent CTA-pair kernel
+template <int MODE>
+nm_status launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &e,
+                      const CUtensorMap &y, const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
+                      int64_t R, int64_t nkb, int m, cudaStream_t s) {
+    using Cfg = PairCfg<MODE>;
+    if (!set_smem_attr<k_gemm_pair<MODE>>(Cfg::SMEM_BYTES)) return NM_ERR_CUDA;
+    const int64_t ntiles = ((T + Cfg::BN - 1) / Cfg::BN) * ((R + 255) / 256);
+    int64_t clusters = sm_count() / 2;
+    if (clusters > ntiles) clusters = ntiles;
+    if (clusters < 1) clusters = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+    cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k_gemm_pair<MODE>, a, b, e, y, X, T, K, ldx, R, nkb, m) !=
+        cudaSuccess)
+        return NM_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -412,15 +828,15 @@ extern "C" nm_status nm_sparse_prepare(const uint16_t *vals, const uint8_t *wmet
     const PackedGeom p = packed_geom(R, K, m);
     if (packed_bytes < static_cast<size_t>(p.vals_bytes + p.meta_bytes)) return NM_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const int64_t n = m - 2;
+    const int n = m - 2;
     const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
     int64_t blocks = (p.Rpad * (p.KLpad / 2) + 255) / 256;
     k_prepare_vals<<<static_cast<unsigned>(blocks < cap ? blocks : cap), 256, 0, s>>>(
-        vals, R, p.G * n, p.Rpad, p.KLpad / 2, static_cast<uint16_t *>(packed));
+        vals, R, p.G, n, m, p.Rpad, p.KLpad / 2, static_cast<uint16_t *>(packed));
     const int64_t nblocks = (p.Rpad / BM) * p.nkb;
     blocks = (nblocks * EBLK_BYTES + 255) / 256;
     k_prepare_meta<<<static_cast<unsigned>(blocks < cap ? blocks : cap), 256, 0, s>>>(
-        wmeta, R, p.nwin, (p.nwin + 1) / 2, p.nkb, nblocks,
+        wmeta, R, p.G, m, (p.nwin + 1) / 2, p.nkb, nblocks,
         static_cast<uint8_t *>(packed) + p.vals_bytes);
     return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
 }
@@ -434,19 +850,19 @@ extern "C" nm_status nm_sparse_gemm(const uint16_t *X, int64_t T, int64_t K, int
     if (!aligned16(X) || !aligned16(Y) || !aligned16(packed) || (ldx % 8) != 0 || (ldy % 8) != 0)
         return NM_ERR_ALIGN;
     const PackedGeom p = packed_geom(R, K, m);
-    CUtensorMap ta, tb, ty;
-    if (!make_tmap_bf16(&ta, packed, p.Rpad, p.KLpad / 2, p.KLpad / 2, 64, BM, true))
-        return NM_ERR_CUDA;
-    if (!make_tmap_bf16(&ty, Y, T, R, ldy, 32, GEMM_BN, false)) return NM_ERR_CUDA;
+    if (p.nkb > 0x7FFFFFFF / 8 || (p.Rpad / BM) * p.nkb * 8 > 0x7FFFFFFF) return NM_ERR_SHAPE;
+    CUtensorMap ta, tb, te, ty;
     const uint8_t *meta = static_cast<const uint8_t *>(packed) + p.vals_bytes;
+    if (!make_tmap_bf16(&ta, packed, p.Rpad, p.KLpad / 2, p.KLpad / 2, 64, BM, true) ||
+        !make_tmap_2d(&te, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, meta, (p.Rpad / BM) * p.nkb * 8, 256,
+                      256, 256, 8, false) ||
+        !make_tmap_bf16(&tb, X, T, K, ldx, 64, 128, true) ||
+        !make_tmap_bf16(&ty, Y, T, R, ldy, 32, 32, false))
+        return NM_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (m == 4) {
-        if (!make_tmap_bf16(&tb, X, T, K, ldx, 64, GEMM_BN, true)) return NM_ERR_CUDA;
-        return launch_gemm<MODE_SP24, GEMM_BN>(ta, tb, ty, meta, p.nkb, m, 1, R, T, s);
-    }
-    if (!make_tmap_bf16(&tb, X, T, K, ldx, 128, GEMM_BN, false)) return NM_ERR_CUDA;
-    return launch_gemm<MODE_SPLIFT, GEMM_BN>(ta, tb, ty, meta, p.nkb, m,
-                                             static_cast<int>(m / 2 - 1), R, T, s);
+    if (m == 4) return launch_pair<PMODE_SP24>(ta, tb, te, ty, X, T, K, ldx, R, p.nkb, m, s);
+    if (m == 8) return launch_pair<PMODE_SP68>(ta, tb, te, ty, X, T, K, ldx, R, p.nkb, m, s);
+    return launch_pair<PMODE_SPLIFT>(ta, tb, te, ty, X, T, K, ldx, R, p.nkb, m, s);
 }
 
 extern "C" nm_status nm_dense_gemm(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
@@ -458,10 +874,35 @@ extern "C" nm_status nm_dense_gemm(const uint16_t *X, int64_t T, int64_t K, int6
         (ldy % 8) != 0)
         return NM_ERR_ALIGN;
     CUtensorMap ta, tb, ty;
-    if (!make_tmap_bf16(&ta, W, R, K, ldw, 64, BM, true)) return NM_ERR_CUDA;
-    if (!make_tmap_bf16(&tb, X, T, K, ldx, 64, GEMM_BN, true)) return NM_ERR_CUDA;
-    if (!make_tmap_bf16(&ty, Y, T, R, ldy, 32, GEMM_BN, false)) return NM_ERR_CUDA;
+    if (!make_tmap_bf16(&ta, W, R, K, ldw, 64, BM, true) ||
+        !make_tmap_bf16(&tb, X, T, K, ldx, 64, 128, true) ||
+        !make_tmap_bf16(&ty, Y, T, R, ldy, 32, 32, false))
+        return NM_ERR_CUDA;
     const int64_t nkb = (K + 63) / 64;
-    return launch_gemm<MODE_DENSE, GEMM_BN>(ta, tb, ty, nullptr, nkb, 4, 1, R, T,
-                                            reinterpret_cast<cudaStream_t>(stream));
+    return launch_pair<PMODE_DENSE>(ta, tb, ta, ty, X, T, K, ldx, R, nkb, 4,
+                                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" nm_status nm_gemm_1cta(int sparse, const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
+                                  const void *W_or_packed, int64_t R, int64_t ldw, uint16_t *Y,
+                                  int64_t ldy, void *stream) {
+    if (!X || !W_or_packed || !Y) return NM_ERR_NULL;
+    if (T < 1 || K < 1 || R < 1 || ldx < K || ldy < R || (!sparse && ldw < K)) return NM_ERR_SHAPE;
+    if (!aligned16(X) || !aligned16(Y) || !aligned16(W_or_packed) || (ldx % 8) != 0 ||
+        (ldy % 8) != 0 || (!sparse && (ldw % 8) != 0))
+        return NM_ERR_ALIGN;
+    CUtensorMap ta, tb, ty;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (!make_tmap_bf16(&ty, Y, T, R, ldy, 32, GEMM_BN, false) ||
+        !make_tmap_bf16(&tb, X, T, K, ldx, 64, GEMM_BN, true))
+        return NM_ERR_CUDA;
+    if (sparse) {
+        const PackedGeom p = packed_geom(R, K, 4);
+        if (!make_tmap_bf16(&ta, W_or_packed, p.Rpad, p.KLpad / 2, p.KLpad / 2, 64, BM, true))
+            return NM_ERR_CUDA;
+        const uint8_t *meta = static_cast<const uint8_t *>(W_or_packed) + p.vals_bytes;
+        return launch_gemm_1cta<MODE_SP24, GEMM_BN>(ta, tb, ty, meta, p.nkb, 4, 1, R, T, s);
+    }
+    if (!make_tmap_bf16(&ta, W_or_packed, R, K, ldw, 64, BM, true)) return NM_ERR_CUDA;
+    return launch_gemm_1cta<MODE_DENSE, GEMM_BN>(ta, tb, ty, nullptr, (K + 63) / 64, 4, 1, R, T, s);
 }

@@ -42,41 +42,78 @@ def packed_geometry(R: int, K: int, m: int):
     G = (K + m - 1) // m
     nwin = G * (m // 2 - 1)
     KL = nwin * 4
-    KLpad = (KL + 127) // 128 * 128
-    Rpad = (R + 127) // 128 * 128
-    return dict(G=G, nwin=nwin, KL=KL, KLpad=KLpad, Rpad=Rpad, nkb=KLpad // 128,
+    nkb = 3 * ((G + 31) // 32) if m == 8 else (KL + 127) // 128
+    KLpad = nkb * 128
+    Rpad = (R + 255) // 256 * 256
+    return dict(G=G, nwin=nwin, KL=KL, KLpad=KLpad, Rpad=Rpad, nkb=nkb,
                 vals_bytes=Rpad * KLpad, meta_bytes=Rpad * KLpad // 8)
 
 
-def decode_packed(packed: np.ndarray, R: int, K: int, m: int):
-    """Undo the GEMM operand layout: returns (vals [R x nwin*2] uint16,
-    window nibbles [R x nwin] uint8, padding_ok bool).
+def slot_windows(m: int, nkb: int):
+    """(group, window) of every slot (4 lifted columns) of the packed K' order:
+    natural for m in (4, 6, 10); for m = 8, per 32 groups: two blocks holding
+    windows 0 and 2 of groups 0-15 and 16-31 (X's own column order), then one
+    block holding window 1 of groups 0-31."""
+    g = np.empty(nkb * 32, dtype=np.int64)
+    w = np.empty(nkb * 32, dtype=np.int64)
+    nwin = m // 2 - 1
+    for kb in range(nkb):
+        for s in range(32):
+            if m == 8:
+                j, typ = divmod(kb, 3)
+                if typ < 2:
+                    gg, ww = 32 * j + 16 * typ + s // 2, 2 * (s % 2)
+                else:
+                    gg, ww = 32 * j + s, 1
+            else:
+                gg, ww = divmod(32 * kb + s, nwin)
+            g[kb * 32 + s], w[kb * 32 + s] = gg, ww
+    return g, w
 
-    Metadata block b of row tile mt and K' block kb (2048 bytes): byte j holds
-    the index pairs of two adjacent windows of one row; with L = j // 16 and
+
+def decode_packed(packed: np.ndarray, R: int, K: int, m: int):
+    """Undo the GEMM operand layout: returns (vals [R x nwin*2] uint16 and
+    window nibbles [R x nwin] uint8, both in (group, window) order, and
+    padding_ok: every padded row or slot holds value 0 and the pair (0,1)).
+
+    Metadata block of row tile mt and K' block kb (2048 bytes): byte j holds
+    the index pairs of two adjacent slots of one row; with L = j // 16 and
     w = j % 16: row = (L % 8) + 8 * ((w // 2) % 2) + 16 * (L // 16) and first
     lifted column = 8 * (w % 2) + 16 * ((L // 8) % 2) + 32 * (w // 4).
     """
-    g = packed_geometry(R, K, m)
-    KLh = g["KLpad"] // 2
-    vals_all = packed[: g["vals_bytes"]].view(np.uint16).reshape(g["Rpad"], KLh)
-    meta = packed[g["vals_bytes"]: g["vals_bytes"] + g["meta_bytes"]]
-    nib = np.zeros((g["Rpad"], g["KLpad"] // 4), dtype=np.uint8)
+    geo = packed_geometry(R, K, m)
+    KLh = geo["KLpad"] // 2
+    vals_all = packed[: geo["vals_bytes"]].view(np.uint16).reshape(geo["Rpad"], KLh)
+    meta = packed[geo["vals_bytes"]: geo["vals_bytes"] + geo["meta_bytes"]]
+    nslots = geo["KLpad"] // 4
+    nib = np.zeros((geo["Rpad"], nslots), dtype=np.uint8)
     j = np.arange(2048)
     L, w = j // 16, j % 16
     rows = (L % 8) + 8 * ((w // 2) % 2) + 16 * (L // 16)
     cols = 8 * (w % 2) + 16 * ((L // 8) % 2) + 32 * (w // 4)
-    blocks = meta.reshape(g["Rpad"] // 128, g["nkb"], 2048)
-    for mt in range(g["Rpad"] // 128):
-        for kb in range(g["nkb"]):
+    blocks = meta.reshape(geo["Rpad"] // 128, geo["nkb"], 2048)
+    for mt in range(geo["Rpad"] // 128):
+        for kb in range(geo["nkb"]):
             b = blocks[mt, kb]
-            win = kb * 32 + cols // 4
-            nib[mt * 128 + rows, win] = b & 0xF
-            nib[mt * 128 + rows, win + 1] = b >> 4
-    nw = g["nwin"]
-    pad_ok = bool(np.all(vals_all[R:] == 0) and np.all(vals_all[:, nw * 2:] == 0)
-                  and np.all(nib[R:] == 4) and np.all(nib[:, nw:] == 4))
-    return vals_all[:R, : nw * 2], nib[:R, :nw], pad_ok
+            slot = kb * 32 + cols // 4
+            nib[mt * 128 + rows, slot] = b & 0xF
+            nib[mt * 128 + rows, slot + 1] = b >> 4
+    sg, sw = slot_windows(m, geo["nkb"])
+    nwin_g = m // 2 - 1
+    real = sg < geo["G"]
+    wi = sg[real] * nwin_g + sw[real]
+    order = np.argsort(wi)
+    assert np.array_equal(wi[order], np.arange(geo["nwin"]))
+    slot_idx = np.nonzero(real)[0][order]          # slot of window wi, in wi order
+    vals = np.empty((R, geo["nwin"] * 2), dtype=np.uint16)
+    vals[:, 0::2] = vals_all[:R, 2 * slot_idx]
+    vals[:, 1::2] = vals_all[:R, 2 * slot_idx + 1]
+    nibs = nib[:R, slot_idx]
+    pad_slots = np.nonzero(~real)[0]
+    pad_ok = bool(np.all(vals_all[R:] == 0) and np.all(nib[R:] == 4)
+                  and np.all(vals_all[:, np.concatenate([2 * pad_slots, 2 * pad_slots + 1])] == 0)
+                  and np.all(nib[:, pad_slots] == 4))
+    return vals, nibs, pad_ok
 
 
 def wmeta_nibbles(wmeta: np.ndarray, nwin: int) -> np.ndarray:
