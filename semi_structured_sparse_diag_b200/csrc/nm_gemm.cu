@@ -378,11 +378,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 //   warp 1      tensor-memory owner; in the leader also the MMA issuer;
 //   warps 4-11  epilogue: tensor memory -> bf16 -> TMA store, 32 weight rows
 //               x 128 tokens each;
-//   warps 12-15 lift (SLIFT / SP68 modes): build this CTA's lifted B half of a
-//               stage from X in global memory (SlideSparse sec. 2B), then
-//               arrive on the leader's lifted[s].
+//   warps 12-15 lift (SPLIFT / SP68 modes, SlideSparse sec. 2B): make this
+//               CTA's lifted B half of each stage and tell the leader it is
+//               ready (lifted[s]):
+//               SPLIFT: copy each window's 4 columns of X from global memory
+//               into the swizzled B buffer with cp.async, up to three stages
+//               in flight (each warp arrives: 4 warps x 2 CTAs);
+//               SP68:   raw blocks are TMA tiles of X (local xfull[s]); warp 2
+//               forwards their arrival to the leader (counted as 4), the lift
+//               warps copy columns 2..5 of every group out of the two raw stages
+//               into the third (odd) stage, then each signals it.
 // Stages: a ring of S shared-memory stages per CTA; empty[s] and acc_full[b]
-// are armed in both CTAs by multicast tcgen05.commit from the leader.
+// are armed in both CTAs by multicast tcgen05.commit from the leader; in the
+// lift modes empty[s] also waits for the 4 local lift warps (a raw stage is
+// not refilled before the lift has read it).
 // ===========================================================================
 enum { PMODE_DENSE = 0, PMODE_SP24 = 1, PMODE_SPLIFT = 2, PMODE_SP68 = 3 };
 
@@ -432,9 +441,9 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
                                                 ~static_cast<uintptr_t>(1023));
     uint8_t *epi_smem = smem + S * C::STAGE_BYTES;
     uint64_t *bars = reinterpret_cast<uint64_t *>(epi_smem + C::EPI_BYTES);
-    uint64_t *full = bars, *empty = bars + S, *lifted = bars + 2 * S;
-    uint64_t *acc_full = bars + 3 * S, *acc_empty = bars + 3 * S + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * S + 4);
+    uint64_t *full = bars, *empty = bars + S, *lifted = bars + 2 * S, *xfull = bars + 3 * S;
+    uint64_t *acc_full = bars + 4 * S, *acc_empty = bars + 4 * S + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * S + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -450,8 +459,9 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-            mbar_init(&lifted[s], 8);
+            mbar_init(&empty[s], C::LIFT ? 5 : 1);
+            mbar_init(&lifted[s], 8);  // 4 lift warps (or the forwarder, x4) per CTA
+            mbar_init(&xfull[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
@@ -487,9 +497,12 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
                     const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
                     if (it >= S && !mbar_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
                     const bool btma = pair_b_by_tma(MODE, kb);
+                    // B tiles go to the leader's full[s], except in SP68 where
+                    // the lift warps of each CTA watch their own xfull[s]
+                    const bool b_to_full = btma && MODE != PMODE_SP68;
                     if (rank == 0) {
                         const uint32_t tx = 2u * static_cast<uint32_t>(
-                            C::A_BYTES + C::E_BYTES + (btma ? C::B_BYTES : 0));
+                            C::A_BYTES + C::E_BYTES + (b_to_full ? C::B_BYTES : 0));
                         mbar_arrive_expect_tx(&full[s], tx);
                     }
                     const uint32_t bar = mapa_shared(&full[s], 0);
@@ -497,7 +510,13 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
                     if (C::SPARSE)
                         tma_load_2d_pair(stE(s), &tmE, bar, 0,
                                          static_cast<int32_t>(((mt2 * 2 + rank) * nkb + kb) * 8));
-                    if (btma) {
+                    if (btma && MODE == PMODE_SP68) {
+                        const int64_t x0 = (kb / 3) * 256 + (kb % 3) * 128;
+                        mbar_arrive_expect_tx(&xfull[s], C::B_BYTES);
+                        tma_load_2d(stB(s), &tmB, &xfull[s], static_cast<int32_t>(x0), brow);
+                        tma_load_2d(stB(s) + C::BH * 128, &tmB, &xfull[s],
+                                    static_cast<int32_t>(x0 + 64), brow);
+                    } else if (btma) {
                         if (MODE == PMODE_DENSE) {
                             tma_load_2d_pair(stB(s), &tmB, bar, static_cast<int32_t>(kb * 64), brow);
                         } else {
@@ -520,7 +539,6 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
         if (rank == 0 && lane == 0) {
             const uint32_t idesc = make_idesc_bf16(256, C::BN, C::SPARSE, 0);
             int64_t it = 0, ti = 0;
-            uint32_t lbits = 0;
             bool ok = true;
             for (int64_t tile = cluster; tile < ntiles && ok; tile += nclusters, ++ti) {
                 const int buf = static_cast<int>(ti % C::ACC_BUFS);
@@ -535,10 +553,7 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
                     const int s = static_cast<int>(it % S);
                     const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
                     if (!mbar_wait(&full[s], ph)) { ok = false; break; }
-                    if (pair_needs_lift(MODE, kb)) {
-                        if (!mbar_wait_cluster(&lifted[s], (lbits >> s) & 1u)) { ok = false; break; }
-                        lbits ^= 1u << s;
-                    }
+                    if (C::LIFT && !mbar_wait_cluster(&lifted[s], ph)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(stA(s)), b0 = smem_u32(stB(s));
                     if (!C::SPARSE) {
@@ -613,64 +628,152 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
         }
         if (lane == 0) bulk_wait_group0();
         __syncwarp();
-    } else if (C::LIFT && warp >= 12) {
-        // ---------------------------------------------------------- lift
-        const int lw = warp - 12;
-        const int nwin = m / 2 - 1;
+    } else if (MODE == PMODE_SP68 && warp == 2) {
+        // ---------------------------------------------------------- forwarder
+        // raw blocks: tell the leader as soon as this CTA's TMA tile has landed
+        const uint32_t lifted_cl0 = mapa_shared(&lifted[0], 0);
         int64_t it = 0;
+        uint32_t xbits = 0;
         bool ok = true;
         for (int64_t tile = cluster; tile < ntiles && ok; tile += nclusters) {
-            const int64_t nt = tile % n_t;
-            const int64_t t0 = nt * C::BN + rank * C::BH;
             for (int64_t kb = 0; kb < nkb; ++kb, ++it) {
-                if (!pair_needs_lift(MODE, kb)) continue;
+                if (kb % 3 == 2) continue;
                 const int s = static_cast<int>(it % S);
-                const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
-                if (it >= S && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u))) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&xfull[s], (xbits >> s) & 1u))) {
                     ok = false;
                     break;
                 }
-                int64_t g;
-                int w;
-                slot_window(m, kb, lane, g, w);
-                const int64_t col = g * m + 2 * w;  // first of the window's 4 columns
-                const bool full_cols = col + 4 <= K;
-                (void)nwin;
-                uint8_t *bs = stB(s);
-                const int chunk = (lane & 15) >> 1, atom = lane >> 4;
-                for (int r0 = lw; r0 < C::BH; r0 += 32) {
-                    uint32_t lo[8], hi[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int row = r0 + 4 * u;
+                xbits ^= 1u << s;
+                if (lane == 0) mbar_arrive_cluster_n(lifted_cl0 + static_cast<uint32_t>(s) * 8u, 4u);
+            }
+        }
+    } else if (C::LIFT && warp >= 12) {
+        // ---------------------------------------------------------- lift
+        const int lw = warp - 12;
+        const uint32_t lifted_cl0 = mapa_shared(&lifted[0], 0);
+        int64_t it = 0;
+        uint32_t xbits = 0;  // phase of xfull[s] (one phase per raw use of stage s)
+        bool ok = true;
+        if (MODE == PMODE_SPLIFT) {
+            // cp.async pipeline: stage of the block issued `d` steps ago, d = 1, 2
+            int pend_s[2] = {-1, -1};
+            for (int64_t tile = cluster; tile < ntiles && ok; tile += nclusters) {
+                const int64_t t0 = (tile % n_t) * C::BN + rank * C::BH;
+                for (int64_t kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = static_cast<int>(it % S);
+                    const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
+                    if (it >= S && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u))) {
+                        ok = false;
+                        break;
+                    }
+                    int64_t g;
+                    int w;
+                    slot_window(m, kb, lane, g, w);
+                    const int64_t col = g * m + 2 * w;  // first of the window's 4 columns
+                    uint8_t *bs = stB(s);
+                    const int chunk = (lane & 15) >> 1, atom = lane >> 4;
+                    for (int row = lw; row < C::BH; row += 4) {
                         const int64_t t = t0 + row;
-                        lo[u] = 0u;
-                        hi[u] = 0u;
-                        if (t < T) {
-                            const uint16_t *src = X + t * ldx + col;
-                            if (full_cols) {
-                                lo[u] = __ldg(reinterpret_cast<const uint32_t *>(src));
-                                hi[u] = __ldg(reinterpret_cast<const uint32_t *>(src) + 1);
-                            } else {
-                                uint32_t e[4];
+                        uint8_t *dst = bs + atom * (C::BH * 128) + row * 128 +
+                                       ((chunk ^ (row & 7)) << 4) + ((lane & 1) << 3);
+                        const bool tin = t < T;
+                        const uint16_t *src = X + (tin ? t : 0) * ldx;
 #pragma unroll
-                                for (int i = 0; i < 4; ++i) e[i] = col + i < K ? __ldg(src + i) : 0u;
-                                lo[u] = e[0] | (e[1] << 16);
-                                hi[u] = e[2] | (e[3] << 16);
+                        for (int hw = 0; hw < 2; ++hw) {
+                            const int64_t c = col + 2 * hw;
+                            if (tin && c + 2 <= K) {
+                                cp_async4(dst + 4 * hw, src + c, 4u);
+                            } else {  // past T or K: zeros (ragged last column keeps its value)
+                                const uint32_t v = (tin && c < K) ? static_cast<uint32_t>(src[c]) : 0u;
+                                *reinterpret_cast<uint32_t *>(dst + 4 * hw) = v;
                             }
                         }
                     }
+                    cp_async_commit();
+                    // the block issued two steps ago has landed: signal it
+                    cp_async_wait_pending<2>();
+                    if (pend_s[1] >= 0) {
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            mbar_arrive_cluster(lifted_cl0 + static_cast<uint32_t>(pend_s[1]) * 8u);
+                            mbar_arrive(&empty[pend_s[1]]);
+                        }
+                    }
+                    pend_s[1] = pend_s[0];
+                    pend_s[0] = s;
+                }
+            }
+            // drain: signal the blocks still in flight, oldest first
+            cp_async_wait_pending<0>();
+            fence_proxy_async_smem();
+            __syncwarp();
+            for (int d = 1; d >= 0; --d) {
+                if (pend_s[d] >= 0 && lane == 0) {
+                    mbar_arrive_cluster(lifted_cl0 + static_cast<uint32_t>(pend_s[d]) * 8u);
+                    mbar_arrive(&empty[pend_s[d]]);
+                }
+            }
+        } else {  // PMODE_SP68
+            for (int64_t tile = cluster; tile < ntiles && ok; tile += nclusters) {
+                for (int64_t kb = 0; kb < nkb && ok; ++kb, ++it) {
+                    const int s = static_cast<int>(it % S);
+                    const int type = static_cast<int>(kb % 3);
+                    if (type < 2) {
+                        // raw block: its B half is a TMA tile of X in this CTA
+                        if (!__all_sync(0xffffffffu, mbar_wait(&xfull[s], (xbits >> s) & 1u))) {
+                            ok = false;
+                            break;
+                        }
+                        xbits ^= 1u << s;
+                        // the odd stage of this super-block must be free
+                        const int64_t it_odd = it + (2 - type);
+                        const int so = static_cast<int>(it_odd % S);
+                        if (type == 0 && it_odd >= S &&
+                            !__all_sync(0xffffffffu,
+                                        mbar_wait(&empty[so], static_cast<uint32_t>(((it_odd / S) & 1) ^ 1)))) {
+                            ok = false;
+                            break;
+                        }
+                        // columns 2..5 of a group = bytes 4..11 of its 16-byte chunk.
+                        // Each quarter-warp reads one 128-byte row segment (one
+                        // (row, atom) pair: 8 groups) with 16-byte loads, so every
+                        // load and store instruction is free of bank conflicts.
+                        const uint8_t *src = stB(s);
+                        uint8_t *dst = stB(so);
+                        const int c = lane & 7, k = lane >> 3;
+                        uint32_t a[16], b[16];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int row = r0 + 4 * u;
-                        uint8_t *dst = bs + atom * (C::BH * 128) + row * 128 +
-                                       ((chunk ^ (row & 7)) << 4) + ((lane & 1) << 3);
-                        *reinterpret_cast<uint2 *>(dst) = make_uint2(lo[u], hi[u]);
+                        for (int i = 0; i < 16; ++i) {
+                            const int p = (lw * 16 + i) * 4 + k;  // (row, atom) pair
+                            const int row = p >> 1, atom = p & 1;
+                            const uint4 v = *reinterpret_cast<const uint4 *>(
+                                src + atom * (C::BH * 128) + row * 128 + ((c ^ (row & 7)) << 4));
+                            a[i] = v.y;
+                            b[i] = v.z;
+                        }
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int p = (lw * 16 + i) * 4 + k;
+                            const int row = p >> 1, atom = p & 1;
+                            const int gl = atom * 8 + c;          // group within the raw block
+                            const int dchunk = gl >> 1;           // slot 16*type + gl
+                            *reinterpret_cast<uint2 *>(dst + type * (C::BH * 128) + row * 128 +
+                                                       ((dchunk ^ (row & 7)) << 4) + ((gl & 1) << 3)) =
+                                make_uint2(a[i], b[i]);
+                        }
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&empty[s]);  // done reading the raw stage
+                    } else {
+                        // odd block: its B half was filled by the two raw steps
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            mbar_arrive_cluster(lifted_cl0 + static_cast<uint32_t>(s) * 8u);
+                            mbar_arrive(&empty[s]);
+                        }
                     }
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(mapa_shared(&lifted[s], 0));
             }
         }
     }
