@@ -77,10 +77,11 @@ __host__ __device__ inline void slot_window(int m, int64_t kb, int s, int64_t &g
             w = 1;
         }
     } else {
-        const int nwin = m / 2 - 1;
+        // nwin = m/2 - 1 is 1, 2 or 4 for m = 4, 6, 10
+        const int sh = m == 4 ? 0 : (m == 6 ? 1 : 2);
         const int64_t wi = 32 * kb + s;
-        g = wi / nwin;
-        w = static_cast<int>(wi - g * nwin);
+        g = wi >> sh;
+        w = static_cast<int>(wi & ((1 << sh) - 1));
     }
 }
 
@@ -99,48 +100,72 @@ __host__ __device__ inline void meta_byte_coords(int b, int &row, int &col) {
     col = 8 * kh + 16 * k1 + 32 * k2;
 }
 
+// values: one thread per 16-byte output chunk (4 slots = 8 values) of a row;
+// grid x = chunks of a row, y (+65535 z) = row
 __global__ void __launch_bounds__(256)
     k_prepare_vals(const uint16_t *__restrict__ vals, int64_t R, int64_t G, int n, int m,
                    int64_t Rpad, int64_t KLh, uint16_t *__restrict__ out) {
-    const int64_t total = Rpad * KLh;
-    const int64_t rowlen = G * n;
-    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
-         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t r = idx / KLh, c = idx - r * KLh;
+    const int64_t r = blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535;
+    const int64_t c8 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // chunk
+    if (r >= Rpad || c8 * 8 >= KLh) return;
+    const int64_t kb = c8 / 8;          // 64 values per K' block
+    const int s0 = static_cast<int>(c8 % 8) * 4;
+    const uint16_t *vrow = vals + r * (G * n);
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
         int64_t g;
         int w;
-        slot_window(m, c / 64, static_cast<int>((c % 64) / 2), g, w);
-        uint16_t v = 0;
-        if (r < R && g < G) v = vals[r * rowlen + g * n + 2 * w + (c & 1)];
-        out[idx] = v;
+        slot_window(m, kb, s0 + i, g, w);
+        uint32_t lo = 0, hi = 0;
+        if (r < R && g < G) {
+            const uint16_t *p = vrow + g * n + 2 * w;
+            lo = __ldg(p);
+            hi = __ldg(p + 1);
+        }
+        o[i] = lo | (hi << 16);
     }
+    *reinterpret_cast<uint4 *>(out + r * KLh + c8 * 8) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// metadata: one thread per tensor-memory lane of a block (16 output bytes);
+// grid x = blocks of 8 metadata blocks (8 x 128 lanes = 1024 threads / 4 ...),
+// each thread: block index blk, lane L.
 __global__ void __launch_bounds__(256)
     k_prepare_meta(const uint8_t *__restrict__ wmeta, int64_t R, int64_t G, int m, int64_t wbytes,
                    int64_t nkb, int64_t nblocks, uint8_t *__restrict__ out) {
-    const int64_t total = nblocks * EBLK_BYTES;
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t blk = tid >> 7;
+    const int L = static_cast<int>(tid & 127);
+    if (blk >= nblocks) return;
     const int nwin = m / 2 - 1;
-    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
-         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t blk = idx / EBLK_BYTES;
-        const int b = static_cast<int>(idx - blk * EBLK_BYTES);
-        const int64_t mt = blk / nkb, kb = blk - mt * nkb;
-        int rl, cl;
-        meta_byte_coords(b, rl, cl);
-        const int64_t row = mt * BM + rl;
-        uint32_t nib[2] = {0x4u, 0x4u};  // padding: pair (0,1) over zero values
-        for (int h = 0; h < 2; ++h) {
-            int64_t g;
-            int w;
-            slot_window(m, kb, cl / 4 + h, g, w);
-            if (row < R && g < G) {
-                const int64_t wi = g * nwin + w;
-                nib[h] = (wmeta[row * wbytes + wi / 2] >> (4 * (wi & 1))) & 0xFu;
+    const int64_t mt = blk / nkb, kb = blk - mt * nkb;
+    uint32_t words[4];
+#pragma unroll
+    for (int wd = 0; wd < 4; ++wd) {
+        uint32_t v = 0;
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) {
+            int rl, cl;
+            meta_byte_coords(L * 16 + wd * 4 + bb, rl, cl);
+            const int64_t row = mt * BM + rl;
+            uint32_t nib[2] = {0x4u, 0x4u};  // padding: pair (0,1) over zero values
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                int64_t g;
+                int w;
+                slot_window(m, kb, cl / 4 + h, g, w);
+                if (row < R && g < G) {
+                    const int64_t wi = g * nwin + w;
+                    nib[h] = (__ldg(wmeta + row * wbytes + wi / 2) >> (4 * (wi & 1))) & 0xFu;
+                }
             }
+            v |= (nib[0] | (nib[1] << 4)) << (8 * bb);
         }
-        out[idx] = static_cast<uint8_t>(nib[0] | (nib[1] << 4));
+        words[wd] = v;
     }
+    *reinterpret_cast<uint4 *>(out + blk * EBLK_BYTES + L * 16) =
+        make_uint4(words[0], words[1], words[2], words[3]);
 }
 
 // ---------------------------------------------------------------------------
@@ -932,13 +957,16 @@ extern "C" nm_status nm_sparse_prepare(const uint16_t *vals, const uint8_t *wmet
     if (packed_bytes < static_cast<size_t>(p.vals_bytes + p.meta_bytes)) return NM_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int n = m - 2;
-    const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
-    int64_t blocks = (p.Rpad * (p.KLpad / 2) + 255) / 256;
-    k_prepare_vals<<<static_cast<unsigned>(blocks < cap ? blocks : cap), 256, 0, s>>>(
-        vals, R, p.G, n, m, p.Rpad, p.KLpad / 2, static_cast<uint16_t *>(packed));
+    const int64_t chunks = p.KLpad / 16;  // 16-byte chunks of a packed row
+    dim3 vgrid(static_cast<unsigned>((chunks + 255) / 256),
+               static_cast<unsigned>(p.Rpad < 65535 ? p.Rpad : 65535),
+               static_cast<unsigned>((p.Rpad + 65534) / 65535));
+    k_prepare_vals<<<vgrid, 256, 0, s>>>(vals, R, p.G, n, m, p.Rpad, p.KLpad / 2,
+                                         static_cast<uint16_t *>(packed));
     const int64_t nblocks = (p.Rpad / BM) * p.nkb;
-    blocks = (nblocks * EBLK_BYTES + 255) / 256;
-    k_prepare_meta<<<static_cast<unsigned>(blocks < cap ? blocks : cap), 256, 0, s>>>(
+    const int64_t mblocks = (nblocks * 128 + 255) / 256;
+    if (mblocks > 0x7FFFFFFF) return NM_ERR_SHAPE;
+    k_prepare_meta<<<static_cast<unsigned>(mblocks), 256, 0, s>>>(
         wmeta, R, p.G, m, (p.nwin + 1) / 2, p.nkb, nblocks,
         static_cast<uint8_t *>(packed) + p.vals_bytes);
     return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;

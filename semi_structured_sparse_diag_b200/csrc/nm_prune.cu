@@ -103,37 +103,54 @@ __device__ __forceinline__ float score_one(const double *__restrict__ H, double 
     return __double2float_rn(__dmul_rn(h, __dmul_rn(w, w)));
 }
 
+// grid: x = 4096-column slice of a row (256 threads x 2 chunks x 8 elements),
+// y (+65535 z) = row.  Both chunks' loads are issued before any arithmetic.
 __global__ void __launch_bounds__(256) k_score(const double *__restrict__ H, double eps,
                                                const uint16_t *__restrict__ W, int64_t R,
                                                int64_t K, int64_t ldw, float *__restrict__ S) {
-    const int64_t cpr = (K + 7) / 8;  // 8-element chunks per row
-    const int64_t total = R * cpr;
-    const bool vec_store = (K % 4) == 0;
-    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
-         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t i = idx / cpr;
-        const int64_t j0 = (idx - i * cpr) * 8;
-        const uint16_t *wrow = W + i * ldw;
-        float *srow = S + i * K;
-        if (j0 + 8 <= K) {
-            const uint4 wv = __ldg(reinterpret_cast<const uint4 *>(wrow + j0));
-            const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
-            float s[8];
+    const int64_t i = blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535;
+    if (i >= R) return;
+    const uint16_t *wrow = W + i * ldw;
+    float *srow = S + i * K;
+    int64_t j0[2];
+    bool full[2];
+    uint4 wv[2];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        j0[c] = (static_cast<int64_t>(blockIdx.x) * 512 + c * 256 + threadIdx.x) * 8;
+        full[c] = j0[c] + 8 <= K;
+        if (full[c]) wv[c] = __ldg(reinterpret_cast<const uint4 *>(wrow + j0[c]));
+    }
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        if (j0[c] >= K) continue;
+        if (!full[c]) {
+            for (int64_t j = j0[c]; j < K; ++j) srow[j] = score_one(H, eps, j, wrow[j]);
+            continue;
+        }
+        const uint32_t wr[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
+        float sv[8];
+        if (H != nullptr) {
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                s[2 * u] = score_one(H, eps, j0 + 2 * u, static_cast<uint16_t>(wr[u] & 0xFFFFu));
-                s[2 * u + 1] = score_one(H, eps, j0 + 2 * u + 1, static_cast<uint16_t>(wr[u] >> 16));
-            }
-            if (vec_store) {
-                float4 *d = reinterpret_cast<float4 *>(srow + j0);
-                d[0] = make_float4(s[0], s[1], s[2], s[3]);
-                d[1] = make_float4(s[4], s[5], s[6], s[7]);
-            } else {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) srow[j0 + u] = s[u];
+                const double2 hv = __ldg(reinterpret_cast<const double2 *>(H + j0[c]) + u);
+                const double wa = bf16_to_f64(static_cast<uint16_t>(wr[u] & 0xFFFFu));
+                const double wb = bf16_to_f64(static_cast<uint16_t>(wr[u] >> 16));
+                sv[2 * u] = __double2float_rn(__dmul_rn(__dadd_rn(hv.x, eps), __dmul_rn(wa, wa)));
+                sv[2 * u + 1] = __double2float_rn(__dmul_rn(__dadd_rn(hv.y, eps), __dmul_rn(wb, wb)));
             }
         } else {
-            for (int64_t j = j0; j < K; ++j) srow[j] = score_one(H, eps, j, wrow[j]);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                sv[u] = fabsf(bf16_to_f32(static_cast<uint16_t>(wr[u >> 1] >> (16 * (u & 1)))));
+        }
+        if ((K & 3) == 0) {
+            float4 *d = reinterpret_cast<float4 *>(srow + j0[c]);
+            d[0] = make_float4(sv[0], sv[1], sv[2], sv[3]);
+            d[1] = make_float4(sv[4], sv[5], sv[6], sv[7]);
+        } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) srow[j0[c] + u] = sv[u];
         }
     }
 }
@@ -149,6 +166,7 @@ template <int M>
 __device__ __forceinline__ void load_group(const float *__restrict__ srow,
                                            const uint16_t *__restrict__ vrow, int64_t c0,
                                            int64_t K, int m_rt, float *s, uint16_t *v) {
+    constexpr int MM = M > 0 ? M : 16;
     const int m = M > 0 ? M : m_rt;
     if (M > 0 && c0 + M <= K) {
         if constexpr (M % 4 == 0) {
@@ -189,9 +207,10 @@ __device__ __forceinline__ void load_group(const float *__restrict__ srow,
             }
         }
     } else {
-        for (int q = 0; q < m; ++q) {
+#pragma unroll
+        for (int q = 0; q < MM; ++q) {
             const int64_t c = c0 + q;
-            if (c < K) { s[q] = __ldg(srow + c); v[q] = __ldg(vrow + c); }
+            if (q < m && c < K) { s[q] = __ldg(srow + c); v[q] = __ldg(vrow + c); }
             else { s[q] = 0.0f; v[q] = 0; }
         }
     }
@@ -202,10 +221,11 @@ __global__ void __launch_bounds__(PRUNE_THREADS)
     k_prune(const float *__restrict__ S, int64_t lds, const uint16_t *__restrict__ V, int64_t ldv,
             int64_t K, int64_t G, int n, int m_rt, uint32_t *__restrict__ mask,
             uint16_t *__restrict__ vals, uint8_t *__restrict__ meta24) {
+    constexpr int MM = M > 0 ? M : 16;  // static trip count (runtime m <= MM)
     const int m = M > 0 ? M : m_rt;
     __shared__ uint32_t words[PRUNE_THREADS / 32][16];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t row = blockIdx.y;
+    const int64_t row = blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535;
     const int64_t g = static_cast<int64_t>(blockIdx.x) * PRUNE_THREADS + threadIdx.x;
     const bool valid = g < G;
     const int64_t mwords = (G * m + 31) / 32;
@@ -213,50 +233,103 @@ __global__ void __launch_bounds__(PRUNE_THREADS)
     if (lane < 16) words[warp][lane] = 0u;
     __syncwarp();
 
-    float s[16];
-    uint16_t v[16];
     uint32_t keepbits = 0;
     uint32_t nib = 0;
     if (valid) {
+        float s[MM];
+        uint16_t v[MM];
         load_group<M>(S + row * lds, V + row * ldv, g * m, K, m, s, v);
-        int kept = 0;
-        uint16_t out[16];
         int i0 = 0, i1 = 0;
+        if (M > 0 && n == m - 2) {
+            // (m-2):m keeps all but the two lowest positions of the order (score
+            // descending, index ascending): find them with two linear scans.  A
+            // later position with an equal score ranks below an earlier one, so
+            // "<=" picks the highest index among equal minima.
+            int d0 = 0;
+            float s0 = s[0];
 #pragma unroll
-        for (int q = 0; q < (M > 0 ? M : 16); ++q) {
-            if (q >= m) break;
-            int rank = 0;
+            for (int q = 1; q < MM; ++q)
+                if (s[q] <= s0) { s0 = s[q]; d0 = q; }
+            int d1 = -1;
+            float s1 = 0.0f;
 #pragma unroll
-            for (int p = 0; p < (M > 0 ? M : 16); ++p) {
-                if (p >= m) break;
-                rank += (s[p] > s[q] || (s[p] == s[q] && p < q)) ? 1 : 0;
+            for (int q = 0; q < MM; ++q)
+                if (q != d0 && (d1 < 0 || s[q] <= s1)) { s1 = s[q]; d1 = q; }
+            const int dlo = d0 < d1 ? d0 : d1, dhi = d0 < d1 ? d1 : d0;
+            keepbits = ((1u << MM) - 1u) & ~(1u << d0) & ~(1u << d1);
+            // output k = v[k], v[k+1] or v[k+2] depending on the dropped positions;
+            // pairs of outputs are packed and stored right here (n = MM - 2 is even)
+            uint16_t *dst = vals + row * (G * n) + g * n;
+#pragma unroll
+            for (int k2 = 0; k2 < (MM - 2) / 2; ++k2) {
+                uint32_t word = 0;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int k = 2 * k2 + h;
+                    const int q = k + (k >= dlo ? 1 : 0) + (k + 1 >= dhi ? 1 : 0);
+                    const uint32_t val =
+                        q == k ? v[k] : (q == k + 1 ? v[k + 1] : v[(k + 2 < MM) ? k + 2 : k]);
+                    word |= val << (16 * h);
+                }
+                reinterpret_cast<uint32_t *>(dst)[k2] = word;
             }
-            if (rank < n) {
-                keepbits |= 1u << q;
-                if (kept == 0) i0 = q;
-                if (kept == 1) i1 = q;
-                out[kept++] = v[q];
+            i0 = (dlo == 0) ? (dhi == 1 ? 2 : 1) : 0;  // first kept position (m == 4 metadata)
+            i1 = 0;
+#pragma unroll
+            for (int q = MM - 1; q >= 0; --q)
+                if (q != dlo && q != dhi && q != i0) i1 = (i1 == 0 || q < i1) ? q : i1;
+        } else {
+            // general n:m: keep position q iff fewer than n positions beat it
+            uint32_t outw[(MM + 1) / 2];
+#pragma unroll
+            for (int k = 0; k < (MM + 1) / 2; ++k) outw[k] = 0u;
+#pragma unroll
+            for (int q = 0; q < MM; ++q) {
+                int rank = 0;
+#pragma unroll
+                for (int p = 0; p < MM; ++p)
+                    rank += (p < m && (s[p] > s[q] || (s[p] == s[q] && p < q))) ? 1 : 0;
+                if (q < m && rank < n) keepbits |= 1u << q;
+            }
+            // compress: output k takes the k-th kept position (ascending); values
+            // are selected with static indices so everything stays in registers
+            uint32_t rem = keepbits;
+#pragma unroll
+            for (int k = 0; k < MM - 1; ++k) {
+                if (k < n) {
+                    const int q = __ffs(rem) - 1;
+                    rem &= rem - 1u;
+                    if (k == 0) i0 = q;
+                    if (k == 1) i1 = q;
+                    uint32_t val = 0;
+#pragma unroll
+                    for (int i = 0; i < MM; ++i) val = (i == q) ? static_cast<uint32_t>(v[i]) : val;
+                    outw[k >> 1] |= val << (16 * (k & 1));
+                }
+            }
+            uint16_t *dst = vals + row * (G * n) + g * n;
+            if (n % 8 == 0) {
+#pragma unroll
+                for (int k = 0; k < (MM - 1) / 8; ++k)
+                    if (8 * k < n)
+                        *reinterpret_cast<uint4 *>(dst + 8 * k) =
+                            make_uint4(outw[4 * k], outw[4 * k + 1], outw[4 * k + 2], outw[4 * k + 3]);
+            } else if (n % 4 == 0) {
+#pragma unroll
+                for (int k = 0; k < (MM - 1) / 4; ++k)
+                    if (4 * k < n)
+                        *reinterpret_cast<uint2 *>(dst + 4 * k) = make_uint2(outw[2 * k], outw[2 * k + 1]);
+            } else if (n % 2 == 0) {
+#pragma unroll
+                for (int k = 0; k < (MM - 1) / 2; ++k)
+                    if (2 * k < n) *reinterpret_cast<uint32_t *>(dst + 2 * k) = outw[k];
+            } else {
+#pragma unroll
+                for (int k = 0; k < MM - 1; ++k)
+                    if (k < n) dst[k] = static_cast<uint16_t>(outw[k >> 1] >> (16 * (k & 1)));
             }
         }
         nib = static_cast<uint32_t>(i0 | (i1 << 2));
-        // compressed values, ascending column order
-        uint16_t *dst = vals + row * (G * n) + g * n;
-        if (M == 4 && n == 2) {
-            *reinterpret_cast<uint32_t *>(dst) = out[0] | (static_cast<uint32_t>(out[1]) << 16);
-        } else if (n % 8 == 0 && ((G * n) % 8) == 0) {
-            for (int k = 0; k < n; k += 8)
-                *reinterpret_cast<uint4 *>(dst + k) = make_uint4(
-                    out[k] | (static_cast<uint32_t>(out[k + 1]) << 16),
-                    out[k + 2] | (static_cast<uint32_t>(out[k + 3]) << 16),
-                    out[k + 4] | (static_cast<uint32_t>(out[k + 5]) << 16),
-                    out[k + 6] | (static_cast<uint32_t>(out[k + 7]) << 16));
-        } else if (n % 2 == 0) {
-            for (int k = 0; k < n; k += 2)
-                *reinterpret_cast<uint32_t *>(dst + k) =
-                    out[k] | (static_cast<uint32_t>(out[k + 1]) << 16);
-        } else {
-            for (int k = 0; k < n; ++k) dst[k] = out[k];
-        }
         // mask bits: this group's m bits at offset (g % 32) * m in the warp's words
         const uint32_t off = static_cast<uint32_t>(lane) * m;
         atomicOr(&words[warp][off >> 5], keepbits << (off & 31));
@@ -278,59 +351,74 @@ __global__ void __launch_bounds__(PRUNE_THREADS)
 }
 
 // ---------------------------------------------------------------------------
-// a4: sliding-window pack.  One thread per group; the window nibbles of a
-// warp's 32 groups are assembled in shared memory and written as bytes.
+// a4: sliding-window pack.  Each thread handles GT consecutive groups whose
+// mask bits start on a 32-bit word boundary (GT*m a multiple of 32) and whose
+// window nibbles fill whole bytes (GT*(m/2-1) even): it reads GT*m/32 words and
+// writes GT*(m/2-1)/2 bytes.  grid: x over runs of a row, y = row.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(PRUNE_THREADS)
-    k_slide_pack(const uint32_t *__restrict__ mask, int64_t G, int m, int64_t mwords,
+template <int M>
+struct SlideRun {
+    static constexpr int NWIN = M / 2 - 1;
+    static constexpr int GT = M == 4 ? 8 : (M == 6 ? 16 : (M == 8 ? 8 : 16));
+    static constexpr int WORDS = GT * M / 32;       // mask words in
+    static constexpr int BYTES = GT * NWIN / 2;     // window bytes out
+};
+
+template <int M>
+__global__ void __launch_bounds__(256)
+    k_slide_pack(const uint32_t *__restrict__ mask, int64_t R, int64_t G, int64_t mwords,
                  int64_t wbytes, uint8_t *__restrict__ wmeta) {
-    const int Ns = m / 2;
-    const int nwin = Ns - 1;
-    __shared__ uint32_t words[PRUNE_THREADS / 32][16];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t row = blockIdx.y;
-    const int64_t g = static_cast<int64_t>(blockIdx.x) * PRUNE_THREADS + threadIdx.x;
-    if (lane < 16) words[warp][lane] = 0u;
-    __syncwarp();
-    if (g < G) {
-        const int64_t b0 = g * m;
-        const uint32_t *mrow = mask + row * mwords;
-        const uint64_t lo = mrow[b0 >> 5];
-        const uint64_t hi = ((b0 >> 5) + 1 < mwords) ? mrow[(b0 >> 5) + 1] : 0u;
-        const uint32_t bits =
-            static_cast<uint32_t>(((hi << 32) | lo) >> (b0 & 31)) & ((1u << m) - 1u);
-        int q[16];
-        int cnt = 0;
-        for (int p = 0; p < m; ++p)
-            if ((bits >> p) & 1u) { if (cnt < 16) q[cnt] = p; ++cnt; }
-        uint32_t nibs = 0;  // nwin nibbles, window w at bits 4w
-        if (cnt != m - 2) {
-            raise_error(ERRBIT_DEVICE);
-        } else {
-            for (int w = 0; w < nwin; ++w) {
-                const int a = q[2 * w] - 2 * w, b = q[2 * w + 1] - 2 * w;
-                if (a < 0 || b > 3 || a >= b) { raise_error(ERRBIT_DEVICE); nibs = 0; break; }
-                nibs |= static_cast<uint32_t>(a | (b << 2)) << (4 * w);
+    using RC = SlideRun<M>;
+    const uint64_t rpr = static_cast<uint64_t>((G + RC::GT - 1) / RC::GT);  // runs per row
+    const uint64_t total = rpr * static_cast<uint64_t>(R);
+    bool bad = false;
+    for (uint64_t idx = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+         idx += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
+        const uint64_t row = idx / rpr, run = idx - row * rpr;
+        const int64_t g0 = static_cast<int64_t>(run) * RC::GT;
+        const uint32_t *mrow = mask + row * mwords + run * RC::WORDS;
+        uint32_t w[RC::WORDS];
+#pragma unroll
+        for (int i = 0; i < RC::WORDS; ++i)
+            w[i] = (static_cast<int64_t>(run) * RC::WORDS + i < mwords) ? __ldg(mrow + i) : 0u;
+        uint32_t ow[(RC::BYTES + 3) / 4];
+#pragma unroll
+        for (int i = 0; i < (RC::BYTES + 3) / 4; ++i) ow[i] = 0u;
+#pragma unroll
+        for (int gi = 0; gi < RC::GT; ++gi) {
+            if (g0 + gi >= G) break;
+            const int b0 = gi * M;  // bit offset of this group in the run
+            uint32_t bits = w[b0 >> 5] >> (b0 & 31);
+            if ((b0 & 31) + M > 32) bits |= w[(b0 >> 5) + 1] << (32 - (b0 & 31));
+            bits &= (1u << M) - 1u;
+            if (__popc(bits) != M - 2) { bad = true; continue; }
+            // survivor k -> window k/2, index q_k - 2*(k/2)
+            uint32_t rem = bits;
+#pragma unroll
+            for (int wv = 0; wv < RC::NWIN; ++wv) {
+                const int qa = __ffs(rem) - 1;
+                rem &= rem - 1u;
+                const int qb = __ffs(rem) - 1;
+                rem &= rem - 1u;
+                const int a = qa - 2 * wv, b = qb - 2 * wv;
+                if (a < 0 || b > 3) bad = true;
+                const int wi = gi * RC::NWIN + wv;                 // nibble index in the run
+                const uint32_t nb = static_cast<uint32_t>((a & 3) | ((b & 3) << 2));
+                ow[wi >> 3] |= nb << (4 * (wi & 7));
             }
         }
-        // warp-local bit offset of this group's first window nibble
-        const uint32_t off = static_cast<uint32_t>(lane) * nwin * 4;
-        const int nb = nwin * 4;
-        atomicOr(&words[warp][off >> 5], nibs << (off & 31));
-        if ((off & 31) + nb > 32) atomicOr(&words[warp][(off >> 5) + 1], nibs >> (32 - (off & 31)));
-    }
-    __syncwarp();
-    // this warp's windows start at window (g - lane) * nwin, an even index
-    const int64_t g_warp0 = g - lane;
-    if (g_warp0 < G) {
-        const int64_t byte0 = g_warp0 * nwin / 2;
-        const int nbytes = 16 * nwin;  // 32 groups * nwin nibbles / 2
-        for (int b = lane; b < nbytes; b += 32) {
-            if (byte0 + b < wbytes)
-                wmeta[row * wbytes + byte0 + b] =
-                    static_cast<uint8_t>((words[warp][b >> 2] >> (8 * (b & 3))) & 0xFFu);
+        const int64_t byte0 = g0 * RC::NWIN / 2;
+        uint8_t *dst = wmeta + row * wbytes + byte0;
+        if (byte0 + RC::BYTES <= wbytes && (reinterpret_cast<uintptr_t>(dst) & 3u) == 0) {
+#pragma unroll
+            for (int i = 0; i < RC::BYTES / 4; ++i) reinterpret_cast<uint32_t *>(dst)[i] = ow[i];
+        } else {
+#pragma unroll
+            for (int i = 0; i < RC::BYTES; ++i)
+                if (byte0 + i < wbytes) dst[i] = static_cast<uint8_t>(ow[i >> 2] >> (8 * (i & 3)));
         }
     }
+    if (bad) raise_error(ERRBIT_DEVICE);
 }
 
 // ---------------------------------------------------------------------------
@@ -507,11 +595,9 @@ extern "C" nm_status nm_score_from_hessian(const double *H, double eps, const ui
     if (!W || !S) return NM_ERR_NULL;
     if (R < 1 || K < 1 || ldw < K) return NM_ERR_SHAPE;
     if (!aligned16(W) || !aligned16(S) || (ldw % 8) != 0) return NM_ERR_ALIGN;
-    const int64_t work = R * ((K + 7) / 8);
-    int64_t blocks = (work + 255) / 256;
-    const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
-    if (blocks > cap) blocks = cap;
-    k_score<<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(H, eps, W, R, K, ldw, S);
+    dim3 grid(static_cast<unsigned>((K + 4095) / 4096), static_cast<unsigned>(R < 65535 ? R : 65535),
+              static_cast<unsigned>((R + 65534) / 65535));
+    k_score<<<grid, 256, 0, as_stream(stream)>>>(H, eps, W, R, K, ldw, S);
     return launch_status();
 }
 
@@ -538,9 +624,10 @@ extern "C" nm_status nm_prune_compress(const float *S, int64_t lds, const uint16
     if (!aligned16(S) || !aligned16(V) || !aligned16(vals) || !aligned16(mask) ||
         (lds % 8) != 0 || (ldv % 8) != 0)
         return NM_ERR_ALIGN;
-    if (R > 65535) return NM_ERR_SHAPE;
+    if (R > 65535LL * 65535LL) return NM_ERR_SHAPE;
     const int64_t G = (K + m - 1) / m;
-    dim3 grid(static_cast<unsigned>((G + PRUNE_THREADS - 1) / PRUNE_THREADS), static_cast<unsigned>(R));
+    dim3 grid(static_cast<unsigned>((G + PRUNE_THREADS - 1) / PRUNE_THREADS),
+              static_cast<unsigned>(R < 65535 ? R : 65535), static_cast<unsigned>((R + 65534) / 65535));
     cudaStream_t s = as_stream(stream);
     uint8_t *meta = (m == 4 && n == 2) ? meta24 : nullptr;
     switch (m) {
@@ -558,12 +645,23 @@ extern "C" nm_status slide_pack(const uint32_t *mask, int64_t R, int64_t K, int 
     if (!mask || !wmeta) return NM_ERR_NULL;
     if (R < 1 || K < 1) return NM_ERR_SHAPE;
     if (m != 4 && m != 6 && m != 8 && m != 10) return NM_ERR_UNSUPPORTED;
-    if (R > 65535) return NM_ERR_SHAPE;
+    if (R > 65535LL * 65535LL) return NM_ERR_SHAPE;
     const int64_t G = (K + m - 1) / m;
     const int64_t mwords = (G * m + 31) / 32;
     const int64_t wbytes = (G * (m / 2 - 1) + 1) / 2;
-    dim3 grid(static_cast<unsigned>((G + PRUNE_THREADS - 1) / PRUNE_THREADS), static_cast<unsigned>(R));
-    k_slide_pack<<<grid, PRUNE_THREADS, 0, as_stream(stream)>>>(mask, G, m, mwords, wbytes, wmeta);
+    cudaStream_t s = as_stream(stream);
+    auto grid_for = [&](int gt) {
+        const int64_t runs = (G + gt - 1) / gt * R;
+        int64_t blocks = (runs + 255) / 256;
+        const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+        return static_cast<unsigned>(blocks < cap ? blocks : cap);
+    };
+    switch (m) {
+        case 4: k_slide_pack<4><<<grid_for(SlideRun<4>::GT), 256, 0, s>>>(mask, R, G, mwords, wbytes, wmeta); break;
+        case 6: k_slide_pack<6><<<grid_for(SlideRun<6>::GT), 256, 0, s>>>(mask, R, G, mwords, wbytes, wmeta); break;
+        case 8: k_slide_pack<8><<<grid_for(SlideRun<8>::GT), 256, 0, s>>>(mask, R, G, mwords, wbytes, wmeta); break;
+        default: k_slide_pack<10><<<grid_for(SlideRun<10>::GT), 256, 0, s>>>(mask, R, G, mwords, wbytes, wmeta); break;
+    }
     return launch_status();
 }
 
