@@ -49,6 +49,30 @@ def peaks():
         return 6650.0, 1590.0, "fallback"
 
 
+PAIR_MODE = {4: "PMODE_SP24", 6: "PMODE_SPLIFT", 8: "PMODE_SP68", 10: "PMODE_SPLIFT"}
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the sparse GEMM from the committed ncu summary
+    profiles/gemm_pair_<workload>.md, if the kernel source is unchanged since."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"gemm_pair_{workload}.md")
+    src = os.path.join(ROOT, "semi_structured_sparse_diag_b200", "csrc", "nm_gemm.cu")
+    try:
+        text = open(path).read()
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    fields = dict(ln.split(":", 1) for ln in text.splitlines()
+                  if ln.startswith(("traffic_bytes_per_launch:", "source_sha256_16:")))
+    if fields.get("source_sha256_16", "").strip() != sha:
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch"].strip())
+    except (KeyError, ValueError):
+        return None
+
+
 def workload_config(layer: datagen.Layer, l2_note: str):
     G = (layer.K + layer.m - 1) // layer.m
     KL = G * (layer.m // 2 - 1) * 4
@@ -323,14 +347,15 @@ def run_ours(args):
         "speedup_bound": round(K / (KL / 2), 4),
         "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": {
-            "kernel": "k_gemm<MODE_SPLIFT>" if m > 4 else "k_gemm<MODE_SP24>",
+            "kernel": f"k_gemm_pair<{PAIR_MODE[m]}>",
             "bound": "tensor",
             "achieved": round(achieved, 2),
             "peak": round(sparse_peak, 1),
             "peak_source": f"2 x {peak_src} dense bf16 burst ({bf16_tf} TFLOP/s)",
             "unit": "TFLOP/s",
             "frac": round(achieved / sparse_peak, 4),
-            "traffic": None,
+            "traffic": recorded_traffic(layer.name),
+            "traffic_source": f"profiles/gemm_pair_{layer.name}.md (ncu dram read+write per launch)",
             "per_unit": "2*R*K'pad flops per token; units per launch = T tokens",
         },
         "e2e": {
