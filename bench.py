@@ -49,7 +49,7 @@ def peaks():
         return 6650.0, 1590.0, "fallback"
 
 
-PAIR_MODE = {4: "PMODE_SP24", 6: "PMODE_SPLIFT", 8: "PMODE_SP68", 10: "PMODE_SPLIFT"}
+PAIR_MODE = {4: "PMODE_SP24", 6: "PMODE_SP24 on K'", 8: "PMODE_SP68T", 10: "PMODE_SP24 on K'"}
 
 
 def recorded_traffic(workload: str):
@@ -175,6 +175,8 @@ def run_ours(args):
     nw = G * (m // 2 - 1)
     wmeta = torch.empty((R, (nw + 1) // 2), dtype=torch.uint8, device=dev) if m > 4 else None
     packed = torch.empty(lib.nm_sparse_prepare_bytes(R, K, m), dtype=torch.uint8, device=dev)
+    gws_bytes = lib.nm_sparse_gemm_workspace_bytes(T, K, m)
+    gws = torch.empty(max(1, gws_bytes), dtype=torch.uint8, device=dev)
     ldy = (R + 7) // 8 * 8
     Y = torch.empty((T, ldy), dtype=torch.bfloat16, device=dev)
     Yd = torch.empty((T, ldy), dtype=torch.bfloat16, device=dev)
@@ -232,9 +234,9 @@ def run_ours(args):
         cnt += 2
         if ev is not None:
             ev[4].record(stream)
-        chk(lib.nm_sparse_gemm(Xs.data_ptr(), T, K, K, packed.data_ptr(), R, m, Y.data_ptr(), ldy, s),
-            "sparse_gemm")
-        cnt += 1
+        chk(lib.nm_sparse_gemm(Xs.data_ptr(), T, K, K, packed.data_ptr(), R, m, Y.data_ptr(), ldy,
+                               gws.data_ptr(), gws_bytes, s), "sparse_gemm")
+        cnt += 1 if m == 4 else 2  # + the middle-window gather (6:8) or the lift (4:6, 8:10)
         if ev is not None:
             ev[5].record(stream)
         chk(lib.nm_dense_gemm(Xs.data_ptr(), T, K, K, Wdense.data_ptr(), R, K, Yd.data_ptr(), ldy, s),

@@ -191,12 +191,22 @@ nm_status nm_sparse_prepare(const uint16_t *vals, const uint8_t *wmeta, int64_t 
  *   Y[t, r] = sum_k X[t,k] * (mask (.) V)[r,k], fp32 accumulation in tensor
  *   memory, bf16 output (round to nearest even).
  *   X : [T x K] bf16, ldx >= K, ldx % 8 == 0.   Y : [T x R] bf16, ldy >= R.
- *   packed: from nm_sparse_prepare(..., R, K, m, ...).  m in {4, 6, 8, 10};
- *   for m > 4 the activations are lifted inside the kernel's shared-memory
- *   staging (no X' in global memory).                                       */
+ *   packed: from nm_sparse_prepare(..., R, K, m, ...).  m in {4, 6, 8, 10}.
+ *   Activation lifting (SlideSparse sec. 2B), by pattern:
+ *     2:4  none;
+ *     6:8  two thirds of the lifted operand are tiles of X itself (windows 0
+ *          and 2 of every group are X's own columns), loaded straight into the
+ *          GEMM's shared-memory staging; the middle windows (columns 2..5 of
+ *          every group) are first gathered into `ws` (T x K/2) and loaded the
+ *          same way;
+ *     4:6, 8:10  the lifted activations X' are written to `ws` (T x K') and the
+ *          product runs as a 2:4 GEMM over K'.
+ *   ws : device scratch of nm_sparse_gemm_workspace_bytes(T, K, m) bytes,
+ *        16-byte aligned (may be NULL when that is 0, i.e. for 2:4).       */
+size_t nm_sparse_gemm_workspace_bytes(int64_t T, int64_t K, int m);
 nm_status nm_sparse_gemm(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
                          const void *packed, int64_t R, int m, uint16_t *Y, int64_t ldy,
-                         void *stream);
+                         void *ws, size_t ws_bytes, void *stream);
 
 /* a8: dense reference GEMM on the tensor cores, Y = X * W^T (W = mask (.) V
  * densified by the caller), fp32 accumulation, bf16 output.                */

@@ -39,6 +39,15 @@ nm_status nm_gemm_1cta(int sparse, const uint16_t *X, int64_t T, int64_t K, int6
                        const void *W_or_packed, int64_t R, int64_t ldw, uint16_t *Y, int64_t ldy,
                        void *stream);
 
+/* Ablation: the same product as nm_sparse_gemm with the whole activation lift
+ * done inside the GEMM (no workspace): for 6:8, lift warps copy columns 2..5
+ * of every group from the two raw X tiles in shared memory into the third
+ * stage; for 4:6 / 8:10 they copy every window's columns from X with cp.async.
+ * Same arguments and output as nm_sparse_gemm (without ws).                */
+nm_status nm_sparse_gemm_fused(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
+                               const void *packed, int64_t R, int m, uint16_t *Y, int64_t ldy,
+                               void *stream);
+
 #ifdef __cplusplus
 }
 #endif

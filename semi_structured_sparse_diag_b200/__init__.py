@@ -29,7 +29,8 @@ EXPORTED = (
     "nm_hessian_workspace_bytes", "nm_hessian_diag", "nm_score", "nm_score_from_hessian",
     "nm_prune_compress", "slide_pack", "lift_activations", "nm_sparse_prepare_bytes",
     "nm_sparse_prepare", "nm_sparse_gemm", "nm_dense_gemm", "nm_ternary_workspace_bytes",
-    "nm_ternary_quantize", "nm_hessian_diag_noalloc", "nm_probe_mma", "nm_probe_copy", "nm_gemm_1cta",
+    "nm_ternary_quantize", "nm_hessian_diag_noalloc", "nm_probe_mma", "nm_probe_copy", "nm_gemm_1cta", "nm_sparse_gemm_workspace_bytes",
+    "nm_sparse_gemm_fused",
 )
 
 _P, _I64, _I, _D, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_size_t
@@ -46,7 +47,9 @@ _SIGS = {
     "lift_activations": (_I, [_P, _I64, _I64, _I64, _I, _P, _I64, _P]),
     "nm_sparse_prepare_bytes": (_SZ, [_I64, _I64, _I]),
     "nm_sparse_prepare": (_I, [_P, _P, _I64, _I64, _I, _P, _SZ, _P]),
-    "nm_sparse_gemm": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I, _P, _I64, _P]),
+    "nm_sparse_gemm": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I, _P, _I64, _P, _SZ, _P]),
+    "nm_sparse_gemm_workspace_bytes": (_SZ, [_I64, _I64, _I]),
+    "nm_sparse_gemm_fused": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I, _P, _I64, _P]),
     "nm_dense_gemm": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _I64, _P]),
     "nm_ternary_workspace_bytes": (_SZ, [_I64]),
     "nm_ternary_quantize": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _SZ, _P]),
@@ -228,13 +231,23 @@ def sparse_prepare(vals, wmeta, R, K, m, packed=None, stream=None):
     return packed
 
 
-def sparse_gemm(X, packed, R, m, Y=None, stream=None):
+def sparse_gemm(X, packed, R, m, Y=None, ws=None, stream=None, fused=False):
+    """Y = X * W_sparse^T.  fused=True runs the in-kernel-lift variant (ablation)."""
     X = _bf16(X, "X")
     T, K = X.shape
+    lib = load()
     if Y is None:
         Y = torch.empty((T, (R + 7) // 8 * 8), dtype=torch.bfloat16, device=X.device)[:, :R]
-    _check(load().nm_sparse_gemm(_ptr(X), T, K, _ld(X), _ptr(packed), R, m, _ptr(Y), _ld(Y),
-                                 _stream(stream)), "nm_sparse_gemm")
+    if fused:
+        _check(lib.nm_sparse_gemm_fused(_ptr(X), T, K, _ld(X), _ptr(packed), R, m, _ptr(Y),
+                                        _ld(Y), _stream(stream)), "nm_sparse_gemm_fused")
+        return Y
+    need = lib.nm_sparse_gemm_workspace_bytes(T, K, m)
+    if ws is None and need:
+        ws = torch.empty(need, dtype=torch.uint8, device=X.device)
+    _check(lib.nm_sparse_gemm(_ptr(X), T, K, _ld(X), _ptr(packed), R, m, _ptr(Y), _ld(Y),
+                              _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)),
+           "nm_sparse_gemm")
     return Y
 
 

@@ -409,16 +409,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 //               SPLIFT: copy each window's 4 columns of X from global memory
 //               into the swizzled B buffer with cp.async, up to three stages
 //               in flight (each warp arrives: 4 warps x 2 CTAs);
-//               SP68:   raw blocks are TMA tiles of X (local xfull[s]); warp 2
-//               forwards their arrival to the leader (counted as 4), the lift
-//               warps copy columns 2..5 of every group out of the two raw stages
-//               into the third (odd) stage, then each signals it.
+//               SP68:   raw blocks are TMA tiles of X counted on the leader's
+//               full[s] like any other operand; warp 2 of the leader relays
+//               their arrival to the peer CTA (xfull[s] there), and the lift
+//               warps copy columns 2..5 of every group out of the two raw
+//               stages into the third (odd) stage, then each signals it.
 // Stages: a ring of S shared-memory stages per CTA; empty[s] and acc_full[b]
 // are armed in both CTAs by multicast tcgen05.commit from the leader; in the
 // lift modes empty[s] also waits for the 4 local lift warps (a raw stage is
 // not refilled before the lift has read it).
 // ===========================================================================
-enum { PMODE_DENSE = 0, PMODE_SP24 = 1, PMODE_SPLIFT = 2, PMODE_SP68 = 3 };
+// PMODE_SP68T: 6:8 with every B block a TMA tile -- raw blocks from X, middle
+// windows from X_mid (gathered by k_gather_mid before the GEMM).
+enum { PMODE_DENSE = 0, PMODE_SP24 = 1, PMODE_SPLIFT = 2, PMODE_SP68 = 3, PMODE_SP68T = 4 };
 
 template <int MODE>
 struct PairCfg {
@@ -450,13 +453,15 @@ __device__ __forceinline__ bool pair_needs_lift(int mode, int64_t kb) {
 
 // B by TMA: the stage's B half is a plain tile of X
 __device__ __forceinline__ bool pair_b_by_tma(int mode, int64_t kb) {
-    return mode == PMODE_DENSE || mode == PMODE_SP24 || (mode == PMODE_SP68 && (kb % 3) != 2);
+    return mode == PMODE_DENSE || mode == PMODE_SP24 || mode == PMODE_SP68T ||
+           (mode == PMODE_SP68 && (kb % 3) != 2);
 }
 
 template <int MODE>
 __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
+                const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmE,
+                const __grid_constant__ CUtensorMap tmY,
                 const uint16_t *__restrict__ X, int64_t T, int64_t K, int64_t ldx, int64_t R,
                 int64_t nkb, int m) {
     using C = PairCfg<MODE>;
@@ -497,6 +502,7 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
         prefetch_tmap(&tmB);
         prefetch_tmap(&tmY);
         if (C::SPARSE) prefetch_tmap(&tmE);
+        if (MODE == PMODE_SP68T) prefetch_tmap(&tmB2);
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
@@ -522,12 +528,9 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
                     const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
                     if (it >= S && !mbar_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
                     const bool btma = pair_b_by_tma(MODE, kb);
-                    // B tiles go to the leader's full[s], except in SP68 where
-                    // the lift warps of each CTA watch their own xfull[s]
-                    const bool b_to_full = btma && MODE != PMODE_SP68;
                     if (rank == 0) {
                         const uint32_t tx = 2u * static_cast<uint32_t>(
-                            C::A_BYTES + C::E_BYTES + (b_to_full ? C::B_BYTES : 0));
+                            C::A_BYTES + C::E_BYTES + (btma ? C::B_BYTES : 0));
                         mbar_arrive_expect_tx(&full[s], tx);
                     }
                     const uint32_t bar = mapa_shared(&full[s], 0);
@@ -535,20 +538,16 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
                     if (C::SPARSE)
                         tma_load_2d_pair(stE(s), &tmE, bar, 0,
                                          static_cast<int32_t>(((mt2 * 2 + rank) * nkb + kb) * 8));
-                    if (btma && MODE == PMODE_SP68) {
-                        const int64_t x0 = (kb / 3) * 256 + (kb % 3) * 128;
-                        mbar_arrive_expect_tx(&xfull[s], C::B_BYTES);
-                        tma_load_2d(stB(s), &tmB, &xfull[s], static_cast<int32_t>(x0), brow);
-                        tma_load_2d(stB(s) + C::BH * 128, &tmB, &xfull[s],
-                                    static_cast<int32_t>(x0 + 64), brow);
-                    } else if (btma) {
+                    if (btma) {
                         if (MODE == PMODE_DENSE) {
                             tma_load_2d_pair(stB(s), &tmB, bar, static_cast<int32_t>(kb * 64), brow);
                         } else {
+                            const bool mid = MODE == PMODE_SP68T && (kb % 3) == 2;
                             const int64_t x0 = MODE == PMODE_SP24 ? kb * 128
-                                                                  : (kb / 3) * 256 + (kb % 3) * 128;
-                            tma_load_2d_pair(stB(s), &tmB, bar, static_cast<int32_t>(x0), brow);
-                            tma_load_2d_pair(stB(s) + C::BH * 128, &tmB, bar,
+                                               : (mid ? (kb / 3) * 128 : (kb / 3) * 256 + (kb % 3) * 128);
+                            const CUtensorMap *tb = mid ? &tmB2 : &tmB;
+                            tma_load_2d_pair(stB(s), tb, bar, static_cast<int32_t>(x0), brow);
+                            tma_load_2d_pair(stB(s) + C::BH * 128, tb, bar,
                                              static_cast<int32_t>(x0 + 64), brow);
                         }
                     }
@@ -564,6 +563,7 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
         if (rank == 0 && lane == 0) {
             const uint32_t idesc = make_idesc_bf16(256, C::BN, C::SPARSE, 0);
             int64_t it = 0, ti = 0;
+            uint32_t lbits = 0;  // phase of lifted[s] (one phase per lifted use of stage s)
             bool ok = true;
             for (int64_t tile = cluster; tile < ntiles && ok; tile += nclusters, ++ti) {
                 const int buf = static_cast<int>(ti % C::ACC_BUFS);
@@ -578,7 +578,10 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
                     const int s = static_cast<int>(it % S);
                     const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
                     if (!mbar_wait(&full[s], ph)) { ok = false; break; }
-                    if (C::LIFT && !mbar_wait_cluster(&lifted[s], ph)) { ok = false; break; }
+                    if (C::LIFT && pair_needs_lift(MODE, kb)) {
+                        if (!mbar_wait_cluster(&lifted[s], (lbits >> s) & 1u)) { ok = false; break; }
+                        lbits ^= 1u << s;
+                    }
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(stA(s)), b0 = smem_u32(stB(s));
                     if (!C::SPARSE) {
@@ -653,23 +656,23 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
         }
         if (lane == 0) bulk_wait_group0();
         __syncwarp();
-    } else if (MODE == PMODE_SP68 && warp == 2) {
-        // ---------------------------------------------------------- forwarder
-        // raw blocks: tell the leader as soon as this CTA's TMA tile has landed
-        const uint32_t lifted_cl0 = mapa_shared(&lifted[0], 0);
+    } else if (MODE == PMODE_SP68 && warp == 2 && rank == 0) {
+        // ---------------------------------------------------------- relay
+        // raw blocks: once the leader's full[s] shows both CTAs' tiles have
+        // landed, tell the peer CTA's lift warps (its xfull[s])
+        const uint32_t xfull_peer0 = mapa_shared(&xfull[0], 1);
         int64_t it = 0;
-        uint32_t xbits = 0;
         bool ok = true;
         for (int64_t tile = cluster; tile < ntiles && ok; tile += nclusters) {
             for (int64_t kb = 0; kb < nkb; ++kb, ++it) {
                 if (kb % 3 == 2) continue;
                 const int s = static_cast<int>(it % S);
-                if (!__all_sync(0xffffffffu, mbar_wait(&xfull[s], (xbits >> s) & 1u))) {
+                const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
+                if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) {
                     ok = false;
                     break;
                 }
-                xbits ^= 1u << s;
-                if (lane == 0) mbar_arrive_cluster_n(lifted_cl0 + static_cast<uint32_t>(s) * 8u, 4u);
+                if (lane == 0) mbar_arrive_cluster(xfull_peer0 + static_cast<uint32_t>(s) * 8u);
             }
         }
     } else if (C::LIFT && warp >= 12) {
@@ -745,12 +748,19 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
                     const int s = static_cast<int>(it % S);
                     const int type = static_cast<int>(kb % 3);
                     if (type < 2) {
-                        // raw block: its B half is a TMA tile of X in this CTA
-                        if (!__all_sync(0xffffffffu, mbar_wait(&xfull[s], (xbits >> s) & 1u))) {
+                        // raw block: its B half is a TMA tile of X in this CTA; the
+                        // leader sees it land on full[s], the peer is told by the relay
+                        bool landed;
+                        if (rank == 0) {
+                            landed = mbar_wait(&full[s], static_cast<uint32_t>((it / S) & 1));
+                        } else {
+                            landed = mbar_wait_cluster(&xfull[s], (xbits >> s) & 1u);
+                            xbits ^= 1u << s;
+                        }
+                        if (!__all_sync(0xffffffffu, landed)) {
                             ok = false;
                             break;
                         }
-                        xbits ^= 1u << s;
                         // the odd stage of this super-block must be free
                         const int64_t it_odd = it + (2 - type);
                         const int so = static_cast<int>(it_odd % S);
@@ -808,6 +818,41 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    }
+}
+
+
+// ---------------------------------------------------------------------------
+// 6:8 middle windows: X_mid[t, 4g + i] = X[t, 8g + 2 + i] (i < 4), zero past K.
+// One thread per two groups: two 16-byte loads, one 16-byte store.
+// grid: x over pairs of groups, y (+65535 z) over tokens.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    k_gather_mid(const uint16_t *__restrict__ X, int64_t T, int64_t K, int64_t ldx, int64_t G,
+                 uint16_t *__restrict__ Xmid, int64_t ldm) {
+    const int64_t t = blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535;
+    const int64_t h = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // group pair
+    if (t >= T || 2 * h >= G) return;
+    const uint16_t *src = X + t * ldx + 16 * h;
+    uint32_t o[4];
+    if (16 * h + 16 <= K) {
+        const uint4 a = __ldg(reinterpret_cast<const uint4 *>(src));
+        const uint4 b = __ldg(reinterpret_cast<const uint4 *>(src) + 1);
+        o[0] = a.y; o[1] = a.z; o[2] = b.y; o[3] = b.z;
+    } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t c = 16 * h + 8 * (j >> 1) + 2 + 2 * (j & 1);
+            const uint32_t lo = c < K ? __ldg(src + (c - 16 * h)) : 0u;
+            const uint32_t hi = c + 1 < K ? __ldg(src + (c + 1 - 16 * h)) : 0u;
+            o[j] = lo | (hi << 16);
+        }
+    }
+    uint16_t *dst = Xmid + t * ldm + 8 * h;
+    if (2 * h + 2 <= G) {
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+    } else {  // last, odd group: four columns only
+        *reinterpret_cast<uint2 *>(dst) = make_uint2(o[0], o[1]);
     }
 }
 
@@ -911,9 +956,9 @@ nm_status launch_gemm_1cta(const CUtensorMap &a, const CUtensorMap &b, const CUt
 
 // ---- persistent CTA-pair kernel
 template <int MODE>
-nm_status launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &e,
-                      const CUtensorMap &y, const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
-                      int64_t R, int64_t nkb, int m, cudaStream_t s) {
+nm_status launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b2,
+                      const CUtensorMap &e, const CUtensorMap &y, const uint16_t *X, int64_t T,
+                      int64_t K, int64_t ldx, int64_t R, int64_t nkb, int m, cudaStream_t s) {
     using Cfg = PairCfg<MODE>;
     if (!set_smem_attr<k_gemm_pair<MODE>>(Cfg::SMEM_BYTES)) return NM_ERR_CUDA;
     const int64_t ntiles = ((T + Cfg::BN - 1) / Cfg::BN) * ((R + 255) / 256);
@@ -932,7 +977,7 @@ nm_status launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensor
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, k_gemm_pair<MODE>, a, b, e, y, X, T, K, ldx, R, nkb, m) !=
+    if (cudaLaunchKernelEx(&cfg, k_gemm_pair<MODE>, a, b, b2, e, y, X, T, K, ldx, R, nkb, m) !=
         cudaSuccess)
         return NM_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
@@ -972,9 +1017,49 @@ extern "C" nm_status nm_sparse_prepare(const uint16_t *vals, const uint8_t *wmet
     return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
 }
 
-extern "C" nm_status nm_sparse_gemm(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
-                                    const void *packed, int64_t R, int m, uint16_t *Y, int64_t ldy,
-                                    void *stream) {
+// extra device memory the online phase needs for (2N-2):2N patterns: the
+// gathered middle windows (6:8) or the lifted activations (4:6, 8:10)
+struct GemmWs {
+    int64_t ld;      // leading dimension (elements) of the staged activations
+    int64_t cols;    // their logical width
+    size_t bytes;
+};
+
+static GemmWs gemm_ws(int64_t T, int64_t K, int m) {
+    GemmWs w{0, 0, 0};
+    if (T < 1 || K < 1 || m == 4) return w;
+    const int64_t G = (K + m - 1) / m;
+    w.cols = m == 8 ? G * 4 : G * (m / 2 - 1) * 4;
+    w.ld = (w.cols + 7) / 8 * 8;
+    w.bytes = static_cast<size_t>(T) * static_cast<size_t>(w.ld) * 2;
+    return w;
+}
+
+extern "C" size_t nm_sparse_gemm_workspace_bytes(int64_t T, int64_t K, int m) {
+    if (m != 4 && m != 6 && m != 8 && m != 10) return 0;
+    return gemm_ws(T, K, m).bytes;
+}
+
+namespace {
+
+struct SparseMaps {
+    CUtensorMap a, e, y;
+    bool ok;
+};
+
+SparseMaps sparse_maps(const void *packed, const PackedGeom &p, const uint16_t *Y, int64_t T,
+                       int64_t R, int64_t ldy) {
+    SparseMaps mp;
+    const uint8_t *meta = static_cast<const uint8_t *>(packed) + p.vals_bytes;
+    mp.ok = make_tmap_bf16(&mp.a, packed, p.Rpad, p.KLpad / 2, p.KLpad / 2, 64, BM, true) &&
+            make_tmap_2d(&mp.e, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, meta, (p.Rpad / BM) * p.nkb * 8,
+                         256, 256, 256, 8, false) &&
+            make_tmap_bf16(&mp.y, Y, T, R, ldy, 32, 32, false);
+    return mp;
+}
+
+nm_status check_sparse_args(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, const void *packed,
+                            int64_t R, int m, const uint16_t *Y, int64_t ldy) {
     if (!X || !packed || !Y) return NM_ERR_NULL;
     if (T < 1 || K < 1 || R < 1 || ldx < K || ldy < R) return NM_ERR_SHAPE;
     if (m != 4 && m != 6 && m != 8 && m != 10) return NM_ERR_UNSUPPORTED;
@@ -982,18 +1067,62 @@ extern "C" nm_status nm_sparse_gemm(const uint16_t *X, int64_t T, int64_t K, int
         return NM_ERR_ALIGN;
     const PackedGeom p = packed_geom(R, K, m);
     if (p.nkb > 0x7FFFFFFF / 8 || (p.Rpad / BM) * p.nkb * 8 > 0x7FFFFFFF) return NM_ERR_SHAPE;
-    CUtensorMap ta, tb, te, ty;
-    const uint8_t *meta = static_cast<const uint8_t *>(packed) + p.vals_bytes;
-    if (!make_tmap_bf16(&ta, packed, p.Rpad, p.KLpad / 2, p.KLpad / 2, 64, BM, true) ||
-        !make_tmap_2d(&te, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, meta, (p.Rpad / BM) * p.nkb * 8, 256,
-                      256, 256, 8, false) ||
-        !make_tmap_bf16(&tb, X, T, K, ldx, 64, 128, true) ||
-        !make_tmap_bf16(&ty, Y, T, R, ldy, 32, 32, false))
-        return NM_ERR_CUDA;
+    return NM_OK;
+}
+
+}  // namespace
+
+extern "C" nm_status nm_sparse_gemm(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
+                                    const void *packed, int64_t R, int m, uint16_t *Y, int64_t ldy,
+                                    void *ws, size_t ws_bytes, void *stream) {
+    nm_status st = check_sparse_args(X, T, K, ldx, packed, R, m, Y, ldy);
+    if (st != NM_OK) return st;
+    const GemmWs w = gemm_ws(T, K, m);
+    if (w.bytes > 0 && (!ws || ws_bytes < w.bytes)) return NM_ERR_WORKSPACE;
+    if (w.bytes > 0 && !aligned16(ws)) return NM_ERR_ALIGN;
+    const PackedGeom p = packed_geom(R, K, m);
+    const SparseMaps mp = sparse_maps(packed, p, Y, T, R, ldy);
+    if (!mp.ok) return NM_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (m == 4) return launch_pair<PMODE_SP24>(ta, tb, te, ty, X, T, K, ldx, R, p.nkb, m, s);
-    if (m == 8) return launch_pair<PMODE_SP68>(ta, tb, te, ty, X, T, K, ldx, R, p.nkb, m, s);
-    return launch_pair<PMODE_SPLIFT>(ta, tb, te, ty, X, T, K, ldx, R, p.nkb, m, s);
+    CUtensorMap tb, tb2;
+    if (m == 4) {
+        if (!make_tmap_bf16(&tb, X, T, K, ldx, 64, 128, true)) return NM_ERR_CUDA;
+        return launch_pair<PMODE_SP24>(mp.a, tb, tb, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, s);
+    }
+    uint16_t *stage = static_cast<uint16_t *>(ws);
+    if (m == 8) {
+        // raw blocks straight from X, middle windows from the gathered X_mid
+        const int64_t pairs = (p.G + 1) / 2;
+        dim3 grid(static_cast<unsigned>((pairs + 255) / 256), static_cast<unsigned>(T < 65535 ? T : 65535),
+                  static_cast<unsigned>((T + 65534) / 65535));
+        k_gather_mid<<<grid, 256, 0, s>>>(X, T, K, ldx, p.G, stage, w.ld);
+        if (cudaGetLastError() != cudaSuccess) return NM_ERR_CUDA;
+        if (!make_tmap_bf16(&tb, X, T, K, ldx, 64, 128, true) ||
+            !make_tmap_bf16(&tb2, stage, T, w.cols, w.ld, 64, 128, true))
+            return NM_ERR_CUDA;
+        return launch_pair<PMODE_SP68T>(mp.a, tb, tb2, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, s);
+    }
+    // 4:6, 8:10: the lifted activations X' (natural window order) then a 2:4
+    // GEMM over K' -- the packed operand is laid out identically
+    st = lift_activations(X, T, K, ldx, m, stage, w.ld, stream);
+    if (st != NM_OK) return st;
+    if (!make_tmap_bf16(&tb, stage, T, w.cols, w.ld, 64, 128, true)) return NM_ERR_CUDA;
+    return launch_pair<PMODE_SP24>(mp.a, tb, tb, mp.e, mp.y, stage, T, w.cols, w.ld, R, p.nkb, 4, s);
+}
+
+extern "C" nm_status nm_sparse_gemm_fused(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
+                                          const void *packed, int64_t R, int m, uint16_t *Y,
+                                          int64_t ldy, void *stream) {
+    nm_status st = check_sparse_args(X, T, K, ldx, packed, R, m, Y, ldy);
+    if (st != NM_OK) return st;
+    const PackedGeom p = packed_geom(R, K, m);
+    const SparseMaps mp = sparse_maps(packed, p, Y, T, R, ldy);
+    CUtensorMap tb;
+    if (!mp.ok || !make_tmap_bf16(&tb, X, T, K, ldx, 64, 128, true)) return NM_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (m == 4) return launch_pair<PMODE_SP24>(mp.a, tb, tb, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, s);
+    if (m == 8) return launch_pair<PMODE_SP68>(mp.a, tb, tb, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, s);
+    return launch_pair<PMODE_SPLIFT>(mp.a, tb, tb, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, s);
 }
 
 extern "C" nm_status nm_dense_gemm(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
@@ -1010,7 +1139,7 @@ extern "C" nm_status nm_dense_gemm(const uint16_t *X, int64_t T, int64_t K, int6
         !make_tmap_bf16(&ty, Y, T, R, ldy, 32, 32, false))
         return NM_ERR_CUDA;
     const int64_t nkb = (K + 63) / 64;
-    return launch_pair<PMODE_DENSE>(ta, tb, ta, ty, X, T, K, ldx, R, nkb, 4,
+    return launch_pair<PMODE_DENSE>(ta, tb, tb, ta, ty, X, T, K, ldx, R, nkb, 4,
                                     reinterpret_cast<cudaStream_t>(stream));
 }
 

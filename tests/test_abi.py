@@ -50,6 +50,10 @@ def test_size_queries():
     assert lib.nm_sparse_prepare_bytes(256, 512, 5) == 0
     assert lib.nm_sparse_prepare_bytes(0, 512, 4) == 0
     assert lib.nm_ternary_workspace_bytes(100) >= 800
+    assert lib.nm_sparse_gemm_workspace_bytes(2048, 4096, 4) == 0
+    assert lib.nm_sparse_gemm_workspace_bytes(2048, 4096, 8) == 2048 * 2048 * 2      # T x K/2
+    assert lib.nm_sparse_gemm_workspace_bytes(7, 1003, 6) == 7 * 1344 * 2           # T x K'
+    assert lib.nm_sparse_gemm_workspace_bytes(16, 8195, 10) == 16 * 13120 * 2
 
 
 # fake but 16-byte aligned device addresses: validation fails before any use
@@ -74,9 +78,12 @@ MIS = 0x10002
     (lambda l: l.lift_activations(A, 4, 8, 8, 8, A, 8, None), 2),
     (lambda l: l.nm_sparse_prepare(A, A, 4, 8, 4, A, 1, None), 5),
     (lambda l: l.nm_sparse_prepare(A, A, 4, 8, 4, MIS, 1 << 20, None), 3),
-    (lambda l: l.nm_sparse_gemm(A, 4, 8, 8, A, 4, 9, A, 8, None), 4),
-    (lambda l: l.nm_sparse_gemm(A, 4, 8, 8, A, 4, 4, A, 12, None), 3),
-    (lambda l: l.nm_sparse_gemm(A, 4, 8, 4, A, 4, 4, A, 8, None), 2),
+    (lambda l: l.nm_sparse_gemm(A, 4, 8, 8, A, 4, 9, A, 8, None, 0, None), 4),
+    (lambda l: l.nm_sparse_gemm(A, 4, 8, 8, A, 4, 4, A, 12, None, 0, None), 3),
+    (lambda l: l.nm_sparse_gemm(A, 4, 8, 4, A, 4, 4, A, 8, None, 0, None), 2),
+    (lambda l: l.nm_sparse_gemm(A, 4, 16, 16, A, 4, 8, A, 8, None, 0, None), 5),
+    (lambda l: l.nm_sparse_gemm(A, 4, 16, 16, A, 4, 8, A, 8, MIS, 1 << 20, None), 3),
+    (lambda l: l.nm_sparse_gemm_fused(A, 4, 8, 8, A, 4, 9, A, 8, None), 4),
     (lambda l: l.nm_dense_gemm(A, 4, 8, 8, None, 4, 8, A, 8, None), 1),
     (lambda l: l.nm_dense_gemm(A, 4, 8, 8, A, 4, 8, MIS, 8, None), 3),
     (lambda l: l.nm_ternary_quantize(A, 4, 8, 8, A, A, A, 1, None), 5),

@@ -155,6 +155,20 @@ def test_sparse_gemm_vs_oracle(nm, m, R, K, T):
     assert rel_err(Y, Y64) <= GEMM_TOL
 
 
+@pytest.mark.parametrize("m,R,K,T", [(6, 256, 1536, 128), (8, 256, 1024, 128), (10, 256, 1280, 128),
+                                     (8, 200, 1030, 257), (6, 131, 1003, 77), (10, 129, 2050, 16),
+                                     (4, 130, 1030, 200)])
+def test_in_kernel_lift_ablation_vs_oracle(nm, m, R, K, T):
+    # the ablation entry point lifts inside the GEMM (no workspace)
+    X, W, res = _layer(R, K, T, m - 2, m, seed=R + K + T + 1, outliers=2)
+    wm = res["meta24"] if m == 4 else res["wmeta"]
+    packed = nm.sparse_prepare(to_dev(res["vals"]), torch.from_numpy(wm).cuda(), R, K, m)
+    Y = nm.sparse_gemm(to_dev(X, (K + 7) // 8 * 8), packed, R, m, fused=True)
+    _sync_ok(nm)
+    Y64 = oracle.gemm_masked(X, res["mask"], W, m)
+    assert rel_err(bf16_to_f64(to_host_u16(Y)), Y64) <= GEMM_TOL
+
+
 @pytest.mark.parametrize("m", [6, 8, 10])
 def test_fused_lift_equals_two_pass(nm, m):
     # lift_activations + a 2:4 GEMM of width K' versus the fused kernel.  For
@@ -163,7 +177,10 @@ def test_fused_lift_equals_two_pass(nm, m):
     # tiles of X first), so it agrees within rounding.
     R, K, T = 256, 1030, 130
     X, W, res = _layer(R, K, T, m - 2, m, seed=m)
-    Yf = _gemm_sparse(nm, X, res, R, K, m, ldx=1032)
+    wm = res["wmeta"]
+    packed = nm.sparse_prepare(to_dev(res["vals"]), torch.from_numpy(wm).cuda(), R, K, m)
+    Yf = bf16_to_f64(to_host_u16(nm.sparse_gemm(to_dev(X, 1032), packed, R, m, fused=True)))
+    Yl = bf16_to_f64(to_host_u16(nm.sparse_gemm(to_dev(X, 1032), packed, R, m)))
     XL = nm.lift_activations(to_dev(X, 1032), m)
     KL = XL.shape[1]
     packed24 = nm.sparse_prepare(to_dev(res["vals"]), torch.from_numpy(res["wmeta"]).cuda(), R, KL, 4)
@@ -171,10 +188,13 @@ def test_fused_lift_equals_two_pass(nm, m):
     _sync_ok(nm)
     Y64 = oracle.gemm_masked(X, res["mask"], W, m)
     assert rel_err(Y2, Y64) <= GEMM_TOL
+    assert rel_err(Yl, Y64) <= GEMM_TOL
     if m == 8:
         assert rel_err(Yf, Y2) <= 2 ** -7
+        assert np.array_equal(Yl, Yf)   # same K' order and tiles, lift done before or inside
     else:
         assert np.array_equal(Y2, Yf)
+        assert np.array_equal(Yl, Yf)
 
 
 @pytest.mark.parametrize("R,K,T", [(256, 512, 128), (384, 4096, 384)])
