@@ -518,6 +518,79 @@ def run_probe(args):
     print(json.dumps(out), flush=True)
 
 
+def run_ablation(args):
+    """Design-choice evidence: the sparse GEMM variants on one workload, each timed
+    alone (median of 10 after 3 warm-ups, L2 flushed before each run)."""
+    import torch
+
+    import semi_structured_sparse_diag_b200 as nm
+    lib = nm.load()
+    dev = torch.device("cuda", 0)
+    layer = datagen.WORKLOADS[args.workload]
+    X_h, W_h = datagen.layer_inputs(layer)
+    R, K, T, n, m = layer.R, layer.K, layer.T, layer.n, layer.m
+    X = torch.from_numpy(X_h.view(np.int16)).to(dev).view(torch.bfloat16)
+    W = torch.from_numpy(W_h.view(np.int16)).to(dev).view(torch.bfloat16)
+    _, S = nm.score(X, W, eps=layer.eps)
+    mask, vals, meta = nm.prune_compress(S, W, n, m)
+    wm = meta if m == 4 else nm.slide_pack(mask, K, m)
+    packed = nm.sparse_prepare(vals, wm, R, K, m)
+    bits = ((mask.unsqueeze(-1) >> torch.arange(32, device=dev, dtype=torch.int32)) & 1)
+    Wd = torch.where(bits.reshape(R, -1)[:, :K].bool(), W, torch.zeros_like(W)).contiguous()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    s = torch.cuda.current_stream().cuda_stream
+    Y = torch.empty((T, (R + 7) // 8 * 8), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(1, lib.nm_sparse_gemm_workspace_bytes(T, K, m)), dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        ts = []
+        for i in range(13):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            st = fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if st != 0:
+                raise nm.NMError(lib.nm_status_string(st).decode())
+            if i >= 3:
+                ts.append(e0.elapsed_time(e1))
+        nm.check_device_error()
+        return sorted(ts)[len(ts) // 2]
+
+    ldy = Y.stride(0)
+    res = {}
+    res["library (TMA operands; 6:8 gather / 4:6, 8:10 lift before the GEMM)"] = timed(
+        lambda: lib.nm_sparse_gemm(X.data_ptr(), T, K, K, packed.data_ptr(), R, m, Y.data_ptr(), ldy,
+                                   ws.data_ptr(), ws.numel(), s))
+    res["in-kernel lift (nm_sparse_gemm_fused)"] = timed(
+        lambda: lib.nm_sparse_gemm_fused(X.data_ptr(), T, K, K, packed.data_ptr(), R, m, Y.data_ptr(),
+                                         ldy, s))
+    res["own dense GEMM, CTA pair (nm_dense_gemm)"] = timed(
+        lambda: lib.nm_dense_gemm(X.data_ptr(), T, K, K, Wd.data_ptr(), R, K, Y.data_ptr(), ldy, s))
+    res["own dense GEMM, single CTA (nm_gemm_1cta)"] = timed(
+        lambda: lib.nm_gemm_1cta(0, X.data_ptr(), T, K, K, Wd.data_ptr(), R, K, Y.data_ptr(), ldy, s))
+    if m == 4:
+        res["2:4 sparse, single CTA (nm_gemm_1cta)"] = timed(
+            lambda: lib.nm_gemm_1cta(1, X.data_ptr(), T, K, K, packed.data_ptr(), R, 0, Y.data_ptr(),
+                                     ldy, s))
+    Yt = torch.empty((T, R), dtype=torch.bfloat16, device=dev)
+    res["torch.matmul bf16 (cuBLAS), context"] = timed(lambda: (torch.matmul(X, Wd.t(), out=Yt), 0)[1])
+    G = (K + m - 1) // m
+    KL = G * (m // 2 - 1) * 4
+    nkb = 3 * ((G + 31) // 32) if m == 8 else (KL + 127) // 128
+    flops_lift = 2.0 * T * R * nkb * 128
+    out = {"ablation": layer.name, "pattern": f"{n}:{m}", "R": R, "K": K, "T": T, "ms": {}, "pct_of_peak": {}}
+    _, bf16_tf, _ = peaks()
+    for k, v in res.items():
+        out["ms"][k] = round(v, 4)
+        sparse = "dense" not in k and "torch" not in k
+        f = flops_lift if sparse else 2.0 * T * R * K
+        pk = 2 * bf16_tf if sparse else bf16_tf
+        out["pct_of_peak"][k] = round(100 * f / (v * 1e-3) / 1e12 / pk, 1)
+    print(json.dumps(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -528,9 +601,13 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--probe", action="store_true", help="run the tensor-pipe / HBM probes instead")
+    ap.add_argument("--ablation", action="store_true", help="time the GEMM variants instead")
     args = ap.parse_args()
     if args.probe:
         run_probe(args)
+        return
+    if args.ablation:
+        run_ablation(args)
         return
     if args.warmup < 3:
         args.warmup = 3
