@@ -177,6 +177,8 @@ def run_ours(args):
     packed = torch.empty(lib.nm_sparse_prepare_bytes(R, K, m), dtype=torch.uint8, device=dev)
     gws_bytes = lib.nm_sparse_gemm_workspace_bytes(T, K, m)
     gws = torch.empty(max(1, gws_bytes), dtype=torch.uint8, device=dev)
+    dws_bytes = lib.nm_dense_gemm_workspace_bytes(T, K, R)
+    dws = torch.empty(max(1, dws_bytes), dtype=torch.uint8, device=dev)
     ldy = (R + 7) // 8 * 8
     Y = torch.empty((T, ldy), dtype=torch.bfloat16, device=dev)
     Yd = torch.empty((T, ldy), dtype=torch.bfloat16, device=dev)
@@ -239,8 +241,8 @@ def run_ours(args):
         cnt += 1 if m == 4 else 2  # + the middle-window gather (6:8) or the lift (4:6, 8:10)
         if ev is not None:
             ev[5].record(stream)
-        chk(lib.nm_dense_gemm(Xs.data_ptr(), T, K, K, Wdense.data_ptr(), R, K, Yd.data_ptr(), ldy, s),
-            "dense_gemm")
+        chk(lib.nm_dense_gemm(Xs.data_ptr(), T, K, K, Wdense.data_ptr(), R, K, Yd.data_ptr(), ldy,
+                              dws.data_ptr(), dws_bytes, s), "dense_gemm")
         cnt += 1
         if ev is not None:
             ev[6].record(stream)
@@ -559,15 +561,24 @@ def run_ablation(args):
         return sorted(ts)[len(ts) // 2]
 
     ldy = Y.stride(0)
+    dws = torch.empty(lib.nm_dense_gemm_workspace_bytes(T, K, R), dtype=torch.uint8, device=dev)
+    sparse_call = lambda: lib.nm_sparse_gemm(X.data_ptr(), T, K, K, packed.data_ptr(), R, m, Y.data_ptr(),
+                                             ldy, ws.data_ptr(), ws.numel(), s)
+    dense_call = lambda: lib.nm_dense_gemm(X.data_ptr(), T, K, K, Wd.data_ptr(), R, K, Y.data_ptr(), ldy,
+                                           dws.data_ptr(), dws.numel(), s)
     res = {}
-    res["library (TMA operands; 6:8 gather / 4:6, 8:10 lift before the GEMM)"] = timed(
-        lambda: lib.nm_sparse_gemm(X.data_ptr(), T, K, K, packed.data_ptr(), R, m, Y.data_ptr(), ldy,
-                                   ws.data_ptr(), ws.numel(), s))
+    res["library (TMA operands; 6:8 gather / 4:6, 8:10 lift before the GEMM)"] = timed(sparse_call)
+    for pol, nm_pol in ((1, "whole tiles"), (2, "stream-K")):
+        nm.set_gemm_schedule(pol)
+        try:
+            res[f"library, {nm_pol} forced"] = timed(sparse_call)
+            res[f"own dense GEMM, CTA pair, {nm_pol} forced"] = timed(dense_call)
+        finally:
+            nm.set_gemm_schedule(0)
     res["in-kernel lift (nm_sparse_gemm_fused)"] = timed(
         lambda: lib.nm_sparse_gemm_fused(X.data_ptr(), T, K, K, packed.data_ptr(), R, m, Y.data_ptr(),
                                          ldy, s))
-    res["own dense GEMM, CTA pair (nm_dense_gemm)"] = timed(
-        lambda: lib.nm_dense_gemm(X.data_ptr(), T, K, K, Wd.data_ptr(), R, K, Y.data_ptr(), ldy, s))
+    res["own dense GEMM, CTA pair (nm_dense_gemm)"] = timed(dense_call)
     res["own dense GEMM, single CTA (nm_gemm_1cta)"] = timed(
         lambda: lib.nm_gemm_1cta(0, X.data_ptr(), T, K, K, Wd.data_ptr(), R, K, Y.data_ptr(), ldy, s))
     if m == 4:

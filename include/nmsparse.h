@@ -24,17 +24,18 @@
  *                     SlideSparse sec. 2B "Elevacao de Ativacao".
  *   nm_sparse_prepare canonical values + window metadata -> the GEMM's operand
  *                     layout. SlideSparse sec. 2C item 2 (initialisation phase).
- *   nm_sparse_gemm    Y = X * W_sparse^T on the sparse tensor cores; for
- *                     (2N-2):2N the lift happens inside the GEMM's shared-memory
- *                     staging. SlideSparse sec. 2C item 3 (online phase).
+ *   nm_sparse_gemm    Y = X * W_sparse^T on the sparse tensor cores, over the
+ *                     lifted activations for (2N-2):2N. SlideSparse sec. 2C
+ *                     item 3 (online phase).
  *   nm_dense_gemm     Y = X * W^T, dense tcgen05 GEMM (the comparison point).
  *   nm_ternary_quantize  gamma = mean|W|, W_q = clip(rint(W/gamma),-1,1)*gamma.
  *                     Sparse-BitNet sec. 1 item 1 (BitNet b1.58 ternary weights).
  *
  * Conventions shared by every call
  *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
- *     allocates nothing; its only state is one device error word and the static
- *     scratch array of nm_hessian_diag_noalloc.
+ *     allocates nothing; its only state is one device error word, the static
+ *     scratch array of nm_hessian_diag_noalloc and the GEMM schedule setting
+ *     of nm_gemm_set_schedule.
  *   - bf16 tensors are passed as uint16_t bit patterns.  Matrices are row-major
  *     with a leading dimension (elements) ld >= the row length.
  *   - X is [T x K] (tokens x in-features), W is [R x K] (out x in features),
@@ -172,8 +173,9 @@ nm_status slide_pack(const uint32_t *mask, int64_t R, int64_t K, int m, uint8_t 
 /* a5 (standalone form): activation lifting (SlideSparse, sec. 2B).
  *   XL[t, g*4(N-1) + 4w + i] = X[t, g*m + 2w + i], 0 where g*m+2w+i >= K.
  *   X : [T x K] bf16, ldx >= K.  XL : [T x G*(N-1)*4] bf16, ldxl >= that.
- * nm_sparse_gemm does this inside its staging; this call exists for tests and
- * for the two-pass (lift, then GEMM on a 2:4 problem of width K') variant.  */
+ * nm_sparse_gemm runs this step itself for 4:6 and 8:10 (into its workspace)
+ * before a 2:4 GEMM of width K'; the standalone call exists for tests and for
+ * callers that keep X' for several layers.                                  */
 nm_status lift_activations(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, int m,
                            uint16_t *XL, int64_t ldxl, void *stream);
 
@@ -201,17 +203,50 @@ nm_status nm_sparse_prepare(const uint16_t *vals, const uint8_t *wmeta, int64_t 
  *          same way;
  *     4:6, 8:10  the lifted activations X' are written to `ws` (T x K') and the
  *          product runs as a 2:4 GEMM over K'.
- *   ws : device scratch of nm_sparse_gemm_workspace_bytes(T, K, m) bytes,
- *        16-byte aligned (may be NULL when that is 0, i.e. for 2:4).       */
+ *   ws : device scratch, 16-byte aligned; nm_sparse_gemm_workspace_bytes(T,
+ *        K, m) bytes give the fastest schedule.  Its first part holds the
+ *        staged activations above (T x K/2 bf16 for 6:8, T x K' for 4:6 and
+ *        8:10, nothing for 2:4; too small -> NM_ERR_WORKSPACE); the rest, at
+ *        the next 256-byte boundary, holds stream-K partial sums (below).  A
+ *        workspace without that part (NULL for 2:4) still works, always with
+ *        whole-tile scheduling.
+ *   Scheduling: a persistent grid of CTA pairs (one per two SMs) walks the
+ *   256 x 256 output tiles.  When the tiles leave part of the last wave idle
+ *   (decode-sized T, few tiles) the K' blocks of all tiles are split evenly
+ *   over the pairs instead (stream-K); the pair that starts a split tile adds
+ *   the fp32 partial sums of the pairs after it in ascending order, so results
+ *   are deterministic for a given device and schedule.  The workspace must
+ *   not be shared by calls that may run at the same time (other streams).
+ *   Waits between pairs are bounded: after one second the call gives up and
+ *   sets NM_ERR_TIMEOUT in the device error word.                          */
 size_t nm_sparse_gemm_workspace_bytes(int64_t T, int64_t K, int m);
 nm_status nm_sparse_gemm(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
                          const void *packed, int64_t R, int m, uint16_t *Y, int64_t ldy,
                          void *ws, size_t ws_bytes, void *stream);
 
 /* a8: dense reference GEMM on the tensor cores, Y = X * W^T (W = mask (.) V
- * densified by the caller), fp32 accumulation, bf16 output.                */
+ * densified by the caller), fp32 accumulation, bf16 output.  Same tiling and
+ * scheduling as nm_sparse_gemm; ws (16-byte aligned, may be NULL: whole-tile
+ * scheduling) of nm_dense_gemm_workspace_bytes(T, K, R) bytes enables
+ * stream-K.                                                                 */
+size_t nm_dense_gemm_workspace_bytes(int64_t T, int64_t K, int64_t R);
 nm_status nm_dense_gemm(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, const uint16_t *W,
-                        int64_t R, int64_t ldw, uint16_t *Y, int64_t ldy, void *stream);
+                        int64_t R, int64_t ldw, uint16_t *Y, int64_t ldy, void *ws,
+                        size_t ws_bytes, void *stream);
+
+/* Upper bound on the CTA pairs a stream-K launch uses (its partial-sum
+ * region is sized for this many: 2*8 slots of 32 x 128 fp32 plus 2*8 64-bit
+ * flags per pair).                                                          */
+#define NM_GEMM_STREAMK_MAX_CLUSTERS 96
+
+/* Process-wide GEMM schedule, for tests and measurements (not thread-safe
+ * against GEMM calls being issued concurrently on other host threads).
+ *   policy   : 0 automatic (default), 1 whole tiles only, 2 stream-K whenever
+ *              the workspace allows it.
+ *   clusters : 0 = as many CTA pairs as fit on the device at once, else at
+ *              most this many.
+ * Returns NM_ERR_SHAPE for a policy outside 0..2 or clusters < 0.          */
+nm_status nm_gemm_set_schedule(int policy, int clusters);
 
 /* Ternary absmean quantisation (Sparse-BitNet sec. 1 item 1), input
  * preparation of the ternary 6:8 layer.

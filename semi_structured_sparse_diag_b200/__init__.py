@@ -21,7 +21,7 @@ from . import build as _build
 __all__ = [
     "NMError", "load", "hessian_diag", "score", "score_from_hessian", "prune_compress",
     "slide_pack", "lift_activations", "sparse_prepare", "sparse_gemm", "dense_gemm",
-    "ternary_quantize", "check_device_error", "EXPORTED",
+    "ternary_quantize", "check_device_error", "set_gemm_schedule", "EXPORTED",
 ]
 
 EXPORTED = (
@@ -30,7 +30,7 @@ EXPORTED = (
     "nm_prune_compress", "slide_pack", "lift_activations", "nm_sparse_prepare_bytes",
     "nm_sparse_prepare", "nm_sparse_gemm", "nm_dense_gemm", "nm_ternary_workspace_bytes",
     "nm_ternary_quantize", "nm_hessian_diag_noalloc", "nm_probe_mma", "nm_probe_copy", "nm_gemm_1cta", "nm_sparse_gemm_workspace_bytes",
-    "nm_sparse_gemm_fused",
+    "nm_sparse_gemm_fused", "nm_dense_gemm_workspace_bytes", "nm_gemm_set_schedule",
 )
 
 _P, _I64, _I, _D, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_size_t
@@ -50,7 +50,9 @@ _SIGS = {
     "nm_sparse_gemm": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I, _P, _I64, _P, _SZ, _P]),
     "nm_sparse_gemm_workspace_bytes": (_SZ, [_I64, _I64, _I]),
     "nm_sparse_gemm_fused": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I, _P, _I64, _P]),
-    "nm_dense_gemm": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _I64, _P]),
+    "nm_dense_gemm": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _I64, _P, _SZ, _P]),
+    "nm_dense_gemm_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
+    "nm_gemm_set_schedule": (_I, [_I, _I]),
     "nm_ternary_workspace_bytes": (_SZ, [_I64]),
     "nm_ternary_quantize": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "nm_hessian_diag_noalloc": (_I, [_P, _I64, _I64, _I64, _P, _P]),
@@ -251,16 +253,25 @@ def sparse_gemm(X, packed, R, m, Y=None, ws=None, stream=None, fused=False):
     return Y
 
 
-def dense_gemm(X, W, Y=None, stream=None):
+def dense_gemm(X, W, Y=None, ws=None, stream=None):
     X = _bf16(X, "X")
     W = _bf16(W, "W")
     T, K = X.shape
     R = W.shape[0]
+    lib = load()
     if Y is None:
         Y = torch.empty((T, (R + 7) // 8 * 8), dtype=torch.bfloat16, device=X.device)[:, :R]
-    _check(load().nm_dense_gemm(_ptr(X), T, K, _ld(X), _ptr(W), R, _ld(W), _ptr(Y), _ld(Y),
-                                _stream(stream)), "nm_dense_gemm")
+    if ws is None:
+        ws = torch.empty(lib.nm_dense_gemm_workspace_bytes(T, K, R), dtype=torch.uint8, device=X.device)
+    _check(lib.nm_dense_gemm(_ptr(X), T, K, _ld(X), _ptr(W), R, _ld(W), _ptr(Y), _ld(Y),
+                             _ptr(ws), ws.numel(), _stream(stream)), "nm_dense_gemm")
     return Y
+
+
+def set_gemm_schedule(policy: int = 0, clusters: int = 0) -> None:
+    """GEMM schedule for this process: policy 0 automatic, 1 whole tiles only,
+    2 stream-K whenever the workspace allows; clusters 0 = all that fit."""
+    _check(load().nm_gemm_set_schedule(policy, clusters), "nm_gemm_set_schedule")
 
 
 def ternary_quantize(W, stream=None):

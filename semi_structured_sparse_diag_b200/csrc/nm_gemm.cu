@@ -16,6 +16,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <chrono>
 #include <mutex>
 
 #include "nm_common.cuh"
@@ -457,14 +459,93 @@ __device__ __forceinline__ bool pair_b_by_tma(int mode, int64_t kb) {
            (mode == PMODE_SP68 && (kb % 3) != 2);
 }
 
+
+// ---------------------------------------------------------------------------
+// Work of one cluster.  Tile mode: whole tiles cluster, cluster + nclusters, ...
+// Stream-K mode: the tiles' K' blocks laid end to end (tile-major) and cut into
+// nclusters equal contiguous ranges; a range may start or end inside a tile.
+// The cluster holding a split tile's first block owns it: it adds the fp32
+// partial sums the later contributors (the next clusters) wrote to their slots,
+// in ascending cluster order, and stores the result.  A contributor's part of a
+// split tile is always the first segment of its range, the owner's part the
+// last, so the owner only waits at the very end of its work.
+// ---------------------------------------------------------------------------
+struct SegIter {
+    bool sk;
+    int64_t nkb, pos, end, step;
+    __device__ SegIter(bool sk_, int64_t cluster, int64_t nclusters, int64_t ntiles, int64_t nkb_)
+        : sk(sk_), nkb(nkb_) {
+        if (sk) {
+            const int64_t total = ntiles * nkb;
+            pos = cluster * total / nclusters;
+            end = (cluster + 1) * total / nclusters;
+            step = 0;
+        } else {
+            pos = cluster;
+            end = ntiles;
+            step = nclusters;
+        }
+    }
+    __device__ bool next(int64_t &tile, int64_t &kb0, int64_t &kb1) {
+        if (pos >= end) return false;
+        if (!sk) {
+            tile = pos;
+            kb0 = 0;
+            kb1 = nkb;
+            pos += step;
+            return true;
+        }
+        tile = pos / nkb;
+        kb0 = pos - tile * nkb;
+        kb1 = kb0 + (end - pos) < nkb ? kb0 + (end - pos) : nkb;
+        pos += kb1 - kb0;
+        return true;
+    }
+};
+
+// stream-K workspace: per (cluster, rank, epilogue warp) a 32 x 128 fp32 slot
+// ([column][row]) and a 64-bit flag that holds the launch's sequence number
+// once the slot is written
+constexpr int SK_SLOT_FLOATS = 32 * 128;
+constexpr int64_t SK_MAX_CLUSTERS = NM_GEMM_STREAMK_MAX_CLUSTERS;
+
+__host__ __device__ inline size_t sk_bytes(int64_t max_clusters) {
+    return static_cast<size_t>(max_clusters) * 2 * 8 * (SK_SLOT_FLOATS * 4 + 8);
+}
+
+__device__ __forceinline__ void st_release_u64(uint64_t *p, uint64_t v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t *p) {
+    uint64_t v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// bounded wait for a stream-K flag (all lanes poll; one second limit)
+__device__ __forceinline__ bool sk_wait_flag(const uint64_t *p, uint64_t seq) {
+    if (ld_acquire_u64(p) == seq) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        __nanosleep(64);
+        if (ld_acquire_u64(p) == seq) return true;
+        if (global_timer_ns() - t0 > WAIT_LIMIT_NS) {
+            raise_error(ERRBIT_TIMEOUT);
+            return false;
+        }
+    }
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmE,
                 const __grid_constant__ CUtensorMap tmY,
                 const uint16_t *__restrict__ X, int64_t T, int64_t K, int64_t ldx, int64_t R,
-                int64_t nkb, int m) {
+                int64_t nkb, int m, uint8_t *__restrict__ sk_ws, uint64_t seq, int stream_k) {
     using C = PairCfg<MODE>;
+    const bool sk = stream_k != 0 && !C::LIFT;
     constexpr int S = C::STAGES;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -519,11 +600,13 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
         if (lane == 0) {
             int64_t it = 0;
             bool ok = true;
-            for (int64_t tile = cluster; tile < ntiles && ok; tile += nclusters) {
+            SegIter seg(sk, cluster, nclusters, ntiles, nkb);
+            int64_t tile, kb0, kb1;
+            while (ok && seg.next(tile, kb0, kb1)) {
                 const int64_t nt = tile % n_t, mt2 = tile / n_t;
                 const int32_t arow = static_cast<int32_t>(mt2 * 256 + rank * 128);
                 const int32_t brow = static_cast<int32_t>(nt * C::BN + rank * C::BH);
-                for (int64_t kb = 0; kb < nkb; ++kb, ++it) {
+                for (int64_t kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = static_cast<int>(it % S);
                     const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
                     if (it >= S && !mbar_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
@@ -565,7 +648,9 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
             int64_t it = 0, ti = 0;
             uint32_t lbits = 0;  // phase of lifted[s] (one phase per lifted use of stage s)
             bool ok = true;
-            for (int64_t tile = cluster; tile < ntiles && ok; tile += nclusters, ++ti) {
+            SegIter seg(sk, cluster, nclusters, ntiles, nkb);
+            int64_t tile, kb0, kb1;
+            for (; ok && seg.next(tile, kb0, kb1); ++ti) {
                 const int buf = static_cast<int>(ti % C::ACC_BUFS);
                 const uint32_t aph = static_cast<uint32_t>((ti / C::ACC_BUFS) & 1);
                 if (ti >= C::ACC_BUFS && !mbar_wait_cluster(&acc_empty[buf], aph ^ 1u)) {
@@ -574,7 +659,7 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
                 }
                 tc_fence_after();
                 const uint32_t dcol = tmem_base + static_cast<uint32_t>(buf * C::BN);
-                for (int64_t kb = 0; kb < nkb; ++kb, ++it) {
+                for (int64_t kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = static_cast<int>(it % S);
                     const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
                     if (!mbar_wait(&full[s], ph)) { ok = false; break; }
@@ -589,7 +674,7 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
                         for (int j = 0; j < 4; ++j)
                             mma_bf16_pair(dcol, make_sdesc(a0 + j * 32, 16, 1024, 2),
                                           make_sdesc(b0 + j * 32, 16, 1024, 2), idesc,
-                                          (kb > 0 || j > 0) ? 1u : 0u);
+                                          (kb > kb0 || j > 0) ? 1u : 0u);
                     } else {
                         const uint32_t te = tmem_base + C::TMEM_E;
                         tmem_cp_128x128b_pair(te, make_sdesc(smem_u32(stE(s)), 2048, 128, 0));
@@ -599,7 +684,7 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
                                 dcol, make_sdesc(a0 + j * 32, 16, 1024, 2),
                                 make_sdesc(b0 + (j >> 1) * (C::BH * 128) + (j & 1) * 64, 16, 1024, 2),
                                 te + (j & ~1), idesc | static_cast<uint32_t>(j & 1),
-                                (kb > 0 || j > 0) ? 1u : 0u);
+                                (kb > kb0 || j > 0) ? 1u : 0u);
                     }
                     mma_commit_pair(&empty[s]);
                 }
@@ -614,23 +699,75 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
         const uint32_t acc_empty_cl0 = mapa_shared(&acc_empty[0], 0);
         const uint32_t acc_empty_cl1 = mapa_shared(&acc_empty[1], 0);
         int64_t ti = 0;
-        for (int64_t tile = cluster; tile < ntiles; tile += nclusters, ++ti) {
+        const int we = warp - 4;  // epilogue warp 0..7
+        float *slots = reinterpret_cast<float *>(sk_ws);
+        uint64_t *flags = reinterpret_cast<uint64_t *>(sk_ws + static_cast<size_t>(nclusters) * 2 * 8 *
+                                                                   SK_SLOT_FLOATS * 4);
+        const int64_t total = ntiles * nkb;
+        SegIter seg(sk, cluster, nclusters, ntiles, nkb);
+        int64_t tile, kb0, kb1;
+        for (; seg.next(tile, kb0, kb1); ++ti) {
             const int64_t nt = tile % n_t, mt2 = tile / n_t;
             const int buf = static_cast<int>(ti % C::ACC_BUFS);
             const uint32_t aph = static_cast<uint32_t>((ti / C::ACC_BUFS) & 1);
             if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], aph))) break;
             tc_fence_after();
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>(buf * C::BN + h * 128);
+            // 32-token chunks of this warp's half that hold real tokens
+            const int64_t tok0 = nt * C::BN + h * 128;
+            const int nvalid = tok0 >= T ? 0 : (T - tok0 >= 128 ? 4 : static_cast<int>((T - tok0 + 31) / 32));
+            if (kb0 > 0) {
+                // later part of a split tile: hand the fp32 partial to the owner
+                // (the stores drain while the next segment's MMAs run)
+                float *slot = slots + static_cast<size_t>((cluster * 2 + rank) * 8 + we) * SK_SLOT_FLOATS;
+#pragma unroll 1
+                for (int c = 0; c < nvalid; ++c) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tbase + c * 32, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) __stcg(slot + (c * 32 + j) * 32 + lane, __uint_as_float(v[j]));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(buf == 0 ? acc_empty_cl0 : acc_empty_cl1);
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release_u64(flags + (cluster * 2 + rank) * 8 + we, seq);
+                continue;
+            }
+            // owner: the clusters after this one that hold the rest of the tile
+            int64_t last_contrib = cluster;
+            if (sk && kb1 < nkb) {
+                while (last_contrib + 1 < nclusters &&
+                       (last_contrib + 1) * total / nclusters < (tile + 1) * nkb)
+                    ++last_contrib;
+                // clusters with an empty range (fewer blocks than clusters) write
+                // nothing; after one wait times out the rest are not waited for
+                bool got = true;
+                for (int64_t cc = cluster + 1; cc <= last_contrib && got; ++cc)
+                    if ((cc + 1) * total / nclusters > cc * total / nclusters)
+                        got = sk_wait_flag(flags + (cc * 2 + rank) * 8 + we, seq);
+            }
             uint32_t packed[64];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                       static_cast<uint32_t>(buf * C::BN + h * 128 + c * 32),
-                                   v);
+                tmem_ld_32x32b_x32(tbase + c * 32, v);
                 tmem_ld_wait();
+                float f[32];
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    packed[c * 16 + i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
+                for (int64_t cc = cluster + 1; cc <= last_contrib && c < nvalid; ++cc) {
+                    if ((cc + 1) * total / nclusters == cc * total / nclusters) continue;
+                    const float *ps = slots + static_cast<size_t>((cc * 2 + rank) * 8 + we) * SK_SLOT_FLOATS +
+                                      c * 32 * 32;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) f[j] += __ldcg(ps + j * 32 + lane);
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) packed[c * 16 + i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
             }
             tc_fence_before();
             __syncwarp();
@@ -955,15 +1092,71 @@ nm_status launch_gemm_1cta(const CUtensorMap &a, const CUtensorMap &b, const CUt
 }
 
 // ---- persistent CTA-pair kernel
+
+// schedule override (0 = automatic, 1 = whole tiles, 2 = stream-K) and
+// cluster count override (0 = as many as fit on the device at once)
+std::atomic<int> g_sched_policy{0};
+std::atomic<int> g_sched_clusters{0};
+
+// launch sequence numbers: unique per launch in this process and, being
+// seeded from the clock, unlikely to equal a stale flag left by another one
+uint64_t next_seq() {
+    static std::atomic<uint64_t> ctr{
+        static_cast<uint64_t>(std::chrono::steady_clock::now().time_since_epoch().count()) | 1u};
+    return ctr.fetch_add(1);
+}
+
+// clusters of two that can be resident at once (per mode and device)
+template <int MODE>
+int64_t resident_clusters() {
+    static int cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return sm_count() / 2;
+    if (cache[dev] == 0) {
+        using Cfg = PairCfg<MODE>;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * static_cast<unsigned>(sm_count() / 2), 1, 1);
+        cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, k_gemm_pair<MODE>, &cfg) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = sm_count() / 2;
+        }
+        cache[dev] = n < sm_count() / 2 ? n : sm_count() / 2;
+    }
+    return cache[dev];
+}
+
 template <int MODE>
 nm_status launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b2,
                       const CUtensorMap &e, const CUtensorMap &y, const uint16_t *X, int64_t T,
-                      int64_t K, int64_t ldx, int64_t R, int64_t nkb, int m, cudaStream_t s) {
+                      int64_t K, int64_t ldx, int64_t R, int64_t nkb, int m, void *sk_ws,
+                      size_t sk_ws_bytes, cudaStream_t s) {
     using Cfg = PairCfg<MODE>;
     if (!set_smem_attr<k_gemm_pair<MODE>>(Cfg::SMEM_BYTES)) return NM_ERR_CUDA;
     const int64_t ntiles = ((T + Cfg::BN - 1) / Cfg::BN) * ((R + 255) / 256);
-    int64_t clusters = sm_count() / 2;
-    if (clusters > ntiles) clusters = ntiles;
+    int64_t res = resident_clusters<MODE>();
+    const int forced = g_sched_clusters.load();
+    if (forced > 0 && forced < res) res = forced;
+    if (res > SK_MAX_CLUSTERS) res = SK_MAX_CLUSTERS;
+    if (res < 1) res = 1;
+    // stream-K when the tiles fill less than half the pairs (decode-sized T):
+    // measured on B200, splitting tiles of a fuller grid (one to two waves)
+    // loses more to the partial-sum traffic and to the clusters working on
+    // unrelated K' blocks at the same time than it gains on the last wave
+    const int policy = g_sched_policy.load();
+    const bool sk_ok = !Cfg::LIFT && sk_ws != nullptr && sk_ws_bytes >= sk_bytes(res) &&
+                       (reinterpret_cast<uintptr_t>(sk_ws) & 15u) == 0;
+    const bool sk = sk_ok && (policy == 2 || (policy == 0 && 2 * ntiles <= res));
+    int64_t clusters = sk ? res : (ntiles < res ? ntiles : res);
     if (clusters < 1) clusters = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
@@ -977,8 +1170,10 @@ nm_status launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensor
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, k_gemm_pair<MODE>, a, b, b2, e, y, X, T, K, ldx, R, nkb, m) !=
-        cudaSuccess)
+    uint8_t *skp = sk ? static_cast<uint8_t *>(sk_ws) : nullptr;
+    const uint64_t seq = sk ? next_seq() : 0;
+    if (cudaLaunchKernelEx(&cfg, k_gemm_pair<MODE>, a, b, b2, e, y, X, T, K, ldx, R, nkb, m, skp, seq,
+                           sk ? 1 : 0) != cudaSuccess)
         return NM_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
 }
@@ -1035,9 +1230,24 @@ static GemmWs gemm_ws(int64_t T, int64_t K, int m) {
     return w;
 }
 
+// the stream-K region follows the staged activations, 256-byte aligned
+static size_t sk_offset(const GemmWs &w) { return (w.bytes + 255) / 256 * 256; }
+
 extern "C" size_t nm_sparse_gemm_workspace_bytes(int64_t T, int64_t K, int m) {
-    if (m != 4 && m != 6 && m != 8 && m != 10) return 0;
-    return gemm_ws(T, K, m).bytes;
+    if (T < 1 || K < 1 || (m != 4 && m != 6 && m != 8 && m != 10)) return 0;
+    return sk_offset(gemm_ws(T, K, m)) + sk_bytes(SK_MAX_CLUSTERS);
+}
+
+extern "C" size_t nm_dense_gemm_workspace_bytes(int64_t T, int64_t K, int64_t R) {
+    if (T < 1 || K < 1 || R < 1) return 0;
+    return sk_bytes(SK_MAX_CLUSTERS);
+}
+
+extern "C" nm_status nm_gemm_set_schedule(int policy, int clusters) {
+    if (policy < 0 || policy > 2 || clusters < 0) return NM_ERR_SHAPE;
+    g_sched_policy.store(policy);
+    g_sched_clusters.store(clusters);
+    return NM_OK;
 }
 
 namespace {
@@ -1079,15 +1289,19 @@ extern "C" nm_status nm_sparse_gemm(const uint16_t *X, int64_t T, int64_t K, int
     if (st != NM_OK) return st;
     const GemmWs w = gemm_ws(T, K, m);
     if (w.bytes > 0 && (!ws || ws_bytes < w.bytes)) return NM_ERR_WORKSPACE;
-    if (w.bytes > 0 && !aligned16(ws)) return NM_ERR_ALIGN;
+    if (ws && !aligned16(ws)) return NM_ERR_ALIGN;
     const PackedGeom p = packed_geom(R, K, m);
     const SparseMaps mp = sparse_maps(packed, p, Y, T, R, ldy);
     if (!mp.ok) return NM_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // stream-K partial sums, when the caller's workspace has room for them
+    const size_t sko = sk_offset(w);
+    void *skw = ws && ws_bytes > sko ? static_cast<uint8_t *>(ws) + sko : nullptr;
+    const size_t skb = skw ? ws_bytes - sko : 0;
     CUtensorMap tb, tb2;
     if (m == 4) {
         if (!make_tmap_bf16(&tb, X, T, K, ldx, 64, 128, true)) return NM_ERR_CUDA;
-        return launch_pair<PMODE_SP24>(mp.a, tb, tb, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, s);
+        return launch_pair<PMODE_SP24>(mp.a, tb, tb, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, skw, skb, s);
     }
     uint16_t *stage = static_cast<uint16_t *>(ws);
     if (m == 8) {
@@ -1100,14 +1314,15 @@ extern "C" nm_status nm_sparse_gemm(const uint16_t *X, int64_t T, int64_t K, int
         if (!make_tmap_bf16(&tb, X, T, K, ldx, 64, 128, true) ||
             !make_tmap_bf16(&tb2, stage, T, w.cols, w.ld, 64, 128, true))
             return NM_ERR_CUDA;
-        return launch_pair<PMODE_SP68T>(mp.a, tb, tb2, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, s);
+        return launch_pair<PMODE_SP68T>(mp.a, tb, tb2, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, skw, skb, s);
     }
     // 4:6, 8:10: the lifted activations X' (natural window order) then a 2:4
     // GEMM over K' -- the packed operand is laid out identically
     st = lift_activations(X, T, K, ldx, m, stage, w.ld, stream);
     if (st != NM_OK) return st;
     if (!make_tmap_bf16(&tb, stage, T, w.cols, w.ld, 64, 128, true)) return NM_ERR_CUDA;
-    return launch_pair<PMODE_SP24>(mp.a, tb, tb, mp.e, mp.y, stage, T, w.cols, w.ld, R, p.nkb, 4, s);
+    return launch_pair<PMODE_SP24>(mp.a, tb, tb, mp.e, mp.y, stage, T, w.cols, w.ld, R, p.nkb, 4, skw,
+                                   skb, s);
 }
 
 extern "C" nm_status nm_sparse_gemm_fused(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
@@ -1120,18 +1335,20 @@ extern "C" nm_status nm_sparse_gemm_fused(const uint16_t *X, int64_t T, int64_t 
     CUtensorMap tb;
     if (!mp.ok || !make_tmap_bf16(&tb, X, T, K, ldx, 64, 128, true)) return NM_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (m == 4) return launch_pair<PMODE_SP24>(mp.a, tb, tb, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, s);
-    if (m == 8) return launch_pair<PMODE_SP68>(mp.a, tb, tb, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, s);
-    return launch_pair<PMODE_SPLIFT>(mp.a, tb, tb, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, s);
+    if (m == 4)
+        return launch_pair<PMODE_SP24>(mp.a, tb, tb, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, nullptr, 0, s);
+    if (m == 8)
+        return launch_pair<PMODE_SP68>(mp.a, tb, tb, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, nullptr, 0, s);
+    return launch_pair<PMODE_SPLIFT>(mp.a, tb, tb, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, nullptr, 0, s);
 }
 
 extern "C" nm_status nm_dense_gemm(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
                                    const uint16_t *W, int64_t R, int64_t ldw, uint16_t *Y,
-                                   int64_t ldy, void *stream) {
+                                   int64_t ldy, void *ws, size_t ws_bytes, void *stream) {
     if (!X || !W || !Y) return NM_ERR_NULL;
     if (T < 1 || K < 1 || R < 1 || ldx < K || ldw < K || ldy < R) return NM_ERR_SHAPE;
     if (!aligned16(X) || !aligned16(W) || !aligned16(Y) || (ldx % 8) != 0 || (ldw % 8) != 0 ||
-        (ldy % 8) != 0)
+        (ldy % 8) != 0 || (ws && !aligned16(ws)))
         return NM_ERR_ALIGN;
     CUtensorMap ta, tb, ty;
     if (!make_tmap_bf16(&ta, W, R, K, ldw, 64, BM, true) ||
@@ -1139,7 +1356,7 @@ extern "C" nm_status nm_dense_gemm(const uint16_t *X, int64_t T, int64_t K, int6
         !make_tmap_bf16(&ty, Y, T, R, ldy, 32, 32, false))
         return NM_ERR_CUDA;
     const int64_t nkb = (K + 63) / 64;
-    return launch_pair<PMODE_DENSE>(ta, tb, tb, ta, ty, X, T, K, ldx, R, nkb, 4,
+    return launch_pair<PMODE_DENSE>(ta, tb, tb, ta, ty, X, T, K, ldx, R, nkb, 4, ws, ws ? ws_bytes : 0,
                                     reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -50,10 +50,18 @@ def test_size_queries():
     assert lib.nm_sparse_prepare_bytes(256, 512, 5) == 0
     assert lib.nm_sparse_prepare_bytes(0, 512, 4) == 0
     assert lib.nm_ternary_workspace_bytes(100) >= 800
-    assert lib.nm_sparse_gemm_workspace_bytes(2048, 4096, 4) == 0
-    assert lib.nm_sparse_gemm_workspace_bytes(2048, 4096, 8) == 2048 * 2048 * 2      # T x K/2
-    assert lib.nm_sparse_gemm_workspace_bytes(7, 1003, 6) == 7 * 1344 * 2           # T x K'
-    assert lib.nm_sparse_gemm_workspace_bytes(16, 8195, 10) == 16 * 13120 * 2
+    # staged activations (rounded up to 256 bytes), then the stream-K region:
+    # per CTA pair 2 x 8 slots of 32 x 128 fp32 and 2 x 8 flags of 8 bytes
+    sk = 96 * 2 * 8 * (32 * 128 * 4 + 8)
+    up = lambda b: (b + 255) // 256 * 256
+    assert lib.nm_sparse_gemm_workspace_bytes(2048, 4096, 4) == sk
+    assert lib.nm_sparse_gemm_workspace_bytes(2048, 4096, 8) == 2048 * 2048 * 2 + sk      # T x K/2
+    assert lib.nm_sparse_gemm_workspace_bytes(7, 1003, 6) == up(7 * 1344 * 2) + sk       # T x K'
+    assert lib.nm_sparse_gemm_workspace_bytes(16, 8195, 10) == up(16 * 13120 * 2) + sk
+    assert lib.nm_sparse_gemm_workspace_bytes(0, 4096, 4) == 0
+    assert lib.nm_sparse_gemm_workspace_bytes(16, 4096, 5) == 0
+    assert lib.nm_dense_gemm_workspace_bytes(16, 4096, 4096) == sk
+    assert lib.nm_dense_gemm_workspace_bytes(16, 0, 4096) == 0
 
 
 # fake but 16-byte aligned device addresses: validation fails before any use
@@ -84,8 +92,14 @@ MIS = 0x10002
     (lambda l: l.nm_sparse_gemm(A, 4, 16, 16, A, 4, 8, A, 8, None, 0, None), 5),
     (lambda l: l.nm_sparse_gemm(A, 4, 16, 16, A, 4, 8, A, 8, MIS, 1 << 20, None), 3),
     (lambda l: l.nm_sparse_gemm_fused(A, 4, 8, 8, A, 4, 9, A, 8, None), 4),
-    (lambda l: l.nm_dense_gemm(A, 4, 8, 8, None, 4, 8, A, 8, None), 1),
-    (lambda l: l.nm_dense_gemm(A, 4, 8, 8, A, 4, 8, MIS, 8, None), 3),
+    (lambda l: l.nm_dense_gemm(A, 4, 8, 8, None, 4, 8, A, 8, None, 0, None), 1),
+    (lambda l: l.nm_dense_gemm(A, 4, 8, 8, A, 4, 8, MIS, 8, None, 0, None), 3),
+    (lambda l: l.nm_dense_gemm(A, 4, 8, 8, A, 4, 8, A, 8, MIS, 1 << 20, None), 3),
+    (lambda l: l.nm_dense_gemm(A, 4, 8, 4, A, 4, 8, A, 8, None, 0, None), 2),
+    (lambda l: l.nm_gemm_set_schedule(3, 0), 2),
+    (lambda l: l.nm_gemm_set_schedule(-1, 0), 2),
+    (lambda l: l.nm_gemm_set_schedule(0, -1), 2),
+    (lambda l: l.nm_gemm_set_schedule(0, 0), 0),
     (lambda l: l.nm_ternary_quantize(A, 4, 8, 8, A, A, A, 1, None), 5),
 ])
 def test_argument_validation(call, expect):

@@ -175,17 +175,23 @@ def test_fused_lift_equals_two_pass(nm, m):
     # 4:6 and 8:10 both use the natural K' order and the same tiles, so the fp32
     # tensor-core sums are identical bits; 6:8 packs K' in another order (raw
     # tiles of X first), so it agrees within rounding.
+    # (whole-tile schedule throughout: the fused kernel has no stream-K form,
+    # and splitting K' would change the fp32 summation order)
     R, K, T = 256, 1030, 130
     X, W, res = _layer(R, K, T, m - 2, m, seed=m)
     wm = res["wmeta"]
     packed = nm.sparse_prepare(to_dev(res["vals"]), torch.from_numpy(wm).cuda(), R, K, m)
-    Yf = bf16_to_f64(to_host_u16(nm.sparse_gemm(to_dev(X, 1032), packed, R, m, fused=True)))
-    Yl = bf16_to_f64(to_host_u16(nm.sparse_gemm(to_dev(X, 1032), packed, R, m)))
-    XL = nm.lift_activations(to_dev(X, 1032), m)
-    KL = XL.shape[1]
-    packed24 = nm.sparse_prepare(to_dev(res["vals"]), torch.from_numpy(res["wmeta"]).cuda(), R, KL, 4)
-    Y2 = bf16_to_f64(to_host_u16(nm.sparse_gemm(XL, packed24, R, 4)))
-    _sync_ok(nm)
+    nm.set_gemm_schedule(1)
+    try:
+        Yf = bf16_to_f64(to_host_u16(nm.sparse_gemm(to_dev(X, 1032), packed, R, m, fused=True)))
+        Yl = bf16_to_f64(to_host_u16(nm.sparse_gemm(to_dev(X, 1032), packed, R, m)))
+        XL = nm.lift_activations(to_dev(X, 1032), m)
+        KL = XL.shape[1]
+        packed24 = nm.sparse_prepare(to_dev(res["vals"]), torch.from_numpy(res["wmeta"]).cuda(), R, KL, 4)
+        Y2 = bf16_to_f64(to_host_u16(nm.sparse_gemm(XL, packed24, R, 4)))
+        _sync_ok(nm)
+    finally:
+        nm.set_gemm_schedule(0)
     Y64 = oracle.gemm_masked(X, res["mask"], W, m)
     assert rel_err(Y2, Y64) <= GEMM_TOL
     assert rel_err(Yl, Y64) <= GEMM_TOL
