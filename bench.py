@@ -351,7 +351,7 @@ def run_ours(args):
         "speedup_bound": round(K / (KL / 2), 4),
         "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": {
-            "kernel": f"k_gemm_pair<{PAIR_MODE[m]}>",
+            "kernel": f"k_gemm_wide<{PAIR_MODE[m]}>",
             "bound": "tensor",
             "achieved": round(achieved, 2),
             "peak": round(sparse_peak, 1),
@@ -575,6 +575,9 @@ def run_ablation(args):
             res[f"own dense GEMM, CTA pair, {nm_pol} forced"] = timed(dense_call)
         finally:
             nm.set_gemm_schedule(0)
+    res["256 x 256 pair tile (nm_sparse_gemm_tile256)"] = timed(
+        lambda: lib.nm_sparse_gemm_tile256(X.data_ptr(), T, K, K, packed.data_ptr(), R, m, Y.data_ptr(),
+                                           ldy, ws.data_ptr(), ws.numel(), s))
     res["in-kernel lift (nm_sparse_gemm_fused)"] = timed(
         lambda: lib.nm_sparse_gemm_fused(X.data_ptr(), T, K, K, packed.data_ptr(), R, m, Y.data_ptr(),
                                          ldy, s))

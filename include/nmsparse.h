@@ -211,7 +211,7 @@ nm_status nm_sparse_prepare(const uint16_t *vals, const uint8_t *wmeta, int64_t 
  *        workspace without that part (NULL for 2:4) still works, always with
  *        whole-tile scheduling.
  *   Scheduling: a persistent grid of CTA pairs (one per two SMs) walks the
- *   256 x 256 output tiles.  When the tiles leave part of the last wave idle
+ *   output tiles of 512 weight rows x up to 240 tokens.  When the tiles leave part of the last wave idle
  *   (decode-sized T, few tiles) the K' blocks of all tiles are split evenly
  *   over the pairs instead (stream-K); the pair that starts a split tile adds
  *   the fp32 partial sums of the pairs after it in ascending order, so results
@@ -235,7 +235,7 @@ nm_status nm_dense_gemm(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, co
                         size_t ws_bytes, void *stream);
 
 /* Upper bound on the CTA pairs a stream-K launch uses (its partial-sum
- * region is sized for this many: 2*8 slots of 32 x 128 fp32 plus 2*8 64-bit
+ * region is sized for this many: 2*8 slots of 32 x 240 fp32 plus 2*8 64-bit
  * flags per pair).                                                          */
 #define NM_GEMM_STREAMK_MAX_CLUSTERS 96
 

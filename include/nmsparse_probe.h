@@ -48,6 +48,14 @@ nm_status nm_sparse_gemm_fused(const uint16_t *X, int64_t T, int64_t K, int64_t 
                                const void *packed, int64_t R, int m, uint16_t *Y, int64_t ldy,
                                void *stream);
 
+/* Ablation: nm_sparse_gemm with the 256-row x 256-token CTA-pair tile (one
+ * M = 256 sparse MMA per step) instead of the library's 512-row x (<= 240)-
+ * token tile (two MMAs per step sharing B).  Same arguments, workspace and
+ * output as nm_sparse_gemm.                                                */
+nm_status nm_sparse_gemm_tile256(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
+                                 const void *packed, int64_t R, int m, uint16_t *Y, int64_t ldy,
+                                 void *ws, size_t ws_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

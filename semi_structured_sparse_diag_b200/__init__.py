@@ -31,6 +31,7 @@ EXPORTED = (
     "nm_sparse_prepare", "nm_sparse_gemm", "nm_dense_gemm", "nm_ternary_workspace_bytes",
     "nm_ternary_quantize", "nm_hessian_diag_noalloc", "nm_probe_mma", "nm_probe_copy", "nm_gemm_1cta", "nm_sparse_gemm_workspace_bytes",
     "nm_sparse_gemm_fused", "nm_dense_gemm_workspace_bytes", "nm_gemm_set_schedule",
+    "nm_sparse_gemm_tile256",
 )
 
 _P, _I64, _I, _D, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_size_t
@@ -50,6 +51,7 @@ _SIGS = {
     "nm_sparse_gemm": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I, _P, _I64, _P, _SZ, _P]),
     "nm_sparse_gemm_workspace_bytes": (_SZ, [_I64, _I64, _I]),
     "nm_sparse_gemm_fused": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I, _P, _I64, _P]),
+    "nm_sparse_gemm_tile256": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I, _P, _I64, _P, _SZ, _P]),
     "nm_dense_gemm": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _I64, _P, _SZ, _P]),
     "nm_dense_gemm_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
     "nm_gemm_set_schedule": (_I, [_I, _I]),
@@ -233,8 +235,9 @@ def sparse_prepare(vals, wmeta, R, K, m, packed=None, stream=None):
     return packed
 
 
-def sparse_gemm(X, packed, R, m, Y=None, ws=None, stream=None, fused=False):
-    """Y = X * W_sparse^T.  fused=True runs the in-kernel-lift variant (ablation)."""
+def sparse_gemm(X, packed, R, m, Y=None, ws=None, stream=None, fused=False, tile256=False):
+    """Y = X * W_sparse^T.  Ablation variants: fused=True lifts inside the GEMM,
+    tile256=True uses the 256 x 256 CTA-pair tile."""
     X = _bf16(X, "X")
     T, K = X.shape
     lib = load()
@@ -247,8 +250,9 @@ def sparse_gemm(X, packed, R, m, Y=None, ws=None, stream=None, fused=False):
     need = lib.nm_sparse_gemm_workspace_bytes(T, K, m)
     if ws is None and need:
         ws = torch.empty(need, dtype=torch.uint8, device=X.device)
-    _check(lib.nm_sparse_gemm(_ptr(X), T, K, _ld(X), _ptr(packed), R, m, _ptr(Y), _ld(Y),
-                              _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)),
+    fn = lib.nm_sparse_gemm_tile256 if tile256 else lib.nm_sparse_gemm
+    _check(fn(_ptr(X), T, K, _ld(X), _ptr(packed), R, m, _ptr(Y), _ld(Y),
+              _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)),
            "nm_sparse_gemm")
     return Y
 

@@ -503,10 +503,11 @@ struct SegIter {
     }
 };
 
-// stream-K workspace: per (cluster, rank, epilogue warp) a 32 x 128 fp32 slot
-// ([column][row]) and a 64-bit flag that holds the launch's sequence number
-// once the slot is written
-constexpr int SK_SLOT_FLOATS = 32 * 128;
+// stream-K workspace: per (cluster, rank, epilogue warp) a slot of up to
+// 32 rows x 240 columns fp32 ([column][row]; the 256-token pair tiles use the
+// first 128 columns of their warp's slot) and a 64-bit flag that holds the
+// launch's sequence number once the slot is written
+constexpr int SK_SLOT_FLOATS = 32 * 240;
 constexpr int64_t SK_MAX_CLUSTERS = NM_GEMM_STREAMK_MAX_CLUSTERS;
 
 __host__ __device__ inline size_t sk_bytes(int64_t max_clusters) {
@@ -958,6 +959,356 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
     }
 }
 
+// ===========================================================================
+// Wide sparse GEMM (library path for every pattern).
+//
+// Shared-memory bandwidth sets the rate of the sparse kernel above: a
+// 2:4-sparse MMA step of the CTA pair (M = 256, N = 256, 32 lifted columns)
+// keeps the tensor core busy for 128 clocks, but each CTA's shared memory must
+// take in and hand out 12 KB of operands for it (4 KB of A, 8 KB of its B
+// half: written by TMA, read by the tensor core), 192 clocks at 128 bytes per
+// clock -- a ceiling of 2/3 of the sparse peak.  Here a pair computes 512
+// weight rows x bn (<= 240) tokens with two MMAs per step that share the B
+// tile: CTA r holds A rows [128r, 128r+128) and [256+128r, 256+128r+128) of
+// the tile, each with its metadata, and bn/2 tokens of B.  Per step and CTA:
+// 8 KB of A and 7.5 KB of B written, 8 KB of A and 2 x 7.5 KB of B read
+// (each MMA reads B once), 308 clocks for 240 clocks of MMA: 78% of peak.
+//
+// Tensor memory (512 columns): accumulator 0 in [0, 240), its metadata at
+// 240, accumulator 1's metadata at 248, accumulator 1 in [256, 496).  One
+// accumulator pair per CTA, so the next tile's MMAs start once the epilogue
+// warps have moved this tile's sums into registers (bf16).
+// Warps: 0 producer, 1 tensor-memory owner and (leader) MMA issuer, 4-11
+// epilogue (lane quarter warp % 4, accumulator (warp - 4) / 4).
+// Tiles where rows 256..511 lie past the padded R (a multiple of 256) skip
+// accumulator 1's loads and MMAs.
+// Schedules as k_gemm_pair: whole tiles, or stream-K (SegIter above).
+// ===========================================================================
+struct WideCfg {
+    static constexpr int BN_MAX = 240;              // tokens per tile (both CTAs)
+    static constexpr int BH_MAX = BN_MAX / 2;       // tokens per CTA
+    static constexpr int A_BYTES = BM * 128;        // 128 rows x 64 values
+    static constexpr int B_ATOM = BH_MAX * 128;     // 64 lifted columns x BH_MAX tokens
+    static constexpr int OFF_A0 = 0, OFF_A1 = A_BYTES, OFF_B = 2 * A_BYTES;
+    static constexpr int OFF_E0 = OFF_B + 2 * B_ATOM, OFF_E1 = OFF_E0 + EBLK_BYTES;
+    static constexpr int STAGE_BYTES = OFF_E1 + EBLK_BYTES;
+    static constexpr int STAGES = 3;
+    static constexpr int EPI_WARPS = 8;
+    static constexpr int EPI_BYTES = EPI_WARPS * 32 * 32 * 2;
+    static constexpr int THREADS = 384;
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int TMEM_D0 = 0, TMEM_E0 = 240, TMEM_E1 = 248, TMEM_D1 = 256;
+    static_assert(STAGE_BYTES % 1024 == 0 && B_ATOM % 1024 == 0, "stage alignment");
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+    static_assert(32 * BN_MAX <= SK_SLOT_FLOATS, "stream-K slot");
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(WideCfg::THREADS, 1)
+    k_gemm_wide(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmE,
+                const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmY16,
+                int64_t T, int64_t R, int64_t nkb, int bn, uint8_t *__restrict__ sk_ws, uint64_t seq,
+                int stream_k) {
+    using C = WideCfg;
+    constexpr int S = C::STAGES;
+    const bool sk = stream_k != 0;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    uint8_t *epi_smem = smem + S * C::STAGE_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(epi_smem + C::EPI_BYTES);
+    uint64_t *full = bars, *empty = bars + S, *acc_full = bars + 2 * S, *acc_empty = bars + 2 * S + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int64_t cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    const int bh = bn >> 1;
+    const int64_t n_t = (T + bn - 1) / bn;
+    const int64_t Rpad = (R + 255) / 256 * 256;
+    const int64_t n_m = (Rpad + 511) / 512;
+    const int64_t ntiles = n_t * n_m;
+    auto stage = [&](int s) { return smem + s * C::STAGE_BYTES; };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 2 * C::EPI_WARPS);
+        fence_barrier_init();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+        prefetch_tmap(&tmE);
+        prefetch_tmap(&tmY);
+        prefetch_tmap(&tmY16);
+        if (MODE == PMODE_SP68T) prefetch_tmap(&tmB2);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            int64_t it = 0;
+            bool ok = true;
+            SegIter seg(sk, cluster, nclusters, ntiles, nkb);
+            int64_t tile, kb0, kb1;
+            const uint32_t b_bytes = static_cast<uint32_t>(bh) * 256u;
+            while (ok && seg.next(tile, kb0, kb1)) {
+                const int64_t nt = tile % n_t, mt = tile / n_t;
+                const bool has1 = mt * 512 + 256 < Rpad;
+                const int32_t arow = static_cast<int32_t>(mt * 512 + rank * 128);
+                const int32_t brow = static_cast<int32_t>(nt * bn + rank * bh);
+                const int64_t e0 = (mt * 4 + rank) * nkb, e1 = (mt * 4 + 2 + rank) * nkb;
+                const uint32_t tx = 2u * ((has1 ? 2u : 1u) * (C::A_BYTES + EBLK_BYTES) + b_bytes);
+                for (int64_t kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int s = static_cast<int>(it % S);
+                    const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
+                    if (it >= S && !mbar_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], tx);
+                    const uint32_t bar = mapa_shared(&full[s], 0);
+                    uint8_t *st = stage(s);
+                    const int32_t ka = static_cast<int32_t>(kb * 64);
+                    tma_load_2d_pair(st + C::OFF_A0, &tmA, bar, ka, arow);
+                    tma_load_2d_pair(st + C::OFF_E0, &tmE, bar, 0, static_cast<int32_t>((e0 + kb) * 8));
+                    if (has1) {
+                        tma_load_2d_pair(st + C::OFF_A1, &tmA, bar, ka, arow + 256);
+                        tma_load_2d_pair(st + C::OFF_E1, &tmE, bar, 0,
+                                         static_cast<int32_t>((e1 + kb) * 8));
+                    }
+                    const bool mid = MODE == PMODE_SP68T && (kb % 3) == 2;
+                    const int64_t x0 = MODE == PMODE_SP24 ? kb * 128
+                                       : (mid ? (kb / 3) * 128 : (kb / 3) * 256 + (kb % 3) * 128);
+                    const CUtensorMap *tb = mid ? &tmB2 : &tmB;
+                    tma_load_2d_pair(st + C::OFF_B, tb, bar, static_cast<int32_t>(x0), brow);
+                    tma_load_2d_pair(st + C::OFF_B + C::B_ATOM, tb, bar, static_cast<int32_t>(x0 + 64),
+                                     brow);
+                }
+            }
+            if (!ok && rank == 0) {  // let copies already issued land before exiting
+                for (int64_t j = (it > S ? it - S : 0); j < it; ++j)
+                    mbar_wait(&full[j % S], static_cast<uint32_t>((j / S) & 1));
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (rank == 0 && lane == 0) {
+            const uint32_t idesc = make_idesc_bf16(256, bn, true, 0);
+            int64_t it = 0, ti = 0;
+            bool ok = true;
+            SegIter seg(sk, cluster, nclusters, ntiles, nkb);
+            int64_t tile, kb0, kb1;
+            for (; ok && seg.next(tile, kb0, kb1); ++ti) {
+                const bool has1 = (tile / n_t) * 512 + 256 < Rpad;
+                if (ti >= 1 && !mbar_wait_cluster(acc_empty, static_cast<uint32_t>((ti - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + C::TMEM_D0, d1 = tmem_base + C::TMEM_D1;
+                const uint32_t te0 = tmem_base + C::TMEM_E0, te1 = tmem_base + C::TMEM_E1;
+                for (int64_t kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int s = static_cast<int>(it % S);
+                    const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
+                    if (!mbar_wait(&full[s], ph)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t st = smem_u32(stage(s));
+                    tmem_cp_128x128b_pair(te0, make_sdesc(st + C::OFF_E0, 2048, 128, 0));
+                    if (has1) tmem_cp_128x128b_pair(te1, make_sdesc(st + C::OFF_E1, 2048, 128, 0));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint64_t bd =
+                            make_sdesc(st + C::OFF_B + (j >> 1) * C::B_ATOM + (j & 1) * 64, 16, 1024, 2);
+                        const uint32_t acc = (kb > kb0 || j > 0) ? 1u : 0u;
+                        const uint32_t id = idesc | static_cast<uint32_t>(j & 1);
+                        mma_sp_bf16_pair(d0, make_sdesc(st + C::OFF_A0 + j * 32, 16, 1024, 2), bd,
+                                         te0 + (j & ~1), id, acc);
+                        if (has1)
+                            mma_sp_bf16_pair(d1, make_sdesc(st + C::OFF_A1 + j * 32, 16, 1024, 2), bd,
+                                             te1 + (j & ~1), id, acc);
+                    }
+                    mma_commit_pair(&empty[s]);
+                }
+                if (ok) mma_commit_pair(acc_full);
+            }
+        }
+    } else if (warp >= 4 && warp < 12) {
+        // ---------------------------------------------------------- epilogue
+        const int q = warp & 3;         // tensor-memory lane quarter
+        const int h = (warp - 4) >> 2;  // accumulator
+        const int we = warp - 4;
+        uint16_t *stage_out = reinterpret_cast<uint16_t *>(epi_smem) + we * 1024;
+        const uint32_t acc_empty_cl = mapa_shared(acc_empty, 0);
+        float *slots = reinterpret_cast<float *>(sk_ws);
+        uint64_t *flags = reinterpret_cast<uint64_t *>(sk_ws + static_cast<size_t>(nclusters) * 2 * 8 *
+                                                                   SK_SLOT_FLOATS * 4);
+        const int64_t total = ntiles * nkb;
+        SegIter seg(sk, cluster, nclusters, ntiles, nkb);
+        int64_t tile, kb0, kb1, ti = 0;
+        for (; seg.next(tile, kb0, kb1); ++ti) {
+            const int64_t nt = tile % n_t, mt = tile / n_t;
+            if (!__all_sync(0xffffffffu, mbar_wait(acc_full, static_cast<uint32_t>(ti & 1)))) break;
+            tc_fence_after();
+            const bool active = h == 0 || mt * 512 + 256 < Rpad;
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>(h ? C::TMEM_D1 : C::TMEM_D0);
+            const int64_t tok0 = nt * bn;
+            const int64_t nv = T - tok0 < bn ? T - tok0 : bn;       // real tokens of the tile
+            const int nch = active ? static_cast<int>((nv + 31) / 32) : 0;
+            if (kb0 > 0) {
+                // later part of a split tile: hand the fp32 partial to the owner
+                float *slot = slots + static_cast<size_t>((cluster * 2 + rank) * 8 + we) * SK_SLOT_FLOATS;
+#pragma unroll 1
+                for (int c = 0; c < nch; ++c) {
+                    if (c < 7) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(tbase + c * 32, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            __stcg(slot + (c * 32 + j) * 32 + lane, __uint_as_float(v[j]));
+                    } else {
+                        uint32_t v[16];
+                        tmem_ld_32x32b_x16(tbase + c * 32, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            __stcg(slot + (c * 32 + j) * 32 + lane, __uint_as_float(v[j]));
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(acc_empty_cl);
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release_u64(flags + (cluster * 2 + rank) * 8 + we, seq);
+                continue;
+            }
+            const int32_t yr = static_cast<int32_t>(mt * 512 + h * 256 + rank * 128 + q * 32);
+            // one bf16 store of chunk c (32 weight rows x 32 tokens, or 16 at
+            // the tile's end) from 16 packed token pairs
+            auto store_chunk = [&](int c, const uint32_t (&w)[16]) {
+                const bool half = c * 32 + 16 >= bn;
+                if (lane == 0) bulk_wait_group_read0();
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    if (half && i >= 8) break;
+                    stage_out[(2 * i) * 32 + lane] = static_cast<uint16_t>(w[i] & 0xFFFFu);
+                    stage_out[(2 * i + 1) * 32 + lane] = static_cast<uint16_t>(w[i] >> 16);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(half ? &tmY16 : &tmY, stage_out, yr, static_cast<int32_t>(tok0 + c * 32));
+                    bulk_commit_group();
+                }
+            };
+            if (sk && kb1 < nkb) {
+                // owner of a split tile (always this cluster's last segment, so
+                // the accumulator may stay busy): wait for the clusters after
+                // this one that hold the rest of the tile, add their partial
+                // sums in ascending order, chunk by chunk
+                int64_t last_contrib = cluster;
+                while (last_contrib + 1 < nclusters &&
+                       (last_contrib + 1) * total / nclusters < (tile + 1) * nkb)
+                    ++last_contrib;
+                bool got = true;
+                for (int64_t cc = cluster + 1; cc <= last_contrib && got; ++cc)
+                    if ((cc + 1) * total / nclusters > cc * total / nclusters)
+                        got = sk_wait_flag(flags + (cc * 2 + rank) * 8 + we, seq);
+#pragma unroll 1
+                for (int c = 0; c < nch; ++c) {
+                    uint32_t v[32];
+                    if (c < 7) {
+                        tmem_ld_32x32b_x32(tbase + c * 32, v);
+                    } else {
+                        uint32_t v16[16];
+                        tmem_ld_32x32b_x16(tbase + c * 32, v16);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) v[j] = v16[j];
+#pragma unroll
+                        for (int j = 16; j < 32; ++j) v[j] = 0;
+                    }
+                    tmem_ld_wait();
+                    const int width = c < 7 ? 32 : 16;
+                    float f[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
+                    for (int64_t cc = cluster + 1; cc <= last_contrib; ++cc) {
+                        if ((cc + 1) * total / nclusters == cc * total / nclusters) continue;
+                        const float *ps = slots + static_cast<size_t>((cc * 2 + rank) * 8 + we) * SK_SLOT_FLOATS +
+                                          c * 32 * 32;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (j < width) f[j] += __ldcg(ps + j * 32 + lane);
+                    }
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
+                    store_chunk(c, w);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(acc_empty_cl);
+                continue;
+            }
+            // whole tile: every chunk into registers (bf16), release the
+            // accumulator, then store
+            uint32_t pk[8][16];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                if (c < nch) {
+                    if (c < 7) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(tbase + c * 32, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            pk[c][i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                    } else {
+                        uint32_t v[16];
+                        tmem_ld_32x32b_x16(tbase + c * 32, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            pk[c][i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+#pragma unroll
+                        for (int i = 8; i < 16; ++i) pk[c][i] = 0;
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty_cl);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                if (c < nch) store_chunk(c, pk[c]);
+        }
+        if (lane == 0) bulk_wait_group0();
+        __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    }
+}
+
 
 // ---------------------------------------------------------------------------
 // 6:8 middle windows: X_mid[t, 4g + i] = X[t, 8g + 2 + i] (i < 4), zero past K.
@@ -1178,6 +1529,75 @@ nm_status launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensor
     return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
 }
 
+// tokens per wide tile: the fewest tiles of at most 240 tokens, as even as
+// multiples of 16 allow
+int64_t wide_bn(int64_t T) {
+    const int64_t nt = (T + WideCfg::BN_MAX - 1) / WideCfg::BN_MAX;
+    const int64_t per = (T + nt - 1) / nt;
+    return (per + 15) / 16 * 16;
+}
+
+template <int MODE>
+nm_status launch_wide(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b2,
+                      const CUtensorMap &e, const CUtensorMap &y, const CUtensorMap &y16, int64_t T,
+                      int64_t R, int64_t nkb, int bn, void *sk_ws, size_t sk_ws_bytes, cudaStream_t s) {
+    using Cfg = WideCfg;
+    if (!set_smem_attr<k_gemm_wide<MODE>>(Cfg::SMEM_BYTES)) return NM_ERR_CUDA;
+    const int64_t Rpad = (R + 255) / 256 * 256;
+    const int64_t ntiles = ((T + bn - 1) / bn) * ((Rpad + 511) / 512);
+    static int cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NM_ERR_CUDA;
+    if (cache[dev] == 0) {
+        cudaLaunchConfig_t q = {};
+        q.gridDim = dim3(2 * static_cast<unsigned>(sm_count() / 2), 1, 1);
+        q.blockDim = dim3(Cfg::THREADS, 1, 1);
+        q.dynamicSmemBytes = Cfg::SMEM_BYTES;
+        cudaLaunchAttribute qa[1];
+        qa[0].id = cudaLaunchAttributeClusterDimension;
+        qa[0].val.clusterDim.x = 2;
+        qa[0].val.clusterDim.y = 1;
+        qa[0].val.clusterDim.z = 1;
+        q.attrs = qa;
+        q.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, k_gemm_wide<MODE>, &q) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = sm_count() / 2;
+        }
+        cache[dev] = n < sm_count() / 2 ? n : sm_count() / 2;
+    }
+    int64_t res = cache[dev];
+    const int forced = g_sched_clusters.load();
+    if (forced > 0 && forced < res) res = forced;
+    if (res > SK_MAX_CLUSTERS) res = SK_MAX_CLUSTERS;
+    if (res < 1) res = 1;
+    const int policy = g_sched_policy.load();
+    const bool sk_ok = sk_ws != nullptr && sk_ws_bytes >= sk_bytes(res) &&
+                       (reinterpret_cast<uintptr_t>(sk_ws) & 15u) == 0;
+    const bool sk = sk_ok && (policy == 2 || (policy == 0 && 2 * ntiles <= res));
+    int64_t clusters = sk ? res : (ntiles < res ? ntiles : res);
+    if (clusters < 1) clusters = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+    cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    uint8_t *skp = sk ? static_cast<uint8_t *>(sk_ws) : nullptr;
+    const uint64_t seq = sk ? next_seq() : 0;
+    if (cudaLaunchKernelEx(&cfg, k_gemm_wide<MODE>, a, b, b2, e, y, y16, T, R, nkb, bn, skp, seq,
+                           sk ? 1 : 0) != cudaSuccess)
+        return NM_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" size_t nm_sparse_prepare_bytes(int64_t R, int64_t K, int m) {
@@ -1282,9 +1702,14 @@ nm_status check_sparse_args(const uint16_t *X, int64_t T, int64_t K, int64_t ldx
 
 }  // namespace
 
-extern "C" nm_status nm_sparse_gemm(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
-                                    const void *packed, int64_t R, int m, uint16_t *Y, int64_t ldy,
-                                    void *ws, size_t ws_bytes, void *stream) {
+namespace {
+
+// the online phase: stage the activations (6:8 middle windows, or the lifted
+// X' for 4:6 and 8:10), then the GEMM with the wide tile (library) or the
+// 256 x 256 pair tile (ablation)
+nm_status sparse_gemm_impl(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, const void *packed,
+                           int64_t R, int m, uint16_t *Y, int64_t ldy, void *ws, size_t ws_bytes,
+                           void *stream, bool wide) {
     nm_status st = check_sparse_args(X, T, K, ldx, packed, R, m, Y, ldy);
     if (st != NM_OK) return st;
     const GemmWs w = gemm_ws(T, K, m);
@@ -1298,31 +1723,54 @@ extern "C" nm_status nm_sparse_gemm(const uint16_t *X, int64_t T, int64_t K, int
     const size_t sko = sk_offset(w);
     void *skw = ws && ws_bytes > sko ? static_cast<uint8_t *>(ws) + sko : nullptr;
     const size_t skb = skw ? ws_bytes - sko : 0;
-    CUtensorMap tb, tb2;
-    if (m == 4) {
-        if (!make_tmap_bf16(&tb, X, T, K, ldx, 64, 128, true)) return NM_ERR_CUDA;
-        return launch_pair<PMODE_SP24>(mp.a, tb, tb, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, skw, skb, s);
-    }
     uint16_t *stage = static_cast<uint16_t *>(ws);
+    // B operand(s): X itself (2:4, and the raw blocks of 6:8), X_mid (6:8), X' (4:6, 8:10)
+    const uint16_t *b_src = X;
+    int64_t b_cols = K, b_ld = ldx;
     if (m == 8) {
-        // raw blocks straight from X, middle windows from the gathered X_mid
         const int64_t pairs = (p.G + 1) / 2;
         dim3 grid(static_cast<unsigned>((pairs + 255) / 256), static_cast<unsigned>(T < 65535 ? T : 65535),
                   static_cast<unsigned>((T + 65534) / 65535));
         k_gather_mid<<<grid, 256, 0, s>>>(X, T, K, ldx, p.G, stage, w.ld);
         if (cudaGetLastError() != cudaSuccess) return NM_ERR_CUDA;
-        if (!make_tmap_bf16(&tb, X, T, K, ldx, 64, 128, true) ||
-            !make_tmap_bf16(&tb2, stage, T, w.cols, w.ld, 64, 128, true))
-            return NM_ERR_CUDA;
-        return launch_pair<PMODE_SP68T>(mp.a, tb, tb2, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, skw, skb, s);
+    } else if (m != 4) {
+        st = lift_activations(X, T, K, ldx, m, stage, w.ld, stream);
+        if (st != NM_OK) return st;
+        b_src = stage;
+        b_cols = w.cols;
+        b_ld = w.ld;
     }
-    // 4:6, 8:10: the lifted activations X' (natural window order) then a 2:4
-    // GEMM over K' -- the packed operand is laid out identically
-    st = lift_activations(X, T, K, ldx, m, stage, w.ld, stream);
-    if (st != NM_OK) return st;
-    if (!make_tmap_bf16(&tb, stage, T, w.cols, w.ld, 64, 128, true)) return NM_ERR_CUDA;
-    return launch_pair<PMODE_SP24>(mp.a, tb, tb, mp.e, mp.y, stage, T, w.cols, w.ld, R, p.nkb, 4, skw,
+    const int bh = wide ? static_cast<int>(wide_bn(T) / 2) : 128;
+    CUtensorMap tb, tb2;
+    if (!make_tmap_bf16(&tb, b_src, T, b_cols, b_ld, 64, static_cast<uint32_t>(bh), true)) return NM_ERR_CUDA;
+    if (m == 8 && !make_tmap_bf16(&tb2, stage, T, w.cols, w.ld, 64, static_cast<uint32_t>(bh), true))
+        return NM_ERR_CUDA;
+    const CUtensorMap &b2 = m == 8 ? tb2 : tb;
+    if (wide) {
+        CUtensorMap y16;
+        if (!make_tmap_bf16(&y16, Y, T, R, ldy, 32, 16, false)) return NM_ERR_CUDA;
+        if (m == 8)
+            return launch_wide<PMODE_SP68T>(mp.a, tb, b2, mp.e, mp.y, y16, T, R, p.nkb, 2 * bh, skw, skb, s);
+        return launch_wide<PMODE_SP24>(mp.a, tb, b2, mp.e, mp.y, y16, T, R, p.nkb, 2 * bh, skw, skb, s);
+    }
+    if (m == 8)
+        return launch_pair<PMODE_SP68T>(mp.a, tb, b2, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, skw, skb, s);
+    return launch_pair<PMODE_SP24>(mp.a, tb, b2, mp.e, mp.y, b_src, T, b_cols, b_ld, R, p.nkb, 4, skw,
                                    skb, s);
+}
+
+}  // namespace
+
+extern "C" nm_status nm_sparse_gemm(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
+                                    const void *packed, int64_t R, int m, uint16_t *Y, int64_t ldy,
+                                    void *ws, size_t ws_bytes, void *stream) {
+    return sparse_gemm_impl(X, T, K, ldx, packed, R, m, Y, ldy, ws, ws_bytes, stream, true);
+}
+
+extern "C" nm_status nm_sparse_gemm_tile256(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
+                                            const void *packed, int64_t R, int m, uint16_t *Y,
+                                            int64_t ldy, void *ws, size_t ws_bytes, void *stream) {
+    return sparse_gemm_impl(X, T, K, ldx, packed, R, m, Y, ldy, ws, ws_bytes, stream, false);
 }
 
 extern "C" nm_status nm_sparse_gemm_fused(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,

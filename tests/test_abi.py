@@ -51,8 +51,8 @@ def test_size_queries():
     assert lib.nm_sparse_prepare_bytes(0, 512, 4) == 0
     assert lib.nm_ternary_workspace_bytes(100) >= 800
     # staged activations (rounded up to 256 bytes), then the stream-K region:
-    # per CTA pair 2 x 8 slots of 32 x 128 fp32 and 2 x 8 flags of 8 bytes
-    sk = 96 * 2 * 8 * (32 * 128 * 4 + 8)
+    # per CTA pair 2 x 8 slots of 32 x 240 fp32 and 2 x 8 flags of 8 bytes
+    sk = 96 * 2 * 8 * (32 * 240 * 4 + 8)
     up = lambda b: (b + 255) // 256 * 256
     assert lib.nm_sparse_gemm_workspace_bytes(2048, 4096, 4) == sk
     assert lib.nm_sparse_gemm_workspace_bytes(2048, 4096, 8) == 2048 * 2048 * 2 + sk      # T x K/2

@@ -155,6 +155,32 @@ def test_sparse_gemm_vs_oracle(nm, m, R, K, T):
     assert rel_err(Y, Y64) <= GEMM_TOL
 
 
+# tokens per wide tile: T <= 240 gives one tile of T rounded up to 16 (the
+# last store of 16 tokens when T % 32 lands in (0, 16]); larger T splits into
+# near-equal tiles of at most 240
+@pytest.mark.parametrize("T", [1, 16, 33, 48, 240, 241, 496, 721])
+@pytest.mark.parametrize("m,R", [(4, 700), (8, 512)])
+def test_sparse_gemm_token_tiling(nm, m, R, T):
+    K = 512
+    X, W, res = _layer(R, K, T, m - 2, m, seed=R + T + m)
+    Y = _gemm_sparse(nm, X, res, R, K, m)
+    Y64 = oracle.gemm_masked(X, res["mask"], W, m)
+    assert rel_err(Y, Y64) <= GEMM_TOL
+
+
+@pytest.mark.parametrize("m,R,K,T", [(4, 256, 512, 128), (4, 1000, 768, 1100), (8, 520, 2056, 700),
+                                     (6, 131, 1003, 77), (10, 260, 2010, 300)])
+def test_tile256_ablation_vs_oracle(nm, m, R, K, T):
+    # the 256 x 256 pair-tile GEMM (ablation entry point) gives the same product
+    X, W, res = _layer(R, K, T, m - 2, m, seed=R + K + T + 2)
+    wm = res["meta24"] if m == 4 else res["wmeta"]
+    packed = nm.sparse_prepare(to_dev(res["vals"]), torch.from_numpy(wm).cuda(), R, K, m)
+    Y = nm.sparse_gemm(to_dev(X, (K + 7) // 8 * 8), packed, R, m, tile256=True)
+    _sync_ok(nm)
+    Y64 = oracle.gemm_masked(X, res["mask"], W, m)
+    assert rel_err(bf16_to_f64(to_host_u16(Y)), Y64) <= GEMM_TOL
+
+
 @pytest.mark.parametrize("m,R,K,T", [(6, 256, 1536, 128), (8, 256, 1024, 128), (10, 256, 1280, 128),
                                      (8, 200, 1030, 257), (6, 131, 1003, 77), (10, 129, 2050, 16),
                                      (4, 130, 1030, 200)])
