@@ -486,6 +486,7 @@ struct SegIter {
             step = nclusters;
         }
     }
+    __device__ bool more() const { return pos < end; }
     __device__ bool next(int64_t &tile, int64_t &kb0, int64_t &kb1) {
         if (pos >= end) return false;
         if (!sk) {
@@ -595,6 +596,9 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
     cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // everything above overlaps the previous kernel's tail (programmatic
+    // dependent launch); global memory is touched only after this
+    grid_dep_wait();
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
@@ -979,7 +983,11 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
 // accumulator pair per CTA, so the next tile's MMAs start once the epilogue
 // warps have moved this tile's sums into registers (bf16).
 // Warps: 0 producer, 1 tensor-memory owner and (leader) MMA issuer, 4-11
-// epilogue (lane quarter warp % 4, accumulator (warp - 4) / 4).
+// epilogue (lane quarter warp % 4, accumulator (warp - 4) / 4): tcgen05.ld of
+// the whole tile into registers as bf16, release of the accumulator, then
+// plain global stores (a warp stores 32 consecutive weight rows of one token,
+// 64 contiguous bytes, per instruction) -- no shared-memory staging, so the
+// stores of one tile overlap the next tile's MMAs without waiting on TMA.
 // Tiles where rows 256..511 lie past the padded R (a multiple of 256) skip
 // accumulator 1's loads and MMAs.
 // Schedules as k_gemm_pair: whole tiles, or stream-K (SegIter above).
@@ -994,10 +1002,9 @@ struct WideCfg {
     static constexpr int STAGE_BYTES = OFF_E1 + EBLK_BYTES;
     static constexpr int STAGES = 3;
     static constexpr int EPI_WARPS = 8;
-    static constexpr int EPI_BYTES = EPI_WARPS * 32 * 32 * 2;
     static constexpr int THREADS = 384;
     static constexpr int BAR_BYTES = 256;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
     static constexpr int TMEM_COLS = 512;
     static constexpr int TMEM_D0 = 0, TMEM_E0 = 240, TMEM_E1 = 248, TMEM_D1 = 256;
     static_assert(STAGE_BYTES % 1024 == 0 && B_ATOM % 1024 == 0, "stage alignment");
@@ -1009,19 +1016,18 @@ template <int MODE>
 __global__ void __launch_bounds__(WideCfg::THREADS, 1)
     k_gemm_wide(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmE,
-                const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmY16,
-                int64_t T, int64_t R, int64_t nkb, int bn, uint8_t *__restrict__ sk_ws, uint64_t seq,
-                int stream_k) {
+                const __grid_constant__ CUtensorMap tmY, uint16_t *__restrict__ Y, int64_t ldy, int64_t T,
+                int64_t R, int64_t nkb, int bn, uint8_t *__restrict__ sk_ws, uint64_t seq, int stream_k) {
     using C = WideCfg;
     constexpr int S = C::STAGES;
     const bool sk = stream_k != 0;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
-    uint8_t *epi_smem = smem + S * C::STAGE_BYTES;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(epi_smem + C::EPI_BYTES);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S * C::STAGE_BYTES);
     uint64_t *full = bars, *empty = bars + S, *acc_full = bars + 2 * S, *acc_empty = bars + 2 * S + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 2);
+    uint64_t *out_ready = bars + 2 * S + 2;  // [2]: an accumulator's output staged (4 warps)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -1040,12 +1046,13 @@ __global__ void __launch_bounds__(WideCfg::THREADS, 1)
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 2 * C::EPI_WARPS);
+        mbar_init(&out_ready[0], 4);
+        mbar_init(&out_ready[1], 4);
         fence_barrier_init();
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
         prefetch_tmap(&tmE);
         prefetch_tmap(&tmY);
-        prefetch_tmap(&tmY16);
         if (MODE == PMODE_SP68T) prefetch_tmap(&tmB2);
     }
     if (warp == 1) {
@@ -1057,6 +1064,9 @@ __global__ void __launch_bounds__(WideCfg::THREADS, 1)
     cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // everything above overlaps the previous kernel's tail (programmatic
+    // dependent launch); global memory is touched only after this
+    grid_dep_wait();
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
@@ -1149,12 +1159,14 @@ __global__ void __launch_bounds__(WideCfg::THREADS, 1)
         const int q = warp & 3;         // tensor-memory lane quarter
         const int h = (warp - 4) >> 2;  // accumulator
         const int we = warp - 4;
-        uint16_t *stage_out = reinterpret_cast<uint16_t *>(epi_smem) + we * 1024;
         const uint32_t acc_empty_cl = mapa_shared(acc_empty, 0);
         float *slots = reinterpret_cast<float *>(sk_ws);
         uint64_t *flags = reinterpret_cast<uint64_t *>(sk_ws + static_cast<size_t>(nclusters) * 2 * 8 *
                                                                    SK_SLOT_FLOATS * 4);
         const int64_t total = ntiles * nkb;
+        // a cluster whose range is empty (fewer K' blocks than clusters) writes nothing
+        auto has_work = [&](int64_t cc) { return (cc + 1) * total / nclusters > cc * total / nclusters; };
+        const bool all_work = total >= nclusters;
         SegIter seg(sk, cluster, nclusters, ntiles, nkb);
         int64_t tile, kb0, kb1, ti = 0;
         for (; seg.next(tile, kb0, kb1); ++ti) {
@@ -1168,25 +1180,26 @@ __global__ void __launch_bounds__(WideCfg::THREADS, 1)
             const int64_t nv = T - tok0 < bn ? T - tok0 : bn;       // real tokens of the tile
             const int nch = active ? static_cast<int>((nv + 31) / 32) : 0;
             if (kb0 > 0) {
-                // later part of a split tile: hand the fp32 partial to the owner
+                // later part of a split tile: hand the fp32 partial (real tokens
+                // only) to the owner; the stores drain while the next segment runs
                 float *slot = slots + static_cast<size_t>((cluster * 2 + rank) * 8 + we) * SK_SLOT_FLOATS;
 #pragma unroll 1
                 for (int c = 0; c < nch; ++c) {
+                    const int64_t wv = nv - c * 32;  // real tokens from this chunk on
+                    uint32_t v[32];
                     if (c < 7) {
-                        uint32_t v[32];
                         tmem_ld_32x32b_x32(tbase + c * 32, v);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            __stcg(slot + (c * 32 + j) * 32 + lane, __uint_as_float(v[j]));
                     } else {
-                        uint32_t v[16];
-                        tmem_ld_32x32b_x16(tbase + c * 32, v);
-                        tmem_ld_wait();
+                        uint32_t v16[16];
+                        tmem_ld_32x32b_x16(tbase + c * 32, v16);
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            __stcg(slot + (c * 32 + j) * 32 + lane, __uint_as_float(v[j]));
+                        for (int j = 0; j < 16; ++j) v[j] = v16[j];
                     }
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (j < wv && (c < 7 || j < 16))
+                            __stcg(slot + (c * 32 + j) * 32 + lane, __uint_as_float(v[j]));
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -1196,39 +1209,72 @@ __global__ void __launch_bounds__(WideCfg::THREADS, 1)
                 if (lane == 0) st_release_u64(flags + (cluster * 2 + rank) * 8 + we, seq);
                 continue;
             }
-            const int32_t yr = static_cast<int32_t>(mt * 512 + h * 256 + rank * 128 + q * 32);
-            // one bf16 store of chunk c (32 weight rows x 32 tokens, or 16 at
-            // the tile's end) from 16 packed token pairs
+            // bf16 out.  The cluster's last segment: every pipeline stage is idle
+            // (its loads landed and its MMAs completed), so the accumulator's
+            // 128 rows x bn tokens are staged there ([token][row]) and leave as
+            // one TMA store of 256-byte rows.  Earlier tiles: straight from
+            // registers, lane = weight row, one store per token (32 consecutive
+            // rows = 64 contiguous bytes), overlapping the next tile's MMAs.
+            const bool last = !seg.more();
+            const int64_t yrow = mt * 512 + h * 256 + rank * 128 + q * 32 + lane;
+            const bool rok = yrow < R;
+            uint16_t *ycol = Y + yrow;
+            uint16_t *stg = reinterpret_cast<uint16_t *>(smem) + h * (128 * C::BN_MAX) + q * 32 + lane;
             auto store_chunk = [&](int c, const uint32_t (&w)[16]) {
-                const bool half = c * 32 + 16 >= bn;
-                if (lane == 0) bulk_wait_group_read0();
-                __syncwarp();
+                if (last) {
+                    uint16_t *sp = stg + c * 32 * 128;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        if (c * 32 + 2 * i >= bn) break;
+                        sp[(2 * i) * 128] = static_cast<uint16_t>(w[i] & 0xFFFFu);
+                        sp[(2 * i + 1) * 128] = static_cast<uint16_t>(w[i] >> 16);
+                    }
+                    return;
+                }
+                const int64_t left = T - (tok0 + c * 32);
+                const int cap = c * 32 + 16 >= bn ? 16 : 32;
+                const int nvt = left < cap ? static_cast<int>(left) : cap;  // tokens to write
+                if (!rok) return;
+                uint16_t *yp = ycol + (tok0 + c * 32) * ldy;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    if (half && i >= 8) break;
-                    stage_out[(2 * i) * 32 + lane] = static_cast<uint16_t>(w[i] & 0xFFFFu);
-                    stage_out[(2 * i + 1) * 32 + lane] = static_cast<uint16_t>(w[i] >> 16);
+                    if (2 * i < nvt) yp[0] = static_cast<uint16_t>(w[i] & 0xFFFFu);
+                    if (2 * i + 1 < nvt) yp[ldy] = static_cast<uint16_t>(w[i] >> 16);
+                    yp += 2 * ldy;
                 }
+            };
+            // after the staged chunks: one TMA store per accumulator, issued by
+            // its lane-quarter-0 warp once the 4 warps have written their rows
+            auto flush_staged = [&]() {
+                if (!last || !active) return;
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(half ? &tmY16 : &tmY, stage_out, yr, static_cast<int32_t>(tok0 + c * 32));
+                if (lane == 0) mbar_arrive(&out_ready[h]);
+                if (q == 0 && lane == 0 && mbar_wait(&out_ready[h], 0)) {
+                    tma_store_2d(&tmY, reinterpret_cast<uint16_t *>(smem) + h * (128 * C::BN_MAX),
+                                 static_cast<int32_t>(mt * 512 + h * 256 + rank * 128),
+                                 static_cast<int32_t>(tok0));
                     bulk_commit_group();
+                    bulk_wait_group0();
                 }
             };
             if (sk && kb1 < nkb) {
                 // owner of a split tile (always this cluster's last segment, so
-                // the accumulator may stay busy): wait for the clusters after
-                // this one that hold the rest of the tile, add their partial
-                // sums in ascending order, chunk by chunk
+                // the accumulator may stay busy): wait for the clusters after this
+                // one that hold the rest of the tile (each lane polls one flag),
+                // then add their partial sums in ascending cluster order
                 int64_t last_contrib = cluster;
                 while (last_contrib + 1 < nclusters &&
                        (last_contrib + 1) * total / nclusters < (tile + 1) * nkb)
                     ++last_contrib;
                 bool got = true;
-                for (int64_t cc = cluster + 1; cc <= last_contrib && got; ++cc)
-                    if ((cc + 1) * total / nclusters > cc * total / nclusters)
-                        got = sk_wait_flag(flags + (cc * 2 + rank) * 8 + we, seq);
+                for (int64_t base = cluster + 1; base <= last_contrib && got; base += 32) {
+                    const int64_t cc = base + lane;
+                    bool mine = true;
+                    if (cc <= last_contrib && (all_work || has_work(cc)))
+                        mine = sk_wait_flag(flags + (cc * 2 + rank) * 8 + we, seq);
+                    got = __all_sync(0xffffffffu, mine);
+                }
 #pragma unroll 1
                 for (int c = 0; c < nch; ++c) {
                     uint32_t v[32];
@@ -1243,62 +1289,105 @@ __global__ void __launch_bounds__(WideCfg::THREADS, 1)
                         for (int j = 16; j < 32; ++j) v[j] = 0;
                     }
                     tmem_ld_wait();
-                    const int width = c < 7 ? 32 : 16;
                     float f[32];
 #pragma unroll
                     for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
-                    for (int64_t cc = cluster + 1; cc <= last_contrib; ++cc) {
-                        if ((cc + 1) * total / nclusters == cc * total / nclusters) continue;
-                        const float *ps = slots + static_cast<size_t>((cc * 2 + rank) * 8 + we) * SK_SLOT_FLOATS +
-                                          c * 32 * 32;
+                    // 16 columns at a time, partials of two clusters in flight
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (j < width) f[j] += __ldcg(ps + j * 32 + lane);
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int64_t wv = nv - c * 32 - hh * 16;  // real tokens from here on
+                        if (wv <= 0 || (c == 7 && hh == 1)) break;
+                        for (int64_t base = cluster + 1; base <= last_contrib; base += 2) {
+                            float pv[2][16];
+                            bool use[2];
+#pragma unroll
+                            for (int k = 0; k < 2; ++k) {
+                                const int64_t cc = base + k;
+                                use[k] = cc <= last_contrib && (all_work || has_work(cc));
+                                const float *ps = slots + (static_cast<size_t>((cc * 2 + rank) * 8 + we) *
+                                                               SK_SLOT_FLOATS +
+                                                           (c * 32 + hh * 16) * 32 + lane);
+#pragma unroll
+                                for (int j = 0; j < 16; ++j)
+                                    pv[k][j] = (use[k] && j < wv) ? __ldcg(ps + j * 32) : 0.0f;
+                            }
+#pragma unroll
+                            for (int k = 0; k < 2; ++k)
+                                if (use[k]) {
+#pragma unroll
+                                    for (int j = 0; j < 16; ++j) f[hh * 16 + j] += pv[k][j];
+                                }
+                        }
                     }
                     uint32_t w[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
                     store_chunk(c, w);
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(acc_empty_cl);
+                flush_staged();  // last segment: the accumulator is not released
                 continue;
             }
-            // whole tile: every chunk into registers (bf16), release the
-            // accumulator, then store
-            uint32_t pk[8][16];
+            if (last) {
+                // last tile: 64 columns per tensor-memory load, straight into
+                // the staging buffer; nothing waits for the accumulator
+#pragma unroll 1
+                for (int c2 = 0; 2 * c2 < nch; ++c2) {
+                    uint32_t v[64];
+                    tmem_ld_32x32b_x64(tbase + c2 * 64, v);
+                    tmem_ld_wait();
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                if (c < nch) {
-                    if (c < 7) {
-                        uint32_t v[32];
-                        tmem_ld_32x32b_x32(tbase + c * 32, v);
-                        tmem_ld_wait();
+                    for (int j = 0; j < 2; ++j) {
+                        if (2 * c2 + j >= nch) break;
+                        uint32_t w[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
-                            pk[c][i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-                    } else {
-                        uint32_t v[16];
-                        tmem_ld_32x32b_x16(tbase + c * 32, v);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            pk[c][i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-#pragma unroll
-                        for (int i = 8; i < 16; ++i) pk[c][i] = 0;
+                            w[i] = pack_bf16x2(__uint_as_float(v[32 * j + 2 * i]),
+                                               __uint_as_float(v[32 * j + 2 * i + 1]));
+                        store_chunk(2 * c2 + j, w);
                     }
                 }
+                flush_staged();
+                continue;
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc_empty_cl);
+            // whole tile, in two halves of four chunks: tensor memory -> bf16
+            // registers -> stores; the accumulator is released once the second
+            // half is in registers, before its stores
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                if (c < nch) store_chunk(c, pk[c]);
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pk[4][16];
+#pragma unroll
+                for (int cc4 = 0; cc4 < 4; ++cc4) {
+                    const int c = half * 4 + cc4;
+                    if (c < nch) {
+                        if (c < 7) {
+                            uint32_t v[32];
+                            tmem_ld_32x32b_x32(tbase + c * 32, v);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                pk[cc4][i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                        } else {
+                            uint32_t v[16];
+                            tmem_ld_32x32b_x16(tbase + c * 32, v);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                pk[cc4][i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+#pragma unroll
+                            for (int i = 8; i < 16; ++i) pk[cc4][i] = 0;
+                        }
+                    }
+                }
+                if (half == 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(acc_empty_cl);
+                }
+#pragma unroll
+                for (int cc4 = 0; cc4 < 4; ++cc4)
+                    if (half * 4 + cc4 < nch) store_chunk(half * 4 + cc4, pk[cc4]);
+            }
         }
-        if (lane == 0) bulk_wait_group0();
-        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
@@ -1318,6 +1407,7 @@ __global__ void __launch_bounds__(WideCfg::THREADS, 1)
 __global__ void __launch_bounds__(256)
     k_gather_mid(const uint16_t *__restrict__ X, int64_t T, int64_t K, int64_t ldx, int64_t G,
                  uint16_t *__restrict__ Xmid, int64_t ldm) {
+    grid_dep_launch();
     const int64_t t = blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535;
     const int64_t h = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // group pair
     if (t >= T || 2 * h >= G) return;
@@ -1514,13 +1604,15 @@ nm_status launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensor
     cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
     cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     uint8_t *skp = sk ? static_cast<uint8_t *>(sk_ws) : nullptr;
     const uint64_t seq = sk ? next_seq() : 0;
     if (cudaLaunchKernelEx(&cfg, k_gemm_pair<MODE>, a, b, b2, e, y, X, T, K, ldx, R, nkb, m, skp, seq,
@@ -1539,7 +1631,7 @@ int64_t wide_bn(int64_t T) {
 
 template <int MODE>
 nm_status launch_wide(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b2,
-                      const CUtensorMap &e, const CUtensorMap &y, const CUtensorMap &y16, int64_t T,
+                      const CUtensorMap &e, const CUtensorMap &y, uint16_t *Y, int64_t ldy, int64_t T,
                       int64_t R, int64_t nkb, int bn, void *sk_ws, size_t sk_ws_bytes, cudaStream_t s) {
     using Cfg = WideCfg;
     if (!set_smem_attr<k_gemm_wide<MODE>>(Cfg::SMEM_BYTES)) return NM_ERR_CUDA;
@@ -1583,16 +1675,18 @@ nm_status launch_wide(const CUtensorMap &a, const CUtensorMap &b, const CUtensor
     cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
     cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     uint8_t *skp = sk ? static_cast<uint8_t *>(sk_ws) : nullptr;
     const uint64_t seq = sk ? next_seq() : 0;
-    if (cudaLaunchKernelEx(&cfg, k_gemm_wide<MODE>, a, b, b2, e, y, y16, T, R, nkb, bn, skp, seq,
+    if (cudaLaunchKernelEx(&cfg, k_gemm_wide<MODE>, a, b, b2, e, y, Y, ldy, T, R, nkb, bn, skp, seq,
                            sk ? 1 : 0) != cudaSuccess)
         return NM_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
@@ -1747,11 +1841,12 @@ nm_status sparse_gemm_impl(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
         return NM_ERR_CUDA;
     const CUtensorMap &b2 = m == 8 ? tb2 : tb;
     if (wide) {
-        CUtensorMap y16;
-        if (!make_tmap_bf16(&y16, Y, T, R, ldy, 32, 16, false)) return NM_ERR_CUDA;
+        // output tile of one accumulator: 128 weight rows x bn tokens
+        CUtensorMap ty;
+        if (!make_tmap_bf16(&ty, Y, T, R, ldy, 128, static_cast<uint32_t>(2 * bh), false)) return NM_ERR_CUDA;
         if (m == 8)
-            return launch_wide<PMODE_SP68T>(mp.a, tb, b2, mp.e, mp.y, y16, T, R, p.nkb, 2 * bh, skw, skb, s);
-        return launch_wide<PMODE_SP24>(mp.a, tb, b2, mp.e, mp.y, y16, T, R, p.nkb, 2 * bh, skw, skb, s);
+            return launch_wide<PMODE_SP68T>(mp.a, tb, b2, mp.e, ty, Y, ldy, T, R, p.nkb, 2 * bh, skw, skb, s);
+        return launch_wide<PMODE_SP24>(mp.a, tb, b2, mp.e, ty, Y, ldy, T, R, p.nkb, 2 * bh, skw, skb, s);
     }
     if (m == 8)
         return launch_pair<PMODE_SP68T>(mp.a, tb, b2, mp.e, mp.y, X, T, K, ldx, R, p.nkb, m, skw, skb, s);

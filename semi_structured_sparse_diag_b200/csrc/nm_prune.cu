@@ -105,52 +105,72 @@ __device__ __forceinline__ float score_one(const double *__restrict__ H, double 
 
 // grid: x = 4096-column slice of a row (256 threads x 2 chunks x 8 elements),
 // y (+65535 z) = row.  Both chunks' loads are issued before any arithmetic.
-__global__ void __launch_bounds__(256) k_score(const double *__restrict__ H, double eps,
+// Each block: SCORE_ROWS rows x 4096 columns; a thread owns two 8-column
+// chunks of each of its rows.  All W loads of a thread are issued before any
+// arithmetic (SCORE_ROWS x 2 x 16 bytes in flight), and H + eps is formed
+// once per column and reused for every row.
+constexpr int SCORE_ROWS = 4;
+
+__global__ void __launch_bounds__(256, 4) k_score(const double *__restrict__ H, double eps,
                                                const uint16_t *__restrict__ W, int64_t R,
                                                int64_t K, int64_t ldw, float *__restrict__ S) {
-    const int64_t i = blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535;
-    if (i >= R) return;
-    const uint16_t *wrow = W + i * ldw;
-    float *srow = S + i * K;
+    const int64_t i0 = (blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535) * SCORE_ROWS;
+    if (i0 >= R) return;
     int64_t j0[2];
     bool full[2];
-    uint4 wv[2];
+    uint4 wv[2][SCORE_ROWS];
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
         j0[c] = (static_cast<int64_t>(blockIdx.x) * 512 + c * 256 + threadIdx.x) * 8;
         full[c] = j0[c] + 8 <= K;
-        if (full[c]) wv[c] = __ldg(reinterpret_cast<const uint4 *>(wrow + j0[c]));
+#pragma unroll
+        for (int r = 0; r < SCORE_ROWS; ++r)
+            if (full[c] && i0 + r < R)
+                wv[c][r] = __ldg(reinterpret_cast<const uint4 *>(W + (i0 + r) * ldw + j0[c]));
     }
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
         if (j0[c] >= K) continue;
         if (!full[c]) {
-            for (int64_t j = j0[c]; j < K; ++j) srow[j] = score_one(H, eps, j, wrow[j]);
+            for (int r = 0; r < SCORE_ROWS && i0 + r < R; ++r)
+                for (int64_t j = j0[c]; j < K; ++j)
+                    S[(i0 + r) * K + j] = score_one(H, eps, j, W[(i0 + r) * ldw + j]);
             continue;
         }
-        const uint32_t wr[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
-        float sv[8];
+        double hp[8];
         if (H != nullptr) {
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const double2 hv = __ldg(reinterpret_cast<const double2 *>(H + j0[c]) + u);
-                const double wa = bf16_to_f64(static_cast<uint16_t>(wr[u] & 0xFFFFu));
-                const double wb = bf16_to_f64(static_cast<uint16_t>(wr[u] >> 16));
-                sv[2 * u] = __double2float_rn(__dmul_rn(__dadd_rn(hv.x, eps), __dmul_rn(wa, wa)));
-                sv[2 * u + 1] = __double2float_rn(__dmul_rn(__dadd_rn(hv.y, eps), __dmul_rn(wb, wb)));
+                hp[2 * u] = __dadd_rn(hv.x, eps);
+                hp[2 * u + 1] = __dadd_rn(hv.y, eps);
             }
-        } else {
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                sv[u] = fabsf(bf16_to_f32(static_cast<uint16_t>(wr[u >> 1] >> (16 * (u & 1)))));
         }
-        if ((K & 3) == 0) {
-            float4 *d = reinterpret_cast<float4 *>(srow + j0[c]);
-            d[0] = make_float4(sv[0], sv[1], sv[2], sv[3]);
-            d[1] = make_float4(sv[4], sv[5], sv[6], sv[7]);
-        } else {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) srow[j0[c] + u] = sv[u];
+        for (int r = 0; r < SCORE_ROWS; ++r) {
+            if (i0 + r >= R) break;
+            const uint32_t wr[4] = {wv[c][r].x, wv[c][r].y, wv[c][r].z, wv[c][r].w};
+            float sv[8];
+            if (H != nullptr) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const double w = bf16_to_f64(static_cast<uint16_t>(wr[u >> 1] >> (16 * (u & 1))));
+                    sv[u] = __double2float_rn(__dmul_rn(hp[u], __dmul_rn(w, w)));
+                }
+            } else {
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    sv[u] = fabsf(bf16_to_f32(static_cast<uint16_t>(wr[u >> 1] >> (16 * (u & 1)))));
+            }
+            float *srow = S + (i0 + r) * K;
+            if ((K & 3) == 0) {
+                float4 *d = reinterpret_cast<float4 *>(srow + j0[c]);
+                d[0] = make_float4(sv[0], sv[1], sv[2], sv[3]);
+                d[1] = make_float4(sv[4], sv[5], sv[6], sv[7]);
+            } else {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) srow[j0[c] + u] = sv[u];
+            }
         }
     }
 }
@@ -216,137 +236,292 @@ __device__ __forceinline__ void load_group(const float *__restrict__ srow,
     }
 }
 
+// one group: keep bits, the 2:4 index pair (i0 | i1 << 2; m == 4), and the
+// compressed values written to dst
+template <int M>
+__device__ __forceinline__ void select_group(const float (&s)[M > 0 ? M : 16],
+                                             const uint16_t (&v)[M > 0 ? M : 16], int n, int m,
+                                             uint16_t *__restrict__ dst, uint32_t &keepbits,
+                                             uint32_t &nib) {
+    constexpr int MM = M > 0 ? M : 16;  // static trip count (runtime m <= MM)
+    int i0 = 0, i1 = 0;
+    if (M > 0 && n == m - 2) {
+        // (m-2):m keeps all but the two lowest positions of the order (score
+        // descending, index ascending): find them with two linear scans.  A
+        // later position with an equal score ranks below an earlier one, so
+        // "<=" picks the highest index among equal minima.
+        int d0 = 0;
+        float s0 = s[0];
+#pragma unroll
+        for (int q = 1; q < MM; ++q)
+            if (s[q] <= s0) { s0 = s[q]; d0 = q; }
+        int d1 = -1;
+        float s1 = 0.0f;
+#pragma unroll
+        for (int q = 0; q < MM; ++q)
+            if (q != d0 && (d1 < 0 || s[q] <= s1)) { s1 = s[q]; d1 = q; }
+        const int dlo = d0 < d1 ? d0 : d1, dhi = d0 < d1 ? d1 : d0;
+        keepbits = ((1u << MM) - 1u) & ~(1u << d0) & ~(1u << d1);
+        // output k = v[k], v[k+1] or v[k+2] depending on the dropped positions;
+        // pairs of outputs are packed and stored right here (n = MM - 2 is even)
+#pragma unroll
+        for (int k2 = 0; k2 < (MM - 2) / 2; ++k2) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int k = 2 * k2 + h;
+                const int q = k + (k >= dlo ? 1 : 0) + (k + 1 >= dhi ? 1 : 0);
+                const uint32_t val =
+                    q == k ? v[k] : (q == k + 1 ? v[k + 1] : v[(k + 2 < MM) ? k + 2 : k]);
+                word |= val << (16 * h);
+            }
+            reinterpret_cast<uint32_t *>(dst)[k2] = word;
+        }
+        i0 = (dlo == 0) ? (dhi == 1 ? 2 : 1) : 0;  // first kept position (m == 4 metadata)
+        i1 = 0;
+#pragma unroll
+        for (int q = MM - 1; q >= 0; --q)
+            if (q != dlo && q != dhi && q != i0) i1 = (i1 == 0 || q < i1) ? q : i1;
+    } else {
+        // general n:m: keep position q iff fewer than n positions beat it
+        uint32_t outw[(MM + 1) / 2];
+#pragma unroll
+        for (int k = 0; k < (MM + 1) / 2; ++k) outw[k] = 0u;
+#pragma unroll
+        for (int q = 0; q < MM; ++q) {
+            int rank = 0;
+#pragma unroll
+            for (int p = 0; p < MM; ++p)
+                rank += (p < m && (s[p] > s[q] || (s[p] == s[q] && p < q))) ? 1 : 0;
+            if (q < m && rank < n) keepbits |= 1u << q;
+        }
+        // compress: output k takes the k-th kept position (ascending); values
+        // are selected with static indices so everything stays in registers
+        uint32_t rem = keepbits;
+#pragma unroll
+        for (int k = 0; k < MM - 1; ++k) {
+            if (k < n) {
+                const int q = __ffs(rem) - 1;
+                rem &= rem - 1u;
+                if (k == 0) i0 = q;
+                if (k == 1) i1 = q;
+                uint32_t val = 0;
+#pragma unroll
+                for (int i = 0; i < MM; ++i) val = (i == q) ? static_cast<uint32_t>(v[i]) : val;
+                outw[k >> 1] |= val << (16 * (k & 1));
+            }
+        }
+                if (n % 8 == 0) {
+#pragma unroll
+            for (int k = 0; k < (MM - 1) / 8; ++k)
+                if (8 * k < n)
+                    *reinterpret_cast<uint4 *>(dst + 8 * k) =
+                        make_uint4(outw[4 * k], outw[4 * k + 1], outw[4 * k + 2], outw[4 * k + 3]);
+        } else if (n % 4 == 0) {
+#pragma unroll
+            for (int k = 0; k < (MM - 1) / 4; ++k)
+                if (4 * k < n)
+                    *reinterpret_cast<uint2 *>(dst + 4 * k) = make_uint2(outw[2 * k], outw[2 * k + 1]);
+        } else if (n % 2 == 0) {
+#pragma unroll
+            for (int k = 0; k < (MM - 1) / 2; ++k)
+                if (2 * k < n) *reinterpret_cast<uint32_t *>(dst + 2 * k) = outw[k];
+        } else {
+#pragma unroll
+            for (int k = 0; k < MM - 1; ++k)
+                if (k < n) dst[k] = static_cast<uint16_t>(outw[k >> 1] >> (16 * (k & 1)));
+        }
+    }
+    nib = static_cast<uint32_t>(i0 | (i1 << 2));
+}
+
+// groups per thread (all loads issued before any selection).  Measured on
+// B200: four groups help 2:4, whose single group is only 24 bytes of loads;
+// for m >= 6 one group per thread is faster (higher occupancy).
+template <int M>
+struct PruneGPT {
+    static constexpr int value = M == 4 ? 4 : 1;
+};
+
+// grid: x over slices of PRUNE_THREADS * GPT groups of a row, y (+65535 z) =
+// row.  Warp w of block b owns groups [32 GPT (8b + w), + 32 GPT); in step i
+// lane l takes group 32 i + l of that range, so every load instruction of a
+// warp reads 32 consecutive groups and every step yields m whole mask words.
 template <int M>
 __global__ void __launch_bounds__(PRUNE_THREADS)
     k_prune(const float *__restrict__ S, int64_t lds, const uint16_t *__restrict__ V, int64_t ldv,
             int64_t K, int64_t G, int n, int m_rt, uint32_t *__restrict__ mask,
             uint16_t *__restrict__ vals, uint8_t *__restrict__ meta24) {
-    constexpr int MM = M > 0 ? M : 16;  // static trip count (runtime m <= MM)
+    constexpr int MM = M > 0 ? M : 16;
+    constexpr int GPT = PruneGPT<M>::value;
     const int m = M > 0 ? M : m_rt;
     __shared__ uint32_t words[PRUNE_THREADS / 32][16];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t row = blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535;
-    const int64_t g = static_cast<int64_t>(blockIdx.x) * PRUNE_THREADS + threadIdx.x;
-    const bool valid = g < G;
+    const int64_t wg0 = (static_cast<int64_t>(blockIdx.x) * (PRUNE_THREADS / 32) + warp) * 32 * GPT;
+    if (wg0 >= G) return;  // warp-uniform
     const int64_t mwords = (G * m + 31) / 32;
+    const float *srow = S + row * lds;
+    const uint16_t *vrow = V + row * ldv;
+    uint16_t *vout = vals + row * (G * n);
 
-    if (lane < 16) words[warp][lane] = 0u;
-    __syncwarp();
-
-    uint32_t keepbits = 0;
-    uint32_t nib = 0;
-    if (valid) {
-        float s[MM];
-        uint16_t v[MM];
-        load_group<M>(S + row * lds, V + row * ldv, g * m, K, m, s, v);
-        int i0 = 0, i1 = 0;
-        if (M > 0 && n == m - 2) {
-            // (m-2):m keeps all but the two lowest positions of the order (score
-            // descending, index ascending): find them with two linear scans.  A
-            // later position with an equal score ranks below an earlier one, so
-            // "<=" picks the highest index among equal minima.
-            int d0 = 0;
-            float s0 = s[0];
+    float s[GPT][MM];
+    uint16_t v[GPT][MM];
 #pragma unroll
-            for (int q = 1; q < MM; ++q)
-                if (s[q] <= s0) { s0 = s[q]; d0 = q; }
-            int d1 = -1;
-            float s1 = 0.0f;
-#pragma unroll
-            for (int q = 0; q < MM; ++q)
-                if (q != d0 && (d1 < 0 || s[q] <= s1)) { s1 = s[q]; d1 = q; }
-            const int dlo = d0 < d1 ? d0 : d1, dhi = d0 < d1 ? d1 : d0;
-            keepbits = ((1u << MM) - 1u) & ~(1u << d0) & ~(1u << d1);
-            // output k = v[k], v[k+1] or v[k+2] depending on the dropped positions;
-            // pairs of outputs are packed and stored right here (n = MM - 2 is even)
-            uint16_t *dst = vals + row * (G * n) + g * n;
-#pragma unroll
-            for (int k2 = 0; k2 < (MM - 2) / 2; ++k2) {
-                uint32_t word = 0;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int k = 2 * k2 + h;
-                    const int q = k + (k >= dlo ? 1 : 0) + (k + 1 >= dhi ? 1 : 0);
-                    const uint32_t val =
-                        q == k ? v[k] : (q == k + 1 ? v[k + 1] : v[(k + 2 < MM) ? k + 2 : k]);
-                    word |= val << (16 * h);
-                }
-                reinterpret_cast<uint32_t *>(dst)[k2] = word;
-            }
-            i0 = (dlo == 0) ? (dhi == 1 ? 2 : 1) : 0;  // first kept position (m == 4 metadata)
-            i1 = 0;
-#pragma unroll
-            for (int q = MM - 1; q >= 0; --q)
-                if (q != dlo && q != dhi && q != i0) i1 = (i1 == 0 || q < i1) ? q : i1;
-        } else {
-            // general n:m: keep position q iff fewer than n positions beat it
-            uint32_t outw[(MM + 1) / 2];
-#pragma unroll
-            for (int k = 0; k < (MM + 1) / 2; ++k) outw[k] = 0u;
-#pragma unroll
-            for (int q = 0; q < MM; ++q) {
-                int rank = 0;
-#pragma unroll
-                for (int p = 0; p < MM; ++p)
-                    rank += (p < m && (s[p] > s[q] || (s[p] == s[q] && p < q))) ? 1 : 0;
-                if (q < m && rank < n) keepbits |= 1u << q;
-            }
-            // compress: output k takes the k-th kept position (ascending); values
-            // are selected with static indices so everything stays in registers
-            uint32_t rem = keepbits;
-#pragma unroll
-            for (int k = 0; k < MM - 1; ++k) {
-                if (k < n) {
-                    const int q = __ffs(rem) - 1;
-                    rem &= rem - 1u;
-                    if (k == 0) i0 = q;
-                    if (k == 1) i1 = q;
-                    uint32_t val = 0;
-#pragma unroll
-                    for (int i = 0; i < MM; ++i) val = (i == q) ? static_cast<uint32_t>(v[i]) : val;
-                    outw[k >> 1] |= val << (16 * (k & 1));
-                }
-            }
-            uint16_t *dst = vals + row * (G * n) + g * n;
-            if (n % 8 == 0) {
-#pragma unroll
-                for (int k = 0; k < (MM - 1) / 8; ++k)
-                    if (8 * k < n)
-                        *reinterpret_cast<uint4 *>(dst + 8 * k) =
-                            make_uint4(outw[4 * k], outw[4 * k + 1], outw[4 * k + 2], outw[4 * k + 3]);
-            } else if (n % 4 == 0) {
-#pragma unroll
-                for (int k = 0; k < (MM - 1) / 4; ++k)
-                    if (4 * k < n)
-                        *reinterpret_cast<uint2 *>(dst + 4 * k) = make_uint2(outw[2 * k], outw[2 * k + 1]);
-            } else if (n % 2 == 0) {
-#pragma unroll
-                for (int k = 0; k < (MM - 1) / 2; ++k)
-                    if (2 * k < n) *reinterpret_cast<uint32_t *>(dst + 2 * k) = outw[k];
-            } else {
-#pragma unroll
-                for (int k = 0; k < MM - 1; ++k)
-                    if (k < n) dst[k] = static_cast<uint16_t>(outw[k >> 1] >> (16 * (k & 1)));
-            }
-        }
-        nib = static_cast<uint32_t>(i0 | (i1 << 2));
-        // mask bits: this group's m bits at offset (g % 32) * m in the warp's words
-        const uint32_t off = static_cast<uint32_t>(lane) * m;
-        atomicOr(&words[warp][off >> 5], keepbits << (off & 31));
-        if ((off & 31) + m > 32) atomicOr(&words[warp][(off >> 5) + 1], keepbits >> (32 - (off & 31)));
+    for (int i = 0; i < GPT; ++i) {
+        const int64_t g = wg0 + i * 32 + lane;
+        if (g < G) load_group<M>(srow, vrow, g * m, K, m, s[i], v[i]);
     }
-    __syncwarp();
-    const int64_t g_warp0 = g - lane;
-    const int64_t w0 = g_warp0 * m / 32;
-    if (lane < m && g_warp0 < G && w0 + lane < mwords) mask[row * mwords + w0 + lane] = words[warp][lane];
-
-    if (M == 4 && meta24 != nullptr && n == 2) {
-        const uint32_t other = __shfl_down_sync(0xffffffffu, nib, 1);
-        const int64_t mbytes = (G + 1) / 2;
-        if ((lane & 1) == 0 && valid) {
-            const uint32_t hi = (g + 1 < G) ? other : 0u;
-            meta24[row * mbytes + g / 2] = static_cast<uint8_t>(nib | (hi << 4));
+#pragma unroll
+    for (int i = 0; i < GPT; ++i) {
+        const int64_t gw = wg0 + i * 32;  // first group of this step
+        if (gw >= G) break;                // warp-uniform
+        const int64_t g = gw + lane;
+        const bool valid = g < G;
+        uint32_t keepbits = 0, nib = 0;
+        if (valid) select_group<M>(s[i], v[i], n, m, vout + g * n, keepbits, nib);
+        const int64_t w0 = gw * m / 32;  // first mask word of this step
+        if constexpr (M == 4 || M == 8) {
+            // 32 / M groups per mask word: OR the lanes' bits together with
+            // shuffles; the first lane of each word stores it
+            constexpr int GPW = 32 / (M > 0 ? M : 32);
+            uint32_t wbits = keepbits << (M * (lane % GPW));
+#pragma unroll
+            for (int o = 1; o < GPW; o <<= 1) wbits |= __shfl_xor_sync(0xffffffffu, wbits, o);
+            const int64_t wi = w0 + lane / GPW;
+            if ((lane % GPW) == 0 && wi < mwords) mask[row * mwords + wi] = wbits;
+        } else {
+            // groups straddle words: assemble the step's m words in shared memory
+            if (lane < 16) words[warp][lane] = 0u;
+            __syncwarp();
+            if (valid) {
+                const uint32_t off = static_cast<uint32_t>(lane) * m;
+                atomicOr(&words[warp][off >> 5], keepbits << (off & 31));
+                if ((off & 31) + m > 32) atomicOr(&words[warp][(off >> 5) + 1], keepbits >> (32 - (off & 31)));
+            }
+            __syncwarp();
+            if (lane < m && w0 + lane < mwords) mask[row * mwords + w0 + lane] = words[warp][lane];
+            __syncwarp();
         }
+        if (M == 4 && meta24 != nullptr && n == 2) {
+            // 8 nibbles (groups gw + 8j .. gw + 8j + 7) per 32-bit word
+            uint32_t mb = nib << (4 * (lane & 7));
+            mb |= __shfl_xor_sync(0xffffffffu, mb, 1);
+            mb |= __shfl_xor_sync(0xffffffffu, mb, 2);
+            mb |= __shfl_xor_sync(0xffffffffu, mb, 4);
+            const int64_t mbytes = (G + 1) / 2;
+            if ((lane & 7) == 0 && valid) {
+                const int64_t b0 = g / 2;  // first byte of this word
+                uint8_t *dst = meta24 + row * mbytes + b0;
+                if (b0 + 4 <= mbytes && (reinterpret_cast<uintptr_t>(dst) & 3u) == 0) {
+                    *reinterpret_cast<uint32_t *>(dst) = mb;
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if (b0 + j < mbytes) dst[j] = static_cast<uint8_t>(mb >> (8 * j));
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a3 for 2:4: one thread per run of 8 groups = 32 columns = one mask word.
+// Loads 128 bytes of S and 64 bytes of V, keeps everything in registers, and
+// writes 32 bytes of values, one mask word and one 32-bit word of metadata (8
+// nibbles) -- no shuffles, no shared memory, four stores per 32 columns.
+// grid: x over runs of a row (128 threads per block), y (+65535 z) = row.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void drop_two_of_4(const float (&s)[4], int &dlo, int &dhi) {
+    // the two positions ranked last (score descending, index ascending):
+    // "<=" picks the highest index among equal minima
+    int d0 = 0;
+    float s0 = s[0];
+#pragma unroll
+    for (int q = 1; q < 4; ++q)
+        if (s[q] <= s0) { s0 = s[q]; d0 = q; }
+    int d1 = -1;
+    float s1 = 0.0f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        if (q != d0 && (d1 < 0 || s[q] <= s1)) { s1 = s[q]; d1 = q; }
+    dlo = d0 < d1 ? d0 : d1;
+    dhi = d0 < d1 ? d1 : d0;
+}
+
+__global__ void __launch_bounds__(128)
+    k_prune24(const float *__restrict__ S, int64_t lds, const uint16_t *__restrict__ V, int64_t ldv,
+              int64_t K, int64_t G, uint32_t *__restrict__ mask, uint16_t *__restrict__ vals,
+              uint8_t *__restrict__ meta24) {
+    const int64_t row = blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535;
+    const int64_t run = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t c0 = run * 32;
+    if (c0 >= K) return;
+    const int64_t mwords = (G * 4 + 31) / 32, mbytes = (G + 1) / 2;
+    const float *srow = S + row * lds + c0;
+    const uint16_t *vrow = V + row * ldv + c0;
+    float sc[32];
+    uint32_t vw[16];
+    if (c0 + 32 <= K) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 f = __ldg(reinterpret_cast<const float4 *>(srow) + j);
+            sc[4 * j] = f.x; sc[4 * j + 1] = f.y; sc[4 * j + 2] = f.z; sc[4 * j + 3] = f.w;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(vrow) + j);
+            vw[4 * j] = u.x; vw[4 * j + 1] = u.y; vw[4 * j + 2] = u.z; vw[4 * j + 3] = u.w;
+        }
+    } else {
+        // ragged end of the row: zero padding (score 0, value 0)
+#pragma unroll
+        for (int j = 0; j < 32; ++j) sc[j] = c0 + j < K ? __ldg(srow + j) : 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const uint32_t lo = c0 + 2 * j < K ? __ldg(vrow + 2 * j) : 0u;
+            const uint32_t hi = c0 + 2 * j + 1 < K ? __ldg(vrow + 2 * j + 1) : 0u;
+            vw[j] = lo | (hi << 16);
+        }
+    }
+    uint32_t mword = 0, nibs = 0, out[8];
+#pragma unroll
+    for (int gi = 0; gi < 8; ++gi) {
+        const float s4[4] = {sc[4 * gi], sc[4 * gi + 1], sc[4 * gi + 2], sc[4 * gi + 3]};
+        int dlo, dhi;
+        drop_two_of_4(s4, dlo, dhi);
+        // kept positions i0 < i1 = the two of {0,1,2,3} other than dlo, dhi
+        const int i0 = dlo == 0 ? (dhi == 1 ? 2 : 1) : 0;
+        const int i1 = dhi == 3 ? (dlo == 2 ? 1 : 2) : 3;
+        const uint32_t v4[4] = {vw[2 * gi] & 0xFFFFu, vw[2 * gi] >> 16, vw[2 * gi + 1] & 0xFFFFu,
+                                vw[2 * gi + 1] >> 16};
+        const uint32_t a = i0 == 0 ? v4[0] : (i0 == 1 ? v4[1] : v4[2]);
+        const uint32_t b = i1 == 3 ? v4[3] : (i1 == 2 ? v4[2] : v4[1]);
+        out[gi] = a | (b << 16);
+        mword |= ((1u << i0) | (1u << i1)) << (4 * gi);
+        nibs |= static_cast<uint32_t>(i0 | (i1 << 2)) << (4 * gi);
+    }
+    const int64_t g0 = c0 / 4;          // first group of the run
+    const int ng = G - g0 < 8 ? static_cast<int>(G - g0) : 8;
+    uint16_t *vdst = vals + row * (G * 2) + g0 * 2;
+    if (ng == 8 && ((reinterpret_cast<uintptr_t>(vdst) & 15u) == 0)) {
+        reinterpret_cast<uint4 *>(vdst)[0] = make_uint4(out[0], out[1], out[2], out[3]);
+        reinterpret_cast<uint4 *>(vdst)[1] = make_uint4(out[4], out[5], out[6], out[7]);
+    } else {
+#pragma unroll
+        for (int gi = 0; gi < 8; ++gi)
+            if (gi < ng) reinterpret_cast<uint32_t *>(vdst)[gi] = out[gi];
+    }
+    if (run < mwords) mask[row * mwords + run] = mword & (ng == 8 ? 0xFFFFFFFFu : ((1u << (4 * ng)) - 1u));
+    uint8_t *mdst = meta24 + row * mbytes + g0 / 2;
+    const int nb = (ng + 1) / 2;
+    if (nb == 4 && ((reinterpret_cast<uintptr_t>(mdst) & 3u) == 0)) {
+        *reinterpret_cast<uint32_t *>(mdst) = nibs;
+    } else {
+        nibs &= ng == 8 ? 0xFFFFFFFFu : ((1u << (4 * ng)) - 1u);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (j < nb) mdst[j] = static_cast<uint8_t>(nibs >> (8 * j));
     }
 }
 
@@ -595,8 +770,9 @@ extern "C" nm_status nm_score_from_hessian(const double *H, double eps, const ui
     if (!W || !S) return NM_ERR_NULL;
     if (R < 1 || K < 1 || ldw < K) return NM_ERR_SHAPE;
     if (!aligned16(W) || !aligned16(S) || (ldw % 8) != 0) return NM_ERR_ALIGN;
-    dim3 grid(static_cast<unsigned>((K + 4095) / 4096), static_cast<unsigned>(R < 65535 ? R : 65535),
-              static_cast<unsigned>((R + 65534) / 65535));
+    const int64_t rb = (R + SCORE_ROWS - 1) / SCORE_ROWS;  // row blocks
+    dim3 grid(static_cast<unsigned>((K + 4095) / 4096), static_cast<unsigned>(rb < 65535 ? rb : 65535),
+              static_cast<unsigned>((rb + 65534) / 65535));
     k_score<<<grid, 256, 0, as_stream(stream)>>>(H, eps, W, R, K, ldw, S);
     return launch_status();
 }
@@ -626,16 +802,28 @@ extern "C" nm_status nm_prune_compress(const float *S, int64_t lds, const uint16
         return NM_ERR_ALIGN;
     if (R > 65535LL * 65535LL) return NM_ERR_SHAPE;
     const int64_t G = (K + m - 1) / m;
-    dim3 grid(static_cast<unsigned>((G + PRUNE_THREADS - 1) / PRUNE_THREADS),
-              static_cast<unsigned>(R < 65535 ? R : 65535), static_cast<unsigned>((R + 65534) / 65535));
     cudaStream_t s = as_stream(stream);
     uint8_t *meta = (m == 4 && n == 2) ? meta24 : nullptr;
+    auto grid_for = [&](int gpt) {
+        const int64_t per = static_cast<int64_t>(PRUNE_THREADS) * gpt;
+        return dim3(static_cast<unsigned>((G + per - 1) / per), static_cast<unsigned>(R < 65535 ? R : 65535),
+                    static_cast<unsigned>((R + 65534) / 65535));
+    };
     switch (m) {
-        case 4: k_prune<4><<<grid, PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
-        case 6: k_prune<6><<<grid, PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
-        case 8: k_prune<8><<<grid, PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
-        case 10: k_prune<10><<<grid, PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
-        default: k_prune<0><<<grid, PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
+        case 4:
+            if (n == 2) {
+                const int64_t runs = (K + 31) / 32;
+                dim3 g24(static_cast<unsigned>((runs + 127) / 128), static_cast<unsigned>(R < 65535 ? R : 65535),
+                         static_cast<unsigned>((R + 65534) / 65535));
+                k_prune24<<<g24, 128, 0, s>>>(S, lds, V, ldv, K, G, mask, vals, meta);
+                break;
+            }
+            k_prune<4><<<grid_for(PruneGPT<4>::value), PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta);
+            break;
+        case 6: k_prune<6><<<grid_for(PruneGPT<6>::value), PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
+        case 8: k_prune<8><<<grid_for(PruneGPT<8>::value), PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
+        case 10: k_prune<10><<<grid_for(PruneGPT<10>::value), PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
+        default: k_prune<0><<<grid_for(PruneGPT<0>::value), PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
     }
     return launch_status();
 }
