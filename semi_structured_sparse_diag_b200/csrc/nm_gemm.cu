@@ -1668,7 +1668,11 @@ nm_status launch_wide(const CUtensorMap &a, const CUtensorMap &b, const CUtensor
     const bool sk_ok = sk_ws != nullptr && sk_ws_bytes >= sk_bytes(res) &&
                        (reinterpret_cast<uintptr_t>(sk_ws) & 15u) == 0;
     const bool sk = sk_ok && (policy == 2 || (policy == 0 && 2 * ntiles <= res));
-    int64_t clusters = sk ? res : (ntiles < res ? ntiles : res);
+    // stream-K: at most ~4 pairs per tile unless the pair count is forced --
+    // each extra contributor costs the tile's owner another round of partial
+    // reads, more than the shorter K' range saves once HBM is the limit
+    int64_t clusters = ntiles < res ? ntiles : res;
+    if (sk) clusters = (forced > 0 || 4 * ntiles >= res) ? res : 4 * ntiles;
     if (clusters < 1) clusters = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
