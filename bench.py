@@ -54,9 +54,9 @@ PAIR_MODE = {4: "PMODE_SP24", 6: "PMODE_SP24 on K'", 8: "PMODE_SP68T", 10: "PMOD
 
 def recorded_traffic(workload: str):
     """DRAM bytes per launch of the sparse GEMM from the committed ncu summary
-    profiles/gemm_pair_<workload>.md, if the kernel source is unchanged since."""
+    profiles/gemm_wide_<workload>.md, if the kernel source is unchanged since."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", f"gemm_pair_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"gemm_wide_{workload}.md")
     src = os.path.join(ROOT, "semi_structured_sparse_diag_b200", "csrc", "nm_gemm.cu")
     try:
         text = open(path).read()
@@ -359,7 +359,7 @@ def run_ours(args):
             "unit": "TFLOP/s",
             "frac": round(achieved / sparse_peak, 4),
             "traffic": recorded_traffic(layer.name),
-            "traffic_source": f"profiles/gemm_pair_{layer.name}.md (ncu dram read+write per launch)",
+            "traffic_source": f"profiles/gemm_wide_{layer.name}.md (ncu dram read+write per launch)",
             "per_unit": "2*R*K'pad flops per token; units per launch = T tokens",
         },
         "e2e": {
