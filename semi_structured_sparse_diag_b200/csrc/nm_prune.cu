@@ -449,7 +449,7 @@ __device__ __forceinline__ void drop_two_of_4(const float (&s)[4], int &dlo, int
     dhi = d0 < d1 ? d1 : d0;
 }
 
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, 8)
     k_prune24(const float *__restrict__ S, int64_t lds, const uint16_t *__restrict__ V, int64_t ldv,
               int64_t K, int64_t G, uint32_t *__restrict__ mask, uint16_t *__restrict__ vals,
               uint8_t *__restrict__ meta24) {
@@ -630,24 +630,60 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------------------------
 // ternary absmean quantisation
 // ---------------------------------------------------------------------------
-__global__ void k_row_abs_sum(const uint16_t *__restrict__ W, int64_t R, int64_t K, int64_t ldw,
-                              double *__restrict__ rowsum) {
-    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (i >= R) return;
-    const uint16_t *w = W + i * ldw;
-    double s = 0.0;
-    int64_t j = 0;
-    for (; j + 8 <= K; j += 8) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(w + j));
-        const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+// Row sums of |W| in the canonical order (each row ascending in column, fp64,
+// sequential).  A block owns 32 rows: all 256 threads stream 32 x 256-column
+// tiles into shared memory with cp.async (coalesced, double-buffered), and
+// warp 0's lane r adds row r's tile left to right.  Rows are padded to 528
+// bytes so a lane's 16-byte reads spread over the banks.
+constexpr int RS_ROWS = 32, RS_COLS = 256, RS_PITCH = RS_COLS + 8;
+
+__global__ void __launch_bounds__(256)
+    k_row_abs_sum(const uint16_t *__restrict__ W, int64_t R, int64_t K, int64_t ldw,
+                  double *__restrict__ rowsum) {
+    __shared__ __align__(16) uint16_t tile[2][RS_ROWS][RS_PITCH];
+    const int64_t r0 = static_cast<int64_t>(blockIdx.x) * RS_ROWS;
+    const int tid = threadIdx.x;
+    const int64_t ntile = (K + RS_COLS - 1) / RS_COLS;
+    auto issue = [&](int64_t t, int buf) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            s = __dadd_rn(s, fabs(bf16_to_f64(static_cast<uint16_t>(q[e] & 0xFFFFu))));
-            s = __dadd_rn(s, fabs(bf16_to_f64(static_cast<uint16_t>(q[e] >> 16))));
+        for (int k = 0; k < 4; ++k) {
+            const int idx = tid + 256 * k;  // 0..1023: row idx / 32, 16-byte chunk idx % 32
+            const int row = idx >> 5, c = idx & 31;
+            const int64_t col = t * RS_COLS + c * 8;
+            const int64_t left = K - col;
+            const uint32_t bytes = (r0 + row < R && left > 0) ? static_cast<uint32_t>(left >= 8 ? 16 : 2 * left) : 0u;
+            const uint16_t *src = bytes ? W + (r0 + row) * ldw + col : W;
+            cp_async16(&tile[buf][row][c * 8], src, bytes);
         }
+        cp_async_commit();
+    };
+    double s = 0.0;
+    issue(0, 0);
+    for (int64_t t = 0; t < ntile; ++t) {
+        if (t + 1 < ntile) {
+            issue(t + 1, static_cast<int>((t + 1) & 1));
+            cp_async_wait_pending<1>();
+        } else {
+            cp_async_wait_pending<0>();
+        }
+        __syncthreads();
+        if (tid < 32) {
+            // zero-filled columns past K add +0 to a non-negative sum: no change
+            const uint16_t *rowp = tile[t & 1][tid];
+#pragma unroll 4
+            for (int c = 0; c < RS_COLS / 8; ++c) {
+                const uint4 u = *reinterpret_cast<const uint4 *>(rowp + c * 8);
+                const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    s = __dadd_rn(s, fabs(bf16_to_f64(static_cast<uint16_t>(q[e] & 0xFFFFu))));
+                    s = __dadd_rn(s, fabs(bf16_to_f64(static_cast<uint16_t>(q[e] >> 16))));
+                }
+            }
+        }
+        __syncthreads();  // buffer t & 1 is refilled by the next iteration's issue
     }
-    for (; j < K; ++j) s = __dadd_rn(s, fabs(bf16_to_f64(w[j])));
-    rowsum[i] = s;
+    if (tid < 32 && r0 + tid < R) rowsum[r0 + tid] = s;
 }
 
 // fp64 -> bf16 bits, round to nearest even, normal range only (0xFFFF if not
@@ -671,11 +707,23 @@ __device__ uint32_t f64_to_bf16_bits(double v) {
     return sign | (static_cast<uint32_t>(e + 127) << 7) | static_cast<uint32_t>(top & 0x7Full);
 }
 
-__global__ void k_gamma(const double *__restrict__ rowsum, int64_t R, int64_t K,
-                        double *__restrict__ gamma_out, uint32_t *__restrict__ gb_out) {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+// gamma = (sum of the row sums, ascending row, fp64 sequential) / (R*K).  The
+// block stages 2048 row sums at a time in shared memory (coalesced loads);
+// thread 0 adds them in order.
+__global__ void __launch_bounds__(256) k_gamma(const double *__restrict__ rowsum, int64_t R, int64_t K,
+                                               double *__restrict__ gamma_out,
+                                               uint32_t *__restrict__ gb_out) {
+    __shared__ double buf[2048];
     double total = 0.0;
-    for (int64_t i = 0; i < R; ++i) total = __dadd_rn(total, rowsum[i]);
+    for (int64_t base = 0; base < R; base += 2048) {
+        const int64_t n = R - base < 2048 ? R - base : 2048;
+        for (int i = threadIdx.x; i < n; i += blockDim.x) buf[i] = rowsum[base + i];
+        __syncthreads();
+        if (threadIdx.x == 0)
+            for (int64_t i = 0; i < n; ++i) total = __dadd_rn(total, buf[i]);
+        __syncthreads();
+    }
+    if (threadIdx.x != 0) return;
     const double gamma = __ddiv_rn(total, __dmul_rn(static_cast<double>(R), static_cast<double>(K)));
     uint32_t gb = f64_to_bf16_bits(gamma);
     if (gamma == 0.0 || gb == 0xFFFFu) {
@@ -686,23 +734,49 @@ __global__ void k_gamma(const double *__restrict__ rowsum, int64_t R, int64_t K,
     *gb_out = gb;
 }
 
+// clip(rint(fl(w / gamma)), -1, 1) without the division.  fl(|w| / gamma) > 0.5
+// exactly when |w| / gamma > 0.5 + 2^-54 (the half-way point to the next
+// double, which rounds to even = 0.5), i.e. |w| > h + 2^-54 gamma with
+// h = gamma / 2.  For h < |w| <= 2h the difference |w| - h is exact (Sterbenz);
+// above 2h the condition holds outright.  rint(x) for |x| > 0.5 is at least 1
+// and clips to 1; |x| <= 0.5 gives 0 (0.5 ties to even).  gamma is a normal
+// double (bf16(gamma) was representable), so gamma / 2 and 2^-54 gamma are
+// exact.  W itself is never NaN here (a NaN would make gamma NaN, which zeroes
+// the output).
+__device__ __forceinline__ uint32_t ternary_one(uint32_t wbits, double h, double tiny, uint32_t gb) {
+    const double a = fabs(bf16_to_f64(static_cast<uint16_t>(wbits)));
+    const bool one = a > 2.0 * h || (a > h && __dsub_rn(a, h) > tiny);
+    return one ? ((wbits & 0x8000u) ? (gb | 0x8000u) : gb) : 0u;
+}
+
+// W_q = clip(rint(W / gamma), -1, 1) * bf16(gamma).  grid: x over 8-column
+// chunks of a row (16-byte load, 16-byte store), y (+65535 z) = row.
 __global__ void __launch_bounds__(256)
     k_ternary_apply(const uint16_t *__restrict__ W, int64_t R, int64_t K, int64_t ldw,
                     const double *__restrict__ gamma_p, const uint32_t *__restrict__ gb_p,
                     uint16_t *__restrict__ Wq) {
+    const int64_t i = blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535;
+    const int64_t j0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+    if (i >= R || j0 >= K) return;
     const double gamma = *gamma_p;
     const uint32_t gb = *gb_p;
-    const int64_t total = R * K;
-    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
-         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t i = idx / K, j = idx - i * K;
-        uint16_t out = 0;
-        if (gb != 0xFFFFu) {
-            double q = rint(__ddiv_rn(bf16_to_f64(W[i * ldw + j]), gamma));
-            q = q > 1.0 ? 1.0 : (q < -1.0 ? -1.0 : q);
-            out = q == 0.0 ? 0 : static_cast<uint16_t>(q > 0.0 ? gb : (gb | 0x8000u));
+    const bool ok = gb != 0xFFFFu;
+    const double h = 0.5 * gamma, tiny = gamma * 0x1p-54;
+    uint16_t *dst = Wq + i * K + j0;
+    if (j0 + 8 <= K && (K & 7) == 0) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(W + i * ldw + j0));
+        const uint32_t in[4] = {u.x, u.y, u.z, u.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const uint32_t lo = ok ? ternary_one(in[e] & 0xFFFFu, h, tiny, gb) : 0u;
+            const uint32_t hi = ok ? ternary_one(in[e] >> 16, h, tiny, gb) : 0u;
+            o[e] = lo | (hi << 16);
         }
-        Wq[idx] = out;
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+    } else {
+        for (int64_t j = j0; j < K && j < j0 + 8; ++j)
+            dst[j - j0] = static_cast<uint16_t>(ok ? ternary_one(W[i * ldw + j], h, tiny, gb) : 0u);
     }
 }
 
@@ -881,12 +955,12 @@ extern "C" nm_status nm_ternary_quantize(const uint16_t *W, int64_t R, int64_t K
     cudaStream_t s = as_stream(stream);
     double *rowsum = static_cast<double *>(ws);
     uint32_t *gb = reinterpret_cast<uint32_t *>(rowsum + R);
-    k_row_abs_sum<<<static_cast<unsigned>((R + 127) / 128), 128, 0, s>>>(W, R, K, ldw, rowsum);
-    k_gamma<<<1, 32, 0, s>>>(rowsum, R, K, gamma, gb);
-    int64_t blocks = (R * K + 255) / 256;
-    const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
-    if (blocks > cap) blocks = cap;
-    k_ternary_apply<<<static_cast<unsigned>(blocks), 256, 0, s>>>(W, R, K, ldw, gamma, gb, Wq);
+    if ((R + RS_ROWS - 1) / RS_ROWS > 0x7FFFFFFF || R > 65535LL * 65535LL) return NM_ERR_SHAPE;
+    k_row_abs_sum<<<static_cast<unsigned>((R + RS_ROWS - 1) / RS_ROWS), 256, 0, s>>>(W, R, K, ldw, rowsum);
+    k_gamma<<<1, 256, 0, s>>>(rowsum, R, K, gamma, gb);
+    dim3 grid(static_cast<unsigned>((K + 2047) / 2048), static_cast<unsigned>(R < 65535 ? R : 65535),
+              static_cast<unsigned>((R + 65534) / 65535));
+    k_ternary_apply<<<grid, 256, 0, s>>>(W, R, K, ldw, gamma, gb, Wq);
     return launch_status();
 }
 
