@@ -7,7 +7,8 @@ One step = one pass of the whole path over one layer of synthetic input:
   a3 top-n per group + compress (nm_prune_compress)
   a4 sliding-window pack       (slide_pack, m > 4)
   a6 operand preparation       (nm_sparse_prepare)
-  a5+a7 lift-in-staging sparse GEMM Y = X W_sparse^T (nm_sparse_gemm)
+  a5+a7 sparse GEMM Y = X W_sparse^T on the lifted activations (nm_sparse_gemm:
+               6:8 middle windows gathered, 4:6 / 8:10 X' lifted, before the GEMM)
   a8 own dense GEMM on the masked W (nm_dense_gemm), the speedup reference.
 
 Prints ONE JSON line.  `value` is the sparse GEMM's effective TFLOP/s,
@@ -134,6 +135,37 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------
+# multi-rank host logic (one process per GPU; weak scaling, no data-path
+# collective: each rank prunes and multiplies its own seeded layer)
+# --------------------------------------------------------------------------
+def rank_env():
+    """(world size, rank, local rank) from the torchrun environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_inputs(layer: datagen.Layer, rank: int):
+    """The seeded (X, W) bf16 bit patterns of this rank's layer."""
+    return datagen.layer_inputs(layer, seed=layer.seed + rank)
+
+
+def max_over_ranks(values, world: int, device=None):
+    """Each rank's timings -> the slowest rank's, element by element."""
+    if world == 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_tflops(world: int, flops_per_rank: float, ms: float) -> float:
+    """Whole-job throughput: all ranks' work over the slowest rank's time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
+# --------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------
 def run_ours(args):
@@ -142,17 +174,14 @@ def run_ours(args):
 
     import semi_structured_sparse_diag_b200 as nm
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local)
     layer = datagen.WORKLOADS[args.workload]
-    # weak scaling: every rank prunes and multiplies its own layer (seed = rank)
-    X_h, W_h = datagen.layer_inputs(layer, seed=layer.seed + rank)
+    X_h, W_h = rank_inputs(layer, rank)
     R, K, T, n, m = layer.R, layer.K, layer.T, layer.n, layer.m
     lib = nm.load()
     stream = torch.cuda.current_stream()
@@ -293,10 +322,7 @@ def run_ours(args):
     step_ms /= args.steps
     gemm_ms = stage_ms["sparse_gemm"]
     dense_ms = stage_ms["dense_gemm"]
-    if world > 1:
-        t = torch.tensor([step_ms, gemm_ms, dense_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms, gemm_ms, dense_ms = t.tolist()
+    step_ms, gemm_ms, dense_ms = max_over_ranks([step_ms, gemm_ms, dense_ms], world, dev)
 
     # ------------------------------------------------ end-to-end through the C ABI
     Xh = torch.from_numpy(X_h.view(np.int16)).pin_memory()
@@ -320,17 +346,14 @@ def run_ours(args):
         torch.cuda.synchronize()
         e2e_ms += e0.elapsed_time(e1)
     e2e_ms /= e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
+    e2e_ms = max_over_ranks([e2e_ms], world, dev)[0]
     nm.check_device_error()
 
     hbm, bf16_tf, peak_src = peaks()
     sparse_peak = 2.0 * bf16_tf  # 2:4 sparse bf16 = 2 x dense bf16 (nominal 4.5 / 2.25)
     flops_eff = 2.0 * T * R * K                 # dense-equivalent of the original layer
     flops_lift = 2.0 * T * R * KLpad            # dense-equivalent of the lifted 2:4 problem
-    value = world * flops_eff / (gemm_ms * 1e-3) / 1e12
+    value = job_tflops(world, flops_eff, gemm_ms)
     achieved = flops_lift / (gemm_ms * 1e-3) / 1e12
     line = {
         "metric": METRIC,
@@ -363,7 +386,7 @@ def run_ours(args):
             "per_unit": "2*R*K'pad flops per token; units per launch = T tokens",
         },
         "e2e": {
-            "value": round(world * flops_eff / (e2e_ms * 1e-3) / 1e12, 3),
+            "value": round(job_tflops(world, flops_eff, e2e_ms), 3),
             "unit": "TFLOP/s",
             "ms_per_step": round(e2e_ms, 4),
             "h2d_bytes_per_step": int(X_h.nbytes + W_h.nbytes),

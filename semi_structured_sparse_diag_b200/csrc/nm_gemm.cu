@@ -1401,36 +1401,50 @@ __global__ void __launch_bounds__(WideCfg::THREADS, 1)
 
 // ---------------------------------------------------------------------------
 // 6:8 middle windows: X_mid[t, 4g + i] = X[t, 8g + 2 + i] (i < 4), zero past K.
-// One thread per two groups: two 16-byte loads, one 16-byte store.
-// grid: x over pairs of groups, y (+65535 z) over tokens.
+// One thread per two groups and GATHER_TOKENS consecutive tokens: all 16-byte
+// loads first (2 per token), then one 16-byte store per token.
+// grid: x over pairs of groups, y (+65535 z) over token runs.
 // ---------------------------------------------------------------------------
+constexpr int GATHER_TOKENS = 4;
+
 __global__ void __launch_bounds__(256)
     k_gather_mid(const uint16_t *__restrict__ X, int64_t T, int64_t K, int64_t ldx, int64_t G,
                  uint16_t *__restrict__ Xmid, int64_t ldm) {
     grid_dep_launch();
-    const int64_t t = blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535;
+    const int64_t t0 = (blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535) * GATHER_TOKENS;
     const int64_t h = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // group pair
-    if (t >= T || 2 * h >= G) return;
-    const uint16_t *src = X + t * ldx + 16 * h;
-    uint32_t o[4];
-    if (16 * h + 16 <= K) {
-        const uint4 a = __ldg(reinterpret_cast<const uint4 *>(src));
-        const uint4 b = __ldg(reinterpret_cast<const uint4 *>(src) + 1);
-        o[0] = a.y; o[1] = a.z; o[2] = b.y; o[3] = b.z;
-    } else {
+    if (t0 >= T || 2 * h >= G) return;
+    const bool full_k = 16 * h + 16 <= K;
+    uint32_t o[GATHER_TOKENS][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int64_t c = 16 * h + 8 * (j >> 1) + 2 + 2 * (j & 1);
-            const uint32_t lo = c < K ? __ldg(src + (c - 16 * h)) : 0u;
-            const uint32_t hi = c + 1 < K ? __ldg(src + (c + 1 - 16 * h)) : 0u;
-            o[j] = lo | (hi << 16);
+    for (int u = 0; u < GATHER_TOKENS; ++u) {
+        const int64_t t = t0 + u;
+        if (t >= T) break;
+        const uint16_t *src = X + t * ldx + 16 * h;
+        if (full_k) {
+            const uint4 a = __ldg(reinterpret_cast<const uint4 *>(src));
+            const uint4 b = __ldg(reinterpret_cast<const uint4 *>(src) + 1);
+            o[u][0] = a.y; o[u][1] = a.z; o[u][2] = b.y; o[u][3] = b.z;
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int64_t c = 16 * h + 8 * (j >> 1) + 2 + 2 * (j & 1);
+                const uint32_t lo = c < K ? __ldg(src + (c - 16 * h)) : 0u;
+                const uint32_t hi = c + 1 < K ? __ldg(src + (c + 1 - 16 * h)) : 0u;
+                o[u][j] = lo | (hi << 16);
+            }
         }
     }
-    uint16_t *dst = Xmid + t * ldm + 8 * h;
-    if (2 * h + 2 <= G) {
-        *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
-    } else {  // last, odd group: four columns only
-        *reinterpret_cast<uint2 *>(dst) = make_uint2(o[0], o[1]);
+#pragma unroll
+    for (int u = 0; u < GATHER_TOKENS; ++u) {
+        const int64_t t = t0 + u;
+        if (t >= T) break;
+        uint16_t *dst = Xmid + t * ldm + 8 * h;
+        if (2 * h + 2 <= G) {
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(o[u][0], o[u][1], o[u][2], o[u][3]);
+        } else {  // last, odd group: four columns only
+            *reinterpret_cast<uint2 *>(dst) = make_uint2(o[u][0], o[u][1]);
+        }
     }
 }
 
@@ -1827,8 +1841,9 @@ nm_status sparse_gemm_impl(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
     int64_t b_cols = K, b_ld = ldx;
     if (m == 8) {
         const int64_t pairs = (p.G + 1) / 2;
-        dim3 grid(static_cast<unsigned>((pairs + 255) / 256), static_cast<unsigned>(T < 65535 ? T : 65535),
-                  static_cast<unsigned>((T + 65534) / 65535));
+        const int64_t runs = (T + GATHER_TOKENS - 1) / GATHER_TOKENS;
+        dim3 grid(static_cast<unsigned>((pairs + 255) / 256), static_cast<unsigned>(runs < 65535 ? runs : 65535),
+                  static_cast<unsigned>((runs + 65534) / 65535));
         k_gather_mid<<<grid, 256, 0, s>>>(X, T, K, ldx, p.G, stage, w.ld);
         if (cudaGetLastError() != cudaSuccess) return NM_ERR_CUDA;
     } else if (m != 4) {
