@@ -358,22 +358,44 @@ void oracle_gemm_lifted(const uint16_t *XL, int64_t T, int64_t KL, const uint16_
 
 /* ------------------------------------------------------------------------ */
 /* Ternary absmean quantisation (Sparse-BitNet, "O Problema" item 1):
- *   gamma = mean |W| over the tensor, fp64: each row summed in ascending
- *           column order, row sums added in ascending row order, then / (R*K);
+ *   gamma = mean |W| over the tensor, fp64, in a fixed order:
+ *     row sum: 32 partial sums; partial l takes the 8-column chunks
+ *              l, l+32, l+64, ... (columns 8c .. 8c+7 of chunk c, those < K),
+ *              each |w| added in ascending column order; then the partials
+ *              are combined by halving: p[l] += p[l+16] (l < 16), then +8,
+ *              +4, +2, +1; the row sum is p[0];
+ *     total:   the row sums in blocks of 1024 consecutive rows, zero-padded,
+ *              each block combined by halving (a[t] += a[t+512] for t < 512,
+ *              then 256, ..., 1), the block sums added in ascending order;
+ *     gamma = total / (R*K)  (one correctly rounded division);
  *   q     = clip(rint(W / gamma), -1, 1), ties to even;
  *   W_q   = q * bf16(gamma), bf16(gamma) rounded to nearest even from fp64.
  * Returns gamma (fp64), or -1.0 if bf16(gamma) is out of the normal range.  */
 double oracle_ternary(const uint16_t *W, int64_t R, int64_t K, int64_t ldw, uint16_t *Wq) {
     double *rowsum = (double *)malloc((size_t)R * sizeof(double));
     if (!rowsum) return -1.0;
+    const int64_t nchunks = (K + 7) / 8;
     #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < R; ++i) {
-        double s = 0.0;
-        for (int64_t j = 0; j < K; ++j) s = s + fabs(bf16_to_f64(W[i * ldw + j]));
-        rowsum[i] = s;
+        double p[32];
+        for (int l = 0; l < 32; ++l) {
+            double s = 0.0;
+            for (int64_t c = l; c < nchunks; c += 32)
+                for (int64_t j = 8 * c; j < 8 * c + 8 && j < K; ++j) s = s + fabs(bf16_to_f64(W[i * ldw + j]));
+            p[l] = s;
+        }
+        for (int stride = 16; stride >= 1; stride /= 2)
+            for (int l = 0; l < stride; ++l) p[l] = p[l] + p[l + stride];
+        rowsum[i] = p[0];
     }
     double total = 0.0;
-    for (int64_t i = 0; i < R; ++i) total = total + rowsum[i];
+    double a[1024];
+    for (int64_t b = 0; b < R; b += 1024) {
+        for (int t = 0; t < 1024; ++t) a[t] = (b + t < R) ? rowsum[b + t] : 0.0;
+        for (int stride = 512; stride >= 1; stride /= 2)
+            for (int t = 0; t < stride; ++t) a[t] = a[t] + a[t + stride];
+        total = total + a[0];
+    }
     free(rowsum);
     double gamma = total / ((double)R * (double)K);
     uint16_t gb = f64_to_bf16_rne(gamma);

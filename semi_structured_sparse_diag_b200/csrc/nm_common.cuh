@@ -442,14 +442,6 @@ __device__ __forceinline__ void cp_async4(void *smem_dst, const void *gsrc, uint
                  : "memory");
 }
 
-// 16-byte global -> shared asynchronous copy, bypassing L1; bytes past
-// src_bytes (0..16) are zero-filled
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
-                 "l"(gsrc), "r"(src_bytes)
-                 : "memory");
-}
-
 __device__ __forceinline__ void cp_async_commit_wait_all() {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }

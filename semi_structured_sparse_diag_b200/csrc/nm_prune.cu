@@ -630,60 +630,55 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------------------------
 // ternary absmean quantisation
 // ---------------------------------------------------------------------------
-// Row sums of |W| in the canonical order (each row ascending in column, fp64,
-// sequential).  A block owns 32 rows: all 256 threads stream 32 x 256-column
-// tiles into shared memory with cp.async (coalesced, double-buffered), and
-// warp 0's lane r adds row r's tile left to right.  Rows are padded to 528
-// bytes so a lane's 16-byte reads spread over the banks.
-constexpr int RS_ROWS = 32, RS_COLS = 256, RS_PITCH = RS_COLS + 8;
-
+// Row sums of |W| in the canonical order: one warp per row; lane l sums the
+// 8-column chunks l, l+32, ... (16-byte loads, a warp instruction reads 512
+// contiguous bytes) left to right, then the 32 partials are combined by
+// halving (lane l adds lane l+16, then +8, +4, +2, +1).
 __global__ void __launch_bounds__(256)
     k_row_abs_sum(const uint16_t *__restrict__ W, int64_t R, int64_t K, int64_t ldw,
                   double *__restrict__ rowsum) {
-    __shared__ __align__(16) uint16_t tile[2][RS_ROWS][RS_PITCH];
-    const int64_t r0 = static_cast<int64_t>(blockIdx.x) * RS_ROWS;
-    const int tid = threadIdx.x;
-    const int64_t ntile = (K + RS_COLS - 1) / RS_COLS;
-    auto issue = [&](int64_t t, int buf) {
+    const int lane = threadIdx.x & 31;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (row >= R) return;  // warp-uniform
+    const uint16_t *w = W + row * ldw;
+    const int64_t nchunks = (K + 7) / 8;
+    double s = 0.0;
+    int64_t c = lane;
+    // four chunks in flight per lane
+    for (; c + 96 < nchunks && 8 * (c + 96) + 8 <= K; c += 128) {
+        uint4 u[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) u[k] = __ldg(reinterpret_cast<const uint4 *>(w + 8 * (c + 32 * k)));
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const int idx = tid + 256 * k;  // 0..1023: row idx / 32, 16-byte chunk idx % 32
-            const int row = idx >> 5, c = idx & 31;
-            const int64_t col = t * RS_COLS + c * 8;
-            const int64_t left = K - col;
-            const uint32_t bytes = (r0 + row < R && left > 0) ? static_cast<uint32_t>(left >= 8 ? 16 : 2 * left) : 0u;
-            const uint16_t *src = bytes ? W + (r0 + row) * ldw + col : W;
-            cp_async16(&tile[buf][row][c * 8], src, bytes);
-        }
-        cp_async_commit();
-    };
-    double s = 0.0;
-    issue(0, 0);
-    for (int64_t t = 0; t < ntile; ++t) {
-        if (t + 1 < ntile) {
-            issue(t + 1, static_cast<int>((t + 1) & 1));
-            cp_async_wait_pending<1>();
-        } else {
-            cp_async_wait_pending<0>();
-        }
-        __syncthreads();
-        if (tid < 32) {
-            // zero-filled columns past K add +0 to a non-negative sum: no change
-            const uint16_t *rowp = tile[t & 1][tid];
-#pragma unroll 4
-            for (int c = 0; c < RS_COLS / 8; ++c) {
-                const uint4 u = *reinterpret_cast<const uint4 *>(rowp + c * 8);
-                const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+            const uint32_t q[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    s = __dadd_rn(s, fabs(bf16_to_f64(static_cast<uint16_t>(q[e] & 0xFFFFu))));
-                    s = __dadd_rn(s, fabs(bf16_to_f64(static_cast<uint16_t>(q[e] >> 16))));
-                }
+            for (int e = 0; e < 4; ++e) {
+                s = __dadd_rn(s, fabs(bf16_to_f64(static_cast<uint16_t>(q[e] & 0xFFFFu))));
+                s = __dadd_rn(s, fabs(bf16_to_f64(static_cast<uint16_t>(q[e] >> 16))));
             }
         }
-        __syncthreads();  // buffer t & 1 is refilled by the next iteration's issue
     }
-    if (tid < 32 && r0 + tid < R) rowsum[r0 + tid] = s;
+    for (; c < nchunks; c += 32) {
+        const int64_t j0 = 8 * c;
+        if (j0 + 8 <= K) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(w + j0));
+            const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                s = __dadd_rn(s, fabs(bf16_to_f64(static_cast<uint16_t>(q[e] & 0xFFFFu))));
+                s = __dadd_rn(s, fabs(bf16_to_f64(static_cast<uint16_t>(q[e] >> 16))));
+            }
+        } else {
+            for (int64_t j = j0; j < K; ++j) s = __dadd_rn(s, fabs(bf16_to_f64(w[j])));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        const double o = __shfl_down_sync(0xffffffffu, s, off);
+        if (lane < off) s = __dadd_rn(s, o);
+    }
+    if (lane == 0) rowsum[row] = s;
 }
 
 // fp64 -> bf16 bits, round to nearest even, normal range only (0xFFFF if not
@@ -707,23 +702,26 @@ __device__ uint32_t f64_to_bf16_bits(double v) {
     return sign | (static_cast<uint32_t>(e + 127) << 7) | static_cast<uint32_t>(top & 0x7Full);
 }
 
-// gamma = (sum of the row sums, ascending row, fp64 sequential) / (R*K).  The
-// block stages 2048 row sums at a time in shared memory (coalesced loads);
-// thread 0 adds them in order.
-__global__ void __launch_bounds__(256) k_gamma(const double *__restrict__ rowsum, int64_t R, int64_t K,
-                                               double *__restrict__ gamma_out,
-                                               uint32_t *__restrict__ gb_out) {
-    __shared__ double buf[2048];
+// gamma = total / (R*K): the row sums in blocks of 1024 rows (zero-padded),
+// each block combined by halving (a[t] += a[t + stride], stride 512 .. 1), the
+// block sums added in ascending order.  One block of 1024 threads.
+__global__ void __launch_bounds__(1024) k_gamma(const double *__restrict__ rowsum, int64_t R, int64_t K,
+                                                double *__restrict__ gamma_out,
+                                                uint32_t *__restrict__ gb_out) {
+    __shared__ double a[1024];
+    const int t = threadIdx.x;
     double total = 0.0;
-    for (int64_t base = 0; base < R; base += 2048) {
-        const int64_t n = R - base < 2048 ? R - base : 2048;
-        for (int i = threadIdx.x; i < n; i += blockDim.x) buf[i] = rowsum[base + i];
+    for (int64_t b = 0; b < R; b += 1024) {
+        a[t] = b + t < R ? rowsum[b + t] : 0.0;
         __syncthreads();
-        if (threadIdx.x == 0)
-            for (int64_t i = 0; i < n; ++i) total = __dadd_rn(total, buf[i]);
+        for (int stride = 512; stride >= 1; stride >>= 1) {
+            if (t < stride) a[t] = __dadd_rn(a[t], a[t + stride]);
+            __syncthreads();
+        }
+        if (t == 0) total = __dadd_rn(total, a[0]);
         __syncthreads();
     }
-    if (threadIdx.x != 0) return;
+    if (t != 0) return;
     const double gamma = __ddiv_rn(total, __dmul_rn(static_cast<double>(R), static_cast<double>(K)));
     uint32_t gb = f64_to_bf16_bits(gamma);
     if (gamma == 0.0 || gb == 0xFFFFu) {
@@ -955,9 +953,9 @@ extern "C" nm_status nm_ternary_quantize(const uint16_t *W, int64_t R, int64_t K
     cudaStream_t s = as_stream(stream);
     double *rowsum = static_cast<double *>(ws);
     uint32_t *gb = reinterpret_cast<uint32_t *>(rowsum + R);
-    if ((R + RS_ROWS - 1) / RS_ROWS > 0x7FFFFFFF || R > 65535LL * 65535LL) return NM_ERR_SHAPE;
-    k_row_abs_sum<<<static_cast<unsigned>((R + RS_ROWS - 1) / RS_ROWS), 256, 0, s>>>(W, R, K, ldw, rowsum);
-    k_gamma<<<1, 256, 0, s>>>(rowsum, R, K, gamma, gb);
+    if ((R + 7) / 8 > 0x7FFFFFFF || R > 65535LL * 65535LL) return NM_ERR_SHAPE;
+    k_row_abs_sum<<<static_cast<unsigned>((R + 7) / 8), 256, 0, s>>>(W, R, K, ldw, rowsum);
+    k_gamma<<<1, 1024, 0, s>>>(rowsum, R, K, gamma, gb);
     dim3 grid(static_cast<unsigned>((K + 2047) / 2048), static_cast<unsigned>(R < 65535 ? R : 65535),
               static_cast<unsigned>((R + 65534) / 65535));
     k_ternary_apply<<<grid, 256, 0, s>>>(W, R, K, ldw, gamma, gb, Wq);

@@ -364,6 +364,28 @@ def test_ternary_gaussian_zero_fraction():
     assert abs(frac - 0.3101) < 0.005
 
 
+def test_ternary_gamma_exact_on_integers():
+    # small-integer |w| (exact in bf16): every partial sum is an exact integer,
+    # so gamma is the correctly rounded mean whatever the order -- a dropped or
+    # doubled element (ragged K: 1003 is not a multiple of 8 or 256) changes it
+    rng = np.random.default_rng(7)
+    Wf = rng.integers(-6, 7, size=(37, 1003)).astype(np.float32)
+    W = datagen.f32_to_bf16_bits(Wf)
+    g, _ = oracle.ternary(W)
+    total = int(np.abs(Wf).astype(np.int64).sum())
+    assert g == total / (37 * 1003)
+
+
+def test_ternary_gamma_close_to_exact_sum():
+    # the fixed order loses at most a few ulps against the exact sum (fsum)
+    import math
+    W = datagen.make_weight(1500, 1030, 0.02, seed=3)
+    g, _ = oracle.ternary(W)
+    absw = np.abs((W.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
+    exact = math.fsum(absw.ravel().tolist()) / absw.size
+    assert abs(g - exact) <= 1e-13 * exact
+
+
 def test_f64_to_bf16_rounding():
     assert oracle.f64_to_bf16(1.0) == 0x3F80
     assert oracle.f64_to_bf16(-2.0) == 0xC000
