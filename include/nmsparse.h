@@ -250,8 +250,12 @@ nm_status nm_gemm_set_schedule(int policy, int clusters);
 
 /* Ternary absmean quantisation (Sparse-BitNet sec. 1 item 1), input
  * preparation of the ternary 6:8 layer.
- *   gamma = (sum over rows, ascending, of each row's ascending-column sum of
- *            |W|, in fp64) / (R*K);
+ *   gamma = (sum of |W| in fp64) / (R*K), summed in a fixed order: per row,
+ *           32 partial sums (partial l: the 8-column chunks l, l+32, ..., each
+ *           in ascending column order) combined by halving (l += l+16, +8, +4,
+ *           +2, +1); the row sums in blocks of 1024 rows, zero-padded, each
+ *           combined by halving (t += t+512, ..., +1), the block sums added in
+ *           ascending order;
  *   q     = clip(rint(W / gamma), -1, 1) (fp64 division, ties to even);
  *   W_q   = q * bf16(gamma), bf16(gamma) rounded to nearest even from fp64,
  *           zeros stored as +0.
