@@ -2,9 +2,11 @@
 """Benchmark of the N:M-pruned linear layer hot path on B200.
 
 One step = one pass of the whole path over one layer of synthetic input:
-  a1 H = mean_t x^2            (nm_hessian_diag, part of nm_score)
-  a2 S = (H + eps) W^2         (nm_score)
-  a3 top-n per group + compress (nm_prune_compress)
+  a1 H = mean_t x^2            (nm_hessian_diag; for the ternary layer the
+                                absmean quantisation, nm_ternary_quantize)
+  a2 S = (H + eps) W^2 and
+  a3 top-n per group + compress, in one pass (nm_score_prune_compress: the
+                                scores stay in registers)
   a4 sliding-window pack       (slide_pack, m > 4)
   a6 operand preparation       (nm_sparse_prepare)
   a5+a7 sparse GEMM Y = X W_sparse^T on the lifted activations (nm_sparse_gemm:
@@ -196,7 +198,6 @@ def run_ours(args):
     KLpad = (KL + 127) // 128 * 128
     # persistent buffers (allocated once, outside the timed region)
     H = torch.empty(K, dtype=torch.float64, device=dev)
-    S = torch.empty((R, K), dtype=torch.float32, device=dev)
     ws = torch.empty(max(1, lib.nm_hessian_workspace_bytes(T, K)), dtype=torch.uint8, device=dev)
     mask = torch.empty((R, (G * m + 31) // 32), dtype=torch.int32, device=dev)
     vals = torch.empty((R, G * n), dtype=torch.bfloat16, device=dev)
@@ -225,7 +226,9 @@ def run_ours(args):
         if st != 0:
             raise nm.NMError(f"{what}: {lib.nm_status_string(st).decode()}")
 
-    stage_names = ["score", "prune", "slide_pack", "prepare", "sparse_gemm", "dense_gemm"]
+    # a1 (or the ternary quantisation of C4-style layers), a2+a3 fused, a4, a6,
+    # a5+a7, a8
+    stage_names = ["hessian_or_ternary", "score_prune", "slide_pack", "prepare", "sparse_gemm", "dense_gemm"]
     launches_per_step = 0
 
     def step(ev=None, Xs=X, Ws=W):
@@ -239,18 +242,16 @@ def run_ours(args):
                                         tws.data_ptr(), tws.numel(), s), "ternary")
             cnt += 3
         if layer.score == "hessian":
-            chk(lib.nm_score(Xs.data_ptr(), T, K, Ws.data_ptr(), R, K, K, layer.eps, H.data_ptr(),
-                             S.data_ptr(), ws.data_ptr(), ws.numel(), s), "score")
-            cnt += 3 if T > 128 else 2  # H chunk (+ finish) + score
-        else:
-            chk(lib.nm_score(None, 0, 0, Ws.data_ptr(), R, K, K, 0.0, None, S.data_ptr(), None, 0, s),
-                "score")
-            cnt += 1
+            chk(lib.nm_hessian_diag(Xs.data_ptr(), T, K, K, H.data_ptr(), ws.data_ptr(), ws.numel(), s),
+                "hessian")
+            cnt += 2 if T > 128 else 1  # H chunk partials (+ ordered finish)
         if ev is not None:
             ev[1].record(stream)
-        chk(lib.nm_prune_compress(S.data_ptr(), K, Vs.data_ptr(), K, R, K, n, m, mask.data_ptr(),
-                                  vals.data_ptr(), meta.data_ptr() if meta is not None else None, s),
-            "prune")
+        # a2 + a3 in one pass: scores formed in registers, never written
+        chk(lib.nm_score_prune_compress(H.data_ptr() if layer.score == "hessian" else None, layer.eps,
+                                        Ws.data_ptr(), K, Vs.data_ptr(), K, R, K, n, m, mask.data_ptr(),
+                                        vals.data_ptr(), meta.data_ptr() if meta is not None else None, s),
+            "score_prune")
         cnt += 1
         if ev is not None:
             ev[2].record(stream)

@@ -18,6 +18,8 @@
  *                     Sparse-BitNet sec. 1 (N:M definition) and sec. 2
  *                     ("Quantizar e depois Mascarar": the values compressed are
  *                     whatever V the caller passes, e.g. ternary W_q).
+ *   nm_score_prune_compress  the two steps above in one pass: the scores are
+ *                     formed in registers and never written.
  *   slide_pack        (2N-2):2N -> N-1 overlapping width-4 windows at stride 2,
  *                     each 2:4. SlideSparse (arXiv 2603.05232) sec. 2A.
  *   lift_activations  X'[t, g*4(N-1) + 4w + i] = X[t, g*2N + 2w + i].
@@ -157,6 +159,19 @@ nm_status nm_score_from_hessian(const double *H, double eps, const uint16_t *W, 
 nm_status nm_prune_compress(const float *S, int64_t lds, const uint16_t *V, int64_t ldv,
                             int64_t R, int64_t K, int n, int m, uint32_t *mask, uint16_t *vals,
                             uint8_t *meta24, void *stream);
+
+/* a2 + a3 fused: exactly nm_score_from_hessian followed by nm_prune_compress
+ * (bit-identical mask, vals and meta24), with each score formed in registers
+ * from W -- fp32((H_j + eps) * W_ij^2), fp64 add and multiplies, rounded once;
+ * or |W_ij| when H == NULL -- and never written: HBM traffic per weight drops
+ * from 2 + 4 (score) + 4 + 2 (prune) bytes read/written to the 2 (+ 2 for a
+ * separate V) read by the selection.
+ *   H : [K] fp64 (8-byte aligned) or NULL.  W : [R x K] bf16, ldw >= K,
+ *   ldw % 8 == 0.  V, mask, vals, meta24 and all rules as nm_prune_compress;
+ *   V may be W itself (then W is read once).                                */
+nm_status nm_score_prune_compress(const double *H, double eps, const uint16_t *W, int64_t ldw,
+                                  const uint16_t *V, int64_t ldv, int64_t R, int64_t K, int n, int m,
+                                  uint32_t *mask, uint16_t *vals, uint8_t *meta24, void *stream);
 
 /* a4: sliding-window pack (SlideSparse, sec. 2A), m = 2N in {4, 6, 8, 10},
  * n = m - 2.  Survivor k (0-based, ascending) of a group goes to window k/2,

@@ -20,7 +20,7 @@ from . import build as _build
 
 __all__ = [
     "NMError", "load", "hessian_diag", "score", "score_from_hessian", "prune_compress",
-    "slide_pack", "lift_activations", "sparse_prepare", "sparse_gemm", "dense_gemm",
+    "score_prune_compress", "slide_pack", "lift_activations", "sparse_prepare", "sparse_gemm", "dense_gemm",
     "ternary_quantize", "check_device_error", "set_gemm_schedule", "EXPORTED",
 ]
 
@@ -31,7 +31,7 @@ EXPORTED = (
     "nm_sparse_prepare", "nm_sparse_gemm", "nm_dense_gemm", "nm_ternary_workspace_bytes",
     "nm_ternary_quantize", "nm_hessian_diag_noalloc", "nm_probe_mma", "nm_probe_copy", "nm_gemm_1cta", "nm_sparse_gemm_workspace_bytes",
     "nm_sparse_gemm_fused", "nm_dense_gemm_workspace_bytes", "nm_gemm_set_schedule",
-    "nm_sparse_gemm_tile256",
+    "nm_sparse_gemm_tile256", "nm_score_prune_compress",
 )
 
 _P, _I64, _I, _D, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_size_t
@@ -44,6 +44,7 @@ _SIGS = {
     "nm_score": (_I, [_P, _I64, _I64, _P, _I64, _I64, _I64, _D, _P, _P, _P, _SZ, _P]),
     "nm_score_from_hessian": (_I, [_P, _D, _P, _I64, _I64, _I64, _P, _P]),
     "nm_prune_compress": (_I, [_P, _I64, _P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P]),
+    "nm_score_prune_compress": (_I, [_P, _D, _P, _I64, _P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P]),
     "slide_pack": (_I, [_P, _I64, _I64, _I, _P, _P]),
     "lift_activations": (_I, [_P, _I64, _I64, _I64, _I, _P, _I64, _P]),
     "nm_sparse_prepare_bytes": (_SZ, [_I64, _I64, _I]),
@@ -195,6 +196,26 @@ def prune_compress(S, V, n, m, K=None, stream=None):
     meta = torch.empty((R, (G + 1) // 2), dtype=torch.uint8, device=dev) if (m == 4 and n == 2) else None
     _check(load().nm_prune_compress(_ptr(S), S.stride(0), _ptr(V), _ld(V), R, K, n, m, _ptr(mask),
                                     _ptr(vals), _ptr(meta), _stream(stream)), "nm_prune_compress")
+    return mask, vals, meta
+
+
+def score_prune_compress(H, W, n, m, V=None, eps=1e-8, stream=None):
+    """a2 + a3 in one pass (scores never written): H fp64 [K] or None (|W|
+    scores); V defaults to W.  Returns (mask, vals, meta24 or None) exactly as
+    prune_compress(score(...), V) would."""
+    W = _bf16(W, "W")
+    V = W if V is None else _bf16(V, "V")
+    if H is not None:
+        _dev(H, "H")
+    R, K = W.shape
+    G = n_groups(K, m)
+    dev = W.device
+    mask = torch.empty((R, (G * m + 31) // 32), dtype=torch.int32, device=dev)
+    vals = torch.empty((R, G * n), dtype=torch.bfloat16, device=dev)
+    meta = torch.empty((R, (G + 1) // 2), dtype=torch.uint8, device=dev) if (m == 4 and n == 2) else None
+    _check(load().nm_score_prune_compress(_ptr(H), eps, _ptr(W), _ld(W), _ptr(V), _ld(V), R, K, n, m,
+                                          _ptr(mask), _ptr(vals), _ptr(meta), _stream(stream)),
+           "nm_score_prune_compress")
     return mask, vals, meta
 
 

@@ -103,6 +103,26 @@ __device__ __forceinline__ float score_one(const double *__restrict__ H, double 
     return __double2float_rn(__dmul_rn(h, __dmul_rn(w, w)));
 }
 
+// Where a3 takes its selection scores from: the stored S, or -- a2 fused into
+// a3, S never written -- computed in registers from W exactly as k_score
+// does: fp32((H_j + eps) * w^2) with fp64 add and multiplies, or |w| when H is
+// null.
+struct ScoreSrc {
+    const float *S;      // stored scores (used when not fused)
+    int64_t lds;
+    const uint16_t *W;   // fused: the weights the scores come from
+    int64_t ldw;
+    const double *H;     // fused: null -> magnitude score
+    double eps;
+};
+
+__device__ __forceinline__ float fused_score(const double *__restrict__ H, double eps, int64_t c,
+                                             uint16_t wb) {
+    if (H == nullptr) return fabsf(bf16_to_f32(wb));
+    const double w = bf16_to_f64(wb);
+    return __double2float_rn(__dmul_rn(__dadd_rn(__ldg(H + c), eps), __dmul_rn(w, w)));
+}
+
 // grid: x = 4096-column slice of a row (256 threads x 2 chunks x 8 elements),
 // y (+65535 z) = row.  Both chunks' loads are issued before any arithmetic.
 // Each block: SCORE_ROWS rows x 4096 columns; a thread owns two 8-column
@@ -181,6 +201,80 @@ __global__ void __launch_bounds__(256, 4) k_score(const double *__restrict__ H, 
 // assembled in shared memory (32*m bits = m whole words, word-aligned).
 // ---------------------------------------------------------------------------
 constexpr int PRUNE_THREADS = 256;
+
+// V values of one group [c0, c0 + m), zero past K (vector loads when whole)
+template <int M>
+__device__ __forceinline__ void load_values(const uint16_t *__restrict__ vrow, int64_t c0, int64_t K,
+                                            int m_rt, uint16_t *v) {
+    constexpr int MM = M > 0 ? M : 16;
+    const int m = M > 0 ? M : m_rt;
+    if (M > 0 && c0 + M <= K) {
+        if constexpr (M % 8 == 0) {
+#pragma unroll
+            for (int q = 0; q < M; q += 8) {
+                const uint4 u = __ldg(reinterpret_cast<const uint4 *>(vrow + c0 + q));
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    v[q + 2 * e] = static_cast<uint16_t>(w[e] & 0xFFFFu);
+                    v[q + 2 * e + 1] = static_cast<uint16_t>(w[e] >> 16);
+                }
+            }
+        } else if constexpr (M % 4 == 0) {
+#pragma unroll
+            for (int q = 0; q < M; q += 4) {
+                const uint2 u = __ldg(reinterpret_cast<const uint2 *>(vrow + c0 + q));
+                v[q] = u.x & 0xFFFFu; v[q + 1] = u.x >> 16; v[q + 2] = u.y & 0xFFFFu; v[q + 3] = u.y >> 16;
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < M; q += 2) {
+                const uint32_t u = __ldg(reinterpret_cast<const uint32_t *>(vrow + c0 + q));
+                v[q] = u & 0xFFFFu; v[q + 1] = u >> 16;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < MM; ++q) {
+            const int64_t c = c0 + q;
+            v[q] = (q < m && c < K) ? __ldg(vrow + c) : static_cast<uint16_t>(0);
+        }
+    }
+}
+
+// fused a2: the group's scores from its weights (zero past K); the values are
+// the weights themselves when V is W
+template <int M>
+__device__ __forceinline__ void load_group_fused(const ScoreSrc &src, int64_t row,
+                                                 const uint16_t *__restrict__ vrow, int64_t c0,
+                                                 int64_t K, int m_rt, float *s, uint16_t *v) {
+    constexpr int MM = M > 0 ? M : 16;
+    const int m = M > 0 ? M : m_rt;
+    const uint16_t *wrow = src.W + row * src.ldw;
+    uint16_t w[MM];
+    load_values<M>(wrow, c0, K, m, w);
+    if (M > 0 && M % 2 == 0 && src.H != nullptr && c0 + M <= K &&
+        (reinterpret_cast<uintptr_t>(src.H + c0) & 15u) == 0) {
+        // whole group: H in 16-byte pairs
+#pragma unroll
+        for (int q = 0; q < MM; q += 2) {
+            const double2 h = __ldg(reinterpret_cast<const double2 *>(src.H + c0 + q));
+            const double wa = bf16_to_f64(w[q]), wb = bf16_to_f64(w[q + 1]);
+            s[q] = __double2float_rn(__dmul_rn(__dadd_rn(h.x, src.eps), __dmul_rn(wa, wa)));
+            s[q + 1] = __double2float_rn(__dmul_rn(__dadd_rn(h.y, src.eps), __dmul_rn(wb, wb)));
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < MM; ++q)
+            s[q] = (q < m && c0 + q < K) ? fused_score(src.H, src.eps, c0 + q, w[q]) : 0.0f;
+    }
+    if (vrow == wrow) {
+#pragma unroll
+        for (int q = 0; q < MM; ++q) v[q] = w[q];
+    } else {
+        load_values<M>(vrow, c0, K, m, v);
+    }
+}
 
 template <int M>
 __device__ __forceinline__ void load_group(const float *__restrict__ srow,
@@ -347,9 +441,9 @@ struct PruneGPT {
 // row.  Warp w of block b owns groups [32 GPT (8b + w), + 32 GPT); in step i
 // lane l takes group 32 i + l of that range, so every load instruction of a
 // warp reads 32 consecutive groups and every step yields m whole mask words.
-template <int M>
+template <int M, bool FUSED>
 __global__ void __launch_bounds__(PRUNE_THREADS)
-    k_prune(const float *__restrict__ S, int64_t lds, const uint16_t *__restrict__ V, int64_t ldv,
+    k_prune(const ScoreSrc src, const uint16_t *__restrict__ V, int64_t ldv,
             int64_t K, int64_t G, int n, int m_rt, uint32_t *__restrict__ mask,
             uint16_t *__restrict__ vals, uint8_t *__restrict__ meta24) {
     constexpr int MM = M > 0 ? M : 16;
@@ -361,7 +455,6 @@ __global__ void __launch_bounds__(PRUNE_THREADS)
     const int64_t wg0 = (static_cast<int64_t>(blockIdx.x) * (PRUNE_THREADS / 32) + warp) * 32 * GPT;
     if (wg0 >= G) return;  // warp-uniform
     const int64_t mwords = (G * m + 31) / 32;
-    const float *srow = S + row * lds;
     const uint16_t *vrow = V + row * ldv;
     uint16_t *vout = vals + row * (G * n);
 
@@ -370,7 +463,10 @@ __global__ void __launch_bounds__(PRUNE_THREADS)
 #pragma unroll
     for (int i = 0; i < GPT; ++i) {
         const int64_t g = wg0 + i * 32 + lane;
-        if (g < G) load_group<M>(srow, vrow, g * m, K, m, s[i], v[i]);
+        if (g < G) {
+            if constexpr (FUSED) load_group_fused<M>(src, row, vrow, g * m, K, m, s[i], v[i]);
+            else load_group<M>(src.S + row * src.lds, vrow, g * m, K, m, s[i], v[i]);
+        }
     }
 #pragma unroll
     for (int i = 0; i < GPT; ++i) {
@@ -449,41 +545,30 @@ __device__ __forceinline__ void drop_two_of_4(const float (&s)[4], int &dlo, int
     dhi = d0 < d1 ? d1 : d0;
 }
 
-__global__ void __launch_bounds__(128, 8)
-    k_prune24(const float *__restrict__ S, int64_t lds, const uint16_t *__restrict__ V, int64_t ldv,
-              int64_t K, int64_t G, uint32_t *__restrict__ mask, uint16_t *__restrict__ vals,
-              uint8_t *__restrict__ meta24) {
-    const int64_t row = blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535;
-    const int64_t run = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const int64_t c0 = run * 32;
-    if (c0 >= K) return;
-    const int64_t mwords = (G * 4 + 31) / 32, mbytes = (G + 1) / 2;
-    const float *srow = S + row * lds + c0;
-    const uint16_t *vrow = V + row * ldv + c0;
-    float sc[32];
-    uint32_t vw[16];
+// 32 bf16 of a row from column c0 as 16 packed words, zero past K
+__device__ __forceinline__ void load_run32(const uint16_t *__restrict__ p, int64_t c0, int64_t K,
+                                           uint32_t (&w)[16]) {
     if (c0 + 32 <= K) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float4 f = __ldg(reinterpret_cast<const float4 *>(srow) + j);
-            sc[4 * j] = f.x; sc[4 * j + 1] = f.y; sc[4 * j + 2] = f.z; sc[4 * j + 3] = f.w;
-        }
-#pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(vrow) + j);
-            vw[4 * j] = u.x; vw[4 * j + 1] = u.y; vw[4 * j + 2] = u.z; vw[4 * j + 3] = u.w;
+            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p) + j);
+            w[4 * j] = u.x; w[4 * j + 1] = u.y; w[4 * j + 2] = u.z; w[4 * j + 3] = u.w;
         }
     } else {
-        // ragged end of the row: zero padding (score 0, value 0)
-#pragma unroll
-        for (int j = 0; j < 32; ++j) sc[j] = c0 + j < K ? __ldg(srow + j) : 0.0f;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-            const uint32_t lo = c0 + 2 * j < K ? __ldg(vrow + 2 * j) : 0u;
-            const uint32_t hi = c0 + 2 * j + 1 < K ? __ldg(vrow + 2 * j + 1) : 0u;
-            vw[j] = lo | (hi << 16);
+            const uint32_t lo = c0 + 2 * j < K ? __ldg(p + 2 * j) : 0u;
+            const uint32_t hi = c0 + 2 * j + 1 < K ? __ldg(p + 2 * j + 1) : 0u;
+            w[j] = lo | (hi << 16);
         }
     }
+}
+
+// select + compress + store one 32-column run (8 groups) of a row
+__device__ __forceinline__ void prune24_run(const float (&sc)[32], const uint32_t (&vw)[16], int64_t row,
+                                            int64_t run, int64_t G, uint32_t *__restrict__ mask,
+                                            uint16_t *__restrict__ vals, uint8_t *__restrict__ meta24) {
+    const int64_t mwords = (G * 4 + 31) / 32, mbytes = (G + 1) / 2;
     uint32_t mword = 0, nibs = 0, out[8];
 #pragma unroll
     for (int gi = 0; gi < 8; ++gi) {
@@ -501,7 +586,7 @@ __global__ void __launch_bounds__(128, 8)
         mword |= ((1u << i0) | (1u << i1)) << (4 * gi);
         nibs |= static_cast<uint32_t>(i0 | (i1 << 2)) << (4 * gi);
     }
-    const int64_t g0 = c0 / 4;          // first group of the run
+    const int64_t g0 = run * 8;  // first group of the run
     const int ng = G - g0 < 8 ? static_cast<int>(G - g0) : 8;
     uint16_t *vdst = vals + row * (G * 2) + g0 * 2;
     if (ng == 8 && ((reinterpret_cast<uintptr_t>(vdst) & 15u) == 0)) {
@@ -522,6 +607,95 @@ __global__ void __launch_bounds__(128, 8)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
             if (j < nb) mdst[j] = static_cast<uint8_t>(nibs >> (8 * j));
+    }
+}
+
+__global__ void __launch_bounds__(128, 8)
+    k_prune24(const ScoreSrc src, const uint16_t *__restrict__ V, int64_t ldv,
+              int64_t K, int64_t G, uint32_t *__restrict__ mask, uint16_t *__restrict__ vals,
+              uint8_t *__restrict__ meta24) {
+    const int64_t row = blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535;
+    const int64_t run = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t c0 = run * 32;
+    if (c0 >= K) return;
+    const uint16_t *vrow = V + row * ldv + c0;
+    const float *srow = src.S + row * src.lds + c0;
+    float sc[32];
+    uint32_t vw[16];
+    if (c0 + 32 <= K) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 f = __ldg(reinterpret_cast<const float4 *>(srow) + j);
+            sc[4 * j] = f.x; sc[4 * j + 1] = f.y; sc[4 * j + 2] = f.z; sc[4 * j + 3] = f.w;
+        }
+    } else {
+        // ragged end of the row: zero padding (score 0, value 0)
+#pragma unroll
+        for (int j = 0; j < 32; ++j) sc[j] = c0 + j < K ? __ldg(srow + j) : 0.0f;
+    }
+    load_run32(vrow, c0, K, vw);
+    prune24_run(sc, vw, row, run, G, mask, vals, meta24);
+}
+
+// 2:4 with a2 fused: the block's 4096 columns of H + eps are staged once in
+// shared memory, transposed so that lane t reading its j-th column hits
+// consecutive words ([j][t], 129-double pitch), and reused for P24F_ROWS rows;
+// each thread scores its 32-column run of W in registers.
+// grid: x = 4096-column slices (128 threads), y (+65535 z) = row blocks.
+constexpr int P24F_ROWS = 4;
+
+__global__ void __launch_bounds__(128, 4)
+    k_prune24_fused(const ScoreSrc src, const uint16_t *__restrict__ V, int64_t ldv, int64_t R,
+                    int64_t K, int64_t G, uint32_t *__restrict__ mask, uint16_t *__restrict__ vals,
+                    uint8_t *__restrict__ meta24) {
+    __shared__ double hs[32 * 129];
+    const int t = threadIdx.x;
+    const int64_t cbase = static_cast<int64_t>(blockIdx.x) * 4096;
+    const int64_t r0 = (blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535) * P24F_ROWS;
+    const bool hess = src.H != nullptr;
+    if (hess) {
+        for (int i = t; i < 4096; i += 128) {
+            const int64_t c = cbase + i;
+            hs[(i & 31) * 129 + (i >> 5)] = c < K ? __dadd_rn(__ldg(src.H + c), src.eps) : 0.0;
+        }
+        __syncthreads();
+    }
+    const int64_t run = cbase / 32 + t;
+    const int64_t c0 = run * 32;
+    if (c0 >= K) return;
+    // the next row's weights are loaded while this row is scored
+    uint32_t wnext[16];
+    load_run32(src.W + r0 * src.ldw + c0, c0, K, wnext);
+#pragma unroll 1
+    for (int rr = 0; rr < P24F_ROWS; ++rr) {
+        const int64_t row = r0 + rr;
+        if (row >= R) break;
+        const uint16_t *wrow = src.W + row * src.ldw + c0;
+        const uint16_t *vrow = V + row * ldv + c0;
+        uint32_t ww[16], vw[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) ww[j] = wnext[j];
+        if (rr + 1 < P24F_ROWS && row + 1 < R) load_run32(wrow + src.ldw, c0, K, wnext);
+        float sc[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const uint16_t wb = static_cast<uint16_t>(ww[j >> 1] >> (16 * (j & 1)));
+            if (c0 + j >= K) {
+                sc[j] = 0.0f;
+            } else if (hess) {
+                const double w = bf16_to_f64(wb);
+                sc[j] = __double2float_rn(__dmul_rn(hs[j * 129 + t], __dmul_rn(w, w)));
+            } else {
+                sc[j] = fabsf(bf16_to_f32(wb));
+            }
+        }
+        if (vrow == wrow) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) vw[j] = ww[j];
+        } else {
+            load_run32(vrow, c0, K, vw);
+        }
+        prune24_run(sc, vw, row, run, G, mask, vals, meta24);
     }
 }
 
@@ -862,6 +1036,47 @@ extern "C" nm_status nm_score(const uint16_t *X, int64_t T, int64_t ldx, const u
     return nm_score_from_hessian(H, eps, W, R, K, ldw, S, stream);
 }
 
+namespace {
+
+// a3 launch (FUSED: with a2 in registers), arguments already validated
+template <bool FUSED>
+nm_status launch_prune(const ScoreSrc &src, const uint16_t *V, int64_t ldv, int64_t R, int64_t K, int n,
+                       int m, uint32_t *mask, uint16_t *vals, uint8_t *meta24, cudaStream_t s) {
+    const int64_t G = (K + m - 1) / m;
+    uint8_t *meta = (m == 4 && n == 2) ? meta24 : nullptr;
+    auto grid_for = [&](int gpt) {
+        const int64_t per = static_cast<int64_t>(PRUNE_THREADS) * gpt;
+        return dim3(static_cast<unsigned>((G + per - 1) / per), static_cast<unsigned>(R < 65535 ? R : 65535),
+                    static_cast<unsigned>((R + 65534) / 65535));
+    };
+    switch (m) {
+        case 4:
+            if (n == 2 && !FUSED) {
+                const int64_t runs = (K + 31) / 32;
+                dim3 g24(static_cast<unsigned>((runs + 127) / 128), static_cast<unsigned>(R < 65535 ? R : 65535),
+                         static_cast<unsigned>((R + 65534) / 65535));
+                k_prune24<<<g24, 128, 0, s>>>(src, V, ldv, K, G, mask, vals, meta);
+                break;
+            }
+            if (n == 2 && FUSED) {
+                const int64_t rb = (R + P24F_ROWS - 1) / P24F_ROWS;
+                dim3 g24(static_cast<unsigned>((K + 4095) / 4096), static_cast<unsigned>(rb < 65535 ? rb : 65535),
+                         static_cast<unsigned>((rb + 65534) / 65535));
+                k_prune24_fused<<<g24, 128, 0, s>>>(src, V, ldv, R, K, G, mask, vals, meta);
+                break;
+            }
+            k_prune<4, FUSED><<<grid_for(PruneGPT<4>::value), PRUNE_THREADS, 0, s>>>(src, V, ldv, K, G, n, m, mask, vals, meta);
+            break;
+        case 6: k_prune<6, FUSED><<<grid_for(PruneGPT<6>::value), PRUNE_THREADS, 0, s>>>(src, V, ldv, K, G, n, m, mask, vals, meta); break;
+        case 8: k_prune<8, FUSED><<<grid_for(PruneGPT<8>::value), PRUNE_THREADS, 0, s>>>(src, V, ldv, K, G, n, m, mask, vals, meta); break;
+        case 10: k_prune<10, FUSED><<<grid_for(PruneGPT<10>::value), PRUNE_THREADS, 0, s>>>(src, V, ldv, K, G, n, m, mask, vals, meta); break;
+        default: k_prune<0, FUSED><<<grid_for(PruneGPT<0>::value), PRUNE_THREADS, 0, s>>>(src, V, ldv, K, G, n, m, mask, vals, meta); break;
+    }
+    return launch_status();
+}
+
+}  // namespace
+
 extern "C" nm_status nm_prune_compress(const float *S, int64_t lds, const uint16_t *V, int64_t ldv,
                                        int64_t R, int64_t K, int n, int m, uint32_t *mask,
                                        uint16_t *vals, uint8_t *meta24, void *stream) {
@@ -873,31 +1088,24 @@ extern "C" nm_status nm_prune_compress(const float *S, int64_t lds, const uint16
         (lds % 8) != 0 || (ldv % 8) != 0)
         return NM_ERR_ALIGN;
     if (R > 65535LL * 65535LL) return NM_ERR_SHAPE;
-    const int64_t G = (K + m - 1) / m;
-    cudaStream_t s = as_stream(stream);
-    uint8_t *meta = (m == 4 && n == 2) ? meta24 : nullptr;
-    auto grid_for = [&](int gpt) {
-        const int64_t per = static_cast<int64_t>(PRUNE_THREADS) * gpt;
-        return dim3(static_cast<unsigned>((G + per - 1) / per), static_cast<unsigned>(R < 65535 ? R : 65535),
-                    static_cast<unsigned>((R + 65534) / 65535));
-    };
-    switch (m) {
-        case 4:
-            if (n == 2) {
-                const int64_t runs = (K + 31) / 32;
-                dim3 g24(static_cast<unsigned>((runs + 127) / 128), static_cast<unsigned>(R < 65535 ? R : 65535),
-                         static_cast<unsigned>((R + 65534) / 65535));
-                k_prune24<<<g24, 128, 0, s>>>(S, lds, V, ldv, K, G, mask, vals, meta);
-                break;
-            }
-            k_prune<4><<<grid_for(PruneGPT<4>::value), PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta);
-            break;
-        case 6: k_prune<6><<<grid_for(PruneGPT<6>::value), PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
-        case 8: k_prune<8><<<grid_for(PruneGPT<8>::value), PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
-        case 10: k_prune<10><<<grid_for(PruneGPT<10>::value), PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
-        default: k_prune<0><<<grid_for(PruneGPT<0>::value), PRUNE_THREADS, 0, s>>>(S, lds, V, ldv, K, G, n, m, mask, vals, meta); break;
-    }
-    return launch_status();
+    const ScoreSrc src{S, lds, nullptr, 0, nullptr, 0.0};
+    return launch_prune<false>(src, V, ldv, R, K, n, m, mask, vals, meta24, as_stream(stream));
+}
+
+extern "C" nm_status nm_score_prune_compress(const double *H, double eps, const uint16_t *W, int64_t ldw,
+                                             const uint16_t *V, int64_t ldv, int64_t R, int64_t K, int n,
+                                             int m, uint32_t *mask, uint16_t *vals, uint8_t *meta24,
+                                             void *stream) {
+    if (!W || !V || !mask || !vals) return NM_ERR_NULL;
+    if (m == 4 && n == 2 && !meta24) return NM_ERR_NULL;
+    if (R < 1 || K < 1 || ldw < K || ldv < K) return NM_ERR_SHAPE;
+    if (m < 2 || m > 16 || n < 1 || n >= m) return NM_ERR_UNSUPPORTED;
+    if (!aligned16(W) || !aligned16(V) || !aligned16(vals) || !aligned16(mask) || (ldw % 8) != 0 ||
+        (ldv % 8) != 0 || (H && (reinterpret_cast<uintptr_t>(H) & 7u)))
+        return NM_ERR_ALIGN;
+    if (R > 65535LL * 65535LL) return NM_ERR_SHAPE;
+    const ScoreSrc src{nullptr, 0, W, ldw, H, eps};
+    return launch_prune<true>(src, V, ldv, R, K, n, m, mask, vals, meta24, as_stream(stream));
 }
 
 extern "C" nm_status slide_pack(const uint32_t *mask, int64_t R, int64_t K, int m, uint8_t *wmeta,

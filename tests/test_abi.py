@@ -80,6 +80,12 @@ MIS = 0x10002
     (lambda l: l.nm_prune_compress(A, 8, A, 8, 4, 8, 4, 4, A, A, A, None), 4),
     (lambda l: l.nm_prune_compress(A, 8, A, 8, 4, 8, 2, 4, A, A, None, None), 1),
     (lambda l: l.nm_prune_compress(A, 8, MIS, 8, 4, 8, 2, 4, A, A, A, None), 3),
+    (lambda l: l.nm_score_prune_compress(None, 0.0, None, 8, A, 8, 4, 8, 2, 4, A, A, A, None), 1),
+    (lambda l: l.nm_score_prune_compress(None, 0.0, A, 8, A, 8, 4, 8, 2, 4, A, A, None, None), 1),
+    (lambda l: l.nm_score_prune_compress(None, 0.0, A, 8, A, 8, 4, 8, 2, 17, A, A, A, None), 4),
+    (lambda l: l.nm_score_prune_compress(None, 0.0, A, 4, A, 8, 4, 8, 2, 4, A, A, A, None), 2),
+    (lambda l: l.nm_score_prune_compress(None, 0.0, MIS, 8, A, 8, 4, 8, 2, 4, A, A, A, None), 3),
+    (lambda l: l.nm_score_prune_compress(A + 4, 0.0, A, 8, A, 8, 4, 8, 2, 4, A, A, A, None), 3),
     (lambda l: l.slide_pack(A, 4, 8, 7, A, None), 4),
     (lambda l: l.slide_pack(A, 4, 8, 12, A, None), 4),
     (lambda l: l.lift_activations(A, 4, 8, 8, 5, A, 8, None), 4),

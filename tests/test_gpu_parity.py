@@ -77,6 +77,41 @@ def test_prune_bitexact(nm, n, m, R, K, kind):
 
 
 # ---------------------------------------------------------------- a4 / a5
+# a2 + a3 fused (scores in registers, never written): the oracle's mask, values
+# and 2:4 metadata, and bit-identical to the two-call path on the GPU
+@pytest.mark.parametrize("n,m,R,K", [(2, 4, 64, 512), (2, 4, 33, 1030), (6, 8, 33, 1030), (4, 6, 17, 1003),
+                                     (8, 10, 9, 207), (2, 4, 3, 9), (1, 4, 8, 64), (3, 4, 8, 60),
+                                     (2, 8, 5, 100), (5, 16, 4, 99), (6, 8, 128, 4096)])
+@pytest.mark.parametrize("mode", ["hessian", "magnitude", "ternary_values", "ties"])
+def test_score_prune_fused_bitexact(nm, n, m, R, K, mode):
+    ld = (K + 7) // 8 * 8
+    X = datagen.make_activations(77, K, seed=R + K, n_outliers=2)
+    if mode == "ties":
+        # small integers: many equal |w| and equal products
+        W = datagen.small_int_bf16((R, K), seed=R, tensor_id=5)
+    else:
+        W = datagen.make_weight(R, K, 0.02, seed=R + 1)
+    score = "magnitude" if mode in ("magnitude", "ternary_values") else "hessian"
+    ref = oracle.run_layer(X, W, n, m, eps=1e-8, score=score, ternary_values=(mode == "ternary_values"))
+    Wd = to_dev(W, ld)
+    Vd = to_dev(ref["V"], ld) if mode == "ternary_values" else None
+    H = nm.hessian_diag(to_dev(X, ld)) if score == "hessian" else None
+    mask, vals, meta = nm.score_prune_compress(H, Wd, n, m, V=Vd, eps=1e-8)
+    # the two-call path on the same device inputs
+    _, S = nm.score(to_dev(X, ld) if score == "hessian" else None, Wd, eps=1e-8)
+    Sp = torch.zeros((R, ld), dtype=torch.float32, device="cuda")
+    Sp[:, :K] = S                                   # prune wants a row stride % 8 == 0
+    mask2, vals2, meta2 = nm.prune_compress(Sp[:, :K], Vd if Vd is not None else Wd, n, m)
+    _sync_ok(nm)
+    assert np.array_equal(to_host(mask).view(np.uint32), ref["mask"])
+    assert np.array_equal(to_host_u16(vals), ref["vals"])
+    assert np.array_equal(to_host(mask), to_host(mask2))
+    assert np.array_equal(to_host_u16(vals), to_host_u16(vals2))
+    if m == 4 and n == 2:
+        assert np.array_equal(to_host(meta), ref["meta24"])
+        assert np.array_equal(to_host(meta), to_host(meta2))
+
+
 @pytest.mark.parametrize("m,R,K", [(4, 64, 512), (6, 20, 1003), (8, 33, 1030), (10, 9, 207),
                                    (8, 4, 8), (6, 128, 4096), (10, 7, 8195)])
 def test_slide_pack_bitexact(nm, m, R, K):
