@@ -499,6 +499,77 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_prep(args):
+    """The HBM-bound prep kernels of one workload's W, each launched alone and
+    timed with CUDA events (L2 flushed): score, prune and fused score + prune
+    (2:4, 6:8 and the workload's pattern), ternary quantisation.  One JSON
+    line.  With --reps 0 every kernel is launched once (the ncu driver)."""
+    import torch
+
+    import semi_structured_sparse_diag_b200 as nm
+    lib = nm.load()
+    dev = torch.device("cuda", 0)
+    layer = datagen.WORKLOADS[args.workload]
+    X_h, W_h = datagen.layer_inputs(layer)
+    R, K = layer.R, layer.K
+    W = torch.from_numpy(W_h.view(np.int16)).to(dev).view(torch.bfloat16)
+    X = torch.from_numpy(X_h.view(np.int16)).to(dev).view(torch.bfloat16)
+    H = nm.hessian_diag(X)
+    S = torch.empty((R, K), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    s = torch.cuda.current_stream().cuda_stream
+
+    def chk(st, what):
+        if st != 0:
+            raise nm.NMError(f"{what}: {lib.nm_status_string(st).decode()}")
+
+    def timed(fn):
+        ts = []
+        for i in range(args.reps + 1):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if i:
+                ts.append(e0.elapsed_time(e1) * 1000)
+        return sorted(ts)[len(ts) // 2] if ts else float("nan")
+
+    out = {"prep": layer.name, "R": R, "K": K, "us": {}, "GBs": {}}
+
+    def rec(name, us, nbytes):
+        if us == us:  # not NaN (--reps 0: launches only, for ncu)
+            out["us"][name] = round(us, 1)
+            out["GBs"][name] = round(nbytes / us / 1e3, 0)
+
+    E = R * K
+    rec("score", timed(lambda: chk(lib.nm_score_from_hessian(H.data_ptr(), layer.eps, W.data_ptr(), R, K, K,
+                                                             S.data_ptr(), s), "score")), 6 * E)
+    for m in sorted({4, 8, layer.m}):
+        n = m - 2
+        G = (K + m - 1) // m
+        mask = torch.empty((R, (G * m + 31) // 32), dtype=torch.int32, device=dev)
+        vals = torch.empty((R, G * n), dtype=torch.bfloat16, device=dev)
+        meta = torch.empty((R, (G + 1) // 2), dtype=torch.uint8, device=dev)
+        mp = meta.data_ptr() if m == 4 else None
+        wr = R * G * n * 2 + mask.numel() * 4 + (meta.numel() if m == 4 else 0)
+        rec(f"prune_{n}of{m}", timed(lambda: chk(lib.nm_prune_compress(
+            S.data_ptr(), K, W.data_ptr(), K, R, K, n, m, mask.data_ptr(), vals.data_ptr(), mp, s), "prune")),
+            6 * E + wr)
+        rec(f"score_prune_{n}of{m}", timed(lambda: chk(lib.nm_score_prune_compress(
+            H.data_ptr(), layer.eps, W.data_ptr(), K, W.data_ptr(), K, R, K, n, m, mask.data_ptr(),
+            vals.data_ptr(), mp, s), "score_prune")), 2 * E + wr)
+    Wq = torch.empty((R, K), dtype=torch.bfloat16, device=dev)
+    gamma = torch.empty(1, dtype=torch.float64, device=dev)
+    tws = torch.empty(lib.nm_ternary_workspace_bytes(R), dtype=torch.uint8, device=dev)
+    rec("ternary_quantize", timed(lambda: chk(lib.nm_ternary_quantize(
+        W.data_ptr(), R, K, K, Wq.data_ptr(), gamma.data_ptr(), tws.data_ptr(), tws.numel(), s), "ternary")),
+        6 * E)
+    nm.check_device_error()
+    print(json.dumps(out), flush=True)
+
+
 def run_probe(args):
     """Tensor-pipe and HBM probes (calibration, not the bench line)."""
     import torch
@@ -640,7 +711,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--probe", action="store_true", help="run the tensor-pipe / HBM probes instead")
     ap.add_argument("--ablation", action="store_true", help="time the GEMM variants instead")
+    ap.add_argument("--prep", action="store_true", help="time the HBM-bound prep kernels instead")
+    ap.add_argument("--reps", type=int, default=5, help="--prep: timed launches per kernel")
     args = ap.parse_args()
+    if args.prep:
+        return run_prep(args)
     if args.probe:
         run_probe(args)
         return
