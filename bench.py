@@ -544,6 +544,17 @@ def run_prep(args):
             out["GBs"][name] = round(nbytes / us / 1e3, 0)
 
     E = R * K
+    T = X.shape[0]
+    Hb = torch.empty(K, dtype=torch.float64, device=dev)
+    hws = torch.empty(max(lib.nm_hessian_workspace_bytes(T, K), 16), dtype=torch.uint8, device=dev)
+    rec("hessian_diag", timed(lambda: chk(lib.nm_hessian_diag(X.data_ptr(), T, K, K, Hb.data_ptr(), hws.data_ptr(),
+                                                             hws.numel(), s), "hessian")), 2 * T * K + 8 * K)
+    # Hutchinson with 16 sign vectors: X is read twice (u = X z, then x * p)
+    zb = torch.from_numpy(datagen.rademacher_bits(16, K, seed=0).view(np.int32)).to(dev)
+    uws = torch.empty(lib.nm_hutchinson_workspace_bytes(T, K, 16), dtype=torch.uint8, device=dev)
+    rec("hutchinson_S16", timed(lambda: chk(lib.nm_hutchinson_diag(
+        X.data_ptr(), T, K, K, zb.data_ptr(), 16, Hb.data_ptr(), uws.data_ptr(), uws.numel(), s), "hutchinson")),
+        4 * T * K + 8 * K)
     rec("score", timed(lambda: chk(lib.nm_score_from_hessian(H.data_ptr(), layer.eps, W.data_ptr(), R, K, K,
                                                              S.data_ptr(), s), "score")), 6 * E)
     for m in sorted({4, 8, layer.m}):

@@ -84,6 +84,18 @@ def tie_heavy_scores(R: int, K: int, seed: int, levels: int = 8) -> np.ndarray:
     return g.integers(0, levels, size=(R, K)).astype(np.float32)
 
 
+def rademacher_bits(S: int, K: int, seed: int) -> np.ndarray:
+    """S random sign vectors of length K as bits: uint32 [S x ceil(K/32)], bit
+    k % 32 of word k / 32 set = -1, clear = +1 (bits past K are clear)."""
+    g = _rng(seed, 23)
+    signs = g.integers(0, 2, size=(S, K), dtype=np.uint8)
+    words = np.zeros((S, (K + 31) // 32), dtype=np.uint32)
+    for b in range(32):
+        col = signs[:, b::32].astype(np.uint32)
+        words[:, : col.shape[1]] |= col << np.uint32(b)
+    return words
+
+
 def small_int_bf16(shape, seed: int, tensor_id: int, lo: int = -4, hi: int = 5) -> np.ndarray:
     """Small integers stored as bf16 bits (exact), so fp64 sums of products are exact."""
     g = _rng(seed, tensor_id)

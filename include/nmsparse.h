@@ -7,6 +7,10 @@
  *                     the input activations. Sparsity Induction for Accurate
  *                     Post-Training Pruning of LLMs (arXiv 2602.21652), sec. 2C
  *                     "Efficientie: Snelle Hessian Update".
+ *   nm_hessian_rescale  H / s^2 under equivalent scaling: the O(d_in) score
+ *                     refresh of Sparsity Induction sec. 2C.
+ *   nm_hutchinson_diag  Rademacher estimate of diag(X^T X / T), SparseForge,
+ *                     "Estimativa de Importancia Consciente do Hessiano".
  *   nm_score          s = (H + eps) * W^2. SparseForge (arXiv 2605.06402),
  *                     "Estimativa de Importancia Consciente do Hessiano".
  *                     With X == NULL: s = |W_latent|, Sparse-BitNet (arXiv
@@ -92,8 +96,9 @@ int nm_version(void);
 /* ------------------------------------------------------------------------ */
 /* a1: diagonal Gauss-Newton proxy (Sparsity Induction, sec. 2C).
  *   H[j] = (1/T) * sum_t X[t,j]^2 in fp64, summed in a fixed order: tokens in
- *   chunks of 128 (each chunk in ascending t), chunk partials in ascending
- *   chunk order, one correctly rounded division by T.  The result is therefore
+ *   chunks of 128; a chunk is runs of 16 tokens, each run summed in ascending
+ *   t, the runs added in ascending order; chunk partials added in ascending
+ *   chunk order; one correctly rounded division by T.  The result is therefore
  *   bit-identical run to run and to any implementation of that order.
  *   X  : [T x K] bf16, ldx >= K.          H : [K] fp64 (output).
  *   ws : scratch of nm_hessian_workspace_bytes(T, K) bytes (may be NULL when
@@ -159,6 +164,37 @@ nm_status nm_score_from_hessian(const double *H, double eps, const uint16_t *W, 
 nm_status nm_prune_compress(const float *S, int64_t lds, const uint16_t *V, int64_t ldv,
                             int64_t R, int64_t K, int n, int m, uint32_t *mask, uint16_t *vals,
                             uint8_t *meta24, void *stream);
+
+/* O(d_in) score refresh (Sparsity Induction sec. 2C "Snelle Hessian Update"):
+ * under the equivalent per-channel scaling W' = W diag(s), X' = X diag(1/s)
+ * the proxy of X' is H'_j = H_j / (s_j * s_j) (fp64: one multiply, one
+ * division), so the scores of W' follow from nm_score_from_hessian(H', ...)
+ * without re-reading X.  H, s, H_out: [K] fp64, 8-byte aligned; H_out may be
+ * H itself.                                                                 */
+nm_status nm_hessian_rescale(const double *H, const double *s, int64_t K, double *H_out, void *stream);
+
+/* Hutchinson's stochastic estimate of diag(A), A = X^T X / T, from S
+ * Rademacher vectors z_s (SparseForge, arXiv 2605.06402, "Estimativa de
+ * Importancia Consciente do Hessiano"; the vectors are inputs, drawn by the
+ * caller):   D_k = (1/S) sum_s z_s[k] (X^T (X z_s))[k] / T.
+ * Its expectation is H_k of nm_hessian_diag; the error falls as 1/sqrt(S).
+ *   X     : bf16 [T x ldx] row-major, 16-byte aligned, ldx % 8 == 0, ldx >= K.
+ *   zbits : uint32 [S x ceil(K/32)], 4-byte aligned; bit k % 32 of word k / 32
+ *           of row s set = z_s[k] = -1, clear = +1.  1 <= S <= 256.
+ *   D     : fp64 [K] (written), 8-byte aligned.
+ *   ws    : nm_hutchinson_workspace_bytes(T, K, S) bytes, 16-byte aligned,
+ *           owned by the caller (u = X z_s in fp32, then per-128-token fp64
+ *           partials of D).
+ * Arithmetic: u[t,s] in fp32 (lane-strided sums, then a shuffle tree);
+ * p[t,k] = sum_s z_s[k] u[t,s] in fp32, s ascending; x[t,k] * p[t,k] rounded
+ * to fp32 and added in fp64 over each 128-token chunk, chunks in ascending
+ * order, then one multiply by 1/(S T).  Deterministic run to run.
+ * Errors: NULL -> NM_ERR_NULL; S outside [1, 256], T or K < 1, ldx < K, a
+ * row of X above 227 KiB (K > 116224) or T above 65535 * 128 -> NM_ERR_SHAPE;
+ * alignment -> NM_ERR_ALIGN; short workspace -> NM_ERR_WORKSPACE.           */
+size_t nm_hutchinson_workspace_bytes(int64_t T, int64_t K, int64_t S);
+nm_status nm_hutchinson_diag(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, const uint32_t *zbits,
+                             int64_t S, double *D, void *ws, size_t ws_bytes, void *stream);
 
 /* a2 + a3 fused: exactly nm_score_from_hessian followed by nm_prune_compress
  * (bit-identical mask, vals and meta24), with each score formed in registers

@@ -8,6 +8,8 @@ file, marshals numpy arrays into it and shapes the outputs.
 
 Function -> passage it follows (page title, section):
   hessian_diag     Sparsity Induction (2602.21652) sec. 2C, diagonal GN proxy
+  hessian_rescale  Sparsity Induction sec. 2C, O(d_in) refresh under equivalent scaling
+  hutchinson_diag  Hutchinson estimate of diag(X^T X / T) from given sign vectors
   score_hessian    SparseForge (2605.06402), Hessian-aware importance s=(H+eps)W^2
   score_magnitude  Sparse-BitNet (2603.05168) sec. 2, mask from latent magnitudes
   prune            SparseForge "Mistura Progressiva" (top-N per group);
@@ -35,7 +37,8 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 _lock = threading.Lock()
 _lib = None
 
-H_CHUNK = 128
+H_CHUNK = 128   # tokens per chunk partial of H
+H_RUN = 16      # tokens per sequential run inside a chunk
 
 
 def build(force: bool = False) -> str:
@@ -58,6 +61,8 @@ def _load():
             P, I64, I, D = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double
             sig = {
                 "oracle_hessian_diag": (None, [P, I64, I64, I64, P]),
+                "oracle_hessian_rescale": (None, [P, P, I64, P]),
+                "oracle_hutchinson_diag": (None, [P, I64, I64, I64, P, I64, P]),
                 "oracle_hessian_diag_naive": (None, [P, I64, I64, I64, P]),
                 "oracle_score_hessian": (None, [P, D, P, I64, I64, I64, P]),
                 "oracle_score_magnitude": (None, [P, I64, I64, I64, P]),
@@ -107,6 +112,25 @@ def hessian_diag(X: np.ndarray, naive: bool = False) -> np.ndarray:
     fn = _load().oracle_hessian_diag_naive if naive else _load().oracle_hessian_diag
     fn(_p(X), T, K, K, _p(H))
     return H
+
+
+def hessian_rescale(H: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """H_j / (s_j * s_j): the proxy of X diag(1/s) (Sparsity Induction sec. 2C)."""
+    H = _c(H, np.float64)
+    s = _c(s, np.float64)
+    out = np.empty_like(H)
+    _load().oracle_hessian_rescale(_p(H), _p(s), H.shape[0], _p(out))
+    return out
+
+
+def hutchinson_diag(X: np.ndarray, zbits: np.ndarray) -> np.ndarray:
+    """(1/S) sum_s z_s * (X^T X z_s) / T in fp64, z_s = -1 where a bit is set."""
+    X = _c(X, np.uint16)
+    zbits = _c(zbits, np.uint32)
+    T, K = X.shape
+    D = np.empty(K, dtype=np.float64)
+    _load().oracle_hutchinson_diag(_p(X), T, K, K, _p(zbits), zbits.shape[0], _p(D))
+    return D
 
 
 def score_hessian(H: np.ndarray, W: np.ndarray, eps: float) -> np.ndarray:

@@ -23,7 +23,8 @@
  *
  * Readings of points the pages leave open (each also listed in the design
  * notes): mean (1/T) with no factor 2 for H; H summed in a canonical order
- * (chunks of 128 tokens, each summed in ascending t, chunk partials summed in
+ * (chunks of 128 tokens; a chunk is runs of 16 tokens, each run summed in
+ * ascending t, the runs added in ascending order; chunk partials summed in
  * ascending chunk order); S rounded once from fp64 to fp32; groups run along
  * the input (K) dimension; ties go to the lower index; a ragged tail group is
  * zero-padded (score 0, value 0); survivor k of a group goes to window k/2.
@@ -37,6 +38,7 @@
 #include <string.h>
 
 #define ORACLE_H_CHUNK 128
+#define ORACLE_H_RUN 16
 
 /* bf16 bit pattern -> fp64 (exact: bf16 is the top half of an fp32). */
 static double bf16_to_f64(uint16_t b) {
@@ -86,15 +88,63 @@ void oracle_hessian_diag(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, d
         for (int64_t c0 = 0; c0 < T; c0 += ORACLE_H_CHUNK) {
             int64_t c1 = c0 + ORACLE_H_CHUNK < T ? c0 + ORACLE_H_CHUNK : T;
             double part = 0.0;
-            for (int64_t t = c0; t < c1; ++t) {
-                double x = bf16_to_f64(X[t * ldx + j]);
-                double sq = x * x;
-                part = part + sq;
+            for (int64_t r0 = c0; r0 < c1; r0 += ORACLE_H_RUN) {
+                int64_t r1 = r0 + ORACLE_H_RUN < c1 ? r0 + ORACLE_H_RUN : c1;
+                double run = 0.0;
+                for (int64_t t = r0; t < r1; ++t) {
+                    double x = bf16_to_f64(X[t * ldx + j]);
+                    double sq = x * x;
+                    run = run + sq;
+                }
+                part = part + run;
             }
             total = total + part;
         }
         H[j] = total / (double)T;
     }
+}
+
+/* O(d_in) refresh of H under per-channel equivalent scaling (Sparsity
+ * Induction, sec. 2C "Snelle Hessian Update"): with W' = W diag(s) and
+ * X' = X diag(1/s) the product is unchanged and the proxy of X' is
+ *   H'_j = H_j / (s_j * s_j)     (fp64: one multiply, one division),
+ * so the scores of W' are refreshed without re-reading X.                  */
+void oracle_hessian_rescale(const double *H, const double *s, int64_t K, double *out) {
+    for (int64_t j = 0; j < K; ++j) out[j] = H[j] / (s[j] * s[j]);
+}
+
+/* Hutchinson's stochastic estimate of diag(A), A = X^T X / T (the Gram
+ * matrix whose diagonal is H), the Rademacher-vector estimator of SparseForge
+ * (arXiv 2605.06402), "Estimativa de Importancia Consciente do Hessiano":
+ *   D_k = (1/S) sum_s z_s[k] (A z_s)[k],   z_s in {-1, +1}^K
+ * with A z = X^T (X z) / T.  Sign s of column k: bit k % 32 of word k / 32
+ * of row s of zbits set = -1.  Plain fp64 loops.                           */
+void oracle_hutchinson_diag(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, const uint32_t *zbits,
+                            int64_t S, double *D) {
+    const int64_t words = (K + 31) / 32;
+    double *u = (double *)malloc((size_t)T * sizeof(double));
+    for (int64_t k = 0; k < K; ++k) D[k] = 0.0;
+    for (int64_t s = 0; s < S; ++s) {
+        const uint32_t *zs = zbits + s * words;
+        #pragma omp parallel for schedule(static)
+        for (int64_t t = 0; t < T; ++t) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < K; ++j) {
+                const double x = bf16_to_f64(X[t * ldx + j]);
+                acc = acc + (((zs[j >> 5] >> (j & 31)) & 1u) ? -x : x);
+            }
+            u[t] = acc;
+        }
+        #pragma omp parallel for schedule(static)
+        for (int64_t k = 0; k < K; ++k) {
+            double v = 0.0;
+            for (int64_t t = 0; t < T; ++t) v = v + bf16_to_f64(X[t * ldx + k]) * u[t];
+            const double z = ((zs[k >> 5] >> (k & 31)) & 1u) ? -1.0 : 1.0;
+            D[k] = D[k] + z * (v / (double)T);
+        }
+    }
+    for (int64_t k = 0; k < K; ++k) D[k] = D[k] / (double)S;
+    free(u);
 }
 
 /* Same quantity, one sequential sum over all tokens (diagnostic only). */

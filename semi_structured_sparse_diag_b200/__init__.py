@@ -20,7 +20,7 @@ from . import build as _build
 
 __all__ = [
     "NMError", "load", "hessian_diag", "score", "score_from_hessian", "prune_compress",
-    "score_prune_compress", "slide_pack", "lift_activations", "sparse_prepare", "sparse_gemm", "dense_gemm",
+    "score_prune_compress", "hessian_rescale", "hutchinson_diag", "slide_pack", "lift_activations", "sparse_prepare", "sparse_gemm", "dense_gemm",
     "ternary_quantize", "check_device_error", "set_gemm_schedule", "EXPORTED",
 ]
 
@@ -31,7 +31,8 @@ EXPORTED = (
     "nm_sparse_prepare", "nm_sparse_gemm", "nm_dense_gemm", "nm_ternary_workspace_bytes",
     "nm_ternary_quantize", "nm_hessian_diag_noalloc", "nm_probe_mma", "nm_probe_copy", "nm_gemm_1cta", "nm_sparse_gemm_workspace_bytes",
     "nm_sparse_gemm_fused", "nm_dense_gemm_workspace_bytes", "nm_gemm_set_schedule",
-    "nm_sparse_gemm_tile256", "nm_score_prune_compress",
+    "nm_sparse_gemm_tile256", "nm_score_prune_compress", "nm_hessian_rescale",
+    "nm_hutchinson_workspace_bytes", "nm_hutchinson_diag",
 )
 
 _P, _I64, _I, _D, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_size_t
@@ -44,6 +45,9 @@ _SIGS = {
     "nm_score": (_I, [_P, _I64, _I64, _P, _I64, _I64, _I64, _D, _P, _P, _P, _SZ, _P]),
     "nm_score_from_hessian": (_I, [_P, _D, _P, _I64, _I64, _I64, _P, _P]),
     "nm_prune_compress": (_I, [_P, _I64, _P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P]),
+    "nm_hessian_rescale": (_I, [_P, _P, _I64, _P, _P]),
+    "nm_hutchinson_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
+    "nm_hutchinson_diag": (_I, [_P, _I64, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
     "nm_score_prune_compress": (_I, [_P, _D, _P, _I64, _P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P]),
     "slide_pack": (_I, [_P, _I64, _I64, _I, _P, _P]),
     "lift_activations": (_I, [_P, _I64, _I64, _I64, _I, _P, _I64, _P]),
@@ -197,6 +201,37 @@ def prune_compress(S, V, n, m, K=None, stream=None):
     _check(load().nm_prune_compress(_ptr(S), S.stride(0), _ptr(V), _ld(V), R, K, n, m, _ptr(mask),
                                     _ptr(vals), _ptr(meta), _stream(stream)), "nm_prune_compress")
     return mask, vals, meta
+
+
+def hessian_rescale(H, s, out=None, stream=None):
+    """H / s^2 per channel (fp64), the O(d_in) refresh under equivalent scaling."""
+    _dev(H, "H")
+    _dev(s, "s")
+    out = torch.empty_like(H) if out is None else out
+    _check(load().nm_hessian_rescale(_ptr(H), _ptr(s), H.shape[0], _ptr(out), _stream(stream)),
+           "nm_hessian_rescale")
+    return out
+
+
+def hutchinson_diag(X, zbits, D=None, ws=None, stream=None):
+    """Hutchinson estimate of diag(X^T X / T): X bf16 [T x K], zbits int32 /
+    uint32 [S x ceil(K/32)] sign bits (set = -1).  Returns fp64 [K]."""
+    X = _bf16(X, "X")
+    _dev(zbits, "zbits")
+    T, K = X.shape
+    S = zbits.shape[0]
+    if zbits.dim() != 2 or zbits.shape[1] != (K + 31) // 32 or zbits.element_size() != 4 \
+            or not zbits.is_contiguous():
+        raise NMError(f"zbits must be contiguous 32-bit words [S x {(K + 31) // 32}]")
+    lib = load()
+    need = lib.nm_hutchinson_workspace_bytes(T, K, S)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=X.device)
+    if D is None:
+        D = torch.empty(K, dtype=torch.float64, device=X.device)
+    _check(lib.nm_hutchinson_diag(_ptr(X), T, K, _ld(X), _ptr(zbits), S, _ptr(D), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream)), "nm_hutchinson_diag")
+    return D
 
 
 def score_prune_compress(H, W, n, m, V=None, eps=1e-8, stream=None):

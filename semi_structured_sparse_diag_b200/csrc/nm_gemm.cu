@@ -21,6 +21,7 @@
 #include <mutex>
 
 #include "nm_common.cuh"
+#include "nm_host.cuh"
 
 namespace nm {
 
@@ -1457,48 +1458,6 @@ using namespace nm;
 
 namespace {
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
-// 2-D tensor map over a row-major [rows x cols] matrix with row stride ld (elements)
-bool make_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, int esize, const void *base,
-                  int64_t rows, int64_t cols, int64_t ld, uint32_t box_cols, uint32_t box_rows,
-                  bool swizzle128) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * esize};
-    cuuint32_t box[2] = {box_cols, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-bool make_tmap_bf16(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, int64_t ld,
-                    uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
-    return make_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, rows, cols, ld, box_cols,
-                        box_rows, swizzle128);
-}
-
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int sm_count() {
@@ -1516,19 +1475,6 @@ int sm_count() {
 
 // one flag per kernel instantiation and device (kernels of different modes
 // share a signature, so the cache is keyed on the kernel itself)
-template <auto kernel>
-bool set_smem_attr(int bytes) {
-    static bool done[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-    if (!done[dev]) {
-        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
-            cudaSuccess)
-            return false;
-        done[dev] = true;
-    }
-    return true;
-}
 
 // ---- single-CTA kernel (ablation baseline)
 constexpr int GEMM_BN = 128;

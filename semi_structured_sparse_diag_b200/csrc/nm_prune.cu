@@ -3,7 +3,8 @@
 // All of these are HBM-streaming kernels: each reads its operand once with
 // coalesced vector loads and writes its outputs once.  Bit-exact by
 // construction with any implementation of the same definitions:
-//   * H uses a fixed summation order (chunks of 128 tokens);
+//   * H uses a fixed summation order (chunks of 128 tokens, each the ordered
+//     sum of eight sequential 16-token runs);
 //   * S uses fp64 add/multiply with explicit round-to-nearest intrinsics (no
 //     FMA contraction) and one fp64 -> fp32 rounding;
 //   * selection is integer logic on fp32 comparisons.
@@ -13,13 +14,17 @@
 #include <mutex>
 
 #include "nm_common.cuh"
+#include "nm_host.cuh"
 
 namespace nm {
 
-constexpr int H_CHUNK = 128;   // tokens per partial sum of H
-constexpr int H_COLS = 2;      // columns per thread in the H reduction
-constexpr int H_THREADS = 256;
-constexpr int H_UNROLL = 16;
+constexpr int H_CHUNK = 128;                  // tokens per chunk partial of H
+constexpr int H_SLICE = 16;                   // tokens per sequential run inside a chunk
+constexpr int H_SLICES = H_CHUNK / H_SLICE;   // 8 runs, one half-warp each
+constexpr int H_VEC = 8;                      // columns per thread: one 16-byte load per token
+constexpr int H_GROUPS = 16;                  // column groups per block (a half-warp's lanes)
+constexpr int H_BLOCK_COLS = H_GROUPS * H_VEC;     // 128 columns per block
+constexpr int H_THREADS = H_GROUPS * H_SLICES;     // 128
 
 __device__ __forceinline__ double bf16_to_f64(uint16_t b) {
     return static_cast<double>(__uint_as_float(static_cast<uint32_t>(b) << 16));
@@ -29,66 +34,127 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t b) {
 }
 
 // ---------------------------------------------------------------------------
-// a1: column sums of squares, one partial per chunk of 128 tokens.
-//   grid.x: column blocks of H_THREADS*H_COLS columns; grid.y: token chunk.
-//   When there is a single chunk the kernel writes H directly.
+// a1: column sums of squares.  A block owns 128 columns and a strided set of
+// 128-token chunks (chunks y, y + gridDim.y, ...).  Each chunk tile
+// [128 tokens x 128 columns] bf16 (32 KB) is brought into shared memory by
+// TMA, three tiles in flight, so that the loads of later chunks overlap the
+// arithmetic on the current one (two blocks per SM).  In a tile, lane g of
+// half-warp r owns columns 8g..8g+7 and tokens 16r..16r+15 and adds x^2 per
+// column in ascending t.  The eight 16-token runs are added in ascending
+// order through shared memory, giving the chunk partial; with a single chunk
+// the kernel writes H directly.  Rows past T and columns past K arrive as
+// zeros from the tensor map, and adding +0.0 leaves a sum of squares as it is.
+//
+// x^2 of a bf16 value is exact in fp64, so fma(x, x, acc) rounds exactly like
+// acc + x*x.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(H_THREADS) k_colsumsq_chunk(const uint16_t *__restrict__ X,
-                                                              int64_t T, int64_t K, int64_t ldx,
-                                                              double *__restrict__ out,
-                                                              int direct) {
-    const int64_t col = (static_cast<int64_t>(blockIdx.x) * H_THREADS + threadIdx.x) * H_COLS;
-    if (col >= K) return;
-    const int64_t t0 = static_cast<int64_t>(blockIdx.y) * H_CHUNK;
-    const int64_t t1 = t0 + H_CHUNK < T ? t0 + H_CHUNK : T;
-    double p0 = 0.0, p1 = 0.0;
-    const uint16_t *base = X + t0 * ldx + col;
-    if (col + 1 < K) {
-        int64_t t = t0;
-        for (; t + H_UNROLL <= t1; t += H_UNROLL) {
-            uint32_t v[H_UNROLL];
-#pragma unroll
-            for (int u = 0; u < H_UNROLL; ++u)
-                v[u] = __ldg(reinterpret_cast<const uint32_t *>(base + (t - t0 + u) * ldx));
-#pragma unroll
-            for (int u = 0; u < H_UNROLL; ++u) {
-                const double a = bf16_to_f64(static_cast<uint16_t>(v[u] & 0xFFFFu));
-                const double b = bf16_to_f64(static_cast<uint16_t>(v[u] >> 16));
-                p0 = __dadd_rn(p0, __dmul_rn(a, a));
-                p1 = __dadd_rn(p1, __dmul_rn(b, b));
-            }
-        }
-        for (; t < t1; ++t) {
-            const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(base + (t - t0) * ldx));
-            const double a = bf16_to_f64(static_cast<uint16_t>(v & 0xFFFFu));
-            const double b = bf16_to_f64(static_cast<uint16_t>(v >> 16));
-            p0 = __dadd_rn(p0, __dmul_rn(a, a));
-            p1 = __dadd_rn(p1, __dmul_rn(b, b));
-        }
-    } else {  // last single column
-        for (int64_t t = t0; t < t1; ++t) {
-            const double a = bf16_to_f64(__ldg(base + (t - t0) * ldx));
-            p0 = __dadd_rn(p0, __dmul_rn(a, a));
+constexpr int H_STAGES = 3;
+constexpr int H_TILE_BYTES = H_CHUNK * H_BLOCK_COLS * 2;  // 32 KB
+constexpr int H_RUN_BYTES = H_SLICES * H_VEC * (H_GROUPS + 1) * 8;
+constexpr int H_SMEM_BYTES = H_STAGES * H_TILE_BYTES + H_RUN_BYTES + 64 + 1024;
+
+__device__ __forceinline__ double bf16lo_to_f64(uint32_t w) {
+    return static_cast<double>(__uint_as_float(w << 16));
+}
+__device__ __forceinline__ double bf16hi_to_f64(uint32_t w) {
+    return static_cast<double>(__uint_as_float(w & 0xFFFF0000u));
+}
+
+__device__ __forceinline__ void sq_acc_conv(uint32_t w, double &a0, double &a1) {
+    const double x0 = bf16lo_to_f64(w), x1 = bf16hi_to_f64(w);
+    a0 = __fma_rn(x0, x0, a0);
+    a1 = __fma_rn(x1, x1, a1);
+}
+
+__global__ void __launch_bounds__(H_THREADS, 2)
+    k_colsumsq_chunk(const __grid_constant__ CUtensorMap tmX, int64_t T, int64_t K, int64_t nchunks,
+                     double *__restrict__ out, int direct) {
+    extern __shared__ uint8_t h_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(h_smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    double(*run)[H_VEC][H_GROUPS + 1] =
+        reinterpret_cast<double(*)[H_VEC][H_GROUPS + 1]>(smem + H_STAGES * H_TILE_BYTES);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + H_STAGES * H_TILE_BYTES + H_RUN_BYTES);
+    grid_dep_launch();
+    const int g = threadIdx.x & (H_GROUPS - 1), r = threadIdx.x / H_GROUPS;
+    const int32_t xcol = static_cast<int32_t>(blockIdx.x) * H_BLOCK_COLS;
+    const int64_t mine = (nchunks - blockIdx.y + gridDim.y - 1) / gridDim.y;  // chunks of this block
+    auto chunk_of = [&](int64_t i) { return static_cast<int64_t>(blockIdx.y) + i * gridDim.y; };
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < H_STAGES; ++s) mbar_init(&full[s], 1);
+        fence_barrier_init();
+        prefetch_tmap(&tmX);
+        for (int64_t i = 0; i < mine && i < H_STAGES; ++i) {
+            mbar_arrive_expect_tx(&full[i], H_TILE_BYTES);
+            tma_load_2d(smem + i * H_TILE_BYTES, &tmX, &full[i], xcol,
+                        static_cast<int32_t>(chunk_of(i) * H_CHUNK));
         }
     }
-    if (direct) {
-        const double dT = static_cast<double>(T);
-        out[col] = __ddiv_rn(p0, dT);
-        if (col + 1 < K) out[col + 1] = __ddiv_rn(p1, dT);
-    } else {
-        double *dst = out + static_cast<int64_t>(blockIdx.y) * K + col;
-        dst[0] = p0;
-        if (col + 1 < K) dst[1] = p1;
+    __syncthreads();
+    int64_t issued = mine < H_STAGES ? mine : H_STAGES;
+    const int c = threadIdx.x;  // the column this thread finishes in the ordered run sum
+    const int64_t col = static_cast<int64_t>(xcol) + c;
+    for (int64_t i = 0; i < mine; ++i) {
+        const int s = static_cast<int>(i % H_STAGES);
+        const bool ok = __syncthreads_and(mbar_wait(&full[s], static_cast<uint32_t>((i / H_STAGES) & 1)));
+        if (!ok) {  // timed out (error word set): let the copies in flight land, then leave
+            if (threadIdx.x == 0)
+                for (int64_t j = i; j < issued; ++j)
+                    mbar_wait(&full[j % H_STAGES], static_cast<uint32_t>((j / H_STAGES) & 1));
+            return;
+        }
+        const uint8_t *tile = smem + s * H_TILE_BYTES + (r * H_SLICE) * (H_BLOCK_COLS * 2) + g * 16;
+        double acc[H_VEC];
+#pragma unroll
+        for (int k = 0; k < H_VEC; ++k) acc[k] = 0.0;
+#pragma unroll 4
+        for (int u = 0; u < H_SLICE; ++u) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(tile + u * (H_BLOCK_COLS * 2));
+            sq_acc_conv(v.x, acc[0], acc[1]);
+            sq_acc_conv(v.y, acc[2], acc[3]);
+            sq_acc_conv(v.z, acc[4], acc[5]);
+            sq_acc_conv(v.w, acc[6], acc[7]);
+        }
+#pragma unroll
+        for (int k = 0; k < H_VEC; ++k) run[r][k][g] = acc[k];
+        __syncthreads();  // tile s consumed by every thread; the runs are complete
+        if (threadIdx.x == 0 && issued < mine) {
+            mbar_arrive_expect_tx(&full[s], H_TILE_BYTES);
+            tma_load_2d(smem + s * H_TILE_BYTES, &tmX, &full[s], xcol,
+                        static_cast<int32_t>(chunk_of(issued) * H_CHUNK));
+            ++issued;
+        }
+        if (col < K) {
+            double total = run[0][c % H_VEC][c / H_VEC];
+#pragma unroll
+            for (int q = 1; q < H_SLICES; ++q) total = __dadd_rn(total, run[q][c % H_VEC][c / H_VEC]);
+            if (direct)
+                out[col] = __ddiv_rn(total, static_cast<double>(T));
+            else
+                out[chunk_of(i) * K + col] = total;
+        }
+        __syncthreads();  // the runs are read before the next chunk overwrites them
     }
 }
 
-// sums the chunk partials in ascending chunk order, then divides by T
-__global__ void k_colsumsq_finish(const double *__restrict__ part, int64_t nchunks, int64_t T,
-                                  int64_t K, double *__restrict__ H) {
+// sums the chunk partials in ascending chunk order, then divides by T;
+// launched as a programmatic dependent of k_colsumsq_chunk
+__global__ void __launch_bounds__(64) k_colsumsq_finish(const double *__restrict__ part, int64_t nchunks,
+                                                         int64_t T, int64_t K, double *__restrict__ H) {
+    grid_dep_wait();
     const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (j >= K) return;
+    // loads run ahead of the (ordered) additions, 32 partials at a time
     double total = 0.0;
-    for (int64_t c = 0; c < nchunks; ++c) total = __dadd_rn(total, part[c * K + j]);
+    int64_t c = 0;
+    for (; c + 32 <= nchunks; c += 32) {
+        double v[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) v[u] = part[(c + u) * K + j];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) total = __dadd_rn(total, v[u]);
+    }
+    for (; c < nchunks; ++c) total = __dadd_rn(total, part[c * K + j]);
     H[j] = __ddiv_rn(total, static_cast<double>(T));
 }
 
@@ -101,6 +167,100 @@ __device__ __forceinline__ float score_one(const double *__restrict__ H, double 
     const double w = bf16_to_f64(wb);
     const double h = __dadd_rn(__ldg(H + j), eps);
     return __double2float_rn(__dmul_rn(h, __dmul_rn(w, w)));
+}
+
+// O(d_in) refresh of H under per-channel equivalent scaling (Sparsity
+// Induction sec. 2C): H'_j = H_j / (s_j * s_j), fp64 multiply then division.
+__global__ void __launch_bounds__(256) k_hessian_rescale(const double *__restrict__ H,
+                                                         const double *__restrict__ sc, int64_t K,
+                                                         double *__restrict__ out) {
+    const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (j < K) out[j] = __ddiv_rn(H[j], __dmul_rn(sc[j], sc[j]));
+}
+
+// ---------------------------------------------------------------------------
+// Hutchinson estimate of diag(A), A = X^T X / T, from S given sign vectors
+// (bit set = -1):  D_k = (1/S) sum_s z_s[k] (X^T (X z_s))[k] / T.
+// Rewritten as D_k = (1/(S T)) sum_t x[t,k] p[t,k] with p[t,k] = sum_s z_s[k]
+// u[t,s] and u[t,s] = sum_j z_s[j] x[t,j]:
+//   k_hutch_u   one block per token: the row in shared memory, warp w forms
+//               u[t, s] for s = w, w+8, ... (lane-strided partial sums, then a
+//               shuffle tree), fp32;
+//   k_hutch_acc (256 columns x 128 tokens) per block: u of the chunk in shared
+//               memory, each thread its column's S signs in registers, p in
+//               fp32, x * p accumulated in fp64 over the chunk's tokens;
+//   k_hutch_fin the chunk partials in ascending order, / (S T).
+// ---------------------------------------------------------------------------
+constexpr int HUTCH_MAX_S = 256, HUTCH_CHUNK = 128;
+
+__global__ void __launch_bounds__(256) k_hutch_u(const uint16_t *__restrict__ X, int64_t T, int64_t K,
+                                                 int64_t ldx, const uint32_t *__restrict__ zbits, int64_t S,
+                                                 float *__restrict__ U) {
+    extern __shared__ uint16_t xrow[];
+    const int64_t t = blockIdx.x + static_cast<int64_t>(blockIdx.y) * 65535;
+    if (t >= T) return;
+    for (int64_t k = threadIdx.x; k < K; k += blockDim.x) xrow[k] = X[t * ldx + k];
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t words = (K + 31) / 32;
+    for (int64_t sidx = warp; sidx < S; sidx += blockDim.x >> 5) {
+        const uint32_t *zs = zbits + sidx * words;
+        float acc = 0.0f;
+        for (int64_t i = 0; i < words; ++i) {
+            const int64_t k = 32 * i + lane;
+            if (k < K) {
+                const float x = bf16_to_f32(xrow[k]);
+                acc += ((__ldg(zs + i) >> lane) & 1u) ? -x : x;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) U[t * S + sidx] = acc;
+    }
+}
+
+__global__ void __launch_bounds__(256) k_hutch_acc(const uint16_t *__restrict__ X, int64_t T, int64_t K,
+                                                   int64_t ldx, const uint32_t *__restrict__ zbits, int64_t S,
+                                                   const float *__restrict__ U, double *__restrict__ part) {
+    extern __shared__ float uchunk[];  // [HUTCH_CHUNK][S]
+    const int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t c = blockIdx.y;
+    const int64_t t0 = c * HUTCH_CHUNK, t1 = t0 + HUTCH_CHUNK < T ? t0 + HUTCH_CHUNK : T;
+    for (int64_t i = threadIdx.x; i < (t1 - t0) * S; i += blockDim.x) uchunk[i] = U[t0 * S + i];
+    __syncthreads();
+    if (k >= K) return;
+    const int64_t words = (K + 31) / 32;
+    uint32_t zb[HUTCH_MAX_S / 32];  // this column's S signs, bit s % 32 of zb[s / 32]
+#pragma unroll
+    for (int w = 0; w < HUTCH_MAX_S / 32; ++w) zb[w] = 0u;
+    for (int64_t sidx = 0; sidx < S; ++sidx) {
+        const uint32_t bit = (__ldg(zbits + sidx * words + (k >> 5)) >> (k & 31)) & 1u;
+#pragma unroll
+        for (int w = 0; w < HUTCH_MAX_S / 32; ++w)
+            if (w == (sidx >> 5)) zb[w] |= bit << (sidx & 31);
+    }
+    double acc = 0.0;
+    for (int64_t t = t0; t < t1; ++t) {
+        const float *ut = uchunk + (t - t0) * S;
+        float p = 0.0f;
+#pragma unroll
+        for (int w = 0; w < HUTCH_MAX_S / 32; ++w) {
+            if (32 * w >= S) break;
+            const uint32_t bits = zb[w];
+            for (int b = 0; b < 32 && 32 * w + b < S; ++b) p += ((bits >> b) & 1u) ? -ut[32 * w + b] : ut[32 * w + b];
+        }
+        acc = __dadd_rn(acc, static_cast<double>(bf16_to_f32(X[t * ldx + k]) * p));
+    }
+    part[c * K + k] = acc;
+}
+
+__global__ void __launch_bounds__(256) k_hutch_fin(const double *__restrict__ part, int64_t nchunks, int64_t K,
+                                                   double scale, double *__restrict__ D) {
+    const int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (k >= K) return;
+    double total = 0.0;
+    for (int64_t c = 0; c < nchunks; ++c) total = __dadd_rn(total, part[c * K + k]);
+    D[k] = __dmul_rn(total, scale);
 }
 
 // Where a3 takes its selection scores from: the stored S, or -- a2 fused into
@@ -981,6 +1141,46 @@ inline int sm_count() {
 
 }  // namespace
 
+namespace {
+
+// the chunk kernel, then (more than one chunk) the ordered finish as its
+// programmatic dependent, so that its launch overlaps the chunk kernel
+nm_status launch_colsumsq(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, double *H, double *part,
+                          cudaStream_t s) {
+    using namespace nm;
+    const int64_t nchunks = (T + H_CHUNK - 1) / H_CHUNK;
+    CUtensorMap tm;
+    if (!make_tmap_bf16(&tm, X, T, K, ldx, H_BLOCK_COLS, H_CHUNK, false)) return NM_ERR_CUDA;
+    if (!set_smem_attr<k_colsumsq_chunk>(H_SMEM_BYTES)) return NM_ERR_CUDA;
+    // two blocks per SM: the column blocks, each with a strided share of the chunks
+    const int64_t cblocks = (K + H_BLOCK_COLS - 1) / H_BLOCK_COLS;
+    int64_t split = 2 * sm_count() / cblocks;
+    split = split < 1 ? 1 : (split > nchunks ? nchunks : split);
+    if (cblocks > 0x7FFFFFFF) return NM_ERR_SHAPE;
+    dim3 grid(static_cast<unsigned>(cblocks), static_cast<unsigned>(split));
+    if (nchunks == 1) {
+        k_colsumsq_chunk<<<grid, H_THREADS, H_SMEM_BYTES, s>>>(tm, T, K, nchunks, H, 1);
+        return launch_status();
+    }
+    k_colsumsq_chunk<<<grid, H_THREADS, H_SMEM_BYTES, s>>>(tm, T, K, nchunks, part, 0);
+    if (cudaGetLastError() != cudaSuccess) return NM_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((K + 63) / 64), 1, 1);
+    cfg.blockDim = dim3(64, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k_colsumsq_finish, static_cast<const double *>(part), nchunks, T, K, H) !=
+        cudaSuccess)
+        return NM_ERR_CUDA;
+    return launch_status();
+}
+
+}  // namespace
+
 extern "C" size_t nm_hessian_workspace_bytes(int64_t T, int64_t K) {
     if (T <= 0 || K <= 0) return 0;
     const int64_t nchunks = (T + H_CHUNK - 1) / H_CHUNK;
@@ -996,17 +1196,52 @@ extern "C" nm_status nm_hessian_diag(const uint16_t *X, int64_t T, int64_t K, in
     if (need > 0 && (!ws || ws_bytes < need)) return NM_ERR_WORKSPACE;
     const int64_t nchunks = (T + H_CHUNK - 1) / H_CHUNK;
     if (nchunks > 65535) return NM_ERR_SHAPE;
-    const int64_t col_threads = (K + H_COLS - 1) / H_COLS;
-    dim3 grid(static_cast<unsigned>((col_threads + H_THREADS - 1) / H_THREADS),
-              static_cast<unsigned>(nchunks));
-    cudaStream_t s = as_stream(stream);
-    if (nchunks == 1) {
-        k_colsumsq_chunk<<<grid, H_THREADS, 0, s>>>(X, T, K, ldx, H, 1);
-        return launch_status();
-    }
-    double *part = static_cast<double *>(ws);
-    k_colsumsq_chunk<<<grid, H_THREADS, 0, s>>>(X, T, K, ldx, part, 0);
-    k_colsumsq_finish<<<static_cast<unsigned>((K + 255) / 256), 256, 0, s>>>(part, nchunks, T, K, H);
+    return launch_colsumsq(X, T, K, ldx, H, static_cast<double *>(ws), as_stream(stream));
+}
+
+extern "C" nm_status nm_hessian_rescale(const double *H, const double *s, int64_t K, double *H_out,
+                                        void *stream) {
+    if (!H || !s || !H_out) return NM_ERR_NULL;
+    if (K < 1 || (K + 255) / 256 > 0x7FFFFFFF) return NM_ERR_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(H) | reinterpret_cast<uintptr_t>(s) |
+         reinterpret_cast<uintptr_t>(H_out)) & 7u)
+        return NM_ERR_ALIGN;
+    k_hessian_rescale<<<static_cast<unsigned>((K + 255) / 256), 256, 0, as_stream(stream)>>>(H, s, K, H_out);
+    return launch_status();
+}
+
+extern "C" size_t nm_hutchinson_workspace_bytes(int64_t T, int64_t K, int64_t S) {
+    if (T < 1 || K < 1 || S < 1) return 0;
+    const int64_t nchunks = (T + HUTCH_CHUNK - 1) / HUTCH_CHUNK;
+    const size_t ub = (static_cast<size_t>(T) * static_cast<size_t>(S) * sizeof(float) + 255) / 256 * 256;
+    return ub + static_cast<size_t>(nchunks) * static_cast<size_t>(K) * sizeof(double);
+}
+
+extern "C" nm_status nm_hutchinson_diag(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
+                                        const uint32_t *zbits, int64_t S, double *D, void *ws,
+                                        size_t ws_bytes, void *stream) {
+    if (!X || !zbits || !D || !ws) return NM_ERR_NULL;
+    if (T < 1 || K < 1 || ldx < K || S < 1 || S > HUTCH_MAX_S) return NM_ERR_SHAPE;
+    if (K * 2 > 227 * 1024 || (T + HUTCH_CHUNK - 1) / HUTCH_CHUNK > 65535) return NM_ERR_SHAPE;
+    if (!aligned16(X) || !aligned16(ws) || (ldx % 8) != 0 || (reinterpret_cast<uintptr_t>(zbits) & 3u) ||
+        (reinterpret_cast<uintptr_t>(D) & 7u))
+        return NM_ERR_ALIGN;
+    if (ws_bytes < nm_hutchinson_workspace_bytes(T, K, S)) return NM_ERR_WORKSPACE;
+    cudaStream_t st = as_stream(stream);
+    float *U = static_cast<float *>(ws);
+    const size_t ub = (static_cast<size_t>(T) * static_cast<size_t>(S) * sizeof(float) + 255) / 256 * 256;
+    double *part = reinterpret_cast<double *>(static_cast<uint8_t *>(ws) + ub);
+    const int64_t nchunks = (T + HUTCH_CHUNK - 1) / HUTCH_CHUNK;
+    const int smem_u = static_cast<int>(K * 2), smem_a = static_cast<int>(HUTCH_CHUNK * S * 4);
+    if (cudaFuncSetAttribute(k_hutch_u, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_u) != cudaSuccess ||
+        cudaFuncSetAttribute(k_hutch_acc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_a) != cudaSuccess)
+        return NM_ERR_CUDA;
+    dim3 gu(static_cast<unsigned>(T < 65535 ? T : 65535), static_cast<unsigned>((T + 65534) / 65535));
+    k_hutch_u<<<gu, 256, smem_u, st>>>(X, T, K, ldx, zbits, S, U);
+    dim3 ga(static_cast<unsigned>((K + 255) / 256), static_cast<unsigned>(nchunks));
+    k_hutch_acc<<<ga, 256, smem_a, st>>>(X, T, K, ldx, zbits, S, U, part);
+    k_hutch_fin<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(
+        part, nchunks, K, 1.0 / (static_cast<double>(S) * static_cast<double>(T)), D);
     return launch_status();
 }
 
@@ -1210,18 +1445,10 @@ extern "C" nm_status nm_hessian_diag_noalloc(const uint16_t *X, int64_t T, int64
     if (nchunks > 65535) return NM_ERR_SHAPE;
     if (nchunks > 1 && nchunks * K > static_cast<int64_t>(NM_HESSIAN_NOALLOC_MAX_PARTIALS))
         return NM_ERR_TOO_LARGE;
-    const int64_t col_threads = (K + H_COLS - 1) / H_COLS;
-    dim3 grid(static_cast<unsigned>((col_threads + H_THREADS - 1) / H_THREADS),
-              static_cast<unsigned>(nchunks));
-    cudaStream_t s = as_stream(stream);
-    if (nchunks == 1) {
-        k_colsumsq_chunk<<<grid, H_THREADS, 0, s>>>(X, T, K, ldx, H, 1);
-        return launch_status();
-    }
     double *part = nullptr;
-    const nm_status st = noalloc_scratch(&part);
-    if (st != NM_OK) return st;
-    k_colsumsq_chunk<<<grid, H_THREADS, 0, s>>>(X, T, K, ldx, part, 0);
-    k_colsumsq_finish<<<static_cast<unsigned>((K + 255) / 256), 256, 0, s>>>(part, nchunks, T, K, H);
-    return launch_status();
+    if (nchunks > 1) {
+        const nm_status st = noalloc_scratch(&part);
+        if (st != NM_OK) return st;
+    }
+    return launch_colsumsq(X, T, K, ldx, H, part, as_stream(stream));
 }

@@ -62,6 +62,10 @@ def test_size_queries():
     assert lib.nm_sparse_gemm_workspace_bytes(16, 4096, 5) == 0
     assert lib.nm_dense_gemm_workspace_bytes(16, 4096, 4096) == sk
     assert lib.nm_dense_gemm_workspace_bytes(16, 0, 4096) == 0
+    # u = X z in fp32 (rounded up to 256 bytes), then one fp64 row per 128 tokens
+    assert lib.nm_hutchinson_workspace_bytes(300, 1000, 7) == up(300 * 7 * 4) + 3 * 1000 * 8
+    assert lib.nm_hutchinson_workspace_bytes(128, 64, 1) == up(128 * 4) + 64 * 8
+    assert lib.nm_hutchinson_workspace_bytes(0, 64, 1) == 0
 
 
 # fake but 16-byte aligned device addresses: validation fails before any use
@@ -86,6 +90,20 @@ MIS = 0x10002
     (lambda l: l.nm_score_prune_compress(None, 0.0, A, 4, A, 8, 4, 8, 2, 4, A, A, A, None), 2),
     (lambda l: l.nm_score_prune_compress(None, 0.0, MIS, 8, A, 8, 4, 8, 2, 4, A, A, A, None), 3),
     (lambda l: l.nm_score_prune_compress(A + 4, 0.0, A, 8, A, 8, 4, 8, 2, 4, A, A, A, None), 3),
+    (lambda l: l.nm_hessian_rescale(None, A, 8, A, None), 1),
+    (lambda l: l.nm_hessian_rescale(A, A, 0, A, None), 2),
+    (lambda l: l.nm_hessian_rescale(A, A + 4, 8, A, None), 3),
+    (lambda l: l.nm_hutchinson_diag(None, 4, 8, 8, A, 2, A, A, 1 << 20, None), 1),
+    (lambda l: l.nm_hutchinson_diag(A, 4, 8, 8, A, 2, A, None, 1 << 20, None), 1),
+    (lambda l: l.nm_hutchinson_diag(A, 4, 8, 4, A, 2, A, A, 1 << 20, None), 2),
+    (lambda l: l.nm_hutchinson_diag(A, 4, 8, 8, A, 0, A, A, 1 << 20, None), 2),
+    (lambda l: l.nm_hutchinson_diag(A, 4, 8, 8, A, 257, A, A, 1 << 20, None), 2),
+    (lambda l: l.nm_hutchinson_diag(A, 4, 8, 12, A, 2, A, A, 1 << 20, None), 3),
+    (lambda l: l.nm_hutchinson_diag(A, 4, 8, 8, A + 2, 2, A, A, 1 << 20, None), 3),
+    (lambda l: l.nm_hutchinson_diag(A, 4, 8, 8, A, 2, A + 4, A, 1 << 20, None), 3),
+    (lambda l: l.nm_hutchinson_diag(A, 4, 8, 8, A, 2, A, A, 16, None), 5),
+    (lambda l: l.nm_hutchinson_diag(A, 4, 200000, 200000, A, 2, A, A, 1 << 30, None), 2),
+    (lambda l: l.nm_hutchinson_diag(A, 65535 * 128 + 1, 8, 8, A, 2, A, A, 1 << 62, None), 2),
     (lambda l: l.slide_pack(A, 4, 8, 7, A, None), 4),
     (lambda l: l.slide_pack(A, 4, 8, 12, A, None), 4),
     (lambda l: l.lift_activations(A, 4, 8, 8, 5, A, 8, None), 4),

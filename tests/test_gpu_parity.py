@@ -31,13 +31,41 @@ def _sync_ok(nm):
 
 
 # ---------------------------------------------------------------- a1 / a2
+# one chunk; ragged runs; one column; a block with several chunks in its
+# three-tile pipeline (K = 40000: more column blocks than SMs, so one split);
+# 65 chunks over the SM-sized split of a 4096-column layer
 @pytest.mark.parametrize("T,K,ld", [(128, 512, 512), (1000, 520, 520), (1, 7, 8), (129, 3, 8),
-                                    (2048, 4096, 4096), (300, 517, 528), (257, 96, 104)])
+                                    (2048, 4096, 4096), (300, 517, 528), (257, 96, 104),
+                                    (1000, 40000, 40000), (8292, 4096, 4104)])
 def test_hessian_bitexact(nm, T, K, ld):
     X = datagen.make_activations(T, K, seed=T + K, n_outliers=min(4, K))
     H = nm.hessian_diag(to_dev(X, ld))
     _sync_ok(nm)
     assert np.array_equal(to_host(H), oracle.hessian_diag(X))
+
+
+def test_hessian_special_values_bitexact(nm):
+    # zeros of both signs, bf16 subnormals, the smallest and largest normals
+    # and infinities, in even and odd columns: every class of value whose
+    # square the reduction must form exactly, against the oracle's fp64
+    T, K = 300, 64
+    X = datagen.make_activations(T, K, seed=5)
+    special = np.array([0x0000, 0x8000, 0x0001, 0x807F, 0x0040, 0x0080, 0x8080, 0x7F7F, 0xFF7F,
+                        0x1F80, 0x2000], dtype=np.uint16)
+    g = np.random.default_rng(5)
+    for j in range(2, 40):                       # a few special values in most columns
+        rows = g.choice(T, size=int(g.integers(1, 6)), replace=False)
+        X[rows, j] = g.choice(special, size=rows.size)
+    X[:, 40] = 0x0001                            # a whole column of subnormals
+    X[:, 41] = 0x8003
+    X[:, 42] = 0x0000                            # and one of zeros
+    X[7, 50] = 0x7F80                            # +inf and -inf
+    X[9, 51] = 0xFF80
+    H = nm.hessian_diag(to_dev(X))
+    _sync_ok(nm)
+    h, ref = to_host(H), oracle.hessian_diag(X)
+    assert np.isinf(ref[50]) and np.isinf(ref[51]) and ref[42] == 0.0 and 0.0 < ref[40] < 1e-70
+    assert np.array_equal(h, ref)
 
 
 @pytest.mark.parametrize("R,K,ld", [(256, 512, 512), (33, 1030, 1032), (5, 13, 16), (64, 4096, 4096)])
@@ -51,6 +79,86 @@ def test_score_bitexact(nm, R, K, ld):
     assert np.array_equal(to_host(H), Ho)
     assert np.array_equal(to_host(S), oracle.score_hessian(Ho, W, 1e-8))
     assert np.array_equal(to_host(Sm), oracle.score_magnitude(W))
+
+
+@pytest.mark.parametrize("K", [1, 517, 4096])
+def test_hessian_rescale_bitexact(nm, K):
+    # the O(d_in) refresh, and for power-of-two scales the proxy recomputed from
+    # the rescaled activations on the GPU
+    X = datagen.make_activations(300, K, seed=K, n_outliers=min(2, K))
+    H = nm.hessian_diag(to_dev(X, (K + 7) // 8 * 8))
+    g = np.random.default_rng(K).uniform(0.3, 3.0, size=K)
+    out = nm.hessian_rescale(H, torch.from_numpy(g).cuda())
+    p2 = np.array([2.0 ** ((j % 7) - 3) for j in range(K)])
+    out2 = nm.hessian_rescale(H, torch.from_numpy(p2).cuda())
+    X2 = datagen.f32_to_bf16_bits(bf16_to_f64(X).astype(np.float32) / p2[None, :].astype(np.float32))
+    H2 = nm.hessian_diag(to_dev(X2, (K + 7) // 8 * 8))
+    _sync_ok(nm)
+    assert np.array_equal(to_host(out), oracle.hessian_rescale(oracle.hessian_diag(X), g))
+    assert np.array_equal(to_host(out2), to_host(H2))
+
+
+def _zbits_dev(zb):
+    return torch.from_numpy(np.ascontiguousarray(zb).view(np.int32)).cuda()
+
+
+def _hutch_scale(X, zb):
+    # per column, (1/(S T)) sum_t |x_tk| sum_s |u_ts| with u = X z_s: the size of
+    # the terms the kernel rounds in fp32 (an error scale, not the estimate)
+    Xf = bf16_to_f64(X)
+    S, K = zb.shape[0], X.shape[1]
+    Z = np.array([[-1.0 if (zb[s, k // 32] >> (k % 32)) & 1 else 1.0 for k in range(K)] for s in range(S)])
+    U = np.abs(Xf @ Z.T).sum(axis=1)
+    return (np.abs(Xf) * U[:, None]).sum(axis=0) / (S * X.shape[0])
+
+
+# (T, K, S): one token / one column, ragged 128-token chunks and 32-column
+# words, S across the 32-bit sign words up to the 256 maximum, a full layer
+@pytest.mark.parametrize("T,K,S", [(1, 1, 1), (7, 33, 3), (300, 1000, 7), (129, 4096, 64),
+                                   (1100, 517, 256), (8192, 4096, 16)])
+def test_hutchinson_vs_oracle(nm, T, K, S):
+    X = datagen.make_activations(T, K, seed=T + S, n_outliers=min(2, K))
+    zb = datagen.rademacher_bits(S, K, seed=K + S)
+    Xd, zd = to_dev(X, (K + 7) // 8 * 8), _zbits_dev(zb)
+    D = nm.hutchinson_diag(Xd, zd)
+    D2 = nm.hutchinson_diag(Xd, zd)
+    _sync_ok(nm)
+    d, d2 = to_host(D), to_host(D2)
+    ref = oracle.hutchinson_diag(X, zb)
+    assert np.array_equal(d, d2)                       # fixed summation order
+    # fp32 u and p: a few ulps of fp32 of the rounded terms' size, per column
+    assert np.all(np.abs(d - ref) <= 1e-6 * _hutch_scale(X, zb) + 1e-300)
+
+
+def test_hutchinson_hadamard_signs_give_h(nm):
+    # K orthogonal sign vectors (Sylvester-Hadamard rows) make the estimate
+    # exact: the GPU estimate equals the GPU's H up to fp32 rounding
+    K, T = 64, 500
+    Hd = np.array([[1.0]])
+    while Hd.shape[0] < K:
+        Hd = np.block([[Hd, Hd], [Hd, -Hd]])
+    zb = np.zeros((K, 2), dtype=np.uint32)
+    for k in range(K):
+        zb[:, k // 32] |= (Hd[:, k] < 0).astype(np.uint32) << np.uint32(k % 32)
+    X = datagen.make_activations(T, K, seed=41, n_outliers=2)
+    Xd = to_dev(X)
+    D = nm.hutchinson_diag(Xd, _zbits_dev(zb))
+    H = nm.hessian_diag(Xd)
+    _sync_ok(nm)
+    assert np.all(np.abs(to_host(D) - to_host(H)) <= 1e-6 * _hutch_scale(X, zb))
+
+
+def test_hutchinson_caller_workspace(nm):
+    # a caller-owned workspace reused across calls of different shapes
+    lib = nm.load()
+    ws = torch.empty(lib.nm_hutchinson_workspace_bytes(1000, 1000, 32), dtype=torch.uint8, device="cuda")
+    for (T, K, S) in ((1000, 1000, 32), (999, 520, 31), (1, 1000, 1)):
+        X = datagen.make_activations(T, K, seed=K, n_outliers=2)
+        zb = datagen.rademacher_bits(S, K, seed=S)
+        D = nm.hutchinson_diag(to_dev(X), _zbits_dev(zb), ws=ws)
+        _sync_ok(nm)
+        ref = oracle.hutchinson_diag(X, zb)
+        assert np.all(np.abs(to_host(D) - ref) <= 1e-6 * _hutch_scale(X, zb) + 1e-300)
 
 
 # ---------------------------------------------------------------- a3

@@ -12,7 +12,8 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 MUTATIONS = [
-    ("part = part + sq;", "part = part + sq + sq;"),                       # doubled term
+    ("run = run + sq;", "run = run + sq + sq;"),                           # doubled term
+    ("part = part + run;", "part = run;"),                                 # dropped run
     ("H[j] = total / (double)T;", "H[j] = total / (double)(T + 1);"),     # wrong divisor
     ("(s[p] == s[q] && p < q)", "(s[p] == s[q] && p > q)"),               # tie direction
     ("if (rank < n) idx", "if (rank <= n) idx"),                          # off by one

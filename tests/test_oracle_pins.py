@@ -64,14 +64,87 @@ def test_H_power_of_two_scaling_is_exact():
     assert np.array_equal(H2, H * (scale.astype(np.float64) ** 2))
 
 
+def test_H_rescale_equals_recomputed_proxy():
+    # equivalent scaling X' = X diag(1/s): for power-of-two s (exact in bf16)
+    # the O(d_in) refresh H / s^2 is bit-identical to recomputing H from X'
+    X = datagen.make_activations(300, 24, seed=9, n_outliers=2)
+    s = np.array([2.0 ** ((j % 7) - 3) for j in range(24)])
+    X2 = bf16(f32(X) / s[None, :].astype(np.float32))
+    assert np.array_equal(f32(X2).astype(np.float64), f32(X).astype(np.float64) / s[None, :])
+    assert np.array_equal(oracle.hessian_rescale(oracle.hessian_diag(X), s), oracle.hessian_diag(X2))
+    # s = 1 is the identity; general s within one rounding of H / s^2 in exact arithmetic
+    H = oracle.hessian_diag(X)
+    assert np.array_equal(oracle.hessian_rescale(H, np.ones(24)), H)
+    g = np.random.default_rng(1).uniform(0.3, 3.0, size=24)
+    out = oracle.hessian_rescale(H, g)
+    for j in range(24):
+        exact = Fraction(float(H[j])) / (Fraction(float(g[j])) ** 2)
+        assert abs(Fraction(float(out[j])) - exact) <= exact * Fraction(3, 2 ** 53)
+
+
+def _bits_from_signs(signs):
+    """[S x K] array of +-1 -> the sign-bit layout (bit set = -1)."""
+    S, K = signs.shape
+    words = np.zeros((S, (K + 31) // 32), dtype=np.uint32)
+    for k in range(K):
+        words[:, k // 32] |= (signs[:, k] < 0).astype(np.uint32) << np.uint32(k % 32)
+    return words
+
+
+def test_hutchinson_exact_with_hadamard_signs():
+    # the rows of a Sylvester-Hadamard matrix are K orthogonal sign vectors:
+    # (1/K) sum_s z_s[k] z_s[j] = delta_kj, so the estimate is diag(A) = H exactly
+    K = 64
+    Hd = np.array([[1]])
+    while Hd.shape[0] < K:
+        Hd = np.block([[Hd, Hd], [Hd, -Hd]])
+    X = datagen.make_activations(96, K, seed=4, n_outliers=3)
+    D = oracle.hutchinson_diag(X, _bits_from_signs(Hd))
+    H = oracle.hessian_diag(X)
+    assert np.all(np.abs(D - H) <= 1e-12 * np.abs(H).max())
+
+
+def test_hutchinson_single_sample_closed_form():
+    # S = 1: D = z * (A z) with A = X^T X / T, formed here by a matmul
+    X = datagen.make_activations(50, 37, seed=6)
+    z = np.where(np.random.default_rng(3).integers(0, 2, 37) == 1, -1.0, 1.0)
+    Xf = f32(X).astype(np.float64)
+    A = Xf.T @ Xf / 50
+    D = oracle.hutchinson_diag(X, _bits_from_signs(z[None, :]))
+    assert np.allclose(D, z * (A @ z), rtol=1e-12, atol=1e-12)
+    # the bit layout of datagen's sign vectors matches the one above
+    zb = datagen.rademacher_bits(5, 37, seed=9)
+    signs = np.array([[-1.0 if (zb[s, k // 32] >> (k % 32)) & 1 else 1.0 for k in range(37)] for s in range(5)])
+    assert np.array_equal(_bits_from_signs(signs), zb)
+
+
+def test_hutchinson_converges_to_H():
+    # unbiased with variance ~ 1/S: the error against H shrinks as S grows
+    X = datagen.make_activations(200, 48, seed=8)
+    H = oracle.hessian_diag(X)
+    err = [np.sqrt(np.mean((oracle.hutchinson_diag(X, datagen.rademacher_bits(S, 48, seed=S)) - H) ** 2))
+           for S in (16, 256, 4096)]
+    assert err[1] < err[0] / 2 and err[2] < err[1] / 2
+
+
 def test_H_canonical_vs_naive_and_single_chunk():
     X = datagen.make_activations(1000, 64, seed=7, n_outliers=2)
     Hc = oracle.hessian_diag(X)
     Hn = oracle.hessian_diag(X, naive=True)
     assert np.all(np.abs(Hc - Hn) <= 1e-12 * np.abs(Hn))
-    # with at most one chunk of tokens the canonical order is the sequential one
-    Xs = X[: oracle.H_CHUNK]
+    # with at most one run of tokens the canonical order is the sequential one
+    Xs = X[: oracle.H_RUN]
     assert np.array_equal(oracle.hessian_diag(Xs), oracle.hessian_diag(Xs, naive=True))
+    # one chunk: the runs of 16 tokens, each sequential, added in ascending order
+    Xc = X[:100]
+    x2 = f32(Xc).astype(np.float64) ** 2
+    expect = np.zeros(64)
+    for r0 in range(0, 100, oracle.H_RUN):
+        run = np.zeros(64)
+        for t in range(r0, min(r0 + oracle.H_RUN, 100)):
+            run = run + x2[t]
+        expect = expect + run
+    assert np.array_equal(oracle.hessian_diag(Xc), expect / 100)
 
 
 def test_H_outlier_channels_scale_400x_in_expectation():
