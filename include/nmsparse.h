@@ -183,15 +183,22 @@ nm_status nm_hessian_rescale(const double *H, const double *s, int64_t K, double
  *           of row s set = z_s[k] = -1, clear = +1.  1 <= S <= 256.
  *   D     : fp64 [K] (written), 8-byte aligned.
  *   ws    : nm_hutchinson_workspace_bytes(T, K, S) bytes, 16-byte aligned,
- *           owned by the caller (u = X z_s in fp32, then per-128-token fp64
- *           partials of D).
- * Arithmetic: u[t,s] in fp32 (lane-strided sums, then a shuffle tree);
- * p[t,k] = sum_s z_s[k] u[t,s] in fp32, s ascending; x[t,k] * p[t,k] rounded
- * to fp32 and added in fp64 over each 128-token chunk, chunks in ascending
- * order, then one multiply by 1/(S T).  Deterministic run to run.
- * Errors: NULL -> NM_ERR_NULL; S outside [1, 256], T or K < 1, ldx < K, a
- * row of X above 227 KiB (K > 116224) or T above 65535 * 128 -> NM_ERR_SHAPE;
- * alignment -> NM_ERR_ALIGN; short workspace -> NM_ERR_WORKSPACE.           */
+ *           owned by the caller; contents on return unspecified.  It holds,
+ *           each region padded to 1 KiB: Z as bf16 [S16 x ldz] (S16 = S
+ *           rounded up to 16, ldz = K rounded up to 8), [Z^T Z^T Z^T] as bf16
+ *           [K x C3] (C3 = 3S rounded up to 64), the fp32 partials of U = X Z^T
+ *           [nsplit x T x S16], U split into bf16 pieces [T x C3] and fp64
+ *           partials of D [ceil(T/128) x K].  nsplit is the value in [1, min(8, ceil(K/64))]
+ *           with the least ceil(n / 148) / n, n = ceil(T/128) * nsplit (the
+ *           smaller on ties): CTAs spread evenly over a B200's 148 SMs.
+ * Arithmetic (tensor cores, bf16 operands, fp32 accumulation): U = X Z^T
+ * over K split into nsplit ranges, the partials added in ascending order;
+ * each u split exactly into three bf16 pieces; P = Z^T U^T from the pieces;
+ * x * P summed in fp32 over 32 tokens, in fp64 over 128-token tiles, the tiles
+ * in ascending order, then one multiply by 1/(S T).  Deterministic run to run.
+ * Errors: NULL -> NM_ERR_NULL; S outside [1, 256], T or K < 1 or above
+ * 2^31 - 128, ldx < K -> NM_ERR_SHAPE; alignment -> NM_ERR_ALIGN; short
+ * workspace -> NM_ERR_WORKSPACE.                                            */
 size_t nm_hutchinson_workspace_bytes(int64_t T, int64_t K, int64_t S);
 nm_status nm_hutchinson_diag(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, const uint32_t *zbits,
                              int64_t S, double *D, void *ws, size_t ws_bytes, void *stream);

@@ -178,91 +178,6 @@ __global__ void __launch_bounds__(256) k_hessian_rescale(const double *__restric
     if (j < K) out[j] = __ddiv_rn(H[j], __dmul_rn(sc[j], sc[j]));
 }
 
-// ---------------------------------------------------------------------------
-// Hutchinson estimate of diag(A), A = X^T X / T, from S given sign vectors
-// (bit set = -1):  D_k = (1/S) sum_s z_s[k] (X^T (X z_s))[k] / T.
-// Rewritten as D_k = (1/(S T)) sum_t x[t,k] p[t,k] with p[t,k] = sum_s z_s[k]
-// u[t,s] and u[t,s] = sum_j z_s[j] x[t,j]:
-//   k_hutch_u   one block per token: the row in shared memory, warp w forms
-//               u[t, s] for s = w, w+8, ... (lane-strided partial sums, then a
-//               shuffle tree), fp32;
-//   k_hutch_acc (256 columns x 128 tokens) per block: u of the chunk in shared
-//               memory, each thread its column's S signs in registers, p in
-//               fp32, x * p accumulated in fp64 over the chunk's tokens;
-//   k_hutch_fin the chunk partials in ascending order, / (S T).
-// ---------------------------------------------------------------------------
-constexpr int HUTCH_MAX_S = 256, HUTCH_CHUNK = 128;
-
-__global__ void __launch_bounds__(256) k_hutch_u(const uint16_t *__restrict__ X, int64_t T, int64_t K,
-                                                 int64_t ldx, const uint32_t *__restrict__ zbits, int64_t S,
-                                                 float *__restrict__ U) {
-    extern __shared__ uint16_t xrow[];
-    const int64_t t = blockIdx.x + static_cast<int64_t>(blockIdx.y) * 65535;
-    if (t >= T) return;
-    for (int64_t k = threadIdx.x; k < K; k += blockDim.x) xrow[k] = X[t * ldx + k];
-    __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t words = (K + 31) / 32;
-    for (int64_t sidx = warp; sidx < S; sidx += blockDim.x >> 5) {
-        const uint32_t *zs = zbits + sidx * words;
-        float acc = 0.0f;
-        for (int64_t i = 0; i < words; ++i) {
-            const int64_t k = 32 * i + lane;
-            if (k < K) {
-                const float x = bf16_to_f32(xrow[k]);
-                acc += ((__ldg(zs + i) >> lane) & 1u) ? -x : x;
-            }
-        }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) U[t * S + sidx] = acc;
-    }
-}
-
-__global__ void __launch_bounds__(256) k_hutch_acc(const uint16_t *__restrict__ X, int64_t T, int64_t K,
-                                                   int64_t ldx, const uint32_t *__restrict__ zbits, int64_t S,
-                                                   const float *__restrict__ U, double *__restrict__ part) {
-    extern __shared__ float uchunk[];  // [HUTCH_CHUNK][S]
-    const int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const int64_t c = blockIdx.y;
-    const int64_t t0 = c * HUTCH_CHUNK, t1 = t0 + HUTCH_CHUNK < T ? t0 + HUTCH_CHUNK : T;
-    for (int64_t i = threadIdx.x; i < (t1 - t0) * S; i += blockDim.x) uchunk[i] = U[t0 * S + i];
-    __syncthreads();
-    if (k >= K) return;
-    const int64_t words = (K + 31) / 32;
-    uint32_t zb[HUTCH_MAX_S / 32];  // this column's S signs, bit s % 32 of zb[s / 32]
-#pragma unroll
-    for (int w = 0; w < HUTCH_MAX_S / 32; ++w) zb[w] = 0u;
-    for (int64_t sidx = 0; sidx < S; ++sidx) {
-        const uint32_t bit = (__ldg(zbits + sidx * words + (k >> 5)) >> (k & 31)) & 1u;
-#pragma unroll
-        for (int w = 0; w < HUTCH_MAX_S / 32; ++w)
-            if (w == (sidx >> 5)) zb[w] |= bit << (sidx & 31);
-    }
-    double acc = 0.0;
-    for (int64_t t = t0; t < t1; ++t) {
-        const float *ut = uchunk + (t - t0) * S;
-        float p = 0.0f;
-#pragma unroll
-        for (int w = 0; w < HUTCH_MAX_S / 32; ++w) {
-            if (32 * w >= S) break;
-            const uint32_t bits = zb[w];
-            for (int b = 0; b < 32 && 32 * w + b < S; ++b) p += ((bits >> b) & 1u) ? -ut[32 * w + b] : ut[32 * w + b];
-        }
-        acc = __dadd_rn(acc, static_cast<double>(bf16_to_f32(X[t * ldx + k]) * p));
-    }
-    part[c * K + k] = acc;
-}
-
-__global__ void __launch_bounds__(256) k_hutch_fin(const double *__restrict__ part, int64_t nchunks, int64_t K,
-                                                   double scale, double *__restrict__ D) {
-    const int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (k >= K) return;
-    double total = 0.0;
-    for (int64_t c = 0; c < nchunks; ++c) total = __dadd_rn(total, part[c * K + k]);
-    D[k] = __dmul_rn(total, scale);
-}
-
 // Where a3 takes its selection scores from: the stored S, or -- a2 fused into
 // a3, S never written -- computed in registers from W exactly as k_score
 // does: fp32((H_j + eps) * w^2) with fp64 add and multiplies, or |w| when H is
@@ -1207,41 +1122,6 @@ extern "C" nm_status nm_hessian_rescale(const double *H, const double *s, int64_
          reinterpret_cast<uintptr_t>(H_out)) & 7u)
         return NM_ERR_ALIGN;
     k_hessian_rescale<<<static_cast<unsigned>((K + 255) / 256), 256, 0, as_stream(stream)>>>(H, s, K, H_out);
-    return launch_status();
-}
-
-extern "C" size_t nm_hutchinson_workspace_bytes(int64_t T, int64_t K, int64_t S) {
-    if (T < 1 || K < 1 || S < 1) return 0;
-    const int64_t nchunks = (T + HUTCH_CHUNK - 1) / HUTCH_CHUNK;
-    const size_t ub = (static_cast<size_t>(T) * static_cast<size_t>(S) * sizeof(float) + 255) / 256 * 256;
-    return ub + static_cast<size_t>(nchunks) * static_cast<size_t>(K) * sizeof(double);
-}
-
-extern "C" nm_status nm_hutchinson_diag(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
-                                        const uint32_t *zbits, int64_t S, double *D, void *ws,
-                                        size_t ws_bytes, void *stream) {
-    if (!X || !zbits || !D || !ws) return NM_ERR_NULL;
-    if (T < 1 || K < 1 || ldx < K || S < 1 || S > HUTCH_MAX_S) return NM_ERR_SHAPE;
-    if (K * 2 > 227 * 1024 || (T + HUTCH_CHUNK - 1) / HUTCH_CHUNK > 65535) return NM_ERR_SHAPE;
-    if (!aligned16(X) || !aligned16(ws) || (ldx % 8) != 0 || (reinterpret_cast<uintptr_t>(zbits) & 3u) ||
-        (reinterpret_cast<uintptr_t>(D) & 7u))
-        return NM_ERR_ALIGN;
-    if (ws_bytes < nm_hutchinson_workspace_bytes(T, K, S)) return NM_ERR_WORKSPACE;
-    cudaStream_t st = as_stream(stream);
-    float *U = static_cast<float *>(ws);
-    const size_t ub = (static_cast<size_t>(T) * static_cast<size_t>(S) * sizeof(float) + 255) / 256 * 256;
-    double *part = reinterpret_cast<double *>(static_cast<uint8_t *>(ws) + ub);
-    const int64_t nchunks = (T + HUTCH_CHUNK - 1) / HUTCH_CHUNK;
-    const int smem_u = static_cast<int>(K * 2), smem_a = static_cast<int>(HUTCH_CHUNK * S * 4);
-    if (cudaFuncSetAttribute(k_hutch_u, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_u) != cudaSuccess ||
-        cudaFuncSetAttribute(k_hutch_acc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_a) != cudaSuccess)
-        return NM_ERR_CUDA;
-    dim3 gu(static_cast<unsigned>(T < 65535 ? T : 65535), static_cast<unsigned>((T + 65534) / 65535));
-    k_hutch_u<<<gu, 256, smem_u, st>>>(X, T, K, ldx, zbits, S, U);
-    dim3 ga(static_cast<unsigned>((K + 255) / 256), static_cast<unsigned>(nchunks));
-    k_hutch_acc<<<ga, 256, smem_a, st>>>(X, T, K, ldx, zbits, S, U, part);
-    k_hutch_fin<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(
-        part, nchunks, K, 1.0 / (static_cast<double>(S) * static_cast<double>(T)), D);
     return launch_status();
 }
 

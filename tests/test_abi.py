@@ -2,6 +2,7 @@
 sm_100a, loads, exports every function include/nmsparse.h declares, and its
 argument validation rejects bad calls before launching anything."""
 import ctypes
+from fractions import Fraction
 import os
 import re
 
@@ -62,10 +63,23 @@ def test_size_queries():
     assert lib.nm_sparse_gemm_workspace_bytes(16, 4096, 5) == 0
     assert lib.nm_dense_gemm_workspace_bytes(16, 4096, 4096) == sk
     assert lib.nm_dense_gemm_workspace_bytes(16, 0, 4096) == 0
-    # u = X z in fp32 (rounded up to 256 bytes), then one fp64 row per 128 tokens
-    assert lib.nm_hutchinson_workspace_bytes(300, 1000, 7) == up(300 * 7 * 4) + 3 * 1000 * 8
-    assert lib.nm_hutchinson_workspace_bytes(128, 64, 1) == up(128 * 4) + 64 * 8
+    # Z [S16 x ldz], [Z^T Z^T Z^T] [K x C3], U partials [nsplit x T x S16] fp32,
+    # U pieces [T x C3] bf16, D partials [T/128 x K] fp64, each padded to
+    # 1 KiB; nsplit in [1, min(8, K/64)] the
+    # one with least ceil(n/148)/n for n = T/128 * nsplit, the smaller on ties
+    k1 = lambda b: (b + 1023) // 1024 * 1024
+
+    def hq(T, K, S):
+        S16, C3, ldz, tt = (S + 15) // 16 * 16, (3 * S + 63) // 64 * 64, (K + 7) // 8 * 8, (T + 127) // 128
+        cost = lambda ns: Fraction(-(-tt * ns // 148), tt * ns)
+        ns = min(range(1, min(8, (K + 63) // 64) + 1), key=lambda n: (cost(n), n))
+        return (k1(S16 * ldz * 2) + k1(K * C3 * 2) + k1(ns * T * S16 * 4) + k1(T * C3 * 2)
+                + k1(tt * K * 8))
+    assert lib.nm_hutchinson_workspace_bytes(300, 1000, 7) == hq(300, 1000, 7)
+    assert lib.nm_hutchinson_workspace_bytes(8192, 4096, 16) == hq(8192, 4096, 16)
+    assert lib.nm_hutchinson_workspace_bytes(1, 1, 256) == hq(1, 1, 256)
     assert lib.nm_hutchinson_workspace_bytes(0, 64, 1) == 0
+    assert lib.nm_hutchinson_workspace_bytes(64, 64, 257) == 0
 
 
 # fake but 16-byte aligned device addresses: validation fails before any use
@@ -102,8 +116,8 @@ MIS = 0x10002
     (lambda l: l.nm_hutchinson_diag(A, 4, 8, 8, A + 2, 2, A, A, 1 << 20, None), 3),
     (lambda l: l.nm_hutchinson_diag(A, 4, 8, 8, A, 2, A + 4, A, 1 << 20, None), 3),
     (lambda l: l.nm_hutchinson_diag(A, 4, 8, 8, A, 2, A, A, 16, None), 5),
-    (lambda l: l.nm_hutchinson_diag(A, 4, 200000, 200000, A, 2, A, A, 1 << 30, None), 2),
-    (lambda l: l.nm_hutchinson_diag(A, 65535 * 128 + 1, 8, 8, A, 2, A, A, 1 << 62, None), 2),
+    (lambda l: l.nm_hutchinson_diag(A, 4, 1 << 31, 1 << 31, A, 2, A, A, 1 << 62, None), 2),
+    (lambda l: l.nm_hutchinson_diag(A, 1 << 31, 8, 8, A, 2, A, A, 1 << 62, None), 2),
     (lambda l: l.slide_pack(A, 4, 8, 7, A, None), 4),
     (lambda l: l.slide_pack(A, 4, 8, 12, A, None), 4),
     (lambda l: l.lift_activations(A, 4, 8, 8, 5, A, 8, None), 4),

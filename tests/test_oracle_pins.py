@@ -118,6 +118,27 @@ def test_hutchinson_single_sample_closed_form():
     assert np.array_equal(_bits_from_signs(signs), zb)
 
 
+def test_hutchinson_integer_inputs_against_exact_rationals():
+    # integer activations: N_k = sum_s z_s[k] (X^T X z_s)[k] is an exact
+    # integer (int64 here, by hand), D_k = N_k / (S T); the oracle's fp64
+    # loops round v / T once per sample and the sample sum S times
+    for (T, K, S, seed) in ((40, 70, 9, 1), (300, 33, 64, 2), (1, 5, 3, 3)):
+        X = datagen.small_int_bf16((T, K), seed=seed, tensor_id=3)
+        zb = datagen.rademacher_bits(S, K, seed=seed)
+        Xi = f32(X).astype(np.int64)
+        Z = np.array([[-1 if (zb[s, k // 32] >> (k % 32)) & 1 else 1 for k in range(K)] for s in range(S)],
+                     dtype=np.int64)
+        N = np.zeros(K, dtype=np.int64)
+        for s in range(S):
+            u = Xi @ Z[s]                         # X z_s
+            for k in range(K):
+                N[k] += Z[s, k] * int(Xi[:, k] @ u)
+        exact = np.array([float(Fraction(int(n), S * T)) for n in N])
+        D = oracle.hutchinson_diag(X, zb)
+        scale = (np.abs(Xi).T @ np.abs(Xi @ Z.T)).sum(axis=1) / (S * T)   # size of the rounded terms
+        assert np.all(np.abs(D - exact) <= (S + 3) * 2.0 ** -52 * (scale + np.abs(exact)))
+
+
 def test_hutchinson_converges_to_H():
     # unbiased with variance ~ 1/S: the error against H shrinks as S grows
     X = datagen.make_activations(200, 48, seed=8)
