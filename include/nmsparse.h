@@ -188,9 +188,9 @@ nm_status nm_hessian_rescale(const double *H, const double *s, int64_t K, double
  *           rounded up to 16, ldz = K rounded up to 8), [Z^T Z^T Z^T] as bf16
  *           [K x C3] (C3 = 3S rounded up to 64), the fp32 partials of U = X Z^T
  *           [nsplit x T x S16], U split into bf16 pieces [T x C3] and fp64
- *           partials of D [ceil(T/128) x K].  nsplit is the value in [1, min(8, ceil(K/64))]
- *           with the least ceil(n / 148) / n, n = ceil(T/128) * nsplit (the
- *           smaller on ties): CTAs spread evenly over a B200's 148 SMs.
+ *           partials of D [ceil(T/128) x K]; nsplit = min(8, ceil(K/64),
+ *           ceil(148 / ceil(T/128))).
+
  * Arithmetic (tensor cores, bf16 operands, fp32 accumulation): U = X Z^T
  * over K split into nsplit ranges, the partials added in ascending order;
  * each u split exactly into three bf16 pieces; P = Z^T U^T from the pieces;

@@ -56,42 +56,45 @@ __device__ __forceinline__ uint16_t sign_bf16(const uint32_t *__restrict__ zbits
     return ((__ldg(zbits + s * words + (k >> 5)) >> (k & 31)) & 1u) ? BF16_MINUS_ONE : BF16_ONE;
 }
 
-// Z [S16 x ldz] (rows past S zero) and Z3 [K x C3] (columns c < 3S hold
-// z_{c mod S}, the rest zero), both bf16, eight values (16 bytes) per thread
-__global__ void __launch_bounds__(256) k_hq_signs(const uint32_t *__restrict__ zbits, int S, int64_t K,
-                                                  int S16, int64_t ldz, int C3, uint16_t *__restrict__ Zb,
-                                                  uint16_t *__restrict__ Z3) {
+// Z [S16 x ldz] (rows past S zero), eight values (16 bytes) per thread
+__global__ void __launch_bounds__(256) k_hq_signs_z(const uint32_t *__restrict__ zbits, int S, int64_t K,
+                                                    int S16, int64_t ldz, uint16_t *__restrict__ Zb) {
     const int64_t words = (K + 31) / 32;
-    const int64_t zrow = ldz / 8, z3row = C3 / 8;
-    const int64_t nz = S16 * zrow, n3 = K * z3row;
+    const int64_t zrow = ldz / 8, nz = S16 * zrow;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nz + n3; i += stride) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nz; i += stride) {
+        const int64_t srow = i / zrow, k0 = (i - srow * zrow) * 8;
         uint32_t o[4] = {0u, 0u, 0u, 0u};
-        if (i < nz) {
-            const int64_t srow = i / zrow, k0 = (i - srow * zrow) * 8;
-            if (srow < S && k0 < K) {
-                const uint32_t bits = __ldg(zbits + srow * words + (k0 >> 5)) >> (k0 & 31);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint32_t v = (k0 + j < K) ? (((bits >> j) & 1u) ? BF16_MINUS_ONE : BF16_ONE) : 0u;
-                    o[j >> 1] |= v << (16 * (j & 1));
-                }
-            }
-            *reinterpret_cast<uint4 *>(Zb + i * 8) = make_uint4(o[0], o[1], o[2], o[3]);
-        } else {
-            const int64_t j3 = i - nz, k = j3 / z3row;
-            const int c0 = static_cast<int>(j3 - k * z3row) * 8;
-            const uint32_t *zk = zbits + (k >> 5);
-            const uint32_t sh = static_cast<uint32_t>(k & 31);
+        if (srow < S && k0 < K) {
+            const uint32_t bits = __ldg(zbits + srow * words + (k0 >> 5)) >> (k0 & 31);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const int c = c0 + j;
-                uint32_t v = 0u;
-                if (c < 3 * S) v = ((__ldg(zk + (c % S) * words) >> sh) & 1u) ? BF16_MINUS_ONE : BF16_ONE;
+                const uint32_t v = (k0 + j < K) ? (((bits >> j) & 1u) ? BF16_MINUS_ONE : BF16_ONE) : 0u;
                 o[j >> 1] |= v << (16 * (j & 1));
             }
-            *reinterpret_cast<uint4 *>(Z3 + j3 * 8) = make_uint4(o[0], o[1], o[2], o[3]);
         }
+        *reinterpret_cast<uint4 *>(Zb + i * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+// Z3 [K x C3]: row k = z_0..z_{S-1} at [k], three times, then zeros.  A block
+// holds 256 / S16 rows, one thread per (row, sample); sample slots past S
+// write the zero padding.
+__global__ void __launch_bounds__(256) k_hq_signs_z3(const uint32_t *__restrict__ zbits, int S, int64_t K,
+                                                     int S16, int C3, uint16_t *__restrict__ Z3) {
+    const int64_t words = (K + 31) / 32;
+    const int rpb = 256 / S16;
+    const int rl = threadIdx.x / S16, sidx = threadIdx.x - rl * S16;
+    if (rl >= rpb) return;
+    for (int64_t k = static_cast<int64_t>(blockIdx.x) * rpb + rl; k < K; k += static_cast<int64_t>(gridDim.x) * rpb) {
+        uint16_t *row = Z3 + k * C3;
+        if (sidx < S) {
+            const uint16_t v = ((__ldg(zbits + sidx * words + (k >> 5)) >> (k & 31)) & 1u) ? BF16_MINUS_ONE : BF16_ONE;
+            row[sidx] = v;
+            row[S + sidx] = v;
+            row[2 * S + sidx] = v;
+        }
+        for (int c = 3 * S + sidx; c < C3; c += S16) row[c] = 0;
     }
 }
 
@@ -204,30 +207,31 @@ __global__ void __launch_bounds__(HQ_THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Step 2: u = sum of the K-split partials (ascending); U3[t][c] = piece c / S
-// of u[t][c % S] for c < 3S (hi, mid, lo: u - hi and the next remainder are
-// exact in fp32), zero for the padding columns.  Block-strided rows, threads
-// over the columns of a row.
+// Step 2: u = sum of the K-split partials (ascending), split into three bf16
+// pieces hi, mid, lo (u - hi and the next remainder are exact in fp32) stored
+// at columns s, S + s, 2S + s of U3; the columns from 3S to C3 are zero.  A
+// block holds 256 / S16 tokens, one thread per (token, sample).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_hq_combine(const float *__restrict__ Up, int64_t T, int S, int S16,
                                                     int nsplit, int C3, uint16_t *__restrict__ U3) {
-    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-        for (int c = threadIdx.x; c < C3; c += blockDim.x) {
-            uint16_t out = 0;
-            if (c < 3 * S) {
-                const int sidx = c % S, piece = c / S;
-                float u = Up[t * S16 + sidx];
-                for (int q = 1; q < nsplit; ++q) u = __fadd_rn(u, Up[(q * T + t) * S16 + sidx]);
-                const __nv_bfloat16 hi = __float2bfloat16_rn(u);
-                const float r1 = __fsub_rn(u, __bfloat162float(hi));
-                const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-                const float r2 = __fsub_rn(r1, __bfloat162float(mid));
-                const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
-                const __nv_bfloat16 pick = piece == 0 ? hi : (piece == 1 ? mid : lo);
-                out = *reinterpret_cast<const uint16_t *>(&pick);
-            }
-            U3[t * C3 + c] = out;
+    const int tpb = 256 / S16;
+    const int tl = threadIdx.x / S16, sidx = threadIdx.x - tl * S16;
+    if (tl >= tpb) return;
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * tpb + tl; t < T; t += static_cast<int64_t>(gridDim.x) * tpb) {
+        uint16_t *row = U3 + t * C3;
+        if (sidx < S) {
+            float u = Up[t * S16 + sidx];
+            for (int q = 1; q < nsplit; ++q) u = __fadd_rn(u, Up[(q * T + t) * S16 + sidx]);
+            const __nv_bfloat16 hi = __float2bfloat16_rn(u);
+            const float r1 = __fsub_rn(u, __bfloat162float(hi));
+            const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+            const float r2 = __fsub_rn(r1, __bfloat162float(mid));
+            const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+            row[sidx] = *reinterpret_cast<const uint16_t *>(&hi);
+            row[S + sidx] = *reinterpret_cast<const uint16_t *>(&mid);
+            row[2 * S + sidx] = *reinterpret_cast<const uint16_t *>(&lo);
         }
+        for (int c = 3 * S + sidx; c < C3; c += S16) row[c] = 0;
     }
 }
 
@@ -440,15 +444,12 @@ HqGeom hq_geometry(int64_t T, int64_t K, int64_t S) {
     g.nkb = (K + 63) / 64;
     g.ttiles = (T + HQ_M - 1) / HQ_M;
     g.ktiles = (K + HQ_M - 1) / HQ_M;
-    // K-split of step 1: the count whose CTAs spread most evenly over 148
-    // SMs (least ceil(n / 148) / n for n = ttiles * nsplit), the smaller on ties
-    const int64_t smax = g.nkb < HQ_MAX_SPLIT ? g.nkb : HQ_MAX_SPLIT;
-    g.nsplit = 1;
-    for (int64_t ns = 2; ns <= smax; ++ns) {
-        const int64_t n = g.ttiles * ns, nb = g.ttiles * g.nsplit;
-        const int64_t w = (n + HQ_TARGET_CTAS - 1) / HQ_TARGET_CTAS, wb = (nb + HQ_TARGET_CTAS - 1) / HQ_TARGET_CTAS;
-        if (w * nb < wb * n) g.nsplit = ns;
-    }
+    // K-split of step 1: enough CTAs to cover 148 SMs, at most 8 and at most
+    // one per 64-column block
+    int64_t ns = (HQ_TARGET_CTAS + g.ttiles - 1) / g.ttiles;
+    ns = ns > HQ_MAX_SPLIT ? HQ_MAX_SPLIT : ns;
+    ns = ns > g.nkb ? g.nkb : ns;
+    g.nsplit = ns < 1 ? 1 : ns;
     size_t off = align1k(static_cast<size_t>(g.S16 * g.ldz) * 2);
     g.off_z3 = off;
     off += align1k(static_cast<size_t>(K * g.C3) * 2);
@@ -519,12 +520,17 @@ extern "C" nm_status nm_hutchinson_diag(const uint16_t *X, int64_t T, int64_t K,
         !set_smem_attr<k_hq_p>(HQ2_SMEM_BYTES))
         return NM_ERR_CUDA;
 
-    const int64_t nsig = g.S16 * g.ldz / 8 + K * g.C3 / 8;
-    k_hq_signs<<<static_cast<unsigned>((nsig + 255) / 256 < 4096 ? (nsig + 255) / 256 : 4096), 256, 0, st>>>(
-        zbits, static_cast<int>(S), K, static_cast<int>(g.S16), g.ldz, static_cast<int>(g.C3), Zb, Z3);
+    const int64_t nz = g.S16 * g.ldz / 8;
+    k_hq_signs_z<<<static_cast<unsigned>((nz + 255) / 256 < 1024 ? (nz + 255) / 256 : 1024), 256, 0, st>>>(
+        zbits, static_cast<int>(S), K, static_cast<int>(g.S16), g.ldz, Zb);
+    const int64_t rpb = 256 / g.S16;
+    const int64_t zblocks = (K + rpb - 1) / rpb;
+    k_hq_signs_z3<<<static_cast<unsigned>(zblocks < 4096 ? zblocks : 4096), 256, 0, st>>>(
+        zbits, static_cast<int>(S), K, static_cast<int>(g.S16), static_cast<int>(g.C3), Z3);
     k_hq_u<<<dim3(static_cast<unsigned>(g.ttiles), static_cast<unsigned>(g.nsplit)), HQ_THREADS, smem1, st>>>(
         tmX1, tmZ, T, g.nkb, static_cast<int>(g.nsplit), static_cast<int>(g.S16), stages, stage_bytes, tcols, Up);
-    k_hq_combine<<<static_cast<unsigned>(T < 16384 ? T : 16384), 256, 0, st>>>(
+    const int64_t cblocks = (T + rpb - 1) / rpb;
+    k_hq_combine<<<static_cast<unsigned>(cblocks < 8192 ? cblocks : 8192), 256, 0, st>>>(
         Up, T, static_cast<int>(S), static_cast<int>(g.S16), static_cast<int>(g.nsplit), static_cast<int>(g.C3),
         U3);
     const int64_t units = g.ktiles * g.ttiles;

@@ -2,7 +2,6 @@
 sm_100a, loads, exports every function include/nmsparse.h declares, and its
 argument validation rejects bad calls before launching anything."""
 import ctypes
-from fractions import Fraction
 import os
 import re
 
@@ -64,15 +63,12 @@ def test_size_queries():
     assert lib.nm_dense_gemm_workspace_bytes(16, 4096, 4096) == sk
     assert lib.nm_dense_gemm_workspace_bytes(16, 0, 4096) == 0
     # Z [S16 x ldz], [Z^T Z^T Z^T] [K x C3], U partials [nsplit x T x S16] fp32,
-    # U pieces [T x C3] bf16, D partials [T/128 x K] fp64, each padded to
-    # 1 KiB; nsplit in [1, min(8, K/64)] the
-    # one with least ceil(n/148)/n for n = T/128 * nsplit, the smaller on ties
+    # U pieces [T x C3] bf16, D partials [T/128 x K] fp64, each padded to 1 KiB
     k1 = lambda b: (b + 1023) // 1024 * 1024
 
     def hq(T, K, S):
         S16, C3, ldz, tt = (S + 15) // 16 * 16, (3 * S + 63) // 64 * 64, (K + 7) // 8 * 8, (T + 127) // 128
-        cost = lambda ns: Fraction(-(-tt * ns // 148), tt * ns)
-        ns = min(range(1, min(8, (K + 63) // 64) + 1), key=lambda n: (cost(n), n))
+        ns = max(1, min(8, (K + 63) // 64, (148 + tt - 1) // tt))
         return (k1(S16 * ldz * 2) + k1(K * C3 * 2) + k1(ns * T * S16 * 4) + k1(T * C3 * 2)
                 + k1(tt * K * 8))
     assert lib.nm_hutchinson_workspace_bytes(300, 1000, 7) == hq(300, 1000, 7)
