@@ -19,6 +19,9 @@ Function -> passage it follows (page title, section):
   lift             SlideSparse sec. 2B, activation lifting
   gemm_*           Y = X * W_sparse^T in fp64
   ternary          Sparse-BitNet sec. 1, ternary absmean quantisation
+  e4m3_*, quant_lift_f8, quant_rows_f8, gemm_f8
+                   SlideSparse sec. 2B / 2C: per-token FP8 quantisation fused
+                   with the lift, FP8 weights, the GEMM on dequantised codes
 
 Every function here has a pin in tests/test_oracle_pins.py; none is unpinned.
 """
@@ -62,6 +65,10 @@ def _load():
             sig = {
                 "oracle_hessian_diag": (None, [P, I64, I64, I64, P]),
                 "oracle_hessian_rescale": (None, [P, P, I64, P]),
+                "oracle_e4m3_value": (D, [ctypes.c_uint8]),
+                "oracle_e4m3_encode": (ctypes.c_uint8, [ctypes.c_float]),
+                "oracle_quant_lift_f8": (I, [P, I64, I64, I64, I, I64, P, P]),
+                "oracle_quant_rows_f8": (None, [P, I64, I64, P, P]),
                 "oracle_hutchinson_diag": (None, [P, I64, I64, I64, P, I64, P]),
                 "oracle_hessian_diag_naive": (None, [P, I64, I64, I64, P]),
                 "oracle_score_hessian": (None, [P, D, P, I64, I64, I64, P]),
@@ -277,3 +284,62 @@ def run_layer(X, W, n, m, eps=1e-8, score="hessian", ternary_values=False):
     mask, vals, meta = prune(S, V, n, m)
     wmeta = slide_pack(mask, W.shape[1], m) if (m % 2 == 0 and n == m - 2) else None
     return dict(H=H, S=S, mask=mask, vals=vals, meta24=meta, wmeta=wmeta, V=V)
+
+
+def e4m3_value(code: int) -> float:
+    return _load().oracle_e4m3_value(code)
+
+
+def e4m3_encode(x: float) -> int:
+    return _load().oracle_e4m3_encode(x)
+
+
+def e4m3_table() -> np.ndarray:
+    """fp64 value of each of the 256 codes (NaN for 0x7F and 0xFF)."""
+    t = np.array([e4m3_value(c) for c in range(256)])
+    t[0x7F] = t[0xFF] = np.nan
+    return t
+
+
+def lifted_cols_f8(K: int, m: int) -> int:
+    """Lifted width rounded up to the FP8 GEMM's 256-column K' block."""
+    return (lifted_cols(K, m) + 255) // 256 * 256
+
+
+def quant_lift_f8(X: np.ndarray, m: int, ldq: int | None = None):
+    """Per-token E4M3 codes of the lifted activations and the fp32 scales."""
+    X = _c(X, np.uint16)
+    T, K = X.shape
+    ldq = lifted_cols_f8(K, m) if ldq is None else ldq
+    Q = np.empty((T, ldq), dtype=np.uint8)
+    sc = np.empty(T, dtype=np.float32)
+    if _load().oracle_quant_lift_f8(_p(X), T, K, K, m, ldq, _p(Q), _p(sc)) != 0:
+        raise ValueError("oracle_quant_lift_f8: unsupported m or ldq")
+    return Q, sc
+
+
+def quant_rows_f8(V: np.ndarray):
+    """Per-row E4M3 codes of kept weight values [R x L] and the fp32 scales."""
+    V = _c(V, np.uint16)
+    R, L = V.shape
+    Q = np.empty((R, L), dtype=np.uint8)
+    sc = np.empty(R, dtype=np.float32)
+    _load().oracle_quant_rows_f8(_p(V), R, L, _p(Q), _p(sc))
+    return Q, sc
+
+
+def gemm_f8(Xq, xs, mask, Wq, ws, K, m, rows=None) -> np.ndarray:
+    """Y64[t, r] = xs[t] ws[r] sum over kept k of e4m3(Xq[t, k]) e4m3(Wq[r, j(k)])
+    in fp64, Xq being the per-token codes of X in its own column order (the
+    lift only duplicates columns, so each lifted code equals one of these)."""
+    tab = e4m3_table()
+    T = Xq.shape[0]
+    sel = np.arange(T) if rows is None else np.asarray(rows)
+    Xd = tab[Xq[sel, :K]]
+    R = Wq.shape[0]
+    words = _c(mask, np.uint32)
+    bits = ((words[:, :, None] >> np.arange(32, dtype=np.uint32)) & 1).reshape(R, -1)[:, :K].astype(bool)
+    Wd = np.zeros((R, K))
+    for r in range(R):
+        Wd[r, bits[r]] = tab[Wq[r, : bits[r].sum()]]
+    return (Xd @ Wd.T) * xs[sel, None].astype(np.float64) * ws[None, :].astype(np.float64)

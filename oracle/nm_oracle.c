@@ -462,4 +462,82 @@ double oracle_ternary(const uint16_t *W, int64_t R, int64_t K, int64_t ldw, uint
 }
 
 /* Exposed for tests of the rounding helper. */
+/* ------------------------------------------------------------------------ */
+/* FP8 path (SlideSparse sec. 2B: the lift is fused into the per-token
+ * INT8/FP8/FP4 quantisation of the activations; sec. 2C: online, one fused
+ * quantise-and-lift kernel, then the sparse GEMM).  Format: E4M3 -- sign,
+ * 4 exponent bits (bias 7), 3 mantissa bits; code e > 0 has the value
+ * 2^(e-7) (1 + m/8), code e = 0 the value m 2^-9; e = 15, m = 7 is NaN, so
+ * the largest finite value is 448 (code 0x7E).  Rounding: to the nearest
+ * finite value, ties to the even code, magnitudes beyond 448 clamp to 448.
+ * Scales (a reading: the pages fix no scale rule): per token (activations)
+ * and per weight row, scale = amax / 448 in fp32 (1 when amax = 0); a value
+ * x becomes the code of fp32(x / scale).                                     */
+double oracle_e4m3_value(uint8_t c) {
+    const int e = (c >> 3) & 15, mant = c & 7;
+    const double v = e == 0 ? ldexp((double)mant, -9) : ldexp(1.0 + mant / 8.0, e - 7);
+    return (c & 0x80) ? -v : v;
+}
+
+/* nearest finite E4M3 code by search over all 127 non-negative codes; codes
+ * are monotone in value and the last code bit is the last mantissa bit, so
+ * "even" is "code bit 0 clear" */
+uint8_t oracle_e4m3_encode(float x) {
+    const double a = fabs((double)x);
+    uint8_t best = 0;
+    double bd = a;
+    for (int c = 1; c <= 0x7E; ++c) {
+        const double d = fabs(oracle_e4m3_value((uint8_t)c) - a);
+        if (d < bd || (d == bd && (c & 1) == 0)) { bd = d; best = (uint8_t)c; }
+    }
+    return signbit(x) ? (uint8_t)(best | 0x80) : best;
+}
+
+static float f8_scale(float amax) { return amax > 0.0f ? amax / 448.0f : 1.0f; }
+
+/* lifted activations (natural window order, as oracle_lift) quantised per
+ * token: Q [T x ldq] codes, columns past the lifted width zero; scale [T] */
+int oracle_quant_lift_f8(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, int m, int64_t ldq, uint8_t *Q,
+                         float *scale) {
+    if (m < 4 || m % 2) return -1;
+    const int Ns = m / 2;
+    const int64_t G = groups_of(K, m);
+    const int64_t KL = G * (Ns - 1) * 4;
+    if (ldq < KL) return -1;
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            const float v = fabsf(bf16_to_f32(X[t * ldx + k]));
+            if (v > amax) amax = v;
+        }
+        const float s = f8_scale(amax);
+        scale[t] = s;
+        for (int64_t c = 0; c < ldq; ++c) Q[t * ldq + c] = 0;
+        for (int64_t g = 0; g < G; ++g)
+            for (int w = 0; w < Ns - 1; ++w)
+                for (int c = 0; c < 4; ++c) {
+                    const int64_t src = g * m + 2 * w + c;
+                    const float v = src < K ? bf16_to_f32(X[t * ldx + src]) : 0.0f;
+                    Q[t * ldq + g * (Ns - 1) * 4 + 4 * w + c] = oracle_e4m3_encode(v / s);
+                }
+    }
+    return 0;
+}
+
+/* kept weight values [R x L] (bf16) quantised per row: Q [R x L], scale [R] */
+void oracle_quant_rows_f8(const uint16_t *V, int64_t R, int64_t L, uint8_t *Q, float *scale) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r) {
+        float amax = 0.0f;
+        for (int64_t j = 0; j < L; ++j) {
+            const float v = fabsf(bf16_to_f32(V[r * L + j]));
+            if (v > amax) amax = v;
+        }
+        const float s = f8_scale(amax);
+        scale[r] = s;
+        for (int64_t j = 0; j < L; ++j) Q[r * L + j] = oracle_e4m3_encode(bf16_to_f32(V[r * L + j]) / s);
+    }
+}
+
 uint16_t oracle_f64_to_bf16(double v) { return f64_to_bf16_rne(v); }

@@ -29,6 +29,8 @@ MUTATIONS = [
      "double p = bf16_to_f64(X[k * ldx + t]) * bf16_to_f64(V[r * ldv + k]);"),  # transposed
     ("s[q] = 0.0f; /* zero-padded tail */", "s[q] = 1e30f;"),              # padding wins
     ("double q = rint(", "double q = round("),                             # ties away
+    ("(d == bd && (c & 1) == 0)", "(d == bd && (c & 1) == 1)"),           # e4m3 ties to odd
+    ("amax > 0.0f ? amax / 448.0f", "amax > 0.0f ? amax / 447.0f"),       # fp8 scale
 ]
 
 

@@ -490,3 +490,84 @@ def test_f64_to_bf16_rounding():
     # agrees with fp32 rounding where no double rounding can occur
     for v in (0.0123, 3.75, 1e-3, 123.456):
         assert oracle.f64_to_bf16(v) == int(datagen.f32_to_bf16_bits(np.array([v], dtype=np.float32))[0])
+
+
+# --------------------------------------------------------------------------
+# FP8 (E4M3) quantisation fused with the lift (SlideSparse sec. 2B / 2C)
+def _e4m3_positive_values():
+    return np.array([oracle.e4m3_value(c) for c in range(0x7F)])
+
+
+def test_e4m3_format_values():
+    v = _e4m3_positive_values()
+    assert v[0] == 0.0 and v[1] == 2.0 ** -9 and v[7] == 7 * 2.0 ** -9     # subnormals m 2^-9
+    assert v[8] == 2.0 ** -6 and v[0x38] == 1.0 and v[0x7E] == 448.0       # normals, largest finite
+    assert np.all(np.diff(v) > 0)                                          # codes are monotone
+    assert oracle.e4m3_value(0xB8) == -1.0
+
+
+def test_e4m3_rounding_round_trip_ties_and_saturation():
+    v = _e4m3_positive_values()
+    for c in range(0x7F):
+        assert oracle.e4m3_encode(float(v[c])) == c
+        assert oracle.e4m3_encode(-float(v[c])) == c | 0x80
+    for c in range(0x7E):
+        mid = np.float32((v[c] + v[c + 1]) / 2)              # exact in fp32
+        assert float(mid) == (v[c] + v[c + 1]) / 2
+        assert oracle.e4m3_encode(float(mid)) == (c if c % 2 == 0 else c + 1)   # ties to even
+        assert oracle.e4m3_encode(float(np.nextafter(mid, np.float32(1e9)))) == c + 1
+        assert oracle.e4m3_encode(float(np.nextafter(mid, np.float32(0)))) == c
+    for big in (448.5, 464.0, 479.0, 1e30):
+        assert oracle.e4m3_encode(big) == 0x7E and oracle.e4m3_encode(-big) == 0xFE
+    assert oracle.e4m3_encode(0.0) == 0 and oracle.e4m3_encode(-0.0) == 0x80
+
+
+def test_e4m3_matches_torch_cast_in_range():
+    torch = pytest.importorskip("torch")
+    g = np.random.default_rng(0)
+    x = np.concatenate([g.normal(0, 60, 4000), g.normal(0, 1e-2, 2000), g.uniform(-448, 448, 2000)]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    ours = np.array([oracle.e4m3_encode(float(a)) for a in x], dtype=np.uint8)
+    assert np.array_equal(ours, ref)
+
+
+def test_quant_lift_f8_scale_duplication_and_padding():
+    X = datagen.make_activations(20, 30, seed=3, n_outliers=2)
+    X[5] = 0                                                  # an all-zero token
+    Q4, s4 = oracle.quant_lift_f8(X, 4)
+    Q8, s8 = oracle.quant_lift_f8(X, 8)
+    assert np.array_equal(s4, s8)
+    amax = np.abs(f32(X)).max(axis=1)
+    assert np.array_equal(s4[amax > 0], (amax[amax > 0] / np.float32(448)).astype(np.float32))
+    assert s4[5] == 1.0 and not Q4[5].any()
+    for t in range(20):                                        # the largest magnitude maps to +-448
+        if amax[t] > 0:
+            k = int(np.argmax(np.abs(f32(X[t]))))
+            assert Q4[t, k] & 0x7F == 0x7E
+    assert Q4.shape[1] == 256 and not Q4[:, 32:].any()        # identity lift, zero padding
+    # 6:8 lift: group g, window w, column c holds source column 8g + 2w + c
+    for g in range(4):
+        for w in range(3):
+            for c in range(4):
+                src = 8 * g + 2 * w + c
+                col = g * 12 + 4 * w + c
+                assert np.array_equal(Q8[:, col], Q4[:, src] if src < 30 else np.zeros(20, np.uint8))
+
+
+def test_gemm_f8_exact_when_codes_are_exact():
+    # each token and weight row holds a 448 (scale 1) and small integers (exact
+    # E4M3 codes): the FP8 GEMM equals the exact product of the bf16 values
+    T, K, R, m = 9, 64, 7, 8
+    g = np.random.default_rng(1)
+    X = bf16(g.integers(-8, 9, size=(T, K)).astype(np.float32))
+    X[:, 3] = bf16(np.full(T, 448.0, np.float32))
+    W = bf16(g.integers(-8, 9, size=(R, K)).astype(np.float32))
+    W[:, 5] = bf16(np.full(R, -448.0, np.float32))
+    res = oracle.run_layer(X, W, m - 2, m, score="magnitude")
+    Xq, xs = oracle.quant_lift_f8(X, 4)
+    Wq, ws = oracle.quant_rows_f8(res["vals"])
+    if not np.any(f32(res["vals"]) == -448.0):
+        pytest.skip("the -448 column was pruned in some row")
+    assert np.all(xs == 1.0) and np.all(ws == 1.0)
+    Y = oracle.gemm_f8(Xq, xs, res["mask"], Wq, ws, K, m)
+    assert np.array_equal(Y, oracle.gemm_masked(X, res["mask"], W, m))
