@@ -581,6 +581,74 @@ def run_prep(args):
     print(json.dumps(out), flush=True)
 
 
+def run_f8(args):
+    """The FP8 form of the layer (SlideSparse sec. 2B/2C): the fused per-token
+    quantise + lift kernel and the kind::f8f6f4 sparse GEMM, each launched
+    alone and timed with CUDA events (L2 flushed), next to the bf16 sparse
+    GEMM on the same layer.  One JSON line."""
+    import torch
+
+    import semi_structured_sparse_diag_b200 as nm
+    lib = nm.load()
+    dev = torch.device("cuda", 0)
+    layer = datagen.WORKLOADS[args.workload]
+    X_h, W_h = datagen.layer_inputs(layer)
+    R, K, m = layer.R, layer.K, layer.m
+    T = X_h.shape[0]
+    W = torch.from_numpy(W_h.view(np.int16)).to(dev).view(torch.bfloat16)
+    X = torch.from_numpy(X_h.view(np.int16)).to(dev).view(torch.bfloat16)
+    H = nm.hessian_diag(X)
+    mask, vals, meta24 = nm.score_prune_compress(H, W, m - 2, m, eps=layer.eps)
+    wmeta = meta24 if m == 4 else nm.slide_pack(mask, K, m)
+    packed8 = nm.sparse_prepare_f8(vals, wmeta, R, K, m)
+    packed16 = nm.sparse_prepare(vals, wmeta, R, K, m)
+    Xq, xs = nm.quant_lift_f8(X, m)
+    Y8 = nm.sparse_gemm_f8(Xq, xs, packed8, R, K, m)
+    Y16 = nm.sparse_gemm(X, packed16, R, m)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    s = torch.cuda.current_stream().cuda_stream
+    KLf = lib.nm_lifted_cols_f8(K, m)
+
+    def timed(fn):
+        ts = []
+        for i in range(args.reps + 1):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if i:
+                ts.append(e0.elapsed_time(e1) * 1000)
+        return sorted(ts)[len(ts) // 2] if ts else float("nan")
+
+    def chk(st, what):
+        if st != 0:
+            raise nm.NMError(f"{what}: {lib.nm_status_string(st).decode()}")
+
+    q_us = timed(lambda: chk(lib.nm_quant_lift_f8(X.data_ptr(), T, K, K, m, Xq.data_ptr(), Xq.shape[1],
+                                                  xs.data_ptr(), s), "quant_lift_f8"))
+    g8_us = timed(lambda: chk(lib.nm_sparse_gemm_f8(Xq.data_ptr(), T, K, Xq.shape[1], xs.data_ptr(),
+                                                    packed8.data_ptr(), R, m, Y8.data_ptr(), Y8.stride(0), s),
+                              "sparse_gemm_f8"))
+    g16_us = timed(lambda: nm.sparse_gemm(X, packed16, R, m, Y=Y16))
+    nm.check_device_error()
+    hbm, bf16_peak, _src = peaks()
+    f8_sparse_peak = 2 * 2 * bf16_peak   # fp8 dense = 2 x bf16 dense (nominal ratio); 2:4 doubles it
+    flops8 = 2.0 * T * R * KLf            # dense-equivalent on the lifted K'
+    out = {"f8": layer.name, "R": R, "K": K, "T": T, "pattern": f"{m - 2}:{m}", "lifted_K_f8": KLf,
+           "us": {"quant_lift_f8": round(q_us, 1), "sparse_gemm_f8": round(g8_us, 1),
+                  "sparse_gemm_bf16": round(g16_us, 1)},
+           "quant_lift_f8_GBs": round((2 * T * K + T * KLf + 4 * T) / q_us / 1e3, 0),
+           "quant_lift_f8_pct_hbm": round(100 * (2 * T * K + T * KLf + 4 * T) / q_us / 1e3 / hbm, 1),
+           "gemm_f8_TFLOPs_on_lifted": round(flops8 / g8_us / 1e6, 1),
+           "gemm_f8_pct_of_f8_2to4_peak": round(100 * flops8 / g8_us / 1e6 / f8_sparse_peak, 1),
+           "f8_2to4_peak_TFLOPs": f8_sparse_peak, "peak_source": "2 x 2 x measured dense bf16 burst",
+           "effective_TFLOPs_on_K": {"f8": round(2.0 * T * R * K / g8_us / 1e6, 1),
+                                     "bf16": round(2.0 * T * R * K / g16_us / 1e6, 1)}}
+    print(json.dumps(out), flush=True)
+
+
 def run_probe(args):
     """Tensor-pipe and HBM probes (calibration, not the bench line)."""
     import torch
@@ -723,10 +791,13 @@ def main():
     ap.add_argument("--probe", action="store_true", help="run the tensor-pipe / HBM probes instead")
     ap.add_argument("--ablation", action="store_true", help="time the GEMM variants instead")
     ap.add_argument("--prep", action="store_true", help="time the HBM-bound prep kernels instead")
-    ap.add_argument("--reps", type=int, default=5, help="--prep: timed launches per kernel")
+    ap.add_argument("--reps", type=int, default=5, help="--prep / --f8: timed launches per kernel")
+    ap.add_argument("--f8", action="store_true", help="time the FP8 quantise+lift and FP8 sparse GEMM instead")
     args = ap.parse_args()
     if args.prep:
         return run_prep(args)
+    if args.f8:
+        return run_f8(args)
     if args.probe:
         run_probe(args)
         return

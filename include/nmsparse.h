@@ -203,6 +203,43 @@ size_t nm_hutchinson_workspace_bytes(int64_t T, int64_t K, int64_t S);
 nm_status nm_hutchinson_diag(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, const uint32_t *zbits,
                              int64_t S, double *D, void *ws, size_t ws_bytes, void *stream);
 
+/* ------------------------------------------------------------------------ */
+/* FP8 path (SlideSparse, arXiv 2603.05232, sec. 2B: the activation lift is
+ * fused into the per-token INT8/FP8/FP4 quantisation kernel; sec. 2C: online,
+ * the fused quantise-and-lift kernel, then the sparse GEMM).  Format E4M3
+ * (largest finite 448); codes are fp32(x / scale) rounded to nearest even,
+ * saturating; scale = amax / 448 in fp32 (1 when amax is 0), per token for
+ * the activations and per weight row (over its kept values) for the weights.
+ * m in {4, 6, 8, 10} (2:4 and the (2N-2):2N patterns); the lifted columns are
+ * in natural window order (window w of group g = columns g m + 2w .. + 3),
+ * padded with zero codes to KLf = nm_lifted_cols_f8(K, m), a multiple of 256.
+ *
+ * nm_quant_lift_f8: X bf16 [T x ldx] (16-byte aligned, ldx % 8 == 0) ->
+ *   Xq E4M3 codes [T x ldq] (16-byte aligned, ldq % 16 == 0, ldq >= KLf; all
+ *   ldq columns are written, zero past the lifted width) and xscale fp32 [T].
+ * nm_sparse_prepare_f8: vals [R x G n] bf16 and window metadata wmeta
+ *   (meta24 for m = 4; nm_slide_pack's for m > 4, one nibble per window, row
+ *   stride ceil(windows / 2) bytes) -> packed: codes [Rpad x KLf/2] (Rpad = R
+ *   rounded up to 128; the kept order is the window order), then metadata
+ *   blocks of 4096 bytes per (128-row tile, 256-column K' block) = two atoms
+ *   of [128 rows x 16 bytes] (row-major; byte i of atom a of block kb holds the
+ *   nibbles of windows 64 kb + 32 a + 2i (low) and + 1 (high)), then the row
+ *   scales fp32 [Rpad].  Size: nm_sparse_prepare_f8_bytes(R, K, m).
+ * nm_sparse_gemm_f8: Y[t, r] = bf16(xscale[t] ws[r] sum E4M3 products), the
+ *   products accumulated in fp32 by tcgen05.mma.sp kind::f8f6f4; Y bf16
+ *   [T x ldy], ldy % 8 == 0, ldy >= R.
+ * Errors: NULL -> NM_ERR_NULL; other m -> NM_ERR_UNSUPPORTED; sizes, ld too
+ * small -> NM_ERR_SHAPE; alignment -> NM_ERR_ALIGN; short packed buffer ->
+ * NM_ERR_WORKSPACE.                                                         */
+int64_t nm_lifted_cols_f8(int64_t K, int m);
+size_t nm_sparse_prepare_f8_bytes(int64_t R, int64_t K, int m);
+nm_status nm_quant_lift_f8(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, int m, uint8_t *Xq, int64_t ldq,
+                           float *xscale, void *stream);
+nm_status nm_sparse_prepare_f8(const uint16_t *vals, const uint8_t *wmeta, int64_t R, int64_t K, int m,
+                               void *packed, size_t packed_bytes, void *stream);
+nm_status nm_sparse_gemm_f8(const uint8_t *Xq, int64_t T, int64_t K, int64_t ldq, const float *xscale,
+                            const void *packed, int64_t R, int m, uint16_t *Y, int64_t ldy, void *stream);
+
 /* a2 + a3 fused: exactly nm_score_from_hessian followed by nm_prune_compress
  * (bit-identical mask, vals and meta24), with each score formed in registers
  * from W -- fp32((H_j + eps) * W_ij^2), fp64 add and multiplies, rounded once;

@@ -20,7 +20,8 @@ from . import build as _build
 
 __all__ = [
     "NMError", "load", "hessian_diag", "score", "score_from_hessian", "prune_compress",
-    "score_prune_compress", "hessian_rescale", "hutchinson_diag", "slide_pack", "lift_activations", "sparse_prepare", "sparse_gemm", "dense_gemm",
+    "score_prune_compress", "hessian_rescale", "hutchinson_diag", "quant_lift_f8", "sparse_prepare_f8",
+    "sparse_gemm_f8", "slide_pack", "lift_activations", "sparse_prepare", "sparse_gemm", "dense_gemm",
     "ternary_quantize", "check_device_error", "set_gemm_schedule", "EXPORTED",
 ]
 
@@ -32,7 +33,8 @@ EXPORTED = (
     "nm_ternary_quantize", "nm_hessian_diag_noalloc", "nm_probe_mma", "nm_probe_copy", "nm_gemm_1cta", "nm_sparse_gemm_workspace_bytes",
     "nm_sparse_gemm_fused", "nm_dense_gemm_workspace_bytes", "nm_gemm_set_schedule",
     "nm_sparse_gemm_tile256", "nm_score_prune_compress", "nm_hessian_rescale",
-    "nm_hutchinson_workspace_bytes", "nm_hutchinson_diag",
+    "nm_hutchinson_workspace_bytes", "nm_hutchinson_diag", "nm_lifted_cols_f8", "nm_sparse_prepare_f8_bytes",
+    "nm_quant_lift_f8", "nm_sparse_prepare_f8", "nm_sparse_gemm_f8",
 )
 
 _P, _I64, _I, _D, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_size_t
@@ -48,6 +50,11 @@ _SIGS = {
     "nm_hessian_rescale": (_I, [_P, _P, _I64, _P, _P]),
     "nm_hutchinson_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
     "nm_hutchinson_diag": (_I, [_P, _I64, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
+    "nm_lifted_cols_f8": (_I64, [_I64, _I]),
+    "nm_sparse_prepare_f8_bytes": (_SZ, [_I64, _I64, _I]),
+    "nm_quant_lift_f8": (_I, [_P, _I64, _I64, _I64, _I, _P, _I64, _P, _P]),
+    "nm_sparse_prepare_f8": (_I, [_P, _P, _I64, _I64, _I, _P, _SZ, _P]),
+    "nm_sparse_gemm_f8": (_I, [_P, _I64, _I64, _I64, _P, _P, _I64, _I, _P, _I64, _P]),
     "nm_score_prune_compress": (_I, [_P, _D, _P, _I64, _P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P]),
     "slide_pack": (_I, [_P, _I64, _I64, _I, _P, _P]),
     "lift_activations": (_I, [_P, _I64, _I64, _I64, _I, _P, _I64, _P]),
@@ -232,6 +239,49 @@ def hutchinson_diag(X, zbits, D=None, ws=None, stream=None):
     _check(lib.nm_hutchinson_diag(_ptr(X), T, K, _ld(X), _ptr(zbits), S, _ptr(D), _ptr(ws),
                                   ws.numel() * ws.element_size(), _stream(stream)), "nm_hutchinson_diag")
     return D
+
+
+def quant_lift_f8(X, m, ldq=None, stream=None):
+    """Per-token E4M3 codes of the lifted activations: (Xq uint8 [T x ldq],
+    xscale fp32 [T]); ldq defaults to nm_lifted_cols_f8(K, m)."""
+    X = _bf16(X, "X")
+    T, K = X.shape
+    lib = load()
+    KLf = lib.nm_lifted_cols_f8(K, m)
+    if KLf == 0:
+        raise NMError(f"unsupported pattern m={m} for the FP8 path")
+    ldq = KLf if ldq is None else ldq
+    Xq = torch.empty((T, ldq), dtype=torch.uint8, device=X.device)
+    xs = torch.empty(T, dtype=torch.float32, device=X.device)
+    _check(lib.nm_quant_lift_f8(_ptr(X), T, K, _ld(X), m, _ptr(Xq), ldq, _ptr(xs), _stream(stream)),
+           "nm_quant_lift_f8")
+    return Xq, xs
+
+
+def sparse_prepare_f8(vals, wmeta, R, K, m, stream=None):
+    """FP8 GEMM operand from the kept values and window metadata (meta24 for
+    2:4): codes, kind::f8f6f4 metadata blocks and row scales in one buffer."""
+    _dev(vals, "vals")
+    _dev(wmeta, "wmeta")
+    lib = load()
+    nbytes = lib.nm_sparse_prepare_f8_bytes(R, K, m)
+    if nbytes == 0:
+        raise NMError(f"unsupported shape or pattern for the FP8 path (R={R}, K={K}, m={m})")
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=vals.device)
+    _check(lib.nm_sparse_prepare_f8(_ptr(vals), _ptr(wmeta), R, K, m, _ptr(packed), nbytes, _stream(stream)),
+           "nm_sparse_prepare_f8")
+    return packed
+
+
+def sparse_gemm_f8(Xq, xscale, packed, R, K, m, Y=None, stream=None):
+    """Y = (xscale ws) * (E4M3 lifted activations x E4M3 packed weights^T), bf16."""
+    _dev(Xq, "Xq")
+    T, ldq = Xq.shape
+    if Y is None:
+        Y = torch.empty((T, (R + 7) // 8 * 8), dtype=torch.bfloat16, device=Xq.device)[:, :R]
+    _check(load().nm_sparse_gemm_f8(_ptr(Xq), T, K, ldq, _ptr(xscale), _ptr(packed), R, m, _ptr(Y), _ld(Y),
+                                    _stream(stream)), "nm_sparse_gemm_f8")
+    return Y
 
 
 def score_prune_compress(H, W, n, m, V=None, eps=1e-8, stream=None):

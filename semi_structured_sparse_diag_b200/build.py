@@ -9,7 +9,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libnmsparse.so")
-SOURCES = ["nm_api.cu", "nm_prune.cu", "nm_gemm.cu", "nm_hutch.cu", "nm_probe.cu"]
+SOURCES = ["nm_api.cu", "nm_prune.cu", "nm_gemm.cu", "nm_hutch.cu", "nm_f8.cu", "nm_probe.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -1,0 +1,395 @@
+// nm_f8.cu -- the FP8 (E4M3) form of the sparse layer.
+//
+// SlideSparse (arXiv 2603.05232) sec. 2B: the activation lift is only an index
+// remap, so it is fused into the per-token INT8/FP8/FP4 quantisation kernel;
+// sec. 2C: online, one fused quantise-and-lift kernel, then the sparse GEMM.
+//
+//   k_quant_lift_f8  one block per token: amax over the row (16-byte loads,
+//                    warp and block max), scale = amax / 448 (1 when amax is
+//                    0), then the lifted row (natural window order, zero past
+//                    the lifted width) as E4M3 codes of fp32(x / scale), round
+//                    to nearest even, saturating; 16 codes per 16-byte store.
+//   k_prepare_f8     one block per weight row: the same per-row scale over the
+//                    kept values, their codes in the packed order (the kept
+//                    order is the window order), and the 2:4 metadata bytes
+//                    rearranged into the kind::f8f6f4 layout: per 128-row tile
+//                    and 256-column K' block two 2 KB atoms of [128 rows x 16
+//                    bytes], row-major, a nibble idx0 | idx1 << 2 per window.
+//   k_gemm_f8        tcgen05.mma.sp kind::f8f6f4, one CTA per 128 weight rows
+//                    x 128 tokens: per 256-column K' block A = codes [128 x
+//                    128 bytes], B = lifted codes [128 x 256 bytes] (two TMA
+//                    boxes, 128-byte swizzle), the metadata copied into tensor
+//                    memory (each MMA, K = 64, reads two columns), four MMAs;
+//                    the epilogue scales by ws[row] * xs[token] and stores bf16.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "nm_common.cuh"
+#include "nm_host.cuh"
+
+namespace nm {
+
+constexpr int F8_BM = 128, F8_BN = 128, F8_THREADS = 256, F8_STAGES = 4;
+constexpr int F8_KB = 256;                                  // lifted columns per stage
+constexpr int F8_A_BYTES = F8_BM * 128;                     // 16 KB
+constexpr int F8_B_BYTES = F8_BN * 256;                     // 32 KB
+constexpr int F8_E_BYTES = 4096;                            // two 2 KB atoms
+constexpr int F8_STAGE_BYTES = F8_A_BYTES + F8_B_BYTES + F8_E_BYTES;
+constexpr int F8_SMEM_BYTES = F8_STAGES * F8_STAGE_BYTES + 1024 + 256;
+constexpr int F8_TMEM_COLS = 256;                           // accumulator 128 + metadata 8
+static_assert(F8_STAGE_BYTES % 1024 == 0, "stage alignment");
+static_assert(F8_BN * F8_BM * 2 <= F8_STAGES * F8_STAGE_BYTES, "epilogue staging");
+
+// two fp32 values -> two E4M3 codes (round to nearest even, saturating); the
+// first argument lands in the low byte
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ float f8_scale(float amax) { return amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f; }
+
+__device__ __forceinline__ float block_max(float v, float *red) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float r = red[0];
+    for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) r = fmaxf(r, red[w]);
+    __syncthreads();  // red is reused by the next call
+    return r;
+}
+
+// lifted column c (natural window order) -> source column of X
+__device__ __forceinline__ int64_t lift_src(int64_t c, int m) {
+    const int64_t per = 2 * m - 4;  // 4 (m/2 - 1) lifted columns per group
+    const int64_t g = c / per, rem = c - g * per;
+    return g * m + 2 * (rem >> 2) + (rem & 3);
+}
+
+__global__ void __launch_bounds__(256) k_quant_lift_f8(const uint16_t *__restrict__ X, int64_t T, int64_t K,
+                                                       int64_t ldx, int m, int64_t KL, uint8_t *__restrict__ Q,
+                                                       int64_t ldq, float *__restrict__ scale) {
+    __shared__ float red[8];
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        const uint16_t *row = X + t * ldx;
+        float amax = 0.0f;
+        const int64_t K8 = K / 8;
+        for (int64_t i = threadIdx.x; i < K8; i += blockDim.x) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(row) + i);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[j] << 16)),
+                                         fabsf(__uint_as_float(w[j] & 0xFFFF0000u))));
+        }
+        for (int64_t k = K8 * 8 + threadIdx.x; k < K; k += blockDim.x)
+            amax = fmaxf(amax, fabsf(__uint_as_float(static_cast<uint32_t>(row[k]) << 16)));
+        amax = block_max(amax, red);
+        const float s = f8_scale(amax);
+        if (threadIdx.x == 0) scale[t] = s;
+        uint8_t *qrow = Q + t * ldq;
+        for (int64_t c0 = 16 * static_cast<int64_t>(threadIdx.x); c0 < ldq; c0 += 16 * blockDim.x) {
+            float v[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int64_t c = c0 + j;
+                float x = 0.0f;
+                if (c < KL) {
+                    const int64_t src = m == 4 ? c : lift_src(c, m);
+                    if (src < K) x = __uint_as_float(static_cast<uint32_t>(__ldg(row + src)) << 16);
+                }
+                v[j] = __fdiv_rn(x, s);
+            }
+            uint32_t o[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                o[q] = e4m3x2(v[4 * q], v[4 * q + 1]) | (e4m3x2(v[4 * q + 2], v[4 * q + 3]) << 16);
+            *reinterpret_cast<uint4 *>(qrow + c0) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
+// one block per padded weight row: codes [Rpad x KLf / 2], metadata blocks,
+// scales [Rpad]; rows past R get zero codes, 0x44 metadata and scale 1
+__global__ void __launch_bounds__(256) k_prepare_f8(const uint16_t *__restrict__ vals, const uint8_t *__restrict__ wmeta,
+                                                    int64_t R, int64_t L, int64_t nwin, int64_t wbytes,
+                                                    int64_t Rpad, int64_t KLf, uint8_t *__restrict__ qv,
+                                                    uint8_t *__restrict__ qmeta, float *__restrict__ qscale) {
+    __shared__ float red[8];
+    const int64_t nkb = KLf / F8_KB, half = KLf / 2;
+    for (int64_t r = blockIdx.x; r < Rpad; r += gridDim.x) {
+        const bool real = r < R;
+        const uint16_t *vrow = vals + r * L;
+        float amax = 0.0f;
+        if (real)
+            for (int64_t j = threadIdx.x; j < L; j += blockDim.x)
+                amax = fmaxf(amax, fabsf(__uint_as_float(static_cast<uint32_t>(vrow[j]) << 16)));
+        amax = block_max(amax, red);
+        const float s = f8_scale(amax);
+        if (threadIdx.x == 0) qscale[r] = s;
+        uint8_t *out = qv + r * half;
+        for (int64_t j0 = 4 * static_cast<int64_t>(threadIdx.x); j0 < half; j0 += 4 * blockDim.x) {
+            float v[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int64_t j = j0 + q;
+                const float x = (real && j < L) ? __uint_as_float(static_cast<uint32_t>(vrow[j]) << 16) : 0.0f;
+                v[q] = __fdiv_rn(x, s);
+            }
+            *reinterpret_cast<uint32_t *>(out + j0) = e4m3x2(v[0], v[1]) | (e4m3x2(v[2], v[3]) << 16);
+        }
+        // metadata: byte i of atom a of K' block kb = windows 64kb + 32a + 2i, +1
+        const int64_t mt = r / F8_BM, lane = r - mt * F8_BM;
+        for (int64_t b = threadIdx.x; b < nkb * 32; b += blockDim.x) {
+            const int64_t kb = b >> 5, a = (b >> 4) & 1, i = b & 15;
+            const int64_t w0 = 64 * kb + 32 * a + 2 * i;
+            uint32_t lo = 0x4u, hi = 0x4u;  // padding window: indices 0 and 1 over zero values
+            if (real) {
+                const uint32_t byte = (w0 / 2 < wbytes) ? wmeta[r * wbytes + w0 / 2] : 0x44u;
+                if (w0 < nwin) lo = byte & 0xFu;
+                if (w0 + 1 < nwin) hi = byte >> 4;
+            }
+            qmeta[((mt * nkb + kb) * 2 + a) * 2048 + lane * 16 + i] = static_cast<uint8_t>(lo | (hi << 4));
+        }
+    }
+}
+
+__device__ __forceinline__ void mma_sp_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t e_tmem,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::1.kind::f8f6f4 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// kind::f8f6f4 instruction descriptor: E4M3 A and B (format 0), fp32 D,
+// both K-major, sparse
+__host__ __device__ constexpr uint32_t make_idesc_f8_sp(uint32_t M, uint32_t N) {
+    return (1u << 2) | (1u << 4) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// Warp roles: 0 = TMA producer, 1 = MMA issuer + tensor-memory owner,
+// 4..7 = epilogue (tensor memory -> scaled bf16 -> TMA store).
+__global__ void __launch_bounds__(F8_THREADS, 1)
+    k_gemm_f8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const __grid_constant__ CUtensorMap tmY, const uint8_t *__restrict__ meta, int64_t nkb,
+              const float *__restrict__ xs, const float *__restrict__ ws, int64_t T) {
+    constexpr int S = F8_STAGES;
+    extern __shared__ __align__(1024) uint8_t f8_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(f8_smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S * F8_STAGE_BYTES);
+    uint64_t *full = bars, *empty = bars + S, *accum = bars + 2 * S;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum + 1);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int mt = blockIdx.x, nt = blockIdx.y;
+    auto stA = [&](int s) { return smem + s * F8_STAGE_BYTES; };
+    auto stB = [&](int s) { return smem + s * F8_STAGE_BYTES + F8_A_BYTES; };
+    auto stE = [&](int s) { return smem + s * F8_STAGE_BYTES + F8_A_BYTES + F8_B_BYTES; };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accum, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+        prefetch_tmap(&tmY);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, F8_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t tmem_e = tmem_base + F8_BN;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int64_t kb = 0;
+            for (; kb < nkb; ++kb) {
+                const int s = static_cast<int>(kb % S);
+                const uint32_t ph = static_cast<uint32_t>((kb / S) & 1);
+                if (kb >= S && !mbar_wait(&empty[s], ph ^ 1u)) { *abort_flag = 1; break; }
+                mbar_arrive_expect_tx(&full[s], F8_STAGE_BYTES);
+                tma_load_2d(stA(s), &tmA, &full[s], static_cast<int32_t>(kb * 128), mt * F8_BM);
+                tma_load_2d(stB(s), &tmB, &full[s], static_cast<int32_t>(kb * F8_KB), nt * F8_BN);
+                tma_load_2d(stB(s) + F8_BN * 128, &tmB, &full[s], static_cast<int32_t>(kb * F8_KB + 128), nt * F8_BN);
+                bulk_load(stE(s), meta + (static_cast<int64_t>(mt) * nkb + kb) * F8_E_BYTES, F8_E_BYTES, &full[s]);
+            }
+            if (*abort_flag)  // let the copies already issued land
+                for (int64_t j = (kb > S ? kb - S : 0); j < kb; ++j)
+                    mbar_wait(&full[j % S], static_cast<uint32_t>((j / S) & 1));
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = make_idesc_f8_sp(F8_BM, F8_BN);
+            bool ok = true;
+            for (int64_t kb = 0; kb < nkb && ok; ++kb) {
+                const int s = static_cast<int>(kb % S);
+                if (!mbar_wait(&full[s], static_cast<uint32_t>((kb / S) & 1))) { ok = false; break; }
+                tc_fence_after();
+                tmem_cp_128x128b(tmem_e, make_sdesc(smem_u32(stE(s)), 2048, 128, 0));
+                tmem_cp_128x128b(tmem_e + 4, make_sdesc(smem_u32(stE(s) + 2048), 2048, 128, 0));
+                const uint32_t a0 = smem_u32(stA(s)), b0 = smem_u32(stB(s));
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint64_t ad = make_sdesc(a0 + j * 32, 16, 1024, 2);
+                    const uint64_t bd = make_sdesc(b0 + (j >> 1) * (F8_BN * 128) + (j & 1) * 64, 16, 1024, 2);
+                    mma_sp_f8(tmem_base, ad, bd, tmem_e + 2 * j, idesc, (kb > 0 || j > 0) ? 1u : 0u);
+                }
+                mma_commit(&empty[s]);
+            }
+            if (ok) mma_commit(accum);
+            else *abort_flag = 1;
+        }
+    } else if (warp >= 4) {
+        const int ew = warp - 4;
+        bool ok = __all_sync(0xffffffffu, mbar_wait(accum, 0));
+        if (ok) {
+            tc_fence_after();
+            const float wsr = ws[mt * F8_BM + ew * 32 + lane];  // ws holds Rpad entries
+            uint16_t *stage_out = reinterpret_cast<uint16_t *>(smem) + ew * (F8_BN * 32);  // [BN][32]
+#pragma unroll 1
+            for (int cc = 0; cc < F8_BN / 32; ++cc) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + cc * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int64_t t = static_cast<int64_t>(nt) * F8_BN + cc * 32 + j;
+                    const float xt = t < T ? __ldg(xs + t) : 0.0f;
+                    const float y = __fmul_rn(__uint_as_float(v[j]), __fmul_rn(wsr, xt));
+                    stage_out[(cc * 32 + j) * 32 + lane] = static_cast<uint16_t>(pack_bf16x2(y, 0.0f) & 0xFFFFu);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(&tmY, stage_out, mt * F8_BM + ew * 32, nt * F8_BN);
+                bulk_commit_group();
+                bulk_wait_group_read0();
+            }
+            __syncwarp();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, F8_TMEM_COLS);
+    }
+}
+
+}  // namespace nm
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+using namespace nm;
+
+namespace {
+
+struct F8Geom {
+    int64_t G, nwin, KL, KLf, nkb, Rpad, wbytes;
+    size_t vals_bytes, meta_bytes, total;
+};
+
+F8Geom f8_geometry(int64_t R, int64_t K, int m) {
+    F8Geom g{};
+    g.G = (K + m - 1) / m;
+    g.nwin = g.G * (m / 2 - 1);
+    g.KL = g.nwin * 4;
+    g.KLf = (g.KL + F8_KB - 1) / F8_KB * F8_KB;
+    g.nkb = g.KLf / F8_KB;
+    g.Rpad = (R + F8_BM - 1) / F8_BM * F8_BM;
+    g.wbytes = (g.nwin + 1) / 2;
+    g.vals_bytes = static_cast<size_t>(g.Rpad) * static_cast<size_t>(g.KLf / 2);
+    g.meta_bytes = static_cast<size_t>(g.Rpad / F8_BM) * static_cast<size_t>(g.nkb) * F8_E_BYTES;
+    g.total = g.vals_bytes + g.meta_bytes + static_cast<size_t>(g.Rpad) * 4;
+    return g;
+}
+
+bool f8_pattern_ok(int m) { return m >= 4 && m <= 10 && (m % 2) == 0; }
+
+}  // namespace
+
+extern "C" int64_t nm_lifted_cols_f8(int64_t K, int m) {
+    if (K < 1 || !f8_pattern_ok(m)) return 0;
+    return f8_geometry(1, K, m).KLf;
+}
+
+extern "C" size_t nm_sparse_prepare_f8_bytes(int64_t R, int64_t K, int m) {
+    if (R < 1 || K < 1 || !f8_pattern_ok(m)) return 0;
+    return f8_geometry(R, K, m).total;
+}
+
+extern "C" nm_status nm_quant_lift_f8(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, int m, uint8_t *Xq,
+                                      int64_t ldq, float *xscale, void *stream) {
+    if (!X || !Xq || !xscale) return NM_ERR_NULL;
+    if (!f8_pattern_ok(m)) return NM_ERR_UNSUPPORTED;
+    if (T < 1 || K < 1 || ldx < K) return NM_ERR_SHAPE;
+    const F8Geom g = f8_geometry(1, K, m);
+    if (ldq < g.KLf) return NM_ERR_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(X) & 15u) || (reinterpret_cast<uintptr_t>(Xq) & 15u) || (ldx % 8) != 0 ||
+        (ldq % 16) != 0 || (reinterpret_cast<uintptr_t>(xscale) & 3u))
+        return NM_ERR_ALIGN;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    k_quant_lift_f8<<<static_cast<unsigned>(T < 65535 * 4 ? T : 65535 * 4), 256, 0, st>>>(X, T, K, ldx, m, g.KL, Xq,
+                                                                                         ldq, xscale);
+    return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
+}
+
+extern "C" nm_status nm_sparse_prepare_f8(const uint16_t *vals, const uint8_t *wmeta, int64_t R, int64_t K, int m,
+                                          void *packed, size_t packed_bytes, void *stream) {
+    if (!vals || !wmeta || !packed) return NM_ERR_NULL;
+    if (!f8_pattern_ok(m)) return NM_ERR_UNSUPPORTED;
+    if (R < 1 || K < 1) return NM_ERR_SHAPE;
+    if (reinterpret_cast<uintptr_t>(packed) & 15u) return NM_ERR_ALIGN;
+    const F8Geom g = f8_geometry(R, K, m);
+    if (packed_bytes < g.total) return NM_ERR_WORKSPACE;
+    uint8_t *p = static_cast<uint8_t *>(packed);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    k_prepare_f8<<<static_cast<unsigned>(g.Rpad < 65535 * 4 ? g.Rpad : 65535 * 4), 256, 0, st>>>(
+        vals, wmeta, R, g.G * (m - 2), g.nwin, g.wbytes, g.Rpad, g.KLf, p, p + g.vals_bytes,
+        reinterpret_cast<float *>(p + g.vals_bytes + g.meta_bytes));
+    return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
+}
+
+extern "C" nm_status nm_sparse_gemm_f8(const uint8_t *Xq, int64_t T, int64_t K, int64_t ldq, const float *xscale,
+                                       const void *packed, int64_t R, int m, uint16_t *Y, int64_t ldy,
+                                       void *stream) {
+    if (!Xq || !xscale || !packed || !Y) return NM_ERR_NULL;
+    if (!f8_pattern_ok(m)) return NM_ERR_UNSUPPORTED;
+    if (T < 1 || K < 1 || R < 1 || ldy < R) return NM_ERR_SHAPE;
+    const F8Geom g = f8_geometry(R, K, m);
+    if (ldq < g.KLf || (T + F8_BN - 1) / F8_BN > 65535) return NM_ERR_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(Xq) & 15u) || (reinterpret_cast<uintptr_t>(packed) & 15u) ||
+        (reinterpret_cast<uintptr_t>(Y) & 15u) || (ldq % 16) != 0 || (ldy % 8) != 0 ||
+        (reinterpret_cast<uintptr_t>(xscale) & 3u))
+        return NM_ERR_ALIGN;
+    const uint8_t *p = static_cast<const uint8_t *>(packed);
+    CUtensorMap ta, tb, ty;
+    if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p, g.Rpad, g.KLf / 2, g.KLf / 2, 128, F8_BM, true) ||
+        !make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Xq, T, g.KLf, ldq, 128, F8_BN, true) ||
+        !make_tmap_bf16(&ty, Y, T, R, ldy, 32, F8_BN, false))
+        return NM_ERR_CUDA;
+    if (!set_smem_attr<k_gemm_f8>(F8_SMEM_BYTES)) return NM_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    dim3 grid(static_cast<unsigned>(g.Rpad / F8_BM), static_cast<unsigned>((T + F8_BN - 1) / F8_BN));
+    k_gemm_f8<<<grid, F8_THREADS, F8_SMEM_BYTES, st>>>(
+        ta, tb, ty, p + g.vals_bytes, g.nkb, xscale,
+        reinterpret_cast<const float *>(p + g.vals_bytes + g.meta_bytes), T);
+    return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
+}

@@ -75,6 +75,15 @@ def test_size_queries():
     assert lib.nm_hutchinson_workspace_bytes(8192, 4096, 16) == hq(8192, 4096, 16)
     assert lib.nm_hutchinson_workspace_bytes(1, 1, 256) == hq(1, 1, 256)
     assert lib.nm_hutchinson_workspace_bytes(0, 64, 1) == 0
+    # FP8: lifted width rounded up to 256; packed = codes [Rpad x KLf/2] +
+    # 4 KB of metadata per (128 rows, 256 lifted columns) + fp32 row scales
+    assert lib.nm_lifted_cols_f8(4096, 4) == 4096 and lib.nm_lifted_cols_f8(4096, 8) == 6144
+    assert lib.nm_lifted_cols_f8(1003, 6) == 1536 and lib.nm_lifted_cols_f8(7, 10) == 256
+    assert lib.nm_lifted_cols_f8(64, 5) == 0 and lib.nm_lifted_cols_f8(64, 12) == 0
+    for (R, K, m) in ((4096, 4096, 8), (131, 1003, 6), (1, 1, 4)):
+        KLf, Rpad = lib.nm_lifted_cols_f8(K, m), (R + 127) // 128 * 128
+        assert lib.nm_sparse_prepare_f8_bytes(R, K, m) == Rpad * KLf // 2 + Rpad // 128 * KLf // 256 * 4096 + Rpad * 4
+    assert lib.nm_sparse_prepare_f8_bytes(0, 8, 4) == 0
     assert lib.nm_hutchinson_workspace_bytes(64, 64, 257) == 0
 
 
@@ -114,6 +123,18 @@ MIS = 0x10002
     (lambda l: l.nm_hutchinson_diag(A, 4, 8, 8, A, 2, A, A, 16, None), 5),
     (lambda l: l.nm_hutchinson_diag(A, 4, 1 << 31, 1 << 31, A, 2, A, A, 1 << 62, None), 2),
     (lambda l: l.nm_hutchinson_diag(A, 1 << 31, 8, 8, A, 2, A, A, 1 << 62, None), 2),
+    (lambda l: l.nm_quant_lift_f8(None, 4, 8, 8, 4, A, 256, A, None), 1),
+    (lambda l: l.nm_quant_lift_f8(A, 4, 8, 8, 5, A, 256, A, None), 4),
+    (lambda l: l.nm_quant_lift_f8(A, 4, 8, 8, 4, A, 128, A, None), 2),
+    (lambda l: l.nm_quant_lift_f8(A, 4, 8, 8, 4, A, 264, A, None), 3),
+    (lambda l: l.nm_quant_lift_f8(A, 4, 8, 8, 4, MIS, 256, A, None), 3),
+    (lambda l: l.nm_sparse_prepare_f8(A, None, 4, 8, 8, A, 1 << 20, None), 1),
+    (lambda l: l.nm_sparse_prepare_f8(A, A, 4, 8, 12, A, 1 << 20, None), 4),
+    (lambda l: l.nm_sparse_prepare_f8(A, A, 4, 8, 8, A, 16, None), 5),
+    (lambda l: l.nm_sparse_gemm_f8(A, 4, 8, 256, None, A, 4, 8, A, 8, None), 1),
+    (lambda l: l.nm_sparse_gemm_f8(A, 4, 8, 128, A, A, 4, 8, A, 8, None), 2),
+    (lambda l: l.nm_sparse_gemm_f8(A, 4, 8, 256, A, A, 4, 8, A, 12, None), 3),
+    (lambda l: l.nm_sparse_gemm_f8(A, 4, 8, 256, A, A, 4, 3, A, 8, None), 4),
     (lambda l: l.slide_pack(A, 4, 8, 7, A, None), 4),
     (lambda l: l.slide_pack(A, 4, 8, 12, A, None), 4),
     (lambda l: l.lift_activations(A, 4, 8, 8, 5, A, 8, None), 4),
