@@ -207,8 +207,9 @@ nm_status nm_hutchinson_diag(const uint16_t *X, int64_t T, int64_t K, int64_t ld
 /* FP8 path (SlideSparse, arXiv 2603.05232, sec. 2B: the activation lift is
  * fused into the per-token INT8/FP8/FP4 quantisation kernel; sec. 2C: online,
  * the fused quantise-and-lift kernel, then the sparse GEMM).  Format E4M3
- * (largest finite 448); codes are fp32(x / scale) rounded to nearest even,
- * saturating; scale = amax / 448 in fp32 (1 when amax is 0), per token for
+ * (largest finite 448); codes are fp32(x * inv), inv = fp32(1 / scale),
+ * rounded to nearest even, saturating; scale = amax / 448 in fp32 (1 when
+ * amax is 0), per token for
  * the activations and per weight row (over its kept values) for the weights.
  * m in {4, 6, 8, 10} (2:4 and the (2N-2):2N patterns); the lifted columns are
  * in natural window order (window w of group g = columns g m + 2w .. + 3),

@@ -472,7 +472,8 @@ double oracle_ternary(const uint16_t *W, int64_t R, int64_t K, int64_t ldw, uint
  * finite value, ties to the even code, magnitudes beyond 448 clamp to 448.
  * Scales (a reading: the pages fix no scale rule): per token (activations)
  * and per weight row, scale = amax / 448 in fp32 (1 when amax = 0); a value
- * x becomes the code of fp32(x / scale).                                     */
+ * x becomes the code of fp32(x * inv), inv = fp32(1 / scale) (multiplying by
+ * the reciprocal, as per-token FP8 quantisers commonly do).                 */
 double oracle_e4m3_value(uint8_t c) {
     const int e = (c >> 3) & 15, mant = c & 7;
     const double v = e == 0 ? ldexp((double)mant, -9) : ldexp(1.0 + mant / 8.0, e - 7);
@@ -511,7 +512,7 @@ int oracle_quant_lift_f8(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, i
             const float v = fabsf(bf16_to_f32(X[t * ldx + k]));
             if (v > amax) amax = v;
         }
-        const float s = f8_scale(amax);
+        const float s = f8_scale(amax), inv = 1.0f / s;
         scale[t] = s;
         for (int64_t c = 0; c < ldq; ++c) Q[t * ldq + c] = 0;
         for (int64_t g = 0; g < G; ++g)
@@ -519,7 +520,7 @@ int oracle_quant_lift_f8(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, i
                 for (int c = 0; c < 4; ++c) {
                     const int64_t src = g * m + 2 * w + c;
                     const float v = src < K ? bf16_to_f32(X[t * ldx + src]) : 0.0f;
-                    Q[t * ldq + g * (Ns - 1) * 4 + 4 * w + c] = oracle_e4m3_encode(v / s);
+                    Q[t * ldq + g * (Ns - 1) * 4 + 4 * w + c] = oracle_e4m3_encode(v * inv);
                 }
     }
     return 0;
@@ -534,9 +535,9 @@ void oracle_quant_rows_f8(const uint16_t *V, int64_t R, int64_t L, uint8_t *Q, f
             const float v = fabsf(bf16_to_f32(V[r * L + j]));
             if (v > amax) amax = v;
         }
-        const float s = f8_scale(amax);
+        const float s = f8_scale(amax), inv = 1.0f / s;
         scale[r] = s;
-        for (int64_t j = 0; j < L; ++j) Q[r * L + j] = oracle_e4m3_encode(bf16_to_f32(V[r * L + j]) / s);
+        for (int64_t j = 0; j < L; ++j) Q[r * L + j] = oracle_e4m3_encode(bf16_to_f32(V[r * L + j]) * inv);
     }
 }
 

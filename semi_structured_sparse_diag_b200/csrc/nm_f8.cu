@@ -4,14 +4,17 @@
 // remap, so it is fused into the per-token INT8/FP8/FP4 quantisation kernel;
 // sec. 2C: online, one fused quantise-and-lift kernel, then the sparse GEMM.
 //
-//   k_quant_lift_f8  one block per token: amax over the row (16-byte loads,
-//                    warp and block max), scale = amax / 448 (1 when amax is
-//                    0), then the lifted row (natural window order, zero past
-//                    the lifted width) as E4M3 codes of fp32(x / scale), round
-//                    to nearest even, saturating; 16 codes per 16-byte store.
+//   k_quant_lift_f8  one block per token: the row into shared memory with
+//                    16-byte loads while taking its amax (warp and block max),
+//                    scale = amax / 448 (1 when amax is 0), then the lifted row
+//                    (natural window order, zero past the lifted width) read
+//                    back from shared memory as E4M3 codes of fp32(x * inv),
+//                    inv = fp32(1 / scale), round to nearest even, saturating;
+//                    16 codes per 16-byte store.  Rows above 48 K columns skip
+//                    the staging and gather from global memory instead.
 //   k_prepare_f8     one block per weight row: the same per-row scale over the
-//                    kept values, their codes in the packed order (the kept
-//                    order is the window order), and the 2:4 metadata bytes
+//                    kept values, their codes (of fp32(w * inv)) in the packed
+//                    order (the kept order is the window order), the metadata
 //                    rearranged into the kind::f8f6f4 layout: per 128-row tile
 //                    and 256-column K' block two 2 KB atoms of [128 rows x 16
 //                    bytes], row-major, a nibble idx0 | idx1 << 2 per window.
@@ -51,6 +54,8 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
 
 __device__ __forceinline__ float f8_scale(float amax) { return amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f; }
 
+constexpr int64_t F8_STAGE_ROW_MAX = 48 * 1024;  // columns of a row staged in shared memory
+
 __device__ __forceinline__ float block_max(float v, float *red) {
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
@@ -62,53 +67,61 @@ __device__ __forceinline__ float block_max(float v, float *red) {
     return r;
 }
 
-// lifted column c (natural window order) -> source column of X
-__device__ __forceinline__ int64_t lift_src(int64_t c, int m) {
-    const int64_t per = 2 * m - 4;  // 4 (m/2 - 1) lifted columns per group
-    const int64_t g = c / per, rem = c - g * per;
+// lifted column c (natural window order) -> source column of X (32-bit: the
+// lifted width is below 2^31)
+__device__ __forceinline__ int lift_src(int c, int m) {
+    const int per = 2 * m - 4;  // 4 (m/2 - 1) lifted columns per group
+    const int g = c / per, rem = c - g * per;
     return g * m + 2 * (rem >> 2) + (rem & 3);
 }
 
-__global__ void __launch_bounds__(256) k_quant_lift_f8(const uint16_t *__restrict__ X, int64_t T, int64_t K,
+constexpr int F8Q_THREADS = 128;  // per token; 12 tokens in flight per SM
+
+__global__ void __launch_bounds__(F8Q_THREADS, 12) k_quant_lift_f8(const uint16_t *__restrict__ X, int64_t T, int64_t K,
                                                        int64_t ldx, int m, int64_t KL, uint8_t *__restrict__ Q,
-                                                       int64_t ldq, float *__restrict__ scale) {
-    __shared__ float red[8];
+                                                       int64_t ldq, float *__restrict__ scale, int staged) {
+    __shared__ float red[F8Q_THREADS / 32];
+    extern __shared__ __align__(16) uint16_t xrow[];  // the row, when staged
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
         const uint16_t *row = X + t * ldx;
         float amax = 0.0f;
         const int64_t K8 = K / 8;
         for (int64_t i = threadIdx.x; i < K8; i += blockDim.x) {
             const uint4 v = __ldg(reinterpret_cast<const uint4 *>(row) + i);
+            if (staged) reinterpret_cast<uint4 *>(xrow)[i] = v;
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[j] << 16)),
                                          fabsf(__uint_as_float(w[j] & 0xFFFF0000u))));
         }
-        for (int64_t k = K8 * 8 + threadIdx.x; k < K; k += blockDim.x)
-            amax = fmaxf(amax, fabsf(__uint_as_float(static_cast<uint32_t>(row[k]) << 16)));
-        amax = block_max(amax, red);
-        const float s = f8_scale(amax);
+        for (int64_t k = K8 * 8 + threadIdx.x; k < K; k += blockDim.x) {
+            const uint16_t b = row[k];
+            if (staged) xrow[k] = b;
+            amax = fmaxf(amax, fabsf(__uint_as_float(static_cast<uint32_t>(b) << 16)));
+        }
+        amax = block_max(amax, red);  // also orders the staging stores before the reads below
+        const float s = f8_scale(amax), inv = __frcp_rn(s);
         if (threadIdx.x == 0) scale[t] = s;
+        const uint16_t *src_row = staged ? xrow : row;
         uint8_t *qrow = Q + t * ldq;
-        for (int64_t c0 = 16 * static_cast<int64_t>(threadIdx.x); c0 < ldq; c0 += 16 * blockDim.x) {
-            float v[16];
+        for (int64_t c0 = 8 * static_cast<int64_t>(threadIdx.x); c0 < ldq; c0 += 8 * blockDim.x) {
+            float v[8];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int64_t c = c0 + j;
+            for (int j = 0; j < 8; ++j) {
+                const int c = static_cast<int>(c0) + j;
                 float x = 0.0f;
                 if (c < KL) {
-                    const int64_t src = m == 4 ? c : lift_src(c, m);
-                    if (src < K) x = __uint_as_float(static_cast<uint32_t>(__ldg(row + src)) << 16);
+                    const int src = m == 4 ? c : lift_src(c, m);
+                    if (src < K) x = __uint_as_float(static_cast<uint32_t>(src_row[src]) << 16);
                 }
-                v[j] = __fdiv_rn(x, s);
+                v[j] = __fmul_rn(x, inv);
             }
-            uint32_t o[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                o[q] = e4m3x2(v[4 * q], v[4 * q + 1]) | (e4m3x2(v[4 * q + 2], v[4 * q + 3]) << 16);
-            *reinterpret_cast<uint4 *>(qrow + c0) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint2 *>(qrow + c0) =
+                make_uint2(e4m3x2(v[0], v[1]) | (e4m3x2(v[2], v[3]) << 16),
+                           e4m3x2(v[4], v[5]) | (e4m3x2(v[6], v[7]) << 16));
         }
+        __syncthreads();  // the staged row is read before the next token overwrites it
     }
 }
 
@@ -128,7 +141,7 @@ __global__ void __launch_bounds__(256) k_prepare_f8(const uint16_t *__restrict__
             for (int64_t j = threadIdx.x; j < L; j += blockDim.x)
                 amax = fmaxf(amax, fabsf(__uint_as_float(static_cast<uint32_t>(vrow[j]) << 16)));
         amax = block_max(amax, red);
-        const float s = f8_scale(amax);
+        const float s = f8_scale(amax), inv = __frcp_rn(s);
         if (threadIdx.x == 0) qscale[r] = s;
         uint8_t *out = qv + r * half;
         for (int64_t j0 = 4 * static_cast<int64_t>(threadIdx.x); j0 < half; j0 += 4 * blockDim.x) {
@@ -137,7 +150,7 @@ __global__ void __launch_bounds__(256) k_prepare_f8(const uint16_t *__restrict__
             for (int q = 0; q < 4; ++q) {
                 const int64_t j = j0 + q;
                 const float x = (real && j < L) ? __uint_as_float(static_cast<uint32_t>(vrow[j]) << 16) : 0.0f;
-                v[q] = __fdiv_rn(x, s);
+                v[q] = __fmul_rn(x, inv);
             }
             *reinterpret_cast<uint32_t *>(out + j0) = e4m3x2(v[0], v[1]) | (e4m3x2(v[2], v[3]) << 16);
         }
@@ -341,13 +354,16 @@ extern "C" nm_status nm_quant_lift_f8(const uint16_t *X, int64_t T, int64_t K, i
     if (!f8_pattern_ok(m)) return NM_ERR_UNSUPPORTED;
     if (T < 1 || K < 1 || ldx < K) return NM_ERR_SHAPE;
     const F8Geom g = f8_geometry(1, K, m);
-    if (ldq < g.KLf) return NM_ERR_SHAPE;
+    if (ldq < g.KLf || ldq > (int64_t(1) << 31) - 8) return NM_ERR_SHAPE;
     if ((reinterpret_cast<uintptr_t>(X) & 15u) || (reinterpret_cast<uintptr_t>(Xq) & 15u) || (ldx % 8) != 0 ||
         (ldq % 16) != 0 || (reinterpret_cast<uintptr_t>(xscale) & 3u))
         return NM_ERR_ALIGN;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    k_quant_lift_f8<<<static_cast<unsigned>(T < 65535 * 4 ? T : 65535 * 4), 256, 0, st>>>(X, T, K, ldx, m, g.KL, Xq,
-                                                                                         ldq, xscale);
+    const int staged = K <= F8_STAGE_ROW_MAX ? 1 : 0;
+    const int smem = staged ? static_cast<int>((K + 7) / 8 * 16) : 0;
+    if (staged && !set_smem_attr<k_quant_lift_f8>(static_cast<int>(F8_STAGE_ROW_MAX * 2))) return NM_ERR_CUDA;
+    k_quant_lift_f8<<<static_cast<unsigned>(T < 65535 * 4 ? T : 65535 * 4), F8Q_THREADS, smem, st>>>(
+        X, T, K, ldx, m, g.KL, Xq, ldq, xscale, staged);
     return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
 }
 
