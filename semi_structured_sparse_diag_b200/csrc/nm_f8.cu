@@ -67,14 +67,6 @@ __device__ __forceinline__ float block_max(float v, float *red) {
     return r;
 }
 
-// lifted column c (natural window order) -> source column of X (32-bit: the
-// lifted width is below 2^31)
-__device__ __forceinline__ int lift_src(int c, int m) {
-    const int per = 2 * m - 4;  // 4 (m/2 - 1) lifted columns per group
-    const int g = c / per, rem = c - g * per;
-    return g * m + 2 * (rem >> 2) + (rem & 3);
-}
-
 constexpr int F8Q_THREADS = 128;  // per token; 12 tokens in flight per SM
 
 __global__ void __launch_bounds__(F8Q_THREADS, 12) k_quant_lift_f8(const uint16_t *__restrict__ X, int64_t T, int64_t K,
@@ -105,17 +97,21 @@ __global__ void __launch_bounds__(F8Q_THREADS, 12) k_quant_lift_f8(const uint16_
         if (threadIdx.x == 0) scale[t] = s;
         const uint16_t *src_row = staged ? xrow : row;
         uint8_t *qrow = Q + t * ldq;
+        const int per = 2 * m - 4;  // lifted columns per group
         for (int64_t c0 = 8 * static_cast<int64_t>(threadIdx.x); c0 < ldq; c0 += 8 * blockDim.x) {
+            // group and offset of the chunk's first column once, then stepped
+            int g = static_cast<int>(c0) / per, rem = static_cast<int>(c0) - g * per;
             float v[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int c = static_cast<int>(c0) + j;
                 float x = 0.0f;
                 if (c < KL) {
-                    const int src = m == 4 ? c : lift_src(c, m);
+                    const int src = g * m + 2 * (rem >> 2) + (rem & 3);
                     if (src < K) x = __uint_as_float(static_cast<uint32_t>(src_row[src]) << 16);
                 }
                 v[j] = __fmul_rn(x, inv);
+                if (++rem == per) { rem = 0; ++g; }
             }
             *reinterpret_cast<uint2 *>(qrow + c0) =
                 make_uint2(e4m3x2(v[0], v[1]) | (e4m3x2(v[2], v[3]) << 16),
