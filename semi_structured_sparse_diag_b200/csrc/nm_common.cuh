@@ -152,20 +152,6 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthread
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// named barrier that also returns the AND of `v` over the nthreads threads
-__device__ __forceinline__ bool named_barrier_and(uint32_t id, uint32_t nthreads, bool v) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
-        : "memory");
-    return r != 0;
-}
-
 // ---------------------------------------------------------------------------
 // tcgen05 (tensor memory + 5th-generation MMA)
 // ---------------------------------------------------------------------------
