@@ -42,9 +42,11 @@ def _wmeta(res, m):
     return res["meta24"] if m == 4 else res["wmeta"]
 
 
-# (T, K, m, ldq extra): one token, ragged K, every pattern, a padded ld
+# (T, K, m, ldq extra): one token, ragged K, every pattern, a padded ld, and
+# rows wider than the 48 K columns staged in shared memory (read from global)
 @pytest.mark.parametrize("T,K,m,extra", [(1, 7, 4, 0), (33, 1030, 8, 16), (300, 4096, 6, 0),
-                                         (5, 2010, 10, 32), (129, 512, 4, 0), (64, 4096, 8, 0)])
+                                         (5, 2010, 10, 32), (129, 512, 4, 0), (64, 4096, 8, 0),
+                                         (3, 50001, 8, 0)])
 def test_quant_lift_f8_bitexact(nm, T, K, m, extra):
     X = datagen.make_activations(T, K, seed=T + K + m, n_outliers=min(2, K))
     X[0, : min(K, 5)] = 0                                  # some exact zeros
