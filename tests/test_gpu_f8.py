@@ -2,8 +2,9 @@
 lift, the FP8 weight operand, and the kind::f8f6f4 sparse GEMM (SlideSparse
 sec. 2B / 2C).
 
-Codes and scales are bit-exact against the oracle (both sides divide in fp32
-and round to the nearest E4M3 code, ties to even, saturating).  The GEMM is
+Codes and scales are bit-exact against the oracle (both sides multiply by
+fp32(1 / scale) and round to the nearest E4M3 code, ties to even,
+saturating).  The GEMM is
 bit-exact where every code is exact and the scales are 1 (integer products
 below 2^24 in fp32, one bf16 rounding), and within the GEMM bar
 max|Y - Y64| / max|Y64| <= 1e-2 of the oracle's fp64 product of the same
