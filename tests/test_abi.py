@@ -159,3 +159,18 @@ MIS = 0x10002
 ])
 def test_argument_validation(call, expect):
     assert call(nm.load()) == expect
+
+
+def test_binding_rejects_host_tensors_and_bad_patterns():
+    # the binding marshals device tensors only: host tensors and unsupported
+    # patterns are refused before any call reaches the library
+    import torch
+    X = torch.zeros((4, 64), dtype=torch.bfloat16)
+    zb = torch.zeros((2, 2), dtype=torch.int32)
+    for call in (lambda: nm.hutchinson_diag(X, zb), lambda: nm.quant_lift_f8(X, 8),
+                 lambda: nm.hessian_rescale(torch.zeros(8, dtype=torch.float64), torch.ones(8, dtype=torch.float64)),
+                 lambda: nm.sparse_gemm_f8(torch.zeros((4, 256), dtype=torch.uint8), torch.ones(4), X, 4, 64, 4)):
+        with pytest.raises(nm.NMError):
+            call()
+    lib = nm.load()
+    assert lib.nm_lifted_cols_f8(64, 7) == 0 and lib.nm_sparse_prepare_f8_bytes(8, 64, 12) == 0
