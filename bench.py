@@ -19,6 +19,11 @@ the same steps and reported in `stages_ms`.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   (the fp64 CPU oracle on a sample)
+
+The default workload is the Llama-7B gate/up projection (11008 x 4096, 2:4)
+at 8192 tokens.  With --gpus N > 1 outside torchrun, the script starts N ranks
+itself (torch.distributed.run, one process per GPU); each rank prunes and
+multiplies its own seeded layer and only the timings meet (max over ranks).
 """
 from __future__ import annotations
 
@@ -37,9 +42,10 @@ sys.path.insert(0, ROOT)
 
 import datagen  # noqa: E402
 
-DEFAULT_WORKLOAD = "slide_6of8_4096"
+DEFAULT_WORKLOAD = "llama7b_gate_T8192"
 METRIC = "N:M sparse GEMM effective TFLOP/s, % of 2:4 TC peak, speedup vs own dense"
 L2_FLUSH_BYTES = 256 << 20
+CHECK_TOL = 1e-2   # max|Y - Yref| / max|Yref| of the GEMM outputs
 
 
 def peaks():
@@ -167,6 +173,67 @@ def job_tflops(world: int, flops_per_rank: float, ms: float) -> float:
     return world * flops_per_rank / (ms * 1e-3) / 1e12
 
 
+def _free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_ranks(nranks: int, argv, timeout_s: float = 1800.0) -> int:
+    """Start `nranks` copies of this script under torch.distributed.run (one
+    process per GPU, rendezvous on 127.0.0.1) with the same arguments; rank 0
+    prints the JSON line.  Returns the launcher's exit status."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={nranks}",
+           "--master-addr=127.0.0.1", f"--master-port={_free_port()}", os.path.abspath(__file__), *argv]
+    env = dict(os.environ)
+    env.setdefault("OMP_NUM_THREADS", "1")
+    try:
+        return subprocess.run(cmd, env=env, timeout=timeout_s).returncode
+    except subprocess.TimeoutExpired:
+        print(json.dumps({"error": f"ranks did not finish within {timeout_s:.0f} s"}), file=sys.stderr)
+        return 124
+
+
+def run_cpu_standin(args):
+    """Host logic of the multi-rank run without a GPU: every rank runs the
+    oracle's whole path on its own seeded layer (gloo process group), the
+    step times meet as a max over ranks, rank 0 prints one line.  It exercises
+    the launcher, the rank environment and the aggregation; its numbers are CPU
+    numbers and say nothing about the GPU path."""
+    import datetime
+
+    import torch.distributed as dist
+
+    import oracle
+    world, rank, _local = rank_env()
+    if world > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+    layer = datagen.WORKLOADS[args.workload]
+    X_h, W_h = rank_inputs(layer, rank)
+    secs = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        res = oracle.run_layer(X_h, W_h, layer.n, layer.m, eps=layer.eps, score=layer.score,
+                               ternary_values=layer.ternary)
+        oracle.gemm_masked(X_h, res["mask"], res["V"], layer.m, rows=np.arange(min(8, layer.T)))
+        if i >= args.warmup:
+            secs.append(time.perf_counter() - t0)
+    if world > 1:
+        dist.barrier()
+    ms = max_over_ranks([1e3 * sum(secs) / len(secs)], world)[0]
+    flops = 2.0 * min(8, layer.T) * layer.R * layer.K
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps({"metric": "cpu stand-in of the multi-rank step (host logic only)",
+                          "value": round(job_tflops(world, flops, ms), 9), "unit": "TFLOP/s",
+                          "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                          "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+                          "standin": "cpu", "config": {"workload": layer.name}}), flush=True)
+
+
 # --------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------
@@ -177,6 +244,8 @@ def run_ours(args):
     import semi_structured_sparse_diag_b200 as nm
 
     world, rank, local = rank_env()
+    if world != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but {world} ranks were started")
     torch.cuda.set_device(local)
     if world > 1:
         import datetime
@@ -350,6 +419,14 @@ def run_ours(args):
     e2e_ms = max_over_ranks([e2e_ms], world, dev)[0]
     nm.check_device_error()
 
+    # output check: the sparse product against the own dense GEMM of the same
+    # masked weights (both fp32 accumulations rounded to bf16)
+    Ys, Yr = Y[:, :R].float(), Yd[:, :R].float()
+    dense_err = ((Ys - Yr).abs().max() / Yr.abs().max().clamp_min(1e-30)).item()
+    check = {"y_vs_own_dense": dense_err, "tol": CHECK_TOL}
+    # a failure on any rank fails the job (same collective on every rank)
+    ok = max_over_ranks([0.0 if dense_err <= CHECK_TOL else 1.0], world, dev)[0] == 0.0
+
     hbm, bf16_tf, peak_src = peaks()
     sparse_peak = 2.0 * bf16_tf  # 2:4 sparse bf16 = 2 x dense bf16 (nominal 4.5 / 2.25)
     flops_eff = 2.0 * T * R * K                 # dense-equivalent of the original layer
@@ -397,28 +474,44 @@ def run_ours(args):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
-    if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(layer, X_h, W_h, budget_s=args.cpu_seconds)
+    if clk:
+        # SM cycles of the sparse GEMM stage at the median clock seen under load
+        clk["sparse_gemm_kcycles_at_median_clock"] = round(gemm_ms * clk["sm_mhz"], 1)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb, Y64, (tok, rows_w) = cpu_baseline(layer, X_h, W_h, budget_s=args.cpu_seconds)
+        line["cpu_baseline"] = cb
+        # the same sampled outputs from the GPU against the oracle's fp64 product
+        Yg = Y[:tok, :rows_w].float().double().cpu().numpy()
+        den = float(np.max(np.abs(Y64))) or 1.0
+        check["y_vs_oracle_sample"] = float(np.max(np.abs(Yg - Y64)) / den)
+        check["oracle_sample"] = f"tokens 0..{tok - 1} x weight rows 0..{rows_w - 1}"
+        ok = ok and check["y_vs_oracle_sample"] <= CHECK_TOL
+    check["ok"] = bool(ok)
+    line["check"] = check
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+    if not ok:
+        raise SystemExit("bench.py: the sparse GEMM output failed its check (see the line's \"check\")")
 
 
 # --------------------------------------------------------------------------
 # the oracle on a bounded sample (CPU baseline and the reference arm)
 # --------------------------------------------------------------------------
 def oracle_sample_step(layer, X_h, W_h, rows_w: int, tok: int):
-    """One oracle step on a sample: H on all of X; S/prune/pack on `rows_w`
-    weight rows; fp64 GEMM of `tok` tokens against those rows.  Returns
-    (seconds, sample flops (dense-equivalent), stage seconds)."""
+    """One oracle step on a sample: H on all of X (for a ternary layer, gamma
+    over all of W); S/prune/pack on `rows_w` weight rows; fp64 GEMM of `tok`
+    tokens against those rows.  Returns (seconds, sample flops
+    (dense-equivalent), stage seconds, the sampled fp64 outputs [tok x rows_w])."""
     import oracle
     t0 = time.perf_counter()
     Wsub = np.ascontiguousarray(W_h[:rows_w])
     V = Wsub
     if layer.ternary:
-        _, V = oracle.ternary(Wsub)
+        _, Vall = oracle.ternary(W_h)    # gamma is a mean over the whole tensor
+        V = np.ascontiguousarray(Vall[:rows_w])
     if layer.score == "hessian":
         H = oracle.hessian_diag(X_h)
         S = oracle.score_hessian(H, Wsub, layer.eps)
@@ -430,10 +523,10 @@ def oracle_sample_step(layer, X_h, W_h, rows_w: int, tok: int):
         oracle.slide_pack(mask, layer.K, layer.m)
     t2 = time.perf_counter()
     rows = np.arange(tok, dtype=np.int64)
-    oracle.gemm_masked(X_h, mask, V, layer.m, rows=rows)
+    Y64 = oracle.gemm_masked(X_h, mask, V, layer.m, rows=rows)
     t3 = time.perf_counter()
     return t3 - t0, 2.0 * tok * rows_w * layer.K, {"score": t1 - t0, "prune_pack": t2 - t1,
-                                                   "gemm": t3 - t2}
+                                                   "gemm": t3 - t2}, Y64
 
 
 def _cores():
@@ -445,14 +538,15 @@ def _cores():
 
 def _sample_size(layer, budget_s):
     # ~1 GFLOP/s-per-core class fp64 loops: size the GEMM sample to the budget
-    rows_w = min(layer.R, 1024)
-    tok = max(1, min(layer.T, int(budget_s * 0.25e9 * _cores() / (2.0 * rows_w * layer.K))))
+    rate = 0.25e9 * _cores()   # fp64 multiply-adds per second, roughly
+    rows_w = max(8, min(layer.R, 1024, int(budget_s * rate / (2.0 * layer.K))))
+    tok = max(1, min(layer.T, int(budget_s * rate / (2.0 * rows_w * layer.K))))
     return rows_w, tok
 
 
 def cpu_baseline(layer, X_h, W_h, budget_s=10.0):
     rows_w, tok = _sample_size(layer, budget_s)
-    sec, flops, stages = oracle_sample_step(layer, X_h, W_h, rows_w, tok)
+    sec, flops, stages, Y64 = oracle_sample_step(layer, X_h, W_h, rows_w, tok)
     return {
         "value": round(flops / stages["gemm"] / 1e12, 6),
         "unit": "TFLOP/s",
@@ -462,7 +556,7 @@ def cpu_baseline(layer, X_h, W_h, budget_s=10.0):
                    f"{layer.R} weight rows, fp64 GEMM of {tok} tokens x {rows_w} rows x K={layer.K}; "
                    f"value = sample GEMM flops / oracle GEMM seconds; step {sec:.2f} s"),
         "stage_seconds": {k: round(v, 3) for k, v in stages.items()},
-    }
+    }, Y64, (tok, rows_w)
 
 
 def run_reference(args):
@@ -472,12 +566,13 @@ def run_reference(args):
         return
     layer = datagen.WORKLOADS[args.workload]
     X_h, W_h = datagen.layer_inputs(layer)
-    rows_w, tok = _sample_size(layer, args.cpu_seconds / 2)
+    # per-step sample sized so that the whole run stays within a few minutes
+    rows_w, tok = _sample_size(layer, min(args.cpu_seconds / 2, 90.0 / (args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_sample_step(layer, X_h, W_h, min(rows_w, 128), 1)
     secs, gsecs, flops = [], [], 0.0
     for _ in range(args.steps):
-        s, f, st = oracle_sample_step(layer, X_h, W_h, rows_w, tok)
+        s, f, st, _ = oracle_sample_step(layer, X_h, W_h, rows_w, tok)
         secs.append(s)
         gsecs.append(st["gemm"])
         flops = f
@@ -782,8 +877,10 @@ def run_ablation(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    # default: ~1 s of timed GPU work on the default workload, so the clock
+    # sampler sees the kernels under load
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(datagen.WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -793,7 +890,13 @@ def main():
     ap.add_argument("--prep", action="store_true", help="time the HBM-bound prep kernels instead")
     ap.add_argument("--reps", type=int, default=5, help="--prep / --f8: timed launches per kernel")
     ap.add_argument("--f8", action="store_true", help="time the FP8 quantise+lift and FP8 sparse GEMM instead")
+    ap.add_argument("--cpu-standin", action="store_true",
+                    help="host logic of the multi-rank run on CPU (gloo, the oracle as per-rank work)")
     args = ap.parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(launch_ranks(args.gpus, sys.argv[1:]))
+    if args.cpu_standin:
+        return run_cpu_standin(args)
     if args.prep:
         return run_prep(args)
     if args.f8:

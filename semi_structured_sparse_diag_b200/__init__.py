@@ -22,7 +22,7 @@ __all__ = [
     "NMError", "load", "hessian_diag", "score", "score_from_hessian", "prune_compress",
     "score_prune_compress", "hessian_rescale", "hutchinson_diag", "quant_lift_f8", "sparse_prepare_f8",
     "sparse_gemm_f8", "slide_pack", "lift_activations", "sparse_prepare", "sparse_gemm", "dense_gemm",
-    "ternary_quantize", "check_device_error", "set_gemm_schedule", "EXPORTED",
+    "ternary_quantize", "check_device_error", "set_gemm_schedule", "set_poison", "EXPORTED",
 ]
 
 EXPORTED = (
@@ -112,6 +112,25 @@ def _stream(stream=None) -> int:
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
+_POISON = False
+
+
+def set_poison(on: bool = True) -> None:
+    """Fill every output and workspace this binding allocates with 0xFF bytes
+    (NaN for fp32 / fp64 / bf16, all-ones for integers) before the call, so
+    that an element a kernel fails to write cannot pass a comparison by
+    holding the bytes of an earlier, identical call.  For tests."""
+    global _POISON
+    _POISON = bool(on)
+
+
+def _out(*shape, dtype, device) -> torch.Tensor:
+    t = torch.empty(*shape, dtype=dtype, device=device)
+    if _POISON and t.numel():
+        t.view(torch.uint8).fill_(0xFF)
+    return t
+
+
 def _ptr(t: torch.Tensor | None):
     return None if t is None else t.data_ptr()
 
@@ -145,10 +164,10 @@ def hessian_diag(X, H=None, ws=None, stream=None):
     T, K = X.shape
     lib = load()
     if H is None:
-        H = torch.empty(K, dtype=torch.float64, device=X.device)
+        H = _out(K, dtype=torch.float64, device=X.device)
     need = lib.nm_hessian_workspace_bytes(T, K)
     if ws is None and need:
-        ws = torch.empty(need, dtype=torch.uint8, device=X.device)
+        ws = _out(need, dtype=torch.uint8, device=X.device)
     _check(lib.nm_hessian_diag(_ptr(X), T, K, _ld(X), _ptr(H), _ptr(ws),
                                ws.numel() * ws.element_size() if ws is not None else 0,
                                _stream(stream)), "nm_hessian_diag")
@@ -159,7 +178,7 @@ def score_from_hessian(H, W, eps, S=None, stream=None):
     W = _bf16(W, "W")
     R, K = W.shape
     if S is None:
-        S = torch.empty((R, K), dtype=torch.float32, device=W.device)
+        S = _out((R, K), dtype=torch.float32, device=W.device)
     _check(load().nm_score_from_hessian(_ptr(H), float(eps), _ptr(W), R, K, _ld(W), _ptr(S),
                                         _stream(stream)), "nm_score_from_hessian")
     return S
@@ -172,7 +191,7 @@ def score(X, W, eps=1e-8, H=None, S=None, ws=None, stream=None):
     R, K = W.shape
     lib = load()
     if S is None:
-        S = torch.empty((R, K), dtype=torch.float32, device=W.device)
+        S = _out((R, K), dtype=torch.float32, device=W.device)
     if X is None:
         _check(lib.nm_score(None, 0, 0, _ptr(W), R, K, _ld(W), 0.0, None, _ptr(S), None, 0,
                             _stream(stream)), "nm_score")
@@ -182,10 +201,10 @@ def score(X, W, eps=1e-8, H=None, S=None, ws=None, stream=None):
     if X.shape[1] != K:
         raise NMError("X and W disagree on K")
     if H is None:
-        H = torch.empty(K, dtype=torch.float64, device=W.device)
+        H = _out(K, dtype=torch.float64, device=W.device)
     need = lib.nm_hessian_workspace_bytes(T, K)
     if ws is None and need:
-        ws = torch.empty(need, dtype=torch.uint8, device=W.device)
+        ws = _out(need, dtype=torch.uint8, device=W.device)
     _check(lib.nm_score(_ptr(X), T, _ld(X), _ptr(W), R, K, _ld(W), float(eps), _ptr(H), _ptr(S),
                         _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)), "nm_score")
     return H, S
@@ -202,9 +221,9 @@ def prune_compress(S, V, n, m, K=None, stream=None):
     R, K = V.shape
     G = n_groups(K, m)
     dev = V.device
-    mask = torch.empty((R, (G * m + 31) // 32), dtype=torch.int32, device=dev)
-    vals = torch.empty((R, G * n), dtype=torch.bfloat16, device=dev)
-    meta = torch.empty((R, (G + 1) // 2), dtype=torch.uint8, device=dev) if (m == 4 and n == 2) else None
+    mask = _out((R, (G * m + 31) // 32), dtype=torch.int32, device=dev)
+    vals = _out((R, G * n), dtype=torch.bfloat16, device=dev)
+    meta = _out((R, (G + 1) // 2), dtype=torch.uint8, device=dev) if (m == 4 and n == 2) else None
     _check(load().nm_prune_compress(_ptr(S), S.stride(0), _ptr(V), _ld(V), R, K, n, m, _ptr(mask),
                                     _ptr(vals), _ptr(meta), _stream(stream)), "nm_prune_compress")
     return mask, vals, meta
@@ -233,9 +252,9 @@ def hutchinson_diag(X, zbits, D=None, ws=None, stream=None):
     lib = load()
     need = lib.nm_hutchinson_workspace_bytes(T, K, S)
     if ws is None:
-        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=X.device)
+        ws = _out(max(need, 16), dtype=torch.uint8, device=X.device)
     if D is None:
-        D = torch.empty(K, dtype=torch.float64, device=X.device)
+        D = _out(K, dtype=torch.float64, device=X.device)
     _check(lib.nm_hutchinson_diag(_ptr(X), T, K, _ld(X), _ptr(zbits), S, _ptr(D), _ptr(ws),
                                   ws.numel() * ws.element_size(), _stream(stream)), "nm_hutchinson_diag")
     return D
@@ -251,8 +270,8 @@ def quant_lift_f8(X, m, ldq=None, stream=None):
     if KLf == 0:
         raise NMError(f"unsupported pattern m={m} for the FP8 path")
     ldq = KLf if ldq is None else ldq
-    Xq = torch.empty((T, ldq), dtype=torch.uint8, device=X.device)
-    xs = torch.empty(T, dtype=torch.float32, device=X.device)
+    Xq = _out((T, ldq), dtype=torch.uint8, device=X.device)
+    xs = _out(T, dtype=torch.float32, device=X.device)
     _check(lib.nm_quant_lift_f8(_ptr(X), T, K, _ld(X), m, _ptr(Xq), ldq, _ptr(xs), _stream(stream)),
            "nm_quant_lift_f8")
     return Xq, xs
@@ -267,7 +286,7 @@ def sparse_prepare_f8(vals, wmeta, R, K, m, stream=None):
     nbytes = lib.nm_sparse_prepare_f8_bytes(R, K, m)
     if nbytes == 0:
         raise NMError(f"unsupported shape or pattern for the FP8 path (R={R}, K={K}, m={m})")
-    packed = torch.empty(nbytes, dtype=torch.uint8, device=vals.device)
+    packed = _out(nbytes, dtype=torch.uint8, device=vals.device)
     _check(lib.nm_sparse_prepare_f8(_ptr(vals), _ptr(wmeta), R, K, m, _ptr(packed), nbytes, _stream(stream)),
            "nm_sparse_prepare_f8")
     return packed
@@ -278,7 +297,7 @@ def sparse_gemm_f8(Xq, xscale, packed, R, K, m, Y=None, stream=None):
     _dev(Xq, "Xq")
     T, ldq = Xq.shape
     if Y is None:
-        Y = torch.empty((T, (R + 7) // 8 * 8), dtype=torch.bfloat16, device=Xq.device)[:, :R]
+        Y = _out((T, (R + 7) // 8 * 8), dtype=torch.bfloat16, device=Xq.device)[:, :R]
     _check(load().nm_sparse_gemm_f8(_ptr(Xq), T, K, ldq, _ptr(xscale), _ptr(packed), R, m, _ptr(Y), _ld(Y),
                                     _stream(stream)), "nm_sparse_gemm_f8")
     return Y
@@ -295,9 +314,9 @@ def score_prune_compress(H, W, n, m, V=None, eps=1e-8, stream=None):
     R, K = W.shape
     G = n_groups(K, m)
     dev = W.device
-    mask = torch.empty((R, (G * m + 31) // 32), dtype=torch.int32, device=dev)
-    vals = torch.empty((R, G * n), dtype=torch.bfloat16, device=dev)
-    meta = torch.empty((R, (G + 1) // 2), dtype=torch.uint8, device=dev) if (m == 4 and n == 2) else None
+    mask = _out((R, (G * m + 31) // 32), dtype=torch.int32, device=dev)
+    vals = _out((R, G * n), dtype=torch.bfloat16, device=dev)
+    meta = _out((R, (G + 1) // 2), dtype=torch.uint8, device=dev) if (m == 4 and n == 2) else None
     _check(load().nm_score_prune_compress(_ptr(H), eps, _ptr(W), _ld(W), _ptr(V), _ld(V), R, K, n, m,
                                           _ptr(mask), _ptr(vals), _ptr(meta), _stream(stream)),
            "nm_score_prune_compress")
@@ -308,7 +327,7 @@ def slide_pack(mask, K, m, stream=None):
     _dev(mask, "mask")
     R = mask.shape[0]
     nw = n_groups(K, m) * (m // 2 - 1)
-    wmeta = torch.empty((R, (nw + 1) // 2), dtype=torch.uint8, device=mask.device)
+    wmeta = _out((R, (nw + 1) // 2), dtype=torch.uint8, device=mask.device)
     _check(load().slide_pack(_ptr(mask), R, K, m, _ptr(wmeta), _stream(stream)), "slide_pack")
     return wmeta
 
@@ -322,7 +341,7 @@ def lift_activations(X, m, XL=None, stream=None):
     T, K = X.shape
     KL = lifted_cols(K, m)
     if XL is None:
-        XL = torch.empty((T, (KL + 7) // 8 * 8), dtype=torch.bfloat16, device=X.device)[:, :KL]
+        XL = _out((T, (KL + 7) // 8 * 8), dtype=torch.bfloat16, device=X.device)[:, :KL]
     _check(load().lift_activations(_ptr(X), T, K, _ld(X), m, _ptr(XL), _ld(XL), _stream(stream)),
            "lift_activations")
     return XL
@@ -334,7 +353,7 @@ def sparse_prepare(vals, wmeta, R, K, m, packed=None, stream=None):
     if need == 0:
         raise NMError("nm_sparse_prepare_bytes: unsupported shape or pattern")
     if packed is None:
-        packed = torch.empty(need, dtype=torch.uint8, device=vals.device)
+        packed = _out(need, dtype=torch.uint8, device=vals.device)
     _check(lib.nm_sparse_prepare(_ptr(vals), _ptr(wmeta), R, K, m, _ptr(packed),
                                  packed.numel() * packed.element_size(), _stream(stream)),
            "nm_sparse_prepare")
@@ -348,14 +367,14 @@ def sparse_gemm(X, packed, R, m, Y=None, ws=None, stream=None, fused=False, tile
     T, K = X.shape
     lib = load()
     if Y is None:
-        Y = torch.empty((T, (R + 7) // 8 * 8), dtype=torch.bfloat16, device=X.device)[:, :R]
+        Y = _out((T, (R + 7) // 8 * 8), dtype=torch.bfloat16, device=X.device)[:, :R]
     if fused:
         _check(lib.nm_sparse_gemm_fused(_ptr(X), T, K, _ld(X), _ptr(packed), R, m, _ptr(Y),
                                         _ld(Y), _stream(stream)), "nm_sparse_gemm_fused")
         return Y
     need = lib.nm_sparse_gemm_workspace_bytes(T, K, m)
     if ws is None and need:
-        ws = torch.empty(need, dtype=torch.uint8, device=X.device)
+        ws = _out(need, dtype=torch.uint8, device=X.device)
     fn = lib.nm_sparse_gemm_tile256 if tile256 else lib.nm_sparse_gemm
     _check(fn(_ptr(X), T, K, _ld(X), _ptr(packed), R, m, _ptr(Y), _ld(Y),
               _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)),
@@ -370,9 +389,9 @@ def dense_gemm(X, W, Y=None, ws=None, stream=None):
     R = W.shape[0]
     lib = load()
     if Y is None:
-        Y = torch.empty((T, (R + 7) // 8 * 8), dtype=torch.bfloat16, device=X.device)[:, :R]
+        Y = _out((T, (R + 7) // 8 * 8), dtype=torch.bfloat16, device=X.device)[:, :R]
     if ws is None:
-        ws = torch.empty(lib.nm_dense_gemm_workspace_bytes(T, K, R), dtype=torch.uint8, device=X.device)
+        ws = _out(lib.nm_dense_gemm_workspace_bytes(T, K, R), dtype=torch.uint8, device=X.device)
     _check(lib.nm_dense_gemm(_ptr(X), T, K, _ld(X), _ptr(W), R, _ld(W), _ptr(Y), _ld(Y),
                              _ptr(ws), ws.numel(), _stream(stream)), "nm_dense_gemm")
     return Y
@@ -389,9 +408,9 @@ def ternary_quantize(W, stream=None):
     W = _bf16(W, "W")
     R, K = W.shape
     lib = load()
-    Wq = torch.empty((R, K), dtype=torch.bfloat16, device=W.device)
-    gamma = torch.empty(1, dtype=torch.float64, device=W.device)
-    ws = torch.empty(lib.nm_ternary_workspace_bytes(R), dtype=torch.uint8, device=W.device)
+    Wq = _out((R, K), dtype=torch.bfloat16, device=W.device)
+    gamma = _out(1, dtype=torch.float64, device=W.device)
+    ws = _out(lib.nm_ternary_workspace_bytes(R), dtype=torch.uint8, device=W.device)
     _check(lib.nm_ternary_quantize(_ptr(W), R, K, _ld(W), _ptr(Wq), _ptr(gamma), _ptr(ws),
                                    ws.numel(), _stream(stream)), "nm_ternary_quantize")
     return Wq, gamma

@@ -25,3 +25,14 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _poison_outputs(request):
+    """GPU tests: every output and workspace the binding allocates starts as
+    0xFF bytes (NaN for floating point), so an element that a kernel never
+    writes cannot pass by holding the bytes of an earlier, identical call."""
+    if "gpu" in request.keywords:
+        import semi_structured_sparse_diag_b200 as nm
+        nm.set_poison(True)
+    yield

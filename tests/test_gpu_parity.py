@@ -253,6 +253,37 @@ def test_score_prune_fused_bitexact(nm, n, m, R, K, mode):
         assert np.array_equal(to_host(meta), to_host(meta2))
 
 
+# the widths of the layers the bench runs and ragged ones: several 4096-column
+# slices of the fused 2:4 kernel (H staged per slice), a ragged last slice,
+# ragged row blocks (R = 9 against four rows per block), every (2N-2):2N
+# pattern; Hessian scores, ternary values under magnitude scores, and
+# small-integer weights (ties) under Hessian scores
+@pytest.mark.parametrize("K", [4097, 8195, 11008, 28672])
+@pytest.mark.parametrize("n,m", [(2, 4), (4, 6), (6, 8), (8, 10)])
+@pytest.mark.parametrize("mode", ["hessian", "ternary_values", "ties"])
+def test_score_prune_fused_wide_k(nm, n, m, K, mode):
+    R = 9
+    ld = (K + 7) // 8 * 8
+    X = datagen.make_activations(77, K, seed=K + m, n_outliers=3)
+    if mode == "ties":
+        W = datagen.small_int_bf16((R, K), seed=K, tensor_id=5)
+    else:
+        W = datagen.make_weight(R, K, 0.02, seed=K + n)
+    score = "magnitude" if mode == "ternary_values" else "hessian"
+    ref = oracle.run_layer(X, W, n, m, eps=1e-8, score=score, ternary_values=(mode == "ternary_values"))
+    Wd = to_dev(W, ld)
+    Vd = to_dev(ref["V"], ld) if mode == "ternary_values" else None
+    H = nm.hessian_diag(to_dev(X, ld)) if score == "hessian" else None
+    mask, vals, meta = nm.score_prune_compress(H, Wd, n, m, V=Vd, eps=1e-8)
+    _sync_ok(nm)
+    if H is not None:
+        assert np.array_equal(to_host(H), ref["H"])
+    assert np.array_equal(to_host(mask).view(np.uint32), ref["mask"])
+    assert np.array_equal(to_host_u16(vals), ref["vals"])
+    if m == 4:
+        assert np.array_equal(to_host(meta), ref["meta24"])
+
+
 @pytest.mark.parametrize("m,R,K", [(4, 64, 512), (6, 20, 1003), (8, 33, 1030), (10, 9, 207),
                                    (8, 4, 8), (6, 128, 4096), (10, 7, 8195)])
 def test_slide_pack_bitexact(nm, m, R, K):
@@ -454,20 +485,22 @@ def test_ternary_bitexact(nm, R, K):
 
 # ---------------------------------------------------------------- whole path
 def _device_pipeline(nm, X, W, n, m, eps=1e-8, score="hessian", ternary=False):
+    # the calls the bench's step makes: H, the fused score + prune, the window
+    # pack, the operand preparation and the sparse GEMM
     Xd, Wd = to_dev(X), to_dev(W)
     V = Wd
     if ternary:
         V, _ = nm.ternary_quantize(Wd)
-    H, S = nm.score(Xd if score == "hessian" else None, Wd, eps=eps)
-    mask, vals, meta = nm.prune_compress(S, V, n, m)
+    H = nm.hessian_diag(Xd) if score == "hessian" else None
+    mask, vals, meta = nm.score_prune_compress(H, Wd, n, m, V=V, eps=eps)
     wm = meta if m == 4 else nm.slide_pack(mask, W.shape[1], m)
     packed = nm.sparse_prepare(vals, wm, W.shape[0], W.shape[1], m)
     Y = nm.sparse_gemm(Xd, packed, W.shape[0], m)
     _sync_ok(nm)
-    return dict(H=H, S=S, mask=mask, vals=vals, wm=wm, Y=Y, V=V)
+    return dict(H=H, mask=mask, vals=vals, wm=wm, Y=Y, V=V)
 
 
-def _check_pipeline(nm, layer, n_rows=64):
+def _check_pipeline(nm, layer, n_rows=512):
     X, W = datagen.layer_inputs(layer)
     out = _device_pipeline(nm, X, W, layer.n, layer.m, layer.eps, layer.score, layer.ternary)
     ref = oracle.run_layer(X, W, layer.n, layer.m, layer.eps, layer.score, layer.ternary)
@@ -486,14 +519,17 @@ def _check_pipeline(nm, layer, n_rows=64):
     assert torch.isfinite(Yall).all()
 
 
+# every workload family; 512 sampled token rows of Y (all of them when T is
+# smaller) against the oracle's fp64 product, the rest checked finite (outputs
+# are poisoned with NaN before each call)
 @pytest.mark.parametrize("name", ["small_2of4", "slide_6of8_4096", "ternary_6of8_gate",
-                                  "llama7b_q_T8192", "llama7b_gate_T2048", "llama7b_down_T128",
-                                  "llama7b_q_T16"])
+                                  "llama7b_q_T8192", "llama7b_gate_T8192", "llama7b_down_T8192",
+                                  "llama7b_gate_T2048", "llama7b_down_T128", "llama7b_q_T16"])
 def test_workload_pipeline(nm, name):
-    _check_pipeline(nm, datagen.WORKLOADS[name], n_rows=128 if name == "small_2of4" else 32)
+    _check_pipeline(nm, datagen.WORKLOADS[name])
 
 
-@pytest.mark.parametrize("name", ["llama70b_up_4of6", "llama70b_down_8of10",
-                                  "llama70b_up_2of4", "llama70b_down_6of8"])
+@pytest.mark.parametrize("name", [f"llama70b_{p}_{nm_}" for p in ("up", "down")
+                                  for nm_ in ("2of4", "4of6", "6of8", "8of10")])
 def test_workload_pipeline_70b(nm, name):
-    _check_pipeline(nm, datagen.WORKLOADS[name], n_rows=8)
+    _check_pipeline(nm, datagen.WORKLOADS[name])

@@ -70,3 +70,34 @@ def test_single_rank_helpers():
     X0, W0 = bench.rank_inputs(layer, 0)
     X0b, _ = datagen.layer_inputs(layer)
     assert np.array_equal(X0, X0b)                   # rank 0 = the workload's own seed
+
+
+def _bench_lines(args, timeout=600):
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), *args], cwd=root,
+                       capture_output=True, text=True, timeout=timeout)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    return [json.loads(ln) for ln in lines]
+
+
+def test_bench_launches_two_ranks_itself():
+    # `bench.py --gpus 2` outside torchrun starts two ranks (torch.distributed.run,
+    # rendezvous on 127.0.0.1); with the CPU stand-in for the per-rank work they
+    # meet over gloo and rank 0 alone prints one line for the whole job
+    lines = _bench_lines(["--gpus", "2", "--cpu-standin", "--workload", "small_2of4",
+                          "--steps", "2", "--warmup", "3"])
+    assert len(lines) == 1
+    assert lines[0]["n_gpus"] == 2 and lines[0]["scaling"] == "weak"
+    assert lines[0]["value"] > 0 and lines[0]["ms_per_step"] > 0
+
+
+def test_reference_arm_under_two_ranks_prints_once():
+    # the reference arm under two ranks: rank 0 runs the oracle, rank 1 exits
+    lines = _bench_lines(["--impl", "reference", "--gpus", "2", "--workload", "small_2of4",
+                          "--steps", "2", "--warmup", "3", "--cpu-seconds", "1"])
+    assert len(lines) == 1
+    assert lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
+    assert lines[0]["cpu_baseline"]["kind"] == "oracle"
