@@ -40,9 +40,6 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 _lock = threading.Lock()
 _lib = None
 
-H_CHUNK = 128   # tokens per chunk partial of H
-H_RUN = 16      # tokens per sequential run inside a chunk
-
 
 def build(force: bool = False) -> str:
     """Compile nm_oracle.c into liboracle.so (gcc, OpenMP, no FMA contraction)."""
@@ -112,7 +109,9 @@ def lifted_cols(K: int, m: int) -> int:
 
 
 def hessian_diag(X: np.ndarray, naive: bool = False) -> np.ndarray:
-    """H [K] fp64 from X [T x K] bf16 bits (canonical chunked order unless naive)."""
+    """H [K] fp64 from X [T x K] bf16 bits: the exact column sums of squares
+    rounded once to fp64, divided by T (naive: one sequential fp64 sum instead,
+    a diagnostic)."""
     X = _c(X, np.uint16)
     T, K = X.shape
     H = np.empty(K, dtype=np.float64)

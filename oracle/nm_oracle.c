@@ -22,12 +22,13 @@
  *     are duplicated so the lifted product equals the original one.
  *
  * Readings of points the pages leave open (each also listed in the design
- * notes): mean (1/T) with no factor 2 for H; H summed in a canonical order
- * (chunks of 128 tokens; a chunk is runs of 16 tokens, each run summed in
- * ascending t, the runs added in ascending order; chunk partials summed in
- * ascending chunk order); S rounded once from fp64 to fp32; groups run along
- * the input (K) dimension; ties go to the lower index; a ragged tail group is
- * zero-padded (score 0, value 0); survivor k of a group goes to window k/2.
+ * notes): mean (1/T) with no factor 2 for H; a mean is the exact sum of its
+ * terms (every term here is a dyadic rational) rounded once to fp64, to
+ * nearest with ties to even, then one IEEE division by the count -- so no
+ * summation order enters the definition; S rounded once from fp64 to fp32;
+ * groups run along the input (K) dimension; ties go to the lower index; a
+ * ragged tail group is zero-padded (score 0, value 0); survivor k of a group
+ * goes to window k/2.
  *
  * Build: gcc -O2 -fopenmp -ffp-contract=off -fPIC -shared (no fast-math, no
  * FMA contraction), so every fp64 operation rounds exactly once as written.
@@ -36,9 +37,6 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
-
-#define ORACLE_H_CHUNK 128
-#define ORACLE_H_RUN 16
 
 /* bf16 bit pattern -> fp64 (exact: bf16 is the top half of an fp32). */
 static double bf16_to_f64(uint16_t b) {
@@ -80,27 +78,82 @@ static uint16_t f64_to_bf16_rne(double v) {
 static int64_t groups_of(int64_t K, int m) { return (K + m - 1) / m; }
 
 /* ------------------------------------------------------------------------ */
-/* O1: diagonal Gauss-Newton proxy H_j = (1/T) sum_t x_{t,j}^2 (canonical). */
+/* Exact sums of bf16-derived terms.  A finite bf16 value with exponent field
+ * e and fraction f has the significand m = 128 + f (e >= 1) or m = f (e = 0)
+ * and the value m * 2^(max(e,1) - 134).  So |x| is an integer multiple of
+ * 2^-134 and x^2 an integer multiple of 2^-268: both sums below are sums of
+ * integers, formed exactly with integer arithmetic and rounded once.        */
+
+#define ORACLE_DIGITS 24   /* 768-bit unsigned integer, 32-bit digits */
+
+/* n += v << shift (v < 2^64) */
+static void big_add_shifted(uint32_t *n, uint64_t v, int shift) {
+    int d = shift / 32, b = shift % 32;
+    /* v << b spans at most three digits */
+    uint64_t lo = (v << b) & 0xFFFFFFFFull;
+    uint64_t mid = b ? ((v >> (32 - b)) & 0xFFFFFFFFull) : ((v >> 32) & 0xFFFFFFFFull);
+    uint64_t hi = b ? (v >> (64 - b)) : 0;
+    uint64_t carry = 0;
+    uint64_t part[3] = {lo, mid, hi};
+    for (int i = d; i < ORACLE_DIGITS; ++i) {
+        uint64_t add = (i - d < 3) ? part[i - d] : 0;
+        uint64_t s = (uint64_t)n[i] + add + carry;
+        n[i] = (uint32_t)s;
+        carry = s >> 32;
+        if (i - d >= 2 && carry == 0) break;
+    }
+}
+
+/* the integer n times 2^-scale, rounded to the nearest fp64 (ties to even).
+ * n < 2^767 and scale <= 268 keep the result a normal, finite double. */
+static double big_round_to_double(const uint32_t *n, int scale) {
+    int top = -1;
+    for (int i = ORACLE_DIGITS - 1; i >= 0 && top < 0; --i)
+        if (n[i])
+            for (int b = 31; b >= 0; --b)
+                if ((n[i] >> b) & 1u) { top = 32 * i + b; break; }
+    if (top < 0) return 0.0;
+    /* bit p of n */
+    #define BIT(p) (((p) >= 0) ? ((n[(p) / 32] >> ((p) % 32)) & 1u) : 0u)
+    uint64_t sig = 0;                        /* the 53 bits from `top` down */
+    for (int p = top; p > top - 53; --p) sig = (sig << 1) | BIT(p);
+    int low = top - 53;                      /* the first bit below the kept ones */
+    int round_bit = (int)BIT(low);
+    int sticky = 0;
+    for (int p = low - 1; p >= 0 && !sticky; --p) sticky = (int)BIT(p);
+    #undef BIT
+    if (round_bit && (sticky || (sig & 1u))) sig += 1;   /* 2^53 stays exact */
+    return ldexp((double)sig, low + 1 - scale);
+}
+
+/* ------------------------------------------------------------------------ */
+/* O1: diagonal Gauss-Newton proxy H_j = (1/T) sum_t x_{t,j}^2:
+ *   the exact sum of the squares rounded once to fp64, then divided by T.
+ * Any NaN in a column makes its H NaN; otherwise any infinity makes it +inf. */
 void oracle_hessian_diag(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, double *H) {
     #pragma omp parallel for schedule(static)
     for (int64_t j = 0; j < K; ++j) {
-        double total = 0.0;
-        for (int64_t c0 = 0; c0 < T; c0 += ORACLE_H_CHUNK) {
-            int64_t c1 = c0 + ORACLE_H_CHUNK < T ? c0 + ORACLE_H_CHUNK : T;
-            double part = 0.0;
-            for (int64_t r0 = c0; r0 < c1; r0 += ORACLE_H_RUN) {
-                int64_t r1 = r0 + ORACLE_H_RUN < c1 ? r0 + ORACLE_H_RUN : c1;
-                double run = 0.0;
-                for (int64_t t = r0; t < r1; ++t) {
-                    double x = bf16_to_f64(X[t * ldx + j]);
-                    double sq = x * x;
-                    run = run + sq;
-                }
-                part = part + run;
+        uint64_t count[256];   /* sum of m^2 over the values with exponent field e */
+        memset(count, 0, sizeof count);
+        int nan = 0, inf = 0;
+        for (int64_t t = 0; t < T; ++t) {
+            uint16_t b = X[t * ldx + j];
+            int e = (b >> 7) & 0xFF, f = b & 0x7F;
+            if (e == 0xFF) {
+                if (f) nan = 1; else inf = 1;
+                continue;
             }
-            total = total + part;
+            uint64_t m = e ? (uint64_t)(128 + f) : (uint64_t)f;
+            count[e] += m * m;
         }
-        H[j] = total / (double)T;
+        if (nan) { H[j] = NAN; continue; }
+        if (inf) { H[j] = INFINITY; continue; }
+        uint32_t n[ORACLE_DIGITS];
+        memset(n, 0, sizeof n);
+        for (int e = 0; e < 255; ++e)
+            if (count[e]) big_add_shifted(n, count[e], 2 * (e ? e : 1));  /* units of 2^-268 */
+        double sum = big_round_to_double(n, 268);
+        H[j] = sum / (double)T;
     }
 }
 
@@ -147,7 +200,8 @@ void oracle_hutchinson_diag(const uint16_t *X, int64_t T, int64_t K, int64_t ldx
     free(u);
 }
 
-/* Same quantity, one sequential sum over all tokens (diagnostic only). */
+/* Same quantity, one sequential fp64 sum over all tokens in ascending t
+ * (diagnostic only: rounds at every addition, so it depends on the order). */
 void oracle_hessian_diag_naive(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, double *H) {
     #pragma omp parallel for schedule(static)
     for (int64_t j = 0; j < K; ++j) {
@@ -408,45 +462,38 @@ void oracle_gemm_lifted(const uint16_t *XL, int64_t T, int64_t KL, const uint16_
 
 /* ------------------------------------------------------------------------ */
 /* Ternary absmean quantisation (Sparse-BitNet, "O Problema" item 1):
- *   gamma = mean |W| over the tensor, fp64, in a fixed order:
- *     row sum: 32 partial sums; partial l takes the 8-column chunks
- *              l, l+32, l+64, ... (columns 8c .. 8c+7 of chunk c, those < K),
- *              each |w| added in ascending column order; then the partials
- *              are combined by halving: p[l] += p[l+16] (l < 16), then +8,
- *              +4, +2, +1; the row sum is p[0];
- *     total:   the row sums in blocks of 1024 consecutive rows, zero-padded,
- *              each block combined by halving (a[t] += a[t+512] for t < 512,
- *              then 256, ..., 1), the block sums added in ascending order;
- *     gamma = total / (R*K)  (one correctly rounded division);
+ *   gamma = mean |W| over the tensor: the exact sum of the |w| rounded once to
+ *           fp64, then divided by R*K;
  *   q     = clip(rint(W / gamma), -1, 1), ties to even;
  *   W_q   = q * bf16(gamma), bf16(gamma) rounded to nearest even from fp64.
- * Returns gamma (fp64), or -1.0 if bf16(gamma) is out of the normal range.  */
+ * Returns gamma (fp64), or -1.0 if bf16(gamma) is out of the normal range or
+ * W holds a NaN or an infinity.                                              */
 double oracle_ternary(const uint16_t *W, int64_t R, int64_t K, int64_t ldw, uint16_t *Wq) {
-    double *rowsum = (double *)malloc((size_t)R * sizeof(double));
-    if (!rowsum) return -1.0;
-    const int64_t nchunks = (K + 7) / 8;
-    #pragma omp parallel for schedule(static)
-    for (int64_t i = 0; i < R; ++i) {
-        double p[32];
-        for (int l = 0; l < 32; ++l) {
-            double s = 0.0;
-            for (int64_t c = l; c < nchunks; c += 32)
-                for (int64_t j = 8 * c; j < 8 * c + 8 && j < K; ++j) s = s + fabs(bf16_to_f64(W[i * ldw + j]));
-            p[l] = s;
-        }
-        for (int stride = 16; stride >= 1; stride /= 2)
-            for (int l = 0; l < stride; ++l) p[l] = p[l] + p[l + stride];
-        rowsum[i] = p[0];
+    uint64_t count[256];   /* sum of m over the values with exponent field e */
+    memset(count, 0, sizeof count);
+    int bad = 0;
+    /* integer counts: each thread counts its rows, the counts are added after */
+    #pragma omp parallel reduction(|:bad)
+    {
+        uint64_t mine[256];
+        memset(mine, 0, sizeof mine);
+        #pragma omp for schedule(static)
+        for (int64_t i = 0; i < R; ++i)
+            for (int64_t j = 0; j < K; ++j) {
+                uint16_t b = W[i * ldw + j];
+                int e = (b >> 7) & 0xFF, f = b & 0x7F;
+                if (e == 0xFF) { bad = 1; continue; }
+                mine[e] += e ? (uint64_t)(128 + f) : (uint64_t)f;
+            }
+        #pragma omp critical
+        for (int e = 0; e < 256; ++e) count[e] += mine[e];
     }
-    double total = 0.0;
-    double a[1024];
-    for (int64_t b = 0; b < R; b += 1024) {
-        for (int t = 0; t < 1024; ++t) a[t] = (b + t < R) ? rowsum[b + t] : 0.0;
-        for (int stride = 512; stride >= 1; stride /= 2)
-            for (int t = 0; t < stride; ++t) a[t] = a[t] + a[t + stride];
-        total = total + a[0];
-    }
-    free(rowsum);
+    if (bad) return -1.0;
+    uint32_t n[ORACLE_DIGITS];
+    memset(n, 0, sizeof n);
+    for (int e = 0; e < 255; ++e)
+        if (count[e]) big_add_shifted(n, count[e], e ? e : 1);   /* units of 2^-134 */
+    double total = big_round_to_double(n, 134);
     double gamma = total / ((double)R * (double)K);
     uint16_t gb = f64_to_bf16_rne(gamma);
     if (gb == 0xFFFF || gamma == 0.0) return -1.0;

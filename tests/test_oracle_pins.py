@@ -40,16 +40,71 @@ def test_H_closed_form_constant_columns():
     assert np.array_equal(H, (c.astype(np.float64) ** 2))
 
 
+def _exact_mean_of_squares(col_bits):
+    """fl(fl(sum x^2) / T) from exact rational arithmetic: the sum of the
+    squares as a Fraction, rounded once to fp64 by Python (correctly rounded),
+    then one IEEE division."""
+    xs = [Fraction(float(v)) for v in f32(np.asarray(col_bits, dtype=np.uint16))]
+    return float(sum(v * v for v in xs)) / len(xs)
+
+
 def test_H_exact_rational_small():
-    # exact rational mean of the bf16 squares bounds the oracle's rounding error
+    # H is the exact sum of the squares rounded once, divided by T: equal to the
+    # exact rational computation, and to math.fsum (a correctly rounded sum)
+    import math
     X = datagen.make_activations(257, 40, seed=3, n_outliers=3)
     H = oracle.hessian_diag(X)
     xs = f32(X).astype(np.float64)
     for j in range(X.shape[1]):
-        exact = sum(Fraction(float(v)) ** 2 for v in xs[:, j]) / X.shape[0]
-        err = abs(Fraction(float(H[j])) - exact)
-        # each of at most T+2 roundings is within 2^-53 relative of a partial sum <= total
-        assert err <= exact * Fraction(X.shape[0] + 2, 2 ** 53)
+        assert H[j] == _exact_mean_of_squares(X[:, j])
+        assert H[j] == math.fsum((xs[:, j] ** 2).tolist()) / X.shape[0]
+
+
+def test_H_is_correctly_rounded_not_summed_in_order():
+    # columns whose rounding a sum in any fixed fp64 order gets wrong:
+    #   2^52 + 2^52 + 1 is a tie between 2^53 and 2^53 + 2 -> even (2^53);
+    #   adding the square of the smallest subnormal, 2^-266, breaks the tie
+    #   upwards (2^53 + 2), which no fp64 partial sum can see;
+    #   and the same terms in other orders give the same H.
+    big, one, sub = 0x4C80, 0x3F80, 0x0001          # 2^26, 1.0, 2^-133
+    tie = np.array([big, big, one], dtype=np.uint16)[:, None]
+    above = np.array([big, big, one, sub], dtype=np.uint16)[:, None]
+    assert oracle.hessian_diag(tie)[0] == 2.0 ** 53 / 3
+    assert oracle.hessian_diag(above)[0] == (2.0 ** 53 + 2) / 4
+    assert oracle.hessian_diag(above, naive=True)[0] == 2.0 ** 53 / 4   # the sequential sum misses it
+    for perm in itertools.permutations(range(4)):
+        assert oracle.hessian_diag(above[list(perm)])[0] == (2.0 ** 53 + 2) / 4
+    # many small terms under a large one: 2^40 + 2^20 * 2^-14 ... exact only if no partial rounds
+    col = np.array([0x5380] + [0x3C00] * 3000, dtype=np.uint16)[:, None]   # 2^40 then 3000 x 2^-7
+    assert oracle.hessian_diag(col)[0] == _exact_mean_of_squares(col[:, 0])
+
+
+def test_H_special_values_against_exact_rationals():
+    # zeros of both signs, subnormals, the smallest and largest normals, mixed
+    # in random columns: equal to the exact rational value; NaN and infinity
+    rng = np.random.default_rng(11)
+    special = np.array([0x0000, 0x8000, 0x0001, 0x807F, 0x0040, 0x0080, 0x8080, 0x7F7F, 0xFF7F,
+                        0x1F80, 0x2000, 0x3F80, 0x4C80], dtype=np.uint16)
+    X = rng.choice(special, size=(50, 30))
+    X[:, 0] = datagen.make_activations(50, 1, seed=2)[:, 0]
+    H = oracle.hessian_diag(X)
+    for j in range(30):
+        assert H[j] == _exact_mean_of_squares(X[:, j])
+    # columns of subnormals only: x = f * 2^-133, so H = 2^-266 * mean(f^2)
+    Xs = np.array([[0x0001, 0x0003, 0x807F], [0x0001, 0x8000, 0x0040], [0x0001, 0x0002, 0x0001]],
+                  dtype=np.uint16)
+    Hs = oracle.hessian_diag(Xs)
+    assert Hs[0] == 2.0 ** -266
+    assert Hs[1] == (9 + 0 + 4) * 2.0 ** -266 / 3
+    assert Hs[2] == (127 * 127 + 64 * 64 + 1) * 2.0 ** -266 / 3
+    Xi = X.copy()
+    Xi[3, 1] = 0x7F80                       # +inf
+    Xi[4, 2] = 0xFF80                       # -inf
+    Xi[5, 3] = 0x7FC1                       # NaN
+    Xi[6, 3] = 0x7F80                       # NaN wins over inf
+    Hi = oracle.hessian_diag(Xi)
+    assert Hi[1] == np.inf and Hi[2] == np.inf and np.isnan(Hi[3])
+    assert np.array_equal(Hi[4:], H[4:])
 
 
 def test_H_power_of_two_scaling_is_exact():
@@ -148,24 +203,16 @@ def test_hutchinson_converges_to_H():
     assert err[1] < err[0] / 2 and err[2] < err[1] / 2
 
 
-def test_H_canonical_vs_naive_and_single_chunk():
+def test_H_exact_vs_naive_order():
+    # the sequential fp64 sum loses at most its own rounding against the exact
+    # value, and agrees with it bit for bit when every partial sum is exact
+    # (small-integer activations)
     X = datagen.make_activations(1000, 64, seed=7, n_outliers=2)
     Hc = oracle.hessian_diag(X)
     Hn = oracle.hessian_diag(X, naive=True)
-    assert np.all(np.abs(Hc - Hn) <= 1e-12 * np.abs(Hn))
-    # with at most one run of tokens the canonical order is the sequential one
-    Xs = X[: oracle.H_RUN]
-    assert np.array_equal(oracle.hessian_diag(Xs), oracle.hessian_diag(Xs, naive=True))
-    # one chunk: the runs of 16 tokens, each sequential, added in ascending order
-    Xc = X[:100]
-    x2 = f32(Xc).astype(np.float64) ** 2
-    expect = np.zeros(64)
-    for r0 in range(0, 100, oracle.H_RUN):
-        run = np.zeros(64)
-        for t in range(r0, min(r0 + oracle.H_RUN, 100)):
-            run = run + x2[t]
-        expect = expect + run
-    assert np.array_equal(oracle.hessian_diag(Xc), expect / 100)
+    assert np.all(np.abs(Hc - Hn) <= (1000 + 2) * 2.0 ** -53 * np.abs(Hc))
+    Xi = datagen.small_int_bf16((300, 16), seed=4, tensor_id=9)
+    assert np.array_equal(oracle.hessian_diag(Xi), oracle.hessian_diag(Xi, naive=True))
 
 
 def test_H_outlier_channels_scale_400x_in_expectation():
@@ -190,6 +237,51 @@ def test_S_special_values():
     # H = 0: score is eps * w^2
     S2 = oracle.score_hessian(np.zeros(4), W, 0.5)
     assert np.array_equal(S2, np.array([[0, 0.5, 2, 0.125], [4.5, 0, 0.5, 0.5]], dtype=np.float32))
+
+
+def _rn32(q: Fraction):
+    """The fp32 value nearest the rational q >= 0 (ties to even), and whether
+    q lies within 2^-40 relative of a tie (where the fp64 steps may decide)."""
+    a = np.float32(float(q))
+    best = None
+    for c in (np.nextafter(a, np.float32(0)), a, np.nextafter(a, np.float32(np.inf))):
+        d = abs(Fraction(float(c)) - q)
+        if best is None or d < best[0] or (d == best[0] and int(np.float32(c).view(np.uint32)) % 2 == 0):
+            best = (d, c)
+    lo, hi = np.nextafter(best[1], np.float32(0)), np.nextafter(best[1], np.float32(np.inf))
+    half = min(abs(Fraction(float(best[1])) - Fraction(float(lo))),
+               abs(Fraction(float(hi)) - Fraction(float(best[1])))) / 2
+    near_tie = abs(abs(Fraction(float(best[1])) - q) - half) <= q * Fraction(1, 2 ** 40)
+    return best[1], near_tie
+
+
+def test_S_single_rounding_against_exact_rationals():
+    # S = fp32((H + eps) w^2) with fp64 intermediates: the exact rational value
+    # of (H + eps) w^2 rounded once to fp32, except within 2^-40 of an fp32 tie
+    # (where the fp64 add may decide), and always within half an fp32 ulp plus
+    # the fp64 steps' 2^-51.  Non-dyadic H and eps: fp32 arithmetic or a
+    # second rounding fails this on many elements.
+    rng = np.random.default_rng(5)
+    H = rng.uniform(0.1, 3.0, size=64) * np.where(rng.random(64) < 0.1, 400.0, 1.0)
+    W = datagen.make_weight(32, 64, 0.02, seed=9)
+    eps = 1e-8
+    S = oracle.score_hessian(H, W, eps)
+    wf = f32(W).astype(np.float64)
+    checked = 0
+    for i in range(32):
+        for j in range(64):
+            exact = (Fraction(float(H[j])) + Fraction(eps)) * Fraction(float(wf[i, j])) ** 2
+            if exact == 0:
+                assert S[i, j] == 0
+                continue
+            want, near_tie = _rn32(exact)
+            got = Fraction(float(S[i, j]))
+            ulp = Fraction(float(np.spacing(np.float32(S[i, j]))))
+            assert abs(got - exact) <= ulp / 2 + exact * Fraction(1, 2 ** 51)
+            if not near_tie:
+                assert S[i, j] == want
+                checked += 1
+    assert checked > 2000
 
 
 def test_S_magnitude_exact():
@@ -470,14 +562,20 @@ def test_ternary_gamma_exact_on_integers():
     assert g == total / (37 * 1003)
 
 
-def test_ternary_gamma_close_to_exact_sum():
-    # the fixed order loses at most a few ulps against the exact sum (fsum)
+def test_ternary_gamma_is_the_rounded_exact_mean():
+    # gamma = fl(fl(sum |w|) / (R K)): equal to math.fsum (correctly rounded)
+    # over the whole tensor divided by R K, and to exact rationals on a tie
     import math
     W = datagen.make_weight(1500, 1030, 0.02, seed=3)
     g, _ = oracle.ternary(W)
-    absw = np.abs((W.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
-    exact = math.fsum(absw.ravel().tolist()) / absw.size
-    assert abs(g - exact) <= 1e-13 * exact
+    absw = np.abs(f32(W).astype(np.float64))
+    assert g == math.fsum(absw.ravel().tolist()) / absw.size
+    # 2^53 + 1 (+ the smallest subnormal) as |w| sums: tie to even, broken up
+    big = 0x5A00                                   # 2^53 (an exact bf16)
+    tie = np.array([[big, 0x3F80, 0x0000, 0x0000]], dtype=np.uint16)   # 2^53 + 1
+    up = np.array([[big, 0x3F80, 0x0001, 0x0000]], dtype=np.uint16)    # + 2^-133
+    assert oracle.ternary(tie)[0] == 2.0 ** 53 / 4
+    assert oracle.ternary(up)[0] == (2.0 ** 53 + 2) / 4
 
 
 def test_f64_to_bf16_rounding():
