@@ -30,6 +30,7 @@
  *                     SlideSparse sec. 2B "Elevacao de Ativacao".
  *   nm_sparse_prepare canonical values + window metadata -> the GEMM's operand
  *                     layout. SlideSparse sec. 2C item 2 (initialisation phase).
+ *   nm_sparse_prepare_from_mask  slide_pack and nm_sparse_prepare in one pass.
  *   nm_sparse_gemm    Y = X * W_sparse^T on the sparse tensor cores, over the
  *                     lifted activations for (2N-2):2N. SlideSparse sec. 2C
  *                     item 3 (online phase).
@@ -80,7 +81,7 @@ typedef enum {
     NM_ERR_CUDA = 6,         /* a CUDA runtime/driver call failed */
     NM_ERR_TIMEOUT = 7,      /* a device-side barrier wait gave up (device error word) */
     NM_ERR_DEVICE = 8,       /* a device-side consistency check failed (device error word) */
-    NM_ERR_TOO_LARGE = 9     /* problem needs more than an allocation-free call's static scratch */
+    NM_ERR_TOO_LARGE = 9     /* reserved: no call returns it */
 } nm_status;
 
 /* Human-readable name of a status code.  Never NULL. */
@@ -95,14 +96,20 @@ int nm_version(void);
 
 /* ------------------------------------------------------------------------ */
 /* a1: diagonal Gauss-Newton proxy (Sparsity Induction, sec. 2C).
- *   H[j] = (1/T) * sum_t X[t,j]^2 in fp64, summed in a fixed order: tokens in
- *   chunks of 128; a chunk is runs of 16 tokens, each run summed in ascending
- *   t, the runs added in ascending order; chunk partials added in ascending
- *   chunk order; one correctly rounded division by T.  The result is therefore
- *   bit-identical run to run and to any implementation of that order.
- *   X  : [T x K] bf16, ldx >= K.          H : [K] fp64 (output).
- *   ws : scratch of nm_hessian_workspace_bytes(T, K) bytes (may be NULL when
- *        that is 0, i.e. T <= 128).  Contents on return are unspecified.   */
+ *   H[j] = fl( fl(sum_t X[t,j]^2) / T ): the exact sum of the squares (each a
+ *   dyadic rational) rounded once to fp64, to nearest with ties to even, then
+ *   one correctly rounded division by T.  No summation order enters the
+ *   result: it equals math.fsum of the squares divided by T, bit for bit, on
+ *   any implementation.  A column holding a NaN gives NaN; otherwise one
+ *   holding an infinity gives +inf.
+ *   X  : [T x K] bf16, ldx >= K, 1 <= T <= NM_HESSIAN_MAX_TOKENS.
+ *   H  : [K] fp64 (output), 8-byte aligned.
+ *   ws : scratch of nm_hessian_workspace_bytes(T, K) bytes, 16-byte aligned
+ *        (may be NULL when that is 0: T <= 128 or K of about 56,000 and
+ *        more); at most a few MB whatever T.  Contents on return unspecified.
+ *   Errors: NULL X or H -> NM_ERR_NULL; T, K < 1, ldx < K, T too large ->
+ *   NM_ERR_SHAPE; alignment -> NM_ERR_ALIGN; short ws -> NM_ERR_WORKSPACE.  */
+#define NM_HESSIAN_MAX_TOKENS 2147483647ll
 size_t nm_hessian_workspace_bytes(int64_t T, int64_t K);
 nm_status nm_hessian_diag(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, double *H,
                           void *ws, size_t ws_bytes, void *stream);
@@ -112,24 +119,32 @@ nm_status nm_hessian_diag(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, 
  * device memory -- for example a plugin running inside a host framework that
  * owns all device memory and hands its plugins no allocator, or a
  * latency-critical loop where a cudaMalloc/cudaFree (which may synchronise the
- * device) is not acceptable.  It computes exactly what nm_hessian_diag computes
- * (same kernels, same summation order, bit-identical H) but keeps the chunk
- * partial sums in a fixed scratch array inside the library instead of a
- * caller-provided workspace.  The caller still passes X and H.
- *   Limit: ceil(T/128) * K <= NM_HESSIAN_NOALLOC_MAX_PARTIALS (8 MiB of fp64
- *   partials, e.g. T = 4096 with K up to 32768, or T = 8192 with K up to
- *   16384); larger problems return NM_ERR_TOO_LARGE and launch nothing.
+ * device) is not acceptable.  It returns exactly what nm_hessian_diag returns
+ * (the same kernels; H is the correctly rounded sum divided by T, so it is
+ * bit-identical) but keeps the blocks' partial sums in a fixed scratch array
+ * inside the library instead of a caller-provided workspace.  The caller
+ * still passes X and H.
+ *   Limit: the array holds NM_HESSIAN_NOALLOC_MAX_PAIRS partial pairs (2 MiB).
+ *   A call never needs more: the number of token ranges is capped at
+ *   NM_HESSIAN_NOALLOC_MAX_PAIRS / K (each block then takes more tokens), and
+ *   a single range, which K above NM_HESSIAN_NOALLOC_MAX_PAIRS / 2 gets,
+ *   needs no scratch.  So every size nm_hessian_diag accepts is accepted;
+ *   sizes beyond that (T > NM_HESSIAN_MAX_TOKENS) return NM_ERR_SHAPE and
+ *   launch nothing.
  *   Memory: the scratch is a static device array; every GPU that loads the
- *   library holds those 8 MiB until the process exits.
- *   Set-up: the first call on each device looks up the array's device address
- *   (with that device current); make that first call before any stream
- *   capture.  It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   library holds those 2 MiB until the process exits.
+ *   Set-up: the first call on each device that needs the array looks up its
+ *   device address (with that device current) and caches it; make that first
+ *   call before any stream capture.  The cached address belongs to the
+ *   device's current context: after cudaDeviceReset the library must be
+ *   unloaded and loaded again before this entry point is used.  It calls no
+ *   cudaMalloc, cudaFree or other allocating routine.
  *   Sharing: all calls on a device share the one array and it keeps the last
- *   call's contents (every partial is written before it is read, so nothing
+ *   call's contents (every pair is written before it is read, so nothing
  *   needs clearing).  Calls whose kernels may overlap on the GPU -- on
  *   different streams, or from different host threads -- race on the array
  *   and must be serialised by the caller.                                   */
-#define NM_HESSIAN_NOALLOC_MAX_PARTIALS 1048576
+#define NM_HESSIAN_NOALLOC_MAX_PAIRS 131072
 nm_status nm_hessian_diag_noalloc(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, double *H,
                                   void *stream);
 
@@ -285,6 +300,20 @@ size_t nm_sparse_prepare_bytes(int64_t R, int64_t K, int m);
 nm_status nm_sparse_prepare(const uint16_t *vals, const uint8_t *wmeta, int64_t R, int64_t K,
                             int m, void *packed, size_t packed_bytes, void *stream);
 
+/* a4 + a6 in one pass: the same packed operand as slide_pack followed by
+ * nm_sparse_prepare, with each window's index pair formed from the mask bits
+ * as the metadata is written (the sliding-window pack of SlideSparse sec. 2A:
+ * survivor k of a group at window k/2, index q_k - 2*(k/2)), so the window
+ * metadata is never stored.  m in {4, 6, 8, 10}, n = m - 2 (for 2:4 the pairs
+ * are meta24's).
+ *   vals  : [R x G n] bf16 from nm_prune_compress, 4-byte aligned.
+ *   mask  : [R x ceil(G m / 32)] u32 from nm_prune_compress, 4-byte aligned.
+ * A group that does not hold exactly m - 2 survivors sets NM_ERR_DEVICE in
+ * the device error word (its pairs are written as padding).  Errors as for
+ * nm_sparse_prepare.                                                        */
+nm_status nm_sparse_prepare_from_mask(const uint16_t *vals, const uint32_t *mask, int64_t R, int64_t K,
+                                      int m, void *packed, size_t packed_bytes, void *stream);
+
 /* a7: sparse GEMM (SlideSparse sec. 2C item 3; 2:4 sparse tensor cores).
  *   Y[t, r] = sum_k X[t,k] * (mask (.) V)[r,k], fp32 accumulation in tensor
  *   memory, bf16 output (round to nearest even).
@@ -346,19 +375,17 @@ nm_status nm_gemm_set_schedule(int policy, int clusters);
 
 /* Ternary absmean quantisation (Sparse-BitNet sec. 1 item 1), input
  * preparation of the ternary 6:8 layer.
- *   gamma = (sum of |W| in fp64) / (R*K), summed in a fixed order: per row,
- *           32 partial sums (partial l: the 8-column chunks l, l+32, ..., each
- *           in ascending column order) combined by halving (l += l+16, +8, +4,
- *           +2, +1); the row sums in blocks of 1024 rows, zero-padded, each
- *           combined by halving (t += t+512, ..., +1), the block sums added in
- *           ascending order;
+ *   gamma = fl( fl(sum of |W|) / (R*K) ): the exact sum of the magnitudes
+ *           rounded once to fp64 (nearest, ties to even), one division -- no
+ *           summation order enters it;
  *   q     = clip(rint(W / gamma), -1, 1) (fp64 division, ties to even);
  *   W_q   = q * bf16(gamma), bf16(gamma) rounded to nearest even from fp64,
  *           zeros stored as +0.
  *   W : [R x K] bf16, ldw >= K.  Wq : [R x K] bf16 (output, row stride K).
  *   gamma : one fp64 on the device (output).  ws : nm_ternary_workspace_bytes(R).
- * If bf16(gamma) falls outside the normal bf16 range the device error word
- * gets NM_ERR_DEVICE and Wq is all zero.                                    */
+ * If bf16(gamma) falls outside the normal bf16 range (W holding an infinity
+ * or a NaN included) the device error word gets NM_ERR_DEVICE and Wq is all
+ * zero.  ws: R * 16 + 16 bytes, 16-byte aligned.                           */
 size_t nm_ternary_workspace_bytes(int64_t R);
 nm_status nm_ternary_quantize(const uint16_t *W, int64_t R, int64_t K, int64_t ldw, uint16_t *Wq,
                               double *gamma, void *ws, size_t ws_bytes, void *stream);

@@ -1,7 +1,8 @@
 /*
- * nmsparse_probe.h -- measurement probes of libnmsparse (not part of the hot
- * path; the papers have no counterpart).  They calibrate the roofline
- * denominators on the chip the library runs on.
+ * nmsparse_probe.h -- measurement probes, ablation GEMMs and test controls
+ * of libnmsparse (not part of the hot path; the papers have no counterpart).
+ * The probes calibrate the roofline denominators on the chip the library
+ * runs on.
  */
 #ifndef NMSPARSE_PROBE_H
 #define NMSPARSE_PROBE_H
@@ -55,6 +56,21 @@ nm_status nm_sparse_gemm_fused(const uint16_t *X, int64_t T, int64_t K, int64_t 
 nm_status nm_sparse_gemm_tile256(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
                                  const void *packed, int64_t R, int m, uint16_t *Y, int64_t ldy,
                                  void *ws, size_t ws_bytes, void *stream);
+
+/* Test controls for the bounded device waits (failure detection without a
+ * GPU fault).  Every barrier and stream-K flag wait gives up after a limit,
+ * records NM_ERR_TIMEOUT in the device error word and lets its kernel finish;
+ * these two calls make such a wait run out on purpose, from the host.
+ *   nm_test_set_wait_limit_ns: the limit for kernels launched afterwards on
+ *     the current device, 1 ns .. 1 s; 0 restores the default of one second
+ *     (larger -> NM_ERR_SHAPE).
+ *   nm_test_withhold_stream_k_flag: the stream-K CTA pair with this index
+ *     (-1: none, the default) still writes its partial sums but never
+ *     publishes their flags, so the pair that owns the tile waits in vain.
+ * Both are synchronous copies to device variables; set them back before
+ * normal use.  Not for production calls.                                   */
+nm_status nm_test_set_wait_limit_ns(unsigned long long ns);
+nm_status nm_test_withhold_stream_k_flag(int cluster);
 
 #ifdef __cplusplus
 }

@@ -21,7 +21,8 @@ from . import build as _build
 __all__ = [
     "NMError", "load", "hessian_diag", "score", "score_from_hessian", "prune_compress",
     "score_prune_compress", "hessian_rescale", "hutchinson_diag", "quant_lift_f8", "sparse_prepare_f8",
-    "sparse_gemm_f8", "slide_pack", "lift_activations", "sparse_prepare", "sparse_gemm", "dense_gemm",
+    "sparse_gemm_f8", "slide_pack", "lift_activations", "sparse_prepare", "sparse_prepare_from_mask",
+    "sparse_gemm", "dense_gemm",
     "ternary_quantize", "check_device_error", "set_gemm_schedule", "set_poison", "EXPORTED",
 ]
 
@@ -34,7 +35,8 @@ EXPORTED = (
     "nm_sparse_gemm_fused", "nm_dense_gemm_workspace_bytes", "nm_gemm_set_schedule",
     "nm_sparse_gemm_tile256", "nm_score_prune_compress", "nm_hessian_rescale",
     "nm_hutchinson_workspace_bytes", "nm_hutchinson_diag", "nm_lifted_cols_f8", "nm_sparse_prepare_f8_bytes",
-    "nm_quant_lift_f8", "nm_sparse_prepare_f8", "nm_sparse_gemm_f8",
+    "nm_quant_lift_f8", "nm_sparse_prepare_f8", "nm_sparse_gemm_f8", "nm_test_set_wait_limit_ns",
+    "nm_test_withhold_stream_k_flag", "nm_sparse_prepare_from_mask",
 )
 
 _P, _I64, _I, _D, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_size_t
@@ -73,6 +75,9 @@ _SIGS = {
     "nm_probe_mma": (_I, [_I, _I, _I, _I, _P, _P, _P]),
     "nm_probe_copy": (_I, [_P, _P, _SZ, _I, _P]),
     "nm_gemm_1cta": (_I, [_I, _P, _I64, _I64, _I64, _P, _I64, _I64, _P, _I64, _P]),
+    "nm_test_set_wait_limit_ns": (_I, [ctypes.c_ulonglong]),
+    "nm_sparse_prepare_from_mask": (_I, [_P, _P, _I64, _I64, _I, _P, _SZ, _P]),
+    "nm_test_withhold_stream_k_flag": (_I, [_I]),
 }
 
 _lock = threading.Lock()
@@ -357,6 +362,23 @@ def sparse_prepare(vals, wmeta, R, K, m, packed=None, stream=None):
     _check(lib.nm_sparse_prepare(_ptr(vals), _ptr(wmeta), R, K, m, _ptr(packed),
                                  packed.numel() * packed.element_size(), _stream(stream)),
            "nm_sparse_prepare")
+    return packed
+
+
+def sparse_prepare_from_mask(vals, mask, R, K, m, packed=None, stream=None):
+    """The GEMM operand straight from the kept values and the mask: the
+    sliding-window pack and the operand preparation in one pass."""
+    _dev(vals, "vals")
+    _dev(mask, "mask")
+    lib = load()
+    need = lib.nm_sparse_prepare_bytes(R, K, m)
+    if need == 0:
+        raise NMError("nm_sparse_prepare_bytes: unsupported shape or pattern")
+    if packed is None:
+        packed = _out(need, dtype=torch.uint8, device=vals.device)
+    _check(lib.nm_sparse_prepare_from_mask(_ptr(vals), _ptr(mask), R, K, m, _ptr(packed),
+                                           packed.numel() * packed.element_size(), _stream(stream)),
+           "nm_sparse_prepare_from_mask")
     return packed
 
 

@@ -6,7 +6,22 @@
 
 namespace nm {
 __device__ uint32_t g_error_word = 0;
+__device__ uint64_t g_wait_limit_ns = WAIT_LIMIT_NS;
+__device__ int g_test_withhold_flag_cluster = -1;
 }  // namespace nm
+
+extern "C" nm_status nm_test_set_wait_limit_ns(unsigned long long ns) {
+    const uint64_t v = ns ? static_cast<uint64_t>(ns) : nm::WAIT_LIMIT_NS;
+    if (v > nm::WAIT_LIMIT_NS) return NM_ERR_SHAPE;
+    return cudaMemcpyToSymbol(nm::g_wait_limit_ns, &v, sizeof(v)) == cudaSuccess ? NM_OK : NM_ERR_CUDA;
+}
+
+extern "C" nm_status nm_test_withhold_stream_k_flag(int cluster) {
+    if (cluster < -1) return NM_ERR_SHAPE;
+    return cudaMemcpyToSymbol(nm::g_test_withhold_flag_cluster, &cluster, sizeof(cluster)) == cudaSuccess
+               ? NM_OK
+               : NM_ERR_CUDA;
+}
 
 extern "C" const char *nm_status_string(int status) {
     switch (status) {

@@ -23,6 +23,16 @@ __device__ __forceinline__ void raise_error(uint32_t bit) { atomicOr(&g_error_wo
 
 // one second: a barrier wait that lasts longer than this is treated as lost
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
+// the limit in force (WAIT_LIMIT_NS unless a test shortened it with
+// nm_test_set_wait_limit_ns); read only once a wait has not succeeded at once
+extern __device__ uint64_t g_wait_limit_ns;
+// test control: a stream-K cluster with this index writes its partial sums but
+// withholds their flags (-1: none), so that the owner's bounded wait runs out
+extern __device__ int g_test_withhold_flag_cluster;
+
+__device__ __forceinline__ uint64_t wait_limit_ns() {
+    return *static_cast<volatile uint64_t *>(&g_wait_limit_ns);
+}
 
 __device__ __forceinline__ uint64_t global_timer_ns() {
     uint64_t t;
@@ -72,14 +82,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// WAIT_LIMIT_NS, records ERRBIT_TIMEOUT and returns false.
+// the wait limit (one second), records ERRBIT_TIMEOUT and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
+    const uint64_t t0 = global_timer_ns(), limit = wait_limit_ns();
     uint32_t spins = 0;
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((++spins & 255u) == 0 && global_timer_ns() - t0 > WAIT_LIMIT_NS) {
+        if ((++spins & 255u) == 0 && global_timer_ns() - t0 > limit) {
             raise_error(ERRBIT_TIMEOUT);
             return false;
         }
@@ -361,11 +371,11 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
 // from the peer CTA)
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
+    const uint64_t t0 = global_timer_ns(), limit = wait_limit_ns();
     uint32_t spins = 0;
     while (true) {
         if (mbar_try_wait_cluster(bar, parity)) return true;
-        if ((++spins & 255u) == 0 && global_timer_ns() - t0 > WAIT_LIMIT_NS) {
+        if ((++spins & 255u) == 0 && global_timer_ns() - t0 > limit) {
             raise_error(ERRBIT_TIMEOUT);
             return false;
         }

@@ -103,72 +103,242 @@ __host__ __device__ inline void meta_byte_coords(int b, int &row, int &col) {
     col = 8 * kh + 16 * k1 + 32 * k2;
 }
 
-// values: one thread per 16-byte output chunk (4 slots = 8 values) of a row;
-// grid x = chunks of a row, y (+65535 z) = row
+// values, natural K' order (m = 4, 6, 10): the packed row is the row of vals
+// (a window's pair of values = one 4-byte word, window wi at word wi) padded
+// with zeros.  One thread per 16-byte output chunk; 16-byte loads when every
+// row of vals starts on 16 bytes (vec), else four 4-byte loads.
+// grid x = chunks of a row, y (+65535 z) = row.
 __global__ void __launch_bounds__(256)
-    k_prepare_vals(const uint16_t *__restrict__ vals, int64_t R, int64_t G, int n, int m,
-                   int64_t Rpad, int64_t KLh, uint16_t *__restrict__ out) {
+    k_prepare_vals(const uint16_t *__restrict__ vals, int64_t R, int64_t words, int64_t Rpad, int64_t KLh,
+                   bool vec, uint16_t *__restrict__ out) {
     const int64_t r = blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535;
     const int64_t c8 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // chunk
     if (r >= Rpad || c8 * 8 >= KLh) return;
-    const int64_t kb = c8 / 8;          // 64 values per K' block
-    const int s0 = static_cast<int>(c8 % 8) * 4;
-    const uint16_t *vrow = vals + r * (G * n);
-    uint32_t o[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        int64_t g;
-        int w;
-        slot_window(m, kb, s0 + i, g, w);
-        uint32_t lo = 0, hi = 0;
-        if (r < R && g < G) {
-            const uint16_t *p = vrow + g * n + 2 * w;
-            lo = __ldg(p);
-            hi = __ldg(p + 1);
+    const uint32_t *vrow = reinterpret_cast<const uint32_t *>(vals) + r * words;
+    const int64_t w0 = 4 * c8;
+    uint4 o = make_uint4(0u, 0u, 0u, 0u);
+    if (r < R) {
+        if (vec && w0 + 4 <= words) {
+            o = __ldg(reinterpret_cast<const uint4 *>(vrow + w0));
+        } else {
+            o.x = w0 < words ? __ldg(vrow + w0) : 0u;
+            o.y = w0 + 1 < words ? __ldg(vrow + w0 + 1) : 0u;
+            o.z = w0 + 2 < words ? __ldg(vrow + w0 + 2) : 0u;
+            o.w = w0 + 3 < words ? __ldg(vrow + w0 + 3) : 0u;
         }
-        o[i] = lo | (hi << 16);
     }
-    *reinterpret_cast<uint4 *>(out + r * KLh + c8 * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4 *>(out + r * KLh + c8 * 8) = o;
 }
 
-// metadata: one thread per tensor-memory lane of a block (16 output bytes);
-// grid x = blocks of 8 metadata blocks (8 x 128 lanes = 1024 threads / 4 ...),
-// each thread: block index blk, lane L.
+// values, 6:8: one warp per (row, 32 groups) = 96 words of vals (3 words per
+// group: windows 0, 1, 2); lane l loads words l, l + 32, l + 64 and the warp
+// writes the three K' blocks of those groups -- windows 0 and 2 of groups
+// 0-15 and of 16-31, then window 1 of all 32 -- one word per lane each, by
+// shuffles.  grid: 8 warps per block over (row, block of 32 groups).
 __global__ void __launch_bounds__(256)
-    k_prepare_meta(const uint8_t *__restrict__ wmeta, int64_t R, int64_t G, int m, int64_t wbytes,
-                   int64_t nkb, int64_t nblocks, uint8_t *__restrict__ out) {
-    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const int64_t blk = tid >> 7;
-    const int L = static_cast<int>(tid & 127);
-    if (blk >= nblocks) return;
-    const int nwin = m / 2 - 1;
+    k_prepare_vals68(const uint16_t *__restrict__ vals, int64_t R, int64_t G, int64_t Rpad, int64_t nj,
+                     int64_t KLh, uint16_t *__restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    const int64_t wid = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (wid >= Rpad * nj) return;  // warp-uniform
+    const int64_t r = wid / nj, j = wid - r * nj;
+    const int64_t words = 3 * G;
+    const uint32_t *src = reinterpret_cast<const uint32_t *>(vals) + r * words + 96 * j;
+    uint32_t v[3];
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+        const int64_t wi = 96 * j + 32 * q + lane;
+        v[q] = (r < R && wi < words) ? __ldg(src + 32 * q + lane) : 0u;
+    }
+    // word i of the 96 lives in lane i % 32, register i / 32
+    auto fetch = [&](int i) {
+        const uint32_t a = __shfl_sync(0xffffffffu, v[0], i & 31);
+        const uint32_t b = __shfl_sync(0xffffffffu, v[1], i & 31);
+        const uint32_t c = __shfl_sync(0xffffffffu, v[2], i & 31);
+        return i < 32 ? a : (i < 64 ? b : c);
+    };
+    // a K' block holds 32 slots = 32 words; blocks 3j, 3j + 1, 3j + 2 of the row
+    uint32_t *dst = reinterpret_cast<uint32_t *>(out + r * KLh) + 96 * j;
+    dst[lane] = fetch(3 * (lane >> 1) + 2 * (lane & 1));              // groups 0-15, windows 0 / 2
+    dst[32 + lane] = fetch(3 * (16 + (lane >> 1)) + 2 * (lane & 1));  // groups 16-31
+    dst[64 + lane] = fetch(3 * lane + 1);                             // window 1 of groups 0-31
+}
+
+// Window index pairs of a (2N-2):2N group from its mask bits (SlideSparse
+// sec. 2A): with the two pruned positions z0 < z1, survivor k sits at
+// k + [k >= z0] + [k >= z1 - 1], and window w (positions 2w .. 2w + 3) takes
+// survivors 2w and 2w + 1: its nibble is (q0 - 2w) | (q1 - 2w) << 2.  The
+// table below holds, for every m-bit value, the nibbles of its windows packed
+// in the order the operand's metadata bytes want them (window w at bits
+// 4w .. 4w+3), or 0xFFFF for a group that does not hold exactly m - 2
+// survivors; it is built at compile time for m = 6, 8, 10 and indexed
+// [offset(m) + bits].
+constexpr int wt_offset(int m) { return m == 6 ? 0 : (m == 8 ? 64 : 64 + 256); }
+constexpr uint16_t wt_entry(int m, uint32_t bits) {
+    uint32_t z = ~bits & ((1u << m) - 1u);
+    int cnt = 0, z0 = -1, z1 = -1;
+    for (int p = 0; p < m; ++p)
+        if ((z >> p) & 1u) {
+            ++cnt;
+            if (z0 < 0) z0 = p; else z1 = p;
+        }
+    if (cnt != 2) return 0xFFFFu;
+    uint32_t out = 0;
+    for (int w = 0; w < m / 2 - 1; ++w) {
+        const int k0 = 2 * w, k1 = 2 * w + 1;
+        const int q0 = k0 + (k0 >= z0) + (k0 >= z1 - 1), q1 = k1 + (k1 >= z0) + (k1 >= z1 - 1);
+        out |= static_cast<uint32_t>((q0 - 2 * w) | ((q1 - 2 * w) << 2)) << (4 * w);
+    }
+    return static_cast<uint16_t>(out);
+}
+struct WinTable {
+    uint16_t v[64 + 256 + 1024];
+    constexpr WinTable() : v() {
+        for (uint32_t b = 0; b < 64; ++b) v[wt_offset(6) + b] = wt_entry(6, b);
+        for (uint32_t b = 0; b < 256; ++b) v[wt_offset(8) + b] = wt_entry(8, b);
+        for (uint32_t b = 0; b < 1024; ++b) v[wt_offset(10) + b] = wt_entry(10, b);
+    }
+};
+__device__ const WinTable g_wintab = WinTable();
+
+// groups of K' block kb: [g_lo, g_hi)
+__device__ __forceinline__ void block_groups(int m, int64_t kb, int64_t &g_lo, int64_t &g_hi) {
+    if (m == 8) {
+        const int64_t j = kb / 3;
+        const int type = static_cast<int>(kb - 3 * j);
+        g_lo = type < 2 ? 32 * j + 16 * type : 32 * j;
+        g_hi = g_lo + (type < 2 ? 16 : 32);
+    } else {
+        const int sh = m == 4 ? 0 : (m == 6 ? 1 : 2);
+        g_lo = (32 * kb) >> sh;
+        g_hi = (32 * kb + 32) >> sh;
+    }
+}
+
+// metadata: one block of 128 threads per (128-row tile mt, K' block kb).
+// (1) The block's input -- the mask words or window-metadata bytes of its
+// groups, for 128 rows -- comes into shared memory with coalesced loads (and,
+// from the mask, the pattern's window table).  (2) Thread r forms the 16
+// bytes of row mt * 128 + r (slot 2p in the low nibble of byte p): from the
+// window metadata (for the natural orders a plain copy), or, with FROM_MASK,
+// by looking each group's mask bits up in the table (the sliding-window pack
+// fused in).  Padding rows and slots get the pair (0, 1).  (3) Thread L
+// writes lane L's 16 bytes in the tensor-memory order of meta_byte_coords:
+// with L = m0 + 8 k1 + 16 m2, word k2 of the lane is half-word k1 + 2 k2 of
+// row m0 + 16 m2 (low half) and of row m0 + 16 m2 + 8 (high half).
+constexpr int PM_IN_WORDS = 13;   // >= input words of a row for any pattern (+1 pitch)
+template <int M, bool FROM_MASK>
+__global__ void __launch_bounds__(128)
+    k_prepare_meta(const uint8_t *__restrict__ wmeta, const uint32_t *__restrict__ mask, int64_t R, int64_t G,
+                   int64_t wbytes, int64_t mwords, int64_t nkb, uint8_t *__restrict__ out) {
+    constexpr int NWIN = M / 2 - 1;
+    __shared__ uint32_t in[BM][PM_IN_WORDS];
+    __shared__ uint32_t rowb[BM][5];  // 16 bytes per row (+1 word pitch)
+    __shared__ uint16_t tab[M == 4 ? 1 : (1 << M)];
+    const int64_t blk = blockIdx.x;
     const int64_t mt = blk / nkb, kb = blk - mt * nkb;
-    uint32_t words[4];
+    const int t = threadIdx.x;
+    if (FROM_MASK && M != 4)
+        for (int i = t; i < (1 << M); i += BM) tab[i] = g_wintab.v[wt_offset(M) + i];
+    int64_t g_lo, g_hi;
+    block_groups(M, kb, g_lo, g_hi);
+    const int64_t g_end = g_hi < G ? g_hi : G;  // real groups [g_lo, g_end)
+    // the input span of a row: mask words or wmeta bytes [u0, u1)
+    int64_t u0 = 0, u1 = 0;
+    if (g_end > g_lo) {
+        if (FROM_MASK) {
+            u0 = (g_lo * M) >> 5;
+            u1 = (g_end * M + 31) >> 5;
+        } else {
+            u0 = (g_lo * NWIN) >> 1;
+            u1 = (g_end * NWIN + 1) >> 1;
+        }
+    }
+    const int nu = static_cast<int>(u1 - u0);   // <= 9 words / <= 48 bytes
+    for (int idx = t; idx < BM * nu; idx += BM) {
+        const int rr = idx / nu, q = idx - rr * nu;
+        const int64_t row = mt * BM + rr;
+        if (FROM_MASK)
+            in[rr][q] = row < R ? __ldg(mask + row * mwords + u0 + q) : 0u;
+        else
+            reinterpret_cast<uint8_t *>(in[rr])[q] = row < R ? __ldg(wmeta + row * wbytes + u0 + q) : 0u;
+    }
+    __syncthreads();
+    const int64_t row = mt * BM + t;
+    const int ng = static_cast<int>(g_end - g_lo);
+    const bool mid = M == 8 && (kb % 3) == 2;
+    constexpr int GPB = M == 4 ? 32 : (M == 8 ? 32 : 32 / NWIN);  // groups a block can hold (6:8: 16 or 32)
+    uint32_t wd[4] = {0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u};  // padding pairs
+    bool bad = false;
+    if (row < R) {
+        const uint8_t *inb = reinterpret_cast<const uint8_t *>(in[t]);
+        if (!FROM_MASK && M != 8 && ng * NWIN == 32) {
+            // natural order, a whole block of real windows: its 16 bytes as they are
 #pragma unroll
-    for (int wd = 0; wd < 4; ++wd) {
-        uint32_t v = 0;
+            for (int q = 0; q < 4; ++q)
+                wd[q] = static_cast<uint32_t>(inb[4 * q]) | (static_cast<uint32_t>(inb[4 * q + 1]) << 8) |
+                        (static_cast<uint32_t>(inb[4 * q + 2]) << 16) | (static_cast<uint32_t>(inb[4 * q + 3]) << 24);
+        } else {
 #pragma unroll
-        for (int bb = 0; bb < 4; ++bb) {
-            int rl, cl;
-            meta_byte_coords(L * 16 + wd * 4 + bb, rl, cl);
-            const int64_t row = mt * BM + rl;
-            uint32_t nib[2] = {0x4u, 0x4u};  // padding: pair (0,1) over zero values
+            for (int gi = 0; gi < GPB; ++gi) {
+                if (gi >= ng || (M == 8 && !mid && gi >= 16)) break;
+                const int64_t g = g_lo + gi;
+                uint32_t nibs;  // window w's nibble at bits 4w
+                if (FROM_MASK) {
+                    const int64_t c = g * M - 32 * u0;  // bit offset within the staged words
+                    const int q = static_cast<int>(c >> 5), off = static_cast<int>(c & 31);
+                    const uint64_t both = (static_cast<uint64_t>(q + 1 < nu ? in[t][q + 1] : 0u) << 32) | in[t][q];
+                    const uint32_t bits = static_cast<uint32_t>(both >> off) & ((1u << M) - 1u);
+                    if (M == 4) {
+                        // 2:4: the two survivors, ascending, are the set bits
+                        const uint32_t s0 = static_cast<uint32_t>(__ffs(bits) - 1);
+                        const uint32_t s1 = static_cast<uint32_t>(__ffs(bits & (bits - 1u)) - 1);
+                        nibs = __popc(bits) == 2 ? (s0 | (s1 << 2)) : 0xFFFFu;
+                    } else {
+                        nibs = tab[bits];
+                    }
+                    if (nibs == 0xFFFFu) {
+                        bad = true;
+                        continue;  // its slots keep the padding pair
+                    }
+                } else {
+                    nibs = 0;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                int64_t g;
-                int w;
-                slot_window(m, kb, cl / 4 + h, g, w);
-                if (row < R && g < G) {
-                    const int64_t wi = g * nwin + w;
-                    nib[h] = (__ldg(wmeta + row * wbytes + wi / 2) >> (4 * (wi & 1))) & 0xFu;
+                    for (int w = 0; w < NWIN; ++w) {
+                        const int64_t wi = g * NWIN + w;
+                        nibs |= ((static_cast<uint32_t>(inb[(wi >> 1) - u0]) >> (4 * (wi & 1))) & 0xFu) << (4 * w);
+                    }
+                }
+                // place the group's slots: natural order window w at slot gi * NWIN + w;
+                // 6:8 blocks 0/1: windows 0 and 2 at slots 2 gi, 2 gi + 1; block 2: window 1 at slot gi
+                auto place = [&](int slot, int width, uint32_t val) {  // slot, width static after unrolling
+                    const int sh = 4 * (slot & 7);
+                    const uint32_t msk = width == 32 ? 0xFFFFFFFFu : (((1u << width) - 1u) << sh);
+                    wd[slot >> 3] = (wd[slot >> 3] & ~msk) | ((val << sh) & msk);
+                };
+                if (M == 8) {
+                    if (mid)
+                        place(gi, 4, (nibs >> 4) & 0xFu);
+                    else
+                        place(2 * gi, 8, (nibs & 0xFu) | (((nibs >> 8) & 0xFu) << 4));
+                } else {
+                    place(gi * NWIN, 4 * NWIN, nibs);
                 }
             }
-            v |= (nib[0] | (nib[1] << 4)) << (8 * bb);
         }
-        words[wd] = v;
     }
-    *reinterpret_cast<uint4 *>(out + blk * EBLK_BYTES + L * 16) =
-        make_uint4(words[0], words[1], words[2], words[3]);
+    if (bad) raise_error(ERRBIT_DEVICE);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) rowb[t][q] = wd[q];
+    __syncthreads();
+    const int m0 = t & 7, k1 = (t >> 3) & 1, m2 = t >> 4;
+    const uint16_t *h0 = reinterpret_cast<const uint16_t *>(rowb[m0 + 16 * m2]);
+    const uint16_t *h1 = reinterpret_cast<const uint16_t *>(rowb[m0 + 16 * m2 + 8]);
+    uint32_t o[4];
+#pragma unroll
+    for (int k2 = 0; k2 < 4; ++k2)
+        o[k2] = static_cast<uint32_t>(h0[k1 + 2 * k2]) | (static_cast<uint32_t>(h1[k1 + 2 * k2]) << 16);
+    *reinterpret_cast<uint4 *>(out + blk * EBLK_BYTES + t * 16) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // ---------------------------------------------------------------------------
@@ -471,6 +641,16 @@ __device__ __forceinline__ bool pair_b_by_tma(int mode, int64_t kb) {
 // split tile is always the first segment of its range, the owner's part the
 // last, so the owner only waits at the very end of its work.
 // ---------------------------------------------------------------------------
+// 6:8: the K' blocks in the order the library kernel's producer visits them --
+// the blocks that are tiles of X itself first, the middle-window blocks (from
+// the gathered X_mid) last -- so that the gather launched just before the GEMM
+// overlaps the first two thirds of every tile's mainloop.  The packed layout
+// is unchanged; only the order of the fp32 accumulation differs.
+__device__ __forceinline__ int64_t visit68(int64_t v, int64_t nkb) {
+    const int64_t nraw = 2 * (nkb / 3);
+    return v < nraw ? 3 * (v >> 1) + (v & 1) : 3 * (v - nraw) + 2;
+}
+
 struct SegIter {
     bool sk;
     int64_t nkb, pos, end, step;
@@ -529,11 +709,11 @@ __device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t *p) {
 // bounded wait for a stream-K flag (all lanes poll; one second limit)
 __device__ __forceinline__ bool sk_wait_flag(const uint64_t *p, uint64_t seq) {
     if (ld_acquire_u64(p) == seq) return true;
-    const uint64_t t0 = global_timer_ns();
+    const uint64_t t0 = global_timer_ns(), limit = wait_limit_ns();
     while (true) {
         __nanosleep(64);
         if (ld_acquire_u64(p) == seq) return true;
-        if (global_timer_ns() - t0 > WAIT_LIMIT_NS) {
+        if (global_timer_ns() - t0 > limit) {
             raise_error(ERRBIT_TIMEOUT);
             return false;
         }
@@ -740,7 +920,8 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
                 if (lane == 0) mbar_arrive_cluster(buf == 0 ? acc_empty_cl0 : acc_empty_cl1);
                 __threadfence();
                 __syncwarp();
-                if (lane == 0) st_release_u64(flags + (cluster * 2 + rank) * 8 + we, seq);
+                if (lane == 0 && cluster != g_test_withhold_flag_cluster)
+                    st_release_u64(flags + (cluster * 2 + rank) * 8 + we, seq);
                 continue;
             }
             // owner: the clusters after this one that hold the rest of the tile
@@ -1066,14 +1247,18 @@ __global__ void __launch_bounds__(WideCfg::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     // everything above overlaps the previous kernel's tail (programmatic
-    // dependent launch); global memory is touched only after this
-    grid_dep_wait();
+    // dependent launch); global memory is touched only after this.  For 6:8
+    // the producer reads only inputs older than that kernel (X, the packed
+    // weights) until its first middle-window block and waits there; the MMA
+    // warp touches no global memory.
+    if (MODE != PMODE_SP68T || warp >= 2) grid_dep_wait();
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
             int64_t it = 0;
             bool ok = true;
+            bool dep_done = MODE != PMODE_SP68T;
             SegIter seg(sk, cluster, nclusters, ntiles, nkb);
             int64_t tile, kb0, kb1;
             const uint32_t b_bytes = static_cast<uint32_t>(bh) * 256u;
@@ -1084,7 +1269,13 @@ __global__ void __launch_bounds__(WideCfg::THREADS, 1)
                 const int32_t brow = static_cast<int32_t>(nt * bn + rank * bh);
                 const int64_t e0 = (mt * 4 + rank) * nkb, e1 = (mt * 4 + 2 + rank) * nkb;
                 const uint32_t tx = 2u * ((has1 ? 2u : 1u) * (C::A_BYTES + EBLK_BYTES) + b_bytes);
-                for (int64_t kb = kb0; kb < kb1; ++kb, ++it) {
+                for (int64_t v = kb0; v < kb1; ++v, ++it) {
+                    const int64_t kb = MODE == PMODE_SP68T ? visit68(v, nkb) : v;
+                    const bool mid = MODE == PMODE_SP68T && (kb % 3) == 2;
+                    if (mid && !dep_done) {  // X_mid is the previous kernel's output
+                        grid_dep_wait();
+                        dep_done = true;
+                    }
                     const int s = static_cast<int>(it % S);
                     const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
                     if (it >= S && !mbar_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
@@ -1099,7 +1290,6 @@ __global__ void __launch_bounds__(WideCfg::THREADS, 1)
                         tma_load_2d_pair(st + C::OFF_E1, &tmE, bar, 0,
                                          static_cast<int32_t>((e1 + kb) * 8));
                     }
-                    const bool mid = MODE == PMODE_SP68T && (kb % 3) == 2;
                     const int64_t x0 = MODE == PMODE_SP24 ? kb * 128
                                        : (mid ? (kb / 3) * 128 : (kb / 3) * 256 + (kb % 3) * 128);
                     const CUtensorMap *tb = mid ? &tmB2 : &tmB;
@@ -1207,7 +1397,8 @@ __global__ void __launch_bounds__(WideCfg::THREADS, 1)
                 if (lane == 0) mbar_arrive_cluster(acc_empty_cl);
                 __threadfence();
                 __syncwarp();
-                if (lane == 0) st_release_u64(flags + (cluster * 2 + rank) * 8 + we, seq);
+                if (lane == 0 && cluster != g_test_withhold_flag_cluster)
+                    st_release_u64(flags + (cluster * 2 + rank) * 8 + we, seq);
                 continue;
             }
             // bf16 out.  The cluster's last segment: every pipeline stage is idle
@@ -1664,30 +1855,77 @@ extern "C" size_t nm_sparse_prepare_bytes(int64_t R, int64_t K, int m) {
     return static_cast<size_t>(p.vals_bytes + p.meta_bytes);
 }
 
+namespace {
+
+// a6 (and, from the mask, a4): the packed values, then the metadata blocks
+nm_status launch_prepare(const uint16_t *vals, const uint8_t *wmeta, const uint32_t *mask, int64_t R,
+                         int64_t K, int m, void *packed, cudaStream_t s) {
+    const PackedGeom p = packed_geom(R, K, m);
+    const int n = m - 2;
+    if (m == 8) {
+        const int64_t nj = p.nkb / 3;
+        const int64_t warps = p.Rpad * nj;
+        if ((warps + 7) / 8 > 0x7FFFFFFF) return NM_ERR_SHAPE;
+        k_prepare_vals68<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, s>>>(
+            vals, R, p.G, p.Rpad, nj, p.KLpad / 2, static_cast<uint16_t *>(packed));
+    } else {
+        const int64_t chunks = p.KLpad / 16;  // 16-byte chunks of a packed row
+        const int64_t words = p.G * n / 2;
+        const bool vec = (words % 4) == 0 && (reinterpret_cast<uintptr_t>(vals) & 15u) == 0;
+        dim3 vgrid(static_cast<unsigned>((chunks + 255) / 256),
+                   static_cast<unsigned>(p.Rpad < 65535 ? p.Rpad : 65535),
+                   static_cast<unsigned>((p.Rpad + 65534) / 65535));
+        k_prepare_vals<<<vgrid, 256, 0, s>>>(vals, R, words, p.Rpad, p.KLpad / 2, vec,
+                                             static_cast<uint16_t *>(packed));
+    }
+    const int64_t nblocks = (p.Rpad / BM) * p.nkb;
+    if (nblocks > 0x7FFFFFFF) return NM_ERR_SHAPE;
+    uint8_t *meta = static_cast<uint8_t *>(packed) + p.vals_bytes;
+    const int64_t mwords = (p.G * m + 31) / 32;
+    const unsigned nb = static_cast<unsigned>(nblocks);
+    const int64_t wb = (p.nwin + 1) / 2;
+#define NM_PREP_META(MM)                                                                                   \
+    (mask ? (k_prepare_meta<MM, true><<<nb, BM, 0, s>>>(nullptr, mask, R, p.G, 0, mwords, p.nkb, meta), 0) \
+          : (k_prepare_meta<MM, false><<<nb, BM, 0, s>>>(wmeta, nullptr, R, p.G, wb, 0, p.nkb, meta), 0))
+    switch (m) {
+        case 4: NM_PREP_META(4); break;
+        case 6: NM_PREP_META(6); break;
+        case 8: NM_PREP_META(8); break;
+        default: NM_PREP_META(10); break;
+    }
+#undef NM_PREP_META
+    return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
+}
+
+nm_status check_prepare(const uint16_t *vals, const void *meta_src, int64_t R, int64_t K, int m,
+                        const void *packed, size_t packed_bytes) {
+    if (!vals || !meta_src || !packed) return NM_ERR_NULL;
+    if (R < 1 || K < 1) return NM_ERR_SHAPE;
+    if (m != 4 && m != 6 && m != 8 && m != 10) return NM_ERR_UNSUPPORTED;
+    if (!aligned16(packed) || (reinterpret_cast<uintptr_t>(vals) & 3u)) return NM_ERR_ALIGN;
+    const PackedGeom p = packed_geom(R, K, m);
+    if (packed_bytes < static_cast<size_t>(p.vals_bytes + p.meta_bytes)) return NM_ERR_WORKSPACE;
+    if (p.Rpad > 65535LL * 65535LL) return NM_ERR_SHAPE;
+    return NM_OK;
+}
+
+}  // namespace
+
 extern "C" nm_status nm_sparse_prepare(const uint16_t *vals, const uint8_t *wmeta, int64_t R,
                                        int64_t K, int m, void *packed, size_t packed_bytes,
                                        void *stream) {
-    if (!vals || !wmeta || !packed) return NM_ERR_NULL;
-    if (R < 1 || K < 1) return NM_ERR_SHAPE;
-    if (m != 4 && m != 6 && m != 8 && m != 10) return NM_ERR_UNSUPPORTED;
-    if (!aligned16(packed)) return NM_ERR_ALIGN;
-    const PackedGeom p = packed_geom(R, K, m);
-    if (packed_bytes < static_cast<size_t>(p.vals_bytes + p.meta_bytes)) return NM_ERR_WORKSPACE;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const int n = m - 2;
-    const int64_t chunks = p.KLpad / 16;  // 16-byte chunks of a packed row
-    dim3 vgrid(static_cast<unsigned>((chunks + 255) / 256),
-               static_cast<unsigned>(p.Rpad < 65535 ? p.Rpad : 65535),
-               static_cast<unsigned>((p.Rpad + 65534) / 65535));
-    k_prepare_vals<<<vgrid, 256, 0, s>>>(vals, R, p.G, n, m, p.Rpad, p.KLpad / 2,
-                                         static_cast<uint16_t *>(packed));
-    const int64_t nblocks = (p.Rpad / BM) * p.nkb;
-    const int64_t mblocks = (nblocks * 128 + 255) / 256;
-    if (mblocks > 0x7FFFFFFF) return NM_ERR_SHAPE;
-    k_prepare_meta<<<static_cast<unsigned>(mblocks), 256, 0, s>>>(
-        wmeta, R, p.G, m, (p.nwin + 1) / 2, p.nkb, nblocks,
-        static_cast<uint8_t *>(packed) + p.vals_bytes);
-    return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
+    const nm_status st = check_prepare(vals, wmeta, R, K, m, packed, packed_bytes);
+    if (st != NM_OK) return st;
+    return launch_prepare(vals, wmeta, nullptr, R, K, m, packed, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" nm_status nm_sparse_prepare_from_mask(const uint16_t *vals, const uint32_t *mask, int64_t R,
+                                                 int64_t K, int m, void *packed, size_t packed_bytes,
+                                                 void *stream) {
+    const nm_status st = check_prepare(vals, mask, R, K, m, packed, packed_bytes);
+    if (st != NM_OK) return st;
+    if (reinterpret_cast<uintptr_t>(mask) & 3u) return NM_ERR_ALIGN;
+    return launch_prepare(vals, nullptr, mask, R, K, m, packed, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // extra device memory the online phase needs for (2N-2):2N patterns: the

@@ -3,8 +3,8 @@
 // All of these are HBM-streaming kernels: each reads its operand once with
 // coalesced vector loads and writes its outputs once.  Bit-exact by
 // construction with any implementation of the same definitions:
-//   * H uses a fixed summation order (chunks of 128 tokens, each the ordered
-//     sum of eight sequential 16-token runs);
+//   * H (and the ternary gamma) is the exact sum rounded once, then divided
+//     once, so no summation order enters it (see "Exact sums" below);
 //   * S uses fp64 add/multiply with explicit round-to-nearest intrinsics (no
 //     FMA contraction) and one fp64 -> fp32 rounding;
 //   * selection is integer logic on fp32 comparisons.
@@ -18,14 +18,6 @@
 
 namespace nm {
 
-constexpr int H_CHUNK = 128;                  // tokens per chunk partial of H
-constexpr int H_SLICE = 16;                   // tokens per sequential run inside a chunk
-constexpr int H_SLICES = H_CHUNK / H_SLICE;   // 8 runs, one half-warp each
-constexpr int H_VEC = 8;                      // columns per thread: one 16-byte load per token
-constexpr int H_GROUPS = 16;                  // column groups per block (a half-warp's lanes)
-constexpr int H_BLOCK_COLS = H_GROUPS * H_VEC;     // 128 columns per block
-constexpr int H_THREADS = H_GROUPS * H_SLICES;     // 128
-
 __device__ __forceinline__ double bf16_to_f64(uint16_t b) {
     return static_cast<double>(__uint_as_float(static_cast<uint32_t>(b) << 16));
 }
@@ -34,128 +26,423 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t b) {
 }
 
 // ---------------------------------------------------------------------------
-// a1: column sums of squares.  A block owns 128 columns and a strided set of
-// 128-token chunks (chunks y, y + gridDim.y, ...).  Each chunk tile
-// [128 tokens x 128 columns] bf16 (32 KB) is brought into shared memory by
-// TMA, three tiles in flight, so that the loads of later chunks overlap the
-// arithmetic on the current one (two blocks per SM).  In a tile, lane g of
-// half-warp r owns columns 8g..8g+7 and tokens 16r..16r+15 and adds x^2 per
-// column in ascending t.  The eight 16-token runs are added in ascending
-// order through shared memory, giving the chunk partial; with a single chunk
-// the kernel writes H directly.  Rows past T and columns past K arrive as
-// zeros from the tensor map, and adding +0.0 leaves a sum of squares as it is.
-//
-// x^2 of a bf16 value is exact in fp64, so fma(x, x, acc) rounds exactly like
-// acc + x*x.
+// Exact sums (H and the ternary gamma).  Both are means of terms that are
+// integer multiples of a power of two: a bf16 value with exponent field e and
+// significand m (m = 128 + fraction for e >= 1, the fraction for e = 0) is
+// m 2^(max(e,1) - 134), its square m^2 2^(2 max(e,1) - 268).  The library
+// returns the exact sum rounded once to fp64 (nearest, ties to even), divided
+// once by the count, so that no summation order enters the result.  Three
+// facts let the kernels sum in any order and still be exact:
+//  (1) fp64 additions of non-negative terms, all integer multiples of a unit
+//      u, are exact while the sum stays below 2^53 u: every partial sum is
+//      then a multiple of u below 2^53 u, hence representable, and once an
+//      addition rounds the running sum is >= 2^53 u for good.  A run whose
+//      result is below that bound was therefore summed exactly; u is the
+//      unit of the run's smallest nonzero term.
+//  (1') The same chain done twice, rounding every step up and then down,
+//      brackets the exact sum (up >= exact >= down, whatever the signs);
+//      equal results are the exact sum.
+//  (2) Knuth's TwoSum splits a + b into s + e exactly (round to nearest), so a
+//      chain of exact partial sums carried as a pair (s, c), the e's summed
+//      into c up and down as in (1'), is the exact total when c's two results
+//      agree; fl(s + c) is then its correct rounding.
+//  (3) Anything that fails a check (a subnormal, an infinity, a NaN, or a
+//      range of magnitudes wider than the checks allow) is summed again in
+//      parts or with integer arithmetic (BigAcc).
 // ---------------------------------------------------------------------------
-constexpr int H_STAGES = 3;
-constexpr int H_TILE_BYTES = H_CHUNK * H_BLOCK_COLS * 2;  // 32 KB
-constexpr int H_RUN_BYTES = H_SLICES * H_VEC * (H_GROUPS + 1) * 8;
-constexpr int H_SMEM_BYTES = H_STAGES * H_TILE_BYTES + H_RUN_BYTES + 64 + 1024;
 
-__device__ __forceinline__ double bf16lo_to_f64(uint32_t w) {
-    return static_cast<double>(__uint_as_float(w << 16));
+// fp64 whose high word is hw and low word zero
+__device__ __forceinline__ double hw_double(uint32_t hw) {
+    return __hiloint2double(static_cast<int>(hw), 0);
 }
-__device__ __forceinline__ double bf16hi_to_f64(uint32_t w) {
-    return static_cast<double>(__uint_as_float(w & 0xFFFF0000u));
+__device__ __forceinline__ uint32_t vmin_s16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("min.s16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
 }
-
-__device__ __forceinline__ void sq_acc_conv(uint32_t w, double &a0, double &a1) {
-    const double x0 = bf16lo_to_f64(w), x1 = bf16hi_to_f64(w);
-    a0 = __fma_rn(x0, x0, a0);
-    a1 = __fma_rn(x1, x1, a1);
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
 }
 
-__global__ void __launch_bounds__(H_THREADS, 2)
-    k_colsumsq_chunk(const __grid_constant__ CUtensorMap tmX, int64_t T, int64_t K, int64_t nchunks,
-                     double *__restrict__ out, int direct) {
-    extern __shared__ uint8_t h_smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(h_smem_raw) + 1023) &
+// TwoSum into (s, c) with c carried both up and down (fact 2)
+__device__ __forceinline__ void two_sum_acc2(double &s, double &cu, double &cd, double a) {
+    const double t = __dadd_rn(s, a);
+    const double bb = __dsub_rn(t, s);
+    const double err = __dadd_rn(__dsub_rn(s, __dsub_rn(t, bb)), __dsub_rn(a, bb));
+    s = t;
+    cu = __dadd_ru(cu, err);
+    cd = __dadd_rd(cd, err);
+}
+
+// Integer accumulator: sum of d[i] 2^(32 i - BIAS), 32-bit digits carried in
+// signed 64-bit limbs (carries resolved once, in round_rn), so up to 2^31 adds.
+template <int NDIG, int BIAS>
+struct BigAcc {
+    long long d[NDIG];
+    __device__ __forceinline__ void clear() {
+#pragma unroll
+        for (int i = 0; i < NDIG; ++i) d[i] = 0;
+    }
+    // += v * 2^(pos - BIAS) (v < 2^53, 0 <= pos), negative when neg
+    __device__ void add_bits(unsigned long long v, int pos, bool neg) {
+        const int q = pos >> 5, b = pos & 31;
+        const unsigned long long lo = (v << b) & 0xFFFFFFFFull;
+        const unsigned long long mid = b ? ((v >> (32 - b)) & 0xFFFFFFFFull) : ((v >> 32) & 0xFFFFFFFFull);
+        const unsigned long long hi = b ? (v >> (64 - b)) : 0ull;
+        const long long sg = neg ? -1 : 1;
+        d[q] += sg * static_cast<long long>(lo);
+        if (q + 1 < NDIG) d[q + 1] += sg * static_cast<long long>(mid);
+        if (q + 2 < NDIG) d[q + 2] += sg * static_cast<long long>(hi);
+    }
+    // += v, v finite and an integer multiple of 2^-BIAS
+    __device__ void add_double(double v) {
+        const unsigned long long u = static_cast<unsigned long long>(__double_as_longlong(v));
+        const int ef = static_cast<int>((u >> 52) & 0x7FF);
+        unsigned long long mant = u & 0xFFFFFFFFFFFFFull;
+        if (ef == 0 && mant == 0) return;
+        if (ef) mant |= 1ull << 52;
+        int pos = (ef ? ef : 1) - 1075 + BIAS;  // position of mant's bit 0
+        if (pos < 0) {                          // only zero bits drop here
+            mant >>= -pos;
+            pos = 0;
+        }
+        add_bits(mant, pos, (u >> 63) != 0);
+    }
+    // the value rounded to the nearest double (ties to even); must be >= 0
+    __device__ double round_rn() const {
+        long long n[NDIG];
+        long long carry = 0;
+#pragma unroll
+        for (int i = 0; i < NDIG; ++i) {
+            const long long v = d[i] + carry;
+            carry = v >> 32;  // arithmetic shift: floor division
+            n[i] = v & 0xFFFFFFFFll;
+        }
+        int top = NDIG - 1;
+        while (top >= 0 && n[top] == 0) --top;
+        if (top < 0) return 0.0;
+        const unsigned long long d2 = static_cast<unsigned long long>(n[top]);
+        const unsigned long long d1 = top >= 1 ? static_cast<unsigned long long>(n[top - 1]) : 0ull;
+        const unsigned long long d0 = top >= 2 ? static_cast<unsigned long long>(n[top - 2]) : 0ull;
+        bool sticky_low = false;
+        for (int i = 0; i < top - 2; ++i) sticky_low |= n[i] != 0;
+        const unsigned __int128 w = (static_cast<unsigned __int128>(d2) << 64) |
+                                    (static_cast<unsigned __int128>(d1) << 32) | d0;
+        const int tb = 64 + 31 - __clz(static_cast<unsigned>(d2));  // top bit of w
+        const int sh = tb - 52;                                       // >= 12
+        unsigned long long sig = static_cast<unsigned long long>(w >> sh);
+        const unsigned __int128 rem = w & ((static_cast<unsigned __int128>(1) << sh) - 1);
+        const bool rbit = ((rem >> (sh - 1)) & 1) != 0;
+        const bool sticky = (rem & ((static_cast<unsigned __int128>(1) << (sh - 1)) - 1)) != 0 || sticky_low;
+        if (rbit && (sticky || (sig & 1ull))) ++sig;  // 2^53 is still exact
+        return scalbn(static_cast<double>(sig), sh + 32 * (top - 2) - BIAS);
+    }
+};
+
+// sums of squares: units of 2^-266 (the square of the smallest subnormal),
+// room for T < 2^31 squares below 2^256
+constexpr int HB_NDIG = 19;
+constexpr int HB_BIAS = 266;
+using SqAcc = BigAcc<HB_NDIG, HB_BIAS>;
+
+// sum of x^2 over one column of X, exactly, rounded once; NaN if the column
+// holds a NaN, else +inf if it holds an infinity.  One thread, plain loads:
+// the path for columns whose fast sums failed a check.
+__device__ __noinline__ double exact_sq_column(const uint16_t *__restrict__ X, int64_t ldx, int64_t T, int64_t col) {
+    SqAcc a;
+    a.clear();
+    bool nan = false, inf = false;
+    for (int64_t t = 0; t < T; ++t) {
+        const uint32_t b = X[t * ldx + col] & 0x7FFFu;
+        const int e = static_cast<int>(b >> 7);
+        const uint32_t f = b & 0x7Fu;
+        if (e == 255) {
+            nan |= f != 0;
+            inf |= f == 0;
+            continue;
+        }
+        if (b == 0) continue;
+        const unsigned long long m = e ? 128u + f : f;
+        a.add_bits(m * m, 2 * (e ? e : 1) - 268 + HB_BIAS, false);
+    }
+    if (nan) return __longlong_as_double(0x7FF8000000000000ll);
+    if (inf) return __longlong_as_double(0x7FF0000000000000ll);
+    return a.round_rn();
+}
+
+// ---------------------------------------------------------------------------
+// a1: H_j = fl(fl(sum_t x_{t,j}^2) / T).
+//
+// Block: 256 threads = 8 warps over one 128-column strip of X and a range of
+// 128-token chunks (blockIdx.y).  Each chunk tile [128 tokens x 128 columns]
+// bf16 (32 KB) comes into shared memory by TMA, three in flight (two blocks
+// per SM); rows past T and columns past K arrive as zeros.  In a tile, warp w
+// owns tokens 16w .. 16w+15 (a run) and lane l columns 4l .. 4l+3 (one 8-byte
+// shared-memory load per token, a warp reads one 256-byte row).  Per run a
+// thread sums x^2 per column twice, rounding up and rounding down (fact 1);
+// equal results are the exact run sum, which goes into the column's TwoSum
+// pair (fact 2).  A run whose two sums differ is summed again from the tile,
+// split into the values within 12 binades of the run's largest and the rest,
+// each part checked the same way; what still fails (an infinity, a NaN, a
+// range wider than that) marks the column for the integer path.  The eight
+// warps' pairs are added in shared memory, again checking c up against down.
+// A block that saw every token divides and writes H; otherwise it writes its
+// exact pair (s, c) -- or NaN in s for a marked column -- and k_hsq_finish
+// adds the pairs of a column.
+//
+// x^2 comes from the bits without a conversion: d = x 2^-896 is the fp64
+// with high word (bits & 0x7FFF) << 13 and g = x 2^896 the same plus
+// 1792 << 20, so d * g = x^2 exactly for every normal x and zero (d = 0), and
+// fma(d, g, acc) rounds like acc + x^2; an infinity or a NaN makes g, hence
+// the sum, inf or NaN, which fails the check.  The check of fact (1) needs the
+// run's smallest nonzero magnitude, kept two columns at a time as a signed
+// 16-bit minimum of t + 0x7FFF over the magnitude bits t (0x7FFF for a zero,
+// the largest; 0x8000 + t - 1, negative and increasing in t, otherwise).  A
+// subnormal (exponent field 0, where g is wrong) fails the check as well.
+// ---------------------------------------------------------------------------
+constexpr int HX_THREADS = 256;
+constexpr int HX_WARPS = HX_THREADS / 32;
+constexpr int HX_VEC = 4;                 // columns per thread
+constexpr int HX_COLS = 32 * HX_VEC;      // columns per block (one TMA box row: 256 bytes)
+constexpr int HX_RUN = 16;                // tokens per checked run (one warp per run)
+constexpr int HX_CHUNK = HX_RUN * HX_WARPS;   // tokens per tile: 128
+constexpr int HX_STAGES = 3;
+constexpr int HX_TILE_BYTES = HX_CHUNK * HX_COLS * 2;                   // 32 KB
+constexpr int HX_SMEM_BYTES = HX_STAGES * HX_TILE_BYTES + 64 + 1024;    // + barriers, alignment
+constexpr int64_t HX_SLOTS = 2 * 148;     // resident blocks at 2 per SM on 148 SMs: the grid's target
+
+struct HPair {
+    double s, c;
+};
+
+// x^2 of the two bf16 halves of a word (low half: w << 13; high half: w >> 3)
+// into the sums of columns k, k + 1, and their smallest magnitudes into key
+__device__ __forceinline__ void sq_word(uint32_t w, double (&a)[HX_VEC], uint32_t &key, int k) {
+    const uint32_t d0 = (w << 13) & 0x0FFFE000u, d1 = (w >> 3) & 0x0FFFE000u;
+    a[k] = __fma_rn(hw_double(d0), hw_double(d0 + 0x70000000u), a[k]);
+    a[k + 1] = __fma_rn(hw_double(d1), hw_double(d1 + 0x70000000u), a[k + 1]);
+    key = vmin_s16x2(key, (w & 0x7FFF7FFFu) + 0x7FFF7FFFu);
+}
+
+// fact (1) for a run: no nonzero value (key 0x7FFF), or a normal smallest
+// value (exponent field e >= 1) and a sum below 2^53 units of its square,
+// 2^(2e - 268 + 53), whose fp64 exponent field is 2e + 808
+__device__ __forceinline__ bool sq_run_exact(double a, uint32_t key16) {
+    if (key16 == 0x7FFFu) return true;
+    const int e = static_cast<int>((key16 - 0x7FFFu) >> 7);
+    return e >= 1 && a < hw_double(static_cast<uint32_t>(2 * e + 808) << 20);
+}
+
+// A run that failed its check, summed again from the tile in two parts: the
+// values within 12 binades of the run's largest (16 squares below
+// 2^(2 emax - 252) on a grid of 2^(2 emax - 292): exact) and the smaller ones,
+// each summed up and down (fact 1').  x = d * 2^896 is exact for subnormals
+// too.  ok = false for an infinity, a NaN, or a run too wide for that split.
+// `col` points at the column's first element of the run in the tile (row
+// pitch HX_COLS elements).
+struct RunSplit {
+    double big, small;
+    bool ok;
+};
+__device__ __noinline__ RunSplit sq_run_split(const uint16_t *col) {
+    RunSplit r{0.0, 0.0, false};
+    uint32_t b[HX_RUN];
+    int emax = 0;
+#pragma unroll
+    for (int u = 0; u < HX_RUN; ++u) {
+        b[u] = col[u * HX_COLS] & 0x7FFFu;
+        if (b[u] >= 0x7F80u) return r;
+        emax = max(emax, static_cast<int>(b[u] >> 7));
+    }
+    const int thr = emax - 12;
+    double bu = 0.0, bd = 0.0, su = 0.0, sd = 0.0;
+#pragma unroll
+    for (int u = 0; u < HX_RUN; ++u) {
+        const double x = __dmul_rn(hw_double(b[u] << 13), 0x1p896);
+        if (static_cast<int>(b[u] >> 7) >= thr) {
+            bu = __fma_ru(x, x, bu);
+            bd = __fma_rd(x, x, bd);
+        } else {
+            su = __fma_ru(x, x, su);
+            sd = __fma_rd(x, x, sd);
+        }
+    }
+    r.big = bu;
+    r.small = su;
+    r.ok = bu == bd && su == sd;
+    return r;
+}
+
+__global__ void __launch_bounds__(HX_THREADS, 2)
+    k_hsq(const __grid_constant__ CUtensorMap tmX, const uint16_t *__restrict__ X, int64_t T, int64_t K,
+          int64_t ldx, HPair *__restrict__ part, double *__restrict__ H) {
+    extern __shared__ uint8_t hx_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(hx_smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
-    double(*run)[H_VEC][H_GROUPS + 1] =
-        reinterpret_cast<double(*)[H_VEC][H_GROUPS + 1]>(smem + H_STAGES * H_TILE_BYTES);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + H_STAGES * H_TILE_BYTES + H_RUN_BYTES);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + HX_STAGES * HX_TILE_BYTES);
     grid_dep_launch();
-    const int g = threadIdx.x & (H_GROUPS - 1), r = threadIdx.x / H_GROUPS;
-    const int32_t xcol = static_cast<int32_t>(blockIdx.x) * H_BLOCK_COLS;
-    const int64_t mine = (nchunks - blockIdx.y + gridDim.y - 1) / gridDim.y;  // chunks of this block
-    auto chunk_of = [&](int64_t i) { return static_cast<int64_t>(blockIdx.y) + i * gridDim.y; };
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int32_t xcol = static_cast<int32_t>(blockIdx.x) * HX_COLS;
+    // token range blockIdx.y of gridDim.y: chunks [y n / split, (y + 1) n / split)
+    const int64_t nchunks = (T + HX_CHUNK - 1) / HX_CHUNK;
+    const int64_t cbeg = static_cast<int64_t>(blockIdx.y) * nchunks / gridDim.y;
+    const int64_t mine = (static_cast<int64_t>(blockIdx.y) + 1) * nchunks / gridDim.y - cbeg;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < H_STAGES; ++s) mbar_init(&full[s], 1);
+        for (int st = 0; st < HX_STAGES; ++st) mbar_init(&full[st], 1);
         fence_barrier_init();
         prefetch_tmap(&tmX);
-        for (int64_t i = 0; i < mine && i < H_STAGES; ++i) {
-            mbar_arrive_expect_tx(&full[i], H_TILE_BYTES);
-            tma_load_2d(smem + i * H_TILE_BYTES, &tmX, &full[i], xcol,
-                        static_cast<int32_t>(chunk_of(i) * H_CHUNK));
+        for (int64_t i = 0; i < mine && i < HX_STAGES; ++i) {
+            mbar_arrive_expect_tx(&full[i], HX_TILE_BYTES);
+            tma_load_2d(smem + i * HX_TILE_BYTES, &tmX, &full[i], xcol, static_cast<int32_t>((cbeg + i) * HX_CHUNK));
         }
     }
     __syncthreads();
-    int64_t issued = mine < H_STAGES ? mine : H_STAGES;
-    const int c = threadIdx.x;  // the column this thread finishes in the ordered run sum
-    const int64_t col = static_cast<int64_t>(xcol) + c;
-    for (int64_t i = 0; i < mine; ++i) {
-        const int s = static_cast<int>(i % H_STAGES);
-        const bool ok = __syncthreads_and(mbar_wait(&full[s], static_cast<uint32_t>((i / H_STAGES) & 1)));
-        if (!ok) {  // timed out (error word set): let the copies in flight land, then leave
-            if (threadIdx.x == 0)
-                for (int64_t j = i; j < issued; ++j)
-                    mbar_wait(&full[j % H_STAGES], static_cast<uint32_t>((j / H_STAGES) & 1));
-            return;
-        }
-        const uint8_t *tile = smem + s * H_TILE_BYTES + (r * H_SLICE) * (H_BLOCK_COLS * 2) + g * 16;
-        double acc[H_VEC];
+    double s[HX_VEC], cu[HX_VEC], cd[HX_VEC];
 #pragma unroll
-        for (int k = 0; k < H_VEC; ++k) acc[k] = 0.0;
-#pragma unroll 4
-        for (int u = 0; u < H_SLICE; ++u) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(tile + u * (H_BLOCK_COLS * 2));
-            sq_acc_conv(v.x, acc[0], acc[1]);
-            sq_acc_conv(v.y, acc[2], acc[3]);
-            sq_acc_conv(v.z, acc[4], acc[5]);
-            sq_acc_conv(v.w, acc[6], acc[7]);
-        }
+    for (int k = 0; k < HX_VEC; ++k) s[k] = cu[k] = cd[k] = 0.0;
+    uint32_t bad = 0;
+    int64_t issued = mine < HX_STAGES ? mine : HX_STAGES;
+    bool ok = true;
+    int64_t i = 0;
+    for (; i < mine; ++i) {
+        const int st = static_cast<int>(i % HX_STAGES);
+        ok = __syncthreads_and(mbar_wait(&full[st], static_cast<uint32_t>((i / HX_STAGES) & 1)));
+        if (!ok) break;  // timed out (error word set)
+        const uint16_t *tile = reinterpret_cast<const uint16_t *>(smem + st * HX_TILE_BYTES) +
+                               (warp * HX_RUN) * HX_COLS + HX_VEC * lane;
+        double a[HX_VEC] = {0.0, 0.0, 0.0, 0.0};
+        uint32_t key0 = 0x7FFF7FFFu, key1 = 0x7FFF7FFFu;
 #pragma unroll
-        for (int k = 0; k < H_VEC; ++k) run[r][k][g] = acc[k];
-        __syncthreads();  // tile s consumed by every thread; the runs are complete
+        for (int u = 0; u < HX_RUN; ++u) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(tile + u * HX_COLS);
+            sq_word(v.x, a, key0, 0);
+            sq_word(v.y, a, key1, 2);
+        }
+        const uint32_t keys[HX_VEC] = {key0 & 0xFFFFu, key0 >> 16, key1 & 0xFFFFu, key1 >> 16};
+#pragma unroll
+        for (int k = 0; k < HX_VEC; ++k) {
+            if (sq_run_exact(a[k], keys[k])) {
+                two_sum_acc2(s[k], cu[k], cd[k], a[k]);
+            } else {
+                const RunSplit r = sq_run_split(tile + k);
+                if (r.ok) {
+                    two_sum_acc2(s[k], cu[k], cd[k], r.big);
+                    two_sum_acc2(s[k], cu[k], cd[k], r.small);
+                } else {
+                    bad |= 1u << k;
+                }
+            }
+        }
+        __syncthreads();  // stage st consumed by every warp
         if (threadIdx.x == 0 && issued < mine) {
-            mbar_arrive_expect_tx(&full[s], H_TILE_BYTES);
-            tma_load_2d(smem + s * H_TILE_BYTES, &tmX, &full[s], xcol,
-                        static_cast<int32_t>(chunk_of(issued) * H_CHUNK));
+            mbar_arrive_expect_tx(&full[st], HX_TILE_BYTES);
+            tma_load_2d(smem + st * HX_TILE_BYTES, &tmX, &full[st], xcol,
+                        static_cast<int32_t>((cbeg + issued) * HX_CHUNK));
             ++issued;
         }
-        if (col < K) {
-            double total = run[0][c % H_VEC][c / H_VEC];
+    }
+    if (!ok) {  // let the copies in flight (chunks i .. issued - 1) land, then leave
+        if (threadIdx.x == 0)
+            for (int64_t j = i; j < issued; ++j)
+                mbar_wait(&full[j % HX_STAGES], static_cast<uint32_t>((j / HX_STAGES) & 1));
+        return;
+    }
+    // the pipeline is drained: stage memory holds the warps' pairs
+    double(*sh_s)[HX_COLS] = reinterpret_cast<double(*)[HX_COLS]>(smem);
+    double(*sh_cu)[HX_COLS] = reinterpret_cast<double(*)[HX_COLS]>(smem + HX_WARPS * HX_COLS * 8);
+    double(*sh_cd)[HX_COLS] = reinterpret_cast<double(*)[HX_COLS]>(smem + 2 * HX_WARPS * HX_COLS * 8);
+    uint8_t(*sh_bad)[HX_COLS] = reinterpret_cast<uint8_t(*)[HX_COLS]>(smem + 3 * HX_WARPS * HX_COLS * 8);
 #pragma unroll
-            for (int q = 1; q < H_SLICES; ++q) total = __dadd_rn(total, run[q][c % H_VEC][c / H_VEC]);
-            if (direct)
-                out[col] = __ddiv_rn(total, static_cast<double>(T));
-            else
-                out[chunk_of(i) * K + col] = total;
-        }
-        __syncthreads();  // the runs are read before the next chunk overwrites them
+    for (int k = 0; k < HX_VEC; ++k) {
+        sh_s[warp][HX_VEC * lane + k] = s[k];
+        sh_cu[warp][HX_VEC * lane + k] = cu[k];
+        sh_cd[warp][HX_VEC * lane + k] = cd[k];
+        sh_bad[warp][HX_VEC * lane + k] = static_cast<uint8_t>((bad >> k) & 1u);
+    }
+    __syncthreads();
+    const int j = threadIdx.x;
+    const int64_t col = static_cast<int64_t>(xcol) + j;
+    if (j >= HX_COLS || col >= K) return;
+    double S = 0.0, CU = 0.0, CD = 0.0;
+    bool marked = false;
+#pragma unroll
+    for (int w = 0; w < HX_WARPS; ++w) {
+        two_sum_acc2(S, CU, CD, sh_s[w][j]);
+        CU = __dadd_ru(CU, sh_cu[w][j]);
+        CD = __dadd_rd(CD, sh_cd[w][j]);
+        marked |= sh_bad[w][j] != 0;
+    }
+    marked |= CU != CD;  // c not exact: its up and down sums differ (fact 2)
+    if (H != nullptr) {  // the block saw every token
+        const double sum = marked ? exact_sq_column(X, ldx, T, col) : __dadd_rn(S, CU);
+        H[col] = __ddiv_rn(sum, static_cast<double>(T));
+    } else {
+        HPair p;
+        p.s = marked ? __longlong_as_double(0x7FF8000000000000ll) : S;
+        p.c = marked ? 0.0 : CU;
+        part[static_cast<int64_t>(blockIdx.y) * K + col] = p;
     }
 }
 
-// sums the chunk partials in ascending chunk order, then divides by T;
-// launched as a programmatic dependent of k_colsumsq_chunk
-__global__ void __launch_bounds__(64) k_colsumsq_finish(const double *__restrict__ part, int64_t nchunks,
-                                                         int64_t T, int64_t K, double *__restrict__ H) {
+// adds the blocks' exact pairs of a column -- with TwoSum, c up and down as
+// in fact 2, or where those differ with integer arithmetic -- and rounds once
+// (a marked pair: the column again, on the integer path); launched as a
+// programmatic dependent of k_hsq
+__global__ void __launch_bounds__(128) k_hsq_finish(const HPair *__restrict__ part, int64_t nparts,
+                                                    const uint16_t *__restrict__ X, int64_t T, int64_t K,
+                                                    int64_t ldx, double *__restrict__ H) {
     grid_dep_wait();
     const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (j >= K) return;
-    // loads run ahead of the (ordered) additions, 32 partials at a time
-    double total = 0.0;
-    int64_t c = 0;
-    for (; c + 32 <= nchunks; c += 32) {
-        double v[32];
+    double S = 0.0, CU = 0.0, CD = 0.0;
+    bool marked = false;
+    // the pairs eight at a time: their loads go out together
+    for (int64_t y0 = 0; y0 < nparts; y0 += 8) {
+        HPair p[8];
 #pragma unroll
-        for (int u = 0; u < 32; ++u) v[u] = part[(c + u) * K + j];
+        for (int q = 0; q < 8; ++q) p[q] = y0 + q < nparts ? part[(y0 + q) * K + j] : HPair{0.0, 0.0};
 #pragma unroll
-        for (int u = 0; u < 32; ++u) total = __dadd_rn(total, v[u]);
+        for (int q = 0; q < 8; ++q) {
+            marked |= isnan(p[q].s);
+            two_sum_acc2(S, CU, CD, p[q].s);
+            CU = __dadd_ru(CU, p[q].c);
+            CD = __dadd_rd(CD, p[q].c);
+        }
     }
-    for (; c < nchunks; ++c) total = __dadd_rn(total, part[c * K + j]);
-    H[j] = __ddiv_rn(total, static_cast<double>(T));
+    double sum;
+    if (marked) {
+        sum = exact_sq_column(X, ldx, T, j);
+    } else if (CU == CD) {
+        sum = __dadd_rn(S, CU);
+    } else {
+        SqAcc a;
+        a.clear();
+        for (int64_t y = 0; y < nparts; ++y) {
+            const HPair p = part[y * K + j];
+            a.add_double(p.s);
+            a.add_double(p.c);
+        }
+        sum = a.round_rn();
+    }
+    H[j] = __ddiv_rn(sum, static_cast<double>(T));
+}
+
+// grid of the H reduction: (column strips, token ranges); the 128-token
+// chunks are spread evenly over the ranges
+struct HGrid {
+    int64_t cblocks, split;
+};
+inline HGrid h_grid(int64_t T, int64_t K, int64_t max_split) {
+    HGrid g;
+    g.cblocks = (K + HX_COLS - 1) / HX_COLS;
+    const int64_t nchunks = (T + HX_CHUNK - 1) / HX_CHUNK;
+    int64_t split = HX_SLOTS / g.cblocks;  // one wave of resident blocks, no partial second one
+    split = split > nchunks ? nchunks : split;
+    split = split > max_split ? max_split : split;
+    g.split = split < 1 ? 1 : split;
+    return g;
 }
 
 // ---------------------------------------------------------------------------
@@ -877,57 +1164,72 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------------------------
-// ternary absmean quantisation
+// ternary absmean quantisation: gamma = fl(fl(sum |w|) / (R K)).
+//
+// k_row_abs_sum: one warp per row; lane l sums |w| of the 8-column chunks
+// l, l + 32, ... in fp64 as d = |w| 2^-896 (high word (bits & 0x7FFF) << 13:
+// exact for zeros and subnormals too), once rounding up and once down (fact
+// 1), and keeps the largest magnitude bits (an infinity or a NaN fails the
+// row).  The 32 lanes' sums are added with TwoSum (fact 2).  The row's exact
+// pair is written scaled back by 2^896 (exact), or NaN in s for a row that
+// failed a check.  k_gamma adds the pairs with integer arithmetic in one
+// block (a marked row summed again on the integer path) and divides once.
 // ---------------------------------------------------------------------------
-// Row sums of |W| in the canonical order: one warp per row; lane l sums the
-// 8-column chunks l, l+32, ... (16-byte loads, a warp instruction reads 512
-// contiguous bytes) left to right, then the 32 partials are combined by
-// halving (lane l adds lane l+16, then +8, +4, +2, +1).
+constexpr int GB_NDIG = 12;   // |w| sums: units of 2^-160, below 2^190
+constexpr int GB_BIAS = 160;
+using AbsAcc = BigAcc<GB_NDIG, GB_BIAS>;
+
+__device__ __forceinline__ void abs_word(uint32_t w, double &up, double &dn, uint32_t &kmax) {
+    const double d0 = hw_double((w << 13) & 0x0FFFE000u), d1 = hw_double((w >> 3) & 0x0FFFE000u);
+    up = __dadd_ru(__dadd_ru(up, d0), d1);
+    dn = __dadd_rd(__dadd_rd(dn, d0), d1);
+    kmax = vmax_u16x2(kmax, w & 0x7FFF7FFFu);
+}
+
 __global__ void __launch_bounds__(256)
-    k_row_abs_sum(const uint16_t *__restrict__ W, int64_t R, int64_t K, int64_t ldw,
-                  double *__restrict__ rowsum) {
+    k_row_abs_sum(const uint16_t *__restrict__ W, int64_t R, int64_t K, int64_t ldw, HPair *__restrict__ rec) {
     const int lane = threadIdx.x & 31;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     if (row >= R) return;  // warp-uniform
     const uint16_t *w = W + row * ldw;
     const int64_t nchunks = (K + 7) / 8;
-    double s = 0.0;
+    double up = 0.0, dn = 0.0;
+    uint32_t kmax = 0u;
     int64_t c = lane;
-    // four chunks in flight per lane
-    for (; c + 96 < nchunks && 8 * (c + 96) + 8 <= K; c += 128) {
+    for (; c + 96 < nchunks && 8 * (c + 96) + 8 <= K; c += 128) {  // four chunks in flight
         uint4 u[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) u[k] = __ldg(reinterpret_cast<const uint4 *>(w + 8 * (c + 32 * k)));
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const uint32_t q[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                s = __dadd_rn(s, fabs(bf16_to_f64(static_cast<uint16_t>(q[e] & 0xFFFFu))));
-                s = __dadd_rn(s, fabs(bf16_to_f64(static_cast<uint16_t>(q[e] >> 16))));
-            }
+            abs_word(u[k].x, up, dn, kmax);
+            abs_word(u[k].y, up, dn, kmax);
+            abs_word(u[k].z, up, dn, kmax);
+            abs_word(u[k].w, up, dn, kmax);
         }
     }
     for (; c < nchunks; c += 32) {
         const int64_t j0 = 8 * c;
         if (j0 + 8 <= K) {
             const uint4 u = __ldg(reinterpret_cast<const uint4 *>(w + j0));
-            const uint32_t q[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                s = __dadd_rn(s, fabs(bf16_to_f64(static_cast<uint16_t>(q[e] & 0xFFFFu))));
-                s = __dadd_rn(s, fabs(bf16_to_f64(static_cast<uint16_t>(q[e] >> 16))));
-            }
+            abs_word(u.x, up, dn, kmax);
+            abs_word(u.y, up, dn, kmax);
+            abs_word(u.z, up, dn, kmax);
+            abs_word(u.w, up, dn, kmax);
         } else {
-            for (int64_t j = j0; j < K; ++j) s = __dadd_rn(s, fabs(bf16_to_f64(w[j])));
+            for (int64_t j = j0; j < K; ++j) abs_word(w[j], up, dn, kmax);  // high half zero
         }
     }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-        const double o = __shfl_down_sync(0xffffffffu, s, off);
-        if (lane < off) s = __dadd_rn(s, o);
-    }
-    if (lane == 0) rowsum[row] = s;
+    const uint32_t mx = max(kmax & 0xFFFFu, kmax >> 16);
+    bool bad = __any_sync(0xffffffffu, mx >= 0x7F80u || up != dn);
+    double S = 0.0, CU = 0.0, CD = 0.0;
+    for (int l = 0; l < 32; ++l) two_sum_acc2(S, CU, CD, __shfl_sync(0xffffffffu, up, l));
+    if (lane != 0) return;
+    bad |= CU != CD;
+    HPair p;
+    p.s = bad ? __longlong_as_double(0x7FF8000000000000ll) : __dmul_rn(S, 0x1p896);
+    p.c = bad ? 0.0 : __dmul_rn(CU, 0x1p896);
+    rec[row] = p;
 }
 
 // fp64 -> bf16 bits, round to nearest even, normal range only (0xFFFF if not
@@ -951,26 +1253,52 @@ __device__ uint32_t f64_to_bf16_bits(double v) {
     return sign | (static_cast<uint32_t>(e + 127) << 7) | static_cast<uint32_t>(top & 0x7Full);
 }
 
-// gamma = total / (R*K): the row sums in blocks of 1024 rows (zero-padded),
-// each block combined by halving (a[t] += a[t + stride], stride 512 .. 1), the
-// block sums added in ascending order.  One block of 1024 threads.
-__global__ void __launch_bounds__(1024) k_gamma(const double *__restrict__ rowsum, int64_t R, int64_t K,
-                                                double *__restrict__ gamma_out,
-                                                uint32_t *__restrict__ gb_out) {
-    __shared__ double a[1024];
-    const int t = threadIdx.x;
-    double total = 0.0;
-    for (int64_t b = 0; b < R; b += 1024) {
-        a[t] = b + t < R ? rowsum[b + t] : 0.0;
-        __syncthreads();
-        for (int stride = 512; stride >= 1; stride >>= 1) {
-            if (t < stride) a[t] = __dadd_rn(a[t], a[t + stride]);
-            __syncthreads();
+// gamma from the rows' exact pairs: every thread adds its rows into an
+// integer accumulator, the block adds the accumulators digit by digit, one
+// rounding, one division by R*K.  One block of 1024 threads.
+__global__ void __launch_bounds__(1024) k_gamma(const HPair *__restrict__ rec, const uint16_t *__restrict__ W,
+                                                int64_t R, int64_t K, int64_t ldw,
+                                                double *__restrict__ gamma_out, uint32_t *__restrict__ gb_out) {
+    __shared__ long long part[32][GB_NDIG];
+    AbsAcc a;
+    a.clear();
+    bool nan = false, inf = false;
+    for (int64_t i = threadIdx.x; i < R; i += blockDim.x) {
+        const HPair p = rec[i];
+        if (!isnan(p.s)) {
+            a.add_double(p.s);
+            a.add_double(p.c);
+            continue;
         }
-        if (t == 0) total = __dadd_rn(total, a[0]);
-        __syncthreads();
+        for (int64_t j = 0; j < K; ++j) {  // the integer path for a marked row
+            const uint32_t b = W[i * ldw + j] & 0x7FFFu;
+            const int e = static_cast<int>(b >> 7);
+            if (e == 255) {
+                nan |= (b & 0x7Fu) != 0;
+                inf |= (b & 0x7Fu) == 0;
+            } else if (b) {
+                a.add_bits(e ? 128u + (b & 0x7Fu) : b, (e ? e : 1) - 134 + GB_BIAS, false);
+            }
+        }
     }
-    if (t != 0) return;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int i = 0; i < GB_NDIG; ++i) {
+        long long v = a.d[i];
+        for (int off = 16; off >= 1; off >>= 1) v += __shfl_down_sync(0xffffffffu, v, off);
+        if (lane == 0) part[warp][i] = v;
+    }
+    nan = __syncthreads_or(nan) != 0;
+    inf = __syncthreads_or(inf) != 0;
+    if (threadIdx.x != 0) return;
+    AbsAcc tot;
+    tot.clear();
+    for (int wv = 0; wv < static_cast<int>(blockDim.x / 32); ++wv)
+#pragma unroll
+        for (int i = 0; i < GB_NDIG; ++i) tot.d[i] += part[wv][i];
+    double total = tot.round_rn();
+    if (nan) total = __longlong_as_double(0x7FF8000000000000ll);
+    else if (inf) total = __longlong_as_double(0x7FF0000000000000ll);
     const double gamma = __ddiv_rn(total, __dmul_rn(static_cast<double>(R), static_cast<double>(K)));
     uint32_t gb = f64_to_bf16_bits(gamma);
     if (gamma == 0.0 || gb == 0xFFFFu) {
@@ -1058,60 +1386,65 @@ inline int sm_count() {
 
 namespace {
 
-// the chunk kernel, then (more than one chunk) the ordered finish as its
-// programmatic dependent, so that its launch overlaps the chunk kernel
-nm_status launch_colsumsq(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, double *H, double *part,
-                          cudaStream_t s) {
+// the H reduction: one launch when a block sees every token; otherwise the
+// partial pairs into `part`, then the finish as a programmatic dependent so
+// that its launch overlaps the main kernel.  `max_split` caps the number of
+// token ranges (the pairs `part` can hold are max_split * K).
+nm_status launch_hsq(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, double *H, HPair *part,
+                     int64_t max_split, cudaStream_t s) {
     using namespace nm;
-    const int64_t nchunks = (T + H_CHUNK - 1) / H_CHUNK;
+    const HGrid g = h_grid(T, K, part ? max_split : 1);
+    if (g.cblocks > 0x7FFFFFFF || g.split > 65535) return NM_ERR_SHAPE;
     CUtensorMap tm;
-    if (!make_tmap_bf16(&tm, X, T, K, ldx, H_BLOCK_COLS, H_CHUNK, false)) return NM_ERR_CUDA;
-    if (!set_smem_attr<k_colsumsq_chunk>(H_SMEM_BYTES)) return NM_ERR_CUDA;
-    // two blocks per SM: the column blocks, each with a strided share of the chunks
-    const int64_t cblocks = (K + H_BLOCK_COLS - 1) / H_BLOCK_COLS;
-    int64_t split = 2 * sm_count() / cblocks;
-    split = split < 1 ? 1 : (split > nchunks ? nchunks : split);
-    if (cblocks > 0x7FFFFFFF) return NM_ERR_SHAPE;
-    dim3 grid(static_cast<unsigned>(cblocks), static_cast<unsigned>(split));
-    if (nchunks == 1) {
-        k_colsumsq_chunk<<<grid, H_THREADS, H_SMEM_BYTES, s>>>(tm, T, K, nchunks, H, 1);
+    if (!make_tmap_bf16(&tm, X, T, K, ldx, HX_COLS, HX_CHUNK, false)) return NM_ERR_CUDA;
+    if (!set_smem_attr<k_hsq>(HX_SMEM_BYTES)) return NM_ERR_CUDA;
+    const dim3 grid(static_cast<unsigned>(g.cblocks), static_cast<unsigned>(g.split));
+    if (g.split == 1) {
+        k_hsq<<<grid, HX_THREADS, HX_SMEM_BYTES, s>>>(tm, X, T, K, ldx, nullptr, H);
         return launch_status();
     }
-    k_colsumsq_chunk<<<grid, H_THREADS, H_SMEM_BYTES, s>>>(tm, T, K, nchunks, part, 0);
+    k_hsq<<<grid, HX_THREADS, HX_SMEM_BYTES, s>>>(tm, X, T, K, ldx, part, nullptr);
     if (cudaGetLastError() != cudaSuccess) return NM_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>((K + 63) / 64), 1, 1);
-    cfg.blockDim = dim3(64, 1, 1);
+    cfg.gridDim = dim3(static_cast<unsigned>((K + 127) / 128), 1, 1);
+    cfg.blockDim = dim3(128, 1, 1);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, k_colsumsq_finish, static_cast<const double *>(part), nchunks, T, K, H) !=
+    if (cudaLaunchKernelEx(&cfg, k_hsq_finish, static_cast<const HPair *>(part), g.split, X, T, K, ldx, H) !=
         cudaSuccess)
         return NM_ERR_CUDA;
     return launch_status();
+}
+
+// the checks shared by both H entry points (no launch, no output touched)
+nm_status check_hessian_args(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, const double *H) {
+    if (!X || !H) return NM_ERR_NULL;
+    if (T < 1 || K < 1 || ldx < K) return NM_ERR_SHAPE;
+    if (T > NM_HESSIAN_MAX_TOKENS || K > 0x3FFFFFFFll) return NM_ERR_SHAPE;
+    if (!aligned16(X) || (ldx % 8) != 0 || (reinterpret_cast<uintptr_t>(H) & 7u)) return NM_ERR_ALIGN;
+    return NM_OK;
 }
 
 }  // namespace
 
 extern "C" size_t nm_hessian_workspace_bytes(int64_t T, int64_t K) {
     if (T <= 0 || K <= 0) return 0;
-    const int64_t nchunks = (T + H_CHUNK - 1) / H_CHUNK;
-    return nchunks > 1 ? static_cast<size_t>(nchunks) * static_cast<size_t>(K) * sizeof(double) : 0;
+    const HGrid g = h_grid(T, K, INT64_MAX);
+    return g.split > 1 ? static_cast<size_t>(g.split) * static_cast<size_t>(K) * sizeof(HPair) : 0;
 }
 
 extern "C" nm_status nm_hessian_diag(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
                                      double *H, void *ws, size_t ws_bytes, void *stream) {
-    if (!X || !H) return NM_ERR_NULL;
-    if (T < 1 || K < 1 || ldx < K) return NM_ERR_SHAPE;
-    if (!aligned16(X) || (ldx % 8) != 0) return NM_ERR_ALIGN;
+    const nm_status st = check_hessian_args(X, T, K, ldx, H);
+    if (st != NM_OK) return st;
     const size_t need = nm_hessian_workspace_bytes(T, K);
     if (need > 0 && (!ws || ws_bytes < need)) return NM_ERR_WORKSPACE;
-    const int64_t nchunks = (T + H_CHUNK - 1) / H_CHUNK;
-    if (nchunks > 65535) return NM_ERR_SHAPE;
-    return launch_colsumsq(X, T, K, ldx, H, static_cast<double *>(ws), as_stream(stream));
+    if (need > 0 && (reinterpret_cast<uintptr_t>(ws) & 15u)) return NM_ERR_ALIGN;
+    return launch_hsq(X, T, K, ldx, H, static_cast<HPair *>(ws), INT64_MAX, as_stream(stream));
 }
 
 extern "C" nm_status nm_hessian_rescale(const double *H, const double *s, int64_t K, double *H_out,
@@ -1263,7 +1596,7 @@ extern "C" nm_status lift_activations(const uint16_t *X, int64_t T, int64_t K, i
 }
 
 extern "C" size_t nm_ternary_workspace_bytes(int64_t R) {
-    return R > 0 ? static_cast<size_t>(R) * sizeof(double) + 16 : 0;
+    return R > 0 ? static_cast<size_t>(R) * sizeof(HPair) + 16 : 0;
 }
 
 extern "C" nm_status nm_ternary_quantize(const uint16_t *W, int64_t R, int64_t K, int64_t ldw,
@@ -1274,11 +1607,11 @@ extern "C" nm_status nm_ternary_quantize(const uint16_t *W, int64_t R, int64_t K
     if (!aligned16(W) || !aligned16(ws) || (ldw % 8) != 0) return NM_ERR_ALIGN;
     if (ws_bytes < nm_ternary_workspace_bytes(R)) return NM_ERR_WORKSPACE;
     cudaStream_t s = as_stream(stream);
-    double *rowsum = static_cast<double *>(ws);
-    uint32_t *gb = reinterpret_cast<uint32_t *>(rowsum + R);
+    HPair *rec = static_cast<HPair *>(ws);
+    uint32_t *gb = reinterpret_cast<uint32_t *>(rec + R);
     if ((R + 7) / 8 > 0x7FFFFFFF || R > 65535LL * 65535LL) return NM_ERR_SHAPE;
-    k_row_abs_sum<<<static_cast<unsigned>((R + 7) / 8), 256, 0, s>>>(W, R, K, ldw, rowsum);
-    k_gamma<<<1, 1024, 0, s>>>(rowsum, R, K, gamma, gb);
+    k_row_abs_sum<<<static_cast<unsigned>((R + 7) / 8), 256, 0, s>>>(W, R, K, ldw, rec);
+    k_gamma<<<1, 1024, 0, s>>>(rec, W, R, K, ldw, gamma, gb);
     dim3 grid(static_cast<unsigned>((K + 2047) / 2048), static_cast<unsigned>(R < 65535 ? R : 65535),
               static_cast<unsigned>((R + 65534) / 65535));
     k_ternary_apply<<<grid, 256, 0, s>>>(W, R, K, ldw, gamma, gb, Wq);
@@ -1286,21 +1619,21 @@ extern "C" nm_status nm_ternary_quantize(const uint16_t *W, int64_t R, int64_t K
 }
 
 // ---------------------------------------------------------------------------
-// Allocation-free H reduction: the chunk partials live in this file-scope
+// Allocation-free H reduction: the partial pairs live in this file-scope
 // device array instead of a caller workspace.  Host code must not pass the
 // array's name to a kernel (on the host it is only a stand-in symbol): its
 // device address is looked up once per device with cudaGetSymbolAddress.
 // ---------------------------------------------------------------------------
 namespace {
 
-static __device__ __align__(256) double g_hessian_noalloc_scratch[NM_HESSIAN_NOALLOC_MAX_PARTIALS];
+static __device__ __align__(256) HPair g_hessian_noalloc_scratch[NM_HESSIAN_NOALLOC_MAX_PAIRS];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-double *g_noalloc_ptr[kMaxDevices] = {};
+HPair *g_noalloc_ptr[kMaxDevices] = {};
 
 // device address of the scratch array for the current device (set-up on first use)
-nm_status noalloc_scratch(double **out) {
+nm_status noalloc_scratch(HPair **out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NM_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
@@ -1308,7 +1641,7 @@ nm_status noalloc_scratch(double **out) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_hessian_noalloc_scratch) != cudaSuccess || p == nullptr)
             return NM_ERR_CUDA;
-        g_noalloc_ptr[dev] = static_cast<double *>(p);
+        g_noalloc_ptr[dev] = static_cast<HPair *>(p);
     }
     *out = g_noalloc_ptr[dev];
     return NM_OK;
@@ -1318,17 +1651,15 @@ nm_status noalloc_scratch(double **out) {
 
 extern "C" nm_status nm_hessian_diag_noalloc(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
                                              double *H, void *stream) {
-    if (!X || !H) return NM_ERR_NULL;
-    if (T < 1 || K < 1 || ldx < K) return NM_ERR_SHAPE;
-    if (!aligned16(X) || (ldx % 8) != 0) return NM_ERR_ALIGN;
-    const int64_t nchunks = (T + H_CHUNK - 1) / H_CHUNK;
-    if (nchunks > 65535) return NM_ERR_SHAPE;
-    if (nchunks > 1 && nchunks * K > static_cast<int64_t>(NM_HESSIAN_NOALLOC_MAX_PARTIALS))
-        return NM_ERR_TOO_LARGE;
-    double *part = nullptr;
-    if (nchunks > 1) {
-        const nm_status st = noalloc_scratch(&part);
-        if (st != NM_OK) return st;
+    const nm_status st = check_hessian_args(X, T, K, ldx, H);
+    if (st != NM_OK) return st;
+    // the token ranges are capped so that their pairs fit the array (a block
+    // then takes more tokens); one range needs no scratch at all
+    const int64_t max_split = NM_HESSIAN_NOALLOC_MAX_PAIRS / K;
+    HPair *part = nullptr;
+    if (max_split > 1 && h_grid(T, K, max_split).split > 1) {
+        const nm_status s2 = noalloc_scratch(&part);
+        if (s2 != NM_OK) return s2;
     }
-    return launch_colsumsq(X, T, K, ldx, H, part, as_stream(stream));
+    return launch_hsq(X, T, K, ldx, H, part, part ? max_split : 1, as_stream(stream));
 }

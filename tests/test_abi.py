@@ -41,15 +41,27 @@ def test_status_strings_and_version():
 
 def test_size_queries():
     lib = nm.load()
+    # H: one (s, c) pair of fp64 per column and token range; the ranges of
+    # 128-token chunks fill one wave of 2 * 148 blocks of 128 columns, and a
+    # single range needs no workspace
+    def h_ws(T, K):
+        cb, chunks = (K + 127) // 128, (T + 127) // 128
+        split = max(1, min(296 // cb, chunks))
+        return split * K * 16 if split > 1 else 0
     assert lib.nm_hessian_workspace_bytes(128, 512) == 0
-    assert lib.nm_hessian_workspace_bytes(129, 512) == 2 * 512 * 8
-    assert lib.nm_hessian_workspace_bytes(8192, 4096) == 64 * 4096 * 8
+    assert lib.nm_hessian_workspace_bytes(129, 512) == 2 * 512 * 16
+    assert lib.nm_hessian_workspace_bytes(8192, 4096) == 9 * 4096 * 16
+    for (T, K) in ((300, 4), (2048, 4096), (8192, 11008), (4096, 28672), (1, 100000), (10 ** 6, 56832)):
+        assert lib.nm_hessian_workspace_bytes(T, K) == h_ws(T, K)
+        # every size fits the allocation-free variant's 2 MiB of pairs
+        assert lib.nm_hessian_workspace_bytes(T, K) <= 131072 * 16
+    assert lib.nm_hessian_workspace_bytes(8192, 40000) == 0
     for (R, K, m) in ((256, 512, 4), (4096, 4096, 8), (131, 1003, 6), (28672, 8192, 10), (1, 1, 4)):
         g = packed_geometry(R, K, m)
         assert lib.nm_sparse_prepare_bytes(R, K, m) == g["vals_bytes"] + g["meta_bytes"]
     assert lib.nm_sparse_prepare_bytes(256, 512, 5) == 0
     assert lib.nm_sparse_prepare_bytes(0, 512, 4) == 0
-    assert lib.nm_ternary_workspace_bytes(100) >= 800
+    assert lib.nm_ternary_workspace_bytes(100) == 100 * 16 + 16
     # staged activations (rounded up to 256 bytes), then the stream-K region:
     # per CTA pair 2 x 8 slots of 32 x 240 fp32 and 2 x 8 flags of 8 bytes
     sk = 96 * 2 * 8 * (32 * 240 * 4 + 8)
@@ -99,6 +111,18 @@ MIS = 0x10002
     (lambda l: l.nm_hessian_diag(MIS, 4, 4, 8, A, None, 0, None), 3),
     (lambda l: l.nm_hessian_diag(A, 4, 4, 12, A, None, 0, None), 3),
     (lambda l: l.nm_hessian_diag(A, 300, 4, 8, A, None, 0, None), 5),
+    (lambda l: l.nm_hessian_diag(A, 300, 4, 8, A, A + 8, 1 << 20, None), 3),
+    (lambda l: l.nm_hessian_diag(A, 4, 4, 8, A + 4, None, 0, None), 3),
+    (lambda l: l.nm_hessian_diag(A, 1 << 31, 4, 8, A, A, 1 << 40, None), 2),
+    # the allocation-free variant: the same checks, before any CUDA call
+    (lambda l: l.nm_hessian_diag_noalloc(None, 4, 4, 8, A, None), 1),
+    (lambda l: l.nm_hessian_diag_noalloc(A, 4, 4, 8, None, None), 1),
+    (lambda l: l.nm_hessian_diag_noalloc(A, 0, 4, 8, A, None), 2),
+    (lambda l: l.nm_hessian_diag_noalloc(A, 4, 9, 8, A, None), 2),
+    (lambda l: l.nm_hessian_diag_noalloc(A, 1 << 31, 4, 8, A, None), 2),
+    (lambda l: l.nm_hessian_diag_noalloc(A, (1 << 62) + 5, 16392, 16392, A, None), 2),
+    (lambda l: l.nm_hessian_diag_noalloc(MIS, 4, 4, 8, A, None), 3),
+    (lambda l: l.nm_hessian_diag_noalloc(A, 4, 4, 12, A, None), 3),
     (lambda l: l.nm_prune_compress(A, 8, A, 8, 4, 8, 2, 17, A, A, A, None), 4),
     (lambda l: l.nm_prune_compress(A, 8, A, 8, 4, 8, 4, 4, A, A, A, None), 4),
     (lambda l: l.nm_prune_compress(A, 8, A, 8, 4, 8, 2, 4, A, A, None, None), 1),
@@ -141,6 +165,12 @@ MIS = 0x10002
     (lambda l: l.lift_activations(A, 4, 8, 8, 8, A, 8, None), 2),
     (lambda l: l.nm_sparse_prepare(A, A, 4, 8, 4, A, 1, None), 5),
     (lambda l: l.nm_sparse_prepare(A, A, 4, 8, 4, MIS, 1 << 20, None), 3),
+    (lambda l: l.nm_sparse_prepare(A + 2, A, 4, 8, 4, A, 1 << 20, None), 3),
+    (lambda l: l.nm_sparse_prepare_from_mask(A, None, 4, 8, 4, A, 1 << 20, None), 1),
+    (lambda l: l.nm_sparse_prepare_from_mask(A, A, 4, 8, 5, A, 1 << 20, None), 4),
+    (lambda l: l.nm_sparse_prepare_from_mask(A, A, 4, 8, 8, A, 1, None), 5),
+    (lambda l: l.nm_sparse_prepare_from_mask(A, A + 2, 4, 8, 8, A, 1 << 20, None), 3),
+    (lambda l: l.nm_sparse_prepare_from_mask(A, A, 0, 8, 8, A, 1 << 20, None), 2),
     (lambda l: l.nm_sparse_gemm(A, 4, 8, 8, A, 4, 9, A, 8, None, 0, None), 4),
     (lambda l: l.nm_sparse_gemm(A, 4, 8, 8, A, 4, 4, A, 12, None, 0, None), 3),
     (lambda l: l.nm_sparse_gemm(A, 4, 8, 4, A, 4, 4, A, 8, None, 0, None), 2),

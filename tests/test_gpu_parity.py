@@ -61,11 +61,44 @@ def test_hessian_special_values_bitexact(nm):
     X[:, 42] = 0x0000                            # and one of zeros
     X[7, 50] = 0x7F80                            # +inf and -inf
     X[9, 51] = 0xFF80
+    X[11, 52] = 0x7FC1                           # NaN, and NaN beside an infinity
+    X[12, 53] = 0xFFC0
+    X[13, 53] = 0x7F80
     H = nm.hessian_diag(to_dev(X))
     _sync_ok(nm)
     h, ref = to_host(H), oracle.hessian_diag(X)
     assert np.isinf(ref[50]) and np.isinf(ref[51]) and ref[42] == 0.0 and 0.0 < ref[40] < 1e-70
-    assert np.array_equal(h, ref)
+    assert np.isnan(ref[52]) and np.isnan(ref[53])
+    assert np.array_equal(h, ref, equal_nan=True)
+
+
+@pytest.mark.parametrize("T", [300, 5000])
+def test_hessian_exact_rounding_paths(nm, T):
+    # columns that need each path of the exact sum, against the oracle:
+    #  0: the tie 2^52 + 2^52 + 1 (rounds to even) and 1: the same broken up by
+    #     the square of the smallest subnormal (the integer path);
+    #  2: a 16-token run holding 2^20 and 2^-12 among ordinary values (its
+    #     check fails; summed again in two parts, each exact);
+    #  3: 2^60 and 2^-60 in two runs of one block (each run exact, the block's
+    #     chain too wide: the integer path); 4: the same in different blocks
+    #     (the finish adds the blocks' exact pairs);
+    #  5: a run of 2^-64 values among ordinary ones; the rest Gaussian
+    K = 40
+    X = datagen.make_activations(T, K, seed=T, n_outliers=4)
+    X[:, :6] = 0
+    X[0, 0], X[1, 0], X[2, 0] = 0x4C80, 0x4C80, 0x3F80
+    X[0, 1], X[1, 1], X[2, 1], X[T - 1, 1] = 0x4C80, 0x4C80, 0x3F80, 0x0001
+    X[:, 2] = datagen.make_activations(T, 1, seed=1)[:, 0]
+    X[17, 2], X[20, 2] = 0x3980, 0x4980                    # 2^-12, 2^20
+    X[5, 3], X[40, 3] = 0x5D80, 0x2180                     # 2^60, 2^-60
+    X[5, 4], X[T - 3, 4] = 0x5D80, 0x2180
+    X[:, 5] = datagen.make_activations(T, 1, seed=2)[:, 0]
+    X[32:48, 5] = 0x1F80                                   # 2^-64
+    H = nm.hessian_diag(to_dev(X, 40))
+    _sync_ok(nm)
+    ref = oracle.hessian_diag(X)
+    assert ref[0] == 2.0 ** 53 / T and ref[1] == (2.0 ** 53 + 2) / T
+    assert np.array_equal(to_host(H), ref)
 
 
 @pytest.mark.parametrize("R,K,ld", [(256, 512, 512), (33, 1030, 1032), (5, 13, 16), (64, 4096, 4096)])
@@ -319,12 +352,16 @@ def test_lift_bitexact(nm, m, T, K):
 
 # ---------------------------------------------------------------- a6
 @pytest.mark.parametrize("m,R,K", [(4, 256, 512), (8, 130, 1030), (6, 64, 1003), (10, 200, 2050),
-                                   (4, 1, 9)])
+                                   (4, 1, 9), (8, 300, 8195), (6, 257, 4100), (10, 129, 4096), (4, 390, 1034)])
 def test_prepare_layout_bitexact(nm, m, R, K):
+    # from the window metadata, and from the mask (the window pack fused in):
+    # both decode to the oracle's values and window index pairs, byte for byte
     W = datagen.make_weight(R, K, 0.02, seed=R * m)
     res = oracle.run_layer(None, W, m - 2, m, score="magnitude")
     wm = res["meta24"] if m == 4 else res["wmeta"]
     packed = nm.sparse_prepare(to_dev(res["vals"]), torch.from_numpy(wm).cuda(), R, K, m)
+    packed_m = nm.sparse_prepare_from_mask(to_dev(res["vals"]), torch.from_numpy(res["mask"].view(np.int32)).cuda(),
+                                           R, K, m)
     _sync_ok(nm)
     g = packed_geometry(R, K, m)
     assert packed.numel() == g["vals_bytes"] + g["meta_bytes"]
@@ -332,6 +369,22 @@ def test_prepare_layout_bitexact(nm, m, R, K):
     assert pad_ok
     assert np.array_equal(vals, res["vals"])
     assert np.array_equal(nib, wmeta_nibbles(wm, g["nwin"]))
+    assert np.array_equal(to_host(packed_m), to_host(packed))
+
+
+def test_prepare_from_mask_flags_bad_mask(nm):
+    # a 5:8 mask is not (m-2):m: NM_ERR_DEVICE in the error word, nothing hangs
+    S = np.zeros((3, 16), dtype=np.float32)
+    S[:, :5] = 1
+    S[:, 8:14] = 1
+    W = datagen.f32_to_bf16_bits(np.ones((3, 16), np.float32))
+    om, ov, _ = oracle.prune(S, W, 5, 8)
+    vals = to_dev(np.zeros((3, 12), dtype=np.uint16))
+    nm.sparse_prepare_from_mask(vals, torch.from_numpy(om.view(np.int32)).cuda(), 3, 16, 8)
+    torch.cuda.synchronize()
+    with pytest.raises(nm.NMError, match="NM_ERR_DEVICE"):
+        nm.check_device_error()
+    nm.check_device_error()
 
 
 # ---------------------------------------------------------------- a7 / a8
@@ -407,7 +460,9 @@ def test_fused_lift_equals_two_pass(nm, m):
     # lift_activations + a 2:4 GEMM of width K' versus the fused kernel.  For
     # 4:6 and 8:10 both use the natural K' order and the same tiles, so the fp32
     # tensor-core sums are identical bits; 6:8 packs K' in another order (raw
-    # tiles of X first), so it agrees within rounding.
+    # tiles of X first), and the library kernel visits its blocks in yet
+    # another (every raw block before every middle-window block), so those
+    # agree within rounding.
     # (whole-tile schedule throughout: the fused kernel has no stream-K form,
     # and splitting K' would change the fp32 summation order)
     R, K, T = 256, 1030, 130
@@ -430,7 +485,7 @@ def test_fused_lift_equals_two_pass(nm, m):
     assert rel_err(Yl, Y64) <= GEMM_TOL
     if m == 8:
         assert rel_err(Yf, Y2) <= 2 ** -7
-        assert np.array_equal(Yl, Yf)   # same K' order and tiles, lift done before or inside
+        assert rel_err(Yl, Yf) <= 2 ** -7
     else:
         assert np.array_equal(Y2, Yf)
         assert np.array_equal(Yl, Yf)
@@ -472,6 +527,30 @@ def test_dense_gemm_vs_oracle_and_torch(nm, R, K, T):
 
 
 # ---------------------------------------------------------------- ternary
+def test_ternary_gamma_exact_rounding_and_specials(nm):
+    # gamma is the correctly rounded sum / (R K): a tie to even, the tie
+    # broken by a subnormal (integer path), a row of subnormals only; an
+    # infinity or a NaN in W is reported, not returned
+    rows = np.zeros((4, 8), dtype=np.uint16)
+    rows[0, :2] = (0x5A00, 0x3F80)                 # 2^53 + 1: a tie, to even
+    rows[1, 0] = 0x0001                            # breaks it upwards
+    rows[2, :] = (0x0001, 0x0003, 0x807F, 0x0040, 0, 0x8001, 0x0002, 0)
+    W = datagen.make_weight(40, 8, 0.02, seed=3)
+    W[:4] = rows
+    Wq, gamma = nm.ternary_quantize(to_dev(W))
+    _sync_ok(nm)
+    g, oWq = oracle.ternary(W)
+    assert to_host(gamma)[0] == g
+    assert np.array_equal(to_host_u16(Wq), oWq)
+    for bad in (0x7F80, 0xFFC1):
+        Wb = W.copy()
+        Wb[7, 5] = bad
+        nm.ternary_quantize(to_dev(Wb))
+        torch.cuda.synchronize()
+        with pytest.raises(nm.NMError, match="NM_ERR_DEVICE"):
+            nm.check_device_error()
+
+
 @pytest.mark.parametrize("R,K", [(64, 256), (11008 // 8, 4096 // 4), (3, 13)])
 def test_ternary_bitexact(nm, R, K):
     W = datagen.make_weight(R, K, 0.02, seed=R)
@@ -486,16 +565,19 @@ def test_ternary_bitexact(nm, R, K):
 # ---------------------------------------------------------------- whole path
 def _device_pipeline(nm, X, W, n, m, eps=1e-8, score="hessian", ternary=False):
     # the calls the bench's step makes: H, the fused score + prune, the window
-    # pack, the operand preparation and the sparse GEMM
+    # pack fused into the operand preparation, and the sparse GEMM
     Xd, Wd = to_dev(X), to_dev(W)
     V = Wd
     if ternary:
         V, _ = nm.ternary_quantize(Wd)
     H = nm.hessian_diag(Xd) if score == "hessian" else None
     mask, vals, meta = nm.score_prune_compress(H, Wd, n, m, V=V, eps=eps)
-    wm = meta if m == 4 else nm.slide_pack(mask, W.shape[1], m)
-    packed = nm.sparse_prepare(vals, wm, W.shape[0], W.shape[1], m)
+    if m == 4:
+        packed = nm.sparse_prepare(vals, meta, W.shape[0], W.shape[1], m)
+    else:
+        packed = nm.sparse_prepare_from_mask(vals, mask, W.shape[0], W.shape[1], m)
     Y = nm.sparse_gemm(Xd, packed, W.shape[0], m)
+    wm = meta if m == 4 else nm.slide_pack(mask, W.shape[1], m)   # the standalone pack, checked too
     _sync_ok(nm)
     return dict(H=H, mask=mask, vals=vals, wm=wm, Y=Y, V=V)
 

@@ -144,3 +144,35 @@ def test_small_workspace_falls_back_to_whole_tiles(nm, schedule):
     Y = nm.sparse_gemm(to_dev(X), packed, R, m, ws=ws)
     _sync_ok(nm)
     assert rel_err(_y(Y), oracle.gemm_masked(X, res["mask"], W, m)) <= GEMM_TOL
+
+
+def test_owner_gives_up_on_a_withheld_flag_and_the_next_launch_is_correct(nm, schedule):
+    # Failure detection without a GPU fault: one tile of 2:4 (R = 256, K' = 32
+    # blocks) cut into four stream-K ranges, so pairs 1..3 hand partial sums to
+    # pair 0.  Pair 2 withholds its flag and the wait limit is 10 ms: pair 0's
+    # bounded poll gives up, records NM_ERR_TIMEOUT and the kernel finishes
+    # (it releases tensor memory and exits as on a normal run; only global
+    # memory polling is involved, no copy is in flight).  The error word
+    # reports it once; a following launch with the controls back is correct.
+    lib = nm.load()
+    R, K, T, m = 256, 4096, 64, 4
+    X, W, res = _layer(R, K, T, m, seed=77)
+    packed = _packed(nm, res, R, K, m)
+    Xd = to_dev(X)
+    Y64 = oracle.gemm_masked(X, res["mask"], W, m)
+    schedule(2, 4)
+    try:
+        assert lib.nm_test_set_wait_limit_ns(10_000_000) == 0
+        assert lib.nm_test_withhold_stream_k_flag(2) == 0
+        nm.sparse_gemm(Xd, packed, R, m)
+        torch.cuda.synchronize()
+        with pytest.raises(nm.NMError, match="NM_ERR_TIMEOUT"):
+            nm.check_device_error()
+    finally:
+        assert lib.nm_test_withhold_stream_k_flag(-1) == 0
+        assert lib.nm_test_set_wait_limit_ns(0) == 0
+    nm.check_device_error()                    # reported once, then cleared
+    Y = nm.sparse_gemm(Xd, packed, R, m)       # same schedule, flags published
+    _sync_ok(nm)
+    assert rel_err(_y(Y), Y64) <= GEMM_TOL
+    assert lib.nm_test_set_wait_limit_ns(2_000_000_000) == 2   # above one second: refused
