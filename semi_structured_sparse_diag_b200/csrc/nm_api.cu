@@ -8,6 +8,7 @@ namespace nm {
 __device__ uint32_t g_error_word = 0;
 __device__ uint64_t g_wait_limit_ns = WAIT_LIMIT_NS;
 __device__ int g_test_withhold_flag_cluster = -1;
+__device__ const WinTable g_wintab = WinTable();
 }  // namespace nm
 
 extern "C" nm_status nm_test_set_wait_limit_ns(unsigned long long ns) {

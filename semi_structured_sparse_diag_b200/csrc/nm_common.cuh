@@ -466,4 +466,43 @@ __device__ __forceinline__ void cp_async_wait_pending() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+
+// Window index pairs of a (2N-2):2N group from its mask bits (SlideSparse
+// sec. 2A): with the two pruned positions z0 < z1, survivor k sits at
+// k + [k >= z0] + [k >= z1 - 1], and window w (positions 2w .. 2w + 3) takes
+// survivors 2w and 2w + 1: its nibble is (q0 - 2w) | (q1 - 2w) << 2.  The
+// table below holds, for every m-bit value, the nibbles of its windows packed
+// in the order the operand's metadata bytes want them (window w at bits
+// 4w .. 4w+3), or 0xFFFF for a group that does not hold exactly m - 2
+// survivors; it is built at compile time for m = 6, 8, 10 and indexed
+// [offset(m) + bits].
+constexpr int wt_offset(int m) { return m == 6 ? 0 : (m == 8 ? 64 : 64 + 256); }
+constexpr uint16_t wt_entry(int m, uint32_t bits) {
+    uint32_t z = ~bits & ((1u << m) - 1u);
+    int cnt = 0, z0 = -1, z1 = -1;
+    for (int p = 0; p < m; ++p)
+        if ((z >> p) & 1u) {
+            ++cnt;
+            if (z0 < 0) z0 = p; else z1 = p;
+        }
+    if (cnt != 2) return 0xFFFFu;
+    uint32_t out = 0;
+    for (int w = 0; w < m / 2 - 1; ++w) {
+        const int k0 = 2 * w, k1 = 2 * w + 1;
+        const int q0 = k0 + (k0 >= z0) + (k0 >= z1 - 1), q1 = k1 + (k1 >= z0) + (k1 >= z1 - 1);
+        out |= static_cast<uint32_t>((q0 - 2 * w) | ((q1 - 2 * w) << 2)) << (4 * w);
+    }
+    return static_cast<uint16_t>(out);
+}
+struct WinTable {
+    uint16_t v[64 + 256 + 1024];
+    constexpr WinTable() : v() {
+        for (uint32_t b = 0; b < 64; ++b) v[wt_offset(6) + b] = wt_entry(6, b);
+        for (uint32_t b = 0; b < 256; ++b) v[wt_offset(8) + b] = wt_entry(8, b);
+        for (uint32_t b = 0; b < 1024; ++b) v[wt_offset(10) + b] = wt_entry(10, b);
+    }
+};
+// defined once, in nm_api.cu
+extern __device__ const WinTable g_wintab;
+
 }  // namespace nm

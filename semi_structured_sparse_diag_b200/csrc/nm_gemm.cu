@@ -105,101 +105,87 @@ __host__ __device__ inline void meta_byte_coords(int b, int &row, int &col) {
 
 // values, natural K' order (m = 4, 6, 10): the packed row is the row of vals
 // (a window's pair of values = one 4-byte word, window wi at word wi) padded
-// with zeros.  One thread per 16-byte output chunk; 16-byte loads when every
-// row of vals starts on 16 bytes (vec), else four 4-byte loads.
-// grid x = chunks of a row, y (+65535 z) = row.
+// with zeros.  A thread moves the same 16-byte chunk of PV_ROWS consecutive
+// rows, every load issued before the first store (64 bytes in flight per
+// thread); 16-byte loads when every row of vals starts on 16 bytes (vec),
+// else four 4-byte loads.  grid x = chunks of a row, y (+65535 z) = blocks
+// of PV_ROWS rows.
+constexpr int PV_ROWS = 4;
 __global__ void __launch_bounds__(256)
     k_prepare_vals(const uint16_t *__restrict__ vals, int64_t R, int64_t words, int64_t Rpad, int64_t KLh,
                    bool vec, uint16_t *__restrict__ out) {
-    const int64_t r = blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535;
+    const int64_t r0 = (blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535) * PV_ROWS;
     const int64_t c8 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // chunk
-    if (r >= Rpad || c8 * 8 >= KLh) return;
-    const uint32_t *vrow = reinterpret_cast<const uint32_t *>(vals) + r * words;
+    if (r0 >= Rpad || c8 * 8 >= KLh) return;
     const int64_t w0 = 4 * c8;
-    uint4 o = make_uint4(0u, 0u, 0u, 0u);
-    if (r < R) {
-        if (vec && w0 + 4 <= words) {
-            o = __ldg(reinterpret_cast<const uint4 *>(vrow + w0));
-        } else {
-            o.x = w0 < words ? __ldg(vrow + w0) : 0u;
-            o.y = w0 + 1 < words ? __ldg(vrow + w0 + 1) : 0u;
-            o.z = w0 + 2 < words ? __ldg(vrow + w0 + 2) : 0u;
-            o.w = w0 + 3 < words ? __ldg(vrow + w0 + 3) : 0u;
+    uint4 o[PV_ROWS];
+#pragma unroll
+    for (int i = 0; i < PV_ROWS; ++i) {
+        const int64_t r = r0 + i;
+        const uint32_t *vrow = reinterpret_cast<const uint32_t *>(vals) + r * words;
+        o[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (r < R) {
+            if (vec && w0 + 4 <= words) {
+                o[i] = __ldg(reinterpret_cast<const uint4 *>(vrow + w0));
+            } else {
+                o[i].x = w0 < words ? __ldg(vrow + w0) : 0u;
+                o[i].y = w0 + 1 < words ? __ldg(vrow + w0 + 1) : 0u;
+                o[i].z = w0 + 2 < words ? __ldg(vrow + w0 + 2) : 0u;
+                o[i].w = w0 + 3 < words ? __ldg(vrow + w0 + 3) : 0u;
+            }
         }
     }
-    *reinterpret_cast<uint4 *>(out + r * KLh + c8 * 8) = o;
+#pragma unroll
+    for (int i = 0; i < PV_ROWS; ++i)
+        if (r0 + i < Rpad) *reinterpret_cast<uint4 *>(out + (r0 + i) * KLh + c8 * 8) = o[i];
 }
 
-// values, 6:8: one warp per (row, 32 groups) = 96 words of vals (3 words per
-// group: windows 0, 1, 2); lane l loads words l, l + 32, l + 64 and the warp
-// writes the three K' blocks of those groups -- windows 0 and 2 of groups
-// 0-15 and of 16-31, then window 1 of all 32 -- one word per lane each, by
-// shuffles.  grid: 8 warps per block over (row, block of 32 groups).
+// values, 6:8: a warp per row, PV68_JW blocks of 32 groups per warp.  A
+// block's 96 words of vals (3 per group: windows 0, 1, 2) sit in the lanes'
+// registers (word 32 c + lane in register c, all loads issued first); the 96
+// output words of the block's three K' blocks -- windows 0 and 2 of groups
+// 0-15, of groups 16-31, then window 1 of all 32 -- are gathered with
+// shuffles: output word 32 c + lane takes source word s0 = 3 (lane / 2) +
+// 2 (lane % 2), s0 + 48 or 3 lane + 1.  grid: x = PV68_JW blocks of 32 groups,
+// y (+65535 z) = 8 rows.
+constexpr int PV68_JW = 4;
 __global__ void __launch_bounds__(256)
     k_prepare_vals68(const uint16_t *__restrict__ vals, int64_t R, int64_t G, int64_t Rpad, int64_t nj,
                      int64_t KLh, uint16_t *__restrict__ out) {
     const int lane = threadIdx.x & 31;
-    const int64_t wid = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    if (wid >= Rpad * nj) return;  // warp-uniform
-    const int64_t r = wid / nj, j = wid - r * nj;
+    const int64_t r = (blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535) * 8 + (threadIdx.x >> 5);
+    if (r >= Rpad) return;  // warp-uniform
+    const int64_t jb = static_cast<int64_t>(blockIdx.x) * PV68_JW;
     const int64_t words = 3 * G;
-    const uint32_t *src = reinterpret_cast<const uint32_t *>(vals) + r * words + 96 * j;
-    uint32_t v[3];
+    const uint32_t *srow = reinterpret_cast<const uint32_t *>(vals) + (r < R ? r : 0) * words;
+    uint32_t *drow = reinterpret_cast<uint32_t *>(out + r * KLh);
+    const int64_t avail = r < R ? words - 96 * jb : 0;  // real words of the row from block jb on
+    uint32_t v[PV68_JW][3];
 #pragma unroll
-    for (int q = 0; q < 3; ++q) {
-        const int64_t wi = 96 * j + 32 * q + lane;
-        v[q] = (r < R && wi < words) ? __ldg(src + 32 * q + lane) : 0u;
+    for (int k = 0; k < PV68_JW; ++k)
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+            const int w = 96 * k + 32 * c + lane;
+            v[k][c] = w < avail ? __ldg(srow + 96 * jb + w) : 0u;
+        }
+    const int s0 = 3 * (lane >> 1) + 2 * (lane & 1), s1 = s0 + 48, s2 = 3 * lane + 1;
+#pragma unroll
+    for (int k = 0; k < PV68_JW; ++k) {
+        if (jb + k >= nj) break;  // warp-uniform
+        const uint32_t a0 = __shfl_sync(0xffffffffu, v[k][0], s0 & 31);
+        const uint32_t a1 = __shfl_sync(0xffffffffu, v[k][1], s0 & 31);
+        const uint32_t b1 = __shfl_sync(0xffffffffu, v[k][1], s1 & 31);
+        const uint32_t b2 = __shfl_sync(0xffffffffu, v[k][2], s1 & 31);
+        const uint32_t c0 = __shfl_sync(0xffffffffu, v[k][0], s2 & 31);
+        const uint32_t c1 = __shfl_sync(0xffffffffu, v[k][1], s2 & 31);
+        const uint32_t c2 = __shfl_sync(0xffffffffu, v[k][2], s2 & 31);
+        uint32_t *d = drow + 96 * (jb + k);
+        d[lane] = s0 < 32 ? a0 : a1;
+        d[32 + lane] = s1 < 64 ? b1 : b2;
+        d[64 + lane] = s2 < 32 ? c0 : (s2 < 64 ? c1 : c2);
     }
-    // word i of the 96 lives in lane i % 32, register i / 32
-    auto fetch = [&](int i) {
-        const uint32_t a = __shfl_sync(0xffffffffu, v[0], i & 31);
-        const uint32_t b = __shfl_sync(0xffffffffu, v[1], i & 31);
-        const uint32_t c = __shfl_sync(0xffffffffu, v[2], i & 31);
-        return i < 32 ? a : (i < 64 ? b : c);
-    };
-    // a K' block holds 32 slots = 32 words; blocks 3j, 3j + 1, 3j + 2 of the row
-    uint32_t *dst = reinterpret_cast<uint32_t *>(out + r * KLh) + 96 * j;
-    dst[lane] = fetch(3 * (lane >> 1) + 2 * (lane & 1));              // groups 0-15, windows 0 / 2
-    dst[32 + lane] = fetch(3 * (16 + (lane >> 1)) + 2 * (lane & 1));  // groups 16-31
-    dst[64 + lane] = fetch(3 * lane + 1);                             // window 1 of groups 0-31
 }
 
-// Window index pairs of a (2N-2):2N group from its mask bits (SlideSparse
-// sec. 2A): with the two pruned positions z0 < z1, survivor k sits at
-// k + [k >= z0] + [k >= z1 - 1], and window w (positions 2w .. 2w + 3) takes
-// survivors 2w and 2w + 1: its nibble is (q0 - 2w) | (q1 - 2w) << 2.  The
-// table below holds, for every m-bit value, the nibbles of its windows packed
-// in the order the operand's metadata bytes want them (window w at bits
-// 4w .. 4w+3), or 0xFFFF for a group that does not hold exactly m - 2
-// survivors; it is built at compile time for m = 6, 8, 10 and indexed
-// [offset(m) + bits].
-constexpr int wt_offset(int m) { return m == 6 ? 0 : (m == 8 ? 64 : 64 + 256); }
-constexpr uint16_t wt_entry(int m, uint32_t bits) {
-    uint32_t z = ~bits & ((1u << m) - 1u);
-    int cnt = 0, z0 = -1, z1 = -1;
-    for (int p = 0; p < m; ++p)
-        if ((z >> p) & 1u) {
-            ++cnt;
-            if (z0 < 0) z0 = p; else z1 = p;
-        }
-    if (cnt != 2) return 0xFFFFu;
-    uint32_t out = 0;
-    for (int w = 0; w < m / 2 - 1; ++w) {
-        const int k0 = 2 * w, k1 = 2 * w + 1;
-        const int q0 = k0 + (k0 >= z0) + (k0 >= z1 - 1), q1 = k1 + (k1 >= z0) + (k1 >= z1 - 1);
-        out |= static_cast<uint32_t>((q0 - 2 * w) | ((q1 - 2 * w) << 2)) << (4 * w);
-    }
-    return static_cast<uint16_t>(out);
-}
-struct WinTable {
-    uint16_t v[64 + 256 + 1024];
-    constexpr WinTable() : v() {
-        for (uint32_t b = 0; b < 64; ++b) v[wt_offset(6) + b] = wt_entry(6, b);
-        for (uint32_t b = 0; b < 256; ++b) v[wt_offset(8) + b] = wt_entry(8, b);
-        for (uint32_t b = 0; b < 1024; ++b) v[wt_offset(10) + b] = wt_entry(10, b);
-    }
-};
-__device__ const WinTable g_wintab = WinTable();
 
 // groups of K' block kb: [g_lo, g_hi)
 __device__ __forceinline__ void block_groups(int m, int64_t kb, int64_t &g_lo, int64_t &g_hi) {
@@ -227,118 +213,265 @@ __device__ __forceinline__ void block_groups(int m, int64_t kb, int64_t &g_lo, i
 // with L = m0 + 8 k1 + 16 m2, word k2 of the lane is half-word k1 + 2 k2 of
 // row m0 + 16 m2 (low half) and of row m0 + 16 m2 + 8 (high half).
 constexpr int PM_IN_WORDS = 13;   // >= input words of a row for any pattern (+1 pitch)
+// 2:4 from the mask: for every 4-bit group value, its nibble s0 | s1 << 2
+// (the two set bits, ascending) and whether it has exactly two bits set
+constexpr uint64_t nib24_table() {
+    uint64_t t = 0;
+    for (int b = 0; b < 16; ++b) {
+        int s[2] = {0, 0}, c = 0;
+        for (int p = 0; p < 4; ++p)
+            if ((b >> p) & 1) {
+                if (c < 2) s[c] = p;
+                ++c;
+            }
+        if (c == 2) t |= static_cast<uint64_t>(s[0] | (s[1] << 2)) << (4 * b);
+    }
+    return t;
+}
+constexpr uint32_t valid24_table() {
+    uint32_t v = 0;
+    for (int b = 0; b < 16; ++b) {
+        int c = 0;
+        for (int p = 0; p < 4; ++p) c += (b >> p) & 1;
+        if (c == 2) v |= 1u << b;
+    }
+    return v;
+}
+constexpr uint64_t kNib24 = nib24_table();
+constexpr uint32_t kValid24 = valid24_table();
+static_assert(kValid24 == 0x1668u, "2:4 group values with two bits set: 3, 5, 6, 9, 10, 12");
+
+// Stages the spans [0, n) of rows row0 .. row0 + 127 (row stride `stride`
+// elements of src) into dst[row][0 .. n): element i = t + 128 k of the
+// flattened spans is row i / n, position i % n (stepped without a division).
+// NE >= n loads per thread, in batches of B, every load of a batch issued
+// before its first store (B = NE: all of them).
+template <int NE, int B, typename E, typename D>
+__device__ __forceinline__ void stage_rows(const E *__restrict__ src, int64_t stride, int n, int64_t row0,
+                                           int64_t R, int t, D (*dst)[sizeof(D) == 1 ? PM_IN_WORDS * 4 : PM_IN_WORDS]) {
+    static_assert(NE % B == 0, "batches");
+    const int dr = BM / n, dq = BM - dr * n;
+    int r = t / n, q = t - r * n;
+#pragma unroll 1
+    for (int k0 = 0; k0 < NE; k0 += B) {
+        if (r >= BM) break;  // this thread's elements are done
+        E v[B];
+        int rr = r, qq = q;
+#pragma unroll
+        for (int k = 0; k < B; ++k) {
+            v[k] = (rr < BM && row0 + rr < R) ? __ldg(src + (row0 + rr) * stride + qq) : E(0);
+            rr += dr;
+            qq += dq;
+            if (qq >= n) {
+                qq -= n;
+                ++rr;
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < B; ++k) {
+            if (r < BM) dst[r][q] = static_cast<D>(v[k]);
+            r += dr;
+            q += dq;
+            if (q >= n) {
+                q -= n;
+                ++r;
+            }
+        }
+    }
+}
+
+// The input span of K' block kb of a row: mask words or window-metadata
+// bytes [u0, u0 + nu) for the real groups [g_lo, g_end).
+template <int M, bool FROM_MASK>
+struct MetaSpan {
+    int64_t g_lo, g_end, u0;
+    int nu;
+    __device__ __forceinline__ MetaSpan(int64_t kb, int64_t G) {
+        constexpr int NWIN = M / 2 - 1;
+        int64_t g_hi;
+        block_groups(M, kb, g_lo, g_hi);
+        g_end = g_hi < G ? g_hi : G;
+        u0 = 0;
+        int64_t u1 = 0;
+        if (g_end > g_lo) {
+            if (FROM_MASK) {
+                u0 = (g_lo * M) >> 5;
+                u1 = (g_end * M + 31) >> 5;
+            } else {
+                u0 = (g_lo * NWIN) >> 1;
+                u1 = (g_end * NWIN + 1) >> 1;
+            }
+        }
+        nu = static_cast<int>(u1 - u0);  // <= 8 words / <= 48 bytes
+    }
+};
+
+// Issues the staging of one K' block's spans for rows row0 .. row0 + 127 into
+// dst (row r, word q at dst[r][q]) as asynchronous 4-byte copies, flattened
+// row after row as in stage_rows (rows at or past R get zeros); window bytes
+// that are not word-aligned are staged with plain loads instead.
+template <int M, bool FROM_MASK>
+__device__ __forceinline__ void meta_stage(const MetaSpan<M, FROM_MASK> &sp, const uint8_t *__restrict__ wmeta,
+                                           const uint32_t *__restrict__ mask, int64_t R, int64_t wbytes,
+                                           int64_t mwords, int64_t row0, int t,
+                                           uint32_t (*dst)[PM_IN_WORDS]) {
+    if (sp.nu <= 0) return;
+    const bool words4 = FROM_MASK || ((wbytes & 3) == 0 && (sp.u0 & 3) == 0 && (sp.nu & 3) == 0 &&
+                                      (reinterpret_cast<uintptr_t>(wmeta) & 3u) == 0);
+    if (!words4) {
+        stage_rows<48, 8>(wmeta + sp.u0, wbytes, sp.nu, row0, R, t,
+                          reinterpret_cast<uint8_t (*)[PM_IN_WORDS * 4]>(dst));
+        return;
+    }
+    const int n = FROM_MASK ? sp.nu : sp.nu >> 2;  // words per row
+    const uint32_t *src = FROM_MASK ? mask + sp.u0 : reinterpret_cast<const uint32_t *>(wmeta + sp.u0);
+    const int64_t stride = FROM_MASK ? mwords : wbytes >> 2;
+    const int dr = BM / n, dq = BM - dr * n;
+    int r = t / n, q = t - r * n;
+#pragma unroll
+    for (int k = 0; k < (FROM_MASK ? 8 : 12); ++k) {
+        if (r < BM) {
+            const bool real = row0 + r < R;
+            cp_async4(&dst[r][q], src + (real ? row0 + r : 0) * stride + q, real ? 4u : 0u);
+        }
+        r += dr;
+        q += dq;
+        if (q >= n) {
+            q -= n;
+            ++r;
+        }
+    }
+}
+
+// metadata: one block of 128 threads per (128-row tile mt, PM_KPB consecutive
+// K' blocks).  For each K' block kb: (1) the block's input -- the mask words
+// or window-metadata bytes of its groups, for 128 rows -- is staged in shared
+// memory by coalesced asynchronous copies, double-buffered: block kb + 1's
+// copies are in flight while kb is formed and stored.  (2) Thread r forms the
+// 16 bytes of row mt * 128 + r (slot 2p in the low nibble of byte p): from the
+// window metadata (for the natural orders a masked copy), or, with FROM_MASK,
+// by looking each group's mask bits up in the window table (the sliding-window
+// pack fused in).  Padding rows and slots get the pair (0, 1).  (3) Thread L
+// writes lane L's 16 bytes in the tensor-memory order of meta_byte_coords:
+// with L = m0 + 8 k1 + 16 m2, word k2 of the lane is half-word k1 + 2 k2 of
+// row m0 + 16 m2 (low half) and of row m0 + 16 m2 + 8 (high half).
+constexpr int PM_KPB = 4;
 template <int M, bool FROM_MASK>
 __global__ void __launch_bounds__(128)
     k_prepare_meta(const uint8_t *__restrict__ wmeta, const uint32_t *__restrict__ mask, int64_t R, int64_t G,
                    int64_t wbytes, int64_t mwords, int64_t nkb, uint8_t *__restrict__ out) {
     constexpr int NWIN = M / 2 - 1;
-    __shared__ uint32_t in[BM][PM_IN_WORDS];
+    __shared__ uint32_t in[2][BM][PM_IN_WORDS];
     __shared__ uint32_t rowb[BM][5];  // 16 bytes per row (+1 word pitch)
     __shared__ uint16_t tab[M == 4 ? 1 : (1 << M)];
-    const int64_t blk = blockIdx.x;
-    const int64_t mt = blk / nkb, kb = blk - mt * nkb;
+    const int64_t nkc = (nkb + PM_KPB - 1) / PM_KPB;
+    const int64_t mt = blockIdx.x / nkc, kc = blockIdx.x - mt * nkc;
+    const int64_t kb0 = kc * PM_KPB, kb1 = kb0 + PM_KPB < nkb ? kb0 + PM_KPB : nkb;
     const int t = threadIdx.x;
+    const int64_t row0 = mt * BM, row = row0 + t;
     if (FROM_MASK && M != 4)
         for (int i = t; i < (1 << M); i += BM) tab[i] = g_wintab.v[wt_offset(M) + i];
-    int64_t g_lo, g_hi;
-    block_groups(M, kb, g_lo, g_hi);
-    const int64_t g_end = g_hi < G ? g_hi : G;  // real groups [g_lo, g_end)
-    // the input span of a row: mask words or wmeta bytes [u0, u1)
-    int64_t u0 = 0, u1 = 0;
-    if (g_end > g_lo) {
-        if (FROM_MASK) {
-            u0 = (g_lo * M) >> 5;
-            u1 = (g_end * M + 31) >> 5;
-        } else {
-            u0 = (g_lo * NWIN) >> 1;
-            u1 = (g_end * NWIN + 1) >> 1;
-        }
-    }
-    const int nu = static_cast<int>(u1 - u0);   // <= 9 words / <= 48 bytes
-    for (int idx = t; idx < BM * nu; idx += BM) {
-        const int rr = idx / nu, q = idx - rr * nu;
-        const int64_t row = mt * BM + rr;
-        if (FROM_MASK)
-            in[rr][q] = row < R ? __ldg(mask + row * mwords + u0 + q) : 0u;
-        else
-            reinterpret_cast<uint8_t *>(in[rr])[q] = row < R ? __ldg(wmeta + row * wbytes + u0 + q) : 0u;
-    }
-    __syncthreads();
-    const int64_t row = mt * BM + t;
-    const int ng = static_cast<int>(g_end - g_lo);
-    const bool mid = M == 8 && (kb % 3) == 2;
-    constexpr int GPB = M == 4 ? 32 : (M == 8 ? 32 : 32 / NWIN);  // groups a block can hold (6:8: 16 or 32)
-    uint32_t wd[4] = {0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u};  // padding pairs
+    meta_stage(MetaSpan<M, FROM_MASK>(kb0, G), wmeta, mask, R, wbytes, mwords, row0, t, in[0]);
+    cp_async_commit();
     bool bad = false;
-    if (row < R) {
-        const uint8_t *inb = reinterpret_cast<const uint8_t *>(in[t]);
-        if (!FROM_MASK && M != 8 && ng * NWIN == 32) {
-            // natural order, a whole block of real windows: its 16 bytes as they are
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                wd[q] = static_cast<uint32_t>(inb[4 * q]) | (static_cast<uint32_t>(inb[4 * q + 1]) << 8) |
-                        (static_cast<uint32_t>(inb[4 * q + 2]) << 16) | (static_cast<uint32_t>(inb[4 * q + 3]) << 24);
+    for (int64_t kb = kb0; kb < kb1; ++kb) {
+        const int cur = static_cast<int>((kb - kb0) & 1);
+        if (kb + 1 < kb1) {
+            meta_stage(MetaSpan<M, FROM_MASK>(kb + 1, G), wmeta, mask, R, wbytes, mwords, row0, t, in[cur ^ 1]);
+            cp_async_commit();
+            cp_async_wait_pending<1>();  // this block's copies have landed (the next one's may not)
         } else {
+            cp_async_wait_pending<0>();
+        }
+        __syncthreads();  // every thread's copies of block kb, the table; rowb free again
+        const MetaSpan<M, FROM_MASK> sp(kb, G);
+        const int64_t g_lo = sp.g_lo, g_end = sp.g_end;
+        const int ng = static_cast<int>(g_end - g_lo);  // real groups of the block (<= its size)
+        const bool mid = M == 8 && (kb % 3) == 2;
+        uint32_t wd[4] = {0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u};  // padding pairs
+        if (row < R && ng > 0) {
+            const uint32_t *iw = in[cur][t];
+            if (!FROM_MASK && M != 8) {
+                // natural window order: the row's nibbles as they are, padding
+                // past the last real window
+                const int nv = ng * NWIN;
 #pragma unroll
-            for (int gi = 0; gi < GPB; ++gi) {
-                if (gi >= ng || (M == 8 && !mid && gi >= 16)) break;
-                const int64_t g = g_lo + gi;
-                uint32_t nibs;  // window w's nibble at bits 4w
-                if (FROM_MASK) {
-                    const int64_t c = g * M - 32 * u0;  // bit offset within the staged words
-                    const int q = static_cast<int>(c >> 5), off = static_cast<int>(c & 31);
-                    const uint64_t both = (static_cast<uint64_t>(q + 1 < nu ? in[t][q + 1] : 0u) << 32) | in[t][q];
-                    const uint32_t bits = static_cast<uint32_t>(both >> off) & ((1u << M) - 1u);
-                    if (M == 4) {
-                        // 2:4: the two survivors, ascending, are the set bits
-                        const uint32_t s0 = static_cast<uint32_t>(__ffs(bits) - 1);
-                        const uint32_t s1 = static_cast<uint32_t>(__ffs(bits & (bits - 1u)) - 1);
-                        nibs = __popc(bits) == 2 ? (s0 | (s1 << 2)) : 0xFFFFu;
-                    } else {
-                        nibs = tab[bits];
-                    }
-                    if (nibs == 0xFFFFu) {
-                        bad = true;
-                        continue;  // its slots keep the padding pair
-                    }
-                } else {
-                    nibs = 0;
-#pragma unroll
-                    for (int w = 0; w < NWIN; ++w) {
-                        const int64_t wi = g * NWIN + w;
-                        nibs |= ((static_cast<uint32_t>(inb[(wi >> 1) - u0]) >> (4 * (wi & 1))) & 0xFu) << (4 * w);
-                    }
+                for (int q = 0; q < 4; ++q) {
+                    const int keep = nv - 8 * q;
+                    const uint32_t m = keep >= 8 ? 0xFFFFFFFFu : (keep <= 0 ? 0u : (1u << (4 * keep)) - 1u);
+                    wd[q] = (iw[q] & m) | (0x44444444u & ~m);
                 }
-                // place the group's slots: natural order window w at slot gi * NWIN + w;
-                // 6:8 blocks 0/1: windows 0 and 2 at slots 2 gi, 2 gi + 1; block 2: window 1 at slot gi
-                auto place = [&](int slot, int width, uint32_t val) {  // slot, width static after unrolling
+            } else {
+                // group by group; every bit and nibble position is a constant
+                // once the loop is unrolled (the mask span of an 8:10 block
+                // starts at bit 0 or 16 of its first word: shifted away first)
+                const int base = M == 10 ? static_cast<int>((g_lo * M) & 31) : 0;
+                auto mword = [&](int q) -> uint32_t {
+                    return M == 10 ? __funnelshift_r(iw[q], iw[q + 1], base) : iw[q];
+                };
+                auto innib = [&](int n) -> uint32_t { return (iw[n >> 3] >> (4 * (n & 7))) & 0xFu; };
+                auto place = [&](int slot, int width, uint32_t val) {
                     const int sh = 4 * (slot & 7);
                     const uint32_t msk = width == 32 ? 0xFFFFFFFFu : (((1u << width) - 1u) << sh);
                     wd[slot >> 3] = (wd[slot >> 3] & ~msk) | ((val << sh) & msk);
                 };
-                if (M == 8) {
-                    if (mid)
-                        place(gi, 4, (nibs >> 4) & 0xFu);
-                    else
-                        place(2 * gi, 8, (nibs & 0xFu) | (((nibs >> 8) & 0xFu) << 4));
+                auto group = [&](int gi) {  // gi: a constant
+                    if (gi >= ng) return;
+                    uint32_t nibs;  // window w's nibble at bits 4w
+                    if (FROM_MASK) {
+                        const int c = gi * M, q = c >> 5, off = c & 31;
+                        const uint32_t raw = off + M <= 32 ? (mword(q) >> off) : __funnelshift_r(mword(q), mword(q + 1), off);
+                        const uint32_t bits = raw & ((1u << M) - 1u);
+                        bool valid;
+                        if (M == 4) {
+                            // 2:4: survivors s0 < s1 (the set bits), nibble s0 | s1 << 2
+                            nibs = static_cast<uint32_t>(kNib24 >> (4 * bits)) & 0xFu;
+                            valid = (kValid24 >> bits) & 1u;
+                        } else {
+                            nibs = tab[bits];
+                            valid = nibs != 0xFFFFu;
+                        }
+                        if (!valid) {
+                            bad = true;
+                            nibs = 0x4444u;  // the group's slots keep the padding pair
+                        }
+                    } else {  // 6:8 window bytes: windows 0, 1, 2 of group gi are nibbles 3 gi + w
+                        nibs = innib(3 * gi) | (innib(3 * gi + 1) << 4) | (innib(3 * gi + 2) << 8);
+                    }
+                    // natural order window w at slot gi * NWIN + w; 6:8 blocks 0 and 1:
+                    // windows 0 and 2 at slots 2 gi, 2 gi + 1; block 2: window 1 at slot gi
+                    if (M == 8) {
+                        if (mid)
+                            place(gi, 4, (nibs >> 4) & 0xFu);
+                        else
+                            place(2 * gi, 8, (nibs & 0xFu) | (((nibs >> 8) & 0xFu) << 4));
+                    } else {
+                        place(gi * NWIN, 4 * NWIN, nibs);
+                    }
+                };
+                if (M == 8 && mid) {
+#pragma unroll
+                    for (int gi = 0; gi < 32; ++gi) group(gi);
                 } else {
-                    place(gi * NWIN, 4 * NWIN, nibs);
+                    constexpr int GPB = M == 8 ? 16 : 32 / NWIN;  // groups of a block
+#pragma unroll
+                    for (int gi = 0; gi < GPB; ++gi) group(gi);
                 }
             }
         }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) rowb[t][q] = wd[q];
+        __syncthreads();  // rowb complete; in[cur] read by every thread
+        const int m0 = t & 7, k1 = (t >> 3) & 1, m2 = t >> 4;
+        const uint16_t *h0 = reinterpret_cast<const uint16_t *>(rowb[m0 + 16 * m2]);
+        const uint16_t *h1 = reinterpret_cast<const uint16_t *>(rowb[m0 + 16 * m2 + 8]);
+        uint32_t o[4];
+#pragma unroll
+        for (int k2 = 0; k2 < 4; ++k2)
+            o[k2] = static_cast<uint32_t>(h0[k1 + 2 * k2]) | (static_cast<uint32_t>(h1[k1 + 2 * k2]) << 16);
+        *reinterpret_cast<uint4 *>(out + (mt * nkb + kb) * EBLK_BYTES + t * 16) = make_uint4(o[0], o[1], o[2], o[3]);
     }
     if (bad) raise_error(ERRBIT_DEVICE);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) rowb[t][q] = wd[q];
-    __syncthreads();
-    const int m0 = t & 7, k1 = (t >> 3) & 1, m2 = t >> 4;
-    const uint16_t *h0 = reinterpret_cast<const uint16_t *>(rowb[m0 + 16 * m2]);
-    const uint16_t *h1 = reinterpret_cast<const uint16_t *>(rowb[m0 + 16 * m2 + 8]);
-    uint32_t o[4];
-#pragma unroll
-    for (int k2 = 0; k2 < 4; ++k2)
-        o[k2] = static_cast<uint32_t>(h0[k1 + 2 * k2]) | (static_cast<uint32_t>(h1[k1 + 2 * k2]) << 16);
-    *reinterpret_cast<uint4 *>(out + blk * EBLK_BYTES + t * 16) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // ---------------------------------------------------------------------------
@@ -651,6 +784,22 @@ __device__ __forceinline__ int64_t visit68(int64_t v, int64_t nkb) {
     return v < nraw ? 3 * (v >> 1) + (v & 1) : 3 * (v - nraw) + 2;
 }
 
+// Output tile order: bands of `gm` row tiles, each band walked token tile
+// by token tile (the band's row tiles side by side).  Concurrent CTA pairs
+// then share a few row tiles of weights and a few token tiles of X, which stay
+// in L2 across the pairs and the waves of a band, instead of every wave
+// streaming all of X again.  A bijection on [0, n_t * n_m); every role of a
+// kernel uses it, so stream-K ranges over the same linear order.
+__device__ __forceinline__ void tile_coords(int64_t tile, int64_t n_t, int64_t n_m, int64_t gm, int64_t &nt,
+                                            int64_t &mt) {
+    const int64_t band = tile / (gm * n_t);
+    const int64_t rem = tile - band * gm * n_t;
+    const int64_t rows = n_m - band * gm < gm ? n_m - band * gm : gm;  // row tiles of this band
+    nt = rem / rows;
+    mt = band * gm + (rem - nt * rows);
+}
+constexpr int64_t BAND_ROWS = 4096;   // weight rows per band of the tile order
+
 struct SegIter {
     bool sk;
     int64_t nkb, pos, end, step;
@@ -789,7 +938,8 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
             SegIter seg(sk, cluster, nclusters, ntiles, nkb);
             int64_t tile, kb0, kb1;
             while (ok && seg.next(tile, kb0, kb1)) {
-                const int64_t nt = tile % n_t, mt2 = tile / n_t;
+                int64_t nt, mt2;
+                tile_coords(tile, n_t, n_m, BAND_ROWS / 256, nt, mt2);
                 const int32_t arow = static_cast<int32_t>(mt2 * 256 + rank * 128);
                 const int32_t brow = static_cast<int32_t>(nt * C::BN + rank * C::BH);
                 for (int64_t kb = kb0; kb < kb1; ++kb, ++it) {
@@ -893,7 +1043,8 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
         SegIter seg(sk, cluster, nclusters, ntiles, nkb);
         int64_t tile, kb0, kb1;
         for (; seg.next(tile, kb0, kb1); ++ti) {
-            const int64_t nt = tile % n_t, mt2 = tile / n_t;
+            int64_t nt, mt2;
+            tile_coords(tile, n_t, n_m, BAND_ROWS / 256, nt, mt2);
             const int buf = static_cast<int>(ti % C::ACC_BUFS);
             const uint32_t aph = static_cast<uint32_t>((ti / C::ACC_BUFS) & 1);
             if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], aph))) break;
@@ -1010,7 +1161,9 @@ __global__ void __launch_bounds__(PairCfg<MODE>::THREADS, 1)
             // cp.async pipeline: stage of the block issued `d` steps ago, d = 1, 2
             int pend_s[2] = {-1, -1};
             for (int64_t tile = cluster; tile < ntiles && ok; tile += nclusters) {
-                const int64_t t0 = (tile % n_t) * C::BN + rank * C::BH;
+                int64_t ntl, mtl;
+                tile_coords(tile, n_t, n_m, BAND_ROWS / 256, ntl, mtl);
+                const int64_t t0 = ntl * C::BN + rank * C::BH;
                 for (int64_t kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = static_cast<int>(it % S);
                     const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
@@ -1263,7 +1416,8 @@ __global__ void __launch_bounds__(WideCfg::THREADS, 1)
             int64_t tile, kb0, kb1;
             const uint32_t b_bytes = static_cast<uint32_t>(bh) * 256u;
             while (ok && seg.next(tile, kb0, kb1)) {
-                const int64_t nt = tile % n_t, mt = tile / n_t;
+                int64_t nt, mt;
+                tile_coords(tile, n_t, n_m, BAND_ROWS / 512, nt, mt);
                 const bool has1 = mt * 512 + 256 < Rpad;
                 const int32_t arow = static_cast<int32_t>(mt * 512 + rank * 128);
                 const int32_t brow = static_cast<int32_t>(nt * bn + rank * bh);
@@ -1312,7 +1466,9 @@ __global__ void __launch_bounds__(WideCfg::THREADS, 1)
             SegIter seg(sk, cluster, nclusters, ntiles, nkb);
             int64_t tile, kb0, kb1;
             for (; ok && seg.next(tile, kb0, kb1); ++ti) {
-                const bool has1 = (tile / n_t) * 512 + 256 < Rpad;
+                int64_t ntm, mtm;
+                tile_coords(tile, n_t, n_m, BAND_ROWS / 512, ntm, mtm);
+                const bool has1 = mtm * 512 + 256 < Rpad;
                 if (ti >= 1 && !mbar_wait_cluster(acc_empty, static_cast<uint32_t>((ti - 1) & 1))) {
                     ok = false;
                     break;
@@ -1361,7 +1517,8 @@ __global__ void __launch_bounds__(WideCfg::THREADS, 1)
         SegIter seg(sk, cluster, nclusters, ntiles, nkb);
         int64_t tile, kb0, kb1, ti = 0;
         for (; seg.next(tile, kb0, kb1); ++ti) {
-            const int64_t nt = tile % n_t, mt = tile / n_t;
+            int64_t nt, mt;
+            tile_coords(tile, n_t, n_m, BAND_ROWS / 512, nt, mt);
             if (!__all_sync(0xffffffffu, mbar_wait(acc_full, static_cast<uint32_t>(ti & 1)))) break;
             tc_fence_after();
             const bool active = h == 0 || mt * 512 + 256 < Rpad;
@@ -1772,26 +1929,42 @@ nm_status launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensor
     return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
 }
 
-// tokens per wide tile: the fewest tiles of at most 240 tokens, as even as
-// multiples of 16 allow
-int64_t wide_bn(int64_t T) {
-    const int64_t nt = (T + WideCfg::BN_MAX - 1) / WideCfg::BN_MAX;
-    const int64_t per = (T + nt - 1) / nt;
-    return (per + 15) / 16 * 16;
+// tokens per wide tile.  Candidates: the fewest tiles of at most 240 tokens
+// and, when that is already several, one or two more, each as even as
+// multiples of 16 allow; the one with the least (waves of tiles over the
+// resident CTA pairs) x (tokens per tile + 32), the N/2 + 32 clocks a sparse
+// MMA of N tokens costs per K' step, so that a last, nearly empty wave is
+// traded for slightly narrower tiles.  (One tile's worth of tokens stays one
+// tile: more would only re-read the weights.)
+int64_t wide_bn(int64_t T, int64_t R, int64_t pairs) {
+    const int64_t n_m = ((R + 255) / 256 * 256 + 511) / 512;
+    const int64_t nt0 = (T + WideCfg::BN_MAX - 1) / WideCfg::BN_MAX;
+    const int64_t nt_last = nt0 >= 2 ? nt0 + 2 : nt0;
+    int64_t best = 0, best_cost = 0;
+    for (int64_t nt = nt0; nt <= nt_last; ++nt) {
+        const int64_t per = (T + nt - 1) / nt;
+        const int64_t bn = (per + 15) / 16 * 16;
+        const int64_t tiles = ((T + bn - 1) / bn) * n_m;
+        const int64_t cost = ((tiles + pairs - 1) / pairs) * (bn + 32);
+        if (best == 0 || cost < best_cost) {
+            best = bn;
+            best_cost = cost;
+        }
+        if (per <= 16) break;
+    }
+    return best;
 }
 
+// CTA pairs of k_gemm_wide<MODE> that can be resident at once on the current
+// device (0 on a CUDA error), cached per device
 template <int MODE>
-nm_status launch_wide(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b2,
-                      const CUtensorMap &e, const CUtensorMap &y, uint16_t *Y, int64_t ldy, int64_t T,
-                      int64_t R, int64_t nkb, int bn, void *sk_ws, size_t sk_ws_bytes, cudaStream_t s) {
+int64_t wide_pairs() {
     using Cfg = WideCfg;
-    if (!set_smem_attr<k_gemm_wide<MODE>>(Cfg::SMEM_BYTES)) return NM_ERR_CUDA;
-    const int64_t Rpad = (R + 255) / 256 * 256;
-    const int64_t ntiles = ((T + bn - 1) / bn) * ((Rpad + 511) / 512);
     static int cache[64] = {};
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NM_ERR_CUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
     if (cache[dev] == 0) {
+        if (!set_smem_attr<k_gemm_wide<MODE>>(Cfg::SMEM_BYTES)) return 0;
         cudaLaunchConfig_t q = {};
         q.gridDim = dim3(2 * static_cast<unsigned>(sm_count() / 2), 1, 1);
         q.blockDim = dim3(Cfg::THREADS, 1, 1);
@@ -1814,7 +1987,20 @@ nm_status launch_wide(const CUtensorMap &a, const CUtensorMap &b, const CUtensor
     const int forced = g_sched_clusters.load();
     if (forced > 0 && forced < res) res = forced;
     if (res > SK_MAX_CLUSTERS) res = SK_MAX_CLUSTERS;
-    if (res < 1) res = 1;
+    return res < 1 ? 1 : res;
+}
+
+template <int MODE>
+nm_status launch_wide(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b2,
+                      const CUtensorMap &e, const CUtensorMap &y, uint16_t *Y, int64_t ldy, int64_t T,
+                      int64_t R, int64_t nkb, int bn, void *sk_ws, size_t sk_ws_bytes, cudaStream_t s) {
+    using Cfg = WideCfg;
+    if (!set_smem_attr<k_gemm_wide<MODE>>(Cfg::SMEM_BYTES)) return NM_ERR_CUDA;
+    const int64_t Rpad = (R + 255) / 256 * 256;
+    const int64_t ntiles = ((T + bn - 1) / bn) * ((Rpad + 511) / 512);
+    const int64_t res = wide_pairs<MODE>();  // with a forced pair count applied
+    if (res == 0) return NM_ERR_CUDA;
+    const int forced = g_sched_clusters.load();
     const int policy = g_sched_policy.load();
     const bool sk_ok = sk_ws != nullptr && sk_ws_bytes >= sk_bytes(res) &&
                        (reinterpret_cast<uintptr_t>(sk_ws) & 15u) == 0;
@@ -1864,17 +2050,18 @@ nm_status launch_prepare(const uint16_t *vals, const uint8_t *wmeta, const uint3
     const int n = m - 2;
     if (m == 8) {
         const int64_t nj = p.nkb / 3;
-        const int64_t warps = p.Rpad * nj;
-        if ((warps + 7) / 8 > 0x7FFFFFFF) return NM_ERR_SHAPE;
-        k_prepare_vals68<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, s>>>(
-            vals, R, p.G, p.Rpad, nj, p.KLpad / 2, static_cast<uint16_t *>(packed));
+        const int64_t rb = (p.Rpad + 7) / 8;
+        dim3 g68(static_cast<unsigned>((nj + PV68_JW - 1) / PV68_JW), static_cast<unsigned>(rb < 65535 ? rb : 65535),
+                 static_cast<unsigned>((rb + 65534) / 65535));
+        k_prepare_vals68<<<g68, 256, 0, s>>>(vals, R, p.G, p.Rpad, nj, p.KLpad / 2,
+                                             static_cast<uint16_t *>(packed));
     } else {
         const int64_t chunks = p.KLpad / 16;  // 16-byte chunks of a packed row
         const int64_t words = p.G * n / 2;
         const bool vec = (words % 4) == 0 && (reinterpret_cast<uintptr_t>(vals) & 15u) == 0;
-        dim3 vgrid(static_cast<unsigned>((chunks + 255) / 256),
-                   static_cast<unsigned>(p.Rpad < 65535 ? p.Rpad : 65535),
-                   static_cast<unsigned>((p.Rpad + 65534) / 65535));
+        const int64_t rb = (p.Rpad + PV_ROWS - 1) / PV_ROWS;
+        dim3 vgrid(static_cast<unsigned>((chunks + 255) / 256), static_cast<unsigned>(rb < 65535 ? rb : 65535),
+                   static_cast<unsigned>((rb + 65534) / 65535));
         k_prepare_vals<<<vgrid, 256, 0, s>>>(vals, R, words, p.Rpad, p.KLpad / 2, vec,
                                              static_cast<uint16_t *>(packed));
     }
@@ -1882,7 +2069,7 @@ nm_status launch_prepare(const uint16_t *vals, const uint8_t *wmeta, const uint3
     if (nblocks > 0x7FFFFFFF) return NM_ERR_SHAPE;
     uint8_t *meta = static_cast<uint8_t *>(packed) + p.vals_bytes;
     const int64_t mwords = (p.G * m + 31) / 32;
-    const unsigned nb = static_cast<unsigned>(nblocks);
+    const unsigned nb = static_cast<unsigned>((p.Rpad / BM) * ((p.nkb + PM_KPB - 1) / PM_KPB));
     const int64_t wb = (p.nwin + 1) / 2;
 #define NM_PREP_META(MM)                                                                                   \
     (mask ? (k_prepare_meta<MM, true><<<nb, BM, 0, s>>>(nullptr, mask, R, p.G, 0, mwords, p.nkb, meta), 0) \
@@ -2037,7 +2224,12 @@ nm_status sparse_gemm_impl(const uint16_t *X, int64_t T, int64_t K, int64_t ldx,
         b_cols = w.cols;
         b_ld = w.ld;
     }
-    const int bh = wide ? static_cast<int>(wide_bn(T) / 2) : 128;
+    int bh = 128;
+    if (wide) {
+        const int64_t pairs = m == 8 ? wide_pairs<PMODE_SP68T>() : wide_pairs<PMODE_SP24>();
+        if (pairs == 0) return NM_ERR_CUDA;
+        bh = static_cast<int>(wide_bn(T, R, pairs) / 2);
+    }
     CUtensorMap tb, tb2;
     if (!make_tmap_bf16(&tb, b_src, T, b_cols, b_ld, 64, static_cast<uint32_t>(bh), true)) return NM_ERR_CUDA;
     if (m == 8 && !make_tmap_bf16(&tb2, stage, T, w.cols, w.ld, 64, static_cast<uint32_t>(bh), true))

@@ -192,15 +192,16 @@ __device__ __noinline__ double exact_sq_column(const uint16_t *__restrict__ X, i
 // exact pair (s, c) -- or NaN in s for a marked column -- and k_hsq_finish
 // adds the pairs of a column.
 //
-// x^2 comes from the bits without a conversion: d = x 2^-896 is the fp64
-// with high word (bits & 0x7FFF) << 13 and g = x 2^896 the same plus
-// 1792 << 20, so d * g = x^2 exactly for every normal x and zero (d = 0), and
-// fma(d, g, acc) rounds like acc + x^2; an infinity or a NaN makes g, hence
-// the sum, inf or NaN, which fails the check.  The check of fact (1) needs the
-// run's smallest nonzero magnitude, kept two columns at a time as a signed
-// 16-bit minimum of t + 0x7FFF over the magnitude bits t (0x7FFF for a zero,
-// the largest; 0x8000 + t - 1, negative and increasing in t, otherwise).  A
-// subnormal (exponent field 0, where g is wrong) fails the check as well.
+// x comes from its bits without a conversion: d = x 2^-896 is the fp64 with
+// high word (bits & 0x7FFF) << 13 (exact for every finite bf16, zeros and
+// subnormals included), |x| = d * 2^896 exactly, and fma(x, x, acc) rounds
+// like acc + x^2 (x^2 exact in fp64, below 2^256).  An infinity or a NaN reads
+// as 2^128 (1 + f/128).  The check of fact (1) needs the run's smallest
+// nonzero magnitude, kept two columns at a time as a signed 16-bit minimum of
+// t + 0x7FFF over the magnitude bits t (0x7FFF for a zero, the largest;
+// 0x8000 + t - 1, negative and increasing in t, otherwise); a run holding an
+// infinity, a NaN or a subnormal (exponent field 255 or 0) fails it and is
+// looked at bit by bit.
 // ---------------------------------------------------------------------------
 constexpr int HX_THREADS = 256;
 constexpr int HX_WARPS = HX_THREADS / 32;
@@ -220,19 +221,22 @@ struct HPair {
 // x^2 of the two bf16 halves of a word (low half: w << 13; high half: w >> 3)
 // into the sums of columns k, k + 1, and their smallest magnitudes into key
 __device__ __forceinline__ void sq_word(uint32_t w, double (&a)[HX_VEC], uint32_t &key, int k) {
-    const uint32_t d0 = (w << 13) & 0x0FFFE000u, d1 = (w >> 3) & 0x0FFFE000u;
-    a[k] = __fma_rn(hw_double(d0), hw_double(d0 + 0x70000000u), a[k]);
-    a[k + 1] = __fma_rn(hw_double(d1), hw_double(d1 + 0x70000000u), a[k + 1]);
+    const double x0 = __dmul_rn(hw_double((w << 13) & 0x0FFFE000u), 0x1p896);
+    const double x1 = __dmul_rn(hw_double((w >> 3) & 0x0FFFE000u), 0x1p896);
+    a[k] = __fma_rn(x0, x0, a[k]);
+    a[k + 1] = __fma_rn(x1, x1, a[k + 1]);
     key = vmin_s16x2(key, (w & 0x7FFF7FFFu) + 0x7FFF7FFFu);
 }
 
 // fact (1) for a run: no nonzero value (key 0x7FFF), or a normal smallest
 // value (exponent field e >= 1) and a sum below 2^53 units of its square,
-// 2^(2e - 268 + 53), whose fp64 exponent field is 2e + 808
+// 2^(2e - 268 + 53), whose fp64 exponent field is 2e + 808, and below 2^256
+// (an infinity or a NaN, read as 2^128 (1 + f/128), squares to at least that;
+// finite squares are smaller)
 __device__ __forceinline__ bool sq_run_exact(double a, uint32_t key16) {
     if (key16 == 0x7FFFu) return true;
     const int e = static_cast<int>((key16 - 0x7FFFu) >> 7);
-    return e >= 1 && a < hw_double(static_cast<uint32_t>(2 * e + 808) << 20);
+    return e >= 1 && a < hw_double(static_cast<uint32_t>(2 * e + 808) << 20) && a < 0x1p256;
 }
 
 // A run that failed its check, summed again from the tile in two parts: the
@@ -1065,7 +1069,7 @@ __global__ void __launch_bounds__(128, 4)
 // a4: sliding-window pack.  Each thread handles GT consecutive groups whose
 // mask bits start on a 32-bit word boundary (GT*m a multiple of 32) and whose
 // window nibbles fill whole bytes (GT*(m/2-1) even): it reads GT*m/32 words and
-// writes GT*(m/2-1)/2 bytes.  grid: x over runs of a row, y = row.
+// writes GT*(m/2-1)/2 bytes.  A grid-stride loop over (row, run) pairs.
 // ---------------------------------------------------------------------------
 template <int M>
 struct SlideRun {
@@ -1080,12 +1084,21 @@ __global__ void __launch_bounds__(256)
     k_slide_pack(const uint32_t *__restrict__ mask, int64_t R, int64_t G, int64_t mwords,
                  int64_t wbytes, uint8_t *__restrict__ wmeta) {
     using RC = SlideRun<M>;
+    // (2N-2):2N: a group's window nibbles come from one lookup in the
+    // compile-time window table (entry 0xFFFF: not exactly m - 2 survivors)
+    __shared__ uint16_t tab[M == 4 ? 1 : (1 << M)];
+    if (M != 4) {
+        for (int i = threadIdx.x; i < (1 << M); i += blockDim.x) tab[i] = g_wintab.v[wt_offset(M) + i];
+        __syncthreads();
+    }
     const uint64_t rpr = static_cast<uint64_t>((G + RC::GT - 1) / RC::GT);  // runs per row
     const uint64_t total = rpr * static_cast<uint64_t>(R);
+    const bool narrow = total <= 0xFFFFFFFFull;
     bool bad = false;
     for (uint64_t idx = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
          idx += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
-        const uint64_t row = idx / rpr, run = idx - row * rpr;
+        const uint64_t row = narrow ? static_cast<uint32_t>(idx) / static_cast<uint32_t>(rpr) : idx / rpr;
+        const uint64_t run = idx - row * rpr;
         const int64_t g0 = static_cast<int64_t>(run) * RC::GT;
         const uint32_t *mrow = mask + row * mwords + run * RC::WORDS;
         uint32_t w[RC::WORDS];
@@ -1102,21 +1115,19 @@ __global__ void __launch_bounds__(256)
             uint32_t bits = w[b0 >> 5] >> (b0 & 31);
             if ((b0 & 31) + M > 32) bits |= w[(b0 >> 5) + 1] << (32 - (b0 & 31));
             bits &= (1u << M) - 1u;
-            if (__popc(bits) != M - 2) { bad = true; continue; }
-            // survivor k -> window k/2, index q_k - 2*(k/2)
-            uint32_t rem = bits;
-#pragma unroll
-            for (int wv = 0; wv < RC::NWIN; ++wv) {
-                const int qa = __ffs(rem) - 1;
-                rem &= rem - 1u;
-                const int qb = __ffs(rem) - 1;
-                rem &= rem - 1u;
-                const int a = qa - 2 * wv, b = qb - 2 * wv;
-                if (a < 0 || b > 3) bad = true;
-                const int wi = gi * RC::NWIN + wv;                 // nibble index in the run
-                const uint32_t nb = static_cast<uint32_t>((a & 3) | ((b & 3) << 2));
-                ow[wi >> 3] |= nb << (4 * (wi & 7));
+            uint32_t nibs;  // window w's nibble at bits 4w
+            if (M == 4) {
+                // 2:4: the two survivors, ascending, are the set bits
+                if (__popc(bits) != 2) { bad = true; continue; }
+                nibs = static_cast<uint32_t>(__ffs(bits) - 1) | (static_cast<uint32_t>(__ffs(bits & (bits - 1u)) - 1) << 2);
+            } else {
+                nibs = tab[bits];
+                if (nibs == 0xFFFFu) { bad = true; continue; }
             }
+            const int wi = gi * RC::NWIN;  // first nibble of the group in the run
+            const int sh = 4 * (wi & 7);
+            ow[wi >> 3] |= nibs << sh;
+            if ((wi & 7) + RC::NWIN > 8) ow[(wi >> 3) + 1] |= nibs >> (32 - sh);
         }
         const int64_t byte0 = g0 * RC::NWIN / 2;
         uint8_t *dst = wmeta + row * wbytes + byte0;
@@ -1188,6 +1199,7 @@ __device__ __forceinline__ void abs_word(uint32_t w, double &up, double &dn, uin
 
 __global__ void __launch_bounds__(256)
     k_row_abs_sum(const uint16_t *__restrict__ W, int64_t R, int64_t K, int64_t ldw, HPair *__restrict__ rec) {
+    grid_dep_launch();
     const int lane = threadIdx.x & 31;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     if (row >= R) return;  // warp-uniform
@@ -1253,50 +1265,142 @@ __device__ uint32_t f64_to_bf16_bits(double v) {
     return sign | (static_cast<uint32_t>(e + 127) << 7) | static_cast<uint32_t>(top & 0x7Full);
 }
 
-// gamma from the rows' exact pairs: every thread adds its rows into an
-// integer accumulator, the block adds the accumulators digit by digit, one
-// rounding, one division by R*K.  One block of 1024 threads.
+// clip(rint(fl(w / gamma)), -1, 1) without the division.  fl(|w| / gamma) > 0.5
+// exactly when |w| / gamma > 0.5 + 2^-54 (the half-way point to the next
+// double, which rounds to even = 0.5), i.e. |w| > h + 2^-54 gamma with
+// h = gamma / 2.  For h < |w| <= 2h the difference |w| - h is exact (Sterbenz);
+// above 2h the condition holds outright.  rint(x) for |x| > 0.5 is at least 1
+// and clips to 1; |x| <= 0.5 gives 0 (0.5 ties to even).  gamma is a normal
+// double (bf16(gamma) was representable), so gamma / 2 and 2^-54 gamma are
+// exact.  The predicate grows with |w|, and non-negative bf16 values grow
+// with their bit patterns, so it holds exactly for the magnitudes
+// (bits & 0x7FFF) at or above one threshold: the smallest pattern for which
+// it holds, found once by bisection over [0, 0x7F80] (0x7F80, +inf, always
+// holds).  W itself is finite whenever bf16(gamma) is representable (an
+// infinity or NaN in W makes gamma infinite or NaN, which zeroes the output).
+__device__ __forceinline__ bool ternary_is_one(uint32_t mag_bits, double h, double tiny) {
+    const double a = bf16_to_f64(static_cast<uint16_t>(mag_bits));
+    return a > 2.0 * h || (a > h && __dsub_rn(a, h) > tiny);
+}
+
+__device__ uint32_t ternary_threshold(double gamma) {
+    const double h = 0.5 * gamma, tiny = gamma * 0x1p-54;
+    uint32_t lo = 0u, hi = 0x7F80u;  // the answer lies in [lo, hi]; hi holds
+    while (lo < hi) {
+        const uint32_t mid = (lo + hi) >> 1;
+        if (ternary_is_one(mid, h, tiny))
+            hi = mid;
+        else
+            lo = mid + 1u;
+    }
+    return lo;
+}
+
+// gamma from the rows' exact pairs.  First with TwoSum (fact 2): every
+// thread adds its rows' pairs, the warps and then the block combine their
+// (s, c up, c down) triples; when no row was marked and c up equals c down
+// the total s + c is exact and is rounded once.  Otherwise every thread adds
+// its rows into an integer accumulator (a marked row summed again from W),
+// the block adds the accumulators digit by digit and rounds once.  Then one
+// division by R*K.  One block of 1024 threads.
+__device__ __forceinline__ void triple_shfl_add(double &S, double &CU, double &CD, int off) {
+    const double s2 = __shfl_down_sync(0xffffffffu, S, off);
+    const double u2 = __shfl_down_sync(0xffffffffu, CU, off);
+    const double d2 = __shfl_down_sync(0xffffffffu, CD, off);
+    two_sum_acc2(S, CU, CD, s2);
+    CU = __dadd_ru(CU, u2);
+    CD = __dadd_rd(CD, d2);
+}
+
 __global__ void __launch_bounds__(1024) k_gamma(const HPair *__restrict__ rec, const uint16_t *__restrict__ W,
                                                 int64_t R, int64_t K, int64_t ldw,
                                                 double *__restrict__ gamma_out, uint32_t *__restrict__ gb_out) {
     __shared__ long long part[32][GB_NDIG];
-    AbsAcc a;
-    a.clear();
-    bool nan = false, inf = false;
-    for (int64_t i = threadIdx.x; i < R; i += blockDim.x) {
-        const HPair p = rec[i];
-        if (!isnan(p.s)) {
-            a.add_double(p.s);
-            a.add_double(p.c);
-            continue;
+    __shared__ double tri[3][32];
+    __shared__ double fast_total;
+    __shared__ int fast_ok;
+    grid_dep_wait();    // the rows' pairs
+    grid_dep_launch();  // the apply grid may start loading W
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    double S = 0.0, CU = 0.0, CD = 0.0;
+    bool marked = false;
+    for (int64_t i0 = threadIdx.x; i0 < R; i0 += 4 * static_cast<int64_t>(blockDim.x)) {
+        HPair p[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int64_t i = i0 + q * static_cast<int64_t>(blockDim.x);
+            p[q] = i < R ? rec[i] : HPair{0.0, 0.0};
         }
-        for (int64_t j = 0; j < K; ++j) {  // the integer path for a marked row
-            const uint32_t b = W[i * ldw + j] & 0x7FFFu;
-            const int e = static_cast<int>(b >> 7);
-            if (e == 255) {
-                nan |= (b & 0x7Fu) != 0;
-                inf |= (b & 0x7Fu) == 0;
-            } else if (b) {
-                a.add_bits(e ? 128u + (b & 0x7Fu) : b, (e ? e : 1) - 134 + GB_BIAS, false);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            marked |= isnan(p[q].s);
+            two_sum_acc2(S, CU, CD, p[q].s);
+            CU = __dadd_ru(CU, p[q].c);
+            CD = __dadd_rd(CD, p[q].c);
+        }
+    }
+    for (int off = 16; off >= 1; off >>= 1) triple_shfl_add(S, CU, CD, off);
+    if (lane == 0) {
+        tri[0][warp] = S;
+        tri[1][warp] = CU;
+        tri[2][warp] = CD;
+    }
+    marked = __syncthreads_or(marked) != 0;
+    if (warp == 0) {
+        const int nw = static_cast<int>(blockDim.x / 32);
+        S = lane < nw ? tri[0][lane] : 0.0;
+        CU = lane < nw ? tri[1][lane] : 0.0;
+        CD = lane < nw ? tri[2][lane] : 0.0;
+        for (int off = 16; off >= 1; off >>= 1) triple_shfl_add(S, CU, CD, off);
+        if (lane == 0) {
+            // a NaN pair (marked row) makes S NaN: then the integer path decides
+            fast_ok = !marked && CU == CD;
+            fast_total = __dadd_rn(S, CU);
+        }
+    }
+    __syncthreads();
+    double total;
+    bool nan = false, inf = false;
+    if (fast_ok) {
+        if (threadIdx.x != 0) return;
+        total = fast_total;
+    } else {
+        AbsAcc a;
+        a.clear();
+        for (int64_t i = threadIdx.x; i < R; i += blockDim.x) {
+            const HPair p = rec[i];
+            if (!isnan(p.s)) {
+                a.add_double(p.s);
+                a.add_double(p.c);
+                continue;
+            }
+            for (int64_t j = 0; j < K; ++j) {  // the integer path for a marked row
+                const uint32_t b = W[i * ldw + j] & 0x7FFFu;
+                const int e = static_cast<int>(b >> 7);
+                if (e == 255) {
+                    nan |= (b & 0x7Fu) != 0;
+                    inf |= (b & 0x7Fu) == 0;
+                } else if (b) {
+                    a.add_bits(e ? 128u + (b & 0x7Fu) : b, (e ? e : 1) - 134 + GB_BIAS, false);
+                }
             }
         }
-    }
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-    for (int i = 0; i < GB_NDIG; ++i) {
-        long long v = a.d[i];
-        for (int off = 16; off >= 1; off >>= 1) v += __shfl_down_sync(0xffffffffu, v, off);
-        if (lane == 0) part[warp][i] = v;
-    }
-    nan = __syncthreads_or(nan) != 0;
-    inf = __syncthreads_or(inf) != 0;
-    if (threadIdx.x != 0) return;
-    AbsAcc tot;
-    tot.clear();
-    for (int wv = 0; wv < static_cast<int>(blockDim.x / 32); ++wv)
+        for (int i = 0; i < GB_NDIG; ++i) {
+            long long v = a.d[i];
+            for (int off = 16; off >= 1; off >>= 1) v += __shfl_down_sync(0xffffffffu, v, off);
+            if (lane == 0) part[warp][i] = v;
+        }
+        nan = __syncthreads_or(nan) != 0;
+        inf = __syncthreads_or(inf) != 0;
+        if (threadIdx.x != 0) return;
+        AbsAcc tot;
+        tot.clear();
+        for (int wv = 0; wv < static_cast<int>(blockDim.x / 32); ++wv)
 #pragma unroll
-        for (int i = 0; i < GB_NDIG; ++i) tot.d[i] += part[wv][i];
-    double total = tot.round_rn();
+            for (int i = 0; i < GB_NDIG; ++i) tot.d[i] += part[wv][i];
+        total = tot.round_rn();
+    }
     if (nan) total = __longlong_as_double(0x7FF8000000000000ll);
     else if (inf) total = __longlong_as_double(0x7FF0000000000000ll);
     const double gamma = __ddiv_rn(total, __dmul_rn(static_cast<double>(R), static_cast<double>(K)));
@@ -1306,52 +1410,41 @@ __global__ void __launch_bounds__(1024) k_gamma(const HPair *__restrict__ rec, c
         gb = 0xFFFFu;
     }
     *gamma_out = gamma;
-    *gb_out = gb;
+    gb_out[0] = gb;
+    gb_out[1] = gb == 0xFFFFu ? 0x7F80u : ternary_threshold(gamma);
 }
 
-// clip(rint(fl(w / gamma)), -1, 1) without the division.  fl(|w| / gamma) > 0.5
-// exactly when |w| / gamma > 0.5 + 2^-54 (the half-way point to the next
-// double, which rounds to even = 0.5), i.e. |w| > h + 2^-54 gamma with
-// h = gamma / 2.  For h < |w| <= 2h the difference |w| - h is exact (Sterbenz);
-// above 2h the condition holds outright.  rint(x) for |x| > 0.5 is at least 1
-// and clips to 1; |x| <= 0.5 gives 0 (0.5 ties to even).  gamma is a normal
-// double (bf16(gamma) was representable), so gamma / 2 and 2^-54 gamma are
-// exact.  W itself is never NaN here (a NaN would make gamma NaN, which zeroes
-// the output).
-__device__ __forceinline__ uint32_t ternary_one(uint32_t wbits, double h, double tiny, uint32_t gb) {
-    const double a = fabs(bf16_to_f64(static_cast<uint16_t>(wbits)));
-    const bool one = a > 2.0 * h || (a > h && __dsub_rn(a, h) > tiny);
-    return one ? ((wbits & 0x8000u) ? (gb | 0x8000u) : gb) : 0u;
+// W_q = clip(rint(W / gamma), -1, 1) * bf16(gamma): +-bf16(gamma) where
+// |w|'s bits reach the threshold, else 0.  grid: x over 8-column chunks of a
+// row (16-byte load, 16-byte store), y (+65535 z) = row.  Launched as a
+// programmatic dependent of k_gamma: W is loaded before the wait for gamma.
+__device__ __forceinline__ uint32_t ternary_pair(uint32_t w2, uint32_t thr, uint32_t gb) {
+    const uint32_t lo = (w2 & 0x7FFFu) >= thr ? ((w2 & 0x8000u) | gb) : 0u;
+    const uint32_t hi = ((w2 >> 16) & 0x7FFFu) >= thr ? (((w2 >> 16) & 0x8000u) | gb) : 0u;
+    return lo | (hi << 16);
 }
 
-// W_q = clip(rint(W / gamma), -1, 1) * bf16(gamma).  grid: x over 8-column
-// chunks of a row (16-byte load, 16-byte store), y (+65535 z) = row.
 __global__ void __launch_bounds__(256)
     k_ternary_apply(const uint16_t *__restrict__ W, int64_t R, int64_t K, int64_t ldw,
-                    const double *__restrict__ gamma_p, const uint32_t *__restrict__ gb_p,
-                    uint16_t *__restrict__ Wq) {
+                    const uint32_t *__restrict__ gb_p, uint16_t *__restrict__ Wq) {
     const int64_t i = blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535;
     const int64_t j0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+    const bool full = i < R && j0 + 8 <= K && (K & 7) == 0;
+    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+    if (full) u = __ldg(reinterpret_cast<const uint4 *>(W + i * ldw + j0));
+    grid_dep_wait();  // gamma, its bf16 bits and the threshold
     if (i >= R || j0 >= K) return;
-    const double gamma = *gamma_p;
-    const uint32_t gb = *gb_p;
+    const uint32_t gb = gb_p[0];
     const bool ok = gb != 0xFFFFu;
-    const double h = 0.5 * gamma, tiny = gamma * 0x1p-54;
+    const uint32_t thr = ok ? gb_p[1] : 0x10000u;  // nothing reaches 0x10000
+    const uint32_t g = ok ? gb : 0u;
     uint16_t *dst = Wq + i * K + j0;
-    if (j0 + 8 <= K && (K & 7) == 0) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(W + i * ldw + j0));
-        const uint32_t in[4] = {u.x, u.y, u.z, u.w};
-        uint32_t o[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const uint32_t lo = ok ? ternary_one(in[e] & 0xFFFFu, h, tiny, gb) : 0u;
-            const uint32_t hi = ok ? ternary_one(in[e] >> 16, h, tiny, gb) : 0u;
-            o[e] = lo | (hi << 16);
-        }
-        *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+    if (full) {
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(ternary_pair(u.x, thr, g), ternary_pair(u.y, thr, g),
+                                                     ternary_pair(u.z, thr, g), ternary_pair(u.w, thr, g));
     } else {
         for (int64_t j = j0; j < K && j < j0 + 8; ++j)
-            dst[j - j0] = static_cast<uint16_t>(ok ? ternary_one(W[i * ldw + j], h, tiny, gb) : 0u);
+            dst[j - j0] = static_cast<uint16_t>(ternary_pair(W[i * ldw + j], thr, g));
     }
 }
 
@@ -1611,10 +1704,25 @@ extern "C" nm_status nm_ternary_quantize(const uint16_t *W, int64_t R, int64_t K
     uint32_t *gb = reinterpret_cast<uint32_t *>(rec + R);
     if ((R + 7) / 8 > 0x7FFFFFFF || R > 65535LL * 65535LL) return NM_ERR_SHAPE;
     k_row_abs_sum<<<static_cast<unsigned>((R + 7) / 8), 256, 0, s>>>(W, R, K, ldw, rec);
-    k_gamma<<<1, 1024, 0, s>>>(rec, W, R, K, ldw, gamma, gb);
-    dim3 grid(static_cast<unsigned>((K + 2047) / 2048), static_cast<unsigned>(R < 65535 ? R : 65535),
-              static_cast<unsigned>((R + 65534) / 65535));
-    k_ternary_apply<<<grid, 256, 0, s>>>(W, R, K, ldw, gamma, gb, Wq);
+    // k_gamma and the apply grid are programmatic dependents: each may start
+    // once its predecessor lets it and waits in-kernel for that one's results
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, 1, 1);
+    cfg.blockDim = dim3(1024, 1, 1);
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k_gamma, static_cast<const HPair *>(rec), W, R, K, ldw, gamma, gb) != cudaSuccess)
+        return NM_ERR_CUDA;
+    cfg.gridDim = dim3(static_cast<unsigned>((K + 2047) / 2048), static_cast<unsigned>(R < 65535 ? R : 65535),
+                       static_cast<unsigned>((R + 65534) / 65535));
+    cfg.blockDim = dim3(256, 1, 1);
+    if (cudaLaunchKernelEx(&cfg, k_ternary_apply, W, R, K, ldw, static_cast<const uint32_t *>(gb), Wq) !=
+        cudaSuccess)
+        return NM_ERR_CUDA;
     return launch_status();
 }
 

@@ -417,7 +417,8 @@ def test_sparse_gemm_vs_oracle(nm, m, R, K, T):
 
 # tokens per wide tile: T <= 240 gives one tile of T rounded up to 16 (the
 # last store of 16 tokens when T % 32 lands in (0, 16]); larger T splits into
-# near-equal tiles of at most 240
+# near-equal tiles of at most 240 (their count chosen against the resident CTA
+# pairs' waves)
 @pytest.mark.parametrize("T", [1, 16, 33, 48, 240, 241, 496, 721])
 @pytest.mark.parametrize("m,R", [(4, 700), (8, 512)])
 def test_sparse_gemm_token_tiling(nm, m, R, T):
@@ -549,6 +550,29 @@ def test_ternary_gamma_exact_rounding_and_specials(nm):
         torch.cuda.synchronize()
         with pytest.raises(nm.NMError, match="NM_ERR_DEVICE"):
             nm.check_device_error()
+
+
+def test_ternary_threshold_at_the_tie(nm):
+    # gamma = mean |w| = 1 exactly: ones everywhere but six values whose
+    # magnitudes also sum to six.  |w| = 0.5 is the tie (rint(0.5) = 0), the
+    # bf16 just below gives 0 and the one just above gives +-bf16(gamma)
+    def bf(v):
+        return np.frombuffer(np.float32(v).tobytes(), dtype=np.uint16)[1]
+    W = np.full((16, 64), bf(1.0), dtype=np.uint16)
+    W[::2, 1::3] |= 0x8000                                   # signs play no part in gamma
+    specials = [(0.5, (3, 5)), (0.498046875, (4, 6)), (0.50390625, (5, 7)),
+                (2.5, (6, 8)), (1.5, (7, 9)), (0.498046875, (8, 10))]
+    for v, (i, j) in specials:
+        W[i, j] = bf(v) | (W[i, j] & 0x8000)
+    Wq, gamma = nm.ternary_quantize(to_dev(W))
+    _sync_ok(nm)
+    assert to_host(gamma)[0] == 1.0
+    q = to_host_u16(Wq)
+    g, oWq = oracle.ternary(W)
+    assert g == 1.0 and np.array_equal(q, oWq)
+    assert q[3, 5] == 0 and q[4, 6] == 0 and q[8, 10] == 0   # 0.5 ties to 0; below
+    assert q[5, 7] & 0x7FFF == bf(1.0)                       # just above the tie
+    assert np.count_nonzero(q) == W.size - 3
 
 
 @pytest.mark.parametrize("R,K", [(64, 256), (11008 // 8, 4096 // 4), (3, 13)])
