@@ -114,6 +114,7 @@ constexpr int PV_ROWS = 4;
 __global__ void __launch_bounds__(256)
     k_prepare_vals(const uint16_t *__restrict__ vals, int64_t R, int64_t words, int64_t Rpad, int64_t KLh,
                    bool vec, uint16_t *__restrict__ out) {
+    grid_dep_launch();  // the metadata grid may run alongside
     const int64_t r0 = (blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535) * PV_ROWS;
     const int64_t c8 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // chunk
     if (r0 >= Rpad || c8 * 8 >= KLh) return;
@@ -152,6 +153,7 @@ constexpr int PV68_JW = 4;
 __global__ void __launch_bounds__(256)
     k_prepare_vals68(const uint16_t *__restrict__ vals, int64_t R, int64_t G, int64_t Rpad, int64_t nj,
                      int64_t KLh, uint16_t *__restrict__ out) {
+    grid_dep_launch();  // the metadata grid may run alongside
     const int lane = threadIdx.x & 31;
     const int64_t r = (blockIdx.y + static_cast<int64_t>(blockIdx.z) * 65535) * 8 + (threadIdx.x >> 5);
     if (r >= Rpad) return;  // warp-uniform
@@ -201,278 +203,234 @@ __device__ __forceinline__ void block_groups(int m, int64_t kb, int64_t &g_lo, i
     }
 }
 
-// metadata: one block of 128 threads per (128-row tile mt, K' block kb).
-// (1) The block's input -- the mask words or window-metadata bytes of its
-// groups, for 128 rows -- comes into shared memory with coalesced loads (and,
-// from the mask, the pattern's window table).  (2) Thread r forms the 16
-// bytes of row mt * 128 + r (slot 2p in the low nibble of byte p): from the
-// window metadata (for the natural orders a plain copy), or, with FROM_MASK,
-// by looking each group's mask bits up in the table (the sliding-window pack
-// fused in).  Padding rows and slots get the pair (0, 1).  (3) Thread L
-// writes lane L's 16 bytes in the tensor-memory order of meta_byte_coords:
-// with L = m0 + 8 k1 + 16 m2, word k2 of the lane is half-word k1 + 2 k2 of
-// row m0 + 16 m2 (low half) and of row m0 + 16 m2 + 8 (high half).
-constexpr int PM_IN_WORDS = 13;   // >= input words of a row for any pattern (+1 pitch)
-// 2:4 from the mask: for every 4-bit group value, its nibble s0 | s1 << 2
-// (the two set bits, ascending) and whether it has exactly two bits set
-constexpr uint64_t nib24_table() {
-    uint64_t t = 0;
-    for (int b = 0; b < 16; ++b) {
-        int s[2] = {0, 0}, c = 0;
-        for (int p = 0; p < 4; ++p)
-            if ((b >> p) & 1) {
-                if (c < 2) s[c] = p;
-                ++c;
-            }
-        if (c == 2) t |= static_cast<uint64_t>(s[0] | (s[1] << 2)) << (4 * b);
-    }
-    return t;
+// 2:4 from the mask, eight groups of a mask word at once: nibble i of the
+// result is s0 | s1 << 2 for the two set bits s0 < s1 of group i (bits 4i ..
+// 4i + 3 of w); a group without exactly two set bits gets the padding pair
+// (0, 1), and sets bad if it is one of the first c (real) groups.  Per group
+// b0..b3: s0 = 0 if b0, else 1 if b1, else 2; s1 = 3 if b3, else 2 if b2,
+// else 1.
+__device__ __forceinline__ uint32_t nib24_word(uint32_t w, int c, bool &bad) {
+    constexpr uint32_t K1 = 0x11111111u;
+    const uint32_t b0 = w & K1, b1 = (w >> 1) & K1, b2 = (w >> 2) & K1, b3 = (w >> 3) & K1;
+    const uint32_t s0lo = b1 & ~b0, s0hi = K1 & ~(b0 | b1);
+    const uint32_t s1lo = b3 | (K1 & ~b2), s1hi = b3 | b2;
+    const uint32_t nib = s0lo | (s0hi << 1) | (s1lo << 2) | (s1hi << 3);
+    const uint32_t x = (b0 + b1 + b2 + b3) ^ 0x22222222u;  // per group: zero iff two bits set
+    const uint32_t z = (x | (x >> 1) | (x >> 2)) & K1;      // bit 4i: group i invalid
+    bad |= (z & (c >= 8 ? 0xFFFFFFFFu : (1u << (4 * c)) - 1u)) != 0u;
+    const uint32_t keep = (K1 & ~z) * 0xFu;
+    return (nib & keep) | (0x44444444u & ~keep);
 }
-constexpr uint32_t valid24_table() {
+
+// keeps the first c nibbles of w (0 <= c <= 8) and pads the rest with 4
+__device__ __forceinline__ uint32_t keep_nibbles(uint32_t w, int c) {
+    const uint32_t m = c >= 8 ? 0xFFFFFFFFu : (c <= 0 ? 0u : (1u << (4 * c)) - 1u);
+    return (w & m) | (0x44444444u & ~m);
+}
+
+// little-endian 32-bit word of row bytes [off, off + 4), zero past `len`
+// bytes; one aligned load when `aligned` (the row and off are 4-byte aligned
+// and the row length a multiple of 4), else byte loads
+__device__ __forceinline__ uint32_t row_word(const uint8_t *__restrict__ row, int64_t off, int64_t len,
+                                             bool aligned) {
+    if (aligned) return off + 4 <= len ? __ldg(reinterpret_cast<const uint32_t *>(row + off)) : 0u;
     uint32_t v = 0;
-    for (int b = 0; b < 16; ++b) {
-        int c = 0;
-        for (int p = 0; p < 4; ++p) c += (b >> p) & 1;
-        if (c == 2) v |= 1u << b;
-    }
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+        if (off + b < len) v |= static_cast<uint32_t>(__ldg(row + off + b)) << (8 * b);
     return v;
 }
-constexpr uint64_t kNib24 = nib24_table();
-constexpr uint32_t kValid24 = valid24_table();
-static_assert(kValid24 == 0x1668u, "2:4 group values with two bits set: 3, 5, 6, 9, 10, 12");
 
-// Stages the spans [0, n) of rows row0 .. row0 + 127 (row stride `stride`
-// elements of src) into dst[row][0 .. n): element i = t + 128 k of the
-// flattened spans is row i / n, position i % n (stepped without a division).
-// NE >= n loads per thread, in batches of B, every load of a batch issued
-// before its first store (B = NE: all of them).
-template <int NE, int B, typename E, typename D>
-__device__ __forceinline__ void stage_rows(const E *__restrict__ src, int64_t stride, int n, int64_t row0,
-                                           int64_t R, int t, D (*dst)[sizeof(D) == 1 ? PM_IN_WORDS * 4 : PM_IN_WORDS]) {
-    static_assert(NE % B == 0, "batches");
-    const int dr = BM / n, dq = BM - dr * n;
-    int r = t / n, q = t - r * n;
-#pragma unroll 1
-    for (int k0 = 0; k0 < NE; k0 += B) {
-        if (r >= BM) break;  // this thread's elements are done
-        E v[B];
-        int rr = r, qq = q;
-#pragma unroll
-        for (int k = 0; k < B; ++k) {
-            v[k] = (rr < BM && row0 + rr < R) ? __ldg(src + (row0 + rr) * stride + qq) : E(0);
-            rr += dr;
-            qq += dq;
-            if (qq >= n) {
-                qq -= n;
-                ++rr;
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < B; ++k) {
-            if (r < BM) dst[r][q] = static_cast<D>(v[k]);
-            r += dr;
-            q += dq;
-            if (q >= n) {
-                q -= n;
-                ++r;
-            }
-        }
-    }
-}
-
-// The input span of K' block kb of a row: mask words or window-metadata
-// bytes [u0, u0 + nu) for the real groups [g_lo, g_end).
-template <int M, bool FROM_MASK>
-struct MetaSpan {
-    int64_t g_lo, g_end, u0;
-    int nu;
-    __device__ __forceinline__ MetaSpan(int64_t kb, int64_t G) {
-        constexpr int NWIN = M / 2 - 1;
-        int64_t g_hi;
-        block_groups(M, kb, g_lo, g_hi);
-        g_end = g_hi < G ? g_hi : G;
-        u0 = 0;
-        int64_t u1 = 0;
-        if (g_end > g_lo) {
-            if (FROM_MASK) {
-                u0 = (g_lo * M) >> 5;
-                u1 = (g_end * M + 31) >> 5;
-            } else {
-                u0 = (g_lo * NWIN) >> 1;
-                u1 = (g_end * NWIN + 1) >> 1;
-            }
-        }
-        nu = static_cast<int>(u1 - u0);  // <= 8 words / <= 48 bytes
-    }
+// Where word k2 (slots 8 k2 .. 8 k2 + 7) of a row's 16 metadata bytes for K'
+// block kb comes from: the groups [g_lo, g_lo + ng) of the block, c of them
+// in this word (c <= 0: padding only).
+struct MetaPos {
+    int64_t kb, g_lo;
+    int ng, c;
+    bool mid;
 };
 
-// Issues the staging of one K' block's spans for rows row0 .. row0 + 127 into
-// dst (row r, word q at dst[r][q]) as asynchronous 4-byte copies, flattened
-// row after row as in stage_rows (rows at or past R get zeros); window bytes
-// that are not word-aligned are staged with plain loads instead.
+template <int M>
+__device__ __forceinline__ MetaPos meta_pos(int64_t kb, int64_t G, int k2) {
+    MetaPos p;
+    int64_t g_hi;
+    block_groups(M, kb, p.g_lo, g_hi);
+    p.kb = kb;
+    p.ng = static_cast<int>((g_hi < G ? g_hi : G) - p.g_lo);
+    p.mid = M == 8 && (kb % 3) == 2;
+    const int gpw = M == 8 ? (p.mid ? 8 : 4) : 8 / (M / 2 - 1);  // groups per output word
+    p.c = p.ng - gpw * k2;
+    return p;
+}
+
+// the input words behind word k2 of row `row` (none for a padding row or word)
 template <int M, bool FROM_MASK>
-__device__ __forceinline__ void meta_stage(const MetaSpan<M, FROM_MASK> &sp, const uint8_t *__restrict__ wmeta,
-                                           const uint32_t *__restrict__ mask, int64_t R, int64_t wbytes,
-                                           int64_t mwords, int64_t row0, int t,
-                                           uint32_t (*dst)[PM_IN_WORDS]) {
-    if (sp.nu <= 0) return;
-    const bool words4 = FROM_MASK || ((wbytes & 3) == 0 && (sp.u0 & 3) == 0 && (sp.nu & 3) == 0 &&
-                                      (reinterpret_cast<uintptr_t>(wmeta) & 3u) == 0);
-    if (!words4) {
-        stage_rows<48, 8>(wmeta + sp.u0, wbytes, sp.nu, row0, R, t,
-                          reinterpret_cast<uint8_t (*)[PM_IN_WORDS * 4]>(dst));
-        return;
-    }
-    const int n = FROM_MASK ? sp.nu : sp.nu >> 2;  // words per row
-    const uint32_t *src = FROM_MASK ? mask + sp.u0 : reinterpret_cast<const uint32_t *>(wmeta + sp.u0);
-    const int64_t stride = FROM_MASK ? mwords : wbytes >> 2;
-    const int dr = BM / n, dq = BM - dr * n;
-    int r = t / n, q = t - r * n;
-#pragma unroll
-    for (int k = 0; k < (FROM_MASK ? 8 : 12); ++k) {
-        if (r < BM) {
-            const bool real = row0 + r < R;
-            cp_async4(&dst[r][q], src + (real ? row0 + r : 0) * stride + q, real ? 4u : 0u);
+__device__ __forceinline__ void meta_fetch(const uint8_t *__restrict__ wmeta, const uint32_t *__restrict__ mask,
+                                           int64_t row, int64_t R, int64_t wbytes, int64_t mwords, bool aligned,
+                                           const MetaPos &p, int k2, uint32_t (&x)[4]) {
+    constexpr int NWIN = M / 2 - 1;
+    x[0] = x[1] = x[2] = x[3] = 0u;
+    if (row >= R || p.c <= 0) return;
+    const uint32_t *mrow = FROM_MASK ? mask + row * mwords : nullptr;
+    const uint8_t *brow = FROM_MASK ? nullptr : wmeta + row * wbytes;
+    auto mw = [&](int64_t q) -> uint32_t { return q < mwords ? __ldg(mrow + q) : 0u; };
+    if (!FROM_MASK && M != 8) {  // natural order: the word itself
+        x[0] = row_word(brow, ((p.g_lo * NWIN) >> 1) + 4 * k2, wbytes, aligned);
+    } else if (!FROM_MASK) {  // 6:8 window bytes: the run of the word's groups
+        const int64_t off = (p.g_lo * 3) / 2 + (p.mid ? 12 * k2 : 6 * k2);
+        const int64_t a = off & ~static_cast<int64_t>(3);
+        x[0] = row_word(brow, a, wbytes, aligned);
+        x[1] = row_word(brow, a + 4, wbytes, aligned);
+        if (p.mid) {  // 12 bytes from a 4-byte boundary or 2 past it
+            x[2] = row_word(brow, a + 8, wbytes, aligned);
+            x[3] = row_word(brow, a + 12, wbytes, aligned);
         }
-        r += dr;
-        q += dq;
-        if (q >= n) {
-            q -= n;
-            ++r;
-        }
+    } else if (M == 4) {
+        x[0] = mw(p.g_lo / 8 + k2);
+    } else if (M == 8) {
+        const int64_t q = p.g_lo / 4 + (p.mid ? 2 * k2 : k2);
+        x[0] = mw(q);
+        if (p.mid) x[1] = mw(q + 1);
+    } else {
+        const int64_t bit0 = p.g_lo * M + static_cast<int64_t>(8 / NWIN * M) * k2;
+        x[0] = mw(bit0 >> 5);
+        x[1] = mw((bit0 >> 5) + 1);
     }
 }
 
-// metadata: one block of 128 threads per (128-row tile mt, PM_KPB consecutive
-// K' blocks).  For each K' block kb: (1) the block's input -- the mask words
-// or window-metadata bytes of its groups, for 128 rows -- is staged in shared
-// memory by coalesced asynchronous copies, double-buffered: block kb + 1's
-// copies are in flight while kb is formed and stored.  (2) Thread r forms the
-// 16 bytes of row mt * 128 + r (slot 2p in the low nibble of byte p): from the
-// window metadata (for the natural orders a masked copy), or, with FROM_MASK,
-// by looking each group's mask bits up in the window table (the sliding-window
-// pack fused in).  Padding rows and slots get the pair (0, 1).  (3) Thread L
-// writes lane L's 16 bytes in the tensor-memory order of meta_byte_coords:
-// with L = m0 + 8 k1 + 16 m2, word k2 of the lane is half-word k1 + 2 k2 of
-// row m0 + 16 m2 (low half) and of row m0 + 16 m2 + 8 (high half).
-constexpr int PM_KPB = 4;
+// word k2 of the row from its input words x (meta_fetch): 8 slot nibbles,
+// the padding pair 4 for a padding row (x unused: R_ok false) or group
 template <int M, bool FROM_MASK>
-__global__ void __launch_bounds__(128)
-    k_prepare_meta(const uint8_t *__restrict__ wmeta, const uint32_t *__restrict__ mask, int64_t R, int64_t G,
-                   int64_t wbytes, int64_t mwords, int64_t nkb, uint8_t *__restrict__ out) {
+__device__ __forceinline__ uint32_t meta_form(const uint32_t (&x)[4], bool row_ok, const MetaPos &p, int k2,
+                                              const uint16_t *tab, bool &bad) {
     constexpr int NWIN = M / 2 - 1;
-    __shared__ uint32_t in[2][BM][PM_IN_WORDS];
-    __shared__ uint32_t rowb[BM][5];  // 16 bytes per row (+1 word pitch)
-    __shared__ uint16_t tab[M == 4 ? 1 : (1 << M)];
-    const int64_t nkc = (nkb + PM_KPB - 1) / PM_KPB;
-    const int64_t mt = blockIdx.x / nkc, kc = blockIdx.x - mt * nkc;
-    const int64_t kb0 = kc * PM_KPB, kb1 = kb0 + PM_KPB < nkb ? kb0 + PM_KPB : nkb;
-    const int t = threadIdx.x;
-    const int64_t row0 = mt * BM, row = row0 + t;
-    if (FROM_MASK && M != 4)
-        for (int i = t; i < (1 << M); i += BM) tab[i] = g_wintab.v[wt_offset(M) + i];
-    meta_stage(MetaSpan<M, FROM_MASK>(kb0, G), wmeta, mask, R, wbytes, mwords, row0, t, in[0]);
-    cp_async_commit();
-    bool bad = false;
-    for (int64_t kb = kb0; kb < kb1; ++kb) {
-        const int cur = static_cast<int>((kb - kb0) & 1);
-        if (kb + 1 < kb1) {
-            meta_stage(MetaSpan<M, FROM_MASK>(kb + 1, G), wmeta, mask, R, wbytes, mwords, row0, t, in[cur ^ 1]);
-            cp_async_commit();
-            cp_async_wait_pending<1>();  // this block's copies have landed (the next one's may not)
-        } else {
-            cp_async_wait_pending<0>();
+    if (!row_ok || p.c <= 0) return 0x44444444u;
+    if (!FROM_MASK && M != 8) return keep_nibbles(x[0], p.c * NWIN);
+    if (M == 4) return keep_nibbles(nib24_word(x[0], p.c, bad), p.c);
+    if (M == 6 || M == 10) {  // groups of 6 or 10 mask bits through the table
+        constexpr int GPW = 8 / NWIN;
+        const int64_t bit0 = p.g_lo * M + static_cast<int64_t>(GPW * M) * k2;
+        const uint32_t v = __funnelshift_r(x[0], x[1], static_cast<uint32_t>(bit0 & 31));
+        constexpr uint32_t wm = (1u << (4 * NWIN)) - 1u;
+        uint32_t W = 0x44444444u;
+#pragma unroll
+        for (int i = 0; i < GPW; ++i) {
+            if (i >= p.c) break;
+            uint32_t e = tab[(v >> (M * i)) & ((1u << M) - 1u)];
+            if (e == 0xFFFFu) {
+                bad = true;
+                e = 0x4444u;
+            }
+            const int sh = 4 * NWIN * i;
+            W = (W & ~(wm << sh)) | ((e & wm) << sh);
         }
-        __syncthreads();  // every thread's copies of block kb, the table; rowb free again
-        const MetaSpan<M, FROM_MASK> sp(kb, G);
-        const int64_t g_lo = sp.g_lo, g_end = sp.g_end;
-        const int ng = static_cast<int>(g_end - g_lo);  // real groups of the block (<= its size)
-        const bool mid = M == 8 && (kb % 3) == 2;
-        uint32_t wd[4] = {0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u};  // padding pairs
-        if (row < R && ng > 0) {
-            const uint32_t *iw = in[cur][t];
-            if (!FROM_MASK && M != 8) {
-                // natural window order: the row's nibbles as they are, padding
-                // past the last real window
-                const int nv = ng * NWIN;
+        return W;
+    }
+    // 6:8: K' blocks 0 and 1 of a triple take windows 0 and 2 of 16 groups
+    // (two slots per group), block 2 window 1 of 32 groups (one slot each)
+    const int GPW = p.mid ? 8 : 4;
+    uint32_t e[8];
+    if (FROM_MASK) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int keep = nv - 8 * q;
-                    const uint32_t m = keep >= 8 ? 0xFFFFFFFFu : (keep <= 0 ? 0u : (1u << (4 * keep)) - 1u);
-                    wd[q] = (iw[q] & m) | (0x44444444u & ~m);
-                }
-            } else {
-                // group by group; every bit and nibble position is a constant
-                // once the loop is unrolled (the mask span of an 8:10 block
-                // starts at bit 0 or 16 of its first word: shifted away first)
-                const int base = M == 10 ? static_cast<int>((g_lo * M) & 31) : 0;
-                auto mword = [&](int q) -> uint32_t {
-                    return M == 10 ? __funnelshift_r(iw[q], iw[q + 1], base) : iw[q];
-                };
-                auto innib = [&](int n) -> uint32_t { return (iw[n >> 3] >> (4 * (n & 7))) & 0xFu; };
-                auto place = [&](int slot, int width, uint32_t val) {
-                    const int sh = 4 * (slot & 7);
-                    const uint32_t msk = width == 32 ? 0xFFFFFFFFu : (((1u << width) - 1u) << sh);
-                    wd[slot >> 3] = (wd[slot >> 3] & ~msk) | ((val << sh) & msk);
-                };
-                auto group = [&](int gi) {  // gi: a constant
-                    if (gi >= ng) return;
-                    uint32_t nibs;  // window w's nibble at bits 4w
-                    if (FROM_MASK) {
-                        const int c = gi * M, q = c >> 5, off = c & 31;
-                        const uint32_t raw = off + M <= 32 ? (mword(q) >> off) : __funnelshift_r(mword(q), mword(q + 1), off);
-                        const uint32_t bits = raw & ((1u << M) - 1u);
-                        bool valid;
-                        if (M == 4) {
-                            // 2:4: survivors s0 < s1 (the set bits), nibble s0 | s1 << 2
-                            nibs = static_cast<uint32_t>(kNib24 >> (4 * bits)) & 0xFu;
-                            valid = (kValid24 >> bits) & 1u;
-                        } else {
-                            nibs = tab[bits];
-                            valid = nibs != 0xFFFFu;
-                        }
-                        if (!valid) {
-                            bad = true;
-                            nibs = 0x4444u;  // the group's slots keep the padding pair
-                        }
-                    } else {  // 6:8 window bytes: windows 0, 1, 2 of group gi are nibbles 3 gi + w
-                        nibs = innib(3 * gi) | (innib(3 * gi + 1) << 4) | (innib(3 * gi + 2) << 8);
-                    }
-                    // natural order window w at slot gi * NWIN + w; 6:8 blocks 0 and 1:
-                    // windows 0 and 2 at slots 2 gi, 2 gi + 1; block 2: window 1 at slot gi
-                    if (M == 8) {
-                        if (mid)
-                            place(gi, 4, (nibs >> 4) & 0xFu);
-                        else
-                            place(2 * gi, 8, (nibs & 0xFu) | (((nibs >> 8) & 0xFu) << 4));
-                    } else {
-                        place(gi * NWIN, 4 * NWIN, nibs);
-                    }
-                };
-                if (M == 8 && mid) {
+        for (int i = 0; i < 8; ++i) {
+            if (i >= GPW) break;
+            const uint32_t bits = ((i < 4 ? x[0] : x[1]) >> (8 * (i & 3))) & 0xFFu;
+            e[i] = i < p.c ? tab[bits] : 0x444u;
+            if (e[i] == 0xFFFFu) {
+                bad = true;
+                e[i] = 0x444u;
+            }
+        }
+    } else {
+        // window bytes: group g's windows are nibbles 3 (g - g_lo) + w of the
+        // span from byte 3 g_lo / 2; the word's run of groups starts at byte
+        // 3 GPW k2 / 2 of the span, 0 or 2 bytes into x[0]
+        const int64_t off = (p.g_lo * 3) / 2 + (p.mid ? 12 * k2 : 6 * k2);
+        const uint32_t sh = static_cast<uint32_t>(8 * (off & 3));
+        const uint32_t y0 = __funnelshift_r(x[0], x[1], sh), y1 = __funnelshift_r(x[1], x[2], sh);
+        const uint32_t y2 = __funnelshift_r(x[2], x[3], sh);
+        auto nib = [&](int n) -> uint32_t {  // nibble n of the run
+            const uint32_t y = n < 8 ? y0 : (n < 16 ? y1 : y2);
+            return (y >> (4 * (n & 7))) & 0xFu;
+        };
 #pragma unroll
-                    for (int gi = 0; gi < 32; ++gi) group(gi);
-                } else {
-                    constexpr int GPB = M == 8 ? 16 : 32 / NWIN;  // groups of a block
+        for (int i = 0; i < 8; ++i) {
+            if (i >= GPW) break;
+            e[i] = i < p.c ? (nib(3 * i) | (nib(3 * i + 1) << 4) | (nib(3 * i + 2) << 8)) : 0x444u;
+        }
+    }
+    uint32_t W = 0u;
 #pragma unroll
-                    for (int gi = 0; gi < GPB; ++gi) group(gi);
-                }
+    for (int i = 0; i < 8; ++i) {
+        if (i >= GPW) break;
+        if (p.mid)
+            W |= ((e[i] >> 4) & 0xFu) << (4 * i);
+        else
+            W |= ((e[i] & 0xFu) | (((e[i] >> 8) & 0xFu) << 4)) << (8 * i);
+    }
+    return W;
+}
+
+// metadata: 256 threads per run of PM_TILES consecutive (128-row tile, K'
+// block) tiles, a grid-stride loop over the runs.  Thread t = k2 + 4 m0 +
+// 32 m2 forms word k2 (slots 8 k2 .. 8 k2 + 7, slot 2p in the low nibble of
+// byte p) of rows A = 16 m2 + m0 and B = A + 8 of each tile straight from
+// global memory -- from the window metadata (natural orders: a masked copy),
+// or, with FROM_MASK, from the mask bits (the sliding-window pack fused in:
+// 2:4 bit-parallel, the other patterns through the window table); all the
+// run's input words are loaded before the first is used.  It writes both in
+// the tensor-memory order of meta_byte_coords: lanes A and A + 8 (k1 = 0, 1)
+// hold in word k2 the low, respectively high, half-words of A's and B's word
+// k2; a warp's two stores per tile cover 256 contiguous bytes.  Padding rows
+// and slots get the pair (0, 1).
+constexpr int PM_TILES = 4;
+template <int M, bool FROM_MASK>
+__global__ void __launch_bounds__(256)
+    k_prepare_meta(const uint8_t *__restrict__ wmeta, const uint32_t *__restrict__ mask, int64_t R, int64_t G,
+                   int64_t wbytes, int64_t mwords, int64_t nkb, int64_t ntiles, uint8_t *__restrict__ out) {
+    __shared__ uint16_t tab[M == 4 ? 1 : (1 << M)];
+    const int t = threadIdx.x;
+    if (FROM_MASK && M != 4) {
+        for (int i = t; i < (1 << M); i += blockDim.x) tab[i] = g_wintab.v[wt_offset(M) + i];
+        __syncthreads();
+    }
+    const int k2 = t & 3, m0 = (t >> 2) & 7, m2 = t >> 5;
+    const int la = m0 + 16 * m2;  // lane of k1 = 0 (and row A); k1 = 1 is la + 8 (row B)
+    const bool aligned = (wbytes & 3) == 0 && (reinterpret_cast<uintptr_t>(wmeta) & 3u) == 0;
+    const int64_t nruns = (ntiles + PM_TILES - 1) / PM_TILES;
+    bool bad = false;
+    for (int64_t run = blockIdx.x; run < nruns; run += gridDim.x) {
+        const int64_t tile0 = run * PM_TILES;
+        int64_t mt = tile0 / nkb, kb = tile0 - mt * nkb;
+        MetaPos pos[PM_TILES];
+        int64_t ra[PM_TILES];
+        uint32_t xa[PM_TILES][4], xb[PM_TILES][4];
+#pragma unroll
+        for (int j = 0; j < PM_TILES; ++j) {
+            pos[j] = meta_pos<M>(kb, G, k2);
+            ra[j] = tile0 + j < ntiles ? mt * BM + la : R;  // past the last tile: nothing to load
+            meta_fetch<M, FROM_MASK>(wmeta, mask, ra[j], R, wbytes, mwords, aligned, pos[j], k2, xa[j]);
+            meta_fetch<M, FROM_MASK>(wmeta, mask, ra[j] + 8, R, wbytes, mwords, aligned, pos[j], k2, xb[j]);
+            if (++kb == nkb) {
+                kb = 0;
+                ++mt;
             }
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) rowb[t][q] = wd[q];
-        __syncthreads();  // rowb complete; in[cur] read by every thread
-        const int m0 = t & 7, k1 = (t >> 3) & 1, m2 = t >> 4;
-        const uint16_t *h0 = reinterpret_cast<const uint16_t *>(rowb[m0 + 16 * m2]);
-        const uint16_t *h1 = reinterpret_cast<const uint16_t *>(rowb[m0 + 16 * m2 + 8]);
-        uint32_t o[4];
-#pragma unroll
-        for (int k2 = 0; k2 < 4; ++k2)
-            o[k2] = static_cast<uint32_t>(h0[k1 + 2 * k2]) | (static_cast<uint32_t>(h1[k1 + 2 * k2]) << 16);
-        *reinterpret_cast<uint4 *>(out + (mt * nkb + kb) * EBLK_BYTES + t * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+        for (int j = 0; j < PM_TILES; ++j) {
+            if (tile0 + j >= ntiles) break;
+            const uint32_t wa = meta_form<M, FROM_MASK>(xa[j], ra[j] < R, pos[j], k2, tab, bad);
+            const uint32_t wb = meta_form<M, FROM_MASK>(xb[j], ra[j] + 8 < R, pos[j], k2, tab, bad);
+            uint32_t *o = reinterpret_cast<uint32_t *>(out + (tile0 + j) * EBLK_BYTES);
+            o[la * 4 + k2] = __byte_perm(wa, wb, 0x5410);
+            o[(la + 8) * 4 + k2] = __byte_perm(wa, wb, 0x7632);
+        }
     }
     if (bad) raise_error(ERRBIT_DEVICE);
+    grid_dep_wait();  // complete only after the values grid (see launch_prepare)
 }
+
+
 
 // ---------------------------------------------------------------------------
 // Single-CTA, one-tile-per-CTA GEMM (kept as the 1-CTA baseline of the
@@ -2069,11 +2027,30 @@ nm_status launch_prepare(const uint16_t *vals, const uint8_t *wmeta, const uint3
     if (nblocks > 0x7FFFFFFF) return NM_ERR_SHAPE;
     uint8_t *meta = static_cast<uint8_t *>(packed) + p.vals_bytes;
     const int64_t mwords = (p.G * m + 31) / 32;
-    const unsigned nb = static_cast<unsigned>((p.Rpad / BM) * ((p.nkb + PM_KPB - 1) / PM_KPB));
+    const int64_t ntiles = (p.Rpad / BM) * p.nkb;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;  // 8 resident blocks of 256 threads per SM
+    const int64_t nruns = (ntiles + PM_TILES - 1) / PM_TILES;
+    const unsigned nb = static_cast<unsigned>(nruns < cap ? nruns : cap);
     const int64_t wb = (p.nwin + 1) / 2;
-#define NM_PREP_META(MM)                                                                                   \
-    (mask ? (k_prepare_meta<MM, true><<<nb, BM, 0, s>>>(nullptr, mask, R, p.G, 0, mwords, p.nkb, meta), 0) \
-          : (k_prepare_meta<MM, false><<<nb, BM, 0, s>>>(wmeta, nullptr, R, p.G, wb, 0, p.nkb, meta), 0))
+    // a programmatic dependent of the values kernel: the two grids write
+    // disjoint parts of the operand from independent inputs and overlap; the
+    // metadata kernel waits for the values grid before it completes, so the
+    // stream's next kernel sees the whole operand
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nb, 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const uint8_t *wm = mask ? nullptr : wmeta;
+    const int64_t wbm = mask ? 0 : wb, mwm = mask ? mwords : 0;
+    cudaError_t e;
+#define NM_PREP_META(MM)                                                                                \
+    e = mask ? cudaLaunchKernelEx(&cfg, k_prepare_meta<MM, true>, wm, mask, R, p.G, wbm, mwm, p.nkb, ntiles, meta) \
+             : cudaLaunchKernelEx(&cfg, k_prepare_meta<MM, false>, wm, mask, R, p.G, wbm, mwm, p.nkb, ntiles, meta)
     switch (m) {
         case 4: NM_PREP_META(4); break;
         case 6: NM_PREP_META(6); break;
@@ -2081,7 +2058,7 @@ nm_status launch_prepare(const uint16_t *vals, const uint8_t *wmeta, const uint3
         default: NM_PREP_META(10); break;
     }
 #undef NM_PREP_META
-    return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
+    return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
 }
 
 nm_status check_prepare(const uint16_t *vals, const void *meta_src, int64_t R, int64_t K, int m,
