@@ -430,6 +430,85 @@ __global__ void __launch_bounds__(256)
     grid_dep_wait();  // complete only after the values grid (see launch_prepare)
 }
 
+// 6:8 metadata from the mask, a K' block triple at a time: blocks 3j and
+// 3j + 1 hold windows 0 and 2 of groups 32j .. 32j + 15 and 32j + 16 ..
+// 32j + 31 (two slots per group), block 3j + 2 window 1 of all 32 (one slot
+// each), and one window-table entry gives a group's three windows.  So 256
+// threads per (128-row tile, triple), thread t = k2 + 4 m0 + 32 m2 looking up
+// groups 32j + 8 k2 .. + 7 of rows A = 16 m2 + m0 and A + 8 once, form
+// three words of each row: word k2 of block 3j + 2, and words 2 (k2 & 1) and
+// 2 (k2 & 1) + 1 of block 3j + (k2 >> 1).  They are written in the
+// tensor-memory order of meta_byte_coords as in k_prepare_meta.  A
+// grid-stride loop over the (tile, triple) pairs.
+__device__ __forceinline__ void meta68_row(uint32_t w0, uint32_t w1, int c, const uint16_t *tab, bool &bad,
+                                           uint32_t &mid, uint32_t &lo, uint32_t &hi) {
+    mid = 0u;
+    lo = 0u;
+    hi = 0u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        uint32_t e = 0x444u;  // a group past the last real one: padding pairs
+        if (i < c) {
+            e = tab[((i < 4 ? w0 : w1) >> (8 * (i & 3))) & 0xFFu];
+            if (e == 0xFFFFu) {
+                bad = true;
+                e = 0x444u;
+            }
+        }
+        mid |= ((e >> 4) & 0xFu) << (4 * i);
+        const uint32_t pair = (e & 0xFu) | (((e >> 8) & 0xFu) << 4);  // windows 0 and 2
+        if (i < 4)
+            lo |= pair << (8 * i);
+        else
+            hi |= pair << (8 * (i - 4));
+    }
+}
+
+__global__ void __launch_bounds__(256)
+    k_prepare_meta68(const uint32_t *__restrict__ mask, int64_t R, int64_t G, int64_t mwords, int64_t nkb,
+                     int64_t ntrip, uint8_t *__restrict__ out) {
+    __shared__ uint16_t tab[256];
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) tab[i] = g_wintab.v[wt_offset(8) + i];
+    __syncthreads();
+    const int t = threadIdx.x;
+    const int k2 = t & 3, m0 = (t >> 2) & 7, m2 = t >> 5;
+    const int la = m0 + 16 * m2;  // lane of k1 = 0 (row A); k1 = 1 is la + 8 (row B)
+    const int64_t nj = nkb / 3;
+    bool bad = false;
+    for (int64_t it = blockIdx.x; it < ntrip; it += gridDim.x) {
+        const int64_t mt = it / nj, j = it - mt * nj;
+        const int64_t g0 = 32 * j + 8 * k2;  // this thread's first group
+        const int c = static_cast<int>(G - g0 < 8 ? G - g0 : 8);  // its real groups (may be <= 0)
+        const int64_t ra = mt * BM + la, rb = ra + 8;
+        const int64_t q = g0 / 4;  // mask word of group g0 (8 bits per group)
+        uint32_t a0 = 0u, a1 = 0u, b0 = 0u, b1 = 0u;
+        if (c > 0) {
+            if (ra < R) {
+                a0 = __ldg(mask + ra * mwords + q);
+                a1 = q + 1 < mwords ? __ldg(mask + ra * mwords + q + 1) : 0u;
+            }
+            if (rb < R) {
+                b0 = __ldg(mask + rb * mwords + q);
+                b1 = q + 1 < mwords ? __ldg(mask + rb * mwords + q + 1) : 0u;
+            }
+        }
+        uint32_t ma, la0, la1, mb, lb0, lb1;
+        meta68_row(a0, a1, ra < R ? c : 0, tab, bad, ma, la0, la1);
+        meta68_row(b0, b1, rb < R ? c : 0, tab, bad, mb, lb0, lb1);
+        uint32_t *om = reinterpret_cast<uint32_t *>(out + (mt * nkb + 3 * j + 2) * EBLK_BYTES);
+        uint32_t *ot = reinterpret_cast<uint32_t *>(out + (mt * nkb + 3 * j + (k2 >> 1)) * EBLK_BYTES);
+        const int w = 2 * (k2 & 1);
+        om[la * 4 + k2] = __byte_perm(ma, mb, 0x5410);
+        om[(la + 8) * 4 + k2] = __byte_perm(ma, mb, 0x7632);
+        ot[la * 4 + w] = __byte_perm(la0, lb0, 0x5410);
+        ot[(la + 8) * 4 + w] = __byte_perm(la0, lb0, 0x7632);
+        ot[la * 4 + w + 1] = __byte_perm(la1, lb1, 0x5410);
+        ot[(la + 8) * 4 + w + 1] = __byte_perm(la1, lb1, 0x7632);
+    }
+    if (bad) raise_error(ERRBIT_DEVICE);
+    grid_dep_wait();  // complete only after the values grid (see launch_prepare)
+}
+
 
 
 // ---------------------------------------------------------------------------
@@ -2048,6 +2127,12 @@ nm_status launch_prepare(const uint16_t *vals, const uint8_t *wmeta, const uint3
     const uint8_t *wm = mask ? nullptr : wmeta;
     const int64_t wbm = mask ? 0 : wb, mwm = mask ? mwords : 0;
     cudaError_t e;
+    if (m == 8 && mask) {  // the main 6:8 path: a K' block triple per thread block
+        const int64_t ntrip = (p.Rpad / BM) * (p.nkb / 3);
+        cfg.gridDim = dim3(static_cast<unsigned>(ntrip < cap ? ntrip : cap), 1, 1);
+        e = cudaLaunchKernelEx(&cfg, k_prepare_meta68, mask, R, p.G, mwords, p.nkb, ntrip, meta);
+        return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
+    }
 #define NM_PREP_META(MM)                                                                                \
     e = mask ? cudaLaunchKernelEx(&cfg, k_prepare_meta<MM, true>, wm, mask, R, p.G, wbm, mwm, p.nkb, ntiles, meta) \
              : cudaLaunchKernelEx(&cfg, k_prepare_meta<MM, false>, wm, mask, R, p.G, wbm, mwm, p.nkb, ntiles, meta)
