@@ -1010,7 +1010,7 @@ __global__ void __launch_bounds__(128, 8)
 // grid: x = 4096-column slices (128 threads), y (+65535 z) = row blocks.
 constexpr int P24F_ROWS = 4;
 
-__global__ void __launch_bounds__(128, 4)
+__global__ void __launch_bounds__(128, 5)  // 96 registers: five blocks (33 KB of H each) per SM
     k_prune24_fused(const ScoreSrc src, const uint16_t *__restrict__ V, int64_t ldv, int64_t R,
                     int64_t K, int64_t G, uint32_t *__restrict__ mask, uint16_t *__restrict__ vals,
                     uint8_t *__restrict__ meta24) {
