@@ -107,6 +107,8 @@ int nm_version(void);
  *   ws : scratch of nm_hessian_workspace_bytes(T, K) bytes, 16-byte aligned
  *        (may be NULL when that is 0: T <= 128 or K of about 56,000 and
  *        more); at most a few MB whatever T.  Contents on return unspecified.
+ *        Unused where the token ranges of a column strip are combined inside
+ *        a thread-block cluster (when every cluster fits on the device).
  *   Errors: NULL X or H -> NM_ERR_NULL; T, K < 1, ldx < K, T too large ->
  *   NM_ERR_SHAPE; alignment -> NM_ERR_ALIGN; short ws -> NM_ERR_WORKSPACE.  */
 #define NM_HESSIAN_MAX_TOKENS 2147483647ll
@@ -139,6 +141,10 @@ nm_status nm_hessian_diag(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, 
  *   device's current context: after cudaDeviceReset the library must be
  *   unloaded and loaded again before this entry point is used.  It calls no
  *   cudaMalloc, cudaFree or other allocating routine.
+ *   Where a column strip's token ranges fit on the device as one
+ *   thread-block cluster each (so on a B200), their partial sums are
+ *   combined in the clusters' shared memory and the array is not used; it
+ *   serves devices where they do not fit.
  *   Sharing: all calls on a device share the one array and it keeps the last
  *   call's contents (every pair is written before it is read, so nothing
  *   needs clearing).  Calls whose kernels may overlap on the GPU -- on

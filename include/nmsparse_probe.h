@@ -72,6 +72,15 @@ nm_status nm_sparse_gemm_tile256(const uint16_t *X, int64_t T, int64_t K, int64_
 nm_status nm_test_set_wait_limit_ns(unsigned long long ns);
 nm_status nm_test_withhold_stream_k_flag(int cluster);
 
+/* Path control for the H reduction.  With several token ranges per column
+ * strip, nm_hessian_diag combines a strip's ranges inside one thread-block
+ * cluster (distributed shared memory) when every cluster fits on the device
+ * at once, and otherwise through the workspace pairs and a second kernel.
+ * on = 0 forces the second path (to test it on a device where clusters fit),
+ * on = 1 restores the automatic choice.  A host setting, not thread-safe
+ * against concurrent calls; not for production use.                        */
+nm_status nm_test_hessian_clusters(int on);
+
 #ifdef __cplusplus
 }
 #endif

@@ -337,6 +337,13 @@ __device__ __forceinline__ uint32_t mapa_shared(const void *p, uint32_t rank) {
     return out;
 }
 
+// fp64 load from another CTA's shared memory (a shared::cluster address)
+__device__ __forceinline__ double ld_dsmem_f64(uint32_t cluster_addr) {
+    double v;
+    asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(cluster_addr) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                      : "memory");

@@ -11,6 +11,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "nm_common.cuh"
@@ -281,7 +282,7 @@ __device__ __noinline__ RunSplit sq_run_split(const uint16_t *col) {
 
 __global__ void __launch_bounds__(HX_THREADS, 2)
     k_hsq(const __grid_constant__ CUtensorMap tmX, const uint16_t *__restrict__ X, int64_t T, int64_t K,
-          int64_t ldx, HPair *__restrict__ part, double *__restrict__ H) {
+          int64_t ldx, HPair *__restrict__ part, double *__restrict__ H, int ccomb) {
     extern __shared__ uint8_t hx_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(hx_smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
@@ -351,43 +352,90 @@ __global__ void __launch_bounds__(HX_THREADS, 2)
         if (threadIdx.x == 0)
             for (int64_t j = i; j < issued; ++j)
                 mbar_wait(&full[j % HX_STAGES], static_cast<uint32_t>((j / HX_STAGES) & 1));
-        return;
+        if (!ccomb) return;  // a cluster member still meets its peers at the barriers
+        __syncthreads();
     }
-    // the pipeline is drained: stage memory holds the warps' pairs
-    double(*sh_s)[HX_COLS] = reinterpret_cast<double(*)[HX_COLS]>(smem);
-    double(*sh_cu)[HX_COLS] = reinterpret_cast<double(*)[HX_COLS]>(smem + HX_WARPS * HX_COLS * 8);
-    double(*sh_cd)[HX_COLS] = reinterpret_cast<double(*)[HX_COLS]>(smem + 2 * HX_WARPS * HX_COLS * 8);
-    uint8_t(*sh_bad)[HX_COLS] = reinterpret_cast<uint8_t(*)[HX_COLS]>(smem + 3 * HX_WARPS * HX_COLS * 8);
-#pragma unroll
-    for (int k = 0; k < HX_VEC; ++k) {
-        sh_s[warp][HX_VEC * lane + k] = s[k];
-        sh_cu[warp][HX_VEC * lane + k] = cu[k];
-        sh_cd[warp][HX_VEC * lane + k] = cd[k];
-        sh_bad[warp][HX_VEC * lane + k] = static_cast<uint8_t>((bad >> k) & 1u);
-    }
-    __syncthreads();
     const int j = threadIdx.x;
     const int64_t col = static_cast<int64_t>(xcol) + j;
-    if (j >= HX_COLS || col >= K) return;
-    double S = 0.0, CU = 0.0, CD = 0.0;
-    bool marked = false;
+    const bool owner = j < HX_COLS && col < K;  // thread j finishes column col
+    // cluster combine: this block's exact pair per column, for rank 0 to read
+    double *res_s = reinterpret_cast<double *>(smem + HX_TILE_BYTES);
+    double *res_c = res_s + HX_COLS;
+    if (ok) {
+        // the pipeline is drained: stage memory holds the warps' pairs
+        double(*sh_s)[HX_COLS] = reinterpret_cast<double(*)[HX_COLS]>(smem);
+        double(*sh_cu)[HX_COLS] = reinterpret_cast<double(*)[HX_COLS]>(smem + HX_WARPS * HX_COLS * 8);
+        double(*sh_cd)[HX_COLS] = reinterpret_cast<double(*)[HX_COLS]>(smem + 2 * HX_WARPS * HX_COLS * 8);
+        uint8_t(*sh_bad)[HX_COLS] = reinterpret_cast<uint8_t(*)[HX_COLS]>(smem + 3 * HX_WARPS * HX_COLS * 8);
 #pragma unroll
-    for (int w = 0; w < HX_WARPS; ++w) {
-        two_sum_acc2(S, CU, CD, sh_s[w][j]);
-        CU = __dadd_ru(CU, sh_cu[w][j]);
-        CD = __dadd_rd(CD, sh_cd[w][j]);
-        marked |= sh_bad[w][j] != 0;
+        for (int k = 0; k < HX_VEC; ++k) {
+            sh_s[warp][HX_VEC * lane + k] = s[k];
+            sh_cu[warp][HX_VEC * lane + k] = cu[k];
+            sh_cd[warp][HX_VEC * lane + k] = cd[k];
+            sh_bad[warp][HX_VEC * lane + k] = static_cast<uint8_t>((bad >> k) & 1u);
+        }
+        __syncthreads();
+        if (owner) {
+            double S = 0.0, CU = 0.0, CD = 0.0;
+            bool marked = false;
+#pragma unroll
+            for (int w = 0; w < HX_WARPS; ++w) {
+                two_sum_acc2(S, CU, CD, sh_s[w][j]);
+                CU = __dadd_ru(CU, sh_cu[w][j]);
+                CD = __dadd_rd(CD, sh_cd[w][j]);
+                marked |= sh_bad[w][j] != 0;
+            }
+            marked |= CU != CD;  // c not exact: its up and down sums differ (fact 2)
+            if (ccomb) {
+                res_s[j] = marked ? __longlong_as_double(0x7FF8000000000000ll) : S;
+                res_c[j] = marked ? 0.0 : CU;
+            } else if (part == nullptr) {  // the block saw every token
+                const double sum = marked ? exact_sq_column(X, ldx, T, col) : __dadd_rn(S, CU);
+                H[col] = __ddiv_rn(sum, static_cast<double>(T));
+            } else {
+                HPair p;
+                p.s = marked ? __longlong_as_double(0x7FF8000000000000ll) : S;
+                p.c = marked ? 0.0 : CU;
+                part[static_cast<int64_t>(blockIdx.y) * K + col] = p;
+            }
+        }
     }
-    marked |= CU != CD;  // c not exact: its up and down sums differ (fact 2)
-    if (H != nullptr) {  // the block saw every token
-        const double sum = marked ? exact_sq_column(X, ldx, T, col) : __dadd_rn(S, CU);
+    if (!ccomb) return;
+    __syncwarp();  // the cluster barrier wants converged warps
+    // the token ranges of the strip are one cluster: rank 0 adds the members'
+    // pairs from their shared memory as k_hsq_finish adds them from global
+    // memory; the second barrier keeps every member resident until then
+    cluster_sync_all();
+    if (ok && owner && cluster_ctarank() == 0) {
+        const int nr = static_cast<int>(gridDim.y);
+        double S = 0.0, CU = 0.0, CD = 0.0;
+        bool marked = false;
+        for (int r = 0; r < nr; ++r) {
+            const double ps = ld_dsmem_f64(mapa_shared(res_s + j, static_cast<uint32_t>(r)));
+            const double pc = ld_dsmem_f64(mapa_shared(res_c + j, static_cast<uint32_t>(r)));
+            marked |= isnan(ps);
+            two_sum_acc2(S, CU, CD, ps);
+            CU = __dadd_ru(CU, pc);
+            CD = __dadd_rd(CD, pc);
+        }
+        double sum;
+        if (marked) {
+            sum = exact_sq_column(X, ldx, T, col);
+        } else if (CU == CD) {
+            sum = __dadd_rn(S, CU);
+        } else {
+            SqAcc acc;
+            acc.clear();
+            for (int r = 0; r < nr; ++r) {
+                acc.add_double(ld_dsmem_f64(mapa_shared(res_s + j, static_cast<uint32_t>(r))));
+                acc.add_double(ld_dsmem_f64(mapa_shared(res_c + j, static_cast<uint32_t>(r))));
+            }
+            sum = acc.round_rn();
+        }
         H[col] = __ddiv_rn(sum, static_cast<double>(T));
-    } else {
-        HPair p;
-        p.s = marked ? __longlong_as_double(0x7FF8000000000000ll) : S;
-        p.c = marked ? 0.0 : CU;
-        part[static_cast<int64_t>(blockIdx.y) * K + col] = p;
     }
+    __syncwarp();
+    cluster_sync_all();
 }
 
 // adds the blocks' exact pairs of a column -- with TwoSum, c up and down as
@@ -1483,6 +1531,36 @@ namespace {
 // partial pairs into `part`, then the finish as a programmatic dependent so
 // that its launch overlaps the main kernel.  `max_split` caps the number of
 // token ranges (the pairs `part` can hold are max_split * K).
+// clusters of k_hsq with `split` blocks that the current device holds at
+// once (0 on an error), cached per device and cluster size
+std::atomic<int> g_hsq_clusters{1};  // 0: the workspace path only (test control)
+
+int hsq_active_clusters(int64_t cblocks, int64_t split) {
+    static int cache[64][9] = {};
+    int dev = 0;
+    if (split < 2 || split > 8 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (cache[dev][split] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(cblocks), static_cast<unsigned>(split), 1);
+        cfg.blockDim = dim3(HX_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = HX_SMEM_BYTES;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = 1;
+        at[0].val.clusterDim.y = static_cast<unsigned>(split);
+        at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, k_hsq, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            return 0;
+        }
+        cache[dev][split] = n > 0 ? n : -1;
+    }
+    return cache[dev][split] > 0 ? cache[dev][split] : 0;
+}
+
 nm_status launch_hsq(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, double *H, HPair *part,
                      int64_t max_split, cudaStream_t s) {
     using namespace nm;
@@ -1493,10 +1571,31 @@ nm_status launch_hsq(const uint16_t *X, int64_t T, int64_t K, int64_t ldx, doubl
     if (!set_smem_attr<k_hsq>(HX_SMEM_BYTES)) return NM_ERR_CUDA;
     const dim3 grid(static_cast<unsigned>(g.cblocks), static_cast<unsigned>(g.split));
     if (g.split == 1) {
-        k_hsq<<<grid, HX_THREADS, HX_SMEM_BYTES, s>>>(tm, X, T, K, ldx, nullptr, H);
+        k_hsq<<<grid, HX_THREADS, HX_SMEM_BYTES, s>>>(tm, X, T, K, ldx, nullptr, H, 0);
         return launch_status();
     }
-    k_hsq<<<grid, HX_THREADS, HX_SMEM_BYTES, s>>>(tm, X, T, K, ldx, part, nullptr);
+    // several token ranges: as one cluster per strip (at most 8 ranges),
+    // combined in distributed shared memory, when every cluster is resident
+    // at once; otherwise through the workspace pairs and k_hsq_finish
+    const HGrid gc = h_grid(T, K, max_split < 8 ? max_split : 8);
+    if (gc.split > 1 && g_hsq_clusters.load() != 0 && hsq_active_clusters(gc.cblocks, gc.split) >= gc.cblocks) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(gc.cblocks), static_cast<unsigned>(gc.split), 1);
+        cfg.blockDim = dim3(HX_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = HX_SMEM_BYTES;
+        cfg.stream = s;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = 1;
+        at[0].val.clusterDim.y = static_cast<unsigned>(gc.split);
+        at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, k_hsq, tm, X, T, K, ldx, static_cast<HPair *>(nullptr), H, 1) != cudaSuccess)
+            return NM_ERR_CUDA;
+        return launch_status();
+    }
+    k_hsq<<<grid, HX_THREADS, HX_SMEM_BYTES, s>>>(tm, X, T, K, ldx, part, nullptr, 0);
     if (cudaGetLastError() != cudaSuccess) return NM_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>((K + 127) / 128), 1, 1);
@@ -1523,6 +1622,12 @@ nm_status check_hessian_args(const uint16_t *X, int64_t T, int64_t K, int64_t ld
 }
 
 }  // namespace
+
+extern "C" nm_status nm_test_hessian_clusters(int on) {
+    if (on != 0 && on != 1) return NM_ERR_SHAPE;
+    g_hsq_clusters.store(on);
+    return NM_OK;
+}
 
 extern "C" size_t nm_hessian_workspace_bytes(int64_t T, int64_t K) {
     if (T <= 0 || K <= 0) return 0;

@@ -31,20 +31,31 @@ def _sync_ok(nm):
 
 
 # ---------------------------------------------------------------- a1 / a2
+@pytest.fixture(params=["clusters", "workspace"])
+def h_path(request, nm):
+    # nm_hessian_diag combines a strip's token ranges inside a thread-block
+    # cluster when the clusters fit on the device, else through the workspace
+    # pairs and a second kernel; both paths must give the same H
+    lib = nm.load()
+    assert lib.nm_test_hessian_clusters(1 if request.param == "clusters" else 0) == 0
+    yield request.param
+    assert lib.nm_test_hessian_clusters(1) == 0
+
+
 # one chunk; ragged runs; one column; a block with several chunks in its
 # three-tile pipeline (K = 40000: more column blocks than SMs, so one split);
 # 65 chunks over the SM-sized split of a 4096-column layer
 @pytest.mark.parametrize("T,K,ld", [(128, 512, 512), (1000, 520, 520), (1, 7, 8), (129, 3, 8),
                                     (2048, 4096, 4096), (300, 517, 528), (257, 96, 104),
                                     (1000, 40000, 40000), (8292, 4096, 4104)])
-def test_hessian_bitexact(nm, T, K, ld):
+def test_hessian_bitexact(nm, h_path, T, K, ld):
     X = datagen.make_activations(T, K, seed=T + K, n_outliers=min(4, K))
     H = nm.hessian_diag(to_dev(X, ld))
     _sync_ok(nm)
     assert np.array_equal(to_host(H), oracle.hessian_diag(X))
 
 
-def test_hessian_special_values_bitexact(nm):
+def test_hessian_special_values_bitexact(nm, h_path):
     # zeros of both signs, bf16 subnormals, the smallest and largest normals
     # and infinities, in even and odd columns: every class of value whose
     # square the reduction must form exactly, against the oracle's fp64
@@ -73,7 +84,7 @@ def test_hessian_special_values_bitexact(nm):
 
 
 @pytest.mark.parametrize("T", [300, 5000])
-def test_hessian_exact_rounding_paths(nm, T):
+def test_hessian_exact_rounding_paths(nm, h_path, T):
     # columns that need each path of the exact sum, against the oracle:
     #  0: the tie 2^52 + 2^52 + 1 (rounds to even) and 1: the same broken up by
     #     the square of the smallest subnormal (the integer path);
