@@ -325,7 +325,7 @@ def run_ours(args):
         if layer.score == "hessian":
             chk(lib.nm_hessian_diag(Xs.data_ptr(), T, K, K, H.data_ptr(), ws.data_ptr(), ws.numel(), s),
                 "hessian")
-            cnt += 2 if ws_needed else 1  # H (+ the finish that adds the blocks' exact pairs)
+            cnt += lib.nm_hessian_launch_count(T, K)  # H (+ a finish kernel where clusters do not fit)
         if ev is not None:
             ev[1].record(stream)
         # a2 + a3 in one pass: scores formed in registers, never written

@@ -81,6 +81,12 @@ nm_status nm_test_withhold_stream_k_flag(int cluster);
  * against concurrent calls; not for production use.                        */
 nm_status nm_test_hessian_clusters(int on);
 
+/* How many kernels nm_hessian_diag(X of T x K) launches on the current device
+ * with the current path setting: 1 (one token range, or the ranges combined
+ * inside clusters) or 2 (the workspace path's second kernel); 0 for T or
+ * K < 1.  A query for launch accounting; launches nothing.                  */
+int nm_hessian_launch_count(int64_t T, int64_t K);
+
 #ifdef __cplusplus
 }
 #endif

@@ -36,7 +36,7 @@ EXPORTED = (
     "nm_sparse_gemm_tile256", "nm_score_prune_compress", "nm_hessian_rescale",
     "nm_hutchinson_workspace_bytes", "nm_hutchinson_diag", "nm_lifted_cols_f8", "nm_sparse_prepare_f8_bytes",
     "nm_quant_lift_f8", "nm_sparse_prepare_f8", "nm_sparse_gemm_f8", "nm_test_set_wait_limit_ns",
-    "nm_test_withhold_stream_k_flag", "nm_test_hessian_clusters", "nm_sparse_prepare_from_mask",
+    "nm_test_withhold_stream_k_flag", "nm_test_hessian_clusters", "nm_hessian_launch_count", "nm_sparse_prepare_from_mask",
 )
 
 _P, _I64, _I, _D, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_size_t
@@ -79,6 +79,7 @@ _SIGS = {
     "nm_sparse_prepare_from_mask": (_I, [_P, _P, _I64, _I64, _I, _P, _SZ, _P]),
     "nm_test_withhold_stream_k_flag": (_I, [_I]),
     "nm_test_hessian_clusters": (_I, [_I]),
+    "nm_hessian_launch_count": (_I, [_I64, _I64]),
 }
 
 _lock = threading.Lock()

@@ -1629,6 +1629,15 @@ extern "C" nm_status nm_test_hessian_clusters(int on) {
     return NM_OK;
 }
 
+extern "C" int nm_hessian_launch_count(int64_t T, int64_t K) {
+    if (T <= 0 || K <= 0) return 0;
+    if (h_grid(T, K, INT64_MAX).split <= 1) return 1;
+    const HGrid gc = h_grid(T, K, 8);
+    if (gc.split > 1 && g_hsq_clusters.load() != 0 && hsq_active_clusters(gc.cblocks, gc.split) >= gc.cblocks)
+        return 1;
+    return 2;
+}
+
 extern "C" size_t nm_hessian_workspace_bytes(int64_t T, int64_t K) {
     if (T <= 0 || K <= 0) return 0;
     const HGrid g = h_grid(T, K, INT64_MAX);

@@ -55,6 +55,21 @@ def test_hessian_bitexact(nm, h_path, T, K, ld):
     assert np.array_equal(to_host(H), oracle.hessian_diag(X))
 
 
+def test_hessian_launch_count(nm):
+    # the launch accounting of the bench: one kernel for one token range or
+    # for ranges combined inside clusters (they fit on a B200), two on the
+    # workspace path
+    lib = nm.load()
+    assert lib.nm_hessian_launch_count(128, 4096) == 1
+    assert lib.nm_hessian_launch_count(8192, 4096) == 1
+    assert lib.nm_test_hessian_clusters(0) == 0
+    try:
+        assert lib.nm_hessian_launch_count(8192, 4096) == 2
+        assert lib.nm_hessian_launch_count(128, 4096) == 1
+    finally:
+        assert lib.nm_test_hessian_clusters(1) == 0
+
+
 def test_hessian_special_values_bitexact(nm, h_path):
     # zeros of both signs, bf16 subnormals, the smallest and largest normals
     # and infinities, in even and odd columns: every class of value whose
