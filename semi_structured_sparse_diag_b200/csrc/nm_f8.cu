@@ -40,9 +40,9 @@ constexpr int F8_B_BYTES = F8_BN * 256;                     // 32 KB
 constexpr int F8_E_BYTES = 4096;                            // two 2 KB atoms
 constexpr int F8_STAGE_BYTES = F8_A_BYTES + F8_B_BYTES + F8_E_BYTES;
 constexpr int F8_SMEM_BYTES = F8_STAGES * F8_STAGE_BYTES + 1024 + 256;
-constexpr int F8_TMEM_COLS = 256;                           // accumulator 128 + metadata 8
+constexpr int F8_TMEM_COLS = 512;                           // two accumulators of 128 + metadata 8
+constexpr int F8_TMEM_E = 2 * F8_BN;                        // metadata columns
 static_assert(F8_STAGE_BYTES % 1024 == 0, "stage alignment");
-static_assert(F8_BN * F8_BM * 2 <= F8_STAGES * F8_STAGE_BYTES, "epilogue staging");
 
 // two fp32 values -> two E4M3 codes (round to nearest even, saturating); the
 // first argument lands in the low byte
@@ -182,22 +182,27 @@ __host__ __device__ constexpr uint32_t make_idesc_f8_sp(uint32_t M, uint32_t N) 
     return (1u << 2) | (1u << 4) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
-// Warp roles: 0 = TMA producer, 1 = MMA issuer + tensor-memory owner,
-// 4..7 = epilogue (tensor memory -> scaled bf16 -> TMA store).
+// Persistent: one CTA per SM walks the (128-row, 128-token) tiles, weight-row
+// tiles fastest (consecutive CTAs share a token tile in L2).  Warp roles: 0 =
+// TMA producer (its stage ring runs on across tiles), 1 = MMA issuer +
+// tensor-memory owner, 4..7 = epilogue.  Two accumulators of 128 columns
+// alternate between tiles, so the epilogue of one tile (tensor memory ->
+// scaled bf16, stored from registers: 32 consecutive weight rows of one token
+// per warp instruction) overlaps the next tile's main loop.
 __global__ void __launch_bounds__(F8_THREADS, 1)
     k_gemm_f8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              const __grid_constant__ CUtensorMap tmY, const uint8_t *__restrict__ meta, int64_t nkb,
-              const float *__restrict__ xs, const float *__restrict__ ws, int64_t T) {
+              const uint8_t *__restrict__ meta, int64_t nkb, const float *__restrict__ xs,
+              const float *__restrict__ ws, int64_t T, int64_t R, int64_t n_m, int64_t ntiles,
+              uint16_t *__restrict__ Y, int64_t ldy) {
     constexpr int S = F8_STAGES;
     extern __shared__ __align__(1024) uint8_t f8_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(f8_smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S * F8_STAGE_BYTES);
-    uint64_t *full = bars, *empty = bars + S, *accum = bars + 2 * S;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum + 1);
+    uint64_t *full = bars, *empty = bars + S, *acc_full = bars + 2 * S, *acc_empty = bars + 2 * S + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 4);
     volatile uint32_t *abort_flag = tmem_slot + 1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int mt = blockIdx.x, nt = blockIdx.y;
     auto stA = [&](int s) { return smem + s * F8_STAGE_BYTES; };
     auto stB = [&](int s) { return smem + s * F8_STAGE_BYTES + F8_A_BYTES; };
     auto stE = [&](int s) { return smem + s * F8_STAGE_BYTES + F8_A_BYTES + F8_B_BYTES; };
@@ -207,12 +212,14 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(accum, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);  // the four epilogue warps
+        }
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
-        prefetch_tmap(&tmY);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, F8_TMEM_COLS);
@@ -222,75 +229,91 @@ __global__ void __launch_bounds__(F8_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const uint32_t tmem_e = tmem_base + F8_BN;
+    const uint32_t tmem_e = tmem_base + F8_TMEM_E;
 
     if (warp == 0) {
         if (lane == 0) {
-            int64_t kb = 0;
-            for (; kb < nkb; ++kb) {
-                const int s = static_cast<int>(kb % S);
-                const uint32_t ph = static_cast<uint32_t>((kb / S) & 1);
-                if (kb >= S && !mbar_wait(&empty[s], ph ^ 1u)) { *abort_flag = 1; break; }
-                mbar_arrive_expect_tx(&full[s], F8_STAGE_BYTES);
-                tma_load_2d(stA(s), &tmA, &full[s], static_cast<int32_t>(kb * 128), mt * F8_BM);
-                tma_load_2d(stB(s), &tmB, &full[s], static_cast<int32_t>(kb * F8_KB), nt * F8_BN);
-                tma_load_2d(stB(s) + F8_BN * 128, &tmB, &full[s], static_cast<int32_t>(kb * F8_KB + 128), nt * F8_BN);
-                bulk_load(stE(s), meta + (static_cast<int64_t>(mt) * nkb + kb) * F8_E_BYTES, F8_E_BYTES, &full[s]);
+            int64_t it = 0;
+            for (int64_t tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
+                const int64_t mt = tile % n_m, nt = tile / n_m;
+                for (int64_t kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = static_cast<int>(it % S);
+                    const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
+                    if (it >= S && !mbar_wait(&empty[s], ph ^ 1u)) { *abort_flag = 1; break; }
+                    mbar_arrive_expect_tx(&full[s], F8_STAGE_BYTES);
+                    tma_load_2d(stA(s), &tmA, &full[s], static_cast<int32_t>(kb * 128), static_cast<int32_t>(mt * F8_BM));
+                    tma_load_2d(stB(s), &tmB, &full[s], static_cast<int32_t>(kb * F8_KB), static_cast<int32_t>(nt * F8_BN));
+                    tma_load_2d(stB(s) + F8_BN * 128, &tmB, &full[s], static_cast<int32_t>(kb * F8_KB + 128),
+                                static_cast<int32_t>(nt * F8_BN));
+                    bulk_load(stE(s), meta + (mt * nkb + kb) * F8_E_BYTES, F8_E_BYTES, &full[s]);
+                }
             }
             if (*abort_flag)  // let the copies already issued land
-                for (int64_t j = (kb > S ? kb - S : 0); j < kb; ++j)
+                for (int64_t j = (it > S ? it - S : 0); j < it; ++j)
                     mbar_wait(&full[j % S], static_cast<uint32_t>((j / S) & 1));
         }
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc = make_idesc_f8_sp(F8_BM, F8_BN);
             bool ok = true;
-            for (int64_t kb = 0; kb < nkb && ok; ++kb) {
-                const int s = static_cast<int>(kb % S);
-                if (!mbar_wait(&full[s], static_cast<uint32_t>((kb / S) & 1))) { ok = false; break; }
-                tc_fence_after();
-                tmem_cp_128x128b(tmem_e, make_sdesc(smem_u32(stE(s)), 2048, 128, 0));
-                tmem_cp_128x128b(tmem_e + 4, make_sdesc(smem_u32(stE(s) + 2048), 2048, 128, 0));
-                const uint32_t a0 = smem_u32(stA(s)), b0 = smem_u32(stB(s));
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint64_t ad = make_sdesc(a0 + j * 32, 16, 1024, 2);
-                    const uint64_t bd = make_sdesc(b0 + (j >> 1) * (F8_BN * 128) + (j & 1) * 64, 16, 1024, 2);
-                    mma_sp_f8(tmem_base, ad, bd, tmem_e + 2 * j, idesc, (kb > 0 || j > 0) ? 1u : 0u);
+            int64_t it = 0, ti = 0;
+            for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++ti) {
+                const int buf = static_cast<int>(ti & 1);
+                if (ti >= 2 && !mbar_wait(&acc_empty[buf], static_cast<uint32_t>(((ti >> 1) - 1) & 1))) {
+                    ok = false;
+                    break;
                 }
-                mma_commit(&empty[s]);
+                tc_fence_after();
+                const uint32_t d = tmem_base + static_cast<uint32_t>(buf * F8_BN);
+                for (int64_t kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = static_cast<int>(it % S);
+                    if (!mbar_wait(&full[s], static_cast<uint32_t>((it / S) & 1))) { ok = false; break; }
+                    tc_fence_after();
+                    tmem_cp_128x128b(tmem_e, make_sdesc(smem_u32(stE(s)), 2048, 128, 0));
+                    tmem_cp_128x128b(tmem_e + 4, make_sdesc(smem_u32(stE(s) + 2048), 2048, 128, 0));
+                    const uint32_t a0 = smem_u32(stA(s)), b0 = smem_u32(stB(s));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint64_t ad = make_sdesc(a0 + j * 32, 16, 1024, 2);
+                        const uint64_t bd = make_sdesc(b0 + (j >> 1) * (F8_BN * 128) + (j & 1) * 64, 16, 1024, 2);
+                        mma_sp_f8(d, ad, bd, tmem_e + 2 * j, idesc, (kb > 0 || j > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&empty[s]);
+                }
+                if (ok) mma_commit(&acc_full[buf]);
             }
-            if (ok) mma_commit(accum);
-            else *abort_flag = 1;
+            if (!ok) *abort_flag = 1;
         }
     } else if (warp >= 4) {
         const int ew = warp - 4;
-        bool ok = __all_sync(0xffffffffu, mbar_wait(accum, 0));
-        if (ok) {
+        int64_t ti = 0;
+        for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++ti) {
+            const int buf = static_cast<int>(ti & 1);
+            if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], static_cast<uint32_t>((ti >> 1) & 1)))) break;
             tc_fence_after();
-            const float wsr = ws[mt * F8_BM + ew * 32 + lane];  // ws holds Rpad entries
-            uint16_t *stage_out = reinterpret_cast<uint16_t *>(smem) + ew * (F8_BN * 32);  // [BN][32]
+            const int64_t mt = tile % n_m, nt = tile / n_m;
+            const int64_t r = mt * F8_BM + ew * 32 + lane;  // this lane's weight row
+            const float wsr = ws[r];                          // ws holds Rpad entries
+            const uint32_t src = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + static_cast<uint32_t>(buf * F8_BN);
 #pragma unroll 1
             for (int cc = 0; cc < F8_BN / 32; ++cc) {
                 uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + cc * 32, v);
+                tmem_ld_32x32b_x32(src + cc * 32, v);
                 tmem_ld_wait();
+                if (cc == F8_BN / 32 - 1) {  // the accumulator is in registers: hand it back
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&acc_empty[buf]);
+                }
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    const int64_t t = static_cast<int64_t>(nt) * F8_BN + cc * 32 + j;
-                    const float xt = t < T ? __ldg(xs + t) : 0.0f;
-                    const float y = __fmul_rn(__uint_as_float(v[j]), __fmul_rn(wsr, xt));
-                    stage_out[(cc * 32 + j) * 32 + lane] = static_cast<uint16_t>(pack_bf16x2(y, 0.0f) & 0xFFFFu);
+                    const int64_t t = nt * F8_BN + cc * 32 + j;
+                    if (t < T) {
+                        const float y = __fmul_rn(__uint_as_float(v[j]), __fmul_rn(wsr, __ldg(xs + t)));
+                        if (r < R) Y[t * ldy + r] = static_cast<uint16_t>(pack_bf16x2(y, 0.0f) & 0xFFFFu);
+                    }
                 }
             }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                tma_store_2d(&tmY, stage_out, mt * F8_BM + ew * 32, nt * F8_BN);
-                bulk_commit_group();
-                bulk_wait_group_read0();
-            }
-            __syncwarp();
         }
     }
     tc_fence_before();
@@ -379,6 +402,15 @@ extern "C" nm_status nm_sparse_prepare_f8(const uint16_t *vals, const uint8_t *w
     return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
 }
 
+// SMs of the current device (148 if the query fails)
+static int f8_sm_count() {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+        return 148;
+    return v;
+}
+
 extern "C" nm_status nm_sparse_gemm_f8(const uint8_t *Xq, int64_t T, int64_t K, int64_t ldq, const float *xscale,
                                        const void *packed, int64_t R, int m, uint16_t *Y, int64_t ldy,
                                        void *stream) {
@@ -392,16 +424,17 @@ extern "C" nm_status nm_sparse_gemm_f8(const uint8_t *Xq, int64_t T, int64_t K, 
         (reinterpret_cast<uintptr_t>(xscale) & 3u))
         return NM_ERR_ALIGN;
     const uint8_t *p = static_cast<const uint8_t *>(packed);
-    CUtensorMap ta, tb, ty;
+    CUtensorMap ta, tb;
     if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p, g.Rpad, g.KLf / 2, g.KLf / 2, 128, F8_BM, true) ||
-        !make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Xq, T, g.KLf, ldq, 128, F8_BN, true) ||
-        !make_tmap_bf16(&ty, Y, T, R, ldy, 32, F8_BN, false))
+        !make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Xq, T, g.KLf, ldq, 128, F8_BN, true))
         return NM_ERR_CUDA;
     if (!set_smem_attr<k_gemm_f8>(F8_SMEM_BYTES)) return NM_ERR_CUDA;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    dim3 grid(static_cast<unsigned>(g.Rpad / F8_BM), static_cast<unsigned>((T + F8_BN - 1) / F8_BN));
+    const int64_t n_m = g.Rpad / F8_BM, ntiles = n_m * ((T + F8_BN - 1) / F8_BN);
+    const int64_t nsm = f8_sm_count();
+    const unsigned grid = static_cast<unsigned>(ntiles < nsm ? ntiles : nsm);
     k_gemm_f8<<<grid, F8_THREADS, F8_SMEM_BYTES, st>>>(
-        ta, tb, ty, p + g.vals_bytes, g.nkb, xscale,
-        reinterpret_cast<const float *>(p + g.vals_bytes + g.meta_bytes), T);
+        ta, tb, p + g.vals_bytes, g.nkb, xscale, reinterpret_cast<const float *>(p + g.vals_bytes + g.meta_bytes),
+        T, R, n_m, ntiles, Y, ldy);
     return cudaGetLastError() == cudaSuccess ? NM_OK : NM_ERR_CUDA;
 }
