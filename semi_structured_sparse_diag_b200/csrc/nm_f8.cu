@@ -99,6 +99,22 @@ __global__ void __launch_bounds__(F8Q_THREADS, 12) k_quant_lift_f8(const uint16_
         uint8_t *qrow = Q + t * ldq;
         const int per = 2 * m - 4;  // lifted columns per group
         for (int64_t c0 = 8 * static_cast<int64_t>(threadIdx.x); c0 < ldq; c0 += 8 * blockDim.x) {
+            if (m == 4 && c0 + 8 <= K) {
+                // 2:4: the lift is the identity; the chunk's 8 columns in one
+                // 16-byte load (rows and chunks start on 16 bytes)
+                const uint4 u = *reinterpret_cast<const uint4 *>(src_row + c0);
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+                float v[8];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    v[2 * j] = __fmul_rn(__uint_as_float(w[j] << 16), inv);
+                    v[2 * j + 1] = __fmul_rn(__uint_as_float(w[j] & 0xFFFF0000u), inv);
+                }
+                *reinterpret_cast<uint2 *>(qrow + c0) =
+                    make_uint2(e4m3x2(v[0], v[1]) | (e4m3x2(v[2], v[3]) << 16),
+                               e4m3x2(v[4], v[5]) | (e4m3x2(v[6], v[7]) << 16));
+                continue;
+            }
             // group and offset of the chunk's first column once, then stepped
             int g = static_cast<int>(c0) / per, rem = static_cast<int>(c0) - g * per;
             float v[8];
