@@ -97,6 +97,40 @@ __global__ void __launch_bounds__(F8Q_THREADS, 12) k_quant_lift_f8(const uint16_
         if (threadIdx.x == 0) scale[t] = s;
         const uint16_t *src_row = staged ? xrow : row;
         uint8_t *qrow = Q + t * ldq;
+        if (staged && m != 4) {
+            // (2N-2):2N from the staged row, a group per thread: window w of a
+            // group is its inputs 2w .. 2w + 3, so with the codes of input
+            // pairs c16[i] = e4m3x2(x[2i], x[2i + 1]) window w is the word
+            // c16[w] | c16[w + 1] << 16 -- every input converted once
+            const int G = static_cast<int>((K + m - 1) / m), nwin = m / 2 - 1;
+            const uint32_t *xw = reinterpret_cast<const uint32_t *>(xrow);
+            uint32_t *qw = reinterpret_cast<uint32_t *>(qrow);
+            for (int g = threadIdx.x; g < G; g += blockDim.x) {
+                uint32_t c16[5];
+#pragma unroll
+                for (int i = 0; i < 5; ++i) {
+                    if (i >= m / 2) break;
+                    const int64_t col = static_cast<int64_t>(g) * m + 2 * i;  // even: a word of the row
+                    uint32_t w2 = 0u;
+                    if (col < K) {
+                        w2 = xw[col / 2];
+                        if (col + 1 >= K) w2 &= 0xFFFFu;  // the last input is the row's last
+                    }
+                    c16[i] = e4m3x2(__fmul_rn(__uint_as_float(w2 << 16), inv),
+                                    __fmul_rn(__uint_as_float(w2 & 0xFFFF0000u), inv));
+                }
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    if (w >= nwin) break;
+                    qw[static_cast<int64_t>(g) * nwin + w] = c16[w] | (c16[w + 1] << 16);
+                }
+            }
+            // lifted columns past the real ones (the row pitch's padding): zero
+            for (int64_t c = KL + 4 * static_cast<int64_t>(threadIdx.x); c < ldq; c += 4 * blockDim.x)
+                *reinterpret_cast<uint32_t *>(qrow + c) = 0u;
+            __syncthreads();  // the staged row is read before the next token overwrites it
+            continue;
+        }
         const int per = 2 * m - 4;  // lifted columns per group
         for (int64_t c0 = 8 * static_cast<int64_t>(threadIdx.x); c0 < ldq; c0 += 8 * blockDim.x) {
             if (m == 4 && c0 + 8 <= K) {
