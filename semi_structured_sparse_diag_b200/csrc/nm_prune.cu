@@ -1540,6 +1540,9 @@ int hsq_active_clusters(int64_t cblocks, int64_t split) {
     int dev = 0;
     if (split < 2 || split > 8 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
     if (cache[dev][split] == 0) {
+        // the kernel's shared-memory size must be allowed before the query
+        // (else it reports that nothing fits); a failed query is not cached
+        if (!set_smem_attr<k_hsq>(HX_SMEM_BYTES)) return 0;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(cblocks), static_cast<unsigned>(split), 1);
         cfg.blockDim = dim3(HX_THREADS, 1, 1);
